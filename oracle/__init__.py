@@ -1,0 +1,141 @@
+"""fp64 CPU oracle for the off-grid cluster attention and KNN gather.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
+benchmark's CPU-baseline / reference leg.  The product library never imports
+it and shares no code with it.  This module is argument marshalling around
+oracle.c (numpy in, numpy out); all arithmetic lives in the C file, which
+cites the passages it follows.
+
+Array conventions (numpy): xy [B, N, 2] float32; q/k/v/dout [B, N, H, D]
+(converted to float64); bias [H, 3]; clusters [B, G, C] int32; nbr [B, G, M]
+int32; table [B, GH, GW, K] int32; queries [B, Q, 2] float32; feats
+[B, N, d]; p [d/32].
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        so = _build.build()
+        L = ct.CDLL(so)
+        for name in ("orc_cluster_batch", "orc_neighbors_batch", "orc_attn_fwd_batch",
+                     "orc_attn_bwd_batch", "orc_knn_table_batch", "orc_knn_fwd_batch",
+                     "orc_knn_bwd_batch", "orc_set_threads"):
+            getattr(L, name).restype = ct.c_int
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ct.c_void_p)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _i32(a):
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def set_threads(n: int) -> int:
+    """Set the OpenMP thread count of the batch drivers; returns the count in use."""
+    return int(lib().orc_set_threads(int(n)))
+
+
+def cluster(xy, C: int = 8) -> np.ndarray:
+    xy = _f32(xy)
+    B, N = xy.shape[:2]
+    G = (N + C - 1) // C
+    out = np.empty((B, G, C), dtype=np.int32)
+    _check(lib().orc_cluster_batch(_p(xy), B, N, C, _p(out)), "cluster")
+    return out
+
+
+def neighbors(xy, clusters, M: int = 48) -> np.ndarray:
+    xy, clusters = _f32(xy), _i32(clusters)
+    B, N = xy.shape[:2]
+    G, C = clusters.shape[1:]
+    out = np.empty((B, G, M), dtype=np.int32)
+    _check(lib().orc_neighbors_batch(_p(xy), _p(clusters), B, N, C, M, _p(out)), "neighbors")
+    return out
+
+
+def attn_fwd(q, k, v, xy, clusters, nbr, bias, scale: float):
+    q, k, v, bias = _f64(q), _f64(k), _f64(v), _f64(bias)
+    xy, clusters, nbr = _f32(xy), _i32(clusters), _i32(nbr)
+    B, N, H, D = q.shape
+    C, M = clusters.shape[2], nbr.shape[2]
+    o = np.empty_like(q)
+    lse = np.empty((B, N, H), dtype=np.float64)
+    _check(lib().orc_attn_fwd_batch(_p(q), _p(k), _p(v), _p(xy), _p(clusters), _p(nbr),
+                                    _p(bias), B, N, H, D, C, M, ct.c_double(scale),
+                                    _p(o), _p(lse)), "attn_fwd")
+    return o, lse
+
+
+def attn_bwd(q, k, v, xy, clusters, nbr, bias, scale: float, dout):
+    q, k, v, bias, dout = _f64(q), _f64(k), _f64(v), _f64(bias), _f64(dout)
+    xy, clusters, nbr = _f32(xy), _i32(clusters), _i32(nbr)
+    B, N, H, D = q.shape
+    C, M = clusters.shape[2], nbr.shape[2]
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    dbias = np.empty((H, 3), dtype=np.float64)
+    _check(lib().orc_attn_bwd_batch(_p(q), _p(k), _p(v), _p(xy), _p(clusters), _p(nbr),
+                                    _p(bias), B, N, H, D, C, M, ct.c_double(scale),
+                                    _p(dout), _p(dq), _p(dk), _p(dv), _p(dbias)), "attn_bwd")
+    return dq, dk, dv, dbias
+
+
+def knn_table(xy, GH: int = 64, GW: int = 64, K: int = 8) -> np.ndarray:
+    xy = _f32(xy)
+    B, N = xy.shape[:2]
+    out = np.empty((B, GH, GW, K), dtype=np.int32)
+    _check(lib().orc_knn_table_batch(_p(xy), B, N, GH, GW, K, _p(out)), "knn_table")
+    return out
+
+
+def knn_fwd(queries, feats, xy, table, p):
+    queries, xy, table = _f32(queries), _f32(xy), _i32(table)
+    feats, p = _f64(feats), _f64(p)
+    B, Q = queries.shape[:2]
+    N, d = feats.shape[1:]
+    GH, GW, K = table.shape[1:]
+    out = np.empty((B, Q, d), dtype=np.float64)
+    _check(lib().orc_knn_fwd_batch(_p(queries), B, Q, _p(feats), _p(xy), N, d, _p(table),
+                                   GH, GW, K, _p(p), _p(out)), "knn_fwd")
+    return out
+
+
+def knn_bwd(queries, feats, xy, table, p, dout):
+    queries, xy, table = _f32(queries), _f32(xy), _i32(table)
+    feats, p, dout = _f64(feats), _f64(p), _f64(dout)
+    B, Q = queries.shape[:2]
+    N, d = feats.shape[1:]
+    GH, GW, K = table.shape[1:]
+    dF = np.empty((B, N, d), dtype=np.float64)
+    dq = np.empty((B, Q, 2), dtype=np.float64)
+    dp = np.empty((d // 32,), dtype=np.float64)
+    _check(lib().orc_knn_bwd_batch(_p(queries), B, Q, _p(feats), _p(xy), N, d, _p(table),
+                                   GH, GW, K, _p(p), _p(dout), _p(dF), _p(dq), _p(dp)),
+           "knn_bwd")
+    return dF, dq, dp

@@ -1,0 +1,616 @@
+/*
+ * oracle.c -- plain, slow fp64 CPU reference for the off-grid cluster attention
+ * and KNN distance-softmax gather.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file: only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg do.  It shares no code, header, table or helper with the CUDA library.
+ *
+ * Sources (page title, section):
+ *   [AFF]  "AFFMAE: Scalable Vision Pre-Training for High-Resolution Microscopy
+ *          Segmentation on Desktop Hardware" (en.papernotes.org notes), Method:
+ *          "Overall Architecture" (tokens carry explicit 2D coordinates; attention
+ *          through local balanced clustering; stages of Local Cluster Attention),
+ *          "Key Designs" 2 (point-wise deformable cross-attention decoder, the
+ *          exponential distance kernel w_i = softmax_i(-p d_i)), "Key Designs" 3
+ *          (KNN cache lookup: an H x W x K table of the K nearest visible tokens
+ *          per grid cell, queries quantised to a cell), "A Complete Example"
+ *          (64 x 64 grid, ~2048 visible tokens, 819 / 328 / 131 after merging).
+ *   [ABS]  "AFFMAE: Scalable and Efficient Vision Pretraining for Desktop
+ *          Graphics Cards" (arXiv abstract page): mixed-precision Flash-style
+ *          cluster attention kernels.
+ * The pages name the operations but leave their details open.  The readings
+ * taken here (recursive median bisection, C tokens per cluster, M = R*C slots
+ * from the R nearest cluster centroids, the bias a*dx + b*dy - c*(dx^2+dy^2)
+ * with dx = key - query, cell-centre lookup with clamping, per-head p) are the
+ * plainest ones consistent with the pages; each is stated where it is used.
+ *
+ * Arithmetic: fp64 throughout; compiled with -ffp-contract=off so that every
+ * product and sum is rounded on its own, in the order written.  Index-producing
+ * geometry (extents, centroids, squared distances) is written as single
+ * expressions whose rounding order the docstrings state.
+ *
+ * Pins: every function here is checked in tests/ against closed forms,
+ * invariants, brute force on tiny inputs, library routines (dense softmax
+ * attention, a KD-tree) and finite differences.  See the test files.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "oracle.h"
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Thread count of the batch drivers (OpenMP over images); returns the count in use. */
+int orc_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* a1: local balanced clustering                                             */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    float a;      /* coordinate on the split axis   */
+    float b;      /* coordinate on the other axis   */
+    int32_t id;   /* token id: the final tie-break  */
+} split_key;
+
+static int cmp_split_key(const void* pa, const void* pb) {
+    const split_key* x = (const split_key*)pa;
+    const split_key* y = (const split_key*)pb;
+    if (x->a < y->a) return -1;
+    if (x->a > y->a) return 1;
+    if (x->b < y->b) return -1;
+    if (x->b > y->b) return 1;
+    return (x->id > y->id) - (x->id < y->id);
+}
+
+static int cmp_i32(const void* pa, const void* pb) {
+    int32_t x = *(const int32_t*)pa, y = *(const int32_t*)pb;
+    return (x > y) - (x < y);
+}
+
+/*
+ * split(S, g): cut the token set S (n tokens) into g clusters.
+ *   g == 1: emit S sorted by token id, padded with -1 to C slots.
+ *   else:   ex = max x - min x, ey = max y - min y over S (fp64 from fp32);
+ *           axis = x when ex >= ey, else y;
+ *           order S by (coordinate on axis, coordinate on the other axis, id);
+ *           the first ceil(g/2)*C tokens form the left part (ceil(g/2)
+ *           clusters), the rest the right part (g - ceil(g/2) clusters);
+ *           recurse left, then right.
+ * Clusters are numbered in emit order.  Because every left part is full, only
+ * the last cluster of the image can hold padding.
+ */
+static void split(const float* xy, int32_t* ids, int n, int g, int C,
+                  int32_t* out, int* next, split_key* keys) {
+    if (g == 1) {
+        int32_t* dst = out + (size_t)(*next) * C;
+        qsort(ids, (size_t)n, sizeof(int32_t), cmp_i32);
+        for (int s = 0; s < C; ++s) dst[s] = (s < n) ? ids[s] : -1;
+        (*next)++;
+        return;
+    }
+    double xmin = INFINITY, xmax = -INFINITY, ymin = INFINITY, ymax = -INFINITY;
+    for (int i = 0; i < n; ++i) {
+        double x = (double)xy[2 * ids[i]], y = (double)xy[2 * ids[i] + 1];
+        if (x < xmin) xmin = x;
+        if (x > xmax) xmax = x;
+        if (y < ymin) ymin = y;
+        if (y > ymax) ymax = y;
+    }
+    double ex = xmax - xmin, ey = ymax - ymin;
+    int axis = (ex >= ey) ? 0 : 1;
+    for (int i = 0; i < n; ++i) {
+        keys[i].a = xy[2 * ids[i] + axis];
+        keys[i].b = xy[2 * ids[i] + (1 - axis)];
+        keys[i].id = ids[i];
+    }
+    qsort(keys, (size_t)n, sizeof(split_key), cmp_split_key);
+    for (int i = 0; i < n; ++i) ids[i] = keys[i].id;
+    int gl = (g + 1) / 2;
+    int nl = gl * C;
+    split(xy, ids, nl, gl, C, out, next, keys);
+    split(xy, ids + nl, n - nl, g - gl, C, out, next, keys);
+}
+
+int orc_cluster(const float* xy, int N, int C, int32_t* clusters) {
+    if (N < 1 || C < 1 || !xy || !clusters) return 1;
+    int G = (N + C - 1) / C;
+    int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)N);
+    split_key* keys = (split_key*)malloc(sizeof(split_key) * (size_t)N);
+    if (!ids || !keys) { free(ids); free(keys); return 2; }
+    for (int i = 0; i < N; ++i) ids[i] = i;
+    int next = 0;
+    split(xy, ids, N, G, C, clusters, &next, keys);
+    free(ids);
+    free(keys);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* a2: cluster-neighbourhood table                                           */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * centroid_g = (sum of the valid slots' x, in slot order, from 0.0) / n_valid,
+ * likewise y, fp64.  dist2(g, h) = dx*dx + dy*dy with dx = cx_h - cx_g,
+ * dy = cy_h - cy_g, each product and the sum rounded separately.
+ * The neighbourhood of g is the first min(R, G) clusters by (dist2, h),
+ * R = M / C; nbr[g][r*C + s] = clusters[h_r][s]; remaining slots -1.
+ */
+int orc_neighbors(const float* xy, const int32_t* clusters, int N, int C, int M,
+                  int32_t* nbr) {
+    if (N < 1 || C < 1 || M < C || M % C != 0 || !xy || !clusters || !nbr) return 1;
+    int G = (N + C - 1) / C;
+    int R = M / C;
+    double* cx = (double*)malloc(sizeof(double) * (size_t)G);
+    double* cy = (double*)malloc(sizeof(double) * (size_t)G);
+    double* d2 = (double*)malloc(sizeof(double) * (size_t)G);
+    char* taken = (char*)malloc((size_t)G);
+    if (!cx || !cy || !d2 || !taken) { free(cx); free(cy); free(d2); free(taken); return 2; }
+    for (int g = 0; g < G; ++g) {
+        double sx = 0.0, sy = 0.0;
+        int cnt = 0;
+        for (int s = 0; s < C; ++s) {
+            int32_t t = clusters[(size_t)g * C + s];
+            if (t < 0) continue;
+            sx = sx + (double)xy[2 * t];
+            sy = sy + (double)xy[2 * t + 1];
+            cnt++;
+        }
+        cx[g] = sx / (double)cnt;
+        cy[g] = sy / (double)cnt;
+    }
+    for (int g = 0; g < G; ++g) {
+        for (int h = 0; h < G; ++h) {
+            double dx = cx[h] - cx[g];
+            double dy = cy[h] - cy[g];
+            double px = dx * dx;
+            double py = dy * dy;
+            d2[h] = px + py;
+            taken[h] = 0;
+        }
+        int32_t* row = nbr + (size_t)g * M;
+        for (int m = 0; m < M; ++m) row[m] = -1;
+        int take = R < G ? R : G;
+        for (int r = 0; r < take; ++r) {
+            int best = -1;
+            for (int h = 0; h < G; ++h) {
+                if (taken[h]) continue;
+                if (best < 0 || d2[h] < d2[best]) best = h;   /* ties: lower h */
+            }
+            taken[best] = 1;
+            for (int s = 0; s < C; ++s) row[r * C + s] = clusters[(size_t)best * C + s];
+        }
+    }
+    free(cx); free(cy); free(d2); free(taken);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* a3 / a4: local cluster attention, forward and backward                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * For a valid token i of cluster g, head h, and every valid key j in nbr(g):
+ *   dx = x_j - x_i, dy = y_j - y_i                       (key minus query)
+ *   s_ij = scale * <q_i, k_j> + a_h dx + b_h dy - c_h (dx^2 + dy^2)
+ *   o_i  = sum_j softmax_j(s_ij) v_j,   lse_i = log sum_j exp(s_ij)
+ * Plain two-pass softmax (max, then exp-sum), no tiling.  A token whose
+ * neighbourhood holds no valid key gets o = 0 and lse = -inf.
+ * Layout: q, k, v, o as [N][H][D]; lse as [N][H]; bias as [H][3] = (a, b, c).
+ */
+static int attn_logits(const double* q, const double* k, const float* xy,
+                       const int32_t* nrow, const double* bias, int i, int h,
+                       int H, int D, int M, double scale, double* s, int* valid) {
+    int any = 0;
+    const double a = bias[3 * h], b = bias[3 * h + 1], c = bias[3 * h + 2];
+    for (int m = 0; m < M; ++m) {
+        int32_t j = nrow[m];
+        valid[m] = (j >= 0);
+        if (j < 0) { s[m] = -INFINITY; continue; }
+        any = 1;
+        double dx = (double)xy[2 * j] - (double)xy[2 * i];
+        double dy = (double)xy[2 * j + 1] - (double)xy[2 * i + 1];
+        double dot = 0.0;
+        const double* qi = q + ((size_t)i * H + h) * D;
+        const double* kj = k + ((size_t)j * H + h) * D;
+        for (int e = 0; e < D; ++e) dot += qi[e] * kj[e];
+        s[m] = scale * dot + a * dx + b * dy - c * (dx * dx + dy * dy);
+    }
+    return any;
+}
+
+int orc_attn_fwd(const double* q, const double* k, const double* v, const float* xy,
+                 const int32_t* clusters, const int32_t* nbr, const double* bias,
+                 int N, int H, int D, int C, int M, double scale,
+                 double* o, double* lse) {
+    if (N < 1 || H < 1 || D < 1 || C < 1 || M < 1) return 1;
+    int G = (N + C - 1) / C;
+    double* s = (double*)malloc(sizeof(double) * (size_t)M);
+    int* valid = (int*)malloc(sizeof(int) * (size_t)M);
+    if (!s || !valid) { free(s); free(valid); return 2; }
+    for (int g = 0; g < G; ++g) {
+        const int32_t* nrow = nbr + (size_t)g * M;
+        for (int sl = 0; sl < C; ++sl) {
+            int32_t i = clusters[(size_t)g * C + sl];
+            if (i < 0) continue;
+            for (int h = 0; h < H; ++h) {
+                double* oi = o + ((size_t)i * H + h) * D;
+                for (int e = 0; e < D; ++e) oi[e] = 0.0;
+                if (!attn_logits(q, k, xy, nrow, bias, i, h, H, D, M, scale, s, valid)) {
+                    lse[(size_t)i * H + h] = -INFINITY;
+                    continue;
+                }
+                double mx = -INFINITY;
+                for (int m = 0; m < M; ++m) if (valid[m] && s[m] > mx) mx = s[m];
+                double sum = 0.0;
+                for (int m = 0; m < M; ++m) if (valid[m]) sum += exp(s[m] - mx);
+                for (int m = 0; m < M; ++m) {
+                    if (!valid[m]) continue;
+                    double p = exp(s[m] - mx) / sum;
+                    const double* vj = v + ((size_t)nrow[m] * H + h) * D;
+                    for (int e = 0; e < D; ++e) oi[e] += p * vj[e];
+                }
+                lse[(size_t)i * H + h] = mx + log(sum);
+            }
+        }
+    }
+    free(s); free(valid);
+    return 0;
+}
+
+/*
+ * Backward by recomputation, from the definition of the forward:
+ *   P_ij = exp(s_ij - lse_i), dP_ij = <dO_i, v_j>, Delta_i = <dO_i, o_i>,
+ *   dS_ij = P_ij (dP_ij - Delta_i),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
+ *   dv_j = sum_i P_ij dO_i,
+ *   da_h = sum dS dx,  db_h = sum dS dy,  dc_h = -sum dS (dx^2 + dy^2).
+ * o and lse are this oracle's own forward results.  Coordinates get no
+ * gradient.  dq, dk, dv are overwritten; dbias [H][3] is overwritten.
+ */
+int orc_attn_bwd(const double* q, const double* k, const double* v, const float* xy,
+                 const int32_t* clusters, const int32_t* nbr, const double* bias,
+                 int N, int H, int D, int C, int M, double scale, const double* dout,
+                 double* dq, double* dk, double* dv, double* dbias) {
+    if (N < 1 || H < 1 || D < 1 || C < 1 || M < 1) return 1;
+    int G = (N + C - 1) / C;
+    size_t nel = (size_t)N * H * D;
+    double* o = (double*)malloc(sizeof(double) * nel);
+    double* lse = (double*)malloc(sizeof(double) * (size_t)N * H);
+    double* s = (double*)malloc(sizeof(double) * (size_t)M);
+    int* valid = (int*)malloc(sizeof(int) * (size_t)M);
+    if (!o || !lse || !s || !valid) { free(o); free(lse); free(s); free(valid); return 2; }
+    int rc = orc_attn_fwd(q, k, v, xy, clusters, nbr, bias, N, H, D, C, M, scale, o, lse);
+    if (rc) { free(o); free(lse); free(s); free(valid); return rc; }
+    memset(dq, 0, sizeof(double) * nel);
+    memset(dk, 0, sizeof(double) * nel);
+    memset(dv, 0, sizeof(double) * nel);
+    memset(dbias, 0, sizeof(double) * (size_t)H * 3);
+    for (int g = 0; g < G; ++g) {
+        const int32_t* nrow = nbr + (size_t)g * M;
+        for (int sl = 0; sl < C; ++sl) {
+            int32_t i = clusters[(size_t)g * C + sl];
+            if (i < 0) continue;
+            for (int h = 0; h < H; ++h) {
+                if (!attn_logits(q, k, xy, nrow, bias, i, h, H, D, M, scale, s, valid)) continue;
+                const double L = lse[(size_t)i * H + h];
+                const double* doi = dout + ((size_t)i * H + h) * D;
+                const double* oi = o + ((size_t)i * H + h) * D;
+                const double* qi = q + ((size_t)i * H + h) * D;
+                double* dqi = dq + ((size_t)i * H + h) * D;
+                double delta = 0.0;
+                for (int e = 0; e < D; ++e) delta += doi[e] * oi[e];
+                for (int m = 0; m < M; ++m) {
+                    if (!valid[m]) continue;
+                    int32_t j = nrow[m];
+                    const double* vj = v + ((size_t)j * H + h) * D;
+                    const double* kj = k + ((size_t)j * H + h) * D;
+                    double* dkj = dk + ((size_t)j * H + h) * D;
+                    double* dvj = dv + ((size_t)j * H + h) * D;
+                    double p = exp(s[m] - L);
+                    double dp = 0.0;
+                    for (int e = 0; e < D; ++e) dp += doi[e] * vj[e];
+                    double ds = p * (dp - delta);
+                    for (int e = 0; e < D; ++e) {
+                        dqi[e] += scale * ds * kj[e];
+                        dkj[e] += scale * ds * qi[e];
+                        dvj[e] += p * doi[e];
+                    }
+                    double dx = (double)xy[2 * j] - (double)xy[2 * i];
+                    double dy = (double)xy[2 * j + 1] - (double)xy[2 * i + 1];
+                    dbias[3 * h] += ds * dx;
+                    dbias[3 * h + 1] += ds * dy;
+                    dbias[3 * h + 2] -= ds * (dx * dx + dy * dy);
+                }
+            }
+        }
+    }
+    free(o); free(lse); free(s); free(valid);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* a5: KNN cache lookup table                                                */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * table[r][c][k] = the k-th token in the order (dist2, id), where
+ * dist2 = dx*dx + dy*dy, dx = x_t - (c + 0.5), dy = y_t - (r + 0.5), fp64,
+ * each operation rounded on its own.  Slots k >= N hold -1.  The table stores
+ * the neighbours of the cell centre (the lookup the pages describe), not of a
+ * particular query.  Brute force over all tokens.
+ */
+int orc_knn_table(const float* xy, int N, int GH, int GW, int K, int32_t* table) {
+    if (N < 1 || GH < 1 || GW < 1 || K < 1 || !xy || !table) return 1;
+    double* d2 = (double*)malloc(sizeof(double) * (size_t)N);
+    char* taken = (char*)malloc((size_t)N);
+    if (!d2 || !taken) { free(d2); free(taken); return 2; }
+    for (int r = 0; r < GH; ++r) {
+        for (int c = 0; c < GW; ++c) {
+            double ccx = (double)c + 0.5, ccy = (double)r + 0.5;
+            for (int t = 0; t < N; ++t) {
+                double dx = (double)xy[2 * t] - ccx;
+                double dy = (double)xy[2 * t + 1] - ccy;
+                double px = dx * dx;
+                double py = dy * dy;
+                d2[t] = px + py;
+                taken[t] = 0;
+            }
+            int32_t* row = table + ((size_t)r * GW + c) * K;
+            for (int kk = 0; kk < K; ++kk) {
+                int best = -1;
+                for (int t = 0; t < N; ++t) {
+                    if (taken[t]) continue;
+                    if (best < 0 || d2[t] < d2[best]) best = t;   /* ties: lower id */
+                }
+                row[kk] = best;
+                if (best >= 0) taken[best] = 1;
+            }
+        }
+    }
+    free(d2); free(taken);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* a6 / a7: KNN distance-softmax gather, forward and backward                */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Query quantisation: cell = (clamp(floor(qy), 0, GH-1), clamp(floor(qx), 0,
+ * GW-1)); with cell centres at +0.5 this is the nearest cell, and clamping
+ * keeps offsets that leave the grid on its border.  A coordinate that is not
+ * >= 0 (negative or NaN) maps to 0.
+ */
+static int quantise(float v, int n) {
+    if (!(v >= 0.0f)) return 0;
+    if (v >= (float)n) return n - 1;
+    int i = (int)floor((double)v);
+    return i > n - 1 ? n - 1 : i;
+}
+
+/*
+ * d_k = ||q - p_{t_k}|| (Euclidean, fp64); per head h (channels h*32..h*32+31):
+ * w_hk = exp(-p_h (d_k - d_min)) / sum_k' exp(-p_h (d_k' - d_min));
+ * out[q][h*32+e] = sum_k w_hk f[t_k][h*32+e].  Table slots holding -1 are
+ * skipped.  A query whose row holds no token gets out = 0.
+ */
+static int knn_weights(const float* qxy, const float* xy, const int32_t* row, int K,
+                       double ph, double* dist, double* w) {
+    double dmin = INFINITY;
+    int any = 0;
+    for (int kk = 0; kk < K; ++kk) {
+        int32_t t = row[kk];
+        if (t < 0) { dist[kk] = INFINITY; continue; }
+        double dx = (double)qxy[0] - (double)xy[2 * t];
+        double dy = (double)qxy[1] - (double)xy[2 * t + 1];
+        dist[kk] = sqrt(dx * dx + dy * dy);
+        if (dist[kk] < dmin) dmin = dist[kk];
+        any = 1;
+    }
+    if (!any) return 0;
+    double sum = 0.0;
+    for (int kk = 0; kk < K; ++kk) {
+        w[kk] = (row[kk] < 0) ? 0.0 : exp(-ph * (dist[kk] - dmin));
+        sum += w[kk];
+    }
+    for (int kk = 0; kk < K; ++kk) w[kk] /= sum;
+    return 1;
+}
+
+int orc_knn_fwd(const float* queries, int Q, const double* feats, const float* xy,
+                int N, int d, const int32_t* table, int GH, int GW, int K,
+                const double* p, double* out) {
+    if (Q < 0 || N < 1 || d < 32 || d % 32 != 0 || K < 1 || K > 64) return 1;
+    int nh = d / 32;
+    double dist[64], w[64];
+    for (int qi = 0; qi < Q; ++qi) {
+        const float* qxy = queries + 2 * (size_t)qi;
+        int cy = quantise(qxy[1], GH), cx = quantise(qxy[0], GW);
+        const int32_t* row = table + ((size_t)cy * GW + cx) * K;
+        double* oq = out + (size_t)qi * d;
+        for (int c = 0; c < d; ++c) oq[c] = 0.0;
+        for (int h = 0; h < nh; ++h) {
+            if (!knn_weights(qxy, xy, row, K, p[h], dist, w)) break;
+            for (int kk = 0; kk < K; ++kk) {
+                int32_t t = row[kk];
+                if (t < 0) continue;
+                const double* f = feats + (size_t)t * d + 32 * h;
+                for (int e = 0; e < 32; ++e) oq[32 * h + e] += w[kk] * f[e];
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Backward of the gather.  With z_hk = -p_h d_k the logits of w_h:
+ *   dw_hk = <dOut_q,h , f_{t_k},h>,  ds_hk = w_hk (dw_hk - sum_k' w_hk' dw_hk'),
+ *   dp_h += sum_k ds_hk (-d_k),
+ *   dq   += sum_{h,k} ds_hk (-p_h) (q - p_{t_k}) / d_k   (term taken as 0 when d_k = 0),
+ *   dF_t += w_hk dOut_q,h for t = t_k.
+ * The cell index is piecewise constant in q and has no gradient; token
+ * coordinates get none.  dfeats [N][d], dq [Q][2] and dp [d/32] are overwritten.
+ */
+int orc_knn_bwd(const float* queries, int Q, const double* feats, const float* xy,
+                int N, int d, const int32_t* table, int GH, int GW, int K,
+                const double* p, const double* dout,
+                double* dfeats, double* dq, double* dp) {
+    if (Q < 0 || N < 1 || d < 32 || d % 32 != 0 || K < 1 || K > 64) return 1;
+    int nh = d / 32;
+    double dist[64], w[64], dw[64];
+    memset(dfeats, 0, sizeof(double) * (size_t)N * d);
+    memset(dq, 0, sizeof(double) * (size_t)Q * 2);
+    memset(dp, 0, sizeof(double) * (size_t)nh);
+    for (int qi = 0; qi < Q; ++qi) {
+        const float* qxy = queries + 2 * (size_t)qi;
+        int cy = quantise(qxy[1], GH), cx = quantise(qxy[0], GW);
+        const int32_t* row = table + ((size_t)cy * GW + cx) * K;
+        const double* g = dout + (size_t)qi * d;
+        for (int h = 0; h < nh; ++h) {
+            if (!knn_weights(qxy, xy, row, K, p[h], dist, w)) break;
+            double sdw = 0.0;
+            for (int kk = 0; kk < K; ++kk) {
+                int32_t t = row[kk];
+                dw[kk] = 0.0;
+                if (t < 0) continue;
+                const double* f = feats + (size_t)t * d + 32 * h;
+                for (int e = 0; e < 32; ++e) dw[kk] += g[32 * h + e] * f[e];
+                sdw += w[kk] * dw[kk];
+            }
+            for (int kk = 0; kk < K; ++kk) {
+                int32_t t = row[kk];
+                if (t < 0) continue;
+                double ds = w[kk] * (dw[kk] - sdw);
+                dp[h] += ds * (-dist[kk]);
+                if (dist[kk] > 0.0) {
+                    double ux = ((double)qxy[0] - (double)xy[2 * t]) / dist[kk];
+                    double uy = ((double)qxy[1] - (double)xy[2 * t + 1]) / dist[kk];
+                    dq[2 * qi] += ds * (-p[h]) * ux;
+                    dq[2 * qi + 1] += ds * (-p[h]) * uy;
+                }
+                double* df = dfeats + (size_t)t * d + 32 * h;
+                for (int e = 0; e < 32; ++e) df[e] += w[kk] * g[32 * h + e];
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* batch drivers: images are independent; OpenMP over images only            */
+/* ------------------------------------------------------------------------ */
+
+int orc_cluster_batch(const float* xy, int B, int N, int C, int32_t* clusters) {
+    int G = (N + C - 1) / C, rc = 0;
+    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    for (int b = 0; b < B; ++b)
+        rc |= orc_cluster(xy + (size_t)b * N * 2, N, C, clusters + (size_t)b * G * C);
+    return rc;
+}
+
+int orc_neighbors_batch(const float* xy, const int32_t* clusters, int B, int N, int C,
+                        int M, int32_t* nbr) {
+    int G = (N + C - 1) / C, rc = 0;
+    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    for (int b = 0; b < B; ++b)
+        rc |= orc_neighbors(xy + (size_t)b * N * 2, clusters + (size_t)b * G * C, N, C, M,
+                            nbr + (size_t)b * G * M);
+    return rc;
+}
+
+int orc_attn_fwd_batch(const double* q, const double* k, const double* v, const float* xy,
+                       const int32_t* clusters, const int32_t* nbr, const double* bias,
+                       int B, int N, int H, int D, int C, int M, double scale,
+                       double* o, double* lse) {
+    int G = (N + C - 1) / C, rc = 0;
+    size_t st = (size_t)N * H * D;
+    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    for (int b = 0; b < B; ++b)
+        rc |= orc_attn_fwd(q + b * st, k + b * st, v + b * st, xy + (size_t)b * N * 2,
+                           clusters + (size_t)b * G * C, nbr + (size_t)b * G * M, bias,
+                           N, H, D, C, M, scale, o + b * st, lse + (size_t)b * N * H);
+    return rc;
+}
+
+int orc_attn_bwd_batch(const double* q, const double* k, const double* v, const float* xy,
+                       const int32_t* clusters, const int32_t* nbr, const double* bias,
+                       int B, int N, int H, int D, int C, int M, double scale,
+                       const double* dout, double* dq, double* dk, double* dv,
+                       double* dbias) {
+    int G = (N + C - 1) / C, rc = 0;
+    size_t st = (size_t)N * H * D;
+    double* part = (double*)calloc((size_t)B * H * 3, sizeof(double));
+    if (!part) return 2;
+    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    for (int b = 0; b < B; ++b)
+        rc |= orc_attn_bwd(q + b * st, k + b * st, v + b * st, xy + (size_t)b * N * 2,
+                           clusters + (size_t)b * G * C, nbr + (size_t)b * G * M, bias,
+                           N, H, D, C, M, scale, dout + b * st, dq + b * st, dk + b * st,
+                           dv + b * st, part + (size_t)b * H * 3);
+    for (int j = 0; j < H * 3; ++j) {
+        double acc = 0.0;
+        for (int b = 0; b < B; ++b) acc += part[(size_t)b * H * 3 + j];
+        dbias[j] = acc;
+    }
+    free(part);
+    return rc;
+}
+
+int orc_knn_table_batch(const float* xy, int B, int N, int GH, int GW, int K,
+                        int32_t* table) {
+    int rc = 0;
+    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    for (int b = 0; b < B; ++b)
+        rc |= orc_knn_table(xy + (size_t)b * N * 2, N, GH, GW, K,
+                            table + (size_t)b * GH * GW * K);
+    return rc;
+}
+
+int orc_knn_fwd_batch(const float* queries, int B, int Q, const double* feats,
+                      const float* xy, int N, int d, const int32_t* table, int GH, int GW,
+                      int K, const double* p, double* out) {
+    int rc = 0;
+    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    for (int b = 0; b < B; ++b)
+        rc |= orc_knn_fwd(queries + (size_t)b * Q * 2, Q, feats + (size_t)b * N * d,
+                          xy + (size_t)b * N * 2, N, d, table + (size_t)b * GH * GW * K,
+                          GH, GW, K, p, out + (size_t)b * Q * d);
+    return rc;
+}
+
+int orc_knn_bwd_batch(const float* queries, int B, int Q, const double* feats,
+                      const float* xy, int N, int d, const int32_t* table, int GH, int GW,
+                      int K, const double* p, const double* dout, double* dfeats,
+                      double* dq, double* dp) {
+    int rc = 0, nh = d / 32;
+    double* part = (double*)calloc((size_t)B * nh, sizeof(double));
+    if (!part) return 2;
+    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    for (int b = 0; b < B; ++b)
+        rc |= orc_knn_bwd(queries + (size_t)b * Q * 2, Q, feats + (size_t)b * N * d,
+                          xy + (size_t)b * N * 2, N, d, table + (size_t)b * GH * GW * K,
+                          GH, GW, K, p, dout + (size_t)b * Q * d, dfeats + (size_t)b * N * d,
+                          dq + (size_t)b * Q * 2, part + (size_t)b * nh);
+    for (int h = 0; h < nh; ++h) {
+        double acc = 0.0;
+        for (int b = 0; b < B; ++b) acc += part[(size_t)b * nh + h];
+        dp[h] = acc;
+    }
+    free(part);
+    return rc;
+}

@@ -1,0 +1,51 @@
+/*
+ * oracle.h -- declarations of the fp64 CPU reference (test infrastructure only;
+ * the CUDA library neither includes nor links it).  Per-image functions take one
+ * image; the *_batch drivers loop over B independent images (OpenMP).  Layouts:
+ * xy [N][2] fp32 (x = column, y = row, grid-cell units); q/k/v/o/dout [N][H][D];
+ * lse [N][H]; bias [H][3] = (a_h, b_h, c_h); clusters [G][C]; nbr [G][M];
+ * table [GH][GW][K]; queries [Q][2]; feats/dfeats [N][d]; out/dout [Q][d];
+ * p [d/32].  Return 0 on success, 1 on bad arguments, 2 on allocation failure.
+ */
+#ifndef ORACLE_H
+#define ORACLE_H
+#include <stdint.h>
+
+int orc_set_threads(int n);
+int orc_cluster(const float* xy, int N, int C, int32_t* clusters);
+int orc_neighbors(const float* xy, const int32_t* clusters, int N, int C, int M, int32_t* nbr);
+int orc_attn_fwd(const double* q, const double* k, const double* v, const float* xy,
+                 const int32_t* clusters, const int32_t* nbr, const double* bias,
+                 int N, int H, int D, int C, int M, double scale, double* o, double* lse);
+int orc_attn_bwd(const double* q, const double* k, const double* v, const float* xy,
+                 const int32_t* clusters, const int32_t* nbr, const double* bias,
+                 int N, int H, int D, int C, int M, double scale, const double* dout,
+                 double* dq, double* dk, double* dv, double* dbias);
+int orc_knn_table(const float* xy, int N, int GH, int GW, int K, int32_t* table);
+int orc_knn_fwd(const float* queries, int Q, const double* feats, const float* xy,
+                int N, int d, const int32_t* table, int GH, int GW, int K,
+                const double* p, double* out);
+int orc_knn_bwd(const float* queries, int Q, const double* feats, const float* xy,
+                int N, int d, const int32_t* table, int GH, int GW, int K,
+                const double* p, const double* dout, double* dfeats, double* dq, double* dp);
+
+int orc_cluster_batch(const float* xy, int B, int N, int C, int32_t* clusters);
+int orc_neighbors_batch(const float* xy, const int32_t* clusters, int B, int N, int C,
+                        int M, int32_t* nbr);
+int orc_attn_fwd_batch(const double* q, const double* k, const double* v, const float* xy,
+                       const int32_t* clusters, const int32_t* nbr, const double* bias,
+                       int B, int N, int H, int D, int C, int M, double scale,
+                       double* o, double* lse);
+int orc_attn_bwd_batch(const double* q, const double* k, const double* v, const float* xy,
+                       const int32_t* clusters, const int32_t* nbr, const double* bias,
+                       int B, int N, int H, int D, int C, int M, double scale,
+                       const double* dout, double* dq, double* dk, double* dv, double* dbias);
+int orc_knn_table_batch(const float* xy, int B, int N, int GH, int GW, int K, int32_t* table);
+int orc_knn_fwd_batch(const float* queries, int B, int Q, const double* feats,
+                      const float* xy, int N, int d, const int32_t* table, int GH, int GW,
+                      int K, const double* p, double* out);
+int orc_knn_bwd_batch(const float* queries, int B, int Q, const double* feats,
+                      const float* xy, int N, int d, const int32_t* table, int GH, int GW,
+                      int K, const double* p, const double* dout, double* dfeats,
+                      double* dq, double* dp);
+#endif

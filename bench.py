@@ -1,0 +1,516 @@
+#!/usr/bin/env python
+"""Benchmark of the off-grid cluster attention + KNN gather hot path on B200.
+
+One *step* is one pass of every step of the path over one batch of seeded
+synthetic input shaped like the AFFMAE pages' stage-1 workload at 1024 px
+(8 images, a 64 x 64 patch grid with a value-noise mask keeping 2048 tokens per
+image, dim 128 = 4 heads x 32, C = 8, M = 48), followed by the decoder's
+KNN gather over that stage (4096 queries per image at cell centre + U(-1,1)^2,
+K = 8, d = 128, one temperature per head):
+
+    acl_cluster -> acl_neighbors -> acl_cluster_attn_fwd -> acl_cluster_attn_bwd
+    -> acl_knn_table -> acl_knn_gather_fwd -> acl_knn_gather_bwd
+
+`value` is whole-job tokens/s: images x tokens processed by all ranks per second
+of the slowest rank's device time.  Inputs sit in HBM before timing starts;
+S input sets rotate so that the sets total at least 4x the L2 size, and each set
+is replayed as one CUDA graph of the seven library calls.  CUDA events inside
+each graph time every call; the roofline figure is taken for the call with the
+largest share of the step.  `e2e` repeats the step through the same C entry
+points from pinned host buffers, with all input copies and all output read-backs
+inside its timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl acl|reference]
+
+With --impl reference the fp64 CPU oracle is timed on the host cores on a
+bounded sample of the same workload (rank 0 only under torchrun).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "cluster-attn fwd+bwd tokens/s & KNN-gather queries/s; % of B200 HBM roofline"
+WORKLOAD = "stage1-1024px-b8-n2048-d128-h4-c8-m48 + decoder-knn-gather-q4096-k8"
+FALLBACK_HBM_GBS = 6650.0
+OPS = ("cluster", "neighbors", "attn_fwd", "attn_bwd", "knn_table", "knn_fwd", "knn_bwd")
+KERNELS = {
+    "cluster": ["cluster_kernel"],
+    "neighbors": ["neighbors_kernel"],
+    "attn_fwd": ["attn_fwd_kernel"],
+    "attn_bwd": ["attn_bwd_query_kernel", "attn_bwd_key_kernel"],
+    "knn_table": ["knn_table_kernel"],
+    "knn_fwd": ["knn_fwd_kernel"],
+    "knn_bwd": ["knn_bwd_query_kernel", "knn_csr_kernel", "knn_bwd_token_kernel"],
+}
+# DRAM bytes per launch measured by ncu for each call (sum over its kernels), with the
+# sha256 of the CUDA source the counters were taken on; a stale hash reports null.
+NCU_TRAFFIC: dict[str, tuple[float, str, str]] = {}
+
+
+# --------------------------------------------------------------------------- helpers
+
+def env_int(name: str, default: int) -> int:
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("acl", "reference"), default="acl")
+    ap.add_argument("--batch", type=int, default=8, help="images per rank (default 8)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="bounded CPU work of the oracle baseline (seconds)")
+    return ap.parse_args(argv)
+
+
+def shard_images(rank: int, world: int, per_rank: int) -> tuple[int, int]:
+    """Images [first, first + per_rank) of the seeded workload handled by this rank."""
+    return rank * per_rank, per_rank
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured (MEASURED_PEAKS.json)"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback 6.65 TB/s"}
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "off_grid_cluster_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def algorithmic_bytes(B, N, H, Q, d, K, GH, GW, C=8, M=48) -> dict:
+    """Bytes each call must move at least once (every tensor counted once)."""
+    G = (N + C - 1) // C
+    per_tok_meta = 8 + 4 + 4 * M * G / N           # coords, cluster slot, neighbour-table share
+    return {
+        "cluster": B * N * (8 + 4),
+        "neighbors": B * (N * 8 + G * C * 4 + G * M * 4),
+        "attn_fwd": B * N * (H * (3 * 64 + 64 + 4) + per_tok_meta) + H * 12,
+        "attn_bwd": B * N * (H * (5 * 64 + 4 + 3 * 64) + per_tok_meta) + 2 * H * 12,
+        "knn_table": B * (N * 8 + GH * GW * K * 4),
+        "knn_fwd": B * (Q * (8 + 4 * K + 2 * d) + N * (2 * d + 8)) + 4 * d // 32,
+        "knn_bwd": B * (Q * (8 + 4 * K + 2 * d + 8) + N * (2 * d + 8 + 2 * d)) + 8 * d // 32,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+class StepSet:
+    """Device buffers of one input set plus the seven library calls of a step."""
+
+    def __init__(self, sb, device, acl, torch):
+        a, k = sb.attn, sb.knn
+        T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
+        bf = torch.bfloat16
+        self.acl, self.torch = acl, torch
+        self.B, self.N, self.H, self.Q, self.d, self.K = a.B, a.N, a.H, k.Q, k.d, k.K
+        self.GH, self.GW, self.scale = k.GH, k.GW, a.scale
+        self.inputs = {
+            "coords": T(a.coords), "q": T(a.q, bf), "k": T(a.k, bf), "v": T(a.v, bf),
+            "do": T(a.do, bf), "bias": T(a.bias), "queries": T(k.queries),
+            "feats": T(k.feats, bf), "dout": T(k.dout, bf), "p": T(k.p),
+        }
+        B, N, H, G = self.B, self.N, self.H, (self.N + 7) // 8
+        e = lambda shape, dt: torch.empty(shape, dtype=dt, device=device)
+        self.outputs = {
+            "clusters": e((B, G, 8), torch.int32), "nbr": e((B, G, 48), torch.int32),
+            "o": e((B, N, H, 32), bf), "lse": e((B, N, H), torch.float32),
+            "dq": e((B, N, H, 32), bf), "dk": e((B, N, H, 32), bf), "dv": e((B, N, H, 32), bf),
+            "dbias": e((H, 3), torch.float32),
+            "table": e((B, self.GH, self.GW, self.K), torch.int32),
+            "out": e((B, self.Q, self.d), bf), "dfeats": e((B, N, self.d), bf),
+            "dqueries": e((B, self.Q, 2), torch.float32), "dp": e((self.d // 32,), torch.float32),
+        }
+        self.ws_attn = e((acl.acl_cluster_attn_workspace(B, N, H, 8, 48),), torch.uint8)
+        self.ws_knn = e((acl.acl_knn_gather_workspace(B, self.Q, N, self.d, self.K),), torch.uint8)
+
+    def bytes(self) -> int:
+        ts = list(self.inputs.values()) + list(self.outputs.values()) + [self.ws_attn, self.ws_knn]
+        return sum(t.numel() * t.element_size() for t in ts)
+
+    def op(self, name: str, stream):
+        i, o, acl = self.inputs, self.outputs, self.acl
+        if name == "cluster":
+            acl.acl_cluster(i["coords"], 8, clusters=o["clusters"], stream=stream)
+        elif name == "neighbors":
+            acl.acl_neighbors(i["coords"], o["clusters"], 48, nbr=o["nbr"], stream=stream)
+        elif name == "attn_fwd":
+            acl.acl_cluster_attn_fwd(i["q"], i["k"], i["v"], i["coords"], o["clusters"], o["nbr"],
+                                     i["bias"], self.scale, O=o["o"], lse=o["lse"], stream=stream)
+        elif name == "attn_bwd":
+            acl.acl_cluster_attn_bwd(i["q"], i["k"], i["v"], i["coords"], o["clusters"], o["nbr"],
+                                     i["bias"], self.scale, o["o"], i["do"], o["lse"], o["dq"],
+                                     o["dk"], o["dv"], o["dbias"], workspace=self.ws_attn,
+                                     stream=stream)
+        elif name == "knn_table":
+            acl.acl_knn_table(i["coords"], self.GH, self.GW, self.K, table=o["table"], stream=stream)
+        elif name == "knn_fwd":
+            acl.acl_knn_gather_fwd(i["queries"], i["feats"], i["coords"], o["table"], i["p"],
+                                   out=o["out"], stream=stream)
+        elif name == "knn_bwd":
+            acl.acl_knn_gather_bwd(i["queries"], i["feats"], i["coords"], o["table"], i["p"],
+                                   i["dout"], dfeats=o["dfeats"], dqueries=o["dqueries"],
+                                   dp=o["dp"], workspace=self.ws_knn, stream=stream)
+        else:
+            raise KeyError(name)
+
+    def step(self, stream, events=None):
+        for j, name in enumerate(OPS):
+            if events is not None:
+                events[j].record(stream)
+            self.op(name, stream)
+        if events is not None:
+            events[len(OPS)].record(stream)
+
+
+def run_gpu(args, rank: int, world: int):
+    import torch
+    import torch.distributed as dist
+
+    import off_grid_cluster_b200 as acl
+    from off_grid_cluster_b200 import synth
+
+    local = env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    first, per_rank = shard_images(rank, world, args.batch)
+    sb = synth.step_batch(B=per_rank, image0=first)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    base = StepSet(sb, device, acl, torch)
+    set_bytes = base.bytes()
+    n_sets = max(2, math.ceil(4 * l2 / set_bytes))
+    sets = [base] + [StepSet(sb, device, acl, torch) for _ in range(n_sets - 1)]
+    stream = torch.cuda.Stream(device)
+
+    # eager warm-up of every call (kernel attributes, lazy module loading), then capture
+    with torch.cuda.stream(stream):
+        for s in sets:
+            s.step(stream)
+    stream.synchronize()
+    n_ev = len(OPS) + 1
+    graphs, events = [], []
+    launches0 = acl.acl_launch_count()
+    for s in sets:
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            s.step(stream, evs)
+        graphs.append(g)
+        events.append(evs)
+    launches_per_step = (acl.acl_launch_count() - launches0) // len(sets)
+    torch.cuda.synchronize()
+
+    for w in range(args.warmup):
+        graphs[w % n_sets].replay()
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(device)
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local)).start()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for it in range(args.steps):
+            graphs[it % n_sets].replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    step_ms_local = t0.elapsed_time(t1) / max(args.steps, 1)
+    # per-call durations from the in-graph events (the last replay of every set)
+    per_op = np.zeros(len(OPS))
+    used = min(n_sets, args.steps)
+    for s_i in range(used):
+        ev = events[s_i]
+        per_op += np.array([ev[j].elapsed_time(ev[j + 1]) for j in range(len(OPS))])
+    per_op /= max(used, 1)
+    # keep the same load on the GPU until the clock sampler has several samples
+    t_wall = time.time()
+    with torch.cuda.stream(stream):
+        it = 0
+        while time.time() - t_wall < 0.8:
+            graphs[it % n_sets].replay()
+            it += 1
+            if it % 64 == 0:
+                stream.synchronize()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+
+    step_ms = max_over_ranks(step_ms_local)
+    B, N, Q = per_rank, sb.attn.N, sb.knn.Q
+    tokens = world * B * N
+    value = tokens / (step_ms * 1e-3)
+    abytes = algorithmic_bytes(B, N, sb.attn.H, Q, sb.knn.d, sb.knn.K, sb.knn.GH, sb.knn.GW)
+    dom = int(np.argmax(per_op))
+    dom_name = OPS[dom]
+    peaks = measured_peaks()
+    achieved = abytes[dom_name] / (per_op[dom] * 1e-3) / 1e9
+    traffic = None
+    if dom_name in NCU_TRAFFIC and NCU_TRAFFIC[dom_name][1] == source_hash():
+        traffic = NCU_TRAFFIC[dom_name][0]
+    breakdown = {}
+    for j, name in enumerate(OPS):
+        gbs = abytes[name] / (per_op[j] * 1e-3) / 1e9
+        breakdown[name] = {"us": round(per_op[j] * 1e3, 2), "alg_MB": round(abytes[name] / 1e6, 3),
+                           "GB_s": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    attn_ms = per_op[OPS.index("attn_fwd")] + per_op[OPS.index("attn_bwd")]
+    knn_ms = per_op[OPS.index("knn_fwd")] + per_op[OPS.index("knn_bwd")]
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, base, stream, torch, acl, tokens_per_step=world * B * N)
+        e2e_ms = max_over_ranks(e2e.pop("_ms"))
+        e2e["value"] = round(world * B * N / (e2e_ms * 1e-3), 1)
+        e2e["ms_per_step"] = round(e2e_ms, 4)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args, sb)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; shapes of the pages' 1024 px stage-1 workload)",
+        "config": {"workload": WORKLOAD, "images_per_gpu": B, "tokens_per_image": N,
+                   "heads": sb.attn.H, "head_dim": 32, "C": 8, "M": 48,
+                   "queries_per_image": Q, "knn_d": sb.knn.d, "K": sb.knn.K, "grid": [64, 64],
+                   "l2": f"rotating {n_sets} input sets, {n_sets * set_bytes / 1e6:.0f} MB total "
+                         f">= 4 x L2 ({l2 / 1e6:.0f} MB)",
+                   "timing": "CUDA graph per set, CUDA events on the launching stream",
+                   "parallelism": f"replicas x{world} (images sharded, no collective)"},
+        "parts": {
+            "knn_queries_per_s": round(world * B * Q / (step_ms * 1e-3), 1),
+            "cluster_attn_fwd_bwd_tokens_per_s": round(world * B * N / (attn_ms * 1e-3), 1),
+            "knn_gather_fwd_bwd_queries_per_s": round(world * B * Q / (knn_ms * 1e-3), 1),
+            "per_call": breakdown,
+        },
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": traffic, "kernel": f"acl_{dom_name} ({', '.join(KERNELS[dom_name])})",
+                     "alg_bytes_per_launch": int(abytes[dom_name]),
+                     "launch_us": round(per_op[dom] * 1e3, 3), "peak_source": peaks["source"]},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": clk,
+    }
+    for g in graphs:
+        g.reset()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, s: StepSet, stream, torch, acl, tokens_per_step: int) -> dict:
+    """The step through the public entry points from pinned host memory, copies inside."""
+    hin = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in s.inputs.items()}
+    for k, v in s.inputs.items():
+        hin[k].copy_(v)
+    hout = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in s.outputs.items()}
+    h2d = sum(t.numel() * t.element_size() for t in hin.values())
+    d2h = sum(t.numel() * t.element_size() for t in hout.values())
+
+    def one():
+        for k, v in hin.items():
+            s.inputs[k].copy_(v, non_blocking=True)
+        s.step(stream)
+        for k, v in s.outputs.items():
+            hout[k].copy_(v, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one()
+    torch.cuda.synchronize()
+    n = max(1, args.e2e_steps)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(n):
+            one()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    return {"value": tokens_per_step / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": n, "_ms": ms}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def oracle_step(sb, images: slice | None = None) -> None:
+    """One pass of the hot path through the fp64 oracle (optionally on a subset of images)."""
+    import oracle
+    a, k = sb.attn, sb.knn
+    sl = images if images is not None else slice(None)
+    xy = a.coords[sl]
+    cl = oracle.cluster(xy, 8)
+    nb = oracle.neighbors(xy, cl, 48)
+    oracle.attn_fwd(a.q[sl], a.k[sl], a.v[sl], xy, cl, nb, a.bias, a.scale)
+    oracle.attn_bwd(a.q[sl], a.k[sl], a.v[sl], xy, cl, nb, a.bias, a.scale, a.do[sl])
+    table = oracle.knn_table(k.coords[sl], k.GH, k.GW, k.K)
+    oracle.knn_fwd(k.queries[sl], k.feats[sl], k.coords[sl], table, k.p)
+    oracle.knn_bwd(k.queries[sl], k.feats[sl], k.coords[sl], table, k.p, k.dout[sl])
+
+
+def cpu_baseline(args, sb) -> dict:
+    import oracle
+    cores = oracle.set_threads(os.cpu_count() or 1)
+    B, N = sb.attn.B, sb.attn.N
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(sb)
+        reps += 1
+        if time.perf_counter() - t0 >= args.cpu_seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(reps * B * N / dt, 1), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{reps} full step(s) of the workload ({B} images), fp64 C, OpenMP over images"}
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    import oracle
+    from off_grid_cluster_b200 import synth
+    cores = oracle.set_threads(os.cpu_count() or 1)
+    sb = synth.step_batch(B=args.batch)
+    B, N = sb.attn.B, sb.attn.N
+    # bounded sample: images per step chosen so that warm-up + steps take about two minutes
+    t = time.perf_counter()
+    oracle_step(sb, slice(0, 1))
+    t_img = max(time.perf_counter() - t, 1e-3)
+    total = args.steps + args.warmup
+    per_step = int(max(1, min(B, 120.0 / (total * t_img))))
+    sl = slice(0, per_step)
+    for _ in range(args.warmup):
+        oracle_step(sb, sl)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(sb, sl)
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    value = per_step * N / dt
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; shapes of the pages' 1024 px stage-1 workload)",
+        "config": {"workload": WORKLOAD, "images_per_gpu": B, "tokens_per_image": N,
+                   "sample_images_per_step": per_step},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{per_step} of {B} images per step, fp64 C oracle"},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = env_int("RANK", 0)
+    world = env_int("WORLD_SIZE", 1)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_gpu(args, rank, world)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,238 @@
+/*
+ * acl.h -- C ABI of the off-grid local cluster attention and KNN gather library
+ * (libacl.so, CUDA, sm_100a).
+ *
+ * What it computes follows the AFFMAE pages:
+ *   "AFFMAE: Scalable Vision Pre-Training for High-Resolution Microscopy
+ *   Segmentation on Desktop Hardware" (en.papernotes.org notes), Method:
+ *   "Overall Architecture" -- every token keeps an explicit 2D coordinate and
+ *   attention runs through local balanced clustering (stages of Local Cluster
+ *   Attention); "Key Designs" 2 -- the decoder gathers the K nearest tokens of a
+ *   sample point with the exponential distance kernel w_i = softmax_i(-p d_i);
+ *   "Key Designs" 3 -- an H x W x K table of each grid cell's K nearest tokens,
+ *   the query quantised to its cell.  The arXiv abstract page ("AFFMAE: Scalable
+ *   and Efficient Vision Pretraining for Desktop Graphics Cards") names the
+ *   Flash-style mixed-precision cluster attention kernels.
+ *
+ * Conventions shared by every call
+ *   - Coordinates are fp32 in grid-cell units: x = column, y = row; cell (r, c)
+ *     covers [c, c+1) x [r, r+1), centre (c + 0.5, r + 0.5).  They must be finite.
+ *   - Feature tensors are bf16 (raw 16-bit patterns, acl_bf16), row-major.
+ *     Attention Q/K/V/O and their gradients: [B][N][H][D] with D = 32.
+ *     Gather features: [B][N][d], channel c belongs to head c / 32.
+ *   - Index tensors are int32; -1 marks an empty slot.
+ *   - Every pointer is a DEVICE pointer owned by the caller, including outputs
+ *     and workspaces.  bf16 tensors must be 16-byte aligned, coordinate and
+ *     query tensors 8-byte aligned, workspaces 256-byte aligned.  The library
+ *     allocates nothing and keeps no state between calls (beyond raising a
+ *     kernel's shared-memory limit once per device); calls are asynchronous on
+ *     `stream` (NULL = legacy default stream) and may be captured into a CUDA
+ *     graph once each call has been made once on the device outside capture.
+ *   - Outputs are overwritten in full (gradients included: nothing accumulates).
+ *   - Images in a batch are independent problems.
+ *   - Host-side validation runs before any launch; a failed call launches
+ *     nothing and returns the status.  After launching, a launch error maps to
+ *     ACL_ERR_CUDA.  Nothing aborts and nothing throws across the ABI.
+ *   - Floating-point results are deterministic: no floating-point atomics, every
+ *     reduction runs in a fixed order; repeated calls give identical bits.
+ */
+#ifndef ACL_H
+#define ACL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ACL_OK = 0,
+    ACL_ERR_INVALID_ARG = 1,   /* null pointer, size out of range, inconsistent sizes  */
+    ACL_ERR_CUDA = 2,          /* a CUDA call or kernel launch failed                  */
+    ACL_ERR_UNSUPPORTED = 3,   /* valid arguments outside what the kernels implement   */
+    ACL_ERR_WORKSPACE = 4,     /* workspace pointer null or smaller than required     */
+    ACL_ERR_DEVICE_CHECK = 5,  /* reserved: device-side consistency check failed      */
+    ACL_ERR_TIMEOUT = 6        /* reserved: a bounded device wait gave up              */
+} acl_status;
+
+/* Same type as cudaStream_t (both are pointers to struct CUstream_st). */
+struct CUstream_st;
+typedef struct CUstream_st* acl_stream_t;
+
+/* Raw bf16 bit pattern (1 sign, 8 exponent, 7 mantissa bits). */
+typedef uint16_t acl_bf16;
+
+/* Implementation limits (ACL_ERR_UNSUPPORTED beyond them). */
+#define ACL_MAX_CLUSTER_N 8192   /* tokens per image for acl_cluster                     */
+#define ACL_MAX_CLUSTER_C 64     /* cluster size for acl_cluster / acl_neighbors         */
+#define ACL_MAX_NEIGHBOR_R 16    /* M / C neighbour clusters                             */
+#define ACL_ATTN_D 32            /* head dim of the attention kernels                    */
+#define ACL_ATTN_C 8             /* cluster size of the attention kernels                */
+#define ACL_ATTN_MAX_M 64        /* neighbourhood slots of the attention kernels          */
+#define ACL_MAX_TABLE_N 16384    /* tokens per image for acl_knn_table                   */
+#define ACL_MAX_KNN_K 16         /* neighbours per cell                                  */
+#define ACL_MAX_GATHER_D 1024    /* channels of the gather                               */
+#define ACL_MAX_GATHER_Q 65535   /* queries per image for acl_knn_gather_bwd             */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* acl_status_string(acl_status s);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int acl_version(void);
+
+/* Number of kernels this process has launched through the library (diagnostic;
+ * counts host-side launches, so a captured CUDA graph's replays add nothing). */
+uint64_t acl_launch_count(void);
+
+/*
+ * acl_cluster -- local balanced clustering (a1).
+ * Passage: AFF notes, Method "Overall Architecture" (attention through local
+ * balanced clustering of tokens with 2D coordinates).  The pages give no
+ * algorithm; this is recursive median bisection:
+ *   split(S, g): if g == 1 emit S ordered by token id, padded with -1 to C slots;
+ *   else cut on the axis of larger fp64 extent (max - min; ties -> x), ordering S
+ *   by (coordinate on that axis, other coordinate, token id); the first
+ *   ceil(g/2) * C tokens form the left part with ceil(g/2) clusters; recurse left
+ *   then right.  The root is split(all N tokens, G = ceil(N / C)).
+ * coords   [B][N][2] fp32.
+ * clusters [B][G][C] int32 out: token ids; only the last cluster of an image may
+ *          hold -1 (when N % C != 0).  Every token appears exactly once.
+ * Limits: 1 <= N <= ACL_MAX_CLUSTER_N, 1 <= C <= ACL_MAX_CLUSTER_C, B >= 1.
+ * The result is bit-exact: comparisons only, and fp64 extents of fp32 values.
+ */
+acl_status acl_cluster(const float* coords, int B, int N, int C,
+                       int32_t* clusters, acl_stream_t stream);
+
+/*
+ * acl_neighbors -- cluster-neighbourhood table (a2).
+ * Passage: AFF notes, Method "Overall Architecture" (Local Cluster Attention);
+ * the pages do not define the neighbourhood.  Reading: the R = M / C clusters of
+ * nearest centroid, the cluster itself first.
+ *   centroid_g = (sum of its valid tokens' x in slot order, from 0.0) / count,
+ *   likewise y, fp64; dist2 = dx*dx + dy*dy (dx = cx_h - cx_g), each operation
+ *   rounded separately (no fused multiply-add); the first min(R, G) clusters by
+ *   (dist2, cluster id).
+ * coords [B][N][2]; clusters [B][G][C] as written by acl_cluster.
+ * nbr    [B][G][M] int32 out: nbr[g][r*C + s] = clusters[h_r][s]; slots beyond
+ *        min(R, G) clusters hold -1.
+ * Limits: M % C == 0, 1 <= M / C <= ACL_MAX_NEIGHBOR_R, C <= ACL_MAX_CLUSTER_C,
+ *         ceil(N / C) <= 14528 (centroids held in shared memory), B <= 65535.  Bit-exact.
+ */
+acl_status acl_neighbors(const float* coords, const int32_t* clusters, int B, int N,
+                         int C, int M, int32_t* nbr, acl_stream_t stream);
+
+/* Workspace bytes acl_cluster_attn_bwd needs for these sizes (0 on bad sizes). */
+size_t acl_cluster_attn_workspace(int B, int N, int H, int C, int M);
+
+/*
+ * acl_cluster_attn_fwd -- local cluster attention, forward (a3).
+ * Passage: AFF notes, Method "Overall Architecture" and the flowchart (Local
+ * Cluster Attention blocks); arXiv abstract page (Flash-style cluster attention).
+ * For each valid token i of cluster g, head h, over the valid keys j of nbr[g]:
+ *   dx = x_j - x_i, dy = y_j - y_i                         (key minus query)
+ *   s_ij = scale * <q_i, k_j> + a_h dx + b_h dy - c_h (dx^2 + dy^2)
+ *   O_i = sum_j softmax_j(s_ij) v_j,   lse_i = log sum_j exp(s_ij)   (natural log)
+ * Q, K, V [B][N][H][D] bf16 (any token order: nbr holds token ids);
+ * coords [B][N][2]; clusters [B][G][C]; nbr [B][G][M] (any token ids, -1 = empty);
+ * bias_coef [H][3] fp32 = (a_h, b_h, c_h); scale e.g. 1/sqrt(32).
+ * O [B][N][H][D] bf16 out (rounded to nearest even), lse [B][N][H] fp32 out.
+ * Rows of tokens that no cluster lists are left untouched; a token whose
+ * neighbourhood is empty gets O = 0 and lse = -inf.
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation, fp32 softmax.
+ * Limits: D == 32, C == 8, M % 8 == 0, 8 <= M <= 64, 1 <= H <= 64.
+ */
+acl_status acl_cluster_attn_fwd(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V,
+                                const float* coords, const int32_t* clusters,
+                                const int32_t* nbr, const float* bias_coef,
+                                int B, int N, int H, int D, int C, int M, float scale,
+                                acl_bf16* O, float* lse, acl_stream_t stream);
+
+/*
+ * acl_cluster_attn_bwd -- local cluster attention, backward (a4), recomputing
+ * P_ij = exp(s_ij - lse_i) from the forward's lse:
+ *   dP_ij = <dO_i, v_j>, Delta_i = <dO_i, O_i>, dS_ij = P_ij (dP_ij - Delta_i),
+ *   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,
+ *   dV_j = sum_i P_ij dO_i,
+ *   dbias_coef[h] = (sum dS dx, sum dS dy, -sum dS (dx^2 + dy^2)) over all images.
+ * Arguments as in the forward, plus O and lse from it and dO [B][N][H][D] bf16.
+ * dQ, dK, dV [B][N][H][D] bf16 out; dbias_coef [H][3] fp32 out.
+ * nbr must be the table acl_neighbors built from `clusters` (each group of C
+ * slots is a whole cluster row): dK/dV are reduced per key cluster over the
+ * query clusters that list it, in a fixed order, without atomics.
+ * workspace: device memory of at least acl_cluster_attn_workspace(B, N, H, C, M)
+ * bytes, 256-byte aligned; its contents on entry do not matter.
+ */
+acl_status acl_cluster_attn_bwd(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V,
+                                const float* coords, const int32_t* clusters,
+                                const int32_t* nbr, const float* bias_coef,
+                                int B, int N, int H, int D, int C, int M, float scale,
+                                const acl_bf16* O, const acl_bf16* dO, const float* lse,
+                                acl_bf16* dQ, acl_bf16* dK, acl_bf16* dV,
+                                float* dbias_coef, void* workspace, size_t ws_bytes,
+                                acl_stream_t stream);
+
+/*
+ * acl_knn_table -- KNN cache lookup table (a5).
+ * Passage: AFF notes, "Key Designs" 3 (KNN Cache Lookup): an H x W x K table of
+ * the K nearest visible tokens of every grid cell.
+ *   table[r][c][k] = the k-th token in the order (dist2, token id), where
+ *   dist2 = dx*dx + dy*dy, dx = x_t - (c + 0.5), dy = y_t - (r + 0.5) in fp64,
+ *   each operation rounded separately.  Slots k >= N hold -1.
+ * coords [B][N][2]; table [B][H][W][K] int32 out.  Bit-exact (a binned search
+ * whose cut-off is conservative in exact arithmetic returns the brute-force set).
+ * Limits: 1 <= N <= ACL_MAX_TABLE_N, 1 <= K <= ACL_MAX_KNN_K, 1 <= H, W <= 4096,
+ *         B <= 65535.
+ */
+acl_status acl_knn_table(const float* coords, int B, int N, int H, int W, int K,
+                         int32_t* table, acl_stream_t stream);
+
+/* Workspace bytes acl_knn_gather_bwd needs for these sizes (0 on bad sizes). */
+size_t acl_knn_gather_workspace(int B, int Q, int N, int d, int K);
+
+/*
+ * acl_knn_gather_fwd -- KNN distance-softmax gather, forward (a6).
+ * Passage: AFF notes, "Key Designs" 2 (w_i = softmax_i(-p d_i) over the K nearest
+ * tokens of the sample point q) and 3 (q quantised to its grid cell, neighbours
+ * read from the table).
+ *   cell = (clamp(floor(q_y), 0, H-1), clamp(floor(q_x), 0, W-1)); a coordinate
+ *   that is not >= 0 maps to 0;
+ *   d_k = ||q - p_{t_k}|| (fp32); per head h: w_hk = softmax_k(-p_h d_k), computed
+ *   as exp(-p_h (d_k - d_min)) / sum; out[h*32 + e] = sum_k w_hk f[t_k][h*32 + e].
+ *   Table slots holding -1 are skipped; a row with no token gives out = 0.
+ * queries [B][Q][2] fp32; feats [B][N][d] bf16; coords [B][N][2]; table
+ * [B][H][W][K] (e.g. from acl_knn_table); p [d/32] fp32 (one temperature per head).
+ * out [B][Q][d] bf16 out.
+ * Limits: d % 32 == 0, 32 <= d <= ACL_MAX_GATHER_D, 1 <= K <= ACL_MAX_KNN_K,
+ *         table entries in [-1, N).
+ */
+acl_status acl_knn_gather_fwd(const float* queries, int B, int Q, const acl_bf16* feats,
+                              const float* coords, int N, int d, const int32_t* table,
+                              int H, int W, int K, const float* p, acl_bf16* out,
+                              acl_stream_t stream);
+
+/*
+ * acl_knn_gather_bwd -- KNN gather, backward (a7).  With z_hk = -p_h d_k:
+ *   dw_hk = <dOut_h, f_{t_k},h>, ds_hk = w_hk (dw_hk - sum_k' w_hk' dw_hk'),
+ *   dp_h = sum over all queries and k of ds_hk (-d_k),
+ *   dq = sum_{h,k} ds_hk (-p_h) (q - p_{t_k}) / d_k (the term is 0 when d_k = 0),
+ *   dF_t = sum over (query, k) with t_k = t of w_hk dOut_h.
+ * The cell index is piecewise constant (no gradient); coords get none.
+ * dF is reduced per token over an inverse index built by a stable counting sort
+ * (fixed order, no atomics).
+ * Arguments as in the forward plus dOut [B][Q][d] bf16.
+ * dfeats [B][N][d] bf16 out; dqueries [B][Q][2] fp32 out; dp [d/32] fp32 out.
+ * workspace: at least acl_knn_gather_workspace(B, Q, N, d, K) bytes, 256-byte
+ * aligned; its contents on entry do not matter.
+ * Limits: as the forward, plus Q <= ACL_MAX_GATHER_Q and N <= ACL_MAX_TABLE_N.
+ */
+acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16* feats,
+                              const float* coords, int N, int d, const int32_t* table,
+                              int H, int W, int K, const float* p, const acl_bf16* dOut,
+                              acl_bf16* dfeats, float* dqueries, float* dp,
+                              void* workspace, size_t ws_bytes, acl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ACL_H */

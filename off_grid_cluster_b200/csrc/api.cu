@@ -1,0 +1,202 @@
+// api.cu -- the exported C ABI (include/acl.h): argument validation, workspace
+// sizing and dispatch to the kernel launchers.  No call allocates, synchronises or
+// keeps state; every check runs on the host before the first launch.
+#include <atomic>
+
+#include "../../include/acl.h"
+#include "internal.h"
+
+namespace acl {
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+}  // namespace acl
+
+namespace {
+
+constexpr size_t kMaxSmem = 227 * 1024;
+constexpr int kMaxAttnN = 262144;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+acl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ACL_OK : ACL_ERR_CUDA; }
+
+cudaStream_t S(acl_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+const acl::bf16* BF(const acl_bf16* p) { return reinterpret_cast<const acl::bf16*>(p); }
+acl::bf16* BFm(acl_bf16* p) { return reinterpret_cast<acl::bf16*>(p); }
+
+acl_status check_attn(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V, const float* coords,
+                      const int32_t* clusters, const int32_t* nbr, const float* bias, int B, int N,
+                      int H, int D, int C, int M) {
+    if (!Q || !K || !V || !coords || !clusters || !nbr || !bias) return ACL_ERR_INVALID_ARG;
+    if (B < 1 || N < 1 || H < 1 || D < 1 || C < 1 || M < 1) return ACL_ERR_INVALID_ARG;
+    if (M % C != 0) return ACL_ERR_INVALID_ARG;
+    if (D != ACL_ATTN_D || C != ACL_ATTN_C || M > ACL_ATTN_MAX_M || H > 1024 || N > kMaxAttnN)
+        return ACL_ERR_UNSUPPORTED;
+    if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(coords, 8))
+        return ACL_ERR_INVALID_ARG;
+    return ACL_OK;
+}
+
+acl_status check_gather(const float* queries, int B, int Q, const acl_bf16* feats,
+                        const float* coords, int N, int d, const int32_t* table, int H, int W,
+                        int K, const float* p) {
+    if ((Q > 0 && !queries) || !feats || !coords || !table || !p) return ACL_ERR_INVALID_ARG;
+    if (B < 1 || Q < 0 || N < 1 || d < 1 || H < 1 || W < 1 || K < 1) return ACL_ERR_INVALID_ARG;
+    if (d % 32 != 0) return ACL_ERR_INVALID_ARG;
+    if (d > ACL_MAX_GATHER_D || K > ACL_MAX_KNN_K) return ACL_ERR_UNSUPPORTED;
+    if (static_cast<long long>(H) * W * K > 0x7fffffffLL) return ACL_ERR_UNSUPPORTED;
+    if (!aligned(feats, 16) || !aligned(queries, 8) || !aligned(coords, 8)) return ACL_ERR_INVALID_ARG;
+    return ACL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* acl_status_string(acl_status s) {
+    switch (s) {
+        case ACL_OK: return "ACL_OK";
+        case ACL_ERR_INVALID_ARG: return "ACL_ERR_INVALID_ARG: null pointer, misaligned pointer or size out of range";
+        case ACL_ERR_CUDA: return "ACL_ERR_CUDA: a CUDA call or kernel launch failed";
+        case ACL_ERR_UNSUPPORTED: return "ACL_ERR_UNSUPPORTED: sizes outside the implemented limits";
+        case ACL_ERR_WORKSPACE: return "ACL_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        case ACL_ERR_DEVICE_CHECK: return "ACL_ERR_DEVICE_CHECK: device-side consistency check failed";
+        case ACL_ERR_TIMEOUT: return "ACL_ERR_TIMEOUT: a bounded device wait gave up";
+    }
+    return "unknown acl_status";
+}
+
+int acl_version(void) { return 10000; }
+
+uint64_t acl_launch_count(void) { return acl::g_launches.load(std::memory_order_relaxed); }
+
+acl_status acl_cluster(const float* coords, int B, int N, int C, int32_t* clusters,
+                       acl_stream_t stream) {
+    if (!coords || !clusters) return ACL_ERR_INVALID_ARG;
+    if (B < 1 || N < 1 || C < 1) return ACL_ERR_INVALID_ARG;
+    if (N > ACL_MAX_CLUSTER_N || C > ACL_MAX_CLUSTER_C) return ACL_ERR_UNSUPPORTED;
+    if (acl::cluster_smem_bytes(N, C) > kMaxSmem) return ACL_ERR_UNSUPPORTED;
+    if (!aligned(coords, 8)) return ACL_ERR_INVALID_ARG;
+    return cuda_status(acl::launch_cluster(coords, B, N, C, clusters, S(stream)));
+}
+
+acl_status acl_neighbors(const float* coords, const int32_t* clusters, int B, int N, int C, int M,
+                         int32_t* nbr, acl_stream_t stream) {
+    if (!coords || !clusters || !nbr) return ACL_ERR_INVALID_ARG;
+    if (B < 1 || N < 1 || C < 1 || M < 1 || M % C != 0) return ACL_ERR_INVALID_ARG;
+    if (C > ACL_MAX_CLUSTER_C || M / C > ACL_MAX_NEIGHBOR_R || B > 65535) return ACL_ERR_UNSUPPORTED;
+    const int G = (N + C - 1) / C;
+    if (acl::neighbors_smem_bytes(G) > kMaxSmem) return ACL_ERR_UNSUPPORTED;
+    return cuda_status(acl::launch_neighbors(coords, clusters, B, N, C, M, nbr, S(stream)));
+}
+
+size_t acl_cluster_attn_workspace(int B, int N, int H, int C, int M) {
+    if (B < 1 || N < 1 || H < 1 || C < 1 || M < C || M % C != 0) return 0;
+    return acl::attn_workspace_layout(B, N, H, C, M).total;
+}
+
+acl_status acl_cluster_attn_fwd(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V,
+                                const float* coords, const int32_t* clusters, const int32_t* nbr,
+                                const float* bias_coef, int B, int N, int H, int D, int C, int M,
+                                float scale, acl_bf16* O, float* lse, acl_stream_t stream) {
+    acl_status st = check_attn(Q, K, V, coords, clusters, nbr, bias_coef, B, N, H, D, C, M);
+    if (st != ACL_OK) return st;
+    if (!O || !lse) return ACL_ERR_INVALID_ARG;
+    if (!aligned(O, 16)) return ACL_ERR_INVALID_ARG;
+    acl::AttnArgs a = {};
+    a.q = BF(Q); a.k = BF(K); a.v = BF(V);
+    a.xy = coords; a.clusters = clusters; a.nbr = nbr; a.bias = bias_coef;
+    a.B = B; a.N = N; a.H = H; a.G = (N + C - 1) / C; a.M = M; a.R = M / C;
+    a.scale = scale;
+    a.o = BFm(O); a.lse = lse;
+    return cuda_status(acl::launch_attn_fwd(a, S(stream)));
+}
+
+acl_status acl_cluster_attn_bwd(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V,
+                                const float* coords, const int32_t* clusters, const int32_t* nbr,
+                                const float* bias_coef, int B, int N, int H, int D, int C, int M,
+                                float scale, const acl_bf16* O, const acl_bf16* dO,
+                                const float* lse, acl_bf16* dQ, acl_bf16* dK, acl_bf16* dV,
+                                float* dbias_coef, void* workspace, size_t ws_bytes,
+                                acl_stream_t stream) {
+    acl_status st = check_attn(Q, K, V, coords, clusters, nbr, bias_coef, B, N, H, D, C, M);
+    if (st != ACL_OK) return st;
+    if (!O || !dO || !lse || !dQ || !dK || !dV || !dbias_coef) return ACL_ERR_INVALID_ARG;
+    if (!aligned(O, 16) || !aligned(dO, 16) || !aligned(dQ, 16) || !aligned(dK, 16) ||
+        !aligned(dV, 16))
+        return ACL_ERR_INVALID_ARG;
+    const acl::AttnWorkspace L = acl::attn_workspace_layout(B, N, H, C, M);
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < L.total) return ACL_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    acl::AttnArgs a = {};
+    a.q = BF(Q); a.k = BF(K); a.v = BF(V);
+    a.xy = coords; a.clusters = clusters; a.nbr = nbr; a.bias = bias_coef;
+    a.B = B; a.N = N; a.H = H; a.G = (N + C - 1) / C; a.M = M; a.R = M / C;
+    a.scale = scale;
+    a.o_in = BF(O); a.dout = BF(dO); a.lse_in = lse;
+    a.dq = BFm(dQ); a.dk = BFm(dK); a.dv = BFm(dV); a.dbias = dbias_coef;
+    a.delta = reinterpret_cast<float*>(ws + L.delta);
+    a.dbias_part = reinterpret_cast<float*>(ws + L.dbias_part);
+    a.tok_cluster = reinterpret_cast<int32_t*>(ws + L.tok_cluster);
+    a.rev_off = reinterpret_cast<int32_t*>(ws + L.rev_off);
+    a.rev_list = reinterpret_cast<int32_t*>(ws + L.rev_list);
+    return cuda_status(acl::launch_attn_bwd(a, S(stream)));
+}
+
+acl_status acl_knn_table(const float* coords, int B, int N, int H, int W, int K, int32_t* table,
+                         acl_stream_t stream) {
+    if (!coords || !table) return ACL_ERR_INVALID_ARG;
+    if (B < 1 || N < 1 || H < 1 || W < 1 || K < 1) return ACL_ERR_INVALID_ARG;
+    if (N > ACL_MAX_TABLE_N || K > ACL_MAX_KNN_K || H > 4096 || W > 4096 || B > 65535)
+        return ACL_ERR_UNSUPPORTED;
+    if (!aligned(coords, 8)) return ACL_ERR_INVALID_ARG;
+    return cuda_status(acl::launch_knn_table(coords, B, N, H, W, K, table, S(stream)));
+}
+
+size_t acl_knn_gather_workspace(int B, int Q, int N, int d, int K) {
+    if (B < 1 || Q < 0 || N < 1 || d < 32 || d % 32 != 0 || K < 1) return 0;
+    return acl::knn_workspace_layout(B, Q, N, d, K).total;
+}
+
+acl_status acl_knn_gather_fwd(const float* queries, int B, int Q, const acl_bf16* feats,
+                              const float* coords, int N, int d, const int32_t* table, int H, int W,
+                              int K, const float* p, acl_bf16* out, acl_stream_t stream) {
+    acl_status st = check_gather(queries, B, Q, feats, coords, N, d, table, H, W, K, p);
+    if (st != ACL_OK) return st;
+    if ((Q > 0 && !out) || !aligned(out, 16)) return ACL_ERR_INVALID_ARG;
+    acl::KnnArgs a = {};
+    a.queries = queries; a.feats = BF(feats); a.xy = coords; a.table = table; a.p = p;
+    a.B = B; a.Q = Q; a.N = N; a.d = d; a.GH = H; a.GW = W; a.K = K;
+    a.out = BFm(out);
+    return cuda_status(acl::launch_knn_fwd(a, S(stream)));
+}
+
+acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16* feats,
+                              const float* coords, int N, int d, const int32_t* table, int H, int W,
+                              int K, const float* p, const acl_bf16* dOut, acl_bf16* dfeats,
+                              float* dqueries, float* dp, void* workspace, size_t ws_bytes,
+                              acl_stream_t stream) {
+    acl_status st = check_gather(queries, B, Q, feats, coords, N, d, table, H, W, K, p);
+    if (st != ACL_OK) return st;
+    if ((Q > 0 && (!dOut || !dqueries)) || !dfeats || !dp) return ACL_ERR_INVALID_ARG;
+    if (!aligned(dOut, 16) || !aligned(dfeats, 16) || !aligned(dqueries, 8)) return ACL_ERR_INVALID_ARG;
+    if (Q > ACL_MAX_GATHER_Q || N > ACL_MAX_TABLE_N) return ACL_ERR_UNSUPPORTED;
+    const acl::KnnWorkspace L = acl::knn_workspace_layout(B, Q, N, d, K);
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < L.total) return ACL_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    acl::KnnArgs a = {};
+    a.queries = queries; a.feats = BF(feats); a.xy = coords; a.table = table; a.p = p;
+    a.B = B; a.Q = Q; a.N = N; a.d = d; a.GH = H; a.GW = W; a.K = K;
+    a.dout = BF(dOut); a.dfeats = BFm(dfeats); a.dq = dqueries; a.dp = dp;
+    a.w = reinterpret_cast<float*>(ws + L.w);
+    a.keys = reinterpret_cast<int32_t*>(ws + L.keys);
+    a.csr = reinterpret_cast<int32_t*>(ws + L.csr);
+    a.csr_off = reinterpret_cast<int32_t*>(ws + L.csr_off);
+    a.dp_part = reinterpret_cast<float*>(ws + L.dp_part);
+    return cuda_status(acl::launch_knn_bwd(a, S(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,116 @@
+// internal.h -- launchers behind the C ABI (not exported).  Each returns the first
+// CUDA error of its launches (cudaSuccess otherwise); argument checks live in api.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "common.cuh"
+
+namespace acl {
+
+// counts every kernel launch issued by the library (see acl_launch_count)
+void note_launch(int n = 1);
+
+// Raise the dynamic shared-memory limit of kernel `Kern` on the current device to at
+// least `bytes`, calling cudaFuncSetAttribute only the first time a larger value is
+// needed on that device (so repeated calls, including calls made while a stream is
+// being captured into a CUDA graph, do no driver work).
+template <auto Kern>
+cudaError_t ensure_smem(size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    static std::atomic<int> done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int want = static_cast<int>(bytes);
+    if (dev < 64 && done[dev].load(std::memory_order_acquire) >= want) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, want);
+    if (e == cudaSuccess && dev < 64) {
+        int cur = done[dev].load(std::memory_order_relaxed);
+        while (cur < want && !done[dev].compare_exchange_weak(cur, want)) {
+        }
+    }
+    return e;
+}
+
+size_t cluster_smem_bytes(int N, int C);
+cudaError_t launch_cluster(const float* xy, int B, int N, int C, int32_t* clusters,
+                           cudaStream_t st);
+size_t neighbors_smem_bytes(int G);
+cudaError_t launch_neighbors(const float* xy, const int32_t* clusters, int B, int N, int C,
+                             int M, int32_t* nbr, cudaStream_t st);
+
+struct AttnArgs {
+    const bf16* q;
+    const bf16* k;
+    const bf16* v;
+    const float* xy;
+    const int32_t* clusters;
+    const int32_t* nbr;
+    const float* bias;
+    int B, N, H, G, M, R;
+    float scale;
+    // forward outputs
+    bf16* o;
+    float* lse;
+    // backward
+    const bf16* o_in;
+    const bf16* dout;
+    const float* lse_in;
+    bf16* dq;
+    bf16* dk;
+    bf16* dv;
+    float* dbias;
+    // backward workspace
+    float* delta;        // [B][N][H]
+    float* dbias_part;   // [B][G][H][3]
+    int32_t* tok_cluster;  // [B][N]
+    int32_t* rev_off;    // [B][G + 1]
+    int32_t* rev_list;   // [B][G * R]
+};
+
+struct AttnWorkspace {
+    size_t delta, dbias_part, tok_cluster, rev_off, rev_list, total;
+};
+AttnWorkspace attn_workspace_layout(int B, int N, int H, int C, int M);
+
+cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_attn_bwd(const AttnArgs& a, cudaStream_t st);
+
+struct KnnArgs {
+    const float* queries;
+    const bf16* feats;
+    const float* xy;
+    const int32_t* table;
+    const float* p;
+    int B, Q, N, d, GH, GW, K;
+    bf16* out;
+    // backward
+    const bf16* dout;
+    bf16* dfeats;
+    float* dq;
+    float* dp;
+    float* w;           // [B][Q][d/32][K]
+    int32_t* keys;      // [B][Q*K]
+    int32_t* csr;       // [B][Q*K]
+    int32_t* csr_off;   // [B][N + 1]
+    float* dp_part;     // [query blocks][d/32]
+};
+
+struct KnnWorkspace {
+    size_t w, keys, csr, csr_off, dp_part, total;
+    int query_blocks;
+};
+KnnWorkspace knn_workspace_layout(int B, int Q, int N, int d, int K);
+
+size_t knn_table_smem_bytes(int N, int nbins);
+cudaError_t launch_knn_table(const float* xy, int B, int N, int GH, int GW, int K,
+                             int32_t* table, cudaStream_t st);
+cudaError_t launch_knn_fwd(const KnnArgs& a, cudaStream_t st);
+cudaError_t launch_knn_bwd(const KnnArgs& a, cudaStream_t st);
+
+}  // namespace acl

@@ -24,3 +24,12 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_sessionstart(session):
+    # build the CUDA library and the oracle in-tree if missing or stale (nvcc and gcc are
+    # available wherever the tests run; the GPU tests then load the in-tree libacl.so)
+    from off_grid_cluster_b200 import build as acl_build
+    from oracle import build as oracle_build
+    acl_build.build()
+    oracle_build.build()

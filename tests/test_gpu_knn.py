@@ -1,0 +1,119 @@
+"""GPU parity of acl_knn_table (bit-exact) and acl_knn_gather_fwd / _bwd with the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import off_grid_cluster_b200 as acl
+import oracle
+from off_grid_cluster_b200 import synth
+from tests.parity import bf16, check_fwd, check_grad, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def table_both(xy: np.ndarray, GH: int, GW: int, K: int) -> np.ndarray:
+    ref = oracle.knn_table(xy, GH, GW, K)
+    got = acl.acl_knn_table(dev(xy), GH, GW, K).cpu().numpy()
+    assert np.array_equal(got, ref), f"table differs ({np.sum(got != ref)} entries)"
+    return ref
+
+
+def gather_both(kb: synth.KnnBatch, bwd: bool = True):
+    table = table_both(kb.coords, kb.GH, kb.GW, kb.K)
+    out_ref = oracle.knn_fwd(kb.queries, kb.feats, kb.coords, table, kb.p)
+    q, f, xy, tt, p = dev(kb.queries), bf16(kb.feats), dev(kb.coords), dev(table), dev(kb.p)
+    out = acl.acl_knn_gather_fwd(q, f, xy, tt, p)
+    stats = check_fwd(host(out), out_ref, "out")
+    if bwd:
+        dF_r, dq_r, dp_r = oracle.knn_bwd(kb.queries, kb.feats, kb.coords, table, kb.p, kb.dout)
+        dF, dq, dp = acl.acl_knn_gather_bwd(q, f, xy, tt, p, bf16(kb.dout))
+        stats["dF"] = check_grad(host(dF), dF_r, "dfeats")
+        stats["dq"] = check_grad(host(dq), dq_r, "dqueries")
+        stats["dp"] = check_grad(host(dp), dp_r, "dp")
+    return stats
+
+
+def test_tables_of_the_decoder_stages():
+    for st in synth.sweep_coords(B=16, wid=synth.WORKLOAD_ID["decoder"]):
+        table_both(st, 64, 64, 8)
+
+
+@pytest.mark.parametrize("N,GH,GW,K", [(1, 8, 8, 8), (5, 16, 16, 8), (7, 9, 13, 16), (300, 64, 64, 1),
+                                       (300, 64, 64, 2), (300, 50, 70, 5), (2048, 64, 64, 16),
+                                       (16384, 64, 64, 8), (64, 256, 256, 8)])
+def test_table_sizes(N, GH, GW, K):
+    xy = synth.uniform(N + 3 * K + GH, 2 * N * 2, -1.0, float(max(GH, GW)) + 1.0)
+    table_both(xy.reshape(2, N, 2).astype(np.float32), GH, GW, K)
+
+
+def test_table_ties_and_out_of_grid():
+    rng = np.random.default_rng(1)
+    xy = rng.integers(-3, 20, size=(2, 400, 2)).astype(np.float32) + 0.5   # duplicates, outside
+    xy[0, :10] = 0.0
+    xy[1, :10] = -0.0
+    table_both(xy, 16, 16, 8)
+
+
+def test_gather_step_workload():
+    # the benchmark workload's gather: 8 images x 4096 queries over 2048 tokens, d = 128
+    sb = synth.step_batch()
+    gather_both(sb.knn)
+
+
+@pytest.mark.parametrize("stage", [0, 1, 2, 3])
+def test_gather_decoder_stage(stage):
+    gather_both(synth.knn_decoder(B=16)[stage])
+
+
+@pytest.mark.parametrize("d,K", [(32, 8), (64, 1), (96, 8), (160, 16), (288, 3), (1024, 8)])
+def test_gather_shapes(d, K):
+    xy = synth.sweep_coords(B=2)[1]
+    kb = synth.knn_batch(xy, d, K=K)
+    gather_both(kb)
+
+
+def test_gather_fewer_tokens_than_k_and_far_queries():
+    xy = synth.sweep_coords(B=2)[3][:, :5]                   # 5 tokens, K = 8
+    kb = synth.knn_batch(np.ascontiguousarray(xy), 64)
+    kb.queries[:, :64] *= np.float32(-1.0)                   # outside the grid
+    kb.queries[:, 64:128] += np.float32(100.0)
+    gather_both(kb)
+
+
+def test_gather_temperature_limits():
+    xy = synth.sweep_coords(B=1)[0]
+    kb = synth.knn_batch(xy, 128)
+    kb.p = np.zeros_like(kb.p)                               # plain mean
+    gather_both(kb)
+    kb.p = np.full_like(kb.p, 60.0)                          # near one-hot
+    gather_both(kb, bwd=False)
+
+
+def test_gather_no_queries():
+    xy = synth.sweep_coords(B=2)[2]
+    kb = synth.knn_batch(xy, 64)
+    table = acl.acl_knn_table(dev(xy))
+    q = torch.zeros(2, 0, 2, device="cuda")
+    f = bf16(kb.feats)
+    out = acl.acl_knn_gather_fwd(q, f, dev(xy), table, dev(kb.p))
+    assert out.shape == (2, 0, 64)
+    dF0 = torch.full_like(f, 7.0)
+    dF, dq, dp = acl.acl_knn_gather_bwd(q, f, dev(xy), table, dev(kb.p),
+                                        torch.zeros(2, 0, 64, dtype=torch.bfloat16, device="cuda"),
+                                        dfeats=dF0)
+    assert torch.count_nonzero(dF) == 0 and torch.count_nonzero(dp) == 0
+
+
+def test_bwd_deterministic_and_overwrites():
+    sb = synth.step_batch(B=2)
+    kb = sb.knn
+    xy = dev(kb.coords)
+    table = acl.acl_knn_table(xy)
+    q, f, p, g = dev(kb.queries), bf16(kb.feats), dev(kb.p), bf16(kb.dout)
+    ws = torch.full((acl.acl_knn_gather_workspace(2, kb.Q, kb.N, kb.d, 8),), 0x55,
+                    dtype=torch.uint8, device="cuda")
+    r1 = acl.acl_knn_gather_bwd(q, f, xy, table, p, g, workspace=ws)
+    outs = [torch.full_like(t, float("nan")) for t in r1]
+    r2 = acl.acl_knn_gather_bwd(q, f, xy, table, p, g, *outs, workspace=ws)
+    for x, y in zip(r1, r2):
+        assert torch.equal(x, y)

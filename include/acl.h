@@ -155,7 +155,10 @@ acl_status acl_cluster_attn_fwd(const acl_bf16* Q, const acl_bf16* K, const acl_
  *   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,
  *   dV_j = sum_i P_ij dO_i,
  *   dbias_coef[h] = (sum dS dx, sum dS dy, -sum dS (dx^2 + dy^2)) over all images.
- * Arguments as in the forward, plus O and lse from it and dO [B][N][H][D] bf16.
+ * Arguments as in the forward, plus lse from it and dO [B][N][H][D] bf16.  O is
+ * accepted for interface symmetry but not read (may be NULL): the whole key row of a
+ * query lies in one tile, so Delta_i is formed as sum_j P_ij dP_ij in fp32, which
+ * equals <dO_i, O_i> without the bf16 rounding of the stored O.
  * dQ, dK, dV [B][N][H][D] bf16 out; dbias_coef [H][3] fp32 out.
  * nbr must be the table acl_neighbors built from `clusters` (each group of C
  * slots is a whole cluster row): dK/dV are reduced per key cluster over the

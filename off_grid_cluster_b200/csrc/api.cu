@@ -124,9 +124,8 @@ acl_status acl_cluster_attn_bwd(const acl_bf16* Q, const acl_bf16* K, const acl_
                                 acl_stream_t stream) {
     acl_status st = check_attn(Q, K, V, coords, clusters, nbr, bias_coef, B, N, H, D, C, M);
     if (st != ACL_OK) return st;
-    if (!O || !dO || !lse || !dQ || !dK || !dV || !dbias_coef) return ACL_ERR_INVALID_ARG;
-    if (!aligned(O, 16) || !aligned(dO, 16) || !aligned(dQ, 16) || !aligned(dK, 16) ||
-        !aligned(dV, 16))
+    if (!dO || !lse || !dQ || !dK || !dV || !dbias_coef) return ACL_ERR_INVALID_ARG;
+    if (!aligned(dO, 16) || !aligned(dQ, 16) || !aligned(dK, 16) || !aligned(dV, 16))
         return ACL_ERR_INVALID_ARG;
     const acl::AttnWorkspace L = acl::attn_workspace_layout(B, N, H, C, M);
     if (!workspace || !aligned(workspace, 256) || ws_bytes < L.total) return ACL_ERR_WORKSPACE;
@@ -136,7 +135,8 @@ acl_status acl_cluster_attn_bwd(const acl_bf16* Q, const acl_bf16* K, const acl_
     a.xy = coords; a.clusters = clusters; a.nbr = nbr; a.bias = bias_coef;
     a.B = B; a.N = N; a.H = H; a.G = (N + C - 1) / C; a.M = M; a.R = M / C;
     a.scale = scale;
-    a.o_in = BF(O); a.dout = BF(dO); a.lse_in = lse;
+    (void)O;  // not read: Delta comes from the recomputed tile
+    a.dout = BF(dO); a.lse_in = lse;
     a.dq = BFm(dQ); a.dk = BFm(dK); a.dv = BFm(dV); a.dbias = dbias_coef;
     a.delta = reinterpret_cast<float*>(ws + L.delta);
     a.dbias_part = reinterpret_cast<float*>(ws + L.dbias_part);

@@ -20,8 +20,10 @@
 // ldmatrix reads without bank conflicts.
 //
 // Backward (recompute, FA2-style, no atomics):
-//   pass 1, query-major (same warp/tile as the forward): Delta = <dO, O>,
-//     recompute P from lse, dP^T = V . dO^T, dS = P (dP - Delta),
+//   pass 1, query-major (same warp/tile as the forward): recompute P from lse,
+//     dP^T = V . dO^T, Delta = rowsum(P o dP) (equal to <dO, O>, but exact in fp32
+//     because the whole key row is in the tile, and O need not be read),
+//     dS = P (dP - Delta),
 //     dQ^T = K^T . dS^T, per-(cluster, head) partial sums of the bias gradient.
 //     B extra CTAs build, per image, the reverse neighbourhood index: for every
 //     key cluster, the query clusters whose table lists it (stable order).
@@ -43,7 +45,7 @@ constexpr int kThreads = 32 * kWarps;
 // ------------------------------------------------------------------ layouts
 
 __host__ __device__ constexpr int fwd_warp_bytes(int MT) { return 140 * MT + 608; }
-__host__ __device__ constexpr int bwdq_warp_bytes(int MT) { return 140 * MT + 1632; }
+__host__ __device__ constexpr int bwdq_warp_bytes(int MT) { return 140 * MT + 1120; }
 constexpr int kBwdKWarpBytes = 3584;
 
 struct FwdTiles {
@@ -145,6 +147,34 @@ __device__ __forceinline__ void xt_b(float (&acc)[2][4], const uint8_t* xs,
     }
 }
 
+// Same as xt_b with B = B_hi + B_lo given as two bf16 fragment sets (a split that keeps
+// about 16 significant bits of B): each A fragment is loaded once and used twice.
+template <int MTILES>
+__device__ __forceinline__ void xt_b2(float (&acc)[2][4], const uint8_t* xs,
+                                      const uint32_t (&bhi)[MTILES][2],
+                                      const uint32_t (&blo)[MTILES][2], int lane) {
+    const int mi = lane >> 3;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+#pragma unroll
+        for (int i = 0; i < MTILES; ++i) {
+            const int row = 16 * i + (lane & 7) + 8 * (mi >> 1);
+            const int ch = 2 * m + (mi & 1);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(smem_addr(xs) + tile64_off(row, ch), a0, a1, a2, a3);
+            mma_bf16(acc[m], a0, a1, a2, a3, blo[i][0], blo[i][1]);
+            mma_bf16(acc[m], a0, a1, a2, a3, bhi[i][0], bhi[i][1]);
+        }
+    }
+}
+
+// bf16 pair (hi) of two floats and the bf16 pair of their remainders (lo).
+__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    hi = pack_bf16(x0, x1);
+    lo = pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
+}
+
 // Write an (e x 8-token) fp32 accumulator pair, transposed to token rows, as bf16 rows of
 // `dst` (token-major [tok][H][32]) through a 512-byte staging tile.
 __device__ __forceinline__ void store_rows_t(const float (&acc)[2][4], float s0, float s1,
@@ -236,23 +266,30 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_kernel(const AttnArgs a) {
     const float m0 = (mx0 == -INFINITY) ? 0.f : mx0;
     const float m1 = (mx1 == -INFINITY) ? 0.f : mx1;
     float l0 = 0.f, l1 = 0.f;
-    uint32_t pb[MTILES][2];
+    uint32_t pbh[MTILES][2], pbl[MTILES][2];
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) {
         const float p0 = exp2f(s[i][0] - m0), p1 = exp2f(s[i][1] - m1);
         const float p2 = exp2f(s[i][2] - m0), p3 = exp2f(s[i][3] - m1);
         l0 += p0 + p2;
         l1 += p1 + p3;
-        pb[i][0] = movm_t(pack_bf16(p0, p1));
-        pb[i][1] = movm_t(pack_bf16(p2, p3));
+        uint32_t h01, l01, h23, l23;
+        split_bf16(p0, p1, h01, l01);
+        split_bf16(p2, p3, h23, l23);
+        pbh[i][0] = movm_t(h01);
+        pbl[i][0] = movm_t(l01);
+        pbh[i][1] = movm_t(h23);
+        pbl[i][1] = movm_t(l23);
     }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
         l0 += __shfl_xor_sync(0xffffffffu, l0, o);
         l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
+    // P is split into bf16 hi + lo parts so that rounding P costs ~2^-17 relative
+    // instead of 2^-9; the output's own bf16 rounding is then the only visible error.
     float oacc[2][4];
-    xt_b<MTILES>(oacc, t.vs, pb, lane);
+    xt_b2<MTILES>(oacc, t.vs, pbh, pbl, lane);
     const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
     const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
     store_rows_t(oacc, i0, i1, t.qs, t.qid, tok0, a.H, h, a.o, lane);
@@ -376,7 +413,6 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_query_kernel(const AttnArgs
     uint8_t* w = smem + warp * bwdq_warp_bytes(MT);
     const FwdTiles t = fwd_tiles(w, MT);
     uint8_t* dos = w + fwd_warp_bytes(MT);
-    uint8_t* os = dos + 512;
     const size_t tok0 = static_cast<size_t>(b) * a.N;
     const int H = a.H;
 
@@ -386,32 +422,12 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_query_kernel(const AttnArgs
         const int id = t.qid[row];
         const size_t off = ((tok0 + (id >= 0 ? id : 0)) * H + h) * 32 + ch * 8;
         cp_async16(smem_addr(dos) + tile64_off(row, ch), a.dout + off, id >= 0);
-        cp_async16(smem_addr(os) + tile64_off(row, ch), a.o_in + off, id >= 0);
     }
     cp_async_commit();
     cp_async_wait<0>();
     __syncwarp();
 
     const int gq = lane >> 2, tq = lane & 3;
-    // Delta_i = <dO_i, O_i>: lane -> (row lane/4, 8 channels)
-    float dsum;
-    {
-        const int row = lane >> 2, ch = lane & 3;
-        const uint4 dv = *reinterpret_cast<const uint4*>(dos + tile64_off(row, ch));
-        const uint4 ov = *reinterpret_cast<const uint4*>(os + tile64_off(row, ch));
-        const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
-        const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
-        dsum = 0.f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            dsum += bf16_lo(dw[j]) * bf16_lo(ow[j]) + bf16_hi(dw[j]) * bf16_hi(ow[j]);
-        dsum += __shfl_xor_sync(0xffffffffu, dsum, 1);
-        dsum += __shfl_xor_sync(0xffffffffu, dsum, 2);
-        const int id = t.qid[row];
-        if (ch == 0 && id >= 0) a.delta[(tok0 + id) * H + h] = dsum;
-    }
-    const float dl0 = __shfl_sync(0xffffffffu, dsum, (2 * tq) * 4);
-    const float dl1 = __shfl_sync(0xffffffffu, dsum, (2 * tq + 1) * 4);
     const int q0 = t.qid[2 * tq], q1 = t.qid[2 * tq + 1];
     float L0 = q0 >= 0 ? a.lse_in[(tok0 + q0) * H + h] * kLog2e : INFINITY;
     float L1 = q1 >= 0 ? a.lse_in[(tok0 + q1) * H + h] * kLog2e : INFINITY;
@@ -429,11 +445,11 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_query_kernel(const AttnArgs
     const float ba = a.bias[3 * h] * kLog2e, bb = a.bias[3 * h + 1] * kLog2e,
                 bc = a.bias[3 * h + 2] * kLog2e;
     const float2 qa = t.qxy[2 * tq], qb = t.qxy[2 * tq + 1];
-    float ga = 0.f, gb = 0.f, gc = 0.f;
-    uint32_t db[MTILES][2];
+    // P from the forward's lse; Delta_i = sum_j P_ij dP_ij (= <dO_i, O_i> exactly, since
+    // the whole key row is in this tile -- no bf16-rounded O enters the gradient)
+    float pd0 = 0.f, pd1 = 0.f;
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) {
-        float ds[4];
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi) {
             const int key = 16 * i + gq + 8 * hi;
@@ -443,15 +459,43 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_query_kernel(const AttnArgs
             for (int qq = 0; qq < 2; ++qq) {
                 const float2 qp = qq ? qb : qa;
                 const float dx = kp.x - qp.x, dy = kp.y - qp.y;
-                const float r2 = dx * dx + dy * dy;
                 const int j = 2 * hi + qq;
-                const float lg = s[i][j] * sc + ba * dx + bb * dy - bc * r2;
+                const float lg = s[i][j] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
                 const float p = kv ? exp2f(lg - (qq ? L1 : L0)) : 0.f;
-                const float v = p * (dp[i][j] - (qq ? dl1 : dl0));
+                s[i][j] = p;
+                if (qq) pd1 += p * dp[i][j];
+                else pd0 += p * dp[i][j];
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        pd0 += __shfl_xor_sync(0xffffffffu, pd0, o);
+        pd1 += __shfl_xor_sync(0xffffffffu, pd1, o);
+    }
+    if (gq == 0) {
+        if (q0 >= 0) a.delta[(tok0 + q0) * H + h] = pd0;
+        if (q1 >= 0) a.delta[(tok0 + q1) * H + h] = pd1;
+    }
+    float ga = 0.f, gb = 0.f, gc = 0.f;
+    uint32_t db[MTILES][2];
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+        float ds[4];
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+            const int key = 16 * i + gq + 8 * hi;
+            const float2 kp = t.kxy[key];
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                const float2 qp = qq ? qb : qa;
+                const float dx = kp.x - qp.x, dy = kp.y - qp.y;
+                const int j = 2 * hi + qq;
+                const float v = s[i][j] * (dp[i][j] - (qq ? pd1 : pd0));
                 ds[j] = v;
                 ga += v * dx;
                 gb += v * dy;
-                gc += v * r2;
+                gc += v * (dx * dx + dy * dy);
             }
         }
         db[i][0] = movm_t(pack_bf16(ds[0], ds[1]));

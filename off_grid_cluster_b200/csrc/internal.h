@@ -58,7 +58,6 @@ struct AttnArgs {
     bf16* o;
     float* lse;
     // backward
-    const bf16* o_in;
     const bf16* dout;
     const float* lse_in;
     bf16* dq;

@@ -79,6 +79,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--serial", action="store_true",
+                    help="run all seven calls on one stream (default: the attention and KNN "
+                         "chains run as two concurrent branches of the step graph)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bounded CPU work of the oracle baseline (seconds)")
     return ap.parse_args(argv)
@@ -248,13 +251,31 @@ class StepSet:
         else:
             raise KeyError(name)
 
-    def step(self, stream, events=None):
+    def step(self, stream, events=None, stream2=None):
+        """The seven calls.  With stream2 the KNN chain (table -> gather fwd -> bwd) runs
+        on stream2 concurrently with the attention chain (cluster -> neighbours -> attn
+        fwd -> bwd) on stream; events[2j], events[2j+1] bracket call j on its stream."""
+        if stream2 is None:
+            for j, name in enumerate(OPS):
+                if events is not None:
+                    events[2 * j].record(stream)
+                self.op(name, stream)
+                if events is not None:
+                    events[2 * j + 1].record(stream)
+            return
+        torch = self.torch
+        fork, join = torch.cuda.Event(), torch.cuda.Event()
+        fork.record(stream)
+        stream2.wait_event(fork)
         for j, name in enumerate(OPS):
+            st = stream2 if name.startswith("knn") else stream
             if events is not None:
-                events[j].record(stream)
-            self.op(name, stream)
-        if events is not None:
-            events[len(OPS)].record(stream)
+                events[2 * j].record(st)
+            self.op(name, st)
+            if events is not None:
+                events[2 * j + 1].record(st)
+        join.record(stream2)
+        stream.wait_event(join)
 
 
 def run_gpu(args, rank: int, world: int):
@@ -284,20 +305,21 @@ def run_gpu(args, rank: int, world: int):
     n_sets = max(2, math.ceil(4 * l2 / set_bytes))
     sets = [base] + [StepSet(sb, device, acl, torch) for _ in range(n_sets - 1)]
     stream = torch.cuda.Stream(device)
+    stream2 = None if args.serial else torch.cuda.Stream(device)
 
     # eager warm-up of every call (kernel attributes, lazy module loading), then capture
     with torch.cuda.stream(stream):
         for s in sets:
             s.step(stream)
     stream.synchronize()
-    n_ev = len(OPS) + 1
+    n_ev = 2 * len(OPS)
     graphs, events = [], []
     launches0 = acl.acl_launch_count()
     for s in sets:
         evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            s.step(stream, evs)
+            s.step(stream, evs, stream2)
         graphs.append(g)
         events.append(evs)
     launches_per_step = (acl.acl_launch_count() - launches0) // len(sets)
@@ -327,7 +349,7 @@ def run_gpu(args, rank: int, world: int):
     used = min(n_sets, args.steps)
     for s_i in range(used):
         ev = events[s_i]
-        per_op += np.array([ev[j].elapsed_time(ev[j + 1]) for j in range(len(OPS))])
+        per_op += np.array([ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(len(OPS))])
     per_op /= max(used, 1)
     # keep the same load on the GPU until the clock sampler has several samples
     t_wall = time.time()
@@ -383,6 +405,7 @@ def run_gpu(args, rank: int, world: int):
                    "l2": f"rotating {n_sets} input sets, {n_sets * set_bytes / 1e6:.0f} MB total "
                          f">= 4 x L2 ({l2 / 1e6:.0f} MB)",
                    "timing": "CUDA graph per set, CUDA events on the launching stream",
+                   "streams": 1 if args.serial else 2,
                    "parallelism": f"replicas x{world} (images sharded, no collective)"},
         "parts": {
             "knn_queries_per_s": round(world * B * Q / (step_ms * 1e-3), 1),

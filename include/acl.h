@@ -140,7 +140,8 @@ size_t acl_cluster_attn_workspace(int B, int N, int H, int C, int M);
  * Rows of tokens that no cluster lists are left untouched; a token whose
  * neighbourhood is empty gets O = 0 and lse = -inf.
  * Arithmetic: bf16 tensor-core products with fp32 accumulation, fp32 softmax.
- * Limits: D == 32, C == 8, M % 8 == 0, 8 <= M <= 64, 1 <= H <= 64.
+ * Limits: D == 32, C == 8, M % 8 == 0, 8 <= M <= 64, 1 <= H <= 1024, B <= 65535,
+ *         N <= 262144.
  */
 acl_status acl_cluster_attn_fwd(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V,
                                 const float* coords, const int32_t* clusters,

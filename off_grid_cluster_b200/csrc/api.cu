@@ -33,7 +33,8 @@ acl_status check_attn(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V, c
     if (!Q || !K || !V || !coords || !clusters || !nbr || !bias) return ACL_ERR_INVALID_ARG;
     if (B < 1 || N < 1 || H < 1 || D < 1 || C < 1 || M < 1) return ACL_ERR_INVALID_ARG;
     if (M % C != 0) return ACL_ERR_INVALID_ARG;
-    if (D != ACL_ATTN_D || C != ACL_ATTN_C || M > ACL_ATTN_MAX_M || H > 1024 || N > kMaxAttnN)
+    if (D != ACL_ATTN_D || C != ACL_ATTN_C || M > ACL_ATTN_MAX_M || H > 1024 || N > kMaxAttnN ||
+        B > 65535)
         return ACL_ERR_UNSUPPORTED;
     if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(coords, 8))
         return ACL_ERR_INVALID_ARG;
@@ -196,6 +197,7 @@ acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16
     a.csr = reinterpret_cast<int32_t*>(ws + L.csr);
     a.csr_off = reinterpret_cast<int32_t*>(ws + L.csr_off);
     a.dp_part = reinterpret_cast<float*>(ws + L.dp_part);
+    a.counter = reinterpret_cast<int*>(ws + L.counter);
     return cuda_status(acl::launch_knn_bwd(a, S(stream)));
 }
 

@@ -15,22 +15,28 @@
 //   S^T (M x 8)  = K (M x 32) . Q^T          -- 2 k-steps per 16-key tile
 //   O^T (32 x 8) = V^T (32 x M) . P^T        -- P^T comes from the S^T
 //                  accumulators by an in-register 8x8 transpose (movmatrix)
-// so no tile is padded beyond M's rounding to 16.  K, V and Q rows are gathered
-// by token id (nbr) with 16-byte cp.async into XOR-swizzled shared tiles that
-// ldmatrix reads without bank conflicts.
+// so no tile is padded beyond M's rounding to 16.
+//
+// A CTA runs kUC = 4 consecutive clusters x kUH = 2 heads (8 warps).  Consecutive
+// clusters are siblings of the bisection tree and their neighbourhoods overlap, so the
+// CTA gathers the union of the group's neighbour blocks once (16-byte cp.async of
+// 128-byte token rows = the two heads) into XOR-swizzled shared tiles, and each warp
+// addresses its own 48 keys inside the union through a block map; ldmatrix reads them
+// without bank conflicts.  This halves the L2 -> SM traffic of the 6x-reused rows.
 //
 // Backward (recompute, FA2-style, no atomics):
-//   pass 1, query-major (same warp/tile as the forward): recompute P from lse,
+//   pass 1, query-major (same CTA shape as the forward): recompute P from lse,
 //     dP^T = V . dO^T, Delta = rowsum(P o dP) (equal to <dO, O>, but exact in fp32
 //     because the whole key row is in the tile, and O need not be read),
-//     dS = P (dP - Delta),
-//     dQ^T = K^T . dS^T, per-(cluster, head) partial sums of the bias gradient.
-//     B extra CTAs build, per image, the reverse neighbourhood index: for every
-//     key cluster, the query clusters whose table lists it (stable order).
-//   pass 2, key-major: one warp per (image, key cluster, head) walks its reverse
-//     list two query clusters at a time (16 queries = one MMA M tile):
-//     S = Q K_h^T, dP = dO V_h^T, dV^T += dO^T P, dK^T += Q^T dS; 3H extra CTAs
-//     reduce the bias-gradient partials in a fixed order.
+//     dS = P (dP - Delta), dQ^T = K^T . dS^T, per-(cluster, head) partial sums of the
+//     bias gradient.  One extra column of CTAs builds, per image, the reverse
+//     neighbourhood index: for every key cluster, the query clusters that list it.
+//   pass 2, key-major: CTA = 4 key clusters x 2 heads; the union of the query clusters
+//     in their reverse lists is gathered once, and each warp walks its own list two
+//     query clusters at a time (16 queries = one MMA M tile): S = Q K_h^T,
+//     dP = dO V_h^T, dV^T += dO^T P, dK^T += Q^T dS.  Extra CTAs reduce the bias
+//     partials in a fixed order.  A group whose lists overflow the union tile falls back
+//     to per-warp direct loads.
 #include <math.h>
 
 #include "internal.h"
@@ -39,137 +45,13 @@ namespace acl {
 
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
 
 // ------------------------------------------------------------------ layouts
 
-__host__ __device__ constexpr int fwd_warp_bytes(int MT) { return 140 * MT + 608; }
-__host__ __device__ constexpr int bwdq_warp_bytes(int MT) { return 140 * MT + 1120; }
 constexpr int kBwdKWarpBytes = 3584;
 
-struct FwdTiles {
-    uint8_t* ks;
-    uint8_t* vs;
-    uint8_t* qs;
-    int* kid;
-    float2* kxy;
-    int* qid;
-    float2* qxy;
-};
-
-__device__ __forceinline__ FwdTiles fwd_tiles(uint8_t* w, int MT) {
-    FwdTiles t;
-    t.ks = w;
-    t.vs = w + MT * 64;
-    t.qs = w + 2 * MT * 64;
-    t.kid = reinterpret_cast<int*>(w + 2 * MT * 64 + 512);
-    t.kxy = reinterpret_cast<float2*>(t.kid + MT);
-    t.qid = reinterpret_cast<int*>(t.kxy + MT);
-    t.qxy = reinterpret_cast<float2*>(t.qid + 8);
-    return t;
-}
-
-// Gather the ids/coordinates of a (cluster, neighbourhood) and issue the cp.async of
-// K, V (and Q) rows of head h.  Empty slots are zero-filled.
-template <int MT>
-__device__ __forceinline__ void load_cluster_tiles(const AttnArgs& a, int b, int g, int h, int lane,
-                                                   const FwdTiles& t, const bf16* qsrc) {
-    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(b) * a.N;
-    const int32_t* nrow = a.nbr + (static_cast<size_t>(b) * a.G + g) * a.M;
-    for (int m = lane; m < MT; m += 32) {
-        int id = (m < a.M) ? nrow[m] : -1;
-        if (id < 0 || id >= a.N) id = -1;
-        t.kid[m] = id;
-        t.kxy[m] = (id >= 0) ? xyb[id] : make_float2(0.f, 0.f);
-    }
-    if (lane < 8) {
-        int id = a.clusters[(static_cast<size_t>(b) * a.G + g) * 8 + lane];
-        if (id < 0 || id >= a.N) id = -1;
-        t.qid[lane] = id;
-        t.qxy[lane] = (id >= 0) ? xyb[id] : make_float2(0.f, 0.f);
-    }
-    __syncwarp();
-    const size_t tok0 = static_cast<size_t>(b) * a.N;
-    const int H = a.H;
-#pragma unroll
-    for (int c = lane; c < MT * 4; c += 32) {
-        const int row = c >> 2, ch = c & 3;
-        const int id = t.kid[row];
-        const size_t off = ((tok0 + (id >= 0 ? id : 0)) * H + h) * 32 + ch * 8;
-        cp_async16(smem_addr(t.ks) + tile64_off(row, ch), a.k + off, id >= 0);
-        cp_async16(smem_addr(t.vs) + tile64_off(row, ch), a.v + off, id >= 0);
-    }
-    {
-        const int row = lane >> 2, ch = lane & 3;
-        const int id = t.qid[row];
-        const size_t off = ((tok0 + (id >= 0 ? id : 0)) * H + h) * 32 + ch * 8;
-        cp_async16(smem_addr(t.qs) + tile64_off(row, ch), qsrc + off, id >= 0);
-    }
-}
-
-// S^T = K . Q^T for all MT/16 key tiles (raw dot products).
-template <int MTILES>
-__device__ __forceinline__ void qk_tiles(float (&s)[MTILES][4], const uint8_t* ks, uint32_t qf0,
-                                         uint32_t qf1, uint32_t qf2, uint32_t qf3, int lane) {
-    const int mi = lane >> 3;
-#pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-        s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            const int row = 16 * i + (lane & 7) + 8 * (mi & 1);
-            const int ch = 2 * kk + (mi >> 1);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(smem_addr(ks) + tile64_off(row, ch), a0, a1, a2, a3);
-            mma_bf16(s[i], a0, a1, a2, a3, kk ? qf2 : qf0, kk ? qf3 : qf1);
-        }
-    }
-}
-
-// acc^T (32 x 8) += X^T (32 x MT) . B^T where X is an MT x 32 row tile and bfr holds the
-// transposed (k-major) B fragments of the MT x 8 matrix.
-template <int MTILES>
-__device__ __forceinline__ void xt_b(float (&acc)[2][4], const uint8_t* xs,
-                                     const uint32_t (&bfr)[MTILES][2], int lane) {
-    const int mi = lane >> 3;
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-        acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
-#pragma unroll
-        for (int i = 0; i < MTILES; ++i) {
-            const int row = 16 * i + (lane & 7) + 8 * (mi >> 1);
-            const int ch = 2 * m + (mi & 1);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(smem_addr(xs) + tile64_off(row, ch), a0, a1, a2, a3);
-            mma_bf16(acc[m], a0, a1, a2, a3, bfr[i][0], bfr[i][1]);
-        }
-    }
-}
-
-// Same as xt_b with B = B_hi + B_lo given as two bf16 fragment sets (a split that keeps
-// about 16 significant bits of B): each A fragment is loaded once and used twice.
-template <int MTILES>
-__device__ __forceinline__ void xt_b2(float (&acc)[2][4], const uint8_t* xs,
-                                      const uint32_t (&bhi)[MTILES][2],
-                                      const uint32_t (&blo)[MTILES][2], int lane) {
-    const int mi = lane >> 3;
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-        acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
-#pragma unroll
-        for (int i = 0; i < MTILES; ++i) {
-            const int row = 16 * i + (lane & 7) + 8 * (mi >> 1);
-            const int ch = 2 * m + (mi & 1);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(smem_addr(xs) + tile64_off(row, ch), a0, a1, a2, a3);
-            mma_bf16(acc[m], a0, a1, a2, a3, blo[i][0], blo[i][1]);
-            mma_bf16(acc[m], a0, a1, a2, a3, bhi[i][0], bhi[i][1]);
-        }
-    }
-}
-
-// bf16 pair (hi) of two floats and the bf16 pair of their remainders (lo).
+// bf16 pair (hi) of two floats and the bf16 pair of their remainders (lo): hi + lo keeps
+// about 16 significant bits.
 __device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uint32_t& lo) {
     hi = pack_bf16(x0, x1);
     lo = pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
@@ -208,54 +90,223 @@ __device__ __forceinline__ void store_rows_t1(const float (&acc)[2][4], float s,
     store_rows_t(acc, s, s, stage, ids, tok0, H, h, dst, lane);
 }
 
-// --------------------------------------------------------------- forward
+// ------------------------------------------------- forward, neighbourhood unions
+//
+// One CTA per (image, group of kUC consecutive clusters, group of kUH heads); warp w owns
+// cluster w / kUH and head w % kUH of the group.  Consecutive clusters are siblings of the
+// bisection tree, so their neighbourhoods overlap: the CTA de-duplicates the group's
+// neighbour blocks (a block is one whole cluster, named by its first token), gathers each
+// union row's K and V once (kUH heads = 128 contiguous bytes per token) and every warp
+// reads its own neighbourhood out of the union tile through a block map.  Rows are
+// 128 bytes with the 16-byte chunk index XOR-ed by (row & 7); a neighbourhood block is 8
+// consecutive union rows, so the 8 rows of every ldmatrix hit 8 distinct bank groups.
+// Empty blocks map to 8 zero rows at the end of the tile.
+constexpr int kUC = 4;
+constexpr int kUH = 2;
+constexpr int kUWarps = kUC * kUH;
+constexpr int kUThreads = 32 * kUWarps;
+constexpr int kURow = 64 * kUH;  // bytes per union row
+
+struct UnionLayout {
+    int ks, vs, qs, stage, blk, utok, uxy, qtok, qxy, krow, nu, total;
+};
+__host__ __device__ __forceinline__ UnionLayout union_layout(int R, int MT) {
+    UnionLayout L;
+    const int rows = kUC * R * 8 + 8;  // union rows + a zero block
+    int o = 0;
+    L.ks = o; o += rows * kURow;
+    L.vs = o; o += rows * kURow;
+    L.qs = o; o += kUC * 8 * kURow;
+    L.stage = o; o += kUWarps * 512;
+    L.blk = o; o += 4 * kUC * R * 2;       // first token, union index
+    L.utok = o; o += 4 * (rows - 8);
+    L.uxy = o; o += 8 * (rows - 8);
+    L.qtok = o; o += 4 * kUC * 8;
+    L.qxy = o; o += 8 * kUC * 8;
+    L.krow = o; o += 4 * kUC * MT;
+    L.nu = o; o += 16;
+    L.total = (o + 15) & ~15;
+    return L;
+}
+
+__device__ __forceinline__ uint32_t urow_off(int row, int ch) {
+    return static_cast<uint32_t>(row * kURow + ((ch ^ (row & 7)) << 4));
+}
 
 template <int MTILES>
-__global__ void __launch_bounds__(kThreads) attn_fwd_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kUThreads) attn_fwd_union_kernel(const AttnArgs a) {
     constexpr int MT = 16 * MTILES;
     extern __shared__ __align__(16) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long task = static_cast<long long>(blockIdx.x) * kWarps + warp;
-    if (task >= static_cast<long long>(a.B) * a.G * a.H) return;
-    const int h = static_cast<int>(task % a.H);
-    const long long bg = task / a.H;
-    const int g = static_cast<int>(bg % a.G), b = static_cast<int>(bg / a.G);
-    const FwdTiles t = fwd_tiles(smem + warp * fwd_warp_bytes(MT), MT);
-    const size_t tok0 = static_cast<size_t>(b) * a.N;
+    const int R = a.R;
+    const UnionLayout L = union_layout(R, MT);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int cg = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+    const int G = a.G, N = a.N, H = a.H, M = a.M;
+    const int g0 = cg * kUC;
+    const int nblk = kUC * R;
+    const int ZR = nblk * 8;
+    uint8_t* ks = smem + L.ks;
+    uint8_t* vs = smem + L.vs;
+    uint8_t* qs = smem + L.qs;
+    int* blk_first = reinterpret_cast<int*>(smem + L.blk);
+    int* ublk = blk_first + nblk;
+    int* utok = reinterpret_cast<int*>(smem + L.utok);
+    float2* uxy = reinterpret_cast<float2*>(smem + L.uxy);
+    int* qtok = reinterpret_cast<int*>(smem + L.qtok);
+    float2* qxy = reinterpret_cast<float2*>(smem + L.qxy);
+    int* krow = reinterpret_cast<int*>(smem + L.krow);
+    int* nu_s = reinterpret_cast<int*>(smem + L.nu);
+    const size_t tok0 = static_cast<size_t>(b) * N;
+    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + tok0;
 
-    load_cluster_tiles<MT>(a, b, g, h, lane, t, a.q);
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncwarp();
+    // 1. neighbour blocks and query tokens of the group
+    for (int i = tid; i < nblk; i += kUThreads) {
+        const int g = g0 + i / R, r = i % R;
+        int f = -1;
+        if (g < G) {
+            f = a.nbr[(static_cast<size_t>(b) * G + g) * M + r * 8];
+            if (f < 0 || f >= N) f = -1;
+        }
+        blk_first[i] = f;
+    }
+    for (int i = tid; i < kUC * 8; i += kUThreads) {
+        const int g = g0 + (i >> 3);
+        int id = -1;
+        if (g < G) {
+            id = a.clusters[(static_cast<size_t>(b) * G + g) * 8 + (i & 7)];
+            if (id < 0 || id >= N) id = -1;
+        }
+        qtok[i] = id;
+        qxy[i] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
+    }
+    __syncthreads();
+    // 2. de-duplicate the blocks (one warp; nblk <= 32)
+    if (warp == 0) {
+        const int f = lane < nblk ? blk_first[lane] : -1;
+        int dup = -1;
+        for (int j = 0; j < nblk; ++j) {
+            const int fj = __shfl_sync(0xffffffffu, f, j);
+            if (j < lane && dup < 0 && f >= 0 && fj == f) dup = j;
+        }
+        const bool isnew = f >= 0 && dup < 0;
+        const unsigned newmask = __ballot_sync(0xffffffffu, isnew);
+        int u = isnew ? __popc(newmask & ((1u << lane) - 1u)) : -1;
+        const int ud = __shfl_sync(0xffffffffu, u, dup >= 0 ? dup : 0);
+        if (dup >= 0) u = ud;
+        if (lane < nblk) ublk[lane] = isnew ? u : (dup >= 0 ? -(u + 2) : -1);  // -(u+2): duplicate
+        if (lane == 0) nu_s[0] = __popc(newmask);
+    }
+    __syncthreads();
+    const int nU = nu_s[0];
+    // 3. union row tokens (from the first occurrence of each block) and the block map
+    for (int i = tid; i < nblk * 8; i += kUThreads) {
+        const int blk = i >> 3, sl = i & 7;
+        const int u = ublk[blk];
+        if (u >= 0) {
+            const int g = g0 + blk / R, r = blk % R;
+            int t = a.nbr[(static_cast<size_t>(b) * G + g) * M + r * 8 + sl];
+            if (t < 0 || t >= N) t = -1;
+            utok[u * 8 + sl] = t;
+            uxy[u * 8 + sl] = t >= 0 ? xyb[t] : make_float2(0.f, 0.f);
+        }
+    }
+    for (int i = tid; i < kUC * MT; i += kUThreads) {
+        const int cw = i / MT, m = i % MT;
+        int row = -1;
+        if (m < M) {
+            int u = ublk[cw * R + (m >> 3)];
+            if (u < -1) u = -u - 2;
+            if (u >= 0) row = u * 8 + (m & 7);
+        }
+        krow[i] = row;
+    }
+    __syncthreads();
+    // 4. gather the union's K and V rows, the group's Q rows, and zero the spare block
+    const int hlo = hg * kUH;
+    for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
+        const int row = i >> 3, ch = i & 7;
+        const int t = row < nU * 8 ? utok[row] : -1;
+        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
+        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
+        const int drow = row < nU * 8 ? row : ZR + (row - nU * 8);
+        cp_async16(smem_addr(ks) + urow_off(drow, ch), a.k + (ok ? off : 0), ok);
+    }
+    for (int i = tid; i < kUC * 8 * 8; i += kUThreads) {
+        const int row = i >> 3, ch = i & 7;
+        const int t = qtok[row];
+        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
+        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
+        cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + (ok ? off : 0), ok);
+    }
+    cp_async_commit();  // group 0: K, Q
+    for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
+        const int row = i >> 3, ch = i & 7;
+        const int t = row < nU * 8 ? utok[row] : -1;
+        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
+        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
+        const int drow = row < nU * 8 ? row : ZR + (row - nU * 8);
+        cp_async16(smem_addr(vs) + urow_off(drow, ch), a.v + (ok ? off : 0), ok);
+    }
+    cp_async_commit();  // group 1: V (lands while S and the softmax run)
+    cp_async_wait<1>();
+    __syncthreads();
 
-    const int gq = lane >> 2, tq = lane & 3;
+    // 5. one (cluster, head) per warp
+    const int cw = warp / kUH, hw = warp % kUH;
+    const int g = g0 + cw;
+    // a warp past the last cluster or head computes on masked data and stores nothing (it
+    // must still reach the barrier before the V tile is read)
+    const bool active = g < G && hlo + hw < H;
+    const int h = active ? hlo + hw : 0;
+    const int gq = lane >> 2, tq = lane & 3, mi = lane >> 3;
+    const int* kr = krow + cw * MT;
+    // row bases of the neighbourhood blocks this lane addresses
+    // row 0 of each neighbourhood block this lane addresses: (mi & 1) picks the block of
+    // the S / dQ operands, (mi >> 1) the block of the transposed V / K operands
+    int base_s[MTILES], base_t[MTILES];
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+        const int s0 = 2 * i + (mi & 1), s1 = 2 * i + (mi >> 1);
+        const int r0 = (s0 * 8 < a.M) ? kr[s0 * 8] : -1;
+        const int r1 = (s1 * 8 < a.M) ? kr[s1 * 8] : -1;
+        base_s[i] = r0 >= 0 ? r0 : ZR;
+        base_t[i] = r1 >= 0 ? r1 : ZR;
+    }
     uint32_t qf0, qf1, qf2, qf3;
-    ldsm_x4(smem_addr(t.qs) + tile64_off(lane & 7, lane >> 3), qf0, qf1, qf2, qf3);
-    float s[MTILES][4];
-    qk_tiles<MTILES>(s, t.ks, qf0, qf1, qf2, qf3, lane);
-
-    // logits in log2 units
+    ldsm_x4(smem_addr(qs) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), qf0, qf1, qf2, qf3);
+    float sacc[MTILES][4];
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+        sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const int row = base_s[i] + (lane & 7);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(smem_addr(ks) + urow_off(row, hw * 4 + 2 * kk + (mi >> 1)), a0, a1, a2, a3);
+            mma_bf16(sacc[i], a0, a1, a2, a3, kk ? qf2 : qf0, kk ? qf3 : qf1);
+        }
+    }
     const float sc = a.scale * kLog2e;
     const float ba = a.bias[3 * h] * kLog2e, bb = a.bias[3 * h + 1] * kLog2e,
                 bc = a.bias[3 * h + 2] * kLog2e;
-    const float2 qa = t.qxy[2 * tq], qb = t.qxy[2 * tq + 1];
+    const float2 qa = qxy[cw * 8 + 2 * tq], qb = qxy[cw * 8 + 2 * tq + 1];
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) {
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi) {
-            const int key = 16 * i + gq + 8 * hi;
-            const bool kv = t.kid[key] >= 0;
-            const float2 kp = t.kxy[key];
+            const int row = kr[16 * i + gq + 8 * hi];
+            const bool kv = row >= 0 && utok[row] >= 0;
+            const float2 kp = kv ? uxy[row] : make_float2(0.f, 0.f);
             float dx = kp.x - qa.x, dy = kp.y - qa.y;
-            const float v0 = s[i][2 * hi] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
+            const float v0 = sacc[i][2 * hi] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
             dx = kp.x - qb.x;
             dy = kp.y - qb.y;
-            const float v1 = s[i][2 * hi + 1] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
-            s[i][2 * hi] = kv ? v0 : -INFINITY;
-            s[i][2 * hi + 1] = kv ? v1 : -INFINITY;
-            mx0 = fmaxf(mx0, s[i][2 * hi]);
-            mx1 = fmaxf(mx1, s[i][2 * hi + 1]);
+            const float v1 = sacc[i][2 * hi + 1] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
+            sacc[i][2 * hi] = kv ? v0 : -INFINITY;
+            sacc[i][2 * hi + 1] = kv ? v1 : -INFINITY;
+            mx0 = fmaxf(mx0, sacc[i][2 * hi]);
+            mx1 = fmaxf(mx1, sacc[i][2 * hi + 1]);
         }
     }
 #pragma unroll
@@ -269,8 +320,8 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_kernel(const AttnArgs a) {
     uint32_t pbh[MTILES][2], pbl[MTILES][2];
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) {
-        const float p0 = exp2f(s[i][0] - m0), p1 = exp2f(s[i][1] - m1);
-        const float p2 = exp2f(s[i][2] - m0), p3 = exp2f(s[i][3] - m1);
+        const float p0 = exp2f(sacc[i][0] - m0), p1 = exp2f(sacc[i][1] - m1);
+        const float p2 = exp2f(sacc[i][2] - m0), p3 = exp2f(sacc[i][3] - m1);
         l0 += p0 + p2;
         l1 += p1 + p3;
         uint32_t h01, l01, h23, l23;
@@ -286,19 +337,29 @@ __global__ void __launch_bounds__(kThreads) attn_fwd_kernel(const AttnArgs a) {
         l0 += __shfl_xor_sync(0xffffffffu, l0, o);
         l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
-    // P is split into bf16 hi + lo parts so that rounding P costs ~2^-17 relative
-    // instead of 2^-9; the output's own bf16 rounding is then the only visible error.
+    cp_async_wait<0>();
+    __syncthreads();  // V tile complete (all threads reach this: no early exit above)
     float oacc[2][4];
-    xt_b2<MTILES>(oacc, t.vs, pbh, pbl, lane);
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        oacc[m][0] = oacc[m][1] = oacc[m][2] = oacc[m][3] = 0.f;
+#pragma unroll
+        for (int i = 0; i < MTILES; ++i) {
+            const int row = base_t[i] + (lane & 7);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(smem_addr(vs) + urow_off(row, hw * 4 + 2 * m + (mi & 1)), a0, a1, a2, a3);
+            mma_bf16(oacc[m], a0, a1, a2, a3, pbl[i][0], pbl[i][1]);
+            mma_bf16(oacc[m], a0, a1, a2, a3, pbh[i][0], pbh[i][1]);
+        }
+    }
     const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
     const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
-    store_rows_t(oacc, i0, i1, t.qs, t.qid, tok0, a.H, h, a.o, lane);
+    if (!active) return;
+    store_rows_t(oacc, i0, i1, smem + L.stage + warp * 512, qtok + cw * 8, tok0, H, h, a.o, lane);
     if (gq == 0) {
-        const int q0 = t.qid[2 * tq], q1 = t.qid[2 * tq + 1];
-        if (q0 >= 0)
-            a.lse[(tok0 + q0) * a.H + h] = l0 > 0.f ? (m0 + log2f(l0)) * kLn2 : -INFINITY;
-        if (q1 >= 0)
-            a.lse[(tok0 + q1) * a.H + h] = l1 > 0.f ? (m1 + log2f(l1)) * kLn2 : -INFINITY;
+        const int q0 = qtok[cw * 8 + 2 * tq], q1 = qtok[cw * 8 + 2 * tq + 1];
+        if (q0 >= 0) a.lse[(tok0 + q0) * H + h] = l0 > 0.f ? (m0 + log2f(l0)) * kLn2 : -INFINITY;
+        if (q1 >= 0) a.lse[(tok0 + q1) * H + h] = l1 > 0.f ? (m1 + log2f(l1)) * kLn2 : -INFINITY;
     }
 }
 
@@ -394,162 +455,15 @@ __device__ void build_reverse_index(const AttnArgs& a, int b, uint8_t* smem) {
     }
 }
 
-// ---------------------------------------------------- backward, query-major
-
-template <int MTILES>
-__global__ void __launch_bounds__(kThreads) attn_bwd_query_kernel(const AttnArgs a, int task_blocks) {
-    constexpr int MT = 16 * MTILES;
-    extern __shared__ __align__(16) uint8_t smem[];
-    if (static_cast<int>(blockIdx.x) >= task_blocks) {
-        build_reverse_index(a, blockIdx.x - task_blocks, smem);
-        return;
-    }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long task = static_cast<long long>(blockIdx.x) * kWarps + warp;
-    if (task >= static_cast<long long>(a.B) * a.G * a.H) return;
-    const int h = static_cast<int>(task % a.H);
-    const long long bg = task / a.H;
-    const int g = static_cast<int>(bg % a.G), b = static_cast<int>(bg / a.G);
-    uint8_t* w = smem + warp * bwdq_warp_bytes(MT);
-    const FwdTiles t = fwd_tiles(w, MT);
-    uint8_t* dos = w + fwd_warp_bytes(MT);
-    const size_t tok0 = static_cast<size_t>(b) * a.N;
-    const int H = a.H;
-
-    load_cluster_tiles<MT>(a, b, g, h, lane, t, a.q);
-    {
-        const int row = lane >> 2, ch = lane & 3;
-        const int id = t.qid[row];
-        const size_t off = ((tok0 + (id >= 0 ? id : 0)) * H + h) * 32 + ch * 8;
-        cp_async16(smem_addr(dos) + tile64_off(row, ch), a.dout + off, id >= 0);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncwarp();
-
-    const int gq = lane >> 2, tq = lane & 3;
-    const int q0 = t.qid[2 * tq], q1 = t.qid[2 * tq + 1];
-    float L0 = q0 >= 0 ? a.lse_in[(tok0 + q0) * H + h] * kLog2e : INFINITY;
-    float L1 = q1 >= 0 ? a.lse_in[(tok0 + q1) * H + h] * kLog2e : INFINITY;
-    if (L0 == -INFINITY) L0 = INFINITY;  // empty neighbourhood: P = 0
-    if (L1 == -INFINITY) L1 = INFINITY;
-
-    uint32_t qf0, qf1, qf2, qf3, df0, df1, df2, df3;
-    ldsm_x4(smem_addr(t.qs) + tile64_off(lane & 7, lane >> 3), qf0, qf1, qf2, qf3);
-    ldsm_x4(smem_addr(dos) + tile64_off(lane & 7, lane >> 3), df0, df1, df2, df3);
-    float s[MTILES][4], dp[MTILES][4];
-    qk_tiles<MTILES>(s, t.ks, qf0, qf1, qf2, qf3, lane);
-    qk_tiles<MTILES>(dp, t.vs, df0, df1, df2, df3, lane);
-
-    const float sc = a.scale * kLog2e;
-    const float ba = a.bias[3 * h] * kLog2e, bb = a.bias[3 * h + 1] * kLog2e,
-                bc = a.bias[3 * h + 2] * kLog2e;
-    const float2 qa = t.qxy[2 * tq], qb = t.qxy[2 * tq + 1];
-    // P from the forward's lse; Delta_i = sum_j P_ij dP_ij (= <dO_i, O_i> exactly, since
-    // the whole key row is in this tile -- no bf16-rounded O enters the gradient)
-    float pd0 = 0.f, pd1 = 0.f;
-#pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-            const int key = 16 * i + gq + 8 * hi;
-            const bool kv = t.kid[key] >= 0;
-            const float2 kp = t.kxy[key];
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const float2 qp = qq ? qb : qa;
-                const float dx = kp.x - qp.x, dy = kp.y - qp.y;
-                const int j = 2 * hi + qq;
-                const float lg = s[i][j] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
-                const float p = kv ? exp2f(lg - (qq ? L1 : L0)) : 0.f;
-                s[i][j] = p;
-                if (qq) pd1 += p * dp[i][j];
-                else pd0 += p * dp[i][j];
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-        pd0 += __shfl_xor_sync(0xffffffffu, pd0, o);
-        pd1 += __shfl_xor_sync(0xffffffffu, pd1, o);
-    }
-    if (gq == 0) {
-        if (q0 >= 0) a.delta[(tok0 + q0) * H + h] = pd0;
-        if (q1 >= 0) a.delta[(tok0 + q1) * H + h] = pd1;
-    }
-    float ga = 0.f, gb = 0.f, gc = 0.f;
-    uint32_t db[MTILES][2];
-#pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-        float ds[4];
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-            const int key = 16 * i + gq + 8 * hi;
-            const float2 kp = t.kxy[key];
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const float2 qp = qq ? qb : qa;
-                const float dx = kp.x - qp.x, dy = kp.y - qp.y;
-                const int j = 2 * hi + qq;
-                const float v = s[i][j] * (dp[i][j] - (qq ? pd1 : pd0));
-                ds[j] = v;
-                ga += v * dx;
-                gb += v * dy;
-                gc += v * (dx * dx + dy * dy);
-            }
-        }
-        db[i][0] = movm_t(pack_bf16(ds[0], ds[1]));
-        db[i][1] = movm_t(pack_bf16(ds[2], ds[3]));
-    }
-    ga = warp_sum(ga);
-    gb = warp_sum(gb);
-    gc = warp_sum(gc);
-    if (lane == 0) {
-        float* part = a.dbias_part + ((static_cast<size_t>(b) * a.G + g) * H + h) * 3;
-        part[0] = ga;
-        part[1] = gb;
-        part[2] = -gc;
-    }
-    float dqacc[2][4];
-    xt_b<MTILES>(dqacc, t.ks, db, lane);
-    store_rows_t(dqacc, a.scale, a.scale, t.qs, t.qid, tok0, H, h, a.dq, lane);
-}
-
 // ------------------------------------------------------ backward, key-major
 
-__global__ void __launch_bounds__(kThreads) attn_bwd_key_kernel(const AttnArgs a, int task_blocks) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (static_cast<int>(blockIdx.x) >= task_blocks) {
-        // bias-gradient reduction: one CTA per (head, coefficient), fixed order
-        const int hj = blockIdx.x - task_blocks;
-        const int hh = hj / 3, j = hj % 3;
-        const int n = a.B * a.G;
-        float acc = 0.f;
-#pragma unroll 4
-        for (int i = threadIdx.x; i < n; i += kThreads)
-            acc += a.dbias_part[(static_cast<size_t>(i) * a.H + hh) * 3 + j];
-        acc = warp_sum(acc);
-        float* red = reinterpret_cast<float*>(smem);
-        if (lane == 0) red[warp] = acc;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float tot = 0.f;
-            for (int w = 0; w < kWarps; ++w) tot += red[w];
-            a.dbias[hh * 3 + j] = tot;
-        }
-        return;
-    }
-    const long long task = static_cast<long long>(blockIdx.x) * kWarps + warp;
-    if (task >= static_cast<long long>(a.B) * a.G * a.H) return;
-    const int h = static_cast<int>(task % a.H);
-    const long long bk = task / a.H;
-    const int kc = static_cast<int>(bk % a.G), b = static_cast<int>(bk / a.G);
+// Key-major backward of one (image, key cluster, head) by one warp, loading the query
+// rows of each pair of listed query clusters straight into its own 3.5 KB of shared memory.
+__device__ void key_major_direct(const AttnArgs& a, int b, int kc, int h, int lane, uint8_t* w) {
     const int H = a.H;
     const size_t tok0 = static_cast<size_t>(b) * a.N;
     const float2* xyb = reinterpret_cast<const float2*>(a.xy) + tok0;
 
-    uint8_t* w = smem + warp * kBwdKWarpBytes;
     uint8_t* ks = w;            // 8 rows
     uint8_t* vs = w + 512;      // 8 rows
     uint8_t* qs = w + 1024;     // 16 rows
@@ -662,31 +576,554 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_key_kernel(const AttnArgs a
     store_rows_t1(dv, 1.f, qs, kid, tok0, H, h, a.dv, lane);
 }
 
+
+// ------------------------------------------------ backward with neighbourhood unions
+
+// Union setup shared by the forward-shaped kernels: neighbour blocks of the CTA's kUC
+// clusters, de-duplicated; union row tokens/coordinates; per-cluster key-slot -> union row
+// map; the group's query tokens.  All threads of the CTA call it.
+__device__ __forceinline__ int union_setup(const AttnArgs& a, int b, int g0, int MT, const UnionLayout& L,
+                                           uint8_t* smem) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = a.G, N = a.N, M = a.M, R = a.R;
+    const int nblk = kUC * R;
+    int* blk_first = reinterpret_cast<int*>(smem + L.blk);
+    int* ublk = blk_first + nblk;
+    int* utok = reinterpret_cast<int*>(smem + L.utok);
+    float2* uxy = reinterpret_cast<float2*>(smem + L.uxy);
+    int* qtok = reinterpret_cast<int*>(smem + L.qtok);
+    float2* qxy = reinterpret_cast<float2*>(smem + L.qxy);
+    int* krow = reinterpret_cast<int*>(smem + L.krow);
+    int* nu_s = reinterpret_cast<int*>(smem + L.nu);
+    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(b) * N;
+    for (int i = tid; i < nblk; i += blockDim.x) {
+        const int g = g0 + i / R, r = i % R;
+        int f = -1;
+        if (g < G) {
+            f = a.nbr[(static_cast<size_t>(b) * G + g) * M + r * 8];
+            if (f < 0 || f >= N) f = -1;
+        }
+        blk_first[i] = f;
+    }
+    for (int i = tid; i < kUC * 8; i += blockDim.x) {
+        const int g = g0 + (i >> 3);
+        int id = -1;
+        if (g < G) {
+            id = a.clusters[(static_cast<size_t>(b) * G + g) * 8 + (i & 7)];
+            if (id < 0 || id >= N) id = -1;
+        }
+        qtok[i] = id;
+        qxy[i] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int f = lane < nblk ? blk_first[lane] : -1;
+        int dup = -1;
+        for (int j = 0; j < nblk; ++j) {
+            const int fj = __shfl_sync(0xffffffffu, f, j);
+            if (j < lane && dup < 0 && f >= 0 && fj == f) dup = j;
+        }
+        const bool isnew = f >= 0 && dup < 0;
+        const unsigned newmask = __ballot_sync(0xffffffffu, isnew);
+        int u = isnew ? __popc(newmask & ((1u << lane) - 1u)) : -1;
+        const int ud = __shfl_sync(0xffffffffu, u, dup >= 0 ? dup : 0);
+        if (dup >= 0) u = ud;
+        if (lane < nblk) ublk[lane] = isnew ? u : (dup >= 0 ? -(u + 2) : -1);
+        if (lane == 0) nu_s[0] = __popc(newmask);
+    }
+    __syncthreads();
+    for (int i = tid; i < nblk * 8; i += blockDim.x) {
+        const int blk = i >> 3, sl = i & 7;
+        const int u = ublk[blk];
+        if (u >= 0) {
+            const int g = g0 + blk / R, r = blk % R;
+            int t = a.nbr[(static_cast<size_t>(b) * G + g) * M + r * 8 + sl];
+            if (t < 0 || t >= N) t = -1;
+            utok[u * 8 + sl] = t;
+            uxy[u * 8 + sl] = t >= 0 ? xyb[t] : make_float2(0.f, 0.f);
+        }
+    }
+    for (int i = tid; i < kUC * MT; i += blockDim.x) {
+        const int cw = i / MT, m = i % MT;
+        int row = -1;
+        if (m < M) {
+            int u = ublk[cw * R + (m >> 3)];
+            if (u < -1) u = -u - 2;
+            if (u >= 0) row = u * 8 + (m & 7);
+        }
+        krow[i] = row;
+    }
+    __syncthreads();
+    return nu_s[0];
+}
+
+// Query-major pass with neighbourhood unions (same CTA shape as the forward), plus one
+// extra CTA column that builds each image's reverse neighbourhood index.
 template <int MTILES>
-cudaError_t fwd_dispatch(const AttnArgs& a, cudaStream_t st) {
-    const size_t smem = static_cast<size_t>(kWarps) * fwd_warp_bytes(16 * MTILES);
-    const long long tasks = static_cast<long long>(a.B) * a.G * a.H;
-    const long long blocks = (tasks + kWarps - 1) / kWarps;
-    attn_fwd_kernel<MTILES><<<static_cast<unsigned>(blocks), kThreads, smem, st>>>(a);
+__global__ void __launch_bounds__(kUThreads) attn_bwd_query_union_kernel(const AttnArgs a, int ncg) {
+    constexpr int MT = 16 * MTILES;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int cg = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+    if (cg >= ncg) {
+        if (hg == 0) build_reverse_index(a, b, smem);
+        return;
+    }
+    const int R = a.R;
+    const UnionLayout L = union_layout(R, MT);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = a.G, N = a.N, H = a.H;
+    const int g0 = cg * kUC;
+    const int ZR = kUC * R * 8;
+    uint8_t* ks = smem + L.ks;
+    uint8_t* vs = smem + L.vs;
+    uint8_t* qs = smem + L.qs;
+    uint8_t* dos = smem + L.stage;  // dO tile (kUC * 8 rows) in the staging area
+    uint8_t* stage = smem + L.total;  // per-warp output staging after the layout
+    const size_t tok0 = static_cast<size_t>(b) * N;
+    const int nU = union_setup(a, b, g0, MT, L, smem);
+    const int* utok = reinterpret_cast<const int*>(smem + L.utok);
+    const float2* uxy = reinterpret_cast<const float2*>(smem + L.uxy);
+    const int* qtok = reinterpret_cast<const int*>(smem + L.qtok);
+    const float2* qxy = reinterpret_cast<const float2*>(smem + L.qxy);
+    const int* krow = reinterpret_cast<const int*>(smem + L.krow);
+    const int hlo = hg * kUH;
+    for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
+        const int row = i >> 3, ch = i & 7;
+        const int t = row < nU * 8 ? utok[row] : -1;
+        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
+        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
+        const int drow = row < nU * 8 ? row : ZR + (row - nU * 8);
+        cp_async16(smem_addr(ks) + urow_off(drow, ch), a.k + (ok ? off : 0), ok);
+        cp_async16(smem_addr(vs) + urow_off(drow, ch), a.v + (ok ? off : 0), ok);
+    }
+    for (int i = tid; i < kUC * 8 * 8; i += kUThreads) {
+        const int row = i >> 3, ch = i & 7;
+        const int t = qtok[row];
+        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
+        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
+        cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + (ok ? off : 0), ok);
+        cp_async16(smem_addr(dos) + urow_off(row, ch), a.dout + (ok ? off : 0), ok);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    const int cw = warp / kUH, hw = warp % kUH;
+    const int g = g0 + cw, h = hlo + hw;
+    if (g >= G || h >= H) return;
+    const int gq = lane >> 2, tq = lane & 3, mi = lane >> 3;
+    const int* kr = krow + cw * MT;
+    // row 0 of each neighbourhood block this lane addresses: (mi & 1) picks the block of
+    // the S / dQ operands, (mi >> 1) the block of the transposed V / K operands
+    int base_s[MTILES], base_t[MTILES];
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+        const int s0 = 2 * i + (mi & 1), s1 = 2 * i + (mi >> 1);
+        const int r0 = (s0 * 8 < a.M) ? kr[s0 * 8] : -1;
+        const int r1 = (s1 * 8 < a.M) ? kr[s1 * 8] : -1;
+        base_s[i] = r0 >= 0 ? r0 : ZR;
+        base_t[i] = r1 >= 0 ? r1 : ZR;
+    }
+    const int q0 = qtok[cw * 8 + 2 * tq], q1 = qtok[cw * 8 + 2 * tq + 1];
+    float L0 = q0 >= 0 ? a.lse_in[(tok0 + q0) * H + h] * kLog2e : INFINITY;
+    float L1 = q1 >= 0 ? a.lse_in[(tok0 + q1) * H + h] * kLog2e : INFINITY;
+    if (L0 == -INFINITY) L0 = INFINITY;
+    if (L1 == -INFINITY) L1 = INFINITY;
+    uint32_t qf0, qf1, qf2, qf3, df0, df1, df2, df3;
+    ldsm_x4(smem_addr(qs) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), qf0, qf1, qf2, qf3);
+    ldsm_x4(smem_addr(dos) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), df0, df1, df2, df3);
+    float sacc[MTILES][4], dp[MTILES][4];
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+        sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
+        dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const int row = base_s[i] + (lane & 7);
+            const uint32_t off = urow_off(row, hw * 4 + 2 * kk + (mi >> 1));
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(smem_addr(ks) + off, a0, a1, a2, a3);
+            mma_bf16(sacc[i], a0, a1, a2, a3, kk ? qf2 : qf0, kk ? qf3 : qf1);
+            ldsm_x4(smem_addr(vs) + off, a0, a1, a2, a3);
+            mma_bf16(dp[i], a0, a1, a2, a3, kk ? df2 : df0, kk ? df3 : df1);
+        }
+    }
+    const float sc = a.scale * kLog2e;
+    const float ba = a.bias[3 * h] * kLog2e, bb = a.bias[3 * h + 1] * kLog2e,
+                bc = a.bias[3 * h + 2] * kLog2e;
+    const float2 qa = qxy[cw * 8 + 2 * tq], qb = qxy[cw * 8 + 2 * tq + 1];
+    float pd0 = 0.f, pd1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+            const int row = kr[16 * i + gq + 8 * hi];
+            const bool kv = row >= 0 && utok[row] >= 0;
+            const float2 kp = kv ? uxy[row] : make_float2(0.f, 0.f);
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                const float2 qp = qq ? qb : qa;
+                const float dx = kp.x - qp.x, dy = kp.y - qp.y;
+                const int j = 2 * hi + qq;
+                const float lg = sacc[i][j] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
+                const float p = kv ? exp2f(lg - (qq ? L1 : L0)) : 0.f;
+                sacc[i][j] = p;
+                if (qq) pd1 += p * dp[i][j];
+                else pd0 += p * dp[i][j];
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        pd0 += __shfl_xor_sync(0xffffffffu, pd0, o);
+        pd1 += __shfl_xor_sync(0xffffffffu, pd1, o);
+    }
+    if (gq == 0) {
+        if (q0 >= 0) a.delta[(tok0 + q0) * H + h] = pd0;
+        if (q1 >= 0) a.delta[(tok0 + q1) * H + h] = pd1;
+    }
+    float ga = 0.f, gb = 0.f, gc = 0.f;
+    uint32_t db[MTILES][2];
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+        float ds[4];
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+            const int row = kr[16 * i + gq + 8 * hi];
+            const bool kv = row >= 0 && utok[row] >= 0;
+            const float2 kp = kv ? uxy[row] : make_float2(0.f, 0.f);
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                const float2 qp = qq ? qb : qa;
+                const float dx = kp.x - qp.x, dy = kp.y - qp.y;
+                const int j = 2 * hi + qq;
+                const float v = sacc[i][j] * (dp[i][j] - (qq ? pd1 : pd0));
+                ds[j] = v;
+                ga += v * dx;
+                gb += v * dy;
+                gc += v * (dx * dx + dy * dy);
+            }
+        }
+        db[i][0] = movm_t(pack_bf16(ds[0], ds[1]));
+        db[i][1] = movm_t(pack_bf16(ds[2], ds[3]));
+    }
+    ga = warp_sum(ga);
+    gb = warp_sum(gb);
+    gc = warp_sum(gc);
+    if (lane == 0) {
+        float* part = a.dbias_part + ((static_cast<size_t>(b) * G + g) * H + h) * 3;
+        part[0] = ga;
+        part[1] = gb;
+        part[2] = -gc;
+    }
+    float dqacc[2][4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        dqacc[m][0] = dqacc[m][1] = dqacc[m][2] = dqacc[m][3] = 0.f;
+#pragma unroll
+        for (int i = 0; i < MTILES; ++i) {
+            const int row = base_t[i] + (lane & 7);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(smem_addr(ks) + urow_off(row, hw * 4 + 2 * m + (mi & 1)), a0, a1, a2, a3);
+            mma_bf16(dqacc[m], a0, a1, a2, a3, db[i][0], db[i][1]);
+        }
+    }
+    store_rows_t(dqacc, a.scale, a.scale, stage + warp * 512, qtok + cw * 8, tok0, H, h, a.dq, lane);
+}
+
+// Key-major pass with query-cluster unions.  CTA = (kUC consecutive key clusters, kUH
+// heads, image).  The reverse lists of its key clusters are concatenated and their query
+// clusters de-duplicated; Q and dO rows of the union (plus lse and Delta) are gathered
+// once and every warp walks its own list two query clusters at a time out of the union
+// tile.  A group whose lists exceed the tile falls back to per-warp direct loading.
+constexpr int kKQ = 24;       // union query clusters held per CTA
+constexpr int kKEnt = 64;     // list entries per CTA
+struct KeyLayout {
+    int qs, dos, ks, vs, stage, ent, eu, es, qtok, qxy, qL, qD, ktok, kxy, misc, total;
+};
+__host__ __device__ __forceinline__ KeyLayout key_layout() {
+    KeyLayout L;
+    const int rows = kKQ * 8 + 8;
+    int o = 0;
+    L.qs = o; o += rows * kURow;
+    L.dos = o; o += rows * kURow;
+    L.ks = o; o += kUC * 8 * kURow;
+    L.vs = o; o += kUC * 8 * kURow;
+    L.stage = o; o += kUWarps * 512;
+    L.ent = o; o += 4 * kKEnt;
+    L.eu = o; o += 4 * kKEnt;
+    L.es = o; o += 4 * (kUC + 1);
+    o = (o + 15) & ~15;
+    L.qtok = o; o += 4 * rows;
+    L.qxy = o; o += 8 * rows;
+    L.qL = o; o += 4 * rows * kUH;
+    L.qD = o; o += 4 * rows * kUH;
+    L.ktok = o; o += 4 * kUC * 8;
+    L.kxy = o; o += 8 * kUC * 8;
+    L.misc = o; o += 16;
+    L.total = (o + 15) & ~15;
+    return L;
+}
+
+__global__ void __launch_bounds__(kUThreads) attn_bwd_key_union_kernel(const AttnArgs a, int ncg) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int cg = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+    const int G = a.G, N = a.N, H = a.H;
+    if (cg >= ncg) {
+        // bias-gradient reduction: one CTA per (head, coefficient), fixed order
+        const int hj = cg - ncg;
+        if (hg != 0 || b != 0 || hj >= 3 * H) return;
+        const int hh = hj / 3, j = hj % 3;
+        const int n = a.B * G;
+        float acc = 0.f;
+#pragma unroll 4
+        for (int i = tid; i < n; i += kUThreads) acc += a.dbias_part[(static_cast<size_t>(i) * H + hh) * 3 + j];
+        acc = warp_sum(acc);
+        float* red = reinterpret_cast<float*>(smem);
+        if (lane == 0) red[warp] = acc;
+        __syncthreads();
+        if (tid == 0) {
+            float tot = 0.f;
+            for (int w = 0; w < kUWarps; ++w) tot += red[w];
+            a.dbias[hh * 3 + j] = tot;
+        }
+        return;
+    }
+    const KeyLayout L = key_layout();
+    const int g0 = cg * kUC;
+    const int hlo = hg * kUH;
+    const int ZR = kKQ * 8;
+    const size_t tok0 = static_cast<size_t>(b) * N;
+    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + tok0;
+    int* ent = reinterpret_cast<int*>(smem + L.ent);
+    int* eu = reinterpret_cast<int*>(smem + L.eu);
+    int* es = reinterpret_cast<int*>(smem + L.es);
+    int* qtok = reinterpret_cast<int*>(smem + L.qtok);
+    float2* qxy = reinterpret_cast<float2*>(smem + L.qxy);
+    float* qL = reinterpret_cast<float*>(smem + L.qL);
+    float* qD = reinterpret_cast<float*>(smem + L.qD);
+    int* ktok = reinterpret_cast<int*>(smem + L.ktok);
+    float2* kxy = reinterpret_cast<float2*>(smem + L.kxy);
+    int* misc = reinterpret_cast<int*>(smem + L.misc);
+    const int32_t* roff = a.rev_off + static_cast<size_t>(b) * (G + 1);
+    const int32_t* rlist = a.rev_list + static_cast<size_t>(b) * G * a.R;
+    if (tid == 0) {
+        int acc = 0;
+        for (int c = 0; c < kUC; ++c) {
+            es[c] = acc;
+            const int kc = g0 + c;
+            if (kc < G) acc += roff[kc + 1] - roff[kc];
+        }
+        es[kUC] = acc;
+    }
+    for (int i = tid; i < kUC * 8; i += kUThreads) {
+        const int kc = g0 + (i >> 3);
+        int id = -1;
+        if (kc < G) {
+            id = a.clusters[(static_cast<size_t>(b) * G + kc) * 8 + (i & 7)];
+            if (id < 0 || id >= N) id = -1;
+        }
+        ktok[i] = id;
+        kxy[i] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
+    }
+    __syncthreads();
+    const int ntot = es[kUC];
+    bool fits = ntot <= kKEnt;
+    if (fits) {
+        for (int i = tid; i < ntot; i += kUThreads) {
+            int c = 0;
+            while (c + 1 < kUC && es[c + 1] <= i) ++c;
+            ent[i] = rlist[roff[g0 + c] + (i - es[c])];
+        }
+        __syncthreads();
+        // first occurrences get consecutive union indices, in list order
+        if (warp == 0) {
+            int run = 0;
+            for (int base = 0; base < ntot; base += 32) {
+                const int i = base + lane;
+                bool first = false;
+                if (i < ntot) {
+                    first = true;
+                    for (int j = 0; j < i; ++j)
+                        if (ent[j] == ent[i]) { first = false; break; }
+                }
+                const unsigned m = __ballot_sync(0xffffffffu, first);
+                if (first) eu[i] = run + __popc(m & ((1u << lane) - 1u));
+                run += __popc(m);
+            }
+            if (lane == 0) misc[0] = run;
+        }
+        __syncthreads();
+        for (int i = tid; i < ntot; i += kUThreads) {
+            int src = i;
+            for (int j = 0; j < i; ++j)
+                if (ent[j] == ent[i]) { src = j; break; }
+            if (src != i) eu[i] = -1 - src;  // resolved below
+        }
+        __syncthreads();
+        for (int i = tid; i < ntot; i += kUThreads)
+            if (eu[i] < 0) eu[i] = eu[-1 - eu[i]];
+        fits = misc[0] <= kKQ;
+        __syncthreads();
+    }
+    if (!fits) {
+        // fallback: every warp handles its (key cluster, head) with direct loads
+        const int cw = warp / kUH, hw = warp % kUH;
+        const int kc = g0 + cw, h = hlo + hw;
+        if (kc < G && h < H) key_major_direct(a, b, kc, h, lane, smem + warp * kBwdKWarpBytes);
+        return;
+    }
+    const int nU = misc[0];
+    // union query rows, their lse / Delta per head of the group
+    for (int i = tid; i < ntot * 8; i += kUThreads) {
+        const int e = i >> 3, sl = i & 7;
+        bool first = true;
+        for (int j = 0; j < e; ++j)
+            if (ent[j] == ent[e]) { first = false; break; }
+        if (!first) continue;
+        const int row = eu[e] * 8 + sl;
+        int t = a.clusters[(static_cast<size_t>(b) * G + ent[e]) * 8 + sl];
+        if (t < 0 || t >= N) t = -1;
+        qtok[row] = t;
+        qxy[row] = t >= 0 ? xyb[t] : make_float2(0.f, 0.f);
+        for (int hw = 0; hw < kUH; ++hw) {
+            const int h = hlo + hw;
+            float Lv = INFINITY, Dv = 0.f;
+            if (t >= 0 && h < H) {
+                Lv = a.lse_in[(tok0 + t) * H + h] * kLog2e;
+                if (Lv == -INFINITY) Lv = INFINITY;
+                Dv = a.delta[(tok0 + t) * H + h];
+            }
+            qL[row * kUH + hw] = Lv;
+            qD[row * kUH + hw] = Dv;
+        }
+    }
+    for (int i = tid; i < 8 * kUH; i += kUThreads) {
+        qL[(ZR + (i / kUH)) * kUH + (i % kUH)] = INFINITY;
+        qD[(ZR + (i / kUH)) * kUH + (i % kUH)] = 0.f;
+    }
+    if (tid < 8) {
+        qtok[ZR + tid] = -1;
+        qxy[ZR + tid] = make_float2(0.f, 0.f);
+    }
+    __syncthreads();
+    uint8_t* qs = smem + L.qs;
+    uint8_t* dos = smem + L.dos;
+    uint8_t* ks = smem + L.ks;
+    uint8_t* vs = smem + L.vs;
+    for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
+        const int row = i >> 3, ch = i & 7;
+        const int drow = row < nU * 8 ? row : ZR + (row - nU * 8);
+        const int t = qtok[drow];
+        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
+        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
+        cp_async16(smem_addr(qs) + urow_off(drow, ch), a.q + (ok ? off : 0), ok);
+        cp_async16(smem_addr(dos) + urow_off(drow, ch), a.dout + (ok ? off : 0), ok);
+    }
+    for (int i = tid; i < kUC * 8 * 8; i += kUThreads) {
+        const int row = i >> 3, ch = i & 7;
+        const int t = ktok[row];
+        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
+        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
+        cp_async16(smem_addr(ks) + urow_off(row, ch), a.k + (ok ? off : 0), ok);
+        cp_async16(smem_addr(vs) + urow_off(row, ch), a.v + (ok ? off : 0), ok);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    const int cw = warp / kUH, hw = warp % kUH;
+    const int kc = g0 + cw, h = hlo + hw;
+    if (kc >= G || h >= H) return;
+    const int gq = lane >> 2, tq = lane & 3, mi = lane >> 3;
+    uint32_t kf0, kf1, kf2, kf3, vf0, vf1, vf2, vf3;
+    ldsm_x4(smem_addr(ks) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), kf0, kf1, kf2, kf3);
+    ldsm_x4(smem_addr(vs) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), vf0, vf1, vf2, vf3);
+    const float sc = a.scale * kLog2e;
+    const float ba = a.bias[3 * h] * kLog2e, bb = a.bias[3 * h + 1] * kLog2e,
+                bc = a.bias[3 * h + 2] * kLog2e;
+    const float2 kp0 = kxy[cw * 8 + 2 * tq], kp1 = kxy[cw * 8 + 2 * tq + 1];
+    float dk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float dv[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    const int e_end = es[cw + 1];
+    for (int e = es[cw]; e < e_end; e += 2) {
+        const int b1 = eu[e] * 8;
+        const int b2 = (e + 1 < e_end) ? eu[e + 1] * 8 : ZR;
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, pacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const int row = ((mi & 1) ? b2 : b1) + (lane & 7);
+            const uint32_t off = urow_off(row, hw * 4 + 2 * kk + (mi >> 1));
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(smem_addr(qs) + off, a0, a1, a2, a3);
+            mma_bf16(sacc, a0, a1, a2, a3, kk ? kf2 : kf0, kk ? kf3 : kf1);
+            ldsm_x4(smem_addr(dos) + off, a0, a1, a2, a3);
+            mma_bf16(pacc, a0, a1, a2, a3, kk ? vf2 : vf0, kk ? vf3 : vf1);
+        }
+        float p[4], ds[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int qrow = ((j >> 1) ? b2 : b1) + gq;
+            const float2 qp = qxy[qrow];
+            const float2 kp = (j & 1) ? kp1 : kp0;
+            const float dx = kp.x - qp.x, dy = kp.y - qp.y;
+            const float lg = sacc[j] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
+            p[j] = exp2f(lg - qL[qrow * kUH + hw]);
+            ds[j] = p[j] * (pacc[j] - qD[qrow * kUH + hw]);
+        }
+        const uint32_t pb0 = movm_t(pack_bf16(p[0], p[1]));
+        const uint32_t pb1 = movm_t(pack_bf16(p[2], p[3]));
+        const uint32_t sb0 = movm_t(pack_bf16(ds[0], ds[1]));
+        const uint32_t sb1 = movm_t(pack_bf16(ds[2], ds[3]));
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int row = ((mi >> 1) ? b2 : b1) + (lane & 7);
+            const uint32_t off = urow_off(row, hw * 4 + 2 * m + (mi & 1));
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(smem_addr(dos) + off, a0, a1, a2, a3);
+            mma_bf16(dv[m], a0, a1, a2, a3, pb0, pb1);
+            ldsm_x4_t(smem_addr(qs) + off, a0, a1, a2, a3);
+            mma_bf16(dk[m], a0, a1, a2, a3, sb0, sb1);
+        }
+    }
+    uint8_t* stage = smem + L.stage + warp * 512;
+    store_rows_t1(dk, a.scale, stage, ktok + cw * 8, tok0, H, h, a.dk, lane);
+    store_rows_t1(dv, 1.f, stage, ktok + cw * 8, tok0, H, h, a.dv, lane);
+}
+
+template <int MTILES>
+cudaError_t fwd_union_dispatch(const AttnArgs& a, cudaStream_t st) {
+    const size_t smem = static_cast<size_t>(union_layout(a.R, 16 * MTILES).total);
+    cudaError_t e = ensure_smem<attn_fwd_union_kernel<MTILES>>(smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((a.G + kUC - 1) / kUC, (a.H + kUH - 1) / kUH, a.B);
+    attn_fwd_union_kernel<MTILES><<<grid, kUThreads, smem, st>>>(a);
     note_launch();
     return cudaGetLastError();
 }
 
 template <int MTILES>
 cudaError_t bwd_dispatch(const AttnArgs& a, cudaStream_t st) {
-    const long long tasks = static_cast<long long>(a.B) * a.G * a.H;
-    const int blocks = static_cast<int>((tasks + kWarps - 1) / kWarps);
-    size_t smem = static_cast<size_t>(kWarps) * bwdq_warp_bytes(16 * MTILES);
+    const int ncg = (a.G + kUC - 1) / kUC;
+    const int nhg = (a.H + kUH - 1) / kUH;
+    // query-major pass (+ one column of reverse-index CTAs)
+    size_t smem = static_cast<size_t>(union_layout(a.R, 16 * MTILES).total) + kUWarps * 512;
     const size_t prep = 4 * static_cast<size_t>(a.G + 1) + 160;
     if (prep > smem) smem = prep;
-    cudaError_t e = ensure_smem<attn_bwd_query_kernel<MTILES>>(smem);
+    cudaError_t e = ensure_smem<attn_bwd_query_union_kernel<MTILES>>(smem);
     if (e != cudaSuccess) return e;
-    attn_bwd_query_kernel<MTILES><<<blocks + a.B, kThreads, smem, st>>>(a, blocks);
+    attn_bwd_query_union_kernel<MTILES><<<dim3(ncg + 1, nhg, a.B), kUThreads, smem, st>>>(a, ncg);
     note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t smem2 = static_cast<size_t>(kWarps) * kBwdKWarpBytes;
-    attn_bwd_key_kernel<<<blocks + 3 * a.H, kThreads, smem2, st>>>(a, blocks);
+    // key-major pass (+ 3H bias-reduction CTAs in the first column block)
+    size_t smem2 = static_cast<size_t>(key_layout().total);
+    if (smem2 < static_cast<size_t>(kUWarps) * kBwdKWarpBytes) smem2 = static_cast<size_t>(kUWarps) * kBwdKWarpBytes;
+    e = ensure_smem<attn_bwd_key_union_kernel>(smem2);
+    if (e != cudaSuccess) return e;
+    const int extra = (3 * a.H + 0);
+    attn_bwd_key_union_kernel<<<dim3(ncg + extra, nhg, a.B), kUThreads, smem2, st>>>(a, ncg);
     note_launch();
     return cudaGetLastError();
 }
@@ -710,10 +1147,10 @@ AttnWorkspace attn_workspace_layout(int B, int N, int H, int C, int M) {
 
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st) {
     switch ((a.M + 15) / 16) {
-        case 1: return fwd_dispatch<1>(a, st);
-        case 2: return fwd_dispatch<2>(a, st);
-        case 3: return fwd_dispatch<3>(a, st);
-        default: return fwd_dispatch<4>(a, st);
+        case 1: return fwd_union_dispatch<1>(a, st);
+        case 2: return fwd_union_dispatch<2>(a, st);
+        case 3: return fwd_union_dispatch<3>(a, st);
+        default: return fwd_union_dispatch<4>(a, st);
     }
 }
 

@@ -43,9 +43,16 @@ __host__ __device__ __forceinline__ int next_pow2(int n) {
     return p;
 }
 
-// Byte offsets of the shared-memory regions of cluster_kernel.
+constexpr int kBucketMax = 32;  // largest bucket the fast path sorts with one thread
+
+// Byte offsets of the shared-memory regions of cluster_kernel:
+//   xs, ys [N] f32 | L0 [2N] u16 (sorted X list, then Y list) |
+//   U = union of { sort keys [2P] u64 (fallback) or bucket counts [2P] i32 (fast path) }
+//             and { level arrays: L1 [2N], scanv [N], scanout [N], posX [N], posY [N],
+//                   pos_cluster [N] (u16), seg_c0, seg_g [G] u16, seg_axis [G] u8 } |
+//   scratch [160] i32
 struct ClusterSmem {
-    size_t region, kid, warp, total;
+    size_t l0, u, scratch, total;
 };
 __host__ __device__ __forceinline__ size_t round16(size_t x) { return (x + 15) & ~size_t(15); }
 __host__ __device__ __forceinline__ ClusterSmem cluster_smem_layout(int N, int C) {
@@ -53,20 +60,102 @@ __host__ __device__ __forceinline__ ClusterSmem cluster_smem_layout(int N, int C
     const size_t G = static_cast<size_t>((N + C - 1) / C);
     const size_t n = static_cast<size_t>(N);
     ClusterSmem L;
-    L.region = round16(8 * n);                                   // xs, ys
-    const size_t sort_keys = 16 * P;                             // 2P u64
-    const size_t levels = 12 * n + 4 * G + n + G + 16;           // lists, scans, segments, flags
-    L.kid = L.region + round16(sort_keys > levels ? sort_keys : levels);
-    L.warp = L.kid + round16(4 * P);                             // 2P u16 ids
-    L.total = L.warp + 32 * sizeof(int);
+    L.l0 = round16(8 * n);
+    L.u = L.l0 + round16(4 * n);
+    const size_t sort_bytes = 16 * P;
+    const size_t level_bytes = 14 * n + 5 * G + 16;
+    L.scratch = L.u + round16(sort_bytes > level_bytes ? sort_bytes : level_bytes);
+    L.total = L.scratch + 160 * sizeof(int);
     return L;
 }
 
+__device__ __forceinline__ uint64_t full_key(float a, float b) {
+    return (static_cast<uint64_t>(order_bits(a)) << 32) | order_bits(b);
+}
+
+// Block-wide min/max of x and y (all threads call; result broadcast through scratch).
+__device__ void block_minmax(const float* xs, const float* ys, int N, int* scratch, float& xmin,
+                             float& xmax, float& ymin, float& ymax) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    float a = INFINITY, b = -INFINITY, c = INFINITY, d = -INFINITY;
+    for (int i = tid; i < N; i += blockDim.x) {
+        a = fminf(a, xs[i]);
+        b = fmaxf(b, xs[i]);
+        c = fminf(c, ys[i]);
+        d = fmaxf(d, ys[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a = fminf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
+        c = fminf(c, __shfl_xor_sync(0xffffffffu, c, o));
+        d = fmaxf(d, __shfl_xor_sync(0xffffffffu, d, o));
+    }
+    float* f = reinterpret_cast<float*>(scratch);
+    __syncthreads();
+    if (lane == 0) {
+        f[4 * warp] = a;
+        f[4 * warp + 1] = b;
+        f[4 * warp + 2] = c;
+        f[4 * warp + 3] = d;
+    }
+    __syncthreads();
+    xmin = ymin = INFINITY;
+    xmax = ymax = -INFINITY;
+    for (int w = 0; w < nw; ++w) {
+        xmin = fminf(xmin, f[4 * w]);
+        xmax = fmaxf(xmax, f[4 * w + 1]);
+        ymin = fminf(ymin, f[4 * w + 2]);
+        ymax = fmaxf(ymax, f[4 * w + 3]);
+    }
+    __syncthreads();
+}
+
+// Exclusive prefix sum of int data[0..n) in place (all threads call); returns the total.
+__device__ int block_scan_int(int* data, int n, int* scratch) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const int per = (n + blockDim.x - 1) / blockDim.x;
+    const int p0 = tid * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i)
+        if (p0 + i < n) local += data[p0 + i];
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = lane < nw ? scratch[lane] : 0;
+        int sc = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, sc, o);
+            if (lane >= o) sc += u;
+        }
+        scratch[lane] = sc - v;
+        if (lane == 31) scratch[32] = sc;
+    }
+    __syncthreads();
+    int run = scratch[warp] + incl - local;
+    for (int i = 0; i < per; ++i) {
+        if (p0 + i < n) {
+            const int v = data[p0 + i];
+            data[p0 + i] = run;
+            run += v;
+        }
+    }
+    const int total = scratch[32];
+    __syncthreads();
+    return total;
+}
+
 // Exclusive prefix sum of vals[0..n) (uint16) into out[0..n); all threads call.
-__device__ void block_exclusive_scan_u16(const uint16_t* vals, uint16_t* out, int n,
-                                         int* warp_tot) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int per = (n + kClusterThreads - 1) / kClusterThreads;
+__device__ void block_exclusive_scan_u16(const uint16_t* vals, uint16_t* out, int n, int* scratch) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const int per = (n + blockDim.x - 1) / blockDim.x;
     const int p0 = tid * per;
     int local = 0;
     for (int i = 0; i < per; ++i)
@@ -74,23 +163,23 @@ __device__ void block_exclusive_scan_u16(const uint16_t* vals, uint16_t* out, in
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        int v = __shfl_up_sync(0xffffffffu, incl, o);
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += v;
     }
-    if (lane == 31) warp_tot[warp] = incl;
+    if (lane == 31) scratch[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        int v = warp_tot[lane];
-        int s = v;
+        const int v = lane < nw ? scratch[lane] : 0;
+        int sc = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int u = __shfl_up_sync(0xffffffffu, s, o);
-            if (lane >= o) s += u;
+            const int u = __shfl_up_sync(0xffffffffu, sc, o);
+            if (lane >= o) sc += u;
         }
-        warp_tot[lane] = s - v;  // exclusive prefix of warp totals
+        scratch[lane] = sc - v;
     }
     __syncthreads();
-    int run = warp_tot[warp] + incl - local;
+    int run = scratch[warp] + incl - local;
     for (int i = 0; i < per; ++i) {
         if (p0 + i < n) {
             out[p0 + i] = static_cast<uint16_t>(run);
@@ -100,9 +189,87 @@ __device__ void block_exclusive_scan_u16(const uint16_t* vals, uint16_t* out, in
     __syncthreads();
 }
 
-// Shared memory: xs, ys [N] f32 | keys [2P] u64 | ids [2P] u16, where the level
-// arrays (list ping-pong, flags, scan, segments) overlay the keys region once the
-// sort is done.
+// Bucket index of v: floor((v - vmin) * scale) clamped to [0, nb - 1].  Every step is
+// monotone non-decreasing in v, so bucket order never contradicts coordinate order.
+__device__ __forceinline__ int bucket_of(float v, float vmin, float scale, int nb) {
+    const float t = (v - vmin) * scale;
+    if (!(t >= 0.f)) return 0;
+    if (t >= static_cast<float>(nb)) return nb - 1;
+    const int i = static_cast<int>(t);
+    return i > nb - 1 ? nb - 1 : i;
+}
+
+// Bitonic sort of 2P packed u64 values in shared memory, [0,P) and [P,2P) independently.
+__device__ void bitonic_2lists(uint64_t* keys, int P) {
+    const int tid = threadIdx.x, nt = blockDim.x;
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < 2 * P; i += nt) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const bool up = ((i & (P - 1)) & k) == 0;
+                    const uint64_t ka = keys[i], kb = keys[ixj];
+                    if ((ka > kb) == up) {
+                        keys[i] = kb;
+                        keys[ixj] = ka;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+// Fallback sort for inputs with crowded buckets (many equal or clustered coordinates),
+// with 48-bit packed keys only.  Round 1 sorts (a, id) per list: T_x = tokens in (x, id)
+// order, T_y = tokens in (y, id) order.  Round 2 sorts the X list by (x, r) where r is a
+// token's position in T_y -- so ties in x fall back to (y, id) -- and the Y list by (y, r)
+// with r its position in T_x; mapping r back through T_y / T_x gives the tokens.
+__device__ void fallback_sort(const float* xs, const float* ys, int N, int P, uint64_t* keys,
+                              uint16_t* L0) {
+    const int tid = threadIdx.x, nt = blockDim.x;
+    for (int i = tid; i < 2 * P; i += nt) {
+        const int li = i & (P - 1);
+        keys[i] = (li < N) ? ((static_cast<uint64_t>(order_bits(i < P ? xs[li] : ys[li])) << 16) | li)
+                           : ~uint64_t(0);
+    }
+    __syncthreads();
+    bitonic_2lists(keys, P);
+    for (int i = tid; i < N; i += nt) {
+        L0[i] = static_cast<uint16_t>(keys[i] & 0xFFFFu);          // T_x
+        L0[N + i] = static_cast<uint16_t>(keys[P + i] & 0xFFFFu);  // T_y
+    }
+    __syncthreads();
+    for (int i = tid; i < 2 * P; i += nt) {
+        const int li = i & (P - 1);
+        uint64_t k = ~uint64_t(0);
+        if (li < N) {
+            if (i < P) {
+                const int t = L0[N + li];  // li-th token of the (y, id) order
+                k = (static_cast<uint64_t>(order_bits(xs[t])) << 16) | li;
+            } else {
+                const int t = L0[li];      // li-th token of the (x, id) order
+                k = (static_cast<uint64_t>(order_bits(ys[t])) << 16) | li;
+            }
+        }
+        keys[i] = k;
+    }
+    __syncthreads();
+    bitonic_2lists(keys, P);
+    for (int i = tid; i < N; i += nt) {
+        const int rx = static_cast<int>(keys[i] & 0xFFFFu);
+        const int ry = static_cast<int>(keys[P + i] & 0xFFFFu);
+        keys[i] = L0[N + rx];
+        keys[P + i] = L0[ry];
+    }
+    __syncthreads();
+    for (int i = tid; i < N; i += nt) {
+        L0[i] = static_cast<uint16_t>(keys[i]);
+        L0[N + i] = static_cast<uint16_t>(keys[P + i]);
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(kClusterThreads)
     cluster_kernel(const float* __restrict__ xy, int N, int C, int32_t* __restrict__ clusters) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -113,67 +280,80 @@ __global__ void __launch_bounds__(kClusterThreads)
     const ClusterSmem L = cluster_smem_layout(N, C);
     float* xs = reinterpret_cast<float*>(smem);
     float* ys = xs + N;
-    uint8_t* region = smem + L.region;
-    uint64_t* keys = reinterpret_cast<uint64_t*>(region);
-    uint16_t* kid = reinterpret_cast<uint16_t*>(smem + L.kid);
-    // level arrays, inside the keys region (sized for both uses)
-    uint16_t* lx0 = reinterpret_cast<uint16_t*>(region);
-    uint16_t* ly0 = lx0 + N;
-    uint16_t* lx1 = ly0 + N;
-    uint16_t* ly1 = lx1 + N;
-    uint16_t* scanv = ly1 + N;
-    uint16_t* scanout = scanv + N;
-    uint16_t* seg_c0 = scanout + N;
-    uint16_t* seg_g = seg_c0 + G;
-    uint8_t* flag = reinterpret_cast<uint8_t*>(seg_g + G);
-    uint8_t* seg_axis = flag + N;
-    int* warp_tot = reinterpret_cast<int*>(smem + L.warp);
+    uint16_t* L0 = reinterpret_cast<uint16_t*>(smem + L.l0);  // [2N]: X list then Y list
+    uint8_t* U = smem + L.u;
+    int* scratch = reinterpret_cast<int*>(smem + L.scratch);
 
-    const float* img = xy + static_cast<size_t>(b) * N * 2;
+    const float2* img = reinterpret_cast<const float2*>(xy) + static_cast<size_t>(b) * N;
     for (int i = tid; i < N; i += kClusterThreads) {
-        float2 p = reinterpret_cast<const float2*>(img)[i];
+        const float2 p = img[i];
         xs[i] = p.x;
         ys[i] = p.y;
     }
     __syncthreads();
 
-    // ---- one bitonic network sorting both lists: [0,P) by (x,y,id), [P,2P) by (y,x,id)
-    for (int i = tid; i < 2 * P; i += kClusterThreads) {
-        const int li = i & (P - 1);
-        if (li < N) {
-            const uint32_t ox = order_bits(xs[li]), oy = order_bits(ys[li]);
-            keys[i] = (i < P) ? ((uint64_t(ox) << 32) | oy) : ((uint64_t(oy) << 32) | ox);
-            kid[i] = static_cast<uint16_t>(li);
-        } else {
-            keys[i] = ~uint64_t(0);
-            kid[i] = 0xFFFFu;
-        }
+    // ---- sort both lists: counting sort into N monotone buckets per axis, then an exact
+    //      insertion sort inside each (small) bucket by (axis coord, other coord, id)
+    float xmin, xmax, ymin, ymax;
+    block_minmax(xs, ys, N, scratch, xmin, xmax, ymin, ymax);
+    const int NB = N;
+    const float sx = (float)NB / (xmax - xmin), sy = (float)NB / (ymax - ymin);
+    int* cnt = reinterpret_cast<int*>(U);  // [2 NB]
+    for (int i = tid; i < 2 * NB; i += kClusterThreads) cnt[i] = 0;
+    __syncthreads();
+    const bool sx_ok = isfinite(sx), sy_ok = isfinite(sy);
+    for (int i = tid; i < N; i += kClusterThreads) {
+        atomicAdd(&cnt[sx_ok ? bucket_of(xs[i], xmin, sx, NB) : 0], 1);
+        atomicAdd(&cnt[NB + (sy_ok ? bucket_of(ys[i], ymin, sy, NB) : 0)], 1);
     }
     __syncthreads();
-    for (int k = 2; k <= P; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < 2 * P; i += kClusterThreads) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const bool up = ((i & (P - 1)) & k) == 0;
-                    const uint64_t ka = keys[i], kb = keys[ixj];
-                    const uint16_t ia = kid[i], ib = kid[ixj];
-                    const bool gt = (ka > kb) || (ka == kb && ia > ib);
-                    if (gt == up) {
-                        keys[i] = kb;
-                        keys[ixj] = ka;
-                        kid[i] = ib;
-                        kid[ixj] = ia;
-                    }
-                }
-            }
-            __syncthreads();
+    int crowded = 0;
+    for (int i = tid; i < 2 * NB; i += kClusterThreads) crowded |= (cnt[i] > kBucketMax);
+    crowded = __syncthreads_or(crowded);
+    if (!crowded) {
+        block_scan_int(cnt, 2 * NB, scratch);
+        for (int i = tid; i < N; i += kClusterThreads) {
+            L0[atomicAdd(&cnt[sx_ok ? bucket_of(xs[i], xmin, sx, NB) : 0], 1)] = static_cast<uint16_t>(i);
+            L0[atomicAdd(&cnt[NB + (sy_ok ? bucket_of(ys[i], ymin, sy, NB) : 0)], 1)] =
+                static_cast<uint16_t>(i);
         }
+        __syncthreads();  // cnt[bb] = end of bucket bb
+        for (int bb = tid; bb < 2 * NB; bb += kClusterThreads) {
+            const int s0 = bb > 0 ? cnt[bb - 1] : 0, s1 = cnt[bb];
+            const bool isx = bb < NB;
+            for (int i = s0 + 1; i < s1; ++i) {
+                const int t = L0[i];
+                const uint64_t kt = isx ? full_key(xs[t], ys[t]) : full_key(ys[t], xs[t]);
+                int j = i - 1;
+                while (j >= s0) {
+                    const int u = L0[j];
+                    const uint64_t ku = isx ? full_key(xs[u], ys[u]) : full_key(ys[u], xs[u]);
+                    if (ku < kt || (ku == kt && u < t)) break;
+                    L0[j + 1] = static_cast<uint16_t>(u);
+                    --j;
+                }
+                L0[j + 1] = static_cast<uint16_t>(t);
+            }
+        }
+        __syncthreads();
+    } else {
+        fallback_sort(xs, ys, N, P, reinterpret_cast<uint64_t*>(U), L0);
     }
-    // ids live above the keys region, so copying them into the level arrays is safe
-    for (int i = tid; i < N; i += kClusterThreads) {
-        lx0[i] = kid[i];
-        ly0[i] = kid[P + i];
+
+    // ---- level arrays (overlay U now that the sort is done)
+    uint16_t* L1 = reinterpret_cast<uint16_t*>(U);  // [2N]
+    uint16_t* scanv = L1 + 2 * N;
+    uint16_t* scanout = scanv + N;
+    uint16_t* posX = scanout + N;
+    uint16_t* posY = posX + N;
+    uint16_t* pos_cluster = posY + N;
+    uint16_t* seg_c0 = pos_cluster + N;
+    uint16_t* seg_g = seg_c0 + G;
+    uint8_t* seg_axis = reinterpret_cast<uint8_t*>(seg_g + G);
+    for (int p = tid; p < N; p += kClusterThreads) {
+        posX[L0[p]] = static_cast<uint16_t>(p);
+        posY[L0[N + p]] = static_cast<uint16_t>(p);
+        pos_cluster[p] = static_cast<uint16_t>(p / C);
     }
     for (int c = tid; c < G; c += kClusterThreads) {
         seg_c0[c] = 0;
@@ -181,48 +361,51 @@ __global__ void __launch_bounds__(kClusterThreads)
     }
     __syncthreads();
 
-    uint16_t *LX = lx0, *LY = ly0, *NX = lx1, *NY = ly1;
+    uint16_t *LX = L0, *LY = L0 + N, *NX = L1, *NY = L1 + N;
+    bool first = true;
     for (int gmax = G; gmax > 1; gmax = (gmax + 1) / 2) {
-        // A: split axis of every segment, from the ends of its sorted lists
+        // A: the previous level's children become segments; then each segment's axis
         for (int c = tid; c < G; c += kClusterThreads) {
-            const int c0 = seg_c0[c], g = seg_g[c];
+            int c0 = seg_c0[c], g = seg_g[c];
+            if (!first && g >= 2) {
+                const int gl = (g + 1) / 2;
+                if (c < c0 + gl) {
+                    g = gl;
+                } else {
+                    c0 += gl;
+                    g -= gl;
+                }
+                seg_c0[c] = static_cast<uint16_t>(c0);
+                seg_g[c] = static_cast<uint16_t>(g);
+            }
             if (c == c0 && g >= 2) {
                 const int lo = c0 * C, hi = min((c0 + g) * C, N) - 1;
-                const double ex = __dsub_rn(static_cast<double>(xs[LX[hi]]),
-                                            static_cast<double>(xs[LX[lo]]));
-                const double ey = __dsub_rn(static_cast<double>(ys[LY[hi]]),
-                                            static_cast<double>(ys[LY[lo]]));
+                const double ex = __dsub_rn(static_cast<double>(xs[LX[hi]]), static_cast<double>(xs[LX[lo]]));
+                const double ey = __dsub_rn(static_cast<double>(ys[LY[hi]]), static_cast<double>(ys[LY[lo]]));
                 seg_axis[c0] = (ex >= ey) ? 0 : 1;
             }
         }
+        first = false;
         __syncthreads();
-        // B: membership of the left part, read off the split-axis list
+        // C: is the other list's element in the left part?  (its rank on the split axis)
         for (int p = tid; p < N; p += kClusterThreads) {
-            const int c = p / C;
-            const int c0 = seg_c0[c], g = seg_g[c];
-            if (g >= 2) {
-                const int lo = c0 * C, nl = ((g + 1) / 2) * C;
-                const uint16_t t = seg_axis[c0] ? LY[p] : LX[p];
-                flag[t] = (p - lo < nl) ? 1 : 0;
-            }
-        }
-        __syncthreads();
-        // C: prefix count of left members along the other list
-        for (int p = tid; p < N; p += kClusterThreads) {
-            const int c = p / C;
+            const int c = pos_cluster[p];
             const int c0 = seg_c0[c], g = seg_g[c];
             uint16_t v = 0;
             if (g >= 2) {
-                const uint16_t t = seg_axis[c0] ? LX[p] : LY[p];
-                v = flag[t];
+                const int lo = c0 * C, nl = ((g + 1) / 2) * C;
+                const int ax = seg_axis[c0];
+                const int t = ax ? LX[p] : LY[p];
+                const int pa = ax ? posY[t] : posX[t];
+                v = (pa - lo < nl) ? 1 : 0;
             }
             scanv[p] = v;
         }
         __syncthreads();
-        block_exclusive_scan_u16(scanv, scanout, N, warp_tot);
+        block_exclusive_scan_u16(scanv, scanout, N, scratch);
         // D: stable partition of the other list; the axis list is already split
         for (int p = tid; p < N; p += kClusterThreads) {
-            const int c = p / C;
+            const int c = pos_cluster[p];
             const int c0 = seg_c0[c], g = seg_g[c];
             if (g < 2) {
                 NX[p] = LX[p];
@@ -235,23 +418,11 @@ __global__ void __launch_bounds__(kClusterThreads)
             if (seg_axis[c0]) {
                 NY[p] = LY[p];
                 NX[dst] = LX[p];
+                posX[LX[p]] = static_cast<uint16_t>(dst);
             } else {
                 NX[p] = LX[p];
                 NY[dst] = LY[p];
-            }
-        }
-        __syncthreads();
-        // E: children become the segments of the next level
-        for (int c = tid; c < G; c += kClusterThreads) {
-            const int c0 = seg_c0[c], g = seg_g[c];
-            if (g >= 2) {
-                const int gl = (g + 1) / 2;
-                if (c < c0 + gl) {
-                    seg_g[c] = static_cast<uint16_t>(gl);
-                } else {
-                    seg_c0[c] = static_cast<uint16_t>(c0 + gl);
-                    seg_g[c] = static_cast<uint16_t>(g - gl);
-                }
+                posY[LY[p]] = static_cast<uint16_t>(dst);
             }
         }
         uint16_t* t0 = LX; LX = NX; NX = t0;
@@ -264,13 +435,13 @@ __global__ void __launch_bounds__(kClusterThreads)
     for (int c = tid; c < G; c += kClusterThreads) {
         const int lo = c * C;
         const int n = min(C, N - lo);
-        for (int s = 0; s < n; ++s) {
-            const int id = LX[lo + s];
+        for (int s2 = 0; s2 < n; ++s2) {
+            const int id = LX[lo + s2];
             int rank = 0;
             for (int u = 0; u < n; ++u) rank += (LX[lo + u] < id);
             out[lo + rank] = id;
         }
-        for (int s = n; s < C; ++s) out[lo + s] = -1;
+        for (int s2 = n; s2 < C; ++s2) out[lo + s2] = -1;
     }
 }
 
@@ -278,8 +449,18 @@ __global__ void __launch_bounds__(kClusterThreads)
 // neighbours: R nearest centroids per cluster
 // ---------------------------------------------------------------------------
 
-constexpr int kNbrThreads = 128;
+constexpr int kNbrThreads = 256;
+constexpr int kNbrWarps = kNbrThreads / 32;
 
+// (d, h) < (d', h') in the neighbour order
+__device__ __forceinline__ bool nbr_less(double d, int h, double d2, int h2) {
+    return d < d2 || (d == d2 && h < h2);
+}
+
+// One warp per query cluster g.  Every CTA first computes the G centroids of its image in
+// shared memory (fp64, slot order, as the header states).  Lane l scores the candidate
+// clusters h = l, l + 32, ... and keeps its own top-RMAX by (dist2, h); R rounds of a
+// warp-wide argmin over the lanes' heads then pop the R nearest in order.
 template <int RMAX>
 __global__ void __launch_bounds__(kNbrThreads)
     neighbors_kernel(const float* __restrict__ xy, const int32_t* __restrict__ clusters, int N,
@@ -309,21 +490,22 @@ __global__ void __launch_bounds__(kNbrThreads)
     }
     __syncthreads();
 
-    const int g = blockIdx.x * kNbrThreads + threadIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = blockIdx.x * kNbrWarps + warp;
     if (g >= G) return;
     double bd[RMAX];
     int bh[RMAX];
 #pragma unroll
     for (int r = 0; r < RMAX; ++r) {
         bd[r] = DBL_MAX;
-        bh[r] = -1;
+        bh[r] = 0x7fffffff;
     }
     const double gx = cx[g], gy = cy[g];
-    for (int h = 0; h < G; ++h) {
+    for (int h = lane; h < G; h += 32) {
         const double dx = __dsub_rn(cx[h], gx);
         const double dy = __dsub_rn(cy[h], gy);
         const double d = __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy));
-        if (d < bd[RMAX - 1]) {  // strict: an equal distance keeps the lower id already held
+        if (d < bd[RMAX - 1]) {  // h ascends within a lane, so equal d keeps the lower id
             bool placed = false;
 #pragma unroll
             for (int r = RMAX - 1; r >= 0; --r) {
@@ -341,12 +523,31 @@ __global__ void __launch_bounds__(kNbrThreads)
         }
     }
     int32_t* row = nbr + (static_cast<size_t>(b) * G + g) * M;
+    for (int r = 0; r < R; ++r) {
+        // warp argmin of the lanes' heads
+        double d = bd[0];
+        int h = bh[0];
 #pragma unroll
-    for (int r = 0; r < RMAX; ++r) {
-        if (r >= R) break;
-        const int h = bh[r];
-        for (int s = 0; s < C; ++s)
-            row[r * C + s] = (h >= 0) ? cl[static_cast<size_t>(h) * C + s] : -1;
+        for (int o = 16; o > 0; o >>= 1) {
+            const double d2 = __shfl_xor_sync(0xffffffffu, d, o);
+            const int h2 = __shfl_xor_sync(0xffffffffu, h, o);
+            if (nbr_less(d2, h2, d, h)) {
+                d = d2;
+                h = h2;
+            }
+        }
+        const bool valid = (h != 0x7fffffff);
+        if (valid && bh[0] == h) {  // the owner pops its head
+#pragma unroll
+            for (int q = 0; q < RMAX - 1; ++q) {
+                bd[q] = bd[q + 1];
+                bh[q] = bh[q + 1];
+            }
+            bd[RMAX - 1] = DBL_MAX;
+            bh[RMAX - 1] = 0x7fffffff;
+        }
+        for (int s = lane; s < C; s += 32)
+            row[r * C + s] = valid ? cl[static_cast<size_t>(h) * C + s] : -1;
     }
 }
 
@@ -370,7 +571,7 @@ cudaError_t launch_neighbors(const float* xy, const int32_t* clusters, int B, in
                              int32_t* nbr, cudaStream_t st) {
     const int G = (N + C - 1) / C;
     const size_t smem = neighbors_smem_bytes(G);
-    dim3 grid((G + kNbrThreads - 1) / kNbrThreads, B);
+    dim3 grid((G + kNbrWarps - 1) / kNbrWarps, B);
     cudaError_t e;
     if (M / C <= 8) {
         e = ensure_smem<neighbors_kernel<8>>(smem);

@@ -98,10 +98,11 @@ struct KnnArgs {
     int32_t* csr;       // [B][Q*K]
     int32_t* csr_off;   // [B][N + 1]
     float* dp_part;     // [query blocks][d/32]
+    int* counter;       // work counter of the token-side kernel
 };
 
 struct KnnWorkspace {
-    size_t w, keys, csr, csr_off, dp_part, total;
+    size_t w, keys, csr, csr_off, dp_part, counter, total;
     int query_blocks;
 };
 KnnWorkspace knn_workspace_layout(int B, int Q, int N, int d, int K);

@@ -176,6 +176,35 @@ acl_status acl_cluster_attn_bwd(const acl_bf16* Q, const acl_bf16* K, const acl_
                                 float* dbias_coef, void* workspace, size_t ws_bytes,
                                 acl_stream_t stream);
 
+/* Size of the library-owned scratch array used by acl_cluster_attn_bwd_noalloc. */
+#define ACL_NOALLOC_ATTN_WS_BYTES (4u << 20)
+
+/*
+ * acl_cluster_attn_bwd_noalloc -- acl_cluster_attn_bwd without a caller workspace.
+ * The pages have no counterpart: this entry point exists for callers that cannot
+ * allocate device memory (a host framework that forbids allocation on its hot path, or a
+ * runtime that only hands out pre-registered buffers).  It computes exactly what
+ * acl_cluster_attn_bwd computes, with the same arguments minus workspace/ws_bytes; its
+ * scratch is a file-scope device array of ACL_NOALLOC_ATTN_WS_BYTES (4 MiB) that every
+ * GPU loading the library holds until the process exits.  Nothing is allocated.
+ *  - Sizes whose acl_cluster_attn_workspace(B, N, H, C, M) exceeds
+ *    ACL_NOALLOC_ATTN_WS_BYTES return ACL_ERR_UNSUPPORTED (the regular entry point with a
+ *    caller workspace has no such limit); bad sizes return ACL_ERR_INVALID_ARG.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before any
+ *    stream capture on the device.
+ *  - All calls share the one array, which keeps the last call's contents; nothing in it
+ *    needs to start at zero (every scratch value is written before it is read).  Calls
+ *    that overlap on the GPU (on different streams, without ordering) race on it.
+ */
+acl_status acl_cluster_attn_bwd_noalloc(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V,
+                                        const float* coords, const int32_t* clusters,
+                                        const int32_t* nbr, const float* bias_coef,
+                                        int B, int N, int H, int D, int C, int M, float scale,
+                                        const acl_bf16* O, const acl_bf16* dO, const float* lse,
+                                        acl_bf16* dQ, acl_bf16* dK, acl_bf16* dV,
+                                        float* dbias_coef, acl_stream_t stream);
+
 /*
  * acl_knn_table -- KNN cache lookup table (a5).
  * Passage: AFF notes, "Key Designs" 3 (KNN Cache Lookup): an H x W x K table of

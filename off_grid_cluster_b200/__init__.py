@@ -37,6 +37,8 @@ SIGNATURES = {
                                   _P, _P, _P]),
     "acl_cluster_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F,
                                   _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P]),
+    "acl_cluster_attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                          _F, _P, _P, _P, _P, _P, _P, _P, _P]),
     "acl_knn_table": (_I, [_P, _I, _I, _I, _I, _I, _P, _P]),
     "acl_knn_gather_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "acl_knn_gather_fwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P]),
@@ -202,6 +204,32 @@ def acl_cluster_attn_bwd(Q, K, V, coords, clusters, nbr, bias_coef, scale: float
           _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbias_coef), _ptr(workspace),
           workspace.numel() * workspace.element_size(), _stream(stream))
     return dQ, dK, dV, dbias_coef
+
+
+def acl_cluster_attn_bwd_noalloc(Q, K, V, coords, clusters, nbr, bias_coef, scale: float | None,
+                                 O, dO, lse, dQ=None, dK=None, dV=None, dbias_coef=None,
+                                 stream=None):
+    """acl_cluster_attn_bwd with the library's own scratch array instead of a workspace.
+
+    For callers that cannot allocate device scratch.  The outputs are allocated here only
+    when not passed in (pass them to allocate nothing).  Raises AclError with
+    ACL_ERR_UNSUPPORTED when the sizes need more than ACL_NOALLOC_ATTN_WS_BYTES.
+    """
+    B, N, H, D, C, M = _attn_shapes(Q, K, V, coords, clusters, nbr, bias_coef)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _need(dO, "dO", torch.bfloat16, (B, N, H, D))
+    _need(lse, "lse", torch.float32, (B, N, H))
+    dQ = _out(dQ, (B, N, H, D), torch.bfloat16, Q, "dQ")
+    dK = _out(dK, (B, N, H, D), torch.bfloat16, Q, "dK")
+    dV = _out(dV, (B, N, H, D), torch.bfloat16, Q, "dV")
+    dbias_coef = _out(dbias_coef, (H, 3), torch.float32, Q, "dbias_coef")
+    _call("acl_cluster_attn_bwd_noalloc", _ptr(Q), _ptr(K), _ptr(V), _ptr(coords), _ptr(clusters),
+          _ptr(nbr), _ptr(bias_coef), B, N, H, D, C, M, scale, _ptr(O), _ptr(dO), _ptr(lse),
+          _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbias_coef), _stream(stream))
+    return dQ, dK, dV, dbias_coef
+
+
+ACL_NOALLOC_ATTN_WS_BYTES = 4 << 20
 
 
 # ---------------------------------------------------------------- KNN gather

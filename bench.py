@@ -45,15 +45,17 @@ sys.path.insert(0, ROOT)
 METRIC = "cluster-attn fwd+bwd tokens/s & KNN-gather queries/s; % of B200 HBM roofline"
 WORKLOAD = "stage1-1024px-b8-n2048-d128-h4-c8-m48 + decoder-knn-gather-q4096-k8"
 FALLBACK_HBM_GBS = 6650.0
-OPS = ("cluster", "neighbors", "attn_fwd", "attn_bwd", "knn_table", "knn_fwd", "knn_bwd")
+OPS = ("cluster", "neighbors", "attn_fwd", "attn_bwd", "knn_table", "knn_index", "knn_fwd",
+       "knn_bwd")
 KERNELS = {
     "cluster": ["cluster_kernel"],
     "neighbors": ["neighbors_kernel"],
-    "attn_fwd": ["attn_fwd_kernel"],
-    "attn_bwd": ["attn_bwd_query_kernel", "attn_bwd_key_kernel"],
+    "attn_fwd": ["attn_fwd_union_kernel"],
+    "attn_bwd": ["attn_bwd_query_union_kernel", "attn_bwd_key_union_kernel"],
     "knn_table": ["knn_table_kernel"],
-    "knn_fwd": ["knn_fwd_kernel"],
-    "knn_bwd": ["knn_bwd_query_kernel", "knn_csr_kernel", "knn_bwd_token_kernel"],
+    "knn_index": ["knn_csr_kernel"],
+    "knn_fwd": ["knn_fwd_shared_kernel"],
+    "knn_bwd": ["knn_bwd_query_shared_kernel", "knn_bwd_token_kernel"],
 }
 # DRAM bytes per launch measured by ncu for each call (sum over its kernels), with the
 # sha256 of the CUDA source the counters were taken on; a stale hash reports null.
@@ -137,6 +139,7 @@ def algorithmic_bytes(B, N, H, Q, d, K, GH, GW, C=8, M=48) -> dict:
         "attn_fwd": B * N * (H * (3 * 64 + 64 + 4) + per_tok_meta) + H * 12,
         "attn_bwd": B * N * (H * (4 * 64 + 4 + 3 * 64) + per_tok_meta) + 2 * H * 12,
         "knn_table": B * (N * 8 + GH * GW * K * 4),
+        "knn_index": B * (Q * 8 + GH * GW * K * 4 + Q * K * 4 + (N + 1) * 4),
         "knn_fwd": B * (Q * (8 + 4 * K + 2 * d) + N * (2 * d + 8)) + 4 * d // 32,
         "knn_bwd": B * (Q * (8 + 4 * K + 2 * d + 8) + N * (2 * d + 8 + 2 * d)) + 8 * d // 32,
     }
@@ -244,18 +247,23 @@ class StepSet:
         elif name == "knn_fwd":
             acl.acl_knn_gather_fwd(i["queries"], i["feats"], i["coords"], o["table"], i["p"],
                                    out=o["out"], stream=stream)
+        elif name == "knn_index":
+            acl.acl_knn_gather_index(i["queries"], o["table"], self.N, self.d, self.ws_knn,
+                                     stream=stream)
         elif name == "knn_bwd":
-            acl.acl_knn_gather_bwd(i["queries"], i["feats"], i["coords"], o["table"], i["p"],
-                                   i["dout"], dfeats=o["dfeats"], dqueries=o["dqueries"],
-                                   dp=o["dp"], workspace=self.ws_knn, stream=stream)
+            acl.acl_knn_gather_bwd_indexed(i["queries"], i["feats"], i["coords"], o["table"],
+                                           i["p"], i["dout"], self.ws_knn, dfeats=o["dfeats"],
+                                           dqueries=o["dqueries"], dp=o["dp"], stream=stream)
         else:
             raise KeyError(name)
 
-    def step(self, stream, events=None, stream2=None):
-        """The seven calls.  With stream2 the KNN chain (table -> gather fwd -> bwd) runs
-        on stream2 concurrently with the attention chain (cluster -> neighbours -> attn
-        fwd -> bwd) on stream; events[2j], events[2j+1] bracket call j on its stream."""
-        if stream2 is None:
+    def step(self, stream, events=None, streams=None):
+        """The eight calls.  With streams = (s2, s3) the KNN chain (table -> gather fwd ->
+        indexed bwd) runs on s2 and the inverse index (after the table) on s3, concurrently
+        with the attention chain (cluster -> neighbours -> attn fwd -> bwd) on stream;
+        events[2j], events[2j+1] bracket call j on its stream."""
+        torch = self.torch
+        if streams is None:
             for j, name in enumerate(OPS):
                 if events is not None:
                     events[2 * j].record(stream)
@@ -263,18 +271,27 @@ class StepSet:
                 if events is not None:
                     events[2 * j + 1].record(stream)
             return
-        torch = self.torch
-        fork, join = torch.cuda.Event(), torch.cuda.Event()
+        s2, s3 = streams
+        home = {"knn_table": s2, "knn_fwd": s2, "knn_bwd": s2, "knn_index": s3}
+        fork, tab, idx, join = (torch.cuda.Event() for _ in range(4))
         fork.record(stream)
-        stream2.wait_event(fork)
+        s2.wait_event(fork)
         for j, name in enumerate(OPS):
-            st = stream2 if name.startswith("knn") else stream
+            st = home.get(name, stream)
+            if name == "knn_index":
+                s3.wait_event(tab)
+            if name == "knn_bwd":
+                s2.wait_event(idx)
             if events is not None:
                 events[2 * j].record(st)
             self.op(name, st)
             if events is not None:
                 events[2 * j + 1].record(st)
-        join.record(stream2)
+            if name == "knn_table":
+                tab.record(s2)
+            if name == "knn_index":
+                idx.record(s3)
+        join.record(s2)
         stream.wait_event(join)
 
 
@@ -305,7 +322,7 @@ def run_gpu(args, rank: int, world: int):
     n_sets = max(2, math.ceil(4 * l2 / set_bytes))
     sets = [base] + [StepSet(sb, device, acl, torch) for _ in range(n_sets - 1)]
     stream = torch.cuda.Stream(device)
-    stream2 = None if args.serial else torch.cuda.Stream(device)
+    streams = None if args.serial else (torch.cuda.Stream(device), torch.cuda.Stream(device))
 
     # eager warm-up of every call (kernel attributes, lazy module loading), then capture
     with torch.cuda.stream(stream):
@@ -319,7 +336,7 @@ def run_gpu(args, rank: int, world: int):
         evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            s.step(stream, evs, stream2)
+            s.step(stream, evs, streams)
         graphs.append(g)
         events.append(evs)
     launches_per_step = (acl.acl_launch_count() - launches0) // len(sets)
@@ -381,11 +398,11 @@ def run_gpu(args, rank: int, world: int):
         breakdown[name] = {"us": round(per_op[j] * 1e3, 2), "alg_MB": round(abytes[name] / 1e6, 3),
                            "GB_s": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
     attn_ms = per_op[OPS.index("attn_fwd")] + per_op[OPS.index("attn_bwd")]
-    knn_ms = per_op[OPS.index("knn_fwd")] + per_op[OPS.index("knn_bwd")]
+    knn_ms = sum(per_op[OPS.index(n)] for n in ("knn_index", "knn_fwd", "knn_bwd"))
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, base, stream, torch, acl, tokens_per_step=world * B * N)
+        e2e = run_e2e(args, base, stream, streams, torch, acl, tokens_per_step=world * B * N)
         e2e_ms = max_over_ranks(e2e.pop("_ms"), world, device)
         e2e["value"] = round(world * B * N / (e2e_ms * 1e-3), 1)
         e2e["ms_per_step"] = round(e2e_ms, 4)
@@ -405,7 +422,7 @@ def run_gpu(args, rank: int, world: int):
                    "l2": f"rotating {n_sets} input sets, {n_sets * set_bytes / 1e6:.0f} MB total "
                          f">= 4 x L2 ({l2 / 1e6:.0f} MB)",
                    "timing": "CUDA graph per set, CUDA events on the launching stream",
-                   "streams": 1 if args.serial else 2,
+                   "streams": 1 if args.serial else 3,
                    "parallelism": f"replicas x{world} (images sharded, no collective)"},
         "parts": {
             "knn_queries_per_s": round(world * B * Q / (step_ms * 1e-3), 1),
@@ -431,7 +448,7 @@ def run_gpu(args, rank: int, world: int):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, s: StepSet, stream, torch, acl, tokens_per_step: int) -> dict:
+def run_e2e(args, s: StepSet, stream, streams, torch, acl, tokens_per_step: int) -> dict:
     """The step through the public entry points from pinned host memory, copies inside."""
     hin = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in s.inputs.items()}
     for k, v in s.inputs.items():
@@ -443,7 +460,7 @@ def run_e2e(args, s: StepSet, stream, torch, acl, tokens_per_step: int) -> dict:
     def one():
         for k, v in hin.items():
             s.inputs[k].copy_(v, non_blocking=True)
-        s.step(stream)
+        s.step(stream, None, streams)
         for k, v in s.outputs.items():
             hout[k].copy_(v, non_blocking=True)
 

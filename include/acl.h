@@ -220,7 +220,8 @@ acl_status acl_cluster_attn_bwd_noalloc(const acl_bf16* Q, const acl_bf16* K, co
 acl_status acl_knn_table(const float* coords, int B, int N, int H, int W, int K,
                          int32_t* table, acl_stream_t stream);
 
-/* Workspace bytes acl_knn_gather_bwd needs for these sizes (0 on bad sizes). */
+/* Workspace bytes acl_knn_gather_bwd (and acl_knn_gather_index +
+ * acl_knn_gather_bwd_indexed) need for these sizes (0 on bad sizes). */
 size_t acl_knn_gather_workspace(int B, int Q, int N, int d, int K);
 
 /*
@@ -264,6 +265,36 @@ acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16
                               int H, int W, int K, const float* p, const acl_bf16* dOut,
                               acl_bf16* dfeats, float* dqueries, float* dp,
                               void* workspace, size_t ws_bytes, acl_stream_t stream);
+
+/*
+ * acl_knn_gather_index -- the first stage of acl_knn_gather_bwd on its own: the inverse
+ * index (for every token, its (query, slot) entries in ascending order, by a stable
+ * counting sort) built from the queries' cells and the table alone, written into the
+ * workspace.  Passage: AFF notes, "Key Designs" 3 (q quantised to its cell; the cell's
+ * table row names its K tokens).  The index depends neither on the features nor on dOut,
+ * so it can be built as soon as the table exists, e.g. on another stream while the
+ * forward gather runs.
+ * queries [B][Q][2] fp32; table [B][H][W][K] int32 (entries in [-1, N)); d selects the
+ * workspace layout and must equal the d of the backward call that uses the index.
+ * workspace: as for acl_knn_gather_bwd (same sizes); only its index regions are written.
+ * Limits: as acl_knn_gather_bwd.
+ */
+acl_status acl_knn_gather_index(const float* queries, int B, int Q, int N, int d,
+                                const int32_t* table, int H, int W, int K, void* workspace,
+                                size_t ws_bytes, acl_stream_t stream);
+
+/*
+ * acl_knn_gather_bwd_indexed -- acl_knn_gather_bwd without its first stage: the same
+ * arguments and results, reading the inverse index that acl_knn_gather_index wrote into
+ * this workspace for the same queries, table and sizes (stream-ordered before this call).
+ * The workspace's other regions are overwritten.  An index built for other inputs gives
+ * wrong dfeats; nothing checks this.
+ */
+acl_status acl_knn_gather_bwd_indexed(const float* queries, int B, int Q, const acl_bf16* feats,
+                                      const float* coords, int N, int d, const int32_t* table,
+                                      int H, int W, int K, const float* p, const acl_bf16* dOut,
+                                      acl_bf16* dfeats, float* dqueries, float* dp,
+                                      void* workspace, size_t ws_bytes, acl_stream_t stream);
 
 #ifdef __cplusplus
 }

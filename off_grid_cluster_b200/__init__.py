@@ -44,6 +44,9 @@ SIGNATURES = {
     "acl_knn_gather_fwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P]),
     "acl_knn_gather_bwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P,
                                 _P, _P, _Z, _P]),
+    "acl_knn_gather_index": (_I, [_P, _I, _I, _I, _I, _P, _I, _I, _I, _P, _Z, _P]),
+    "acl_knn_gather_bwd_indexed": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P,
+                                        _P, _P, _P, _P, _Z, _P]),
 }
 
 
@@ -269,9 +272,35 @@ def acl_knn_gather_fwd(queries, feats, coords, table, p, out=None, stream=None):
     return out
 
 
+def acl_knn_gather_index(queries, table, N: int, d: int, workspace: torch.Tensor, stream=None):
+    """Build the backward's inverse index (from the queries' cells and the table) in
+    `workspace` (at least acl_knn_gather_workspace(B, Q, N, d, K) bytes)."""
+    _need(queries, "queries", torch.float32)
+    B, Q = queries.shape[:2]
+    _need(table, "table", torch.int32)
+    H, W, K = table.shape[1:]
+    _call("acl_knn_gather_index", _ptr(queries), B, Q, N, d, _ptr(table), H, W, K,
+          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    return workspace
+
+
+def acl_knn_gather_bwd_indexed(queries, feats, coords, table, p, dOut, workspace: torch.Tensor,
+                               dfeats=None, dqueries=None, dp=None, stream=None):
+    """acl_knn_gather_bwd reading the inverse index that acl_knn_gather_index wrote into
+    `workspace` -> (dfeats, dqueries, dp)."""
+    return _gather_bwd("acl_knn_gather_bwd_indexed", queries, feats, coords, table, p, dOut,
+                       dfeats, dqueries, dp, workspace, stream)
+
+
 def acl_knn_gather_bwd(queries, feats, coords, table, p, dOut, dfeats=None, dqueries=None,
                        dp=None, workspace: torch.Tensor | None = None, stream=None):
     """KNN gather backward -> (dfeats [B,N,d] bf16, dqueries [B,Q,2] f32, dp [d/32] f32)."""
+    return _gather_bwd("acl_knn_gather_bwd", queries, feats, coords, table, p, dOut, dfeats,
+                       dqueries, dp, workspace, stream)
+
+
+def _gather_bwd(fn, queries, feats, coords, table, p, dOut, dfeats, dqueries, dp, workspace,
+                stream):
     B, Q, N, d, H, W, K = _gather_shapes(queries, feats, coords, table, p)
     _need(dOut, "dOut", torch.bfloat16, (B, Q, d))
     dfeats = _out(dfeats, (B, N, d), torch.bfloat16, feats, "dfeats")
@@ -280,7 +309,7 @@ def acl_knn_gather_bwd(queries, feats, coords, table, p, dOut, dfeats=None, dque
     need = acl_knn_gather_workspace(B, Q, N, d, K)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=feats.device)
-    _call("acl_knn_gather_bwd", _ptr(queries), B, Q, _ptr(feats), _ptr(coords), N, d,
+    _call(fn, _ptr(queries), B, Q, _ptr(feats), _ptr(coords), N, d,
           _ptr(table), H, W, K, _ptr(p), _ptr(dOut), _ptr(dfeats), _ptr(dqueries), _ptr(dp),
           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     return dfeats, dqueries, dp

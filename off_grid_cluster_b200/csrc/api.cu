@@ -53,6 +53,39 @@ acl_status check_gather(const float* queries, int B, int Q, const acl_bf16* feat
     return ACL_OK;
 }
 
+void map_knn_workspace(acl::KnnArgs& a, uint8_t* ws, const acl::KnnWorkspace& L) {
+    a.w = reinterpret_cast<float*>(ws + L.w);
+    a.keys = reinterpret_cast<int32_t*>(ws + L.keys);
+    a.csr = reinterpret_cast<int32_t*>(ws + L.csr);
+    a.csr_off = reinterpret_cast<int32_t*>(ws + L.csr_off);
+    a.dp_part = reinterpret_cast<float*>(ws + L.dp_part);
+    a.chunk_tok = reinterpret_cast<int32_t*>(ws + L.chunk_tok);
+    a.chunk_off = reinterpret_cast<int32_t*>(ws + L.chunk_off);
+    a.heavy = reinterpret_cast<int32_t*>(ws + L.heavy);
+    a.heavy_count = reinterpret_cast<int32_t*>(ws + L.heavy_count);
+    a.heavy_cap = L.heavy_cap;
+}
+
+// Validation and argument set-up shared by the two backward entry points.
+acl_status setup_gather_bwd(const float* queries, int B, int Q, const acl_bf16* feats,
+                            const float* coords, int N, int d, const int32_t* table, int H, int W,
+                            int K, const float* p, const acl_bf16* dOut, acl_bf16* dfeats,
+                            float* dqueries, float* dp, void* workspace, size_t ws_bytes,
+                            acl::KnnArgs& a) {
+    acl_status st = check_gather(queries, B, Q, feats, coords, N, d, table, H, W, K, p);
+    if (st != ACL_OK) return st;
+    if ((Q > 0 && (!dOut || !dqueries)) || !dfeats || !dp) return ACL_ERR_INVALID_ARG;
+    if (!aligned(dOut, 16) || !aligned(dfeats, 16) || !aligned(dqueries, 8)) return ACL_ERR_INVALID_ARG;
+    if (Q > ACL_MAX_GATHER_Q || N > ACL_MAX_TABLE_N) return ACL_ERR_UNSUPPORTED;
+    const acl::KnnWorkspace L = acl::knn_workspace_layout(B, Q, N, d, K);
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < L.total) return ACL_ERR_WORKSPACE;
+    a.queries = queries; a.feats = BF(feats); a.xy = coords; a.table = table; a.p = p;
+    a.B = B; a.Q = Q; a.N = N; a.d = d; a.GH = H; a.GW = W; a.K = K;
+    a.dout = BF(dOut); a.dfeats = BFm(dfeats); a.dq = dqueries; a.dp = dp;
+    map_knn_workspace(a, static_cast<uint8_t*>(workspace), L);
+    return ACL_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -175,29 +208,46 @@ acl_status acl_knn_gather_fwd(const float* queries, int B, int Q, const acl_bf16
     return cuda_status(acl::launch_knn_fwd(a, S(stream)));
 }
 
+acl_status acl_knn_gather_index(const float* queries, int B, int Q, int N, int d,
+                                const int32_t* table, int H, int W, int K, void* workspace,
+                                size_t ws_bytes, acl_stream_t stream) {
+    if ((Q > 0 && !queries) || !table) return ACL_ERR_INVALID_ARG;
+    if (B < 1 || Q < 0 || N < 1 || d < 32 || d % 32 != 0 || H < 1 || W < 1 || K < 1)
+        return ACL_ERR_INVALID_ARG;
+    if (d > ACL_MAX_GATHER_D || K > ACL_MAX_KNN_K || Q > ACL_MAX_GATHER_Q || N > ACL_MAX_TABLE_N)
+        return ACL_ERR_UNSUPPORTED;
+    if (static_cast<long long>(H) * W * K > 0x7fffffffLL) return ACL_ERR_UNSUPPORTED;
+    if (!aligned(queries, 8)) return ACL_ERR_INVALID_ARG;
+    const acl::KnnWorkspace L = acl::knn_workspace_layout(B, Q, N, d, K);
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < L.total) return ACL_ERR_WORKSPACE;
+    acl::KnnArgs a = {};
+    a.queries = queries; a.table = table;
+    a.B = B; a.Q = Q; a.N = N; a.d = d; a.GH = H; a.GW = W; a.K = K;
+    map_knn_workspace(a, static_cast<uint8_t*>(workspace), L);
+    return cuda_status(acl::launch_knn_index(a, S(stream)));
+}
+
+acl_status acl_knn_gather_bwd_indexed(const float* queries, int B, int Q, const acl_bf16* feats,
+                                      const float* coords, int N, int d, const int32_t* table,
+                                      int H, int W, int K, const float* p, const acl_bf16* dOut,
+                                      acl_bf16* dfeats, float* dqueries, float* dp,
+                                      void* workspace, size_t ws_bytes, acl_stream_t stream) {
+    acl::KnnArgs a = {};
+    const acl_status st = setup_gather_bwd(queries, B, Q, feats, coords, N, d, table, H, W, K, p,
+                                           dOut, dfeats, dqueries, dp, workspace, ws_bytes, a);
+    if (st != ACL_OK) return st;
+    return cuda_status(acl::launch_knn_bwd_indexed(a, S(stream)));
+}
+
 acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16* feats,
                               const float* coords, int N, int d, const int32_t* table, int H, int W,
                               int K, const float* p, const acl_bf16* dOut, acl_bf16* dfeats,
                               float* dqueries, float* dp, void* workspace, size_t ws_bytes,
                               acl_stream_t stream) {
-    acl_status st = check_gather(queries, B, Q, feats, coords, N, d, table, H, W, K, p);
-    if (st != ACL_OK) return st;
-    if ((Q > 0 && (!dOut || !dqueries)) || !dfeats || !dp) return ACL_ERR_INVALID_ARG;
-    if (!aligned(dOut, 16) || !aligned(dfeats, 16) || !aligned(dqueries, 8)) return ACL_ERR_INVALID_ARG;
-    if (Q > ACL_MAX_GATHER_Q || N > ACL_MAX_TABLE_N) return ACL_ERR_UNSUPPORTED;
-    const acl::KnnWorkspace L = acl::knn_workspace_layout(B, Q, N, d, K);
-    if (!workspace || !aligned(workspace, 256) || ws_bytes < L.total) return ACL_ERR_WORKSPACE;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
     acl::KnnArgs a = {};
-    a.queries = queries; a.feats = BF(feats); a.xy = coords; a.table = table; a.p = p;
-    a.B = B; a.Q = Q; a.N = N; a.d = d; a.GH = H; a.GW = W; a.K = K;
-    a.dout = BF(dOut); a.dfeats = BFm(dfeats); a.dq = dqueries; a.dp = dp;
-    a.w = reinterpret_cast<float*>(ws + L.w);
-    a.keys = reinterpret_cast<int32_t*>(ws + L.keys);
-    a.csr = reinterpret_cast<int32_t*>(ws + L.csr);
-    a.csr_off = reinterpret_cast<int32_t*>(ws + L.csr_off);
-    a.dp_part = reinterpret_cast<float*>(ws + L.dp_part);
-    a.counter = reinterpret_cast<int*>(ws + L.counter);
+    const acl_status st = setup_gather_bwd(queries, B, Q, feats, coords, N, d, table, H, W, K, p,
+                                           dOut, dfeats, dqueries, dp, workspace, ws_bytes, a);
+    if (st != ACL_OK) return st;
     return cuda_status(acl::launch_knn_bwd(a, S(stream)));
 }
 

@@ -13,8 +13,10 @@
 // GPU design.  One 1024-thread CTA per image holds all of the image in shared
 // memory.  Instead of re-sorting every segment at every level (what a literal
 // recursion does), the CTA sorts the tokens once by (x, y, id) and once by
-// (y, x, id) -- one bitonic network over both lists -- and then walks the
-// bisection tree breadth first: at each level a segment's extent is read off
+// (y, x, id) -- a counting sort into N monotone buckets per axis followed by an
+// exact insertion sort inside each bucket, or, when some bucket is crowded
+// (repeated or tightly packed coordinates), a bitonic network over packed keys --
+// and then walks the bisection tree breadth first: at each level a segment's extent is read off
 // the ends of its two sorted lists, its left part is the first ceil(g/2)*C
 // entries of the list on its split axis, and the other list is stably
 // partitioned with one block-wide prefix sum.  Both lists stay sorted inside

@@ -93,17 +93,21 @@ struct KnnArgs {
     bf16* dfeats;
     float* dq;
     float* dp;
-    float* w;           // [B][Q][d/32][K]
-    int32_t* keys;      // [B][Q*K]
+    float* w;           // [B][Q][K][d/32]
+    int32_t* keys;      // [B][Q*K] token of every (query, slot) entry
     int32_t* csr;       // [B][Q*K]
     int32_t* csr_off;   // [B][N + 1]
     float* dp_part;     // [query blocks][d/32]
-    int* counter;       // work counter of the token-side kernel
+    int32_t* chunk_tok;  // [B][chunks + 1] first token of every light chunk of the token pass
+    int32_t* chunk_off;  // [B][chunks + 1] first entry of that token
+    int32_t* heavy;     // [B][slices][heavy_cap] tokens with many entries, per CSR slice
+    int32_t* heavy_count;  // [B][slices]
+    int heavy_cap;
 };
 
 struct KnnWorkspace {
-    size_t w, keys, csr, csr_off, dp_part, counter, total;
-    int query_blocks;
+    size_t w, keys, csr, csr_off, dp_part, chunk_tok, chunk_off, heavy, heavy_count, total;
+    int query_blocks, heavy_cap;
 };
 KnnWorkspace knn_workspace_layout(int B, int Q, int N, int d, int K);
 
@@ -111,6 +115,8 @@ size_t knn_table_smem_bytes(int N, int nbins);
 cudaError_t launch_knn_table(const float* xy, int B, int N, int GH, int GW, int K,
                              int32_t* table, cudaStream_t st);
 cudaError_t launch_knn_fwd(const KnnArgs& a, cudaStream_t st);
+cudaError_t launch_knn_index(const KnnArgs& a, cudaStream_t st);
+cudaError_t launch_knn_bwd_indexed(const KnnArgs& a, cudaStream_t st);
 cudaError_t launch_knn_bwd(const KnnArgs& a, cudaStream_t st);
 
 }  // namespace acl

@@ -23,9 +23,10 @@
 // Backward without atomics.  Query side: recompute w, dw = <dOut, f> (reduced over
 // the 4 lanes of a head), ds, dq, dp partials; store w and the token ids.  An
 // inverse index -- for every token, its (query, slot) entries in ascending order --
-// is built per image by a stable counting sort (per-warp chunk histograms with
-// __match_any_sync, no floating point).  Token side: one lane group per token sums
-// w * dOut over its entries in that fixed order.
+// is built per image by a stable counting sort (integer only).  Token side: a warp
+// (or, for a token with many entries, a whole CTA) sums w * dOut over the token's
+// entries in a fixed order of streams and combining steps.
+#include <climits>
 #include <float.h>
 #include <math.h>
 
@@ -356,11 +357,6 @@ __global__ void __launch_bounds__(kGatherThreads) knn_bwd_query_kernel(const Knn
         qp = reinterpret_cast<const float2*>(a.queries)[gq];
         dmin = load_neighbours<KT>(a, gq, qp, nb);
         b = static_cast<int>(gq / a.Q);
-        if (sub == 0) {
-#pragma unroll
-            for (int j = 0; j < KT; ++j)
-                if (j < a.K) a.keys[static_cast<size_t>(gq) * a.K + j] = nb[j].t;
-        }
     } else {
 #pragma unroll
         for (int j = 0; j < KT; ++j) {
@@ -546,11 +542,6 @@ __global__ void __launch_bounds__(kGatherThreads)
         const float2 qp = live ? reinterpret_cast<const float2*>(a.queries)[gq] : make_float2(0.f, 0.f);
         GroupNbrs nb[KT];
         const float dmin = group_neighbours<KT>(a, gq, live, qp, sub, LPQ, nb);
-        if (live && sub == 0) {
-#pragma unroll
-            for (int j = 0; j < KT; ++j)
-                if (j < a.K) a.keys[static_cast<size_t>(gq) * a.K + j] = nb[j].t;
-        }
         const int b = live ? static_cast<int>(gq / a.Q) : 0;
         const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d;
         float dqx = 0.f, dqy = 0.f;
@@ -628,22 +619,34 @@ __global__ void __launch_bounds__(kGatherThreads)
 }
 
 // Stable counting sort of an image's (query, slot) entries by token id, integer only,
-// spread over `slices` CTAs per image: CTA (slice, b) owns the tokens [t_lo, t_hi).  Warp w
-// owns the contiguous entry chunk [lo_w, hi_w) of the image:
-//   compaction: one pass over its keys (16 per lane in flight) appends the entries of the
-//     slice, in entry order, to the warp's shared-memory list (ballot + popc) and counts
-//     the entries whose token lies below t_lo;
-//   counts and prefix: per-(warp, token) counts of the lists; each warp's first slot per
-//     token is (entries of smaller tokens) + (entries of this token in earlier warps);
+// spread over `slices` CTAs per image: CTA (slice, b) owns the tokens [t_lo, t_hi).
+//   compaction: warp w scans the contiguous entry chunk [lo_w, hi_w) of the image twice
+//     (16 keys per lane in flight): first it counts the slice's entries and the entries
+//     whose token lies below t_lo, then, after a prefix over the warps' counts, it writes
+//     the slice's entries in entry order into one shared-memory list (ballot + popc).
+//     Queries come in raster order and tokens are numbered spatially, so a chunk's
+//     entries cluster in one or two slices; the one list keeps the work per warp equal;
+//   counts and prefix: warp w takes the w-th equal, contiguous share of the list; per-
+//     (warp, token) counts of the shares; each warp's first slot per token is (entries of
+//     smaller tokens) + (entries of this token in earlier shares);
 //   placement: each listed entry goes to its warp's next slot for its token plus its rank
 //     among equal tokens in its group of 32 (lanes OR their bit into a per-warp hashed
 //     mask -- OR commutes, so the mask does not depend on timing).
+//   A slice with more than kCsrListCap entries counts and places straight from the keys,
+//     warp w over its own chunk.
 // The list of a token ends up in ascending entry order; entries are stored packed as
-// (query << 4) | slot.  CTA (0, 0) also resets the token kernel's work counter.
+// (query << 4) | slot.  Each CTA also lists its slice's tokens with more than
+// kHeavyEntries entries (ascending) and writes the chunk starts of the token pass.
 constexpr int kCsrSteps = 16;
 constexpr int kCsrHash = 256;
 constexpr int kCsrWarps = kCsrThreads / 32;
-constexpr int kCsrCap = 384;  // listed entries per warp held in shared memory
+constexpr int kCsrListCap = 12288;  // entries of a slice listed in shared memory
+constexpr int kHeavyEntries = 96;  // tokens with more entries are reduced by a whole CTA
+constexpr int kChunkUnits = 64;   // work units (1 per token + 1 per entry) per light chunk
+constexpr int kChunkIds = 192;    // staged ids per warp (>= kChunkUnits + kHeavyEntries)
+constexpr int kHeavyCtas = 128;   // CTAs of the token pass that take the heavy tokens
+static_assert(kChunkUnits <= kHeavyEntries + 1, "a chunk's tokens other than its last must be light");
+static_assert(kChunkIds >= kChunkUnits + kHeavyEntries, "a chunk's light entries must fit the staging");
 
 struct CsrSmem {
     size_t pre, off, hash, lanes, ckey, cent, scratch, total;
@@ -656,18 +659,34 @@ __host__ __device__ __forceinline__ CsrSmem csr_smem_layout(int NS) {
     L.hash = L.off + ((4 * static_cast<size_t>(NS + 1) + 15) & ~size_t(15));
     L.lanes = L.hash + 4 * static_cast<size_t>(kCsrHash) * kCsrWarps;
     L.ckey = L.lanes + 4 * 32 * static_cast<size_t>(kCsrWarps);
-    L.cent = L.ckey + 2 * static_cast<size_t>(kCsrCap) * kCsrWarps;
-    L.scratch = L.cent + 4 * static_cast<size_t>(kCsrCap) * kCsrWarps;
-    L.total = L.scratch + 40 * 4;
+    L.cent = L.ckey + 2 * static_cast<size_t>(kCsrListCap);
+    L.scratch = L.cent + 4 * static_cast<size_t>(kCsrListCap);
+    L.total = L.scratch + 80 * 4;
     return L;
 }
 
-__global__ void __launch_bounds__(kCsrThreads) knn_csr_kernel(const KnnArgs a, int slices) {
+// Token of every (query, slot) entry: the slot of the query's table row (-1 for an empty
+// slot).  One thread per query; keys [B][Q * K].
+__global__ void __launch_bounds__(256) knn_keys_kernel(const KnnArgs a) {
+    const long long gq = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gq >= static_cast<long long>(a.B) * a.Q) return;
+    const int b = static_cast<int>(gq / a.Q);
+    const float2 qp = reinterpret_cast<const float2*>(a.queries)[gq];
+    const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
+    const int32_t* row = a.table + ((static_cast<size_t>(b) * a.GH + cy) * a.GW + cx) * a.K;
+    int32_t* out = a.keys + gq * a.K;
+    for (int j = 0; j < a.K; ++j) {
+        const int t = __ldg(row + j);
+        out[j] = (t >= a.N) ? -1 : t;
+    }
+}
+
+__global__ void __launch_bounds__(kCsrThreads)
+    knn_csr_kernel(const KnnArgs a, int slices, int chunks) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int b = blockIdx.y, sl = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = a.N, K = a.K;
-    if (b == 0 && sl == 0 && tid == 0) *a.counter = 0;
     const int t_lo = static_cast<int>(static_cast<long long>(sl) * N / slices);
     const int t_hi = static_cast<int>(static_cast<long long>(sl + 1) * N / slices);
     const int NS = t_hi - t_lo;
@@ -677,9 +696,9 @@ __global__ void __launch_bounds__(kCsrThreads) knn_csr_kernel(const KnnArgs a, i
     int* off = reinterpret_cast<int*>(smem + L.off);
     uint32_t* hb = reinterpret_cast<uint32_t*>(smem + L.hash) + warp * kCsrHash;
     int* ks = reinterpret_cast<int*>(smem + L.lanes) + warp * 32;
-    uint16_t* ckey = reinterpret_cast<uint16_t*>(smem + L.ckey) + warp * kCsrCap;  // key - t_lo
-    int* cent = reinterpret_cast<int*>(smem + L.cent) + warp * kCsrCap;              // entry
-    int* scratch = reinterpret_cast<int*>(smem + L.scratch);
+    uint16_t* ckey = reinterpret_cast<uint16_t*>(smem + L.ckey);  // [kCsrListCap] key - t_lo
+    int* cent = reinterpret_cast<int*>(smem + L.cent);              // [kCsrListCap] entry
+    int* scratch = reinterpret_cast<int*>(smem + L.scratch);        // [40] scan, [40..72) counts
     const int E = a.Q * K;
     const int32_t* keys = a.keys + static_cast<size_t>(b) * E;
     int32_t* csr = a.csr + static_cast<size_t>(b) * E;
@@ -689,54 +708,79 @@ __global__ void __launch_bounds__(kCsrThreads) knn_csr_kernel(const KnnArgs a, i
     const int hi = static_cast<int>(static_cast<long long>(warp + 1) * E / kCsrWarps);
     uint16_t* mine = pre + warp * NS2;
     const unsigned below_lanes = (1u << lane) - 1u;
-    // compaction + count below the slice
-    int ncomp = 0, below = 0;
+    // pass 1: per warp, the entries of the slice and the entries below it
+    int cnt = 0, below = 0;
     for (int base = lo; base < hi; base += 32 * kCsrSteps) {
         int k[kCsrSteps];
 #pragma unroll
         for (int st = 0; st < kCsrSteps; ++st) {
             const int e = base + st * 32 + lane;
-            const int v = (e < hi) ? __ldg(keys + e) : -1;
-            k[st] = (v >= N) ? -1 : v;
+            k[st] = (e < hi) ? __ldg(keys + e) : -1;
         }
 #pragma unroll
         for (int st = 0; st < kCsrSteps; ++st) {
             const int key = k[st];
             below += (key >= 0 && key < t_lo);
-            const bool in = key >= t_lo && key < t_hi;
-            const unsigned m = __ballot_sync(0xffffffffu, in);
-            if (in) {
-                const int pos = ncomp + __popc(m & below_lanes);
-                if (pos < kCsrCap) {
-                    ckey[pos] = static_cast<uint16_t>(key - t_lo);
-                    cent[pos] = base + st * 32 + lane;
-                }
-            }
-            ncomp += __popc(m);
+            cnt += __popc(__ballot_sync(0xffffffffu, key >= t_lo && key < t_hi));
         }
     }
-    __syncthreads();  // pre / hash zeroed by all threads before any count
-    const bool listed = ncomp <= kCsrCap;
+    below = __reduce_add_sync(0xffffffffu, below);
+    if (lane == 0) {
+        scratch[warp] = below;
+        scratch[40 + warp] = cnt;
+    }
+    __syncthreads();  // also: pre / hash zeroed by all threads before any count
+    int wbase = 0, n = 0, base_slot = 0;
+    for (int w = 0; w < kCsrWarps; ++w) {
+        const int c = scratch[40 + w];
+        wbase += (w < warp) ? c : 0;
+        n += c;
+        base_slot += scratch[w];
+    }
+    // pass 2: the slice's entries, in entry order, into one list (warps in order); each
+    // warp then takes an equal, contiguous share of the list
+    const bool listed = n <= kCsrListCap;
     if (listed) {
-        for (int i = lane; i < ncomp; i += 32) {
+        int pos = wbase;
+        for (int base = lo; base < hi; base += 32 * kCsrSteps) {
+            int k[kCsrSteps];
+#pragma unroll
+            for (int st = 0; st < kCsrSteps; ++st) {
+                const int e = base + st * 32 + lane;
+                k[st] = (e < hi) ? __ldg(keys + e) : -1;
+            }
+#pragma unroll
+            for (int st = 0; st < kCsrSteps; ++st) {
+                const int key = k[st];
+                const bool in = key >= t_lo && key < t_hi;
+                const unsigned m = __ballot_sync(0xffffffffu, in);
+                if (in) {
+                    const int p = pos + __popc(m & below_lanes);
+                    ckey[p] = static_cast<uint16_t>(key - t_lo);
+                    cent[p] = base + st * 32 + lane;
+                }
+                pos += __popc(m);
+            }
+        }
+    }
+    __syncthreads();
+    const int l0 = static_cast<int>(static_cast<long long>(warp) * n / kCsrWarps);
+    const int l1 = static_cast<int>(static_cast<long long>(warp + 1) * n / kCsrWarps);
+    if (listed) {
+        for (int i = l0 + lane; i < l1; i += 32) {
             const int idx = warp * NS2 + ckey[i];
             atomicAdd(reinterpret_cast<uint32_t*>(pre) + (idx >> 1), 1u << (16 * (idx & 1)));
         }
     } else {
         for (int base = lo; base < hi; base += 32) {
             const int e = base + lane;
-            int key = (e < hi) ? __ldg(keys + e) : -1;
+            const int key = (e < hi) ? __ldg(keys + e) : -1;
             if (key >= t_lo && key < t_hi) {
                 const int idx = warp * NS2 + (key - t_lo);
                 atomicAdd(reinterpret_cast<uint32_t*>(pre) + (idx >> 1), 1u << (16 * (idx & 1)));
             }
         }
     }
-    below = __reduce_add_sync(0xffffffffu, below);
-    if (lane == 0) scratch[warp] = below;
-    __syncthreads();
-    int base_slot = 0;
-    for (int w = 0; w < kCsrWarps; ++w) base_slot += scratch[w];
     __syncthreads();
     for (int t = tid; t < NS; t += kCsrThreads) {
         int run = 0;
@@ -750,12 +794,51 @@ __global__ void __launch_bounds__(kCsrThreads) knn_csr_kernel(const KnnArgs a, i
     __syncthreads();
     const int tot = block_scan(off, NS, scratch);
     int32_t* coff = a.csr_off + static_cast<size_t>(b) * (N + 1);
+    // tokens with many entries go to this slice's heavy list (token order), for the
+    // token kernel's CTA-wide path
+    if (warp == 0) {
+        int nh = 0;
+        int32_t* hl = a.heavy + (static_cast<size_t>(b) * slices + sl) * a.heavy_cap;
+        for (int t0 = 0; t0 < NS; t0 += 32) {
+            const int t = t0 + lane;
+            const int cnt = (t < NS) ? ((t + 1 < NS ? off[t + 1] : tot) - off[t]) : 0;
+            const bool hv = cnt > kHeavyEntries;
+            const unsigned m = __ballot_sync(0xffffffffu, hv);
+            if (hv) hl[nh + __popc(m & below_lanes)] = t_lo + t;
+            nh += __popc(m);
+        }
+        if (lane == 0) a.heavy_count[static_cast<size_t>(b) * slices + sl] = nh;
+    }
+    __syncthreads();
     for (int t = tid; t < NS; t += kCsrThreads) {
         off[t] += base_slot;
         coff[t_lo + t] = off[t];
     }
     if (tid == 0 && sl == slices - 1) coff[N] = base_slot + tot;
     __syncthreads();
+    // chunk starts of the token pass: chunk c begins at the first token t whose unit offset
+    // start(t) + t reaches c * kChunkUnits (the boundaries inside (start(t) + t, start(t + 1)
+    // + t + 1] belong to token t + 1); chunk_off[c] = start of that token
+    int32_t* ctok = a.chunk_tok + static_cast<size_t>(b) * (chunks + 1);
+    int32_t* cofs = a.chunk_off + static_cast<size_t>(b) * (chunks + 1);
+    for (int t = tid; t < NS; t += kCsrThreads) {
+        const int e1 = t + 1 < NS ? off[t + 1] : base_slot + tot;  // first entry of token t + 1
+        const int s0 = off[t] + t_lo + t;
+        const int s1 = e1 + t_lo + t + 1;
+        for (int c = s0 / kChunkUnits + 1; c <= s1 / kChunkUnits; ++c) {
+            ctok[c] = t_lo + t + 1;
+            cofs[c] = e1;
+        }
+    }
+    if (sl == 0 && tid == 0) {
+        ctok[0] = 0;
+        cofs[0] = 0;
+    }
+    if (sl == slices - 1)
+        for (int c = (base_slot + tot + N) / kChunkUnits + 1 + tid; c <= chunks; c += kCsrThreads) {
+            ctok[c] = N;
+            cofs[c] = base_slot + tot;
+        }
     auto place = [&](bool in, int kk, int e) {
         const int h = kk & (kCsrHash - 1);
         ks[lane] = in ? kk : -1;
@@ -782,16 +865,15 @@ __global__ void __launch_bounds__(kCsrThreads) knn_csr_kernel(const KnnArgs a, i
         __syncwarp();
     };
     if (listed) {
-        for (int i0 = 0; i0 < ncomp; i0 += 32) {
+        for (int i0 = l0; i0 < l1; i0 += 32) {
             const int i = i0 + lane;
-            const bool in = i < ncomp;
+            const bool in = i < l1;
             place(in, in ? ckey[i] : -1, in ? cent[i] : 0);
         }
     } else {
         for (int base = lo; base < hi; base += 32) {
             const int e = base + lane;
-            int key = (e < hi) ? __ldg(keys + e) : -1;
-            if (key >= N) key = -1;
+            const int key = (e < hi) ? __ldg(keys + e) : -1;
             const bool in = key >= t_lo && key < t_hi;
             if (__ballot_sync(0xffffffffu, in) == 0u) continue;
             place(in, in ? key - t_lo : -1, e);
@@ -799,86 +881,250 @@ __global__ void __launch_bounds__(kCsrThreads) knn_csr_kernel(const KnnArgs a, i
     }
 }
 
-// Token side of the gather backward.  dF_t = sum of w * dOut over the token's entries, in
-// the entry order the CSR holds.  Entry counts are very uneven (tokens on the rim of an
-// empty region are the neighbours of many cells), so warps are persistent and take
-// tokens from a work counter; all 32 / LPQ lane groups of a warp work on the same token,
-// each on every S-th entry, and the group sums are combined by a fixed shuffle tree.
-// Only the scheduling uses an atomic: each token's sum is formed the same way whichever
-// warp runs it, so the result is bit-reproducible.  The first NH CTAs first reduce dp.
+// Token side of the gather backward.  dF_t = sum of w * dOut over the token's entries, with
+// no atomics and a static, balanced split of the work:
+//   light tokens (at most kHeavyEntries entries): the CSR build cuts each image's token
+//     sequence into chunks of kChunkUnits "units" (a token weighs 1 + its entry count), so
+//     every chunk holds about the same work, and lists for every chunk the first token that
+//     starts in it.  One lane group per chunk stages the entry ids of its tokens in shared
+//     memory (one round of independent loads), then walks them with the next batch's w and
+//     dOut loads in flight, summing each token's entries in ascending order;
+//   heavy tokens (listed per CSR slice): the first kHeavyCtas CTAs take them in a fixed
+//     stride; all 8 warps x (32 / LPQ) lane groups stream every S-th entry, combined by a
+//     fixed shuffle tree and a fixed-order pass over warps.
+// Every token's sum is formed the same way on every run: bit-reproducible.  The first NH
+// CTAs also reduce dp in a fixed order.
 template <int CH>
-__global__ void __launch_bounds__(kGatherThreads)
-    knn_bwd_token_kernel(const KnnArgs a, int lpq_log2, int query_blocks) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ void token_streams(const KnnArgs& a, int b, int lo, int hi, int sid,
+                                             int nstreams, int sub, int LPQ, int ch,
+                                             float (&acc)[8]) {
     const int NH = a.d >> 5;
-    if (static_cast<int>(blockIdx.x) < NH) {
-        __shared__ float red[kGatherWarps];
-        const int h = blockIdx.x;
-        float acc = 0.f;
-        for (int i = threadIdx.x; i < query_blocks; i += kGatherThreads)
-            acc += a.dp_part[static_cast<size_t>(i) * NH + h];
-        acc = warp_sum(acc);
-        if (lane == 0) red[warp] = acc;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float tot = 0.f;
-            for (int w = 0; w < kGatherWarps; ++w) tot += red[w];
-            a.dp[h] = tot;
+    const int KN = a.K * NH;
+    const int c0 = ch * LPQ * 8 + sub * 8;
+    const bool on = c0 < a.d;
+    const int hh = on ? (c0 >> 5) : 0;
+    const size_t qbase = static_cast<size_t>(b) * a.Q;
+    const float* wb = a.w + qbase * KN + hh;
+    const bf16* gb = a.dout + qbase * a.d + (on ? c0 : 0);
+    const int32_t* csr = a.csr + static_cast<size_t>(b) * a.Q * a.K;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+    // this stream's entries are lo + sid + nstreams * k; lanes of the group hold LPQ of them
+    const int n = (hi - lo - sid + nstreams - 1) / nstreams;  // entries of this stream (>= 0)
+    const unsigned gmask = (LPQ == 32) ? 0xffffffffu : (((1u << LPQ) - 1u) << (threadIdx.x & 31 & ~(LPQ - 1)));
+    for (int k0 = 0; k0 < n; k0 += LPQ) {
+        const int kk = k0 + sub;
+        const int mine = (kk < n) ? __ldg(csr + lo + sid + nstreams * kk) : 0;
+        const int cnt = min(LPQ, n - k0);
+        int u = 0;
+        for (; u + 4 <= cnt; u += 4) {
+            float wv[4];
+            uint4 gv[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int e = __shfl_sync(gmask, mine, u + x, LPQ);
+                const int q = e >> 4, j = e & 15;
+                wv[x] = __ldg(wb + q * KN + j * NH);
+                gv[x] = on ? ldg16(gb + q * a.d) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x) fma8(acc, wv[x], gv[x]);
+        }
+        for (; u < cnt; ++u) {
+            const int e = __shfl_sync(gmask, mine, u, LPQ);
+            const int q = e >> 4, j = e & 15;
+            fma8(acc, __ldg(wb + q * KN + j * NH), on ? ldg16(gb + q * a.d) : make_uint4(0u, 0u, 0u, 0u));
         }
     }
-    const int LPQ = 1 << lpq_log2, S = 32 >> lpq_log2;
-    const int sub = lane & (LPQ - 1), grp = lane >> lpq_log2;
-    const int total = a.B * a.N;
-    const int KN = a.K * NH;
-    int next = 0;
-    if (lane == 0) next = atomicAdd(a.counter, 1);
-    next = __shfl_sync(0xffffffffu, next, 0);
-    while (next < total) {
-        const int gt = next;
-        if (lane == 0) next = atomicAdd(a.counter, 1);  // fetch the following token early
-        const int b = gt / a.N, t = gt - b * a.N;
-        const int32_t* coff = a.csr_off + static_cast<size_t>(b) * (a.N + 1);
-        const int lo = coff[t], hi = coff[t + 1];
-        const int32_t* csr = a.csr + static_cast<size_t>(b) * a.Q * a.K;
-        const size_t qbase = static_cast<size_t>(b) * a.Q;
+}
+
+// One heavy token by the whole CTA (all threads call).
+__device__ void heavy_token(const KnnArgs& a, int b, int t, int l2, float (*part)[256]) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int LPQ = 1 << l2, S = 32 >> l2;
+    const int sub = lane & (LPQ - 1), grp = lane >> l2;
+    const int CH = (a.d + 8 * LPQ - 1) / (8 * LPQ);
+    const int32_t* coff = a.csr_off + static_cast<size_t>(b) * (a.N + 1);
+    const int lo = coff[t], hi = coff[t + 1];
+    for (int ch = 0; ch < CH; ++ch) {
+        float acc[8];
+        token_streams<1>(a, b, lo, hi, warp * S + grp, kGatherWarps * S, sub, LPQ, ch, acc);
+        for (int o = LPQ; o < 32; o <<= 1) {
 #pragma unroll
-        for (int ch = 0; ch < CH; ++ch) {
-            const int c0 = ch * LPQ * 8 + sub * 8;
+            for (int v = 0; v < 8; ++v) acc[v] += __shfl_xor_sync(0xffffffffu, acc[v], o);
+        }
+        if (grp == 0) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) part[warp][sub * 8 + v] = acc[v];
+        }
+        __syncthreads();
+        const int c0 = ch * LPQ * 8 + threadIdx.x * 8;
+        if (threadIdx.x < LPQ && c0 < a.d) {
+            float tot[8];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                float x = 0.f;
+                for (int w = 0; w < kGatherWarps; ++w) x += part[w][threadIdx.x * 8 + v];
+                tot[v] = x;
+            }
+            *reinterpret_cast<uint4*>(a.dfeats + (static_cast<size_t>(b) * a.N + t) * a.d + c0) =
+                pack8(tot, 1.f);
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(kGatherThreads, 4)
+    knn_bwd_token_kernel(const KnnArgs a, int lpq_log2, int query_blocks, int nlists, int chunks) {
+    constexpr int STEPS = 4;  // warp steps whose loads are in flight together
+    __shared__ float part[kGatherWarps][256];
+    __shared__ int hpre[kGatherThreads];
+    __shared__ int scan_scratch[kGatherWarps + 1];
+    __shared__ int ids_smem[kGatherWarps][kChunkIds];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NH = a.d >> 5;
+    if (static_cast<int>(blockIdx.x) < kHeavyCtas) {
+        const int h = blockIdx.x;
+        if (h < NH) {
+            float acc = 0.f;
+            for (int i = threadIdx.x; i < query_blocks; i += kGatherThreads)
+                acc += a.dp_part[static_cast<size_t>(i) * NH + h];
+            acc = warp_sum(acc);
+            if (lane == 0) part[warp][0] = acc;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                float tot = 0.f;
+                for (int w = 0; w < kGatherWarps; ++w) tot += part[w][0];
+                a.dp[h] = tot;
+            }
+            __syncthreads();
+        }
+        // heavy items h, h + kHeavyCtas, ... of the concatenated per-(image, slice) lists,
+        // scanned kGatherThreads lists at a time
+        const int slices = nlists / a.B;
+        int run = 0;
+        for (int l0 = 0; l0 < nlists; l0 += kGatherThreads) {
+            const int nl = min(kGatherThreads, nlists - l0);
+            hpre[threadIdx.x] = (static_cast<int>(threadIdx.x) < nl) ? a.heavy_count[l0 + threadIdx.x] : 0;
+            __syncthreads();
+            const int tot = block_scan(hpre, kGatherThreads, scan_scratch);  // hpre: exclusive
+            int i = run + ((h - run % kHeavyCtas) + kHeavyCtas) % kHeavyCtas;  // first i >= run, i = h mod
+            for (; i < run + tot; i += kHeavyCtas) {
+                const int r = i - run;
+                int li = 0, hl = nl - 1;  // last list whose prefix is <= r
+                while (li < hl) {
+                    const int mid = (li + hl + 1) >> 1;
+                    if (hpre[mid] <= r) li = mid; else hl = mid - 1;
+                }
+                const int lg = l0 + li;
+                const int t = a.heavy[static_cast<size_t>(lg) * a.heavy_cap + (r - hpre[li])];
+                heavy_token(a, lg / slices, t, lpq_log2, part);
+            }
+            run += tot;
+            __syncthreads();
+        }
+        return;
+    }
+    // light tokens: warp gid owns chunk gid (image b, chunk c) and takes its tokens in order.
+    // A token's entries are dealt round robin to the warp's EPS = 32 / LPQ slots (slot =
+    // lane / LPQ; the lanes of a slot hold 8 channels each), STEPS entries per slot are
+    // loaded together, and the slots are combined by a fixed xor tree at the token's end.
+    const int LPQ = 1 << lpq_log2, EPS = 32 >> lpq_log2;
+    const int slot = lane >> lpq_log2, sub = lane & (LPQ - 1);
+    const int gid = (static_cast<int>(blockIdx.x) - kHeavyCtas) * kGatherWarps + warp;
+    const int b = gid / chunks;
+    if (b >= a.B) return;  // whole warps leave together
+    const int c = gid - b * chunks;
+    int* ids = ids_smem[warp];
+    const int32_t* ctok = a.chunk_tok + static_cast<size_t>(b) * (chunks + 1);
+    const int32_t* coff = a.csr_off + static_cast<size_t>(b) * (a.N + 1);
+    const int32_t* csr = a.csr + static_cast<size_t>(b) * a.Q * a.K;
+    const int ta = ctok[c], tb = ctok[c + 1];
+    const int* cofs = a.chunk_off + static_cast<size_t>(b) * (chunks + 1);
+    const int C0 = cofs[c];
+    const int KN = a.K * NH;
+    const size_t qbase = static_cast<size_t>(b) * a.Q;
+    bf16* dfb = a.dfeats + static_cast<size_t>(b) * a.N * a.d;
+    const int passes = (a.d + 8 * LPQ - 1) / (8 * LPQ);
+    {
+        // the chunk's light entries all lie in its first kChunkUnits + kHeavyEntries entries
+        const int nst = min(cofs[c + 1] - C0, kChunkIds);
+        int v[kChunkIds / 32];
+#pragma unroll
+        for (int x = 0; x < kChunkIds / 32; ++x) {
+            const int i = x * 32 + lane;
+            v[x] = (i < nst) ? __ldg(csr + C0 + i) : 0;
+        }
+#pragma unroll
+        for (int x = 0; x < kChunkIds / 32; ++x) {
+            const int i = x * 32 + lane;
+            if (i < nst) ids[i] = v[x];
+        }
+    }
+    __syncwarp();
+    for (int t0 = ta; t0 < tb; t0 += 31) {
+        const int nt = min(31, tb - t0);
+        const int offv = (lane <= nt) ? coff[t0 + lane] - C0 : 0;  // relative to the chunk
+        // only the chunk's last token can be heavy; it is left to the heavy CTAs
+        const int last_cnt = __shfl_sync(0xffffffffu, offv, nt) - __shfl_sync(0xffffffffu, offv, nt - 1);
+        const int nl = (t0 + nt == tb && last_cnt > kHeavyEntries) ? nt - 1 : nt;
+#pragma unroll 1
+        for (int ps = 0; ps < passes; ++ps) {
+            const int c0 = ps * LPQ * 8 + sub * 8;
             const bool on = c0 < a.d;
             const int hh = on ? (c0 >> 5) : 0;
             const float* wb = a.w + qbase * KN + hh;
             const bf16* gb = a.dout + qbase * a.d + (on ? c0 : 0);
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            int i = lo + grp;
-            for (; i + 3 * S < hi; i += 4 * S) {
-                int e[4];
-                float wv[4];
-                uint4 gv[4];
+            int lo = __shfl_sync(0xffffffffu, offv, 0);
+            for (int k = 0; k < nl; ++k) {
+                const int hi = __shfl_sync(0xffffffffu, offv, k + 1);
+                float acc[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) e[u] = __ldg(csr + i + u * S);
+                for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+                for (int i0 = lo; i0 < hi; i0 += STEPS * EPS) {
+                    float w[STEPS];
+                    uint4 g[STEPS];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int q = e[u] >> 4, j = e[u] & 15;
-                    wv[u] = __ldg(wb + q * KN + j * NH);
-                    gv[u] = on ? ldg16(gb + q * a.d) : make_uint4(0u, 0u, 0u, 0u);
+                    for (int x = 0; x < STEPS; ++x) {
+                        const int i = i0 + x * EPS + slot;
+                        w[x] = 0.f;
+                        g[x] = make_uint4(0u, 0u, 0u, 0u);
+                        if (i < hi) {
+                            const int e = ids[i];
+                            const int q = e >> 4, sl = e & 15;
+                            w[x] = __ldg(wb + q * KN + sl * NH);
+                            if (on) g[x] = ldg16(gb + static_cast<size_t>(q) * a.d);
+                        }
+                    }
+#pragma unroll
+                    for (int x = 0; x < STEPS; ++x) fma8(acc, w[x], g[x]);
                 }
+                for (int o = LPQ; o < 32; o <<= 1) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) fma8(acc, wv[u], gv[u]);
+                    for (int v = 0; v < 8; ++v) acc[v] += __shfl_xor_sync(0xffffffffu, acc[v], o);
+                }
+                if (on && slot == 0)
+                    *reinterpret_cast<uint4*>(dfb + static_cast<size_t>(t0 + k) * a.d + c0) = pack8(acc, 1.f);
+                lo = hi;
             }
-            for (; i < hi; i += S) {
-                const int e = __ldg(csr + i);
-                const int q = e >> 4, j = e & 15;
-                fma8(acc, __ldg(wb + q * KN + j * NH), on ? ldg16(gb + q * a.d) : make_uint4(0u, 0u, 0u, 0u));
-            }
-            for (int o = LPQ; o < 32; o <<= 1) {
-#pragma unroll
-                for (int v = 0; v < 8; ++v) acc[v] += __shfl_xor_sync(0xffffffffu, acc[v], o);
-            }
-            if (on && grp == 0)
-                *reinterpret_cast<uint4*>(a.dfeats + static_cast<size_t>(gt) * a.d + c0) = pack8(acc, 1.f);
         }
-        next = __shfl_sync(0xffffffffu, next, 0);
+        __syncwarp();
     }
+}
+
+// light chunks of the token pass per image: (Q*K entries + N tokens) / kChunkUnits + 1
+int knn_chunks(int Q, int K, int N) {
+    return static_cast<int>((static_cast<long long>(Q) * K + N) / kChunkUnits) + 1;
+}
+
+// token slices of the CSR build per image (B * slices <= 148 CTAs, at most 8)
+int csr_slices(int B, int N) {
+    int slices = 148 / (B > 0 ? B : 1);
+    if (slices > 8) slices = 8;
+    if (slices < 1) slices = 1;
+    if (slices > (N + 31) / 32) slices = (N + 31) / 32;
+    if (slices < 1) slices = 1;
+    return slices;
 }
 
 // lanes per query: d/8 rounded up to a power of two, capped at 32
@@ -993,7 +1239,16 @@ KnnWorkspace knn_workspace_layout(int B, int Q, int N, int d, int K) {
     w.csr = off;     off += up(sizeof(int32_t) * BQ * K);
     w.csr_off = off; off += up(sizeof(int32_t) * static_cast<size_t>(B) * (N + 1));
     w.dp_part = off; off += up(sizeof(float) * static_cast<size_t>(w.query_blocks) * NH);
-    w.counter = off; off += up(sizeof(int));
+    w.chunk_tok = off;
+    off += up(sizeof(int32_t) * static_cast<size_t>(B) * (knn_chunks(Q, K, N) + 1));
+    w.chunk_off = off;
+    off += up(sizeof(int32_t) * static_cast<size_t>(B) * (knn_chunks(Q, K, N) + 1));
+    {
+        const int sl = csr_slices(B, N);
+        w.heavy_cap = (N + sl - 1) / sl;
+        w.heavy = off; off += up(sizeof(int32_t) * static_cast<size_t>(B) * sl * w.heavy_cap);
+        w.heavy_count = off; off += up(sizeof(int32_t) * static_cast<size_t>(B) * sl);
+    }
     w.total = off;
     return w;
 }
@@ -1010,7 +1265,23 @@ cudaError_t launch_knn_fwd(const KnnArgs& a, cudaStream_t st) {
     return e;
 }
 
-cudaError_t launch_knn_bwd(const KnnArgs& a, cudaStream_t st) {
+cudaError_t launch_knn_index(const KnnArgs& a, cudaStream_t st) {
+    // built even for Q == 0 (it then writes empty lists)
+    const int slices = csr_slices(a.B, a.N);
+    const size_t csmem = csr_smem_layout((a.N + slices - 1) / slices).total;
+    cudaError_t e = ensure_smem<knn_csr_kernel>(csmem);
+    if (e != cudaSuccess) return e;
+    const long long nq = static_cast<long long>(a.B) * a.Q;
+    if (nq > 0) {
+        knn_keys_kernel<<<static_cast<unsigned>((nq + 255) / 256), 256, 0, st>>>(a);
+        note_launch();
+    }
+    knn_csr_kernel<<<dim3(slices, a.B), kCsrThreads, csmem, st>>>(a, slices, knn_chunks(a.Q, a.K, a.N));
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_knn_bwd_indexed(const KnnArgs& a, cudaStream_t st) {
     const int l2 = lpq_log2_for(a.d);
     const int lanes = 1 << l2;
     const int ch = (a.d + 8 * lanes - 1) / (8 * lanes);
@@ -1028,28 +1299,21 @@ cudaError_t launch_knn_bwd(const KnnArgs& a, cudaStream_t st) {
         note_launch();
         if (e != cudaSuccess) return e;
     }
-    // the inverse index is built even for Q == 0 (it then writes empty lists)
-    int slices = 148 / (a.B > 0 ? a.B : 1);
-    if (slices > 8) slices = 8;
-    if (slices < 1) slices = 1;
-    if (slices > (a.N + 31) / 32) slices = (a.N + 31) / 32;
-    const size_t csmem = csr_smem_layout((a.N + slices - 1) / slices).total;
-    e = ensure_smem<knn_csr_kernel>(csmem);
-    if (e != cudaSuccess) return e;
-    knn_csr_kernel<<<dim3(slices, a.B), kCsrThreads, csmem, st>>>(a, slices);
-    note_launch();
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    const int slices = csr_slices(a.B, a.N);
+    const int chunks = knn_chunks(a.Q, a.K, a.N);
     const int qb = static_cast<int>(qblocks);
-    const unsigned tblocks = static_cast<unsigned>(148 * 4 > NH ? 148 * 4 : NH);
-    switch (ch) {
-        case 1: knn_bwd_token_kernel<1><<<tblocks, kGatherThreads, 0, st>>>(a, l2, qb); break;
-        case 2: knn_bwd_token_kernel<2><<<tblocks, kGatherThreads, 0, st>>>(a, l2, qb); break;
-        case 3: knn_bwd_token_kernel<3><<<tblocks, kGatherThreads, 0, st>>>(a, l2, qb); break;
-        default: knn_bwd_token_kernel<4><<<tblocks, kGatherThreads, 0, st>>>(a, l2, qb); break;
-    }
+    const long long warps = static_cast<long long>(a.B) * chunks;
+    const unsigned tblocks = static_cast<unsigned>(kHeavyCtas + (warps + kGatherWarps - 1) / kGatherWarps);
+    const int nlists = a.B * slices;
+    knn_bwd_token_kernel<<<tblocks, kGatherThreads, 0, st>>>(a, l2, qb, nlists, chunks);
     note_launch();
     return cudaGetLastError();
+}
+
+cudaError_t launch_knn_bwd(const KnnArgs& a, cudaStream_t st) {
+    const cudaError_t e = launch_knn_index(a, st);
+    if (e != cudaSuccess) return e;
+    return launch_knn_bwd_indexed(a, st);
 }
 
 }  // namespace acl

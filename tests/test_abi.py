@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("acl_cluster", "acl_neighbors", "acl_cluster_attn_fwd", "acl_cluster_attn_bwd",
               "acl_cluster_attn_workspace", "acl_knn_table", "acl_knn_gather_fwd",
-              "acl_knn_gather_bwd", "acl_knn_gather_workspace", "acl_status_string"):
+              "acl_knn_gather_bwd", "acl_knn_gather_workspace", "acl_knn_gather_index",
+              "acl_knn_gather_bwd_indexed", "acl_status_string"):
         assert n in names
 
 
@@ -116,6 +117,20 @@ def test_knn_validation():
                                                     P, P, P, P, P, wsb, None)
     assert bwd(wsb=16) == WORKSPACE
     assert bwd(Q=70000, wsb=1 << 40) == UNSUPPORTED
+    bwdi = lambda Q=10, wsb=ws: L.acl_knn_gather_bwd_indexed(P, 1, Q, P, P, 100, 128, P, 64, 64,
+                                                             8, P, P, P, P, P, P, wsb, None)
+    assert bwdi(wsb=16) == WORKSPACE
+    assert bwdi(Q=70000, wsb=1 << 40) == UNSUPPORTED
+    idx = lambda Q=10, d=128, K=8, q=P, t=P, wsb=ws, w=P: L.acl_knn_gather_index(
+        q, 1, Q, 100, d, t, 64, 64, K, w, wsb, None)
+    assert idx(t=None) == INVALID
+    assert idx(q=None) == INVALID
+    assert idx(d=100) == INVALID
+    assert idx(K=17) == UNSUPPORTED
+    assert idx(Q=70000) == UNSUPPORTED
+    assert idx(q=P + 4) == INVALID
+    assert idx(wsb=16) == WORKSPACE
+    assert idx(w=P + 16) == WORKSPACE
 
 
 def test_workspace_sizes_scale_with_inputs():

@@ -117,3 +117,22 @@ def test_bwd_deterministic_and_overwrites():
     r2 = acl.acl_knn_gather_bwd(q, f, xy, table, p, g, *outs, workspace=ws)
     for x, y in zip(r1, r2):
         assert torch.equal(x, y)
+
+
+def test_staged_backward_matches_one_call():
+    """Index built on a side stream, then the indexed backward: bit-identical results."""
+    sb = synth.step_batch(B=2)
+    kb = sb.knn
+    xy = dev(kb.coords)
+    table = acl.acl_knn_table(xy)
+    q, f, p, g = dev(kb.queries), bf16(kb.feats), dev(kb.p), bf16(kb.dout)
+    need = acl.acl_knn_gather_workspace(2, kb.Q, kb.N, kb.d, 8)
+    r1 = acl.acl_knn_gather_bwd(q, f, xy, table, p, g)
+    ws = torch.full((need,), 0xAB, dtype=torch.uint8, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    acl.acl_knn_gather_index(q, table, kb.N, kb.d, ws, stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    r2 = acl.acl_knn_gather_bwd_indexed(q, f, xy, table, p, g, ws)
+    for x, y in zip(r1, r2):
+        assert torch.equal(x, y)

@@ -8,17 +8,21 @@ image, dim 128 = 4 heads x 32, C = 8, M = 48), followed by the decoder's
 KNN gather over that stage (4096 queries per image at cell centre + U(-1,1)^2,
 K = 8, d = 128, one temperature per head):
 
-    acl_cluster -> acl_neighbors -> acl_cluster_attn_fwd -> acl_cluster_attn_bwd
-    -> acl_knn_table -> acl_knn_gather_fwd -> acl_knn_gather_bwd
+    attention chain: acl_cluster -> acl_neighbors -> acl_cluster_attn_fwd
+                     -> acl_cluster_attn_bwd
+    KNN chain:       acl_knn_table -> (acl_knn_gather_index || acl_knn_gather_fwd)
+                     -> acl_knn_gather_bwd_indexed
 
 `value` is whole-job tokens/s: images x tokens processed by all ranks per second
 of the slowest rank's device time.  Inputs sit in HBM before timing starts;
-S input sets rotate so that the sets total at least 4x the L2 size, and each set
-is replayed as one CUDA graph of the seven library calls.  CUDA events inside
-each graph time every call; the roofline figure is taken for the call with the
-largest share of the step.  `e2e` repeats the step through the same C entry
-points from pinned host buffers, with all input copies and all output read-backs
-inside its timed region.
+S input sets rotate so that the sets total at least 4x the L2 size.  Each set's
+two chains are captured as two CUDA graphs and replayed on two streams (the
+attention chain, the longer one, at the higher priority; the inverse index on a
+third stream inside the KNN graph).  CUDA events inside the graphs time every
+call; the roofline figure is taken for the call with the largest share of the
+step.  `e2e` runs the same calls through the C entry points with every step's
+inputs copied in from pinned host buffers and all of its outputs read back, the
+copies pipelined against the neighbouring steps' compute.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl acl|reference]
 
@@ -80,7 +84,7 @@ def parse_args(argv=None):
     ap.add_argument("--batch", type=int, default=8, help="images per rank (default 8)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--serial", action="store_true",
                     help="run all seven calls on one stream (default: the attention and KNN "
                          "chains run as two concurrent branches of the step graph)")
@@ -257,40 +261,46 @@ class StepSet:
         else:
             raise KeyError(name)
 
-    def step(self, stream, events=None, streams=None):
-        """The eight calls.  With streams = (s2, s3) the KNN chain (table -> gather fwd ->
-        indexed bwd) runs on s2 and the inverse index (after the table) on s3, concurrently
-        with the attention chain (cluster -> neighbours -> attn fwd -> bwd) on stream;
-        events[2j], events[2j+1] bracket call j on its stream."""
+    ATTN = ("cluster", "neighbors", "attn_fwd", "attn_bwd")
+    KNN = ("knn_table", "knn_index", "knn_fwd", "knn_bwd")
+
+    def chain(self, names, stream, events=None, s3=None):
+        """The calls of one chain in order on `stream`; with s3 the inverse index runs on
+        s3 after the table and the indexed backward waits for it."""
         torch = self.torch
-        if streams is None:
-            for j, name in enumerate(OPS):
-                if events is not None:
-                    events[2 * j].record(stream)
-                self.op(name, stream)
-                if events is not None:
-                    events[2 * j + 1].record(stream)
-            return
-        s2, s3 = streams
-        home = {"knn_table": s2, "knn_fwd": s2, "knn_bwd": s2, "knn_index": s3}
-        fork, tab, idx, join = (torch.cuda.Event() for _ in range(4))
-        fork.record(stream)
-        s2.wait_event(fork)
-        for j, name in enumerate(OPS):
-            st = home.get(name, stream)
-            if name == "knn_index":
+        tab, idx = torch.cuda.Event(), torch.cuda.Event()
+        for name in names:
+            j = OPS.index(name)
+            st = s3 if (name == "knn_index" and s3 is not None) else stream
+            if name == "knn_index" and s3 is not None:
                 s3.wait_event(tab)
-            if name == "knn_bwd":
-                s2.wait_event(idx)
+            if name == "knn_bwd" and s3 is not None:
+                stream.wait_event(idx)
             if events is not None:
                 events[2 * j].record(st)
             self.op(name, st)
             if events is not None:
                 events[2 * j + 1].record(st)
             if name == "knn_table":
-                tab.record(s2)
+                tab.record(stream)
             if name == "knn_index":
-                idx.record(s3)
+                idx.record(st)
+
+    def step(self, stream, events=None, streams=None):
+        """The eight calls.  With streams = (s2, s3) the KNN chain (table -> gather fwd ->
+        indexed bwd; the inverse index on s3 after the table) runs on s2 concurrently with
+        the attention chain (cluster -> neighbours -> attn fwd -> bwd) on stream;
+        events[2j], events[2j+1] bracket call j on its stream."""
+        if streams is None:
+            self.chain(OPS, stream, events)
+            return
+        torch = self.torch
+        s2, s3 = streams
+        fork, join = torch.cuda.Event(), torch.cuda.Event()
+        fork.record(stream)
+        s2.wait_event(fork)
+        self.chain(StepSet.ATTN, stream, events)
+        self.chain(StepSet.KNN, s2, events, s3=s3)
         join.record(s2)
         stream.wait_event(join)
 
@@ -321,8 +331,12 @@ def run_gpu(args, rank: int, world: int):
     set_bytes = base.bytes()
     n_sets = max(2, math.ceil(4 * l2 / set_bytes))
     sets = [base] + [StepSet(sb, device, acl, torch) for _ in range(n_sets - 1)]
-    stream = torch.cuda.Stream(device)
-    streams = None if args.serial else (torch.cuda.Stream(device), torch.cuda.Stream(device))
+    # the attention chain is the longer one: its stream gets the higher priority so its
+    # CTAs are scheduled first and the KNN chain fills the remaining SMs
+    # (a lower number is a higher priority; out-of-range values map to the nearest valid one)
+    stream = torch.cuda.Stream(device, priority=-100)
+    streams = None if args.serial else (torch.cuda.Stream(device, priority=0),
+                                        torch.cuda.Stream(device, priority=0))
 
     # eager warm-up of every call (kernel attributes, lazy module loading), then capture
     with torch.cuda.stream(stream):
@@ -334,16 +348,60 @@ def run_gpu(args, rank: int, world: int):
     launches0 = acl.acl_launch_count()
     for s in sets:
         evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            s.step(stream, evs, streams)
-        graphs.append(g)
+        if streams is None:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                s.step(stream, evs)
+            graphs.append((g,))
+        else:
+            # one graph per chain, replayed on its own stream (graph nodes run at the
+            # priority of the stream the graph is launched into)
+            ga, gk = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ga, stream=stream):
+                s.chain(StepSet.ATTN, stream, evs)
+            with torch.cuda.graph(gk, stream=streams[0]):
+                s.chain(StepSet.KNN, streams[0], evs, s3=streams[1])
+            graphs.append((ga, gk))
         events.append(evs)
     launches_per_step = (acl.acl_launch_count() - launches0) // len(sets)
+    # single-stream graphs of the same sets: the per-call breakdown and the roofline come
+    # from these, where no call shares the GPU with another
+    serial_graphs, serial_events = [], []
+    if streams is None:
+        serial_graphs, serial_events = [gs[0] for gs in graphs], events
+    else:
+        for s in sets:
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                s.step(stream, evs)
+            serial_graphs.append(g)
+            serial_events.append(evs)
     torch.cuda.synchronize()
 
+    def replay(i):
+        gs = graphs[i % n_sets]
+        if len(gs) == 1:
+            with torch.cuda.stream(stream):
+                gs[0].replay()
+            return
+        with torch.cuda.stream(stream):
+            gs[0].replay()
+        with torch.cuda.stream(streams[0]):
+            gs[1].replay()
+
+    def fork():
+        if streams is not None:
+            streams[0].wait_stream(stream)
+
+    def join():
+        if streams is not None:
+            stream.wait_stream(streams[0])
+
+    fork()
     for w in range(args.warmup):
-        graphs[w % n_sets].replay()
+        replay(w)
+    join()
     torch.cuda.synchronize()
 
     props = torch.cuda.get_device_properties(device)
@@ -353,30 +411,41 @@ def run_gpu(args, rank: int, world: int):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        t0.record(stream)
-        for it in range(args.steps):
-            graphs[it % n_sets].replay()
-        t1.record(stream)
+    t0.record(stream)
+    fork()
+    for it in range(args.steps):
+        replay(it)
+    join()
+    t1.record(stream)
     torch.cuda.synchronize()
     barrier()
     step_ms_local = t0.elapsed_time(t1) / max(args.steps, 1)
-    # per-call durations from the in-graph events (the last replay of every set)
-    per_op = np.zeros(len(OPS))
-    used = min(n_sets, args.steps)
-    for s_i in range(used):
-        ev = events[s_i]
-        per_op += np.array([ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(len(OPS))])
-    per_op /= max(used, 1)
+    def per_call(evsets, used):
+        acc = np.zeros(len(OPS))
+        for s_i in range(used):
+            ev = evsets[s_i]
+            acc += np.array([ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(len(OPS))])
+        return acc / max(used, 1)
+
+    # per-call durations inside the timed region (the last replay of every set); with
+    # concurrent chains each includes the time it shared the GPU with the other chain
+    per_op_concurrent = per_call(events, min(n_sets, args.steps))
+    # per-call durations with one call at a time: 2 rounds over the sets, after warm-up
+    with torch.cuda.stream(stream):
+        for it in range(3 * n_sets):
+            serial_graphs[it % n_sets].replay()
+    torch.cuda.synchronize()
+    per_op = per_call(serial_events, n_sets)
     # keep the same load on the GPU until the clock sampler has several samples
     t_wall = time.time()
-    with torch.cuda.stream(stream):
-        it = 0
-        while time.time() - t_wall < 0.8:
-            graphs[it % n_sets].replay()
+    it = 0
+    while time.time() - t_wall < 0.8:
+        fork()
+        for _ in range(64):
+            replay(it)
             it += 1
-            if it % 64 == 0:
-                stream.synchronize()
+        join()
+        stream.synchronize()
     torch.cuda.synchronize()
     clk = clocks.stop()
 
@@ -402,7 +471,8 @@ def run_gpu(args, rank: int, world: int):
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, base, stream, streams, torch, acl, tokens_per_step=world * B * N)
+        e2e = run_e2e(args, base, stream, streams, torch, acl, tokens_per_step=world * B * N,
+                      sb=sb, device=device)
         e2e_ms = max_over_ranks(e2e.pop("_ms"), world, device)
         e2e["value"] = round(world * B * N / (e2e_ms * 1e-3), 1)
         e2e["ms_per_step"] = round(e2e_ms, 4)
@@ -422,13 +492,17 @@ def run_gpu(args, rank: int, world: int):
                    "l2": f"rotating {n_sets} input sets, {n_sets * set_bytes / 1e6:.0f} MB total "
                          f">= 4 x L2 ({l2 / 1e6:.0f} MB)",
                    "timing": "CUDA graph per set, CUDA events on the launching stream",
-                   "streams": 1 if args.serial else 3,
+                   "streams": "1" if args.serial else "3 (attention chain at high priority)",
                    "parallelism": f"replicas x{world} (images sharded, no collective)"},
         "parts": {
             "knn_queries_per_s": round(world * B * Q / (step_ms * 1e-3), 1),
             "cluster_attn_fwd_bwd_tokens_per_s": round(world * B * N / (attn_ms * 1e-3), 1),
             "knn_gather_fwd_bwd_queries_per_s": round(world * B * Q / (knn_ms * 1e-3), 1),
             "per_call": breakdown,
+            "per_call_note": "one call at a time (single-stream graphs of the same sets, "
+                             "after the timed region); the step overlaps the two chains",
+            "per_call_concurrent_us": {n: round(per_op_concurrent[j] * 1e3, 2)
+                                       for j, n in enumerate(OPS)},
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -440,45 +514,84 @@ def run_gpu(args, rank: int, world: int):
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": clk,
     }
-    for g in graphs:
-        g.reset()
+    for gs in graphs:
+        for g in gs:
+            g.reset()
+    if streams is not None:
+        for g in serial_graphs:
+            g.reset()
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, s: StepSet, stream, streams, torch, acl, tokens_per_step: int) -> dict:
-    """The step through the public entry points from pinned host memory, copies inside."""
+def run_e2e(args, s: StepSet, stream, streams, torch, acl, tokens_per_step: int, sb=None,
+            device=None) -> dict:
+    """The step through the public entry points from pinned host memory, copies inside.
+
+    Every step copies its inputs host -> device and its results device -> host.  Two
+    device sets and two copy streams pipeline the steps: the inputs of step k + 1 travel
+    in and the results of step k - 1 travel out while step k computes (PCIe is full
+    duplex), with events ordering each set's copy-in, compute and copy-out."""
+    sets = [s, StepSet(sb, device, acl, torch)] if sb is not None else [s, s]
     hin = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in s.inputs.items()}
     for k, v in s.inputs.items():
         hin[k].copy_(v)
-    hout = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in s.outputs.items()}
+    hout = [{k: torch.empty_like(v, device="cpu").pin_memory() for k, v in s.outputs.items()}
+            for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in hin.values())
-    d2h = sum(t.numel() * t.element_size() for t in hout.values())
+    d2h = sum(t.numel() * t.element_size() for t in hout[0].values())
+    cp_in, cp_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    recorded = [False, False]
 
-    def one():
-        for k, v in hin.items():
-            s.inputs[k].copy_(v, non_blocking=True)
-        s.step(stream, None, streams)
-        for k, v in s.outputs.items():
-            hout[k].copy_(v, non_blocking=True)
+    def one(k):
+        i = k % 2
+        S = sets[i]
+        if recorded[i]:
+            cp_in.wait_event(ev_done[i])    # step k - 2 has finished reading set i's inputs
+        with torch.cuda.stream(cp_in):
+            for name, v in hin.items():
+                S.inputs[name].copy_(v, non_blocking=True)
+        ev_in[i].record(cp_in)
+        stream.wait_event(ev_in[i])
+        if recorded[i]:
+            stream.wait_event(ev_out[i])    # step k - 2's results have left set i
+        with torch.cuda.stream(stream):
+            S.step(stream, None, streams)
+        ev_done[i].record(stream)
+        cp_out.wait_event(ev_done[i])
+        with torch.cuda.stream(cp_out):
+            for name, v in S.outputs.items():
+                hout[i][name].copy_(v, non_blocking=True)
+        ev_out[i].record(cp_out)
+        recorded[i] = True
 
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            one()
+    def drain():
+        stream.wait_stream(cp_out)
+        stream.wait_stream(cp_in)
+
+    for k in range(4):
+        one(k)
+    drain()
     torch.cuda.synchronize()
     n = max(1, args.e2e_steps)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        a.record(stream)
-        for _ in range(n):
-            one()
-        b.record(stream)
+    a.record(stream)
+    cp_in.wait_stream(stream)
+    cp_out.wait_stream(stream)
+    for k in range(n):
+        one(k)
+    drain()
+    b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / n
     return {"value": tokens_per_step / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "steps": n, "_ms": ms}
+            "d2h_bytes_per_step": int(d2h), "steps": n, "_ms": ms,
+            "pipelining": "2 device sets, copy-in / compute / copy-out streams"}
 
 
 # --------------------------------------------------------------------------- CPU oracle

@@ -102,14 +102,30 @@ __device__ void block_minmax(const float* xs, const float* ys, int N, int* scrat
         f[4 * warp + 3] = d;
     }
     __syncthreads();
-    xmin = ymin = INFINITY;
-    xmax = ymax = -INFINITY;
-    for (int w = 0; w < nw; ++w) {
-        xmin = fminf(xmin, f[4 * w]);
-        xmax = fmaxf(xmax, f[4 * w + 1]);
-        ymin = fminf(ymin, f[4 * w + 2]);
-        ymax = fmaxf(ymax, f[4 * w + 3]);
+    if (warp == 0) {
+        a = lane < nw ? f[4 * lane] : INFINITY;
+        b = lane < nw ? f[4 * lane + 1] : -INFINITY;
+        c = lane < nw ? f[4 * lane + 2] : INFINITY;
+        d = lane < nw ? f[4 * lane + 3] : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            a = fminf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
+            c = fminf(c, __shfl_xor_sync(0xffffffffu, c, o));
+            d = fmaxf(d, __shfl_xor_sync(0xffffffffu, d, o));
+        }
+        if (lane == 0) {
+            f[128] = a;
+            f[129] = b;
+            f[130] = c;
+            f[131] = d;
+        }
     }
+    __syncthreads();
+    xmin = f[128];
+    xmax = f[129];
+    ymin = f[130];
+    ymax = f[131];
     __syncthreads();
 }
 
@@ -432,18 +448,20 @@ __global__ void __launch_bounds__(kClusterThreads)
         __syncthreads();
     }
 
-    // leaves: ids ascending, padding (-1) after the valid ones
+    // leaves: ids ascending, padding (-1) after the valid ones; one thread per slot ranks
+    // its id among its cluster's ids
     int32_t* out = clusters + static_cast<size_t>(b) * G * C;
-    for (int c = tid; c < G; c += kClusterThreads) {
-        const int lo = c * C;
+    for (int q = tid; q < G * C; q += kClusterThreads) {
+        const int lo = (q / C) * C;
         const int n = min(C, N - lo);
-        for (int s2 = 0; s2 < n; ++s2) {
-            const int id = LX[lo + s2];
-            int rank = 0;
-            for (int u = 0; u < n; ++u) rank += (LX[lo + u] < id);
-            out[lo + rank] = id;
+        if (q - lo >= n) {
+            out[q] = -1;
+            continue;
         }
-        for (int s2 = n; s2 < C; ++s2) out[lo + s2] = -1;
+        const int id = LX[q];
+        int rank = 0;
+        for (int u = 0; u < n; ++u) rank += (LX[lo + u] < id);
+        out[lo + rank] = id;
     }
 }
 

@@ -36,7 +36,8 @@ namespace acl {
 
 namespace {
 
-constexpr int kTableThreads = 256;
+constexpr int kTableThreads = 512;
+constexpr int kTableSub = 4;  // lanes per cell in the table search
 constexpr int kGatherWarps = 8;
 constexpr int kGatherThreads = 32 * kGatherWarps;
 constexpr int kCsrThreads = 1024;
@@ -102,39 +103,88 @@ __device__ __forceinline__ int bin_coord(float v, float inv_s, int nb) {
     return i > nb - 1 ? nb - 1 : i;
 }
 
+// (d, t) < (d', t') in the table's order: distance, then token id
+__device__ __forceinline__ bool dt_less(double d, int t, double d2, int t2) {
+    return d < d2 || (d == d2 && t < t2);
+}
+
+// Insert (d, t) into the ascending top-K list: every slot compares with the new pair at
+// once (the list is sorted, so the slots below it form a prefix), then shifts or takes it.
 template <int KMAX>
-__device__ __forceinline__ void topk_insert(double (&bd)[KMAX], int (&bi)[KMAX], double d, int t) {
-    if (d < bd[KMAX - 1] || (d == bd[KMAX - 1] && t < bi[KMAX - 1])) {
-        bool placed = false;
+__device__ __forceinline__ void topk_insert_par(double (&bd)[KMAX], int (&bi)[KMAX], double d, int t) {
+    if (!dt_less(d, t, bd[KMAX - 1], bi[KMAX - 1])) return;
+    bool lt[KMAX];
 #pragma unroll
-        for (int r = KMAX - 1; r >= 0; --r) {
-            if (!placed) {
-                if (r > 0 && (bd[r - 1] > d || (bd[r - 1] == d && bi[r - 1] > t))) {
-                    bd[r] = bd[r - 1];
-                    bi[r] = bi[r - 1];
-                } else {
-                    bd[r] = d;
-                    bi[r] = t;
-                    placed = true;
+    for (int r = 0; r < KMAX; ++r) lt[r] = dt_less(bd[r], bi[r], d, t);
+#pragma unroll
+    for (int r = KMAX - 1; r >= 1; --r) {
+        if (!lt[r]) {
+            bd[r] = lt[r - 1] ? d : bd[r - 1];
+            bi[r] = lt[r - 1] ? t : bi[r - 1];
+        }
+    }
+    if (!lt[0]) {
+        bd[0] = d;
+        bi[0] = t;
+    }
+}
+
+// In place: the K smallest of this lane's ascending list and the list of lane ^ o, as a
+// bitonic sequence (element r is the smaller of A[r] and B[K-1-r]).
+template <int KMAX>
+__device__ __forceinline__ void merge_lows(double (&bd)[KMAX], int (&bi)[KMAX], int o) {
+    double od[KMAX];
+    int oi[KMAX];
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r) {
+        od[r] = __shfl_xor_sync(0xffffffffu, bd[r], o);
+        oi[r] = __shfl_xor_sync(0xffffffffu, bi[r], o);
+    }
+#pragma unroll
+    for (int r = 0; r < KMAX; ++r) {
+        if (!dt_less(bd[r], bi[r], od[KMAX - 1 - r], oi[KMAX - 1 - r])) {
+            bd[r] = od[KMAX - 1 - r];
+            bi[r] = oi[KMAX - 1 - r];
+        }
+    }
+}
+
+// Sort a bitonic sequence ascending (half-cleaners of decreasing span).
+template <int KMAX>
+__device__ __forceinline__ void bitonic_finish(double (&cd)[KMAX], int (&ci)[KMAX]) {
+#pragma unroll
+    for (int span = KMAX / 2; span >= 1; span >>= 1) {
+#pragma unroll
+        for (int r = 0; r < KMAX; ++r) {
+            if ((r & span) == 0) {
+                const int u = r + span;
+                if (dt_less(cd[u], ci[u], cd[r], ci[r])) {
+                    const double td = cd[r]; cd[r] = cd[u]; cd[u] = td;
+                    const int ti = ci[r]; ci[r] = ci[u]; ci[u] = ti;
                 }
             }
         }
     }
 }
 
-// One warp per 8 x 4 tile of cells, one lane per cell.  Bin rows are contiguous runs of
-// the bin-sorted tokens, and all lanes of the warp read the same candidate (a
-// shared-memory broadcast).  A candidate whose fp32 squared distance exceeds the current K-th best by
-// more than the fp32 rounding bound cannot enter the fp64 (distance, id) top-K and is
-// skipped; the rest go through the exact fp64 comparison.  Bins are visited in rings
-// around the tile's own bins, nearest first, so the lists fill with near tokens and the
-// threshold tightens early.  After each ring every lane checks that its K-th distance is
-// below its distance to the scanned rectangle's edge (tokens outside lie beyond it, and
-// rounding is monotone); the warp stops once all lanes are proven.
+// One warp per 4 x 2 tile of cells, kTableSub lanes per cell (lane = cell * kTableSub +
+// sub).  Bin rows are contiguous runs of the bin-sorted tokens; sub-lane p of every cell
+// takes the run's candidates i = p (mod kTableSub), all cells reading the same candidate
+// (a shared-memory broadcast), and keeps its own ascending (fp64 distance, id) top-K.  A
+// candidate whose fp32 squared distance exceeds a bound of the cell's K-th best by more
+// than the fp32 rounding bound cannot enter the top-K and is skipped.  Bins are visited in
+// rings around the tile's own bins, nearest first.  After each ring the cell's K-th best
+// is bounded above by the largest of its sub-lanes' ceil(K / kTableSub)-th entries (those
+// prefixes hold at least K distinct tokens); every cell checks that the bound is below its
+// distance to the scanned rectangle's edge (tokens outside lie beyond it, and rounding is
+// monotone), and the warp stops once all cells are proven.  The sub-lanes' lists are then
+// merged (bitonic, over shuffles); each token was seen by exactly one sub-lane, so the
+// merged list is the top-K of all candidates.
 template <int KMAX>
-__global__ void __launch_bounds__(kTableThreads)
+__global__ void __launch_bounds__(kTableThreads, KMAX <= 8 ? 2 : 1)
     knn_table_kernel(const float* __restrict__ xy, int N, int GH, int GW, int K, BinGrid bg,
                      int32_t* __restrict__ table) {
+    static_assert(kTableSub == 4, "the merge below takes two levels");
     extern __shared__ __align__(16) uint8_t smem[];
     const int b = blockIdx.y, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -162,11 +212,12 @@ __global__ void __launch_bounds__(kTableThreads)
     }
     __syncthreads();  // cnt[bin] = end of bin; start = cnt[bin - 1]
 
-    const int tiles_x = (GW + 7) >> 3, tiles_y = (GH + 3) >> 2;
+    const int tiles_x = (GW + 3) >> 2, tiles_y = (GH + 1) >> 1;
     const int tile = blockIdx.x * (kTableThreads / 32) + warp;
     if (tile >= tiles_x * tiles_y) return;
-    const int tx0 = (tile % tiles_x) * 8, ty0 = (tile / tiles_x) * 4;
-    const int c = tx0 + (lane & 7), r = ty0 + (lane >> 3);
+    const int tx0 = (tile % tiles_x) * 4, ty0 = (tile / tiles_x) * 2;
+    const int cell = lane / kTableSub, sub = lane % kTableSub;
+    const int c = tx0 + (cell & 3), r = ty0 + (cell >> 2);
     const int cc = min(c, GW - 1), rr = min(r, GH - 1);  // lanes past the edge shadow a real cell
     const double px = static_cast<double>(cc) + 0.5, py = static_cast<double>(rr) + 0.5;
     const float pxf = static_cast<float>(cc) + 0.5f, pyf = static_cast<float>(rr) + 0.5f;
@@ -179,29 +230,32 @@ __global__ void __launch_bounds__(kTableThreads)
         bi[k] = 0x7fffffff;
     }
     float thr = INFINITY;
-    // scan one contiguous run of bins [b0, b1] (one bin row): every lane reads the same token
+    auto tighten = [&](double kth) {
+        if (kth < DBL_MAX) thr = fminf(thr, static_cast<float>(kth) * (1.0f + 1.0f / 1048576.0f));
+    };
+    // scan one contiguous run of bins [b0, b1] (one bin row), this sub-lane's share
     auto scan_run = [&](int b0, int b1) {
         const int s0 = b0 > 0 ? cnt[b0 - 1] : 0, s1 = cnt[b1];
-        for (int i = s0; i < s1; ++i) {
+        for (int i = s0 + sub; i < s1; i += kTableSub) {
             const float2 p = txy[i];
             const float dxf = p.x - pxf, dyf = p.y - pyf;
             const float d2f = fmaf(dxf, dxf, dyf * dyf);
             if (d2f <= thr) {
                 const double dx = __dsub_rn(static_cast<double>(p.x), px);
                 const double dy = __dsub_rn(static_cast<double>(p.y), py);
-                topk_insert<KMAX>(bd, bi, __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)), tidv[i]);
-                if (bd[KMAX - 1] < DBL_MAX)
-                    thr = static_cast<float>(bd[KMAX - 1]) * (1.0f + 1.0f / 1048576.0f);
+                topk_insert_par<KMAX>(bd, bi, __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)), tidv[i]);
+                tighten(bd[KMAX - 1]);
             }
         }
     };
     // the tile's footprint in bins; rings of bins around it are scanned nearest first
     const int tbx0 = bin_coord(static_cast<float>(tx0) + 0.5f, bg.inv_s, bg.nbx);
-    const int tbx1 = bin_coord(static_cast<float>(min(tx0 + 8, GW)) - 0.5f, bg.inv_s, bg.nbx);
+    const int tbx1 = bin_coord(static_cast<float>(min(tx0 + 4, GW)) - 0.5f, bg.inv_s, bg.nbx);
     const int tby0 = bin_coord(static_cast<float>(ty0) + 0.5f, bg.inv_s, bg.nby);
-    const int tby1 = bin_coord(static_cast<float>(min(ty0 + 4, GH)) - 0.5f, bg.inv_s, bg.nby);
+    const int tby1 = bin_coord(static_cast<float>(min(ty0 + 2, GH)) - 0.5f, bg.inv_s, bg.nby);
     const double s = static_cast<double>(bg.s);
     const int maxring = max(bg.nbx, bg.nby);
+    const int kq = (K + kTableSub - 1) / kTableSub - 1;
     for (int rho = 0; rho <= maxring; ++rho) {
         const int bx_lo = tbx0 - rho, bx_hi = tbx1 + rho, by_lo = tby0 - rho, by_hi = tby1 + rho;
         const int cx_lo = max(bx_lo, 0), cx_hi = min(bx_hi, bg.nbx - 1);
@@ -216,6 +270,15 @@ __global__ void __launch_bounds__(kTableThreads)
                 if (bx_hi < bg.nbx) scan_run(by * bg.nbx + bx_hi, by * bg.nbx + bx_hi);
             }
         }
+        // an upper bound of the cell's K-th best: the sub-lanes' first ceil(K / kTableSub)
+        // entries are at least K distinct tokens, so the K-th best is at most their maximum
+        double kth = DBL_MAX;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k)
+            if (k == kq) kth = bd[k];
+        kth = fmax(kth, __shfl_xor_sync(0xffffffffu, kth, 1));
+        kth = fmax(kth, __shfl_xor_sync(0xffffffffu, kth, 2));
+        tighten(kth);
         // distance from the cell centre to the edge of the scanned rectangle; a side on the
         // grid border is unbounded (tokens outside the grid fall into border bins)
         double m = DBL_MAX;
@@ -223,10 +286,15 @@ __global__ void __launch_bounds__(kTableThreads)
         if (bx_hi < bg.nbx - 1) m = fmin(m, (bx_hi + 1) * s - px);
         if (by_lo > 0) m = fmin(m, py - by_lo * s);
         if (by_hi < bg.nby - 1) m = fmin(m, (by_hi + 1) * s - py);
-        const bool proven = (m == DBL_MAX) || (bd[KMAX - 1] < m * m);
+        const bool proven = (m == DBL_MAX) || (kth < m * m);
         if (__all_sync(0xffffffffu, proven)) break;
     }
-    if (c >= GW || r >= GH) return;
+    // final list: merge the sub-lanes' lists (two levels), sub-lane 0 writes it
+    merge_lows<KMAX>(bd, bi, 1);
+    bitonic_finish<KMAX>(bd, bi);
+    merge_lows<KMAX>(bd, bi, 2);
+    bitonic_finish<KMAX>(bd, bi);
+    if (sub != 0 || c >= GW || r >= GH) return;
     int32_t* out = table + static_cast<size_t>(b) * GH * GW * K + (static_cast<size_t>(r) * GW + c) * K;
 #pragma unroll
     for (int k = 0; k < KMAX; ++k)
@@ -1210,7 +1278,7 @@ cudaError_t launch_knn_table(const float* xy, int B, int N, int GH, int GW, int 
                              cudaStream_t st) {
     const BinGrid bg = choose_bins(N, GH, GW);
     const size_t smem = knn_table_smem_bytes(N, bg.nbx * bg.nby);
-    const int tiles = ((GW + 7) / 8) * ((GH + 3) / 4);
+    const int tiles = ((GW + 3) / 4) * ((GH + 1) / 2);
     dim3 grid((tiles + kTableThreads / 32 - 1) / (kTableThreads / 32), B);
     cudaError_t e;
 #define ACL_TABLE_CASE(KM)                                                                        \

@@ -54,6 +54,14 @@ def test_cluster_sizes(C, M):
     run_both(xy, C, M)
 
 
+@pytest.mark.parametrize("N,C", [(6000, 1), (8065, 63), (8192, 4), (3000, 5)])
+def test_deep_trees_and_largest_warp_nodes(N, C):
+    # the levels below the fifth run one warp per node; (8065, 63) gives the largest such
+    # node (315 tokens), C = 1 the deepest tree
+    xy = synth.uniform(1000 + N + C, 2 * N, -5.0, 70.0).reshape(1, N, 2).astype(np.float32)
+    run_both(xy, C, 2 * C if C <= 8 else C)
+
+
 def test_ties_negative_zero_and_duplicates():
     # exact duplicates, -0.0 vs +0.0, integer lattice: every tie-break path
     rng = np.random.default_rng(0)

@@ -108,7 +108,7 @@ constexpr int kUThreads = 32 * kUWarps;
 constexpr int kURow = 64 * kUH;  // bytes per union row
 
 struct UnionLayout {
-    int ks, vs, qs, stage, blk, utok, uxy, qtok, qxy, krow, nu, total;
+    int ks, vs, qs, stage, utok, uxy, qtok, qxy, krow, nbs, total;
 };
 __host__ __device__ __forceinline__ UnionLayout union_layout(int R, int MT) {
     UnionLayout L;
@@ -118,19 +118,101 @@ __host__ __device__ __forceinline__ UnionLayout union_layout(int R, int MT) {
     L.vs = o; o += rows * kURow;
     L.qs = o; o += kUC * 8 * kURow;
     L.stage = o; o += kUWarps * 512;
-    L.blk = o; o += 4 * kUC * R * 2;       // first token, union index
     L.utok = o; o += 4 * (rows - 8);
     L.uxy = o; o += 8 * (rows - 8);
     L.qtok = o; o += 4 * kUC * 8;
     L.qxy = o; o += 8 * kUC * 8;
     L.krow = o; o += 4 * kUC * MT;
-    L.nu = o; o += 16;
+    L.nbs = o; o += 4 * kUC * R * 8;        // the group's neighbour rows
     L.total = (o + 15) & ~15;
     return L;
 }
 
 __device__ __forceinline__ uint32_t urow_off(int row, int ch) {
     return static_cast<uint32_t>(row * kURow + ((ch ^ (row & 7)) << 4));
+}
+
+// Union setup shared by the forward-shaped kernels: the neighbour rows of the CTA's kUC
+// clusters (one global round, into shared memory), their blocks de-duplicated by first
+// token (every warp computes the same map in registers, so no barrier is needed before
+// it is used), union row tokens, the per-cluster key-slot -> union row map and the
+// group's query tokens.  Coordinates follow with the tiles (union_coords_async).  All
+// threads of the CTA call it; returns the number of distinct blocks.
+__device__ __forceinline__ int union_setup(const AttnArgs& a, int b, int g0, int MT, const UnionLayout& L,
+                                           uint8_t* smem) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int G = a.G, N = a.N, M = a.M, R = a.R;
+    const int nblk = kUC * R;
+    int* utok = reinterpret_cast<int*>(smem + L.utok);
+    int* qtok = reinterpret_cast<int*>(smem + L.qtok);
+    int* krow = reinterpret_cast<int*>(smem + L.krow);
+    int* nbs = reinterpret_cast<int*>(smem + L.nbs);
+    for (int i = tid; i < nblk * 8; i += blockDim.x) {
+        const int cw = i / M, m = i - cw * M;
+        const int g = g0 + cw;
+        int t = -1;
+        if (g < G) {
+            t = a.nbr[(static_cast<size_t>(b) * G + g) * M + m];
+            if (t < 0 || t >= N) t = -1;
+        }
+        nbs[i] = t;
+    }
+    for (int i = tid; i < kUC * 8; i += blockDim.x) {
+        const int g = g0 + (i >> 3);
+        int id = -1;
+        if (g < G) {
+            id = a.clusters[(static_cast<size_t>(b) * G + g) * 8 + (i & 7)];
+            if (id < 0 || id >= N) id = -1;
+        }
+        qtok[i] = id;
+    }
+    __syncthreads();
+    // lane j < nblk: block j's union index, or the index of its first occurrence
+    const int f = lane < nblk ? nbs[lane * 8] : -1;
+    int dup = -1;
+    for (int j = 0; j < nblk; ++j) {
+        const int fj = __shfl_sync(0xffffffffu, f, j);
+        if (j < lane && dup < 0 && f >= 0 && fj == f) dup = j;
+    }
+    const bool isnew = f >= 0 && dup < 0;
+    const unsigned newmask = __ballot_sync(0xffffffffu, isnew);
+    int u = isnew ? __popc(newmask & ((1u << lane) - 1u)) : -1;
+    const int ud = __shfl_sync(0xffffffffu, u, dup >= 0 ? dup : 0);
+    if (dup >= 0) u = ud;
+    const int nU = __popc(newmask);
+    for (int base = 0; base < nblk * 8; base += blockDim.x) {
+        const int i = base + tid;
+        const int blk = min(i >> 3, 31);
+        const int ub = __shfl_sync(0xffffffffu, u, blk);
+        const bool first = __shfl_sync(0xffffffffu, isnew ? 1 : 0, blk) != 0;
+        if (i < nblk * 8 && first) utok[ub * 8 + (i & 7)] = nbs[i];
+    }
+    for (int base = 0; base < kUC * MT; base += blockDim.x) {
+        const int i = base + tid;
+        const int cw = i / MT, m = i - cw * MT;
+        const int blk = min(cw * R + (m >> 3), 31);
+        const int ub = __shfl_sync(0xffffffffu, u, blk);
+        if (i < kUC * MT) krow[i] = (m < M && ub >= 0) ? ub * 8 + (m & 7) : -1;
+    }
+    __syncthreads();
+    return nU;
+}
+
+// Coordinates of the union rows and of the group's queries, as asynchronous copies in
+// the caller's current cp.async group (rows without a token read as (0, 0)).
+__device__ __forceinline__ void union_coords_async(const AttnArgs& a, int b, int nU, const UnionLayout& L,
+                                                   uint8_t* smem) {
+    const int* utok = reinterpret_cast<const int*>(smem + L.utok);
+    const int* qtok = reinterpret_cast<const int*>(smem + L.qtok);
+    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(b) * a.N;
+    for (int i = threadIdx.x; i < nU * 8; i += blockDim.x) {
+        const int t = utok[i];
+        cp_async8(smem_addr(smem + L.uxy) + 8 * i, xyb + (t >= 0 ? t : 0), t >= 0);
+    }
+    for (int i = threadIdx.x; i < kUC * 8; i += blockDim.x) {
+        const int t = qtok[i];
+        cp_async8(smem_addr(smem + L.qxy) + 8 * i, xyb + (t >= 0 ? t : 0), t >= 0);
+    }
 }
 
 template <int MTILES>
@@ -141,86 +223,22 @@ __global__ void __launch_bounds__(kUThreads) attn_fwd_union_kernel(const AttnArg
     const UnionLayout L = union_layout(R, MT);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int cg = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-    const int G = a.G, N = a.N, H = a.H, M = a.M;
+    const int G = a.G, N = a.N, H = a.H;
     const int g0 = cg * kUC;
     const int nblk = kUC * R;
     const int ZR = nblk * 8;
     uint8_t* ks = smem + L.ks;
     uint8_t* vs = smem + L.vs;
     uint8_t* qs = smem + L.qs;
-    int* blk_first = reinterpret_cast<int*>(smem + L.blk);
-    int* ublk = blk_first + nblk;
-    int* utok = reinterpret_cast<int*>(smem + L.utok);
-    float2* uxy = reinterpret_cast<float2*>(smem + L.uxy);
-    int* qtok = reinterpret_cast<int*>(smem + L.qtok);
-    float2* qxy = reinterpret_cast<float2*>(smem + L.qxy);
-    int* krow = reinterpret_cast<int*>(smem + L.krow);
-    int* nu_s = reinterpret_cast<int*>(smem + L.nu);
+    const int* utok = reinterpret_cast<const int*>(smem + L.utok);
+    const float2* uxy = reinterpret_cast<const float2*>(smem + L.uxy);
+    const int* qtok = reinterpret_cast<const int*>(smem + L.qtok);
+    const float2* qxy = reinterpret_cast<const float2*>(smem + L.qxy);
+    const int* krow = reinterpret_cast<const int*>(smem + L.krow);
     const size_t tok0 = static_cast<size_t>(b) * N;
-    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + tok0;
 
-    // 1. neighbour blocks and query tokens of the group
-    for (int i = tid; i < nblk; i += kUThreads) {
-        const int g = g0 + i / R, r = i % R;
-        int f = -1;
-        if (g < G) {
-            f = a.nbr[(static_cast<size_t>(b) * G + g) * M + r * 8];
-            if (f < 0 || f >= N) f = -1;
-        }
-        blk_first[i] = f;
-    }
-    for (int i = tid; i < kUC * 8; i += kUThreads) {
-        const int g = g0 + (i >> 3);
-        int id = -1;
-        if (g < G) {
-            id = a.clusters[(static_cast<size_t>(b) * G + g) * 8 + (i & 7)];
-            if (id < 0 || id >= N) id = -1;
-        }
-        qtok[i] = id;
-        qxy[i] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
-    }
-    __syncthreads();
-    // 2. de-duplicate the blocks (one warp; nblk <= 32)
-    if (warp == 0) {
-        const int f = lane < nblk ? blk_first[lane] : -1;
-        int dup = -1;
-        for (int j = 0; j < nblk; ++j) {
-            const int fj = __shfl_sync(0xffffffffu, f, j);
-            if (j < lane && dup < 0 && f >= 0 && fj == f) dup = j;
-        }
-        const bool isnew = f >= 0 && dup < 0;
-        const unsigned newmask = __ballot_sync(0xffffffffu, isnew);
-        int u = isnew ? __popc(newmask & ((1u << lane) - 1u)) : -1;
-        const int ud = __shfl_sync(0xffffffffu, u, dup >= 0 ? dup : 0);
-        if (dup >= 0) u = ud;
-        if (lane < nblk) ublk[lane] = isnew ? u : (dup >= 0 ? -(u + 2) : -1);  // -(u+2): duplicate
-        if (lane == 0) nu_s[0] = __popc(newmask);
-    }
-    __syncthreads();
-    const int nU = nu_s[0];
-    // 3. union row tokens (from the first occurrence of each block) and the block map
-    for (int i = tid; i < nblk * 8; i += kUThreads) {
-        const int blk = i >> 3, sl = i & 7;
-        const int u = ublk[blk];
-        if (u >= 0) {
-            const int g = g0 + blk / R, r = blk % R;
-            int t = a.nbr[(static_cast<size_t>(b) * G + g) * M + r * 8 + sl];
-            if (t < 0 || t >= N) t = -1;
-            utok[u * 8 + sl] = t;
-            uxy[u * 8 + sl] = t >= 0 ? xyb[t] : make_float2(0.f, 0.f);
-        }
-    }
-    for (int i = tid; i < kUC * MT; i += kUThreads) {
-        const int cw = i / MT, m = i % MT;
-        int row = -1;
-        if (m < M) {
-            int u = ublk[cw * R + (m >> 3)];
-            if (u < -1) u = -u - 2;
-            if (u >= 0) row = u * 8 + (m & 7);
-        }
-        krow[i] = row;
-    }
-    __syncthreads();
+    // 1-3. the group's neighbour rows, de-duplicated blocks, union rows and block map
+    const int nU = union_setup(a, b, g0, MT, L, smem);
     // 4. gather the union's K and V rows, the group's Q rows, and zero the spare block
     const int hlo = hg * kUH;
     for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
@@ -238,7 +256,8 @@ __global__ void __launch_bounds__(kUThreads) attn_fwd_union_kernel(const AttnArg
         const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
         cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + (ok ? off : 0), ok);
     }
-    cp_async_commit();  // group 0: K, Q
+    union_coords_async(a, b, nU, L, smem);
+    cp_async_commit();  // group 0: K, Q, coordinates
     for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
         const int row = i >> 3, ch = i & 7;
         const int t = row < nU * 8 ? utok[row] : -1;
@@ -579,83 +598,6 @@ __device__ void key_major_direct(const AttnArgs& a, int b, int kc, int h, int la
 
 // ------------------------------------------------ backward with neighbourhood unions
 
-// Union setup shared by the forward-shaped kernels: neighbour blocks of the CTA's kUC
-// clusters, de-duplicated; union row tokens/coordinates; per-cluster key-slot -> union row
-// map; the group's query tokens.  All threads of the CTA call it.
-__device__ __forceinline__ int union_setup(const AttnArgs& a, int b, int g0, int MT, const UnionLayout& L,
-                                           uint8_t* smem) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int G = a.G, N = a.N, M = a.M, R = a.R;
-    const int nblk = kUC * R;
-    int* blk_first = reinterpret_cast<int*>(smem + L.blk);
-    int* ublk = blk_first + nblk;
-    int* utok = reinterpret_cast<int*>(smem + L.utok);
-    float2* uxy = reinterpret_cast<float2*>(smem + L.uxy);
-    int* qtok = reinterpret_cast<int*>(smem + L.qtok);
-    float2* qxy = reinterpret_cast<float2*>(smem + L.qxy);
-    int* krow = reinterpret_cast<int*>(smem + L.krow);
-    int* nu_s = reinterpret_cast<int*>(smem + L.nu);
-    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(b) * N;
-    for (int i = tid; i < nblk; i += blockDim.x) {
-        const int g = g0 + i / R, r = i % R;
-        int f = -1;
-        if (g < G) {
-            f = a.nbr[(static_cast<size_t>(b) * G + g) * M + r * 8];
-            if (f < 0 || f >= N) f = -1;
-        }
-        blk_first[i] = f;
-    }
-    for (int i = tid; i < kUC * 8; i += blockDim.x) {
-        const int g = g0 + (i >> 3);
-        int id = -1;
-        if (g < G) {
-            id = a.clusters[(static_cast<size_t>(b) * G + g) * 8 + (i & 7)];
-            if (id < 0 || id >= N) id = -1;
-        }
-        qtok[i] = id;
-        qxy[i] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const int f = lane < nblk ? blk_first[lane] : -1;
-        int dup = -1;
-        for (int j = 0; j < nblk; ++j) {
-            const int fj = __shfl_sync(0xffffffffu, f, j);
-            if (j < lane && dup < 0 && f >= 0 && fj == f) dup = j;
-        }
-        const bool isnew = f >= 0 && dup < 0;
-        const unsigned newmask = __ballot_sync(0xffffffffu, isnew);
-        int u = isnew ? __popc(newmask & ((1u << lane) - 1u)) : -1;
-        const int ud = __shfl_sync(0xffffffffu, u, dup >= 0 ? dup : 0);
-        if (dup >= 0) u = ud;
-        if (lane < nblk) ublk[lane] = isnew ? u : (dup >= 0 ? -(u + 2) : -1);
-        if (lane == 0) nu_s[0] = __popc(newmask);
-    }
-    __syncthreads();
-    for (int i = tid; i < nblk * 8; i += blockDim.x) {
-        const int blk = i >> 3, sl = i & 7;
-        const int u = ublk[blk];
-        if (u >= 0) {
-            const int g = g0 + blk / R, r = blk % R;
-            int t = a.nbr[(static_cast<size_t>(b) * G + g) * M + r * 8 + sl];
-            if (t < 0 || t >= N) t = -1;
-            utok[u * 8 + sl] = t;
-            uxy[u * 8 + sl] = t >= 0 ? xyb[t] : make_float2(0.f, 0.f);
-        }
-    }
-    for (int i = tid; i < kUC * MT; i += blockDim.x) {
-        const int cw = i / MT, m = i % MT;
-        int row = -1;
-        if (m < M) {
-            int u = ublk[cw * R + (m >> 3)];
-            if (u < -1) u = -u - 2;
-            if (u >= 0) row = u * 8 + (m & 7);
-        }
-        krow[i] = row;
-    }
-    __syncthreads();
-    return nu_s[0];
-}
 
 // Query-major pass with neighbourhood unions (same CTA shape as the forward), plus one
 // extra CTA column that builds each image's reverse neighbourhood index.
@@ -704,6 +646,7 @@ __global__ void __launch_bounds__(kUThreads) attn_bwd_query_union_kernel(const A
         cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + (ok ? off : 0), ok);
         cp_async16(smem_addr(dos) + urow_off(row, ch), a.dout + (ok ? off : 0), ok);
     }
+    union_coords_async(a, b, nU, L, smem);
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
@@ -852,7 +795,7 @@ __host__ __device__ __forceinline__ KeyLayout key_layout() {
     L.stage = o; o += kUWarps * 512;
     L.ent = o; o += 4 * kKEnt;
     L.eu = o; o += 4 * kKEnt;
-    L.es = o; o += 4 * (kUC + 1);
+    L.es = o; o += 4 * (kUC + 1 + kKEnt);  // [kUC] count, then first-occurrence flags
     o = (o + 15) & ~15;
     L.qtok = o; o += 4 * rows;
     L.qxy = o; o += 8 * rows;
@@ -908,65 +851,82 @@ __global__ void __launch_bounds__(kUThreads) attn_bwd_key_union_kernel(const Att
     int* misc = reinterpret_cast<int*>(smem + L.misc);
     const int32_t* roff = a.rev_off + static_cast<size_t>(b) * (G + 1);
     const int32_t* rlist = a.rev_list + static_cast<size_t>(b) * G * a.R;
-    if (tid == 0) {
-        int acc = 0;
-        for (int c = 0; c < kUC; ++c) {
-            es[c] = acc;
-            const int kc = g0 + c;
-            if (kc < G) acc += roff[kc + 1] - roff[kc];
+    static_assert(kKEnt == 64 && kUC < 32, "warp 0 holds two list entries per lane");
+    if (warp == 0) {
+        // list offsets of the kUC key clusters (lane c), their prefix, then the entries
+        // (lanes hold entries lane and lane + 32) and their de-duplication in registers
+        int cnt = 0;
+        if (lane < kUC && g0 + lane < G) cnt = roff[g0 + lane + 1] - roff[g0 + lane];
+        const int start = (lane < kUC && g0 + lane < G) ? roff[g0 + lane] : 0;
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
-        es[kUC] = acc;
-    }
-    for (int i = tid; i < kUC * 8; i += kUThreads) {
-        const int kc = g0 + (i >> 3);
-        int id = -1;
-        if (kc < G) {
-            id = a.clusters[(static_cast<size_t>(b) * G + kc) * 8 + (i & 7)];
-            if (id < 0 || id >= N) id = -1;
-        }
-        ktok[i] = id;
-        kxy[i] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
-    }
-    __syncthreads();
-    const int ntot = es[kUC];
-    bool fits = ntot <= kKEnt;
-    if (fits) {
-        for (int i = tid; i < ntot; i += kUThreads) {
-            int c = 0;
-            while (c + 1 < kUC && es[c + 1] <= i) ++c;
-            ent[i] = rlist[roff[g0 + c] + (i - es[c])];
-        }
-        __syncthreads();
-        // first occurrences get consecutive union indices, in list order
-        if (warp == 0) {
-            int run = 0;
-            for (int base = 0; base < ntot; base += 32) {
-                const int i = base + lane;
-                bool first = false;
-                if (i < ntot) {
-                    first = true;
-                    for (int j = 0; j < i; ++j)
-                        if (ent[j] == ent[i]) { first = false; break; }
-                }
+        const int ntot_w = __shfl_sync(0xffffffffu, incl, kUC - 1);
+        int e[2] = {-1, -1};
+        if (ntot_w <= kKEnt) {
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int i = x * 32 + lane;
+                int c = 0;  // the key cluster whose list holds entry i (all lanes shuffle)
+#pragma unroll
+                for (int cc = 1; cc < kUC; ++cc)
+                    c += (i >= __shfl_sync(0xffffffffu, incl - cnt, cc)) ? 1 : 0;
+                const int es_c = __shfl_sync(0xffffffffu, incl - cnt, c);
+                const int st_c = __shfl_sync(0xffffffffu, start, c);
+                if (i < ntot_w) e[x] = rlist[st_c + (i - es_c)];
+            }
+            // first occurrence of each entry's value (src = its index), in list order
+            int src[2] = {0x7fffffff, 0x7fffffff};
+#pragma unroll 8
+            for (int j = 0; j < kKEnt; ++j) {
+                const int vj = __shfl_sync(0xffffffffu, j < 32 ? e[0] : e[1], j & 31);
+#pragma unroll
+                for (int x = 0; x < 2; ++x)
+                    if (j < src[x] && vj == e[x] && j < ntot_w) src[x] = j;
+            }
+            int run = 0, ui[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int i = x * 32 + lane;
+                const bool first = i < ntot_w && src[x] == i;
                 const unsigned m = __ballot_sync(0xffffffffu, first);
-                if (first) eu[i] = run + __popc(m & ((1u << lane) - 1u));
+                ui[x] = first ? run + __popc(m & ((1u << lane) - 1u)) : -1;
                 run += __popc(m);
+            }
+            // a repeated entry takes the union index of its first occurrence
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int i = x * 32 + lane;
+                const int s2 = (i < ntot_w) ? src[x] : i;
+                const int from0 = __shfl_sync(0xffffffffu, ui[0], s2 & 31);
+                const int from1 = __shfl_sync(0xffffffffu, ui[1], s2 & 31);
+                if (i < ntot_w) {
+                    ent[i] = e[x];
+                    eu[i] = (s2 < 32) ? from0 : from1;
+                    es[kUC + 1 + i] = (src[x] == i) ? 1 : 0;  // first occurrence
+                }
             }
             if (lane == 0) misc[0] = run;
         }
-        __syncthreads();
-        for (int i = tid; i < ntot; i += kUThreads) {
-            int src = i;
-            for (int j = 0; j < i; ++j)
-                if (ent[j] == ent[i]) { src = j; break; }
-            if (src != i) eu[i] = -1 - src;  // resolved below
+        if (lane <= kUC) es[lane] = incl - cnt;  // list start of key cluster lane; es[kUC] = total
+    } else {
+        for (int i = tid - 32; i < kUC * 8; i += kUThreads - 32) {
+            const int kc = g0 + (i >> 3);
+            int id = -1;
+            if (kc < G) {
+                id = a.clusters[(static_cast<size_t>(b) * G + kc) * 8 + (i & 7)];
+                if (id < 0 || id >= N) id = -1;
+            }
+            ktok[i] = id;
+            kxy[i] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
         }
-        __syncthreads();
-        for (int i = tid; i < ntot; i += kUThreads)
-            if (eu[i] < 0) eu[i] = eu[-1 - eu[i]];
-        fits = misc[0] <= kKQ;
-        __syncthreads();
     }
+    __syncthreads();
+    const int ntot = es[kUC];
+    const bool fits = ntot <= kKEnt && misc[0] <= kKQ;
     if (!fits) {
         // fallback: every warp handles its (key cluster, head) with direct loads
         const int cw = warp / kUH, hw = warp % kUH;
@@ -978,10 +938,7 @@ __global__ void __launch_bounds__(kUThreads) attn_bwd_key_union_kernel(const Att
     // union query rows, their lse / Delta per head of the group
     for (int i = tid; i < ntot * 8; i += kUThreads) {
         const int e = i >> 3, sl = i & 7;
-        bool first = true;
-        for (int j = 0; j < e; ++j)
-            if (ent[j] == ent[e]) { first = false; break; }
-        if (!first) continue;
+        if (!es[kUC + 1 + e]) continue;  // a repeated list entry
         const int row = eu[e] * 8 + sl;
         int t = a.clusters[(static_cast<size_t>(b) * G + ent[e]) * 8 + sl];
         if (t < 0 || t >= N) t = -1;

@@ -167,14 +167,13 @@ __device__ __forceinline__ int union_setup(const AttnArgs& a, int b, int g0, int
         qtok[i] = id;
     }
     __syncthreads();
-    // lane j < nblk: block j's union index, or the index of its first occurrence
+    // lane j < nblk: block j's union index, or the index of its first occurrence (the
+    // lowest lane holding the same first token)
     const int f = lane < nblk ? nbs[lane * 8] : -1;
-    int dup = -1;
-    for (int j = 0; j < nblk; ++j) {
-        const int fj = __shfl_sync(0xffffffffu, f, j);
-        if (j < lane && dup < 0 && f >= 0 && fj == f) dup = j;
-    }
-    const bool isnew = f >= 0 && dup < 0;
+    const unsigned peers = __match_any_sync(0xffffffffu, f);
+    const int lead = __ffs(peers) - 1;
+    const int dup = (f >= 0 && lead != lane) ? lead : -1;
+    const bool isnew = f >= 0 && lead == lane;
     const unsigned newmask = __ballot_sync(0xffffffffu, isnew);
     int u = isnew ? __popc(newmask & ((1u << lane) - 1u)) : -1;
     const int ud = __shfl_sync(0xffffffffu, u, dup >= 0 ? dup : 0);
@@ -239,32 +238,32 @@ __global__ void __launch_bounds__(kUThreads) attn_fwd_union_kernel(const AttnArg
 
     // 1-3. the group's neighbour rows, de-duplicated blocks, union rows and block map
     const int nU = union_setup(a, b, g0, MT, L, smem);
-    // 4. gather the union's K and V rows, the group's Q rows, and zero the spare block
+    // 4. gather the union's K and V rows, the group's Q rows, and zero the spare block;
+    //    thread tid copies 16-byte chunk tid % 8 of rows tid / 8, tid / 8 + 32, ...
     const int hlo = hg * kUH;
-    for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
-        const int row = i >> 3, ch = i & 7;
-        const int t = row < nU * 8 ? utok[row] : -1;
-        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
-        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
-        const int drow = row < nU * 8 ? row : ZR + (row - nU * 8);
-        cp_async16(smem_addr(ks) + urow_off(drow, ch), a.k + (ok ? off : 0), ok);
+    const int ch = tid & 7;
+    const bool ch_ok = hlo + (ch >> 2) < H;
+    const size_t cbase = (tok0 * H + hlo) * 32 + ch * 8;
+    const size_t tstride = static_cast<size_t>(H) * 32;
+    const int urows = nU * 8;
+    for (int row = tid >> 3; row < urows + 8; row += kUThreads / 8) {
+        const int t = row < urows ? utok[row] : -1;
+        const bool ok = t >= 0 && ch_ok;
+        const int drow = row < urows ? row : ZR + (row - urows);
+        cp_async16(smem_addr(ks) + urow_off(drow, ch), a.k + (ok ? cbase + t * tstride : 0), ok);
     }
-    for (int i = tid; i < kUC * 8 * 8; i += kUThreads) {
-        const int row = i >> 3, ch = i & 7;
+    for (int row = tid >> 3; row < kUC * 8; row += kUThreads / 8) {
         const int t = qtok[row];
-        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
-        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
-        cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + (ok ? off : 0), ok);
+        const bool ok = t >= 0 && ch_ok;
+        cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + (ok ? cbase + t * tstride : 0), ok);
     }
     union_coords_async(a, b, nU, L, smem);
     cp_async_commit();  // group 0: K, Q, coordinates
-    for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
-        const int row = i >> 3, ch = i & 7;
-        const int t = row < nU * 8 ? utok[row] : -1;
-        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
-        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
-        const int drow = row < nU * 8 ? row : ZR + (row - nU * 8);
-        cp_async16(smem_addr(vs) + urow_off(drow, ch), a.v + (ok ? off : 0), ok);
+    for (int row = tid >> 3; row < urows + 8; row += kUThreads / 8) {
+        const int t = row < urows ? utok[row] : -1;
+        const bool ok = t >= 0 && ch_ok;
+        const int drow = row < urows ? row : ZR + (row - urows);
+        cp_async16(smem_addr(vs) + urow_off(drow, ch), a.v + (ok ? cbase + t * tstride : 0), ok);
     }
     cp_async_commit();  // group 1: V (lands while S and the softmax run)
     cp_async_wait<1>();
@@ -629,22 +628,28 @@ __global__ void __launch_bounds__(kUThreads) attn_bwd_query_union_kernel(const A
     const float2* qxy = reinterpret_cast<const float2*>(smem + L.qxy);
     const int* krow = reinterpret_cast<const int*>(smem + L.krow);
     const int hlo = hg * kUH;
-    for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
-        const int row = i >> 3, ch = i & 7;
-        const int t = row < nU * 8 ? utok[row] : -1;
-        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
-        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
-        const int drow = row < nU * 8 ? row : ZR + (row - nU * 8);
-        cp_async16(smem_addr(ks) + urow_off(drow, ch), a.k + (ok ? off : 0), ok);
-        cp_async16(smem_addr(vs) + urow_off(drow, ch), a.v + (ok ? off : 0), ok);
-    }
-    for (int i = tid; i < kUC * 8 * 8; i += kUThreads) {
-        const int row = i >> 3, ch = i & 7;
-        const int t = qtok[row];
-        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
-        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
-        cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + (ok ? off : 0), ok);
-        cp_async16(smem_addr(dos) + urow_off(row, ch), a.dout + (ok ? off : 0), ok);
+    {
+        // thread tid copies 16-byte chunk tid % 8 of rows tid / 8, tid / 8 + 32, ...
+        const int ch = tid & 7;
+        const bool ch_ok = hlo + (ch >> 2) < H;
+        const size_t cbase = (tok0 * H + hlo) * 32 + ch * 8;
+        const size_t tstride = static_cast<size_t>(H) * 32;
+        const int urows = nU * 8;
+        for (int row = tid >> 3; row < urows + 8; row += kUThreads / 8) {
+            const int t = row < urows ? utok[row] : -1;
+            const bool ok = t >= 0 && ch_ok;
+            const int drow = row < urows ? row : ZR + (row - urows);
+            const size_t off = ok ? cbase + t * tstride : 0;
+            cp_async16(smem_addr(ks) + urow_off(drow, ch), a.k + off, ok);
+            cp_async16(smem_addr(vs) + urow_off(drow, ch), a.v + off, ok);
+        }
+        for (int row = tid >> 3; row < kUC * 8; row += kUThreads / 8) {
+            const int t = qtok[row];
+            const bool ok = t >= 0 && ch_ok;
+            const size_t off = ok ? cbase + t * tstride : 0;
+            cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + off, ok);
+            cp_async16(smem_addr(dos) + urow_off(row, ch), a.dout + off, ok);
+        }
     }
     union_coords_async(a, b, nU, L, smem);
     cp_async_commit();
@@ -969,22 +974,28 @@ __global__ void __launch_bounds__(kUThreads) attn_bwd_key_union_kernel(const Att
     uint8_t* dos = smem + L.dos;
     uint8_t* ks = smem + L.ks;
     uint8_t* vs = smem + L.vs;
-    for (int i = tid; i < (nU * 8 + 8) * 8; i += kUThreads) {
-        const int row = i >> 3, ch = i & 7;
-        const int drow = row < nU * 8 ? row : ZR + (row - nU * 8);
-        const int t = qtok[drow];
-        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
-        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
-        cp_async16(smem_addr(qs) + urow_off(drow, ch), a.q + (ok ? off : 0), ok);
-        cp_async16(smem_addr(dos) + urow_off(drow, ch), a.dout + (ok ? off : 0), ok);
-    }
-    for (int i = tid; i < kUC * 8 * 8; i += kUThreads) {
-        const int row = i >> 3, ch = i & 7;
-        const int t = ktok[row];
-        const bool ok = t >= 0 && hlo + (ch >> 2) < H;
-        const size_t off = ((tok0 + (ok ? t : 0)) * H + hlo) * 32 + ch * 8;
-        cp_async16(smem_addr(ks) + urow_off(row, ch), a.k + (ok ? off : 0), ok);
-        cp_async16(smem_addr(vs) + urow_off(row, ch), a.v + (ok ? off : 0), ok);
+    {
+        // thread tid copies 16-byte chunk tid % 8 of rows tid / 8, tid / 8 + 32, ...
+        const int ch = tid & 7;
+        const bool ch_ok = hlo + (ch >> 2) < H;
+        const size_t cbase = (tok0 * H + hlo) * 32 + ch * 8;
+        const size_t tstride = static_cast<size_t>(H) * 32;
+        const int urows = nU * 8;
+        for (int row = tid >> 3; row < urows + 8; row += kUThreads / 8) {
+            const int drow = row < urows ? row : ZR + (row - urows);
+            const int t = qtok[drow];
+            const bool ok = t >= 0 && ch_ok;
+            const size_t off = ok ? cbase + t * tstride : 0;
+            cp_async16(smem_addr(qs) + urow_off(drow, ch), a.q + off, ok);
+            cp_async16(smem_addr(dos) + urow_off(drow, ch), a.dout + off, ok);
+        }
+        for (int row = tid >> 3; row < kUC * 8; row += kUThreads / 8) {
+            const int t = ktok[row];
+            const bool ok = t >= 0 && ch_ok;
+            const size_t off = ok ? cbase + t * tstride : 0;
+            cp_async16(smem_addr(ks) + urow_off(row, ch), a.k + off, ok);
+            cp_async16(smem_addr(vs) + urow_off(row, ch), a.v + off, ok);
+        }
     }
     cp_async_commit();
     cp_async_wait<0>();

@@ -63,7 +63,11 @@ KERNELS = {
 }
 # DRAM bytes per launch measured by ncu for each call (sum over its kernels), with the
 # sha256 of the CUDA source the counters were taken on; a stale hash reports null.
-NCU_TRAFFIC: dict[str, tuple[float, str, str]] = {}
+NCU_TRAFFIC: dict[str, tuple[float, str, str]] = {
+    "attn_fwd": (13202176.0, "139177723ccca99c", "profiles/attn_kernels_step_workload.md"),
+    "attn_bwd": (35377408.0, "139177723ccca99c", "profiles/attn_kernels_step_workload.md"),
+    "knn_table": (178432.0, "139177723ccca99c", "profiles/knn_kernels_step_workload.md"),
+}
 
 
 # --------------------------------------------------------------------------- helpers
@@ -459,8 +463,9 @@ def run_gpu(args, rank: int, world: int):
     peaks = measured_peaks()
     achieved = abytes[dom_name] / (per_op[dom] * 1e-3) / 1e9
     traffic = None
+    traffic_src = None
     if dom_name in NCU_TRAFFIC and NCU_TRAFFIC[dom_name][1] == source_hash():
-        traffic = NCU_TRAFFIC[dom_name][0]
+        traffic, traffic_src = NCU_TRAFFIC[dom_name][0], NCU_TRAFFIC[dom_name][2]
     breakdown = {}
     for j, name in enumerate(OPS):
         gbs = abytes[name] / (per_op[j] * 1e-3) / 1e9
@@ -506,7 +511,8 @@ def run_gpu(args, rank: int, world: int):
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "traffic": traffic, "kernel": f"acl_{dom_name} ({', '.join(KERNELS[dom_name])})",
+                     "traffic": traffic, "traffic_unit": "bytes per launch (ncu DRAM read + write)",
+                     "traffic_source": traffic_src, "kernel": f"acl_{dom_name} ({', '.join(KERNELS[dom_name])})",
                      "alg_bytes_per_launch": int(abytes[dom_name]),
                      "launch_us": round(per_op[dom] * 1e3, 3), "peak_source": peaks["source"]},
         "cpu_baseline": cpu,
@@ -622,9 +628,21 @@ def cpu_baseline(args, sb) -> dict:
         if time.perf_counter() - t0 >= args.cpu_seconds:
             break
     dt = time.perf_counter() - t0
+    # the same on one thread, over the first image only (a few seconds)
+    oracle.set_threads(1)
+    reps1, t1 = 0, time.perf_counter()
+    while True:
+        oracle_step(sb, images=slice(0, 1))
+        reps1 += 1
+        if time.perf_counter() - t1 >= max(2.0, args.cpu_seconds / 4):
+            break
+    dt1 = time.perf_counter() - t1
+    oracle.set_threads(cores)
     return {"value": round(reps * B * N / dt, 1), "unit": "tokens/s", "cores": cores,
             "kind": "oracle",
-            "sample": f"{reps} full step(s) of the workload ({B} images), fp64 C, OpenMP over images"}
+            "sample": f"{reps} full step(s) of the workload ({B} images), fp64 C, OpenMP over images",
+            "value_1_thread": round(reps1 * N / dt1, 1),
+            "sample_1_thread": f"{reps1} step(s) of one image on 1 thread"}
 
 
 def run_reference(args, rank: int, world: int) -> None:

@@ -592,7 +592,7 @@ __global__ void __launch_bounds__(kGatherThreads)
 }
 
 template <int KT, int CH>
-__global__ void __launch_bounds__(kGatherThreads)
+__global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 3 : 1)
     knn_bwd_query_shared_kernel(const KnnArgs a, int lpq_log2, int iters) {
     extern __shared__ __align__(16) float sdp[];  // [warps][groups][heads]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1185,10 +1185,10 @@ int knn_chunks(int Q, int K, int N) {
     return static_cast<int>((static_cast<long long>(Q) * K + N) / kChunkUnits) + 1;
 }
 
-// token slices of the CSR build per image (B * slices <= 148 CTAs, at most 8)
+// token slices of the CSR build per image (B * slices <= 148 CTAs, at most 16)
 int csr_slices(int B, int N) {
     int slices = 148 / (B > 0 ? B : 1);
-    if (slices > 8) slices = 8;
+    if (slices > 16) slices = 16;
     if (slices < 1) slices = 1;
     if (slices > (N + 31) / 32) slices = (N + 31) / 32;
     if (slices < 1) slices = 1;
@@ -1203,12 +1203,15 @@ int lpq_log2_for(int d) {
     return l2;
 }
 
-// Launch shape of the query-side gather kernels (used by the workspace layout too).
+// Launch shape of the query-side gather kernels (the backward's also sizes the workspace).
 struct GatherPlan {
     int l2, ch, iters, blocks;
     bool shared;  // lane j of a query group owns neighbour j (needs K <= lanes per query)
 };
-GatherPlan gather_plan(int B, int Q, int d, int K) {
+// Launch shape of the query-side gather kernels.  A CTA walks `iters` consecutive blocks of
+// queries; iters is chosen so the grid fits one wave of the kernel's resident CTAs (the
+// backward's query pass holds fewer CTAs per SM than the forward: more registers).
+GatherPlan gather_plan(int B, int Q, int d, int K, bool bwd) {
     GatherPlan g;
     g.l2 = lpq_log2_for(d);
     const int lanes = 1 << g.l2;
@@ -1216,7 +1219,13 @@ GatherPlan gather_plan(int B, int Q, int d, int K) {
     g.shared = K <= lanes;
     const long long per_iter = static_cast<long long>(kGatherWarps) * (32 >> g.l2);
     const long long total = static_cast<long long>(B) * Q;
-    g.iters = (g.shared && total >= per_iter * 4 * 148 * 2) ? 4 : 1;
+    const int resident = bwd ? ((K <= 8 && g.ch == 1) ? 3 : 2) : 4;
+    long long it = 1;
+    if (g.shared) {
+        it = (total + per_iter * 148 * resident - 1) / (per_iter * 148 * resident);
+        it = it < 1 ? 1 : (it > 8 ? 8 : it);
+    }
+    g.iters = static_cast<int>(it);
     g.blocks = static_cast<int>((total + per_iter * g.iters - 1) / (per_iter * g.iters));
     return g;
 }
@@ -1300,7 +1309,7 @@ KnnWorkspace knn_workspace_layout(int B, int Q, int N, int d, int K) {
     const size_t NH = static_cast<size_t>(d / 32);
     const size_t BQ = static_cast<size_t>(B) * Q;
     KnnWorkspace w;
-    w.query_blocks = gather_plan(B, Q, d, K).blocks;
+    w.query_blocks = gather_plan(B, Q, d, K, true).blocks;
     size_t off = 0;
     w.w = off;       off += up(sizeof(float) * BQ * NH * K);
     w.keys = off;    off += up(sizeof(int32_t) * BQ * K);
@@ -1322,7 +1331,7 @@ KnnWorkspace knn_workspace_layout(int B, int Q, int N, int d, int K) {
 }
 
 cudaError_t launch_knn_fwd(const KnnArgs& a, cudaStream_t st) {
-    const GatherPlan g = gather_plan(a.B, a.Q, a.d, a.K);
+    const GatherPlan g = gather_plan(a.B, a.Q, a.d, a.K, false);
     if (g.blocks == 0) return cudaSuccess;
     cudaError_t e;
     if (g.shared)
@@ -1356,7 +1365,7 @@ cudaError_t launch_knn_bwd_indexed(const KnnArgs& a, cudaStream_t st) {
     const int NH = a.d / 32;
     const KnnWorkspace ws = knn_workspace_layout(a.B, a.Q, a.N, a.d, a.K);
     const unsigned qblocks = static_cast<unsigned>(ws.query_blocks);
-    const GatherPlan g = gather_plan(a.B, a.Q, a.d, a.K);
+    const GatherPlan g = gather_plan(a.B, a.Q, a.d, a.K, true);
     cudaError_t e = cudaSuccess;
     if (qblocks > 0) {
         const size_t smem = sizeof(float) * kGatherWarps * (32 >> l2) * NH;

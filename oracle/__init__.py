@@ -114,7 +114,10 @@ def knn_table(xy, GH: int = 64, GW: int = 64, K: int = 8) -> np.ndarray:
     return out
 
 
-def knn_fwd(queries, feats, xy, table, p):
+KNN_EXP, KNN_INVPOW = 0, 1  # weight kernels: softmax(-p d) and d^-p / sum d^-p
+
+
+def knn_fwd(queries, feats, xy, table, p, kind=KNN_EXP):
     queries, xy, table = _f32(queries), _f32(xy), _i32(table)
     feats, p = _f64(feats), _f64(p)
     B, Q = queries.shape[:2]
@@ -122,11 +125,11 @@ def knn_fwd(queries, feats, xy, table, p):
     GH, GW, K = table.shape[1:]
     out = np.empty((B, Q, d), dtype=np.float64)
     _check(lib().orc_knn_fwd_batch(_p(queries), B, Q, _p(feats), _p(xy), N, d, _p(table),
-                                   GH, GW, K, _p(p), _p(out)), "knn_fwd")
+                                   GH, GW, K, _p(p), int(kind), _p(out)), "knn_fwd")
     return out
 
 
-def knn_bwd(queries, feats, xy, table, p, dout):
+def knn_bwd(queries, feats, xy, table, p, dout, kind=KNN_EXP):
     queries, xy, table = _f32(queries), _f32(xy), _i32(table)
     feats, p, dout = _f64(feats), _f64(p), _f64(dout)
     B, Q = queries.shape[:2]
@@ -136,6 +139,7 @@ def knn_bwd(queries, feats, xy, table, p, dout):
     dq = np.empty((B, Q, 2), dtype=np.float64)
     dp = np.empty((d // 32,), dtype=np.float64)
     _check(lib().orc_knn_bwd_batch(_p(queries), B, Q, _p(feats), _p(xy), N, d, _p(table),
-                                   GH, GW, K, _p(p), _p(dout), _p(dF), _p(dq), _p(dp)),
+                                   GH, GW, K, _p(p), int(kind), _p(dout), _p(dF), _p(dq),
+                                   _p(dp)),
            "knn_bwd")
     return dF, dq, dp

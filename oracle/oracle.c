@@ -404,13 +404,21 @@ static int quantise(float v, int n) {
 }
 
 /*
- * d_k = ||q - p_{t_k}|| (Euclidean, fp64); per head h (channels h*32..h*32+31):
- * w_hk = exp(-p_h (d_k - d_min)) / sum_k' exp(-p_h (d_k' - d_min));
- * out[q][h*32+e] = sum_k w_hk f[t_k][h*32+e].  Table slots holding -1 are
- * skipped.  A query whose row holds no token gets out = 0.
+ * d_k = ||q - p_{t_k}|| (Euclidean, fp64); per head h (channels h*32..h*32+31) the
+ * weights of the K neighbours, for the two kernels the AFFMAE notes compare ("Key Designs"
+ * 2):
+ *   kind 0, exponential (the method):  w_hk = exp(-p_h (d_k - d_min)) / sum_k' (same),
+ *     i.e. softmax_k(-p_h d_k);
+ *   kind 1, inverse power (the original AFF kernel the notes replace):
+ *     w_hk = d_k^(-p_h) / sum_k' d_k'^(-p_h), evaluated as (d_min / d_k)^p_h / sum (same),
+ *     the same ratio with both terms divided by d_min^(-p_h); a neighbour at d_min gets
+ *     the factor 1 (so when the query sits on tokens, d_min = 0, they share the weight and
+ *     the others get 0, the limit of the definition), and p_h = 0 gives equal weights.
+ * out[q][h*32+e] = sum_k w_hk f[t_k][h*32+e].  Table slots holding -1 are skipped.  A
+ * query whose row holds no token gets out = 0.
  */
 static int knn_weights(const float* qxy, const float* xy, const int32_t* row, int K,
-                       double ph, double* dist, double* w) {
+                       double ph, int kind, double* dist, double* w) {
     double dmin = INFINITY;
     int any = 0;
     for (int kk = 0; kk < K; ++kk) {
@@ -425,7 +433,9 @@ static int knn_weights(const float* qxy, const float* xy, const int32_t* row, in
     if (!any) return 0;
     double sum = 0.0;
     for (int kk = 0; kk < K; ++kk) {
-        w[kk] = (row[kk] < 0) ? 0.0 : exp(-ph * (dist[kk] - dmin));
+        if (row[kk] < 0) w[kk] = 0.0;
+        else if (kind == 0) w[kk] = exp(-ph * (dist[kk] - dmin));
+        else w[kk] = (dist[kk] == dmin || ph == 0.0) ? 1.0 : pow(dmin / dist[kk], ph);
         sum += w[kk];
     }
     for (int kk = 0; kk < K; ++kk) w[kk] /= sum;
@@ -434,7 +444,7 @@ static int knn_weights(const float* qxy, const float* xy, const int32_t* row, in
 
 int orc_knn_fwd(const float* queries, int Q, const double* feats, const float* xy,
                 int N, int d, const int32_t* table, int GH, int GW, int K,
-                const double* p, double* out) {
+                const double* p, int kind, double* out) {
     if (Q < 0 || N < 1 || d < 32 || d % 32 != 0 || K < 1 || K > 64) return 1;
     int nh = d / 32;
     double dist[64], w[64];
@@ -445,7 +455,7 @@ int orc_knn_fwd(const float* queries, int Q, const double* feats, const float* x
         double* oq = out + (size_t)qi * d;
         for (int c = 0; c < d; ++c) oq[c] = 0.0;
         for (int h = 0; h < nh; ++h) {
-            if (!knn_weights(qxy, xy, row, K, p[h], dist, w)) break;
+            if (!knn_weights(qxy, xy, row, K, p[h], kind, dist, w)) break;
             for (int kk = 0; kk < K; ++kk) {
                 int32_t t = row[kk];
                 if (t < 0) continue;
@@ -458,17 +468,21 @@ int orc_knn_fwd(const float* queries, int Q, const double* feats, const float* x
 }
 
 /*
- * Backward of the gather.  With z_hk = -p_h d_k the logits of w_h:
+ * Backward of the gather.  With z_hk the logits of w_h (w_h = softmax_k(z_hk)):
+ * z_hk = -p_h d_k (kind 0) or -p_h ln d_k (kind 1), and
  *   dw_hk = <dOut_q,h , f_{t_k},h>,  ds_hk = w_hk (dw_hk - sum_k' w_hk' dw_hk'),
- *   dp_h += sum_k ds_hk (-d_k),
- *   dq   += sum_{h,k} ds_hk (-p_h) (q - p_{t_k}) / d_k   (term taken as 0 when d_k = 0),
+ *   dp_h += sum_k ds_hk dz_hk/dp_h,  dz/dp = -d_k (kind 0), -ln d_k (kind 1),
+ *   dq   += sum_{h,k} ds_hk dz_hk/dq, dz/dq = -p_h (q - p_{t_k}) / d_k (kind 0),
+ *           -p_h (q - p_{t_k}) / d_k^2 (kind 1),
  *   dF_t += w_hk dOut_q,h for t = t_k.
+ * Terms of a neighbour at d_k = 0 are taken as 0 in dq (both kinds) and in dp (kind 1),
+ * where the derivatives are undefined.
  * The cell index is piecewise constant in q and has no gradient; token
  * coordinates get none.  dfeats [N][d], dq [Q][2] and dp [d/32] are overwritten.
  */
 int orc_knn_bwd(const float* queries, int Q, const double* feats, const float* xy,
                 int N, int d, const int32_t* table, int GH, int GW, int K,
-                const double* p, const double* dout,
+                const double* p, int kind, const double* dout,
                 double* dfeats, double* dq, double* dp) {
     if (Q < 0 || N < 1 || d < 32 || d % 32 != 0 || K < 1 || K > 64) return 1;
     int nh = d / 32;
@@ -482,7 +496,7 @@ int orc_knn_bwd(const float* queries, int Q, const double* feats, const float* x
         const int32_t* row = table + ((size_t)cy * GW + cx) * K;
         const double* g = dout + (size_t)qi * d;
         for (int h = 0; h < nh; ++h) {
-            if (!knn_weights(qxy, xy, row, K, p[h], dist, w)) break;
+            if (!knn_weights(qxy, xy, row, K, p[h], kind, dist, w)) break;
             double sdw = 0.0;
             for (int kk = 0; kk < K; ++kk) {
                 int32_t t = row[kk];
@@ -496,10 +510,12 @@ int orc_knn_bwd(const float* queries, int Q, const double* feats, const float* x
                 int32_t t = row[kk];
                 if (t < 0) continue;
                 double ds = w[kk] * (dw[kk] - sdw);
-                dp[h] += ds * (-dist[kk]);
+                if (kind == 0) dp[h] += ds * (-dist[kk]);
+                else if (dist[kk] > 0.0) dp[h] += ds * (-log(dist[kk]));
                 if (dist[kk] > 0.0) {
-                    double ux = ((double)qxy[0] - (double)xy[2 * t]) / dist[kk];
-                    double uy = ((double)qxy[1] - (double)xy[2 * t + 1]) / dist[kk];
+                    double r = kind == 0 ? dist[kk] : dist[kk] * dist[kk];
+                    double ux = ((double)qxy[0] - (double)xy[2 * t]) / r;
+                    double uy = ((double)qxy[1] - (double)xy[2 * t + 1]) / r;
                     dq[2 * qi] += ds * (-p[h]) * ux;
                     dq[2 * qi + 1] += ds * (-p[h]) * uy;
                 }
@@ -583,19 +599,19 @@ int orc_knn_table_batch(const float* xy, int B, int N, int GH, int GW, int K,
 
 int orc_knn_fwd_batch(const float* queries, int B, int Q, const double* feats,
                       const float* xy, int N, int d, const int32_t* table, int GH, int GW,
-                      int K, const double* p, double* out) {
+                      int K, const double* p, int kind, double* out) {
     int rc = 0;
     #pragma omp parallel for schedule(dynamic) reduction(|:rc)
     for (int b = 0; b < B; ++b)
         rc |= orc_knn_fwd(queries + (size_t)b * Q * 2, Q, feats + (size_t)b * N * d,
                           xy + (size_t)b * N * 2, N, d, table + (size_t)b * GH * GW * K,
-                          GH, GW, K, p, out + (size_t)b * Q * d);
+                          GH, GW, K, p, kind, out + (size_t)b * Q * d);
     return rc;
 }
 
 int orc_knn_bwd_batch(const float* queries, int B, int Q, const double* feats,
                       const float* xy, int N, int d, const int32_t* table, int GH, int GW,
-                      int K, const double* p, const double* dout, double* dfeats,
+                      int K, const double* p, int kind, const double* dout, double* dfeats,
                       double* dq, double* dp) {
     int rc = 0, nh = d / 32;
     double* part = (double*)calloc((size_t)B * nh, sizeof(double));
@@ -604,7 +620,7 @@ int orc_knn_bwd_batch(const float* queries, int B, int Q, const double* feats,
     for (int b = 0; b < B; ++b)
         rc |= orc_knn_bwd(queries + (size_t)b * Q * 2, Q, feats + (size_t)b * N * d,
                           xy + (size_t)b * N * 2, N, d, table + (size_t)b * GH * GW * K,
-                          GH, GW, K, p, dout + (size_t)b * Q * d, dfeats + (size_t)b * N * d,
+                          GH, GW, K, p, kind, dout + (size_t)b * Q * d, dfeats + (size_t)b * N * d,
                           dq + (size_t)b * Q * 2, part + (size_t)b * nh);
     for (int h = 0; h < nh; ++h) {
         double acc = 0.0;

@@ -22,12 +22,14 @@ int orc_attn_bwd(const double* q, const double* k, const double* v, const float*
                  int N, int H, int D, int C, int M, double scale, const double* dout,
                  double* dq, double* dk, double* dv, double* dbias);
 int orc_knn_table(const float* xy, int N, int GH, int GW, int K, int32_t* table);
+/* kind: 0 = exponential kernel softmax(-p d), 1 = inverse power d^-p / sum d^-p */
 int orc_knn_fwd(const float* queries, int Q, const double* feats, const float* xy,
                 int N, int d, const int32_t* table, int GH, int GW, int K,
-                const double* p, double* out);
+                const double* p, int kind, double* out);
 int orc_knn_bwd(const float* queries, int Q, const double* feats, const float* xy,
                 int N, int d, const int32_t* table, int GH, int GW, int K,
-                const double* p, const double* dout, double* dfeats, double* dq, double* dp);
+                const double* p, int kind, const double* dout, double* dfeats, double* dq,
+                double* dp);
 
 int orc_cluster_batch(const float* xy, int B, int N, int C, int32_t* clusters);
 int orc_neighbors_batch(const float* xy, const int32_t* clusters, int B, int N, int C,
@@ -43,9 +45,9 @@ int orc_attn_bwd_batch(const double* q, const double* k, const double* v, const 
 int orc_knn_table_batch(const float* xy, int B, int N, int GH, int GW, int K, int32_t* table);
 int orc_knn_fwd_batch(const float* queries, int B, int Q, const double* feats,
                       const float* xy, int N, int d, const int32_t* table, int GH, int GW,
-                      int K, const double* p, double* out);
+                      int K, const double* p, int kind, double* out);
 int orc_knn_bwd_batch(const float* queries, int B, int Q, const double* feats,
                       const float* xy, int N, int d, const int32_t* table, int GH, int GW,
-                      int K, const double* p, const double* dout, double* dfeats,
+                      int K, const double* p, int kind, const double* dout, double* dfeats,
                       double* dq, double* dp);
 #endif

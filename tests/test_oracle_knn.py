@@ -171,3 +171,130 @@ def test_backward_finite_differences():
             assert dq[0, i, j] == pytest.approx(fd, rel=2e-4, abs=2e-5), (i, j)
             checked += 1
     assert checked > 200
+
+
+# ------------------------------------------------------------------ inverse-power kernel
+# AFFMAE notes, "Key Designs" 2: the original AFF weighting w_i proportional to d_i^-p,
+# which the notes replace by the exponential kernel because it overflows at short range and
+# underflows at long range in mixed precision.
+
+INV = oracle.KNN_INVPOW
+
+
+def _one_row_table(GH, GW, ids):
+    t = np.empty((1, GH, GW, len(ids)), dtype=np.int32)
+    t[...] = np.asarray(ids, dtype=np.int32)
+    return t
+
+
+def test_invpow_two_neighbours_closed_form():
+    # w_1 = 1 / (1 + (d1/d2)^p), w_2 = 1 - w_1 for two tokens at distances d1, d2
+    xy = np.array([[[3.0, 2.0], [2.0, 6.0]]], dtype=np.float32)
+    q = np.array([[[2.0, 2.5]]], dtype=np.float32)
+    feats = np.random.default_rng(3).standard_normal((1, 2, 32))
+    table = _one_row_table(8, 8, [0, 1])
+    d1, d2 = np.hypot(1.0, 0.5), np.hypot(0.0, 3.5)
+    for p in (0.5, 1.0, 2.5, 7.0):
+        out = oracle.knn_fwd(q, feats, xy, table, np.array([p]), kind=INV)[0, 0]
+        w1 = 1.0 / (1.0 + (d1 / d2) ** p)
+        np.testing.assert_allclose(out, w1 * feats[0, 0] + (1 - w1) * feats[0, 1], rtol=1e-12)
+
+
+def test_invpow_scale_invariance_and_exp_is_not():
+    # d^-p weights only see distance ratios: scaling every token's offset from the query by
+    # s leaves them unchanged; softmax(-p d) weights change
+    rng = np.random.default_rng(5)
+    K = 6
+    off = rng.uniform(-1.5, 1.5, size=(K, 2))
+    q = np.array([[[20.5, 20.5]]], dtype=np.float32)
+    feats = rng.standard_normal((1, K, 64))
+    table = _one_row_table(32, 32, list(range(K)))
+    p = np.array([1.3, 3.0])
+    outs = {}
+    for kind in (oracle.KNN_EXP, INV):
+        for s in (1.0, 4.0):
+            xy = (q[0, 0].astype(np.float64) + s * off).astype(np.float32)[None]
+            outs[kind, s] = oracle.knn_fwd(q, feats, xy, table, p, kind=kind)[0, 0]
+    np.testing.assert_allclose(outs[INV, 1.0], outs[INV, 4.0], rtol=1e-6, atol=1e-6)
+    assert np.abs(outs[oracle.KNN_EXP, 1.0] - outs[oracle.KNN_EXP, 4.0]).max() > 1e-2
+
+
+def test_invpow_query_on_tokens_and_zero_temperature():
+    # the limit d -> 0: a query on a token takes that token's features (shared equally by
+    # coincident tokens); p = 0 gives the plain mean
+    xy = np.array([[[1.25, 1.75], [1.25, 1.75], [3.0, 0.5], [0.1, 3.9]]], dtype=np.float32)
+    feats = np.random.default_rng(7).standard_normal((1, 4, 32))
+    table = _one_row_table(4, 4, [0, 1, 2, 3])
+    q = np.array([[[1.25, 1.75], [3.0, 0.5]]], dtype=np.float32)
+    out = oracle.knn_fwd(q, feats, xy, table, np.array([2.0]), kind=INV)[0]
+    np.testing.assert_allclose(out[0], 0.5 * (feats[0, 0] + feats[0, 1]), rtol=1e-12)
+    np.testing.assert_allclose(out[1], feats[0, 2], rtol=1e-12)
+    out = oracle.knn_fwd(q, feats, xy, table, np.array([0.0]), kind=INV)[0]
+    np.testing.assert_allclose(out[0], feats[0].mean(axis=0), rtol=1e-12)
+    dF, dq, dp = oracle.knn_bwd(q, feats, xy, table, np.array([2.0]),
+                                np.ones((1, 2, 32)), kind=INV)
+    assert np.isfinite(dq).all() and np.isfinite(dp).all() and np.isfinite(dF).all()
+
+
+def _loss_inv(q, feats, xy, table, p, dout):
+    return float((oracle.knn_fwd(q, feats, xy, table, p, kind=INV) * dout).sum())
+
+
+def test_invpow_backward_finite_differences():
+    xy, feats, q, p, table = _problem(N=150, d=64, Q=120, seed=11)
+    dout = np.random.default_rng(4).standard_normal((1, 120, 64))
+    dF, dq, dp = oracle.knn_bwd(q, feats, xy, table, p, dout, kind=INV)
+    rng = np.random.default_rng(8)
+    eps = 1e-6
+    for _ in range(40):
+        idx = (0, int(rng.integers(0, 150)), int(rng.integers(0, 64)))
+        fp, fm = feats.copy(), feats.copy()
+        fp[idx] += eps
+        fm[idx] -= eps
+        fd = (_loss_inv(q, fp, xy, table, p, dout) - _loss_inv(q, fm, xy, table, p, dout)) / (2 * eps)
+        assert dF[idx] == pytest.approx(fd, rel=1e-6, abs=1e-8)
+    for h in range(2):
+        pp, pm = p.copy(), p.copy()
+        pp[h] += eps
+        pm[h] -= eps
+        fd = (_loss_inv(q, feats, xy, table, pp, dout) - _loss_inv(q, feats, xy, table, pm, dout)) / (2 * eps)
+        assert dp[h] == pytest.approx(fd, rel=1e-6, abs=1e-8)
+    e = 2.0 ** -12
+    checked = 0
+    for i in range(120):
+        for j in range(2):
+            v = float(q[0, i, j])
+            if abs(v - np.round(v)) < 4 * e:
+                continue
+            qp, qm = q.copy(), q.copy()
+            qp[0, i, j] = np.float32(v + e)
+            qm[0, i, j] = np.float32(v - e)
+            fd = (_loss_inv(qp, feats, xy, table, p, dout) - _loss_inv(qm, feats, xy, table, p, dout)) / (2 * e)
+            assert dq[0, i, j] == pytest.approx(fd, rel=5e-4, abs=5e-5), (i, j)
+            checked += 1
+    assert checked > 200
+
+
+def test_invpow_half_precision_range_versus_exp_kernel():
+    # the reason the notes give for the exponential kernel: evaluated directly in half
+    # precision, d^-p overflows for close tokens and underflows for far ones, so the
+    # normalised weights become nan or lose every term; softmax(-p d) with the minimum
+    # subtracted stays in [0, 1].  (The oracle and the CUDA path evaluate the inverse power
+    # as (d_min / d)^p, which stays in [0, 1] as well.)
+    p = np.float16(4.0)
+    near = np.array([0.05, 0.3, 0.6], dtype=np.float16)        # cell units
+    far = np.array([40.0, 55.0, 60.0], dtype=np.float16)
+    with np.errstate(over="ignore", divide="ignore", invalid="ignore"):
+        w_near = near ** -p                                        # fp16: 0.05^-4 = 160000
+        assert np.isinf(w_near[0])
+        assert np.isnan(w_near / w_near.sum()).any()
+        w_far = far ** -np.float16(8.0)                            # ~1e-13: below fp16 range
+        assert (w_far == 0).all()
+        bf_near = (near.astype(np.float32) ** -np.float32(30.0))   # bf16 range = fp32 range
+        assert np.isinf(bf_near[0])
+    for dist in (near, far):
+        z = -p * (dist - dist.min())                                # exponential kernel
+        w = np.exp(z.astype(np.float16))
+        assert np.isfinite(w).all() and w.max() == np.float16(1.0)
+        r = (dist.min() / dist) ** p                                # the ratio form
+        assert np.isfinite(r).all() and r.max() == np.float16(1.0)

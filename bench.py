@@ -236,7 +236,7 @@ class StepSet:
         ts = list(self.inputs.values()) + list(self.outputs.values()) + [self.ws_attn, self.ws_knn]
         return sum(t.numel() * t.element_size() for t in ts)
 
-    def op(self, name: str, stream):
+    def op(self, name: str, stream, kind: int = 0):
         i, o, acl = self.inputs, self.outputs, self.acl
         if name == "cluster":
             acl.acl_cluster(i["coords"], 8, clusters=o["clusters"], stream=stream)
@@ -254,14 +254,15 @@ class StepSet:
             acl.acl_knn_table(i["coords"], self.GH, self.GW, self.K, table=o["table"], stream=stream)
         elif name == "knn_fwd":
             acl.acl_knn_gather_fwd(i["queries"], i["feats"], i["coords"], o["table"], i["p"],
-                                   out=o["out"], stream=stream)
+                                   out=o["out"], stream=stream, kind=kind)
         elif name == "knn_index":
             acl.acl_knn_gather_index(i["queries"], o["table"], self.N, self.d, self.ws_knn,
                                      stream=stream)
         elif name == "knn_bwd":
             acl.acl_knn_gather_bwd_indexed(i["queries"], i["feats"], i["coords"], o["table"],
                                            i["p"], i["dout"], self.ws_knn, dfeats=o["dfeats"],
-                                           dqueries=o["dqueries"], dp=o["dp"], stream=stream)
+                                           dqueries=o["dqueries"], dp=o["dp"], stream=stream,
+                                           kind=kind)
         else:
             raise KeyError(name)
 
@@ -440,6 +441,21 @@ def run_gpu(args, rank: int, world: int):
             serial_graphs[it % n_sets].replay()
     torch.cuda.synchronize()
     per_op = per_call(serial_events, n_sets)
+    # the inverse-power weight kernel (the original AFF weighting) on the same gathers:
+    # forward and backward of set 0, one call at a time
+    inv_us = {}
+    s0 = sets[0]
+    with torch.cuda.stream(stream):
+        for name in ("knn_fwd", "knn_bwd"):
+            for _ in range(3):
+                s0.op(name, stream, kind=acl.ACL_KNN_INVPOW)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(20):
+                s0.op(name, stream, kind=acl.ACL_KNN_INVPOW)
+            e1.record(stream)
+            e1.synchronize()
+            inv_us[name] = round(e0.elapsed_time(e1) / 20 * 1e3, 2)
     # keep the same load on the GPU until the clock sampler has several samples
     t_wall = time.time()
     it = 0
@@ -508,6 +524,8 @@ def run_gpu(args, rank: int, world: int):
                              "after the timed region); the step overlaps the two chains",
             "per_call_concurrent_us": {n: round(per_op_concurrent[j] * 1e3, 2)
                                        for j, n in enumerate(OPS)},
+            "knn_invpow_us": {**inv_us, "note": "inverse-power weight kernel (d^-p), same "
+                              "gathers, set 0, L2-warm (one set): compare with per_call"},
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),

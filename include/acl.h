@@ -246,6 +246,28 @@ acl_status acl_knn_gather_fwd(const float* queries, int B, int Q, const acl_bf16
                               acl_stream_t stream);
 
 /*
+ * Weight kernels of the gather.  AFF notes, "Key Designs" 2: the method uses the
+ * exponential distance kernel w_k = softmax_k(-p d_k); the original AFF weighting it
+ * replaced is the inverse power w_k = d_k^-p / sum_k' d_k'^-p, which the notes describe as
+ * overflowing at short range and underflowing at long range in mixed precision.  Here the
+ * inverse power is evaluated as (d_min / d_k)^p / sum (the same ratio, in [0, 1]): a
+ * neighbour at d_min gets 1 (a query on a token, d_min = 0, puts all weight on the tokens
+ * at its position, the d -> 0 limit), p = 0 gives equal weights; p must be >= 0.  In the
+ * backward, dz/dp = -ln d_k and dz/dq = -p (q - x_k) / d_k^2; terms of a neighbour at
+ * d_k = 0 are 0.
+ */
+typedef enum {
+    ACL_KNN_EXP = 0,     /* softmax(-p d): the method's kernel (the plain entry points)   */
+    ACL_KNN_INVPOW = 1   /* d^-p / sum d^-p: the original AFF weighting                   */
+} acl_knn_kernel;
+
+/* acl_knn_gather_fwd with a choice of weight kernel (ACL_ERR_INVALID_ARG for any other). */
+acl_status acl_knn_gather_fwd_ex(const float* queries, int B, int Q, const acl_bf16* feats,
+                                 const float* coords, int N, int d, const int32_t* table,
+                                 int H, int W, int K, const float* p, acl_knn_kernel kind,
+                                 acl_bf16* out, acl_stream_t stream);
+
+/*
  * acl_knn_gather_bwd -- KNN gather, backward (a7).  With z_hk = -p_h d_k:
  *   dw_hk = <dOut_h, f_{t_k},h>, ds_hk = w_hk (dw_hk - sum_k' w_hk' dw_hk'),
  *   dp_h = sum over all queries and k of ds_hk (-d_k),
@@ -265,6 +287,14 @@ acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16
                               int H, int W, int K, const float* p, const acl_bf16* dOut,
                               acl_bf16* dfeats, float* dqueries, float* dp,
                               void* workspace, size_t ws_bytes, acl_stream_t stream);
+
+/* acl_knn_gather_bwd with a choice of weight kernel (the kind of the forward). */
+acl_status acl_knn_gather_bwd_ex(const float* queries, int B, int Q, const acl_bf16* feats,
+                                 const float* coords, int N, int d, const int32_t* table,
+                                 int H, int W, int K, const float* p, acl_knn_kernel kind,
+                                 const acl_bf16* dOut, acl_bf16* dfeats, float* dqueries,
+                                 float* dp, void* workspace, size_t ws_bytes,
+                                 acl_stream_t stream);
 
 /*
  * acl_knn_gather_index -- the first stage of acl_knn_gather_bwd on its own: the inverse
@@ -295,6 +325,16 @@ acl_status acl_knn_gather_bwd_indexed(const float* queries, int B, int Q, const 
                                       int H, int W, int K, const float* p, const acl_bf16* dOut,
                                       acl_bf16* dfeats, float* dqueries, float* dp,
                                       void* workspace, size_t ws_bytes, acl_stream_t stream);
+
+/* acl_knn_gather_bwd_indexed with a choice of weight kernel (the index does not depend on
+ * it). */
+acl_status acl_knn_gather_bwd_indexed_ex(const float* queries, int B, int Q,
+                                         const acl_bf16* feats, const float* coords, int N, int d,
+                                         const int32_t* table, int H, int W, int K,
+                                         const float* p, acl_knn_kernel kind,
+                                         const acl_bf16* dOut, acl_bf16* dfeats, float* dqueries,
+                                         float* dp, void* workspace, size_t ws_bytes,
+                                         acl_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -45,6 +45,11 @@ SIGNATURES = {
     "acl_knn_gather_bwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P,
                                 _P, _P, _Z, _P]),
     "acl_knn_gather_index": (_I, [_P, _I, _I, _I, _I, _P, _I, _I, _I, _P, _Z, _P]),
+    "acl_knn_gather_fwd_ex": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _I, _P, _P]),
+    "acl_knn_gather_bwd_ex": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _I, _P, _P,
+                                   _P, _P, _P, _Z, _P]),
+    "acl_knn_gather_bwd_indexed_ex": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _I,
+                                           _P, _P, _P, _P, _P, _Z, _P]),
     "acl_knn_gather_bwd_indexed": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P,
                                         _P, _P, _P, _P, _Z, _P]),
 }
@@ -263,12 +268,16 @@ def _gather_shapes(queries, feats, coords, table, p):
     return B, Q, N, d, H, W, K
 
 
-def acl_knn_gather_fwd(queries, feats, coords, table, p, out=None, stream=None):
-    """KNN distance-softmax gather forward -> out [B,Q,d] bf16."""
+ACL_KNN_EXP, ACL_KNN_INVPOW = 0, 1  # weight kernels: softmax(-p d), d^-p / sum d^-p
+
+
+def acl_knn_gather_fwd(queries, feats, coords, table, p, out=None, stream=None,
+                       kind: int = ACL_KNN_EXP):
+    """KNN distance-weighted gather forward -> out [B,Q,d] bf16."""
     B, Q, N, d, H, W, K = _gather_shapes(queries, feats, coords, table, p)
     out = _out(out, (B, Q, d), torch.bfloat16, feats, "out")
-    _call("acl_knn_gather_fwd", _ptr(queries), B, Q, _ptr(feats), _ptr(coords), N, d,
-          _ptr(table), H, W, K, _ptr(p), _ptr(out), _stream(stream))
+    _call("acl_knn_gather_fwd_ex", _ptr(queries), B, Q, _ptr(feats), _ptr(coords), N, d,
+          _ptr(table), H, W, K, _ptr(p), int(kind), _ptr(out), _stream(stream))
     return out
 
 
@@ -285,22 +294,24 @@ def acl_knn_gather_index(queries, table, N: int, d: int, workspace: torch.Tensor
 
 
 def acl_knn_gather_bwd_indexed(queries, feats, coords, table, p, dOut, workspace: torch.Tensor,
-                               dfeats=None, dqueries=None, dp=None, stream=None):
+                               dfeats=None, dqueries=None, dp=None, stream=None,
+                               kind: int = ACL_KNN_EXP):
     """acl_knn_gather_bwd reading the inverse index that acl_knn_gather_index wrote into
     `workspace` -> (dfeats, dqueries, dp)."""
-    return _gather_bwd("acl_knn_gather_bwd_indexed", queries, feats, coords, table, p, dOut,
-                       dfeats, dqueries, dp, workspace, stream)
+    return _gather_bwd("acl_knn_gather_bwd_indexed_ex", queries, feats, coords, table, p, dOut,
+                       dfeats, dqueries, dp, workspace, stream, kind)
 
 
 def acl_knn_gather_bwd(queries, feats, coords, table, p, dOut, dfeats=None, dqueries=None,
-                       dp=None, workspace: torch.Tensor | None = None, stream=None):
+                       dp=None, workspace: torch.Tensor | None = None, stream=None,
+                       kind: int = ACL_KNN_EXP):
     """KNN gather backward -> (dfeats [B,N,d] bf16, dqueries [B,Q,2] f32, dp [d/32] f32)."""
-    return _gather_bwd("acl_knn_gather_bwd", queries, feats, coords, table, p, dOut, dfeats,
-                       dqueries, dp, workspace, stream)
+    return _gather_bwd("acl_knn_gather_bwd_ex", queries, feats, coords, table, p, dOut, dfeats,
+                       dqueries, dp, workspace, stream, kind)
 
 
 def _gather_bwd(fn, queries, feats, coords, table, p, dOut, dfeats, dqueries, dp, workspace,
-                stream):
+                stream, kind):
     B, Q, N, d, H, W, K = _gather_shapes(queries, feats, coords, table, p)
     _need(dOut, "dOut", torch.bfloat16, (B, Q, d))
     dfeats = _out(dfeats, (B, N, d), torch.bfloat16, feats, "dfeats")
@@ -310,7 +321,8 @@ def _gather_bwd(fn, queries, feats, coords, table, p, dOut, dfeats, dqueries, dp
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=feats.device)
     _call(fn, _ptr(queries), B, Q, _ptr(feats), _ptr(coords), N, d,
-          _ptr(table), H, W, K, _ptr(p), _ptr(dOut), _ptr(dfeats), _ptr(dqueries), _ptr(dp),
+          _ptr(table), H, W, K, _ptr(p), int(kind), _ptr(dOut), _ptr(dfeats), _ptr(dqueries),
+          _ptr(dp),
           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     return dfeats, dqueries, dp
 

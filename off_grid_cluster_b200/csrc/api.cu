@@ -69,11 +69,12 @@ void map_knn_workspace(acl::KnnArgs& a, uint8_t* ws, const acl::KnnWorkspace& L)
 // Validation and argument set-up shared by the two backward entry points.
 acl_status setup_gather_bwd(const float* queries, int B, int Q, const acl_bf16* feats,
                             const float* coords, int N, int d, const int32_t* table, int H, int W,
-                            int K, const float* p, const acl_bf16* dOut, acl_bf16* dfeats,
-                            float* dqueries, float* dp, void* workspace, size_t ws_bytes,
-                            acl::KnnArgs& a) {
+                            int K, const float* p, acl_knn_kernel kind, const acl_bf16* dOut,
+                            acl_bf16* dfeats, float* dqueries, float* dp, void* workspace,
+                            size_t ws_bytes, acl::KnnArgs& a) {
     acl_status st = check_gather(queries, B, Q, feats, coords, N, d, table, H, W, K, p);
     if (st != ACL_OK) return st;
+    if (kind != ACL_KNN_EXP && kind != ACL_KNN_INVPOW) return ACL_ERR_INVALID_ARG;
     if ((Q > 0 && (!dOut || !dqueries)) || !dfeats || !dp) return ACL_ERR_INVALID_ARG;
     if (!aligned(dOut, 16) || !aligned(dfeats, 16) || !aligned(dqueries, 8)) return ACL_ERR_INVALID_ARG;
     if (Q > ACL_MAX_GATHER_Q || N > ACL_MAX_TABLE_N) return ACL_ERR_UNSUPPORTED;
@@ -82,6 +83,7 @@ acl_status setup_gather_bwd(const float* queries, int B, int Q, const acl_bf16* 
     a.queries = queries; a.feats = BF(feats); a.xy = coords; a.table = table; a.p = p;
     a.B = B; a.Q = Q; a.N = N; a.d = d; a.GH = H; a.GW = W; a.K = K;
     a.dout = BF(dOut); a.dfeats = BFm(dfeats); a.dq = dqueries; a.dp = dp;
+    a.kind = static_cast<int>(kind);
     map_knn_workspace(a, static_cast<uint8_t*>(workspace), L);
     return ACL_OK;
 }
@@ -195,17 +197,27 @@ size_t acl_knn_gather_workspace(int B, int Q, int N, int d, int K) {
     return acl::knn_workspace_layout(B, Q, N, d, K).total;
 }
 
-acl_status acl_knn_gather_fwd(const float* queries, int B, int Q, const acl_bf16* feats,
-                              const float* coords, int N, int d, const int32_t* table, int H, int W,
-                              int K, const float* p, acl_bf16* out, acl_stream_t stream) {
+acl_status acl_knn_gather_fwd_ex(const float* queries, int B, int Q, const acl_bf16* feats,
+                                 const float* coords, int N, int d, const int32_t* table, int H,
+                                 int W, int K, const float* p, acl_knn_kernel kind, acl_bf16* out,
+                                 acl_stream_t stream) {
     acl_status st = check_gather(queries, B, Q, feats, coords, N, d, table, H, W, K, p);
     if (st != ACL_OK) return st;
+    if (kind != ACL_KNN_EXP && kind != ACL_KNN_INVPOW) return ACL_ERR_INVALID_ARG;
     if ((Q > 0 && !out) || !aligned(out, 16)) return ACL_ERR_INVALID_ARG;
     acl::KnnArgs a = {};
     a.queries = queries; a.feats = BF(feats); a.xy = coords; a.table = table; a.p = p;
     a.B = B; a.Q = Q; a.N = N; a.d = d; a.GH = H; a.GW = W; a.K = K;
+    a.kind = static_cast<int>(kind);
     a.out = BFm(out);
     return cuda_status(acl::launch_knn_fwd(a, S(stream)));
+}
+
+acl_status acl_knn_gather_fwd(const float* queries, int B, int Q, const acl_bf16* feats,
+                              const float* coords, int N, int d, const int32_t* table, int H, int W,
+                              int K, const float* p, acl_bf16* out, acl_stream_t stream) {
+    return acl_knn_gather_fwd_ex(queries, B, Q, feats, coords, N, d, table, H, W, K, p, ACL_KNN_EXP,
+                                 out, stream);
 }
 
 acl_status acl_knn_gather_index(const float* queries, int B, int Q, int N, int d,
@@ -227,16 +239,39 @@ acl_status acl_knn_gather_index(const float* queries, int B, int Q, int N, int d
     return cuda_status(acl::launch_knn_index(a, S(stream)));
 }
 
+acl_status acl_knn_gather_bwd_indexed_ex(const float* queries, int B, int Q,
+                                         const acl_bf16* feats, const float* coords, int N, int d,
+                                         const int32_t* table, int H, int W, int K, const float* p,
+                                         acl_knn_kernel kind, const acl_bf16* dOut,
+                                         acl_bf16* dfeats, float* dqueries, float* dp,
+                                         void* workspace, size_t ws_bytes, acl_stream_t stream) {
+    acl::KnnArgs a = {};
+    const acl_status st = setup_gather_bwd(queries, B, Q, feats, coords, N, d, table, H, W, K, p,
+                                           kind, dOut, dfeats, dqueries, dp, workspace, ws_bytes, a);
+    if (st != ACL_OK) return st;
+    return cuda_status(acl::launch_knn_bwd_indexed(a, S(stream)));
+}
+
 acl_status acl_knn_gather_bwd_indexed(const float* queries, int B, int Q, const acl_bf16* feats,
                                       const float* coords, int N, int d, const int32_t* table,
                                       int H, int W, int K, const float* p, const acl_bf16* dOut,
                                       acl_bf16* dfeats, float* dqueries, float* dp,
                                       void* workspace, size_t ws_bytes, acl_stream_t stream) {
+    return acl_knn_gather_bwd_indexed_ex(queries, B, Q, feats, coords, N, d, table, H, W, K, p,
+                                         ACL_KNN_EXP, dOut, dfeats, dqueries, dp, workspace,
+                                         ws_bytes, stream);
+}
+
+acl_status acl_knn_gather_bwd_ex(const float* queries, int B, int Q, const acl_bf16* feats,
+                                 const float* coords, int N, int d, const int32_t* table, int H,
+                                 int W, int K, const float* p, acl_knn_kernel kind,
+                                 const acl_bf16* dOut, acl_bf16* dfeats, float* dqueries, float* dp,
+                                 void* workspace, size_t ws_bytes, acl_stream_t stream) {
     acl::KnnArgs a = {};
     const acl_status st = setup_gather_bwd(queries, B, Q, feats, coords, N, d, table, H, W, K, p,
-                                           dOut, dfeats, dqueries, dp, workspace, ws_bytes, a);
+                                           kind, dOut, dfeats, dqueries, dp, workspace, ws_bytes, a);
     if (st != ACL_OK) return st;
-    return cuda_status(acl::launch_knn_bwd_indexed(a, S(stream)));
+    return cuda_status(acl::launch_knn_bwd(a, S(stream)));
 }
 
 acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16* feats,
@@ -244,11 +279,8 @@ acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16
                               int K, const float* p, const acl_bf16* dOut, acl_bf16* dfeats,
                               float* dqueries, float* dp, void* workspace, size_t ws_bytes,
                               acl_stream_t stream) {
-    acl::KnnArgs a = {};
-    const acl_status st = setup_gather_bwd(queries, B, Q, feats, coords, N, d, table, H, W, K, p,
-                                           dOut, dfeats, dqueries, dp, workspace, ws_bytes, a);
-    if (st != ACL_OK) return st;
-    return cuda_status(acl::launch_knn_bwd(a, S(stream)));
+    return acl_knn_gather_bwd_ex(queries, B, Q, feats, coords, N, d, table, H, W, K, p, ACL_KNN_EXP,
+                                 dOut, dfeats, dqueries, dp, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"

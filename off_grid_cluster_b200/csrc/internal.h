@@ -87,6 +87,7 @@ struct KnnArgs {
     const int32_t* table;
     const float* p;
     int B, Q, N, d, GH, GW, K;
+    int kind;           // 0: exponential kernel softmax(-p d); 1: inverse power d^-p / sum
     bf16* out;
     // backward
     const bf16* dout;

@@ -321,6 +321,22 @@ struct Nbrs {
     float d, x, y;
 };
 
+// The two weight kernels share one form: w_k = 2^(-p (v_k - v_min)) / sum, with
+// v = d log2(e) for the exponential kernel (exp(-p (d - d_min))) and v = log2(d) for the
+// inverse power ((d_min / d)^p).  A neighbour at v_min gets 1 (for the inverse power at
+// d_min = 0 that is the d -> 0 limit); p = 0 gives equal weights.
+__device__ __forceinline__ float knn_v(float d, int kind) { return kind ? log2f(d) : d * kLog2e; }
+__device__ __forceinline__ float knn_weight(float v, float vmin, float p) {
+    if (v == vmin || p == 0.f) return 1.f;
+    return exp2f(-p * (v - vmin));
+}
+// -dz/dp for z = -p d (d) or z = -p ln d (ln d; 0 at d = 0), from v
+__device__ __forceinline__ float knn_dzdp(float v) { return v == -INFINITY ? 0.f : v * kLn2; }
+// f with dz/dq = -p f (q - x): 1 / d or 1 / d^2, 0 at d = 0
+__device__ __forceinline__ float knn_dq_factor(float d, int kind) {
+    return d > 0.f ? (kind ? 1.f / (d * d) : 1.f / d) : 0.f;
+}
+
 // Lane-group prologue shared by the forward and the query side of the backward.
 template <int KT>
 __device__ __forceinline__ float load_neighbours(const KnnArgs& a, long long gq, float2 qp,
@@ -378,14 +394,17 @@ __global__ void __launch_bounds__(kGatherThreads) knn_fwd_kernel(const KnnArgs a
     if (gq >= total) return;  // no cross-lane communication below
     const float2 qp = reinterpret_cast<const float2*>(a.queries)[gq];
     Nbrs nb[KT];
-    const float dmin = load_neighbours<KT>(a, gq, qp, nb);
+    const float vmin = knn_v(load_neighbours<KT>(a, gq, qp, nb), a.kind);
+    float v[KT];
+#pragma unroll
+    for (int j = 0; j < KT; ++j) v[j] = knn_v(nb[j].d, a.kind);
     const int b = static_cast<int>(gq / a.Q);
     const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d;
 #pragma unroll
     for (int ch = 0; ch < CH; ++ch) {
         const int c0 = ch * LPQ * 8 + sub * 8;
         if (c0 >= a.d) break;
-        const float ph = a.p[c0 >> 5] * kLog2e;
+        const float ph = a.p[c0 >> 5];
         uint4 f[KT];
 #pragma unroll
         for (int j = 0; j < KT; ++j)
@@ -395,7 +414,7 @@ __global__ void __launch_bounds__(kGatherThreads) knn_fwd_kernel(const KnnArgs a
         float sum = 0.f;
 #pragma unroll
         for (int j = 0; j < KT; ++j) {
-            const float w = (nb[j].t >= 0) ? exp2f(-ph * (nb[j].d - dmin)) : 0.f;
+            const float w = (nb[j].t >= 0) ? knn_weight(v[j], vmin, ph) : 0.f;
             sum += w;
             fma8(acc, w, f[j]);
         }
@@ -434,6 +453,10 @@ __global__ void __launch_bounds__(kGatherThreads) knn_bwd_query_kernel(const Knn
         }
     }
     const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d;
+    const float vmin = knn_v(dmin, a.kind);
+    float v[KT];
+#pragma unroll
+    for (int j = 0; j < KT; ++j) v[j] = knn_v(nb[j].d, a.kind);
     float dqx = 0.f, dqy = 0.f;
 #pragma unroll
     for (int ch = 0; ch < CH; ++ch) {
@@ -456,11 +479,11 @@ __global__ void __launch_bounds__(kGatherThreads) knn_bwd_query_kernel(const Knn
         float sum = 0.f;
 #pragma unroll
         for (int j = 0; j < KT; ++j) {
-            const bool v = on && nb[j].t >= 0;
-            w[j] = v ? exp2f(-ph * kLog2e * (nb[j].d - dmin)) : 0.f;
+            const bool ok = on && nb[j].t >= 0;
+            w[j] = ok ? knn_weight(v[j], vmin, ph) : 0.f;
             sum += w[j];
-            const uint4 f = v ? ldg16(fb + static_cast<size_t>(nb[j].t) * a.d + c0)
-                              : make_uint4(0u, 0u, 0u, 0u);
+            const uint4 f = ok ? ldg16(fb + static_cast<size_t>(nb[j].t) * a.d + c0)
+                               : make_uint4(0u, 0u, 0u, 0u);
             const uint32_t u[4] = {f.x, f.y, f.z, f.w};
             float acc = 0.f;
 #pragma unroll
@@ -484,12 +507,10 @@ __global__ void __launch_bounds__(kGatherThreads) knn_bwd_query_kernel(const Knn
                 if (j < a.K) wout[j * NH] = w[j];
                 if (nb[j].t < 0) continue;
                 const float ds = w[j] * (dw[j] - sdw);
-                dph -= ds * nb[j].d;
-                if (nb[j].d > 0.f) {
-                    const float cf = -ds * ph / nb[j].d;
-                    dqx += cf * (qp.x - nb[j].x);
-                    dqy += cf * (qp.y - nb[j].y);
-                }
+                dph -= ds * knn_dzdp(v[j]);
+                const float cf = -ds * ph * knn_dq_factor(nb[j].d, a.kind);
+                dqx += cf * (qp.x - nb[j].x);
+                dqy += cf * (qp.y - nb[j].y);
             }
             sdp[(warp * QPW + grp) * NH + hh] = dph;
         }
@@ -515,14 +536,14 @@ __global__ void __launch_bounds__(kGatherThreads) knn_bwd_query_kernel(const Knn
 // of their tokens) run on one SM and find each other's feature rows in L1.
 struct GroupNbrs {
     int t;
-    float d, ux, uy;  // id, distance, unit vector (q - p) / d (0 when d == 0)
+    float v, ux, uy;  // id, weight exponent knn_v(d), (q - p) * knn_dq_factor(d)
 };
 
 template <int KT>
 __device__ __forceinline__ float group_neighbours(const KnnArgs& a, long long gq, bool live, float2 qp,
                                                   int sub, int LPQ, GroupNbrs (&nb)[KT]) {
     int t = -1;
-    float d = INFINITY, ux = 0.f, uy = 0.f;
+    float v = INFINITY, ux = 0.f, uy = 0.f;
     if (live && sub < a.K) {
         const int b = static_cast<int>(gq / a.Q);
         const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
@@ -531,23 +552,48 @@ __device__ __forceinline__ float group_neighbours(const KnnArgs& a, long long gq
         if (t >= 0) {
             const float2 p = reinterpret_cast<const float2*>(a.xy)[static_cast<size_t>(b) * a.N + t];
             const float dx = qp.x - p.x, dy = qp.y - p.y;
-            d = sqrtf(dx * dx + dy * dy);
-            if (d > 0.f) {
-                ux = dx / d;
-                uy = dy / d;
-            }
+            const float d = sqrtf(dx * dx + dy * dy);
+            v = knn_v(d, a.kind);
+            const float f = knn_dq_factor(d, a.kind);
+            ux = dx * f;
+            uy = dy * f;
         }
     }
-    float dmin = d;
-    for (int o = 1; o < LPQ; o <<= 1) dmin = fminf(dmin, __shfl_xor_sync(0xffffffffu, dmin, o, LPQ));
+    float vmin = v;
+    for (int o = 1; o < LPQ; o <<= 1) vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o, LPQ));
 #pragma unroll
     for (int j = 0; j < KT; ++j) {
         nb[j].t = __shfl_sync(0xffffffffu, t, j, LPQ);
-        nb[j].d = __shfl_sync(0xffffffffu, d, j, LPQ);
+        nb[j].v = __shfl_sync(0xffffffffu, v, j, LPQ);
         nb[j].ux = __shfl_sync(0xffffffffu, ux, j, LPQ);
         nb[j].uy = __shfl_sync(0xffffffffu, uy, j, LPQ);
     }
-    return dmin;
+    return vmin;
+}
+
+// The neighbour that lane sub (< K) of a query's lane group owns: token id, weight
+// exponent v = knn_v(d), and (q - p) * knn_dq_factor(d); returns the group's minimum v.
+__device__ __forceinline__ float own_neighbour(const KnnArgs& a, long long gq, bool live, float2 qp,
+                                               int sub, int LPQ, int& t, float& v, float& ux,
+                                               float& uy) {
+    if (live && sub < a.K) {
+        const int b = static_cast<int>(gq / a.Q);
+        const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
+        t = a.table[((static_cast<size_t>(b) * a.GH + cy) * a.GW + cx) * a.K + sub];
+        if (t >= a.N) t = -1;
+        if (t >= 0) {
+            const float2 p = reinterpret_cast<const float2*>(a.xy)[static_cast<size_t>(b) * a.N + t];
+            const float dx = qp.x - p.x, dy = qp.y - p.y;
+            const float d = sqrtf(dx * dx + dy * dy);
+            v = knn_v(d, a.kind);
+            const float f = knn_dq_factor(d, a.kind);
+            ux = dx * f;
+            uy = dy * f;
+        }
+    }
+    float vmin = v;
+    for (int o = 1; o < LPQ; o <<= 1) vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o, LPQ));
+    return vmin;
 }
 
 template <int KT, int CH>
@@ -563,7 +609,7 @@ __global__ void __launch_bounds__(kGatherThreads)
         const bool live = gq < total;
         const float2 qp = live ? reinterpret_cast<const float2*>(a.queries)[gq] : make_float2(0.f, 0.f);
         GroupNbrs nb[KT];
-        const float dmin = group_neighbours<KT>(a, gq, live, qp, sub, LPQ, nb);
+        const float vmin = group_neighbours<KT>(a, gq, live, qp, sub, LPQ, nb);
         if (!live) continue;
         const int b = static_cast<int>(gq / a.Q);
         const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d;
@@ -571,7 +617,7 @@ __global__ void __launch_bounds__(kGatherThreads)
         for (int ch = 0; ch < CH; ++ch) {
             const int c0 = ch * LPQ * 8 + sub * 8;
             if (c0 >= a.d) break;
-            const float ph = a.p[c0 >> 5] * kLog2e;
+            const float ph = a.p[c0 >> 5];
             uint4 f[KT];
 #pragma unroll
             for (int j = 0; j < KT; ++j)
@@ -581,7 +627,7 @@ __global__ void __launch_bounds__(kGatherThreads)
             float sum = 0.f;
 #pragma unroll
             for (int j = 0; j < KT; ++j) {
-                const float w = (nb[j].t >= 0) ? exp2f(-ph * (nb[j].d - dmin)) : 0.f;
+                const float w = (nb[j].t >= 0) ? knn_weight(nb[j].v, vmin, ph) : 0.f;
                 sum += w;
                 fma8(acc, w, f[j]);
             }
@@ -592,7 +638,7 @@ __global__ void __launch_bounds__(kGatherThreads)
 }
 
 template <int KT, int CH>
-__global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 3 : 1)
+__global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 4 : 2)
     knn_bwd_query_shared_kernel(const KnnArgs a, int lpq_log2, int iters) {
     extern __shared__ __align__(16) float sdp[];  // [warps][groups][heads]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -608,10 +654,17 @@ __global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 3 : 1)
         if ((gq - grp) >= total) break;  // uniform per warp
         const bool live = gq < total;
         const float2 qp = live ? reinterpret_cast<const float2*>(a.queries)[gq] : make_float2(0.f, 0.f);
-        GroupNbrs nb[KT];
-        const float dmin = group_neighbours<KT>(a, gq, live, qp, sub, LPQ, nb);
+        // lane j < K of the group owns neighbour j; every lane gets all K token ids
+        int my_t = -1;
+        float my_v = INFINITY, my_ux = 0.f, my_uy = 0.f;
+        const float vmin = own_neighbour(a, gq, live, qp, sub, LPQ, my_t, my_v, my_ux, my_uy);
+        int tk[KT];
+#pragma unroll
+        for (int j = 0; j < KT; ++j) tk[j] = __shfl_sync(0xffffffffu, my_t, j, LPQ);
         const int b = live ? static_cast<int>(gq / a.Q) : 0;
         const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d;
+        const int r = sub & 3;  // lane within the 4 lanes of a head
+        constexpr int KQ = KT / 4;  // neighbours per lane after the reduce-scatter: j = r + 4 u
         float dqx = 0.f, dqy = 0.f;
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch) {
@@ -630,47 +683,77 @@ __global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 3 : 1)
                     g[2 * i + 1] = bf16_hi(u[i]);
                 }
             }
-            uint4 f[KT];
+            // this lane's 8-channel share of dw_j = <dOut_h, f_j,h> for every neighbour
+            float dwp[KT];
+            {
+                uint4 f[KT];
 #pragma unroll
-            for (int j = 0; j < KT; ++j)
-                f[j] = (on && nb[j].t >= 0) ? ldg16(fb + static_cast<size_t>(nb[j].t) * a.d + c0)
-                                            : make_uint4(0u, 0u, 0u, 0u);
-            float w[KT], dw[KT];
+                for (int j = 0; j < KT; ++j)
+                    f[j] = (on && tk[j] >= 0) ? ldg16(fb + static_cast<size_t>(tk[j]) * a.d + c0)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int j = 0; j < KT; ++j) {
+                    const uint32_t u[4] = {f[j].x, f[j].y, f[j].z, f[j].w};
+                    float acc = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc += g[2 * i] * bf16_lo(u[i]) + g[2 * i + 1] * bf16_hi(u[i]);
+                    dwp[j] = acc;
+                }
+            }
+            // reduce-scatter over the head's 4 lanes: after the xor-2 step a lane holds the
+            // j whose bit 1 matches bit 1 of r, after the xor-1 step the j = r + 4 u
+            float dh[KT / 2];
+#pragma unroll
+            for (int s2 = 0; s2 < KT / 2; ++s2) {
+                const int jlo = (s2 & 1) | ((s2 >> 1) << 2), jhi = jlo | 2;
+                const float send = (r & 2) ? dwp[jlo] : dwp[jhi];
+                const float keep = (r & 2) ? dwp[jhi] : dwp[jlo];
+                dh[s2] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+            }
+            float dw[KQ], w[KQ], vj[KQ], uxj[KQ], uyj[KQ];
+            bool okj[KQ];
             float sum = 0.f;
 #pragma unroll
-            for (int j = 0; j < KT; ++j) {
-                w[j] = (on && nb[j].t >= 0) ? exp2f(-ph * kLog2e * (nb[j].d - dmin)) : 0.f;
-                sum += w[j];
-                const uint32_t u[4] = {f[j].x, f[j].y, f[j].z, f[j].w};
-                float acc = 0.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc += g[2 * i] * bf16_lo(u[i]) + g[2 * i + 1] * bf16_hi(u[i]);
-                dw[j] = acc;
+            for (int u = 0; u < KQ; ++u) {
+                const float send = (r & 1) ? dh[2 * u] : dh[2 * u + 1];
+                const float keep = (r & 1) ? dh[2 * u + 1] : dh[2 * u];
+                dw[u] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                const int j = r + 4 * u;
+                const int t = __shfl_sync(0xffffffffu, my_t, j, LPQ);
+                vj[u] = __shfl_sync(0xffffffffu, my_v, j, LPQ);
+                uxj[u] = __shfl_sync(0xffffffffu, my_ux, j, LPQ);
+                uyj[u] = __shfl_sync(0xffffffffu, my_uy, j, LPQ);
+                okj[u] = on && j < a.K && t >= 0;
+                w[u] = okj[u] ? knn_weight(vj[u], vmin, ph) : 0.f;
+                sum += w[u];
             }
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
             const float inv = sum > 0.f ? 1.f / sum : 0.f;
             float sdw = 0.f;
 #pragma unroll
-            for (int j = 0; j < KT; ++j) {
-                dw[j] += __shfl_xor_sync(0xffffffffu, dw[j], 1);
-                dw[j] += __shfl_xor_sync(0xffffffffu, dw[j], 2);
-                w[j] *= inv;
-                sdw += w[j] * dw[j];
+            for (int u = 0; u < KQ; ++u) {
+                w[u] *= inv;
+                sdw += w[u] * dw[u];
             }
-            if (on && (sub & 3) == 0) {
-                float dph = 0.f;
-                float* wout = a.w + static_cast<size_t>(gq) * a.K * NH + hh;
+            sdw += __shfl_xor_sync(0xffffffffu, sdw, 1);
+            sdw += __shfl_xor_sync(0xffffffffu, sdw, 2);
+            float dph = 0.f;
+            float* wout = a.w + static_cast<size_t>(gq) * a.K * NH + hh;
 #pragma unroll
-                for (int j = 0; j < KT; ++j) {
-                    if (j < a.K) wout[j * NH] = w[j];
-                    if (nb[j].t < 0) continue;
-                    const float ds = w[j] * (dw[j] - sdw);
-                    dph -= ds * nb[j].d;
-                    const float cf = -ds * ph;
-                    dqx += cf * nb[j].ux;
-                    dqy += cf * nb[j].uy;
-                }
-                sdp[(warp * QPW + grp) * NH + hh] += dph;
+            for (int u = 0; u < KQ; ++u) {
+                const int j = r + 4 * u;
+                if (on && j < a.K) wout[j * NH] = w[u];
+                if (!okj[u]) continue;
+                const float ds = w[u] * (dw[u] - sdw);
+                dph -= ds * knn_dzdp(vj[u]);
+                const float cf = -ds * ph;
+                dqx += cf * uxj[u];
+                dqy += cf * uyj[u];
             }
+            dph += __shfl_xor_sync(0xffffffffu, dph, 1);
+            dph += __shfl_xor_sync(0xffffffffu, dph, 2);
+            if (on && r == 0) sdp[(warp * QPW + grp) * NH + hh] += dph;
         }
         for (int o = 1; o < LPQ; o <<= 1) {
             dqx += __shfl_xor_sync(0xffffffffu, dqx, o);
@@ -1209,8 +1292,9 @@ struct GatherPlan {
     bool shared;  // lane j of a query group owns neighbour j (needs K <= lanes per query)
 };
 // Launch shape of the query-side gather kernels.  A CTA walks `iters` consecutive blocks of
-// queries; iters is chosen so the grid fits one wave of the kernel's resident CTAs (the
-// backward's query pass holds fewer CTAs per SM than the forward: more registers).
+// queries; iters is chosen so the grid fits one wave of the kernel's resident CTAs (4 per
+// SM; 2 for the backward's query pass with K > 8 or more than one channel pass, which
+// needs up to 128 registers).
 GatherPlan gather_plan(int B, int Q, int d, int K, bool bwd) {
     GatherPlan g;
     g.l2 = lpq_log2_for(d);
@@ -1219,7 +1303,7 @@ GatherPlan gather_plan(int B, int Q, int d, int K, bool bwd) {
     g.shared = K <= lanes;
     const long long per_iter = static_cast<long long>(kGatherWarps) * (32 >> g.l2);
     const long long total = static_cast<long long>(B) * Q;
-    const int resident = bwd ? ((K <= 8 && g.ch == 1) ? 3 : 2) : 4;
+    const int resident = bwd ? ((K <= 8 && g.ch == 1) ? 4 : 2) : 4;
     long long it = 1;
     if (g.shared) {
         it = (total + per_iter * 148 * resident - 1) / (per_iter * 148 * resident);

@@ -119,6 +119,13 @@ def test_knn_validation():
     assert bwd(Q=70000, wsb=1 << 40) == UNSUPPORTED
     bwdi = lambda Q=10, wsb=ws: L.acl_knn_gather_bwd_indexed(P, 1, Q, P, P, 100, 128, P, 64, 64,
                                                              8, P, P, P, P, P, P, wsb, None)
+    assert L.acl_knn_gather_fwd_ex(P, 1, 10, P, P, 100, 128, P, 64, 64, 8, P, 2, P, None) == INVALID
+    assert L.acl_knn_gather_bwd_ex(P, 1, 10, P, P, 100, 128, P, 64, 64, 8, P, -1, P, P, P, P,
+                                   P, ws, None) == INVALID
+    assert L.acl_knn_gather_bwd_indexed_ex(P, 1, 10, P, P, 100, 128, P, 64, 64, 8, P, 7, P, P,
+                                           P, P, P, ws, None) == INVALID
+    assert L.acl_knn_gather_bwd_ex(P, 1, 10, P, P, 100, 128, P, 64, 64, 8, P, 1, P, P, P, P,
+                                   P, 16, None) == WORKSPACE
     assert bwdi(wsb=16) == WORKSPACE
     assert bwdi(Q=70000, wsb=1 << 40) == UNSUPPORTED
     idx = lambda Q=10, d=128, K=8, q=P, t=P, wsb=ws, w=P: L.acl_knn_gather_index(

@@ -18,15 +18,16 @@ def table_both(xy: np.ndarray, GH: int, GW: int, K: int) -> np.ndarray:
     return ref
 
 
-def gather_both(kb: synth.KnnBatch, bwd: bool = True):
+def gather_both(kb: synth.KnnBatch, bwd: bool = True, kind: int = acl.ACL_KNN_EXP):
     table = table_both(kb.coords, kb.GH, kb.GW, kb.K)
-    out_ref = oracle.knn_fwd(kb.queries, kb.feats, kb.coords, table, kb.p)
+    out_ref = oracle.knn_fwd(kb.queries, kb.feats, kb.coords, table, kb.p, kind=kind)
     q, f, xy, tt, p = dev(kb.queries), bf16(kb.feats), dev(kb.coords), dev(table), dev(kb.p)
-    out = acl.acl_knn_gather_fwd(q, f, xy, tt, p)
+    out = acl.acl_knn_gather_fwd(q, f, xy, tt, p, kind=kind)
     stats = check_fwd(host(out), out_ref, "out")
     if bwd:
-        dF_r, dq_r, dp_r = oracle.knn_bwd(kb.queries, kb.feats, kb.coords, table, kb.p, kb.dout)
-        dF, dq, dp = acl.acl_knn_gather_bwd(q, f, xy, tt, p, bf16(kb.dout))
+        dF_r, dq_r, dp_r = oracle.knn_bwd(kb.queries, kb.feats, kb.coords, table, kb.p, kb.dout,
+                                          kind=kind)
+        dF, dq, dp = acl.acl_knn_gather_bwd(q, f, xy, tt, p, bf16(kb.dout), kind=kind)
         stats["dF"] = check_grad(host(dF), dF_r, "dfeats")
         stats["dq"] = check_grad(host(dq), dq_r, "dqueries")
         stats["dp"] = check_grad(host(dp), dp_r, "dp")
@@ -134,5 +135,50 @@ def test_staged_backward_matches_one_call():
     acl.acl_knn_gather_index(q, table, kb.N, kb.d, ws, stream=side)
     torch.cuda.current_stream().wait_stream(side)
     r2 = acl.acl_knn_gather_bwd_indexed(q, f, xy, table, p, g, ws)
+    for x, y in zip(r1, r2):
+        assert torch.equal(x, y)
+
+
+# ------------------------------------------------------------------ inverse-power kernel
+
+INV = acl.ACL_KNN_INVPOW
+
+
+def test_invpow_step_workload():
+    gather_both(synth.step_batch(B=2).knn, kind=INV)
+
+
+@pytest.mark.parametrize("stage", [0, 3])
+def test_invpow_decoder_stage(stage):
+    gather_both(synth.knn_decoder(B=16)[stage], kind=INV)
+
+
+@pytest.mark.parametrize("d,K", [(32, 8), (96, 8), (160, 16), (288, 3)])
+def test_invpow_shapes(d, K):
+    xy = synth.sweep_coords(B=2)[1]
+    gather_both(synth.knn_batch(xy, d, K=K), kind=INV)
+
+
+def test_invpow_queries_on_tokens_and_temperature_limits():
+    xy = synth.sweep_coords(B=1)[1]
+    kb = synth.knn_batch(xy, 128)
+    kb.queries[:, :300] = kb.coords[:, :300]            # d_min = 0: the d -> 0 limit
+    gather_both(kb, kind=INV)
+    kb.p = np.zeros_like(kb.p)                           # plain mean
+    gather_both(kb, kind=INV)
+    kb.p = np.full_like(kb.p, 40.0)                      # near one-hot
+    gather_both(kb, bwd=False, kind=INV)
+
+
+def test_invpow_staged_backward_matches_one_call():
+    kb = synth.step_batch(B=2).knn
+    xy = dev(kb.coords)
+    table = acl.acl_knn_table(xy)
+    q, f, p, g = dev(kb.queries), bf16(kb.feats), dev(kb.p), bf16(kb.dout)
+    r1 = acl.acl_knn_gather_bwd(q, f, xy, table, p, g, kind=INV)
+    ws = torch.empty((acl.acl_knn_gather_workspace(2, kb.Q, kb.N, kb.d, 8),), dtype=torch.uint8,
+                     device="cuda")
+    acl.acl_knn_gather_index(q, table, kb.N, kb.d, ws)
+    r2 = acl.acl_knn_gather_bwd_indexed(q, f, xy, table, p, g, ws, kind=INV)
     for x, y in zip(r1, r2):
         assert torch.equal(x, y)

@@ -50,7 +50,7 @@ TAG_Q, TAG_K, TAG_V, TAG_DO = 10, 11, 12, 13
 TAG_QUERY, TAG_FEAT, TAG_P, TAG_DOUT = 20, 21, 22, 23
 
 WORKLOAD_ID = {"tiny": 1, "stage1": 2, "stage3": 3, "sweep": 4, "decoder": 5,
-               "step": 6}
+               "step": 6, "hires": 7}
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -359,3 +359,13 @@ def step_batch(B: int = 8, image0: int = 0) -> StepBatch:
     a = attn_stage1(B, image0)
     kb = knn_batch(a.coords, 128, image0, 0, wid=WORKLOAD_ID["step"])
     return StepBatch(a, kb, {"workload": "stage1-1024px+decoder-gather", "B": B})
+
+
+def hires_batch(B: int = 2, image0: int = 0, grid: int = 128, keep: int | None = None,
+                d: int = 128) -> KnnBatch:
+    """Decoder gather at high resolution: a grid x grid patch grid (128 x 128 = a 2048 px image
+    at 16 px patches), the value-noise mask keeping half the cells, one query per cell."""
+    wid = WORKLOAD_ID["hires"]
+    keep = grid * grid // 2 if keep is None else keep
+    xy = np.stack([stage1_coords(wid, i, grid, grid, keep) for i in range(image0, image0 + B)])
+    return knn_batch(xy, d, image0, 0, wid=wid, gh=grid, gw=grid)

@@ -30,7 +30,7 @@ def lib():
         L = ct.CDLL(so)
         for name in ("orc_cluster_batch", "orc_neighbors_batch", "orc_attn_fwd_batch",
                      "orc_attn_bwd_batch", "orc_knn_table_batch", "orc_knn_fwd_batch",
-                     "orc_knn_bwd_batch", "orc_set_threads"):
+                     "orc_knn_bwd_batch", "orc_set_threads", "orc_token_order_batch"):
             getattr(L, name).restype = ct.c_int
         _lib = L
     return _lib
@@ -143,3 +143,12 @@ def knn_bwd(queries, feats, xy, table, p, dout, kind=KNN_EXP):
                                    _p(dp)),
            "knn_bwd")
     return dF, dq, dp
+
+
+def token_order(xy, GH, GW):
+    """Token ids of each image in Z-order of their cells on the GH x GW grid -> [B, N] int32."""
+    xy = _f32(xy)
+    B, N = xy.shape[:2]
+    perm = np.empty((B, N), dtype=np.int32)
+    _check(lib().orc_token_order_batch(_p(xy), B, N, GH, GW, _p(perm)), "token_order")
+    return perm

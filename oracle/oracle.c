@@ -527,6 +527,41 @@ int orc_knn_bwd(const float* queries, int Q, const double* feats, const float* x
     return 0;
 }
 
+/*
+ * Space-filling token order (AFFMAE notes, "Limitations": the dense lookup table and the
+ * gathers are bandwidth-bound, and space-filling curves are suggested to keep neighbouring
+ * tokens close in memory).  Each token's cell on the H x W grid (quantised as the gather
+ * quantises a query) gets its Z-order (Morton) code: bit i of the column goes to bit 2i,
+ * bit i of the row to bit 2i + 1.  perm lists the token ids by (code, id) ascending.
+ */
+static uint32_t morton_code(uint32_t r, uint32_t c) {
+    uint32_t code = 0;
+    for (int i = 0; i < 16; ++i) {
+        code |= ((c >> i) & 1u) << (2 * i);
+        code |= ((r >> i) & 1u) << (2 * i + 1);
+    }
+    return code;
+}
+
+static int cmp_u64(const void* pa, const void* pb) {
+    uint64_t a = *(const uint64_t*)pa, b = *(const uint64_t*)pb;
+    return (a > b) - (a < b);
+}
+
+int orc_token_order(const float* xy, int N, int GH, int GW, int32_t* perm) {
+    if (N < 1 || GH < 1 || GW < 1 || GH > 65536 || GW > 65536) return 1;
+    uint64_t* key = (uint64_t*)malloc(sizeof(uint64_t) * (size_t)N);
+    if (!key) return 2;
+    for (int t = 0; t < N; ++t) {
+        uint32_t r = (uint32_t)quantise(xy[2 * t + 1], GH), c = (uint32_t)quantise(xy[2 * t], GW);
+        key[t] = ((uint64_t)morton_code(r, c) << 32) | (uint32_t)t;
+    }
+    qsort(key, (size_t)N, sizeof(uint64_t), cmp_u64);
+    for (int i = 0; i < N; ++i) perm[i] = (int32_t)(key[i] & 0xffffffffu);
+    free(key);
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* batch drivers: images are independent; OpenMP over images only            */
 /* ------------------------------------------------------------------------ */
@@ -628,5 +663,13 @@ int orc_knn_bwd_batch(const float* queries, int B, int Q, const double* feats,
         dp[h] = acc;
     }
     free(part);
+    return rc;
+}
+
+int orc_token_order_batch(const float* xy, int B, int N, int GH, int GW, int32_t* perm) {
+    int rc = 0;
+    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    for (int b = 0; b < B; ++b)
+        rc |= orc_token_order(xy + (size_t)b * N * 2, N, GH, GW, perm + (size_t)b * N);
     return rc;
 }

@@ -31,6 +31,9 @@ int orc_knn_bwd(const float* queries, int Q, const double* feats, const float* x
                 const double* p, int kind, const double* dout, double* dfeats, double* dq,
                 double* dp);
 
+/* token ids in Z-order of their cells on the GH x GW grid, ties by id */
+int orc_token_order(const float* xy, int N, int GH, int GW, int32_t* perm);
+
 int orc_cluster_batch(const float* xy, int B, int N, int C, int32_t* clusters);
 int orc_neighbors_batch(const float* xy, const int32_t* clusters, int B, int N, int C,
                         int M, int32_t* nbr);
@@ -50,4 +53,5 @@ int orc_knn_bwd_batch(const float* queries, int B, int Q, const double* feats,
                       const float* xy, int N, int d, const int32_t* table, int GH, int GW,
                       int K, const double* p, int kind, const double* dout, double* dfeats,
                       double* dq, double* dp);
+int orc_token_order_batch(const float* xy, int B, int N, int GH, int GW, int32_t* perm);
 #endif

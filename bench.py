@@ -456,6 +456,7 @@ def run_gpu(args, rank: int, world: int):
             e1.record(stream)
             e1.synchronize()
             inv_us[name] = round(e0.elapsed_time(e1) / 20 * 1e3, 2)
+    hires = hires_gather_times(torch, acl, synth, device, stream) if world == 1 else None
     # keep the same load on the GPU until the clock sampler has several samples
     t_wall = time.time()
     it = 0
@@ -526,6 +527,7 @@ def run_gpu(args, rank: int, world: int):
                                        for j, n in enumerate(OPS)},
             "knn_invpow_us": {**inv_us, "note": "inverse-power weight kernel (d^-p), same "
                               "gathers, set 0, L2-warm (one set): compare with per_call"},
+            "hires_gather_us": hires,
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -548,6 +550,50 @@ def run_gpu(args, rank: int, world: int):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def hires_gather_times(torch, acl, synth, device, stream, B: int = 4, reps: int = 10) -> dict:
+    """Decoder gather at 128 x 128 cells (4 images, 8192 tokens, 16384 queries, d = 128):
+    Z-order token order, then table + gather fwd + bwd in raster and in Z-order, one call at a
+    time with CUDA events."""
+    kb = synth.hires_batch(B=B)
+    T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
+    xy, f = T(kb.coords), T(kb.feats, torch.bfloat16)
+    q, p, g = T(kb.queries), T(kb.p), T(kb.dout, torch.bfloat16)
+    ws = torch.empty((acl.acl_knn_gather_workspace(B, kb.Q, kb.N, kb.d, 8),), dtype=torch.uint8,
+                     device=device)
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+        e1.synchronize()
+        return round(e0.elapsed_time(e1) / reps * 1e3, 2)
+
+    res = {"workload": f"{B} images, 128x128 cells, {kb.N} tokens, {kb.Q} queries, d = {kb.d}, K = 8"}
+    perm = acl.acl_token_order(xy, 128, 128, stream=stream)
+    res["token_order"] = timed(lambda: acl.acl_token_order(xy, 128, 128, perm=perm, stream=stream))
+    torch.cuda.synchronize()
+    bidx = torch.arange(B, device=device)[:, None]
+    pl = perm.long()
+    variants = {"raster": (xy, f), "z_order": (xy[bidx, pl].contiguous(), f[bidx, pl].contiguous())}
+    for name, (xv, fv) in variants.items():
+        table = acl.acl_knn_table(xv, 128, 128, 8, stream=stream)
+        out = acl.acl_knn_gather_fwd(q, fv, xv, table, p, stream=stream)
+        dF, dq, dp = acl.acl_knn_gather_bwd(q, fv, xv, table, p, g, workspace=ws, stream=stream)
+        res[name] = {
+            "knn_table": timed(lambda: acl.acl_knn_table(xv, 128, 128, 8, table=table, stream=stream)),
+            "knn_fwd": timed(lambda: acl.acl_knn_gather_fwd(q, fv, xv, table, p, out=out,
+                                                            stream=stream)),
+            "knn_bwd": timed(lambda: acl.acl_knn_gather_bwd(q, fv, xv, table, p, g, dF, dq, dp,
+                                                            workspace=ws, stream=stream)),
+        }
+    return res
 
 
 def run_e2e(args, s: StepSet, stream, streams, torch, acl, tokens_per_step: int, sb=None,

@@ -220,6 +220,22 @@ acl_status acl_cluster_attn_bwd_noalloc(const acl_bf16* Q, const acl_bf16* K, co
 acl_status acl_knn_table(const float* coords, int B, int N, int H, int W, int K,
                          int32_t* table, acl_stream_t stream);
 
+/*
+ * acl_token_order -- space-filling (Z-order) token order.  Passage: AFF notes,
+ * "Limitations" (the lookup table and the gathers are bound by memory traffic; space-filling
+ * curves are suggested so that tokens close on the image are close in memory).
+ *   cell(t) = (clamp(floor(y_t), 0, H-1), clamp(floor(x_t), 0, W-1)) as for a query;
+ *   code(t) = Morton code of the cell: column bit i at bit 2i, row bit i at bit 2i + 1;
+ *   perm[b][i] = the id of the i-th token by (code, id) ascending.
+ * Permuting a stage's tokens (coordinates, features) by perm before the table and the
+ * gathers puts every aligned 2^k x 2^k block of cells in one contiguous run of tokens.
+ * coords [B][N][2] fp32 (8-byte aligned); perm [B][N] int32 out (a permutation of 0..N-1).
+ * Bit-exact (integer keys only).  Limits: 1 <= N <= ACL_MAX_TABLE_N, 1 <= H, W <= 4096,
+ * B <= 65535.
+ */
+acl_status acl_token_order(const float* coords, int B, int N, int H, int W, int32_t* perm,
+                           acl_stream_t stream);
+
 /* Workspace bytes acl_knn_gather_bwd (and acl_knn_gather_index +
  * acl_knn_gather_bwd_indexed) need for these sizes (0 on bad sizes). */
 size_t acl_knn_gather_workspace(int B, int Q, int N, int d, int K);

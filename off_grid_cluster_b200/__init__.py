@@ -40,6 +40,7 @@ SIGNATURES = {
     "acl_cluster_attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                           _F, _P, _P, _P, _P, _P, _P, _P, _P]),
     "acl_knn_table": (_I, [_P, _I, _I, _I, _I, _I, _P, _P]),
+    "acl_token_order": (_I, [_P, _I, _I, _I, _I, _P, _P]),
     "acl_knn_gather_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "acl_knn_gather_fwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P]),
     "acl_knn_gather_bwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P,
@@ -250,6 +251,16 @@ def acl_knn_table(coords: torch.Tensor, H: int = 64, W: int = 64, K: int = 8,
     table = _out(table, (B, H, W, K), torch.int32, coords, "table")
     _call("acl_knn_table", _ptr(coords), B, N, H, W, K, _ptr(table), _stream(stream))
     return table
+
+
+def acl_token_order(coords: torch.Tensor, H: int, W: int, perm: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """Token ids of each image in Z-order of their cells on the H x W grid -> [B,N] int32."""
+    _need(coords, "coords", torch.float32)
+    B, N = coords.shape[:2]
+    perm = _out(perm, (B, N), torch.int32, coords, "perm")
+    _call("acl_token_order", _ptr(coords), B, N, H, W, _ptr(perm), _stream(stream))
+    return perm
 
 
 def acl_knn_gather_workspace(B: int, Q: int, N: int, d: int, K: int = 8) -> int:

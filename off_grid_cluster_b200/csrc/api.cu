@@ -192,6 +192,16 @@ acl_status acl_knn_table(const float* coords, int B, int N, int H, int W, int K,
     return cuda_status(acl::launch_knn_table(coords, B, N, H, W, K, table, S(stream)));
 }
 
+acl_status acl_token_order(const float* coords, int B, int N, int H, int W, int32_t* perm,
+                           acl_stream_t stream) {
+    if (!coords || !perm) return ACL_ERR_INVALID_ARG;
+    if (B < 1 || N < 1 || H < 1 || W < 1) return ACL_ERR_INVALID_ARG;
+    if (N > ACL_MAX_TABLE_N || H > 4096 || W > 4096 || B > 65535) return ACL_ERR_UNSUPPORTED;
+    if (acl::token_order_smem_bytes(N) > kMaxSmem) return ACL_ERR_UNSUPPORTED;
+    if (!aligned(coords, 8)) return ACL_ERR_INVALID_ARG;
+    return cuda_status(acl::launch_token_order(coords, B, N, H, W, perm, S(stream)));
+}
+
 size_t acl_knn_gather_workspace(int B, int Q, int N, int d, int K) {
     if (B < 1 || Q < 0 || N < 1 || d < 32 || d % 32 != 0 || K < 1) return 0;
     return acl::knn_workspace_layout(B, Q, N, d, K).total;

@@ -100,4 +100,13 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Grid cell of a coordinate on an axis of n cells: clamp(floor(v), 0, n - 1); a value that
+// is not >= 0 (negative or NaN) maps to 0.  Used for queries (gather) and tokens (order).
+__device__ __forceinline__ int quantise(float v, int n) {
+    if (!(v >= 0.f)) return 0;
+    if (v >= static_cast<float>(n)) return n - 1;
+    const int i = static_cast<int>(v);
+    return i > n - 1 ? n - 1 : i;
+}
+
 }  // namespace acl

@@ -113,6 +113,9 @@ struct KnnWorkspace {
 KnnWorkspace knn_workspace_layout(int B, int Q, int N, int d, int K);
 
 size_t knn_table_smem_bytes(int N, int nbins);
+size_t token_order_smem_bytes(int N);
+cudaError_t launch_token_order(const float* xy, int B, int N, int GH, int GW, int32_t* perm,
+                               cudaStream_t st);
 cudaError_t launch_knn_table(const float* xy, int B, int N, int GH, int GW, int K,
                              int32_t* table, cudaStream_t st);
 cudaError_t launch_knn_fwd(const KnnArgs& a, cudaStream_t st);

@@ -42,13 +42,6 @@ constexpr int kGatherWarps = 8;
 constexpr int kGatherThreads = 32 * kGatherWarps;
 constexpr int kCsrThreads = 1024;
 
-__device__ __forceinline__ int quantise(float v, int n) {
-    if (!(v >= 0.f)) return 0;
-    if (v >= static_cast<float>(n)) return n - 1;
-    const int i = static_cast<int>(v);
-    return i > n - 1 ? n - 1 : i;
-}
-
 // Exclusive prefix sum in place by the whole block; returns the total.
 __device__ int block_scan(int* data, int n, int* scratch) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;

@@ -99,6 +99,17 @@ def test_attention_validation():
     assert L.acl_cluster_attn_bwd(*args, P + 16, ws, None) == WORKSPACE
 
 
+def test_token_order_validation():
+    L = _lib()
+    assert L.acl_token_order(None, 1, 10, 8, 8, P, None) == INVALID
+    assert L.acl_token_order(P, 1, 10, 8, 8, None, None) == INVALID
+    assert L.acl_token_order(P, 1, 0, 8, 8, P, None) == INVALID
+    assert L.acl_token_order(P, 1, 10, 0, 8, P, None) == INVALID
+    assert L.acl_token_order(P, 1, 16385, 8, 8, P, None) == UNSUPPORTED
+    assert L.acl_token_order(P, 1, 10, 4097, 8, P, None) == UNSUPPORTED
+    assert L.acl_token_order(P + 4, 1, 10, 8, 8, P, None) == INVALID
+
+
 def test_knn_validation():
     L = _lib()
     assert L.acl_knn_table(P, 1, 0, 64, 64, 8, P, None) == INVALID

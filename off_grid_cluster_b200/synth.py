@@ -50,7 +50,7 @@ TAG_Q, TAG_K, TAG_V, TAG_DO = 10, 11, 12, 13
 TAG_QUERY, TAG_FEAT, TAG_P, TAG_DOUT = 20, 21, 22, 23
 
 WORKLOAD_ID = {"tiny": 1, "stage1": 2, "stage3": 3, "sweep": 4, "decoder": 5,
-               "step": 6, "hires": 7}
+               "step": 6, "hires": 7, "merge": 8}
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -369,3 +369,50 @@ def hires_batch(B: int = 2, image0: int = 0, grid: int = 128, keep: int | None =
     keep = grid * grid // 2 if keep is None else keep
     xy = np.stack([stage1_coords(wid, i, grid, grid, keep) for i in range(image0, image0 + B)])
     return knn_batch(xy, d, image0, 0, wid=wid, gh=grid, gw=grid)
+
+
+@dataclass
+class MergeBatch:
+    """Token merging between stages: B images of N tokens (d channels) -> k anchors, with a
+    seeded random scoring MLP (W1 [d][h], b1 [h], w2 [h], b2) and upstream gradients."""
+    coords: np.ndarray            # [B, N, 2] fp32
+    feats: np.ndarray             # [B, N, d] bf16 values in fp32
+    w1: np.ndarray                # [d, h] fp32
+    b1: np.ndarray                # [h] fp32
+    w2: np.ndarray                # [h] fp32
+    b2: float
+    k: int
+    dmerged: np.ndarray           # [B, k, d] bf16 values in fp32
+    dmcoords: np.ndarray          # [B, k, 2] fp32
+
+    @property
+    def B(self): return self.coords.shape[0]
+
+    @property
+    def N(self): return self.coords.shape[1]
+
+    @property
+    def d(self): return self.feats.shape[2]
+
+    @property
+    def h(self): return self.w1.shape[1]
+
+
+def merge_batch(coords: np.ndarray, d: int = 128, ds: float = 0.4, image0: int = 0,
+                hidden: int | None = None) -> MergeBatch:
+    """Merge of one stage's tokens: k = round(ds N) anchors, hidden width d/4 by default;
+    W1 ~ N(0, 1/d), w2 ~ N(0, 1/h), biases ~ 0.1 N(0, 1); features and gradients N(0, 1)."""
+    wid = WORKLOAD_ID["merge"]
+    B, N = coords.shape[:2]
+    h = d // 4 if hidden is None else hidden
+    k = int(math.floor(N * ds + 0.5))
+    imgs = range(image0, image0 + B)
+    feats = np.stack([normal_bf16(stream_seed(wid, i, TAG_FEAT), (N, d)) for i in imgs])
+    w1 = (normal(stream_seed(wid, 0, TAG_Q, 1), d * h) / math.sqrt(d)).reshape(d, h).astype(np.float32)
+    b1 = (0.1 * normal(stream_seed(wid, 0, TAG_K, 1), h)).astype(np.float32)
+    w2 = (normal(stream_seed(wid, 0, TAG_V, 1), h) / math.sqrt(h)).astype(np.float32)
+    b2 = float(np.float32(0.1 * normal(stream_seed(wid, 0, TAG_DO, 1), 1)[0]))
+    dm = np.stack([normal_bf16(stream_seed(wid, i, TAG_DOUT), (k, d)) for i in imgs])
+    dxy = np.stack([normal(stream_seed(wid, i, TAG_QUERY, 1), 2 * k).reshape(k, 2)
+                    for i in imgs]).astype(np.float32)
+    return MergeBatch(coords.astype(np.float32), feats, w1, b1, w2, b2, k, dm, dxy)

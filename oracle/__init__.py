@@ -30,7 +30,8 @@ def lib():
         L = ct.CDLL(so)
         for name in ("orc_cluster_batch", "orc_neighbors_batch", "orc_attn_fwd_batch",
                      "orc_attn_bwd_batch", "orc_knn_table_batch", "orc_knn_fwd_batch",
-                     "orc_knn_bwd_batch", "orc_set_threads", "orc_token_order_batch"):
+                     "orc_knn_bwd_batch", "orc_set_threads", "orc_token_order_batch",
+                     "orc_merge_scores", "orc_merge_select", "orc_merge_fwd", "orc_merge_bwd"):
             getattr(L, name).restype = ct.c_int
         _lib = L
     return _lib
@@ -152,3 +153,62 @@ def token_order(xy, GH, GW):
     perm = np.empty((B, N), dtype=np.int32)
     _check(lib().orc_token_order_batch(_p(xy), B, N, GH, GW, _p(perm)), "token_order")
     return perm
+
+
+# ------------------------------------------------------------------ token merging
+
+def merge_scores(feats, w1, b1, w2, b2):
+    """Importance scores s = w2 . gelu(W1^T f + b1) + b2 -> [B, N] fp64."""
+    feats, w1, b1, w2 = _f64(feats), _f64(w1), _f64(b1), _f64(w2)
+    B, N, d = feats.shape
+    h = w1.shape[1]
+    out = np.empty((B, N), dtype=np.float64)
+    for b in range(B):
+        _check(lib().orc_merge_scores(_p(feats[b]), N, d, _p(w1), _p(b1), _p(w2),
+                                      ct.c_double(float(b2)), h, _p(out[b])), "merge_scores")
+    return out
+
+
+def merge_select(scores, xy, k):
+    """Anchors (top-k scores, ties by id, ascending id) and nearest-anchor assignment."""
+    scores, xy = _f64(scores), _f32(xy)
+    B, N = scores.shape
+    anchors = np.empty((B, k), dtype=np.int32)
+    assign = np.empty((B, N), dtype=np.int32)
+    for b in range(B):
+        _check(lib().orc_merge_select(_p(scores[b]), _p(xy[b]), N, k, _p(anchors[b]),
+                                      _p(assign[b])), "merge_select")
+    return anchors, assign
+
+
+def merge_fwd(feats, xy, scores, k, assign):
+    """Merged features [B, k, d] and coordinates [B, k, 2] (softmax-of-score weights)."""
+    feats, xy, scores, assign = _f64(feats), _f32(xy), _f64(scores), _i32(assign)
+    B, N, d = feats.shape
+    merged = np.empty((B, k, d), dtype=np.float64)
+    mxy = np.empty((B, k, 2), dtype=np.float64)
+    for b in range(B):
+        _check(lib().orc_merge_fwd(_p(feats[b]), _p(xy[b]), N, d, _p(scores[b]), k,
+                                   _p(assign[b]), _p(merged[b]), _p(mxy[b])), "merge_fwd")
+    return merged, mxy
+
+
+def merge_bwd(feats, xy, w1, b1, w2, b2, k, assign, dmerged, dmxy):
+    """(dfeats, dcoords, dW1, db1, dw2, db2) for fixed anchors/assignment; parameter
+    gradients summed over the images."""
+    feats, xy, assign = _f64(feats), _f32(xy), _i32(assign)
+    w1, b1, w2 = _f64(w1), _f64(b1), _f64(w2)
+    dmerged, dmxy = _f64(dmerged), _f64(dmxy)
+    B, N, d = feats.shape
+    h = w1.shape[1]
+    df = np.empty((B, N, d)); dxy = np.empty((B, N, 2))
+    dw1 = np.zeros((d, h)); db1 = np.zeros(h); dw2 = np.zeros(h); db2 = 0.0
+    for b in range(B):
+        t1, t2, t3 = np.empty((d, h)), np.empty(h), np.empty(h)
+        t4 = ct.c_double(0.0)
+        _check(lib().orc_merge_bwd(_p(feats[b]), _p(xy[b]), N, d, _p(w1), _p(b1), _p(w2),
+                                   ct.c_double(float(b2)), h, k, _p(assign[b]), _p(dmerged[b]),
+                                   _p(dmxy[b]), _p(df[b]), _p(dxy[b]), _p(t1), _p(t2), _p(t3),
+                                   ct.byref(t4)), "merge_bwd")
+        dw1 += t1; db1 += t2; dw2 += t3; db2 += t4.value
+    return df, dxy, dw1, db1, dw2, db2

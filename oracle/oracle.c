@@ -562,6 +562,173 @@ int orc_token_order(const float* xy, int N, int GH, int GW, int32_t* perm) {
     return 0;
 }
 
+/*
+ * Token merging between stages (AFFMAE notes, "Key Designs" 1, adaptive off-grid token
+ * merging): a lightweight MLP scores every token, the top-k by score are kept as anchors
+ * at the retention rate, and every other token is merged differentiably into its nearest
+ * anchor, fusing features and spatial support.  The notes fix no more than that; the
+ * readings taken:
+ *   score s_i = w2 . gelu(W1^T f_i + b1) + b2, W1 [d][h], gelu(z) = z (1 + erf(z/sqrt 2))/2;
+ *   anchors: the k largest scores, ties by lower id, listed by ascending id;
+ *   assignment: the nearest anchor by squared distance (dx*dx + dy*dy in fp64, dx = x_i -
+ *     x_a), ties by lower anchor id; an anchor is its own group;
+ *   merge: group G_j of anchor j, weights w_i = exp(s_i - max_G s) / sum_G exp(.) (the
+ *     softmax of the scores: differentiable in the scores, so the MLP is trained through
+ *     the merge); merged feature F_j = sum_G w_i f_i, merged coordinate X_j = sum_G w_i x_i.
+ */
+static const double kPi = 3.14159265358979323846;
+static double gelu(double z) { return 0.5 * z * (1.0 + erf(z / sqrt(2.0))); }
+static double gelu_grad(double z) {
+    return 0.5 * (1.0 + erf(z / sqrt(2.0))) + z * exp(-0.5 * z * z) / sqrt(2.0 * kPi);
+}
+
+int orc_merge_scores(const double* f, int N, int d, const double* w1, const double* b1,
+                     const double* w2, double b2, int h, double* scores) {
+    if (N < 1 || d < 1 || h < 1) return 1;
+    for (int i = 0; i < N; ++i) {
+        double s = b2;
+        for (int u = 0; u < h; ++u) {
+            double z = b1[u];
+            for (int c = 0; c < d; ++c) z += f[(size_t)i * d + c] * w1[(size_t)c * h + u];
+            s += w2[u] * gelu(z);
+        }
+        scores[i] = s;
+    }
+    return 0;
+}
+
+typedef struct { double s; int id; } score_id;
+static int cmp_score_desc(const void* pa, const void* pb) {
+    const score_id* a = (const score_id*)pa;
+    const score_id* b = (const score_id*)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->id > b->id) - (a->id < b->id);
+}
+
+int orc_merge_select(const double* scores, const float* xy, int N, int k, int32_t* anchors,
+                     int32_t* assign) {
+    if (N < 1 || k < 1 || k > N) return 1;
+    score_id* o = (score_id*)malloc(sizeof(score_id) * (size_t)N);
+    int32_t* rank = (int32_t*)malloc(sizeof(int32_t) * (size_t)N);
+    if (!o || !rank) { free(o); free(rank); return 2; }
+    for (int i = 0; i < N; ++i) { o[i].s = scores[i]; o[i].id = i; rank[i] = -1; }
+    qsort(o, (size_t)N, sizeof(score_id), cmp_score_desc);
+    for (int j = 0; j < k; ++j) anchors[j] = o[j].id;
+    qsort(anchors, (size_t)k, sizeof(int32_t), cmp_i32);
+    for (int j = 0; j < k; ++j) rank[anchors[j]] = j;
+    for (int i = 0; i < N; ++i) {
+        if (rank[i] >= 0) { assign[i] = rank[i]; continue; }
+        double best = INFINITY;
+        int bj = 0;
+        for (int j = 0; j < k; ++j) {
+            int a = anchors[j];
+            double dx = (double)xy[2 * i] - (double)xy[2 * a];
+            double dy = (double)xy[2 * i + 1] - (double)xy[2 * a + 1];
+            double d2 = dx * dx + dy * dy;
+            if (d2 < best) { best = d2; bj = j; }   /* strict: ties keep the lower id */
+        }
+        assign[i] = bj;
+    }
+    free(o);
+    free(rank);
+    return 0;
+}
+
+int orc_merge_fwd(const double* f, const float* xy, int N, int d, const double* scores, int k,
+                  const int32_t* assign, double* merged, double* mxy) {
+    if (N < 1 || d < 1 || k < 1) return 1;
+    double* gmax = (double*)malloc(sizeof(double) * (size_t)k);
+    double* gsum = (double*)calloc((size_t)k, sizeof(double));
+    if (!gmax || !gsum) { free(gmax); free(gsum); return 2; }
+    for (int j = 0; j < k; ++j) gmax[j] = -INFINITY;
+    for (int i = 0; i < N; ++i) if (scores[i] > gmax[assign[i]]) gmax[assign[i]] = scores[i];
+    for (int i = 0; i < N; ++i) gsum[assign[i]] += exp(scores[i] - gmax[assign[i]]);
+    memset(merged, 0, sizeof(double) * (size_t)k * d);
+    memset(mxy, 0, sizeof(double) * (size_t)k * 2);
+    for (int i = 0; i < N; ++i) {
+        int j = assign[i];
+        double w = exp(scores[i] - gmax[j]) / gsum[j];
+        for (int c = 0; c < d; ++c) merged[(size_t)j * d + c] += w * f[(size_t)i * d + c];
+        mxy[2 * j] += w * (double)xy[2 * i];
+        mxy[2 * j + 1] += w * (double)xy[2 * i + 1];
+    }
+    free(gmax);
+    free(gsum);
+    return 0;
+}
+
+/*
+ * Backward of the merge and of the scoring MLP for fixed anchors and assignment (both are
+ * piecewise constant in the inputs).  With g_i = <dF_j, f_i> + <dX_j, x_i> for i in G_j:
+ *   df_i = w_i dF_j + W1 dh_i,  dx_i = w_i dX_j,
+ *   ds_i = w_i (g_i - sum_G w g),  dh_i = ds_i w2 * gelu'(z_i),
+ *   dW1 = sum_i f_i dh_i^T, db1 = sum_i dh_i, dw2 = sum_i ds_i gelu(z_i), db2 = sum_i ds_i.
+ * The scores are recomputed from the MLP.  Outputs are overwritten; dW1 ... db2 hold this
+ * image's sums.
+ */
+int orc_merge_bwd(const double* f, const float* xy, int N, int d, const double* w1,
+                  const double* b1, const double* w2, double b2, int h, int k,
+                  const int32_t* assign, const double* dmerged, const double* dmxy,
+                  double* df, double* dxy, double* dw1, double* db1, double* dw2, double* db2) {
+    if (N < 1 || d < 1 || h < 1 || k < 1) return 1;
+    double* s = (double*)malloc(sizeof(double) * (size_t)N);
+    double* z = (double*)malloc(sizeof(double) * (size_t)N * h);
+    double* g = (double*)malloc(sizeof(double) * (size_t)N);
+    double* gmax = (double*)malloc(sizeof(double) * (size_t)k);
+    double* gsum = (double*)calloc((size_t)k, sizeof(double));
+    double* gws = (double*)calloc((size_t)k, sizeof(double));
+    if (!s || !z || !g || !gmax || !gsum || !gws) {
+        free(s); free(z); free(g); free(gmax); free(gsum); free(gws);
+        return 2;
+    }
+    for (int i = 0; i < N; ++i) {
+        double si = b2;
+        for (int u = 0; u < h; ++u) {
+            double zz = b1[u];
+            for (int c = 0; c < d; ++c) zz += f[(size_t)i * d + c] * w1[(size_t)c * h + u];
+            z[(size_t)i * h + u] = zz;
+            si += w2[u] * gelu(zz);
+        }
+        s[i] = si;
+    }
+    for (int j = 0; j < k; ++j) gmax[j] = -INFINITY;
+    for (int i = 0; i < N; ++i) if (s[i] > gmax[assign[i]]) gmax[assign[i]] = s[i];
+    for (int i = 0; i < N; ++i) gsum[assign[i]] += exp(s[i] - gmax[assign[i]]);
+    for (int i = 0; i < N; ++i) {
+        int j = assign[i];
+        double gi = dmxy[2 * j] * (double)xy[2 * i] + dmxy[2 * j + 1] * (double)xy[2 * i + 1];
+        for (int c = 0; c < d; ++c) gi += dmerged[(size_t)j * d + c] * f[(size_t)i * d + c];
+        g[i] = gi;
+        gws[j] += exp(s[i] - gmax[j]) / gsum[j] * gi;
+    }
+    memset(dw1, 0, sizeof(double) * (size_t)d * h);
+    memset(db1, 0, sizeof(double) * (size_t)h);
+    memset(dw2, 0, sizeof(double) * (size_t)h);
+    *db2 = 0.0;
+    for (int i = 0; i < N; ++i) {
+        int j = assign[i];
+        double w = exp(s[i] - gmax[j]) / gsum[j];
+        double ds = w * (g[i] - gws[j]);
+        dxy[2 * i] = w * dmxy[2 * j];
+        dxy[2 * i + 1] = w * dmxy[2 * j + 1];
+        for (int c = 0; c < d; ++c) df[(size_t)i * d + c] = w * dmerged[(size_t)j * d + c];
+        *db2 += ds;
+        for (int u = 0; u < h; ++u) {
+            double zz = z[(size_t)i * h + u];
+            double dh = ds * w2[u] * gelu_grad(zz);
+            dw2[u] += ds * gelu(zz);
+            db1[u] += dh;
+            for (int c = 0; c < d; ++c) {
+                df[(size_t)i * d + c] += w1[(size_t)c * h + u] * dh;
+                dw1[(size_t)c * h + u] += f[(size_t)i * d + c] * dh;
+            }
+        }
+    }
+    free(s); free(z); free(g); free(gmax); free(gsum); free(gws);
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* batch drivers: images are independent; OpenMP over images only            */
 /* ------------------------------------------------------------------------ */

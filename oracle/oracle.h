@@ -34,6 +34,18 @@ int orc_knn_bwd(const float* queries, int Q, const double* feats, const float* x
 /* token ids in Z-order of their cells on the GH x GW grid, ties by id */
 int orc_token_order(const float* xy, int N, int GH, int GW, int32_t* perm);
 
+/* token merging: MLP scores, top-k anchors + nearest-anchor assignment, merge, backward */
+int orc_merge_scores(const double* f, int N, int d, const double* w1, const double* b1,
+                     const double* w2, double b2, int h, double* scores);
+int orc_merge_select(const double* scores, const float* xy, int N, int k, int32_t* anchors,
+                     int32_t* assign);
+int orc_merge_fwd(const double* f, const float* xy, int N, int d, const double* scores, int k,
+                  const int32_t* assign, double* merged, double* mxy);
+int orc_merge_bwd(const double* f, const float* xy, int N, int d, const double* w1,
+                  const double* b1, const double* w2, double b2, int h, int k,
+                  const int32_t* assign, const double* dmerged, const double* dmxy,
+                  double* df, double* dxy, double* dw1, double* db1, double* dw2, double* db2);
+
 int orc_cluster_batch(const float* xy, int B, int N, int C, int32_t* clusters);
 int orc_neighbors_batch(const float* xy, const int32_t* clusters, int B, int N, int C,
                         int M, int32_t* nbr);

@@ -457,6 +457,7 @@ def run_gpu(args, rank: int, world: int):
             e1.synchronize()
             inv_us[name] = round(e0.elapsed_time(e1) / 20 * 1e3, 2)
     hires = hires_gather_times(torch, acl, synth, device, stream) if world == 1 else None
+    merge_us = token_merge_times(torch, acl, synth, sb, device, stream) if world == 1 else None
     # keep the same load on the GPU until the clock sampler has several samples
     t_wall = time.time()
     it = 0
@@ -528,6 +529,7 @@ def run_gpu(args, rank: int, world: int):
             "knn_invpow_us": {**inv_us, "note": "inverse-power weight kernel (d^-p), same "
                               "gathers, set 0, L2-warm (one set): compare with per_call"},
             "hires_gather_us": hires,
+            "token_merge_us": merge_us,
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -550,6 +552,39 @@ def run_gpu(args, rank: int, world: int):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def token_merge_times(torch, acl, synth, sb, device, stream, reps: int = 10) -> dict:
+    """Token merging of the stage-1 tokens into round(0.4 N) anchors (d = 128, hidden 32),
+    forward and backward, one call at a time with CUDA events."""
+    mb = synth.merge_batch(sb.attn.coords, d=128)
+    T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
+    f, xy = T(mb.feats, torch.bfloat16), T(mb.coords)
+    w1, b1, w2 = T(mb.w1), T(mb.b1), T(mb.w2)
+    dm, dx = T(mb.dmerged, torch.bfloat16), T(mb.dmcoords)
+    ws = torch.empty((acl.acl_token_merge_workspace(mb.B, mb.N, mb.d, mb.h, mb.k),),
+                     dtype=torch.uint8, device=device)
+    out = acl.acl_token_merge_fwd(f, xy, w1, b1, w2, mb.b2, mb.k, workspace=ws, stream=stream)
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+        e1.synchronize()
+        return round(e0.elapsed_time(e1) / reps * 1e3, 2)
+
+    return {
+        "workload": f"{mb.B} images, N = {mb.N} -> k = {mb.k}, d = {mb.d}, hidden {mb.h}",
+        "fwd": timed(lambda: acl.acl_token_merge_fwd(f, xy, w1, b1, w2, mb.b2, mb.k, workspace=ws,
+                                                     stream=stream)),
+        "bwd": timed(lambda: acl.acl_token_merge_bwd(f, xy, w1, b1, w2, mb.b2, mb.k, out[0], out[2],
+                                                     dm, dx, workspace=ws, stream=stream)),
+    }
 
 
 def hires_gather_times(torch, acl, synth, device, stream, B: int = 4, reps: int = 10) -> dict:

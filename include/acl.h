@@ -236,6 +236,48 @@ acl_status acl_knn_table(const float* coords, int B, int N, int H, int W, int K,
 acl_status acl_token_order(const float* coords, int B, int N, int H, int W, int32_t* perm,
                            acl_stream_t stream);
 
+/*
+ * Token merging between stages -- AFF notes, "Key Designs" 1 (adaptive off-grid token
+ * merging): a lightweight MLP scores every token, the top-k are kept as anchors at the
+ * retention rate, and the other tokens are merged differentiably into their nearest anchor,
+ * fusing features and spatial support.  The notes fix no more; this library takes:
+ *   s_i = w2 . gelu(W1^T f_i + b1) + b2, gelu(z) = z (1 + erf(z / sqrt 2)) / 2, fp32;
+ *   anchors: the k largest s_i, ties by lower id, listed by ascending token id;
+ *   assign_i: the rank (0..k-1) of the anchor nearest to token i (squared distance of the
+ *     fp32 coordinates in fp64, ties by lower anchor id); an anchor is its own group;
+ *   merged_j = sum_{i in G_j} w_i f_i and mcoords_j = sum w_i x_i, w = softmax of the
+ *     group's scores (so the scores, and the MLP, receive gradients).
+ * feats [B][N][d] bf16 (16-byte aligned); coords [B][N][2] fp32; W1 [d][h], b1 [h], w2 [h]
+ * fp32 (device); scores [B][N] fp32, anchors [B][k] int32, assign [B][N] int32, merged
+ * [B][k][d] bf16, mcoords [B][k][2] fp32 out.  The anchor choice is an integer decision on
+ * fp32 scores; ties and near-ties follow the fp32 values.
+ * workspace: acl_token_merge_workspace(B, N, d, h, k) bytes, 256-byte aligned.
+ * Limits: d % 32 == 0, 32 <= d <= ACL_MAX_GATHER_D, 1 <= h <= 256, 1 <= k <= N <=
+ * ACL_MAX_TABLE_N.  No atomics in any sum: results are bit-reproducible.
+ */
+size_t acl_token_merge_workspace(int B, int N, int d, int h, int k);
+acl_status acl_token_merge_fwd(const acl_bf16* feats, const float* coords, int B, int N, int d,
+                               const float* w1, const float* b1, const float* w2, float b2,
+                               int h, int k, float* scores, int32_t* anchors, int32_t* assign,
+                               acl_bf16* merged, float* mcoords, void* workspace,
+                               size_t ws_bytes, acl_stream_t stream);
+/*
+ * Backward for the forward's scores and assignment (anchors and assignment are piecewise
+ * constant: no gradient flows through them):
+ *   g_i = <dmerged_j, f_i> + <dmcoords_j, x_i>, ds_i = w_i (g_i - sum_G w g),
+ *   dfeats_i = w_i dmerged_j + W1 dh_i, dh_i = ds_i w2 * gelu'(z_i), dcoords_i = w_i dmcoords_j,
+ *   dW1 = sum_i f_i dh_i^T, db1 = sum dh_i, dw2 = sum ds_i gelu(z_i), db2 = sum ds_i
+ *   (sums over all images).  All outputs are overwritten.
+ * dmerged [B][k][d] bf16, dmcoords [B][k][2] fp32 in; dfeats [B][N][d] bf16, dcoords
+ * [B][N][2], dW1 [d][h], db1 [h], dw2 [h], db2 [1] fp32 out.
+ */
+acl_status acl_token_merge_bwd(const acl_bf16* feats, const float* coords, int B, int N, int d,
+                               const float* w1, const float* b1, const float* w2, float b2,
+                               int h, int k, const float* scores, const int32_t* assign,
+                               const acl_bf16* dmerged, const float* dmcoords, acl_bf16* dfeats,
+                               float* dcoords, float* dw1, float* db1, float* dw2, float* db2,
+                               void* workspace, size_t ws_bytes, acl_stream_t stream);
+
 /* Workspace bytes acl_knn_gather_bwd (and acl_knn_gather_index +
  * acl_knn_gather_bwd_indexed) need for these sizes (0 on bad sizes). */
 size_t acl_knn_gather_workspace(int B, int Q, int N, int d, int K);

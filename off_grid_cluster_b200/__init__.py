@@ -41,6 +41,11 @@ SIGNATURES = {
                                           _F, _P, _P, _P, _P, _P, _P, _P, _P]),
     "acl_knn_table": (_I, [_P, _I, _I, _I, _I, _I, _P, _P]),
     "acl_token_order": (_I, [_P, _I, _I, _I, _I, _P, _P]),
+    "acl_token_merge_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "acl_token_merge_fwd": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _F, _I, _I, _P, _P, _P, _P, _P,
+                                 _P, _Z, _P]),
+    "acl_token_merge_bwd": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _F, _I, _I, _P, _P, _P, _P, _P,
+                                 _P, _P, _P, _P, _P, _P, _Z, _P]),
     "acl_knn_gather_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "acl_knn_gather_fwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P]),
     "acl_knn_gather_bwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P,
@@ -261,6 +266,63 @@ def acl_token_order(coords: torch.Tensor, H: int, W: int, perm: torch.Tensor | N
     perm = _out(perm, (B, N), torch.int32, coords, "perm")
     _call("acl_token_order", _ptr(coords), B, N, H, W, _ptr(perm), _stream(stream))
     return perm
+
+
+def acl_token_merge_workspace(B: int, N: int, d: int, h: int, k: int) -> int:
+    return int(lib().acl_token_merge_workspace(B, N, d, h, k))
+
+
+def _merge_shapes(feats, coords, w1, b1, w2):
+    _need(feats, "feats", torch.bfloat16)
+    B, N, d = feats.shape
+    _need(coords, "coords", torch.float32, (B, N, 2))
+    _need(w1, "w1", torch.float32)
+    h = w1.shape[1]
+    _need(w1, "w1", torch.float32, (d, h))
+    _need(b1, "b1", torch.float32, (h,))
+    _need(w2, "w2", torch.float32, (h,))
+    return B, N, d, h
+
+
+def acl_token_merge_fwd(feats, coords, w1, b1, w2, b2: float, k: int, workspace=None, stream=None):
+    """Token merging -> (scores [B,N] f32, anchors [B,k] i32, assign [B,N] i32,
+    merged [B,k,d] bf16, mcoords [B,k,2] f32)."""
+    B, N, d, h = _merge_shapes(feats, coords, w1, b1, w2)
+    dev = feats.device
+    scores = torch.empty((B, N), dtype=torch.float32, device=dev)
+    anchors = torch.empty((B, k), dtype=torch.int32, device=dev)
+    assign = torch.empty((B, N), dtype=torch.int32, device=dev)
+    merged = torch.empty((B, k, d), dtype=torch.bfloat16, device=dev)
+    mcoords = torch.empty((B, k, 2), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(acl_token_merge_workspace(B, N, d, h, k), 1),
+                                dtype=torch.uint8, device=dev)
+    _call("acl_token_merge_fwd", _ptr(feats), _ptr(coords), B, N, d, _ptr(w1), _ptr(b1),
+          _ptr(w2), float(b2), h, k, _ptr(scores), _ptr(anchors), _ptr(assign), _ptr(merged),
+          _ptr(mcoords), _ptr(workspace), workspace.numel(), _stream(stream))
+    return scores, anchors, assign, merged, mcoords
+
+
+def acl_token_merge_bwd(feats, coords, w1, b1, w2, b2: float, k: int, scores, assign, dmerged,
+                        dmcoords, workspace=None, stream=None):
+    """Token merging backward -> (dfeats [B,N,d] bf16, dcoords [B,N,2], dW1 [d,h], db1 [h],
+    dw2 [h], db2 [1] f32)."""
+    B, N, d, h = _merge_shapes(feats, coords, w1, b1, w2)
+    dev = feats.device
+    _need(dmerged, "dmerged", torch.bfloat16, (B, k, d))
+    _need(dmcoords, "dmcoords", torch.float32, (B, k, 2))
+    dfeats = torch.empty_like(feats)
+    dcoords = torch.empty_like(coords)
+    dw1, db1, dw2 = torch.empty_like(w1), torch.empty_like(b1), torch.empty_like(w2)
+    db2 = torch.empty((1,), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(acl_token_merge_workspace(B, N, d, h, k), 1),
+                                dtype=torch.uint8, device=dev)
+    _call("acl_token_merge_bwd", _ptr(feats), _ptr(coords), B, N, d, _ptr(w1), _ptr(b1),
+          _ptr(w2), float(b2), h, k, _ptr(scores), _ptr(assign), _ptr(dmerged), _ptr(dmcoords),
+          _ptr(dfeats), _ptr(dcoords), _ptr(dw1), _ptr(db1), _ptr(dw2), _ptr(db2),
+          _ptr(workspace), workspace.numel(), _stream(stream))
+    return dfeats, dcoords, dw1, db1, dw2, db2
 
 
 def acl_knn_gather_workspace(B: int, Q: int, N: int, d: int, K: int = 8) -> int:

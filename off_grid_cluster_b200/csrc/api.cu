@@ -202,6 +202,84 @@ acl_status acl_token_order(const float* coords, int B, int N, int H, int W, int3
     return cuda_status(acl::launch_token_order(coords, B, N, H, W, perm, S(stream)));
 }
 
+size_t acl_token_merge_workspace(int B, int N, int d, int h, int k) {
+    if (B < 1 || N < 1 || d < 32 || d % 32 != 0 || h < 1 || k < 1 || k > N) return 0;
+    return acl::merge_workspace_layout(B, N, d, h, k).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+acl_status check_merge(const acl_bf16* feats, const float* coords, int B, int N, int d,
+                       const float* w1, const float* b1, const float* w2, int h, int k,
+                       void* workspace, size_t ws_bytes) {
+    if (!feats || !coords || !w1 || !b1 || !w2) return ACL_ERR_INVALID_ARG;
+    if (B < 1 || N < 1 || d < 32 || d % 32 != 0 || h < 1 || k < 1 || k > N) return ACL_ERR_INVALID_ARG;
+    if (N > ACL_MAX_TABLE_N || d > ACL_MAX_GATHER_D || h > 256 || B > 65535) return ACL_ERR_UNSUPPORTED;
+    if (acl::merge_smem_bytes(N, k, d, h) > kMaxSmem) return ACL_ERR_UNSUPPORTED;
+    if (!aligned(feats, 16) || !aligned(coords, 8)) return ACL_ERR_INVALID_ARG;
+    const acl::MergeWorkspace L = acl::merge_workspace_layout(B, N, d, h, k);
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < L.total) return ACL_ERR_WORKSPACE;
+    return ACL_OK;
+}
+
+void map_merge(acl::MergeArgs& m, const acl_bf16* feats, const float* coords, int B, int N, int d,
+               const float* w1, const float* b1, const float* w2, float b2, int h, int k,
+               void* workspace) {
+    const acl::MergeWorkspace L = acl::merge_workspace_layout(B, N, d, h, k);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    m.feats = BF(feats); m.xy = coords; m.B = B; m.N = N; m.d = d; m.h = h; m.k = k;
+    m.w1 = w1; m.b1 = b1; m.w2 = w2; m.b2 = b2;
+    m.rank = reinterpret_cast<int32_t*>(ws + L.rank);
+    m.members = reinterpret_cast<int32_t*>(ws + L.members);
+    m.goff = reinterpret_cast<int32_t*>(ws + L.goff);
+    m.ds = reinterpret_cast<float*>(ws + L.ds);
+    m.dh = reinterpret_cast<float*>(ws + L.dh);
+    m.gz = reinterpret_cast<float*>(ws + L.gz);
+    m.part = reinterpret_cast<float*>(ws + L.part);
+}
+
+}  // namespace
+
+extern "C" {
+
+acl_status acl_token_merge_fwd(const acl_bf16* feats, const float* coords, int B, int N, int d,
+                               const float* w1, const float* b1, const float* w2, float b2, int h,
+                               int k, float* scores, int32_t* anchors, int32_t* assign,
+                               acl_bf16* merged, float* mcoords, void* workspace, size_t ws_bytes,
+                               acl_stream_t stream) {
+    acl_status st = check_merge(feats, coords, B, N, d, w1, b1, w2, h, k, workspace, ws_bytes);
+    if (st != ACL_OK) return st;
+    if (!scores || !anchors || !assign || !merged || !mcoords) return ACL_ERR_INVALID_ARG;
+    if (!aligned(merged, 16) || !aligned(mcoords, 8)) return ACL_ERR_INVALID_ARG;
+    acl::MergeArgs m = {};
+    map_merge(m, feats, coords, B, N, d, w1, b1, w2, b2, h, k, workspace);
+    m.scores = scores; m.anchors = anchors; m.assign = assign; m.merged = BFm(merged); m.mxy = mcoords;
+    return cuda_status(acl::launch_merge_fwd(m, S(stream)));
+}
+
+acl_status acl_token_merge_bwd(const acl_bf16* feats, const float* coords, int B, int N, int d,
+                               const float* w1, const float* b1, const float* w2, float b2, int h,
+                               int k, const float* scores, const int32_t* assign,
+                               const acl_bf16* dmerged, const float* dmcoords, acl_bf16* dfeats,
+                               float* dcoords, float* dw1, float* db1, float* dw2, float* db2,
+                               void* workspace, size_t ws_bytes, acl_stream_t stream) {
+    acl_status st = check_merge(feats, coords, B, N, d, w1, b1, w2, h, k, workspace, ws_bytes);
+    if (st != ACL_OK) return st;
+    if (!scores || !assign || !dmerged || !dmcoords || !dfeats || !dcoords || !dw1 || !db1 || !dw2 ||
+        !db2)
+        return ACL_ERR_INVALID_ARG;
+    if (!aligned(dmerged, 16) || !aligned(dfeats, 16) || !aligned(dcoords, 8) || !aligned(dmcoords, 8))
+        return ACL_ERR_INVALID_ARG;
+    acl::MergeArgs m = {};
+    map_merge(m, feats, coords, B, N, d, w1, b1, w2, b2, h, k, workspace);
+    m.scores = const_cast<float*>(scores); m.assign = const_cast<int32_t*>(assign);
+    m.dmerged = BF(dmerged); m.dmxy = dmcoords; m.dfeats = BFm(dfeats); m.dxy = dcoords;
+    m.dw1 = dw1; m.db1 = db1; m.dw2 = dw2; m.db2 = db2;
+    return cuda_status(acl::launch_merge_bwd(m, S(stream)));
+}
+
 size_t acl_knn_gather_workspace(int B, int Q, int N, int d, int K) {
     if (B < 1 || Q < 0 || N < 1 || d < 32 || d % 32 != 0 || K < 1) return 0;
     return acl::knn_workspace_layout(B, Q, N, d, K).total;

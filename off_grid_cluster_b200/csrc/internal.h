@@ -112,6 +112,46 @@ struct KnnWorkspace {
 };
 KnnWorkspace knn_workspace_layout(int B, int Q, int N, int d, int K);
 
+struct MergeArgs {
+    const bf16* feats;
+    const float* xy;
+    int B, N, d, h, k;
+    const float* w1;
+    const float* b1;
+    const float* w2;
+    float b2;
+    float* scores;       // [B][N] (written by the forward, read by the backward)
+    int32_t* anchors;    // [B][k]
+    int32_t* assign;     // [B][N]
+    bf16* merged;        // [B][k][d]
+    float* mxy;          // [B][k][2]
+    // backward
+    const bf16* dmerged;
+    const float* dmxy;
+    bf16* dfeats;
+    float* dxy;
+    float* dw1;
+    float* db1;
+    float* dw2;
+    float* db2;
+    // workspace
+    int32_t* rank;
+    int32_t* members;
+    int32_t* goff;
+    float* ds;
+    float* dh;
+    float* gz;
+    float* part;
+};
+
+struct MergeWorkspace {
+    size_t rank, members, goff, ds, dh, gz, part, total;
+};
+MergeWorkspace merge_workspace_layout(int B, int N, int d, int h, int k);
+size_t merge_smem_bytes(int N, int k, int d, int h);
+cudaError_t launch_merge_fwd(const MergeArgs& m, cudaStream_t st);
+cudaError_t launch_merge_bwd(const MergeArgs& m, cudaStream_t st);
+
 size_t knn_table_smem_bytes(int N, int nbins);
 size_t token_order_smem_bytes(int N);
 cudaError_t launch_token_order(const float* xy, int B, int N, int GH, int GW, int32_t* perm,

@@ -99,6 +99,28 @@ def test_attention_validation():
     assert L.acl_cluster_attn_bwd(*args, P + 16, ws, None) == WORKSPACE
 
 
+def test_token_merge_validation():
+    L = _lib()
+    ws = acl.acl_token_merge_workspace(2, 2048, 128, 32, 819)
+    assert ws > 0
+    assert acl.acl_token_merge_workspace(2, 2048, 100, 32, 819) == 0
+    assert acl.acl_token_merge_workspace(2, 2048, 128, 32, 4096) == 0
+    fwd = lambda N=2048, d=128, h=32, k=819, f=P, wsb=ws, out=P: L.acl_token_merge_fwd(
+        f, P, 2, N, d, P, P, P, 0.0, h, k, out, P, P, P, P, P, wsb, None)
+    assert fwd(f=None) == INVALID
+    assert fwd(d=100) == INVALID
+    assert fwd(k=0) == INVALID and fwd(k=2049) == INVALID
+    assert fwd(h=257) == UNSUPPORTED
+    assert fwd(N=16385, k=10) == UNSUPPORTED
+    assert fwd(f=P + 2) == INVALID
+    assert fwd(wsb=16) == WORKSPACE
+    assert fwd(out=None) == INVALID
+    bwd = lambda wsb=ws, dw=P: L.acl_token_merge_bwd(P, P, 2, 2048, 128, P, P, P, 0.0, 32, 819,
+                                                    P, P, P, P, P, P, dw, P, P, P, P, wsb, None)
+    assert bwd(dw=None) == INVALID
+    assert bwd(wsb=16) == WORKSPACE
+
+
 def test_token_order_validation():
     L = _lib()
     assert L.acl_token_order(None, 1, 10, 8, 8, P, None) == INVALID

@@ -445,17 +445,10 @@ def run_gpu(args, rank: int, world: int):
     # forward and backward of set 0, one call at a time
     inv_us = {}
     s0 = sets[0]
-    with torch.cuda.stream(stream):
-        for name in ("knn_fwd", "knn_bwd"):
-            for _ in range(3):
-                s0.op(name, stream, kind=acl.ACL_KNN_INVPOW)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(20):
-                s0.op(name, stream, kind=acl.ACL_KNN_INVPOW)
-            e1.record(stream)
-            e1.synchronize()
-            inv_us[name] = round(e0.elapsed_time(e1) / 20 * 1e3, 2)
+    for name in ("knn_fwd", "knn_bwd"):
+        for kind, key in ((acl.ACL_KNN_EXP, "exp"), (acl.ACL_KNN_INVPOW, "invpow")):
+            inv_us[f"{name}_{key}"] = graph_time(
+                torch, stream, lambda: s0.op(name, stream, kind=kind), 20)
     hires = hires_gather_times(torch, acl, synth, device, stream) if world == 1 else None
     merge_us = token_merge_times(torch, acl, synth, sb, device, stream) if world == 1 else None
     # keep the same load on the GPU until the clock sampler has several samples
@@ -526,8 +519,8 @@ def run_gpu(args, rank: int, world: int):
                              "after the timed region); the step overlaps the two chains",
             "per_call_concurrent_us": {n: round(per_op_concurrent[j] * 1e3, 2)
                                        for j, n in enumerate(OPS)},
-            "knn_invpow_us": {**inv_us, "note": "inverse-power weight kernel (d^-p), same "
-                              "gathers, set 0, L2-warm (one set): compare with per_call"},
+            "knn_kernels_us": {**inv_us, "note": "exponential and inverse-power weight kernels "
+                               "on the same gathers (set 0, one graph per call, L2-warm)"},
             "hires_gather_us": hires,
             "token_merge_us": merge_us,
         },
@@ -554,6 +547,28 @@ def run_gpu(args, rank: int, world: int):
         print(json.dumps(line), flush=True)
 
 
+def graph_time(torch, stream, fn, reps: int = 10) -> float:
+    """Device time of one call of fn in microseconds: fn captured once as a CUDA graph and
+    replayed `reps` times between CUDA events on `stream` (no host work inside)."""
+    with torch.cuda.stream(stream):
+        fn()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    g.reset()
+    return round(e0.elapsed_time(e1) / reps * 1e3, 2)
+
+
 def token_merge_times(torch, acl, synth, sb, device, stream, reps: int = 10) -> dict:
     """Token merging of the stage-1 tokens into round(0.4 N) anchors (d = 128, hidden 32),
     forward and backward, one call at a time with CUDA events."""
@@ -565,19 +580,7 @@ def token_merge_times(torch, acl, synth, sb, device, stream, reps: int = 10) -> 
     ws = torch.empty((acl.acl_token_merge_workspace(mb.B, mb.N, mb.d, mb.h, mb.k),),
                      dtype=torch.uint8, device=device)
     out = acl.acl_token_merge_fwd(f, xy, w1, b1, w2, mb.b2, mb.k, workspace=ws, stream=stream)
-
-    def timed(fn):
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                fn()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(reps):
-                fn()
-            e1.record(stream)
-        e1.synchronize()
-        return round(e0.elapsed_time(e1) / reps * 1e3, 2)
-
+    timed = lambda fn: graph_time(torch, stream, fn, reps)
     return {
         "workload": f"{mb.B} images, N = {mb.N} -> k = {mb.k}, d = {mb.d}, hidden {mb.h}",
         "fwd": timed(lambda: acl.acl_token_merge_fwd(f, xy, w1, b1, w2, mb.b2, mb.k, workspace=ws,
@@ -598,18 +601,7 @@ def hires_gather_times(torch, acl, synth, device, stream, B: int = 4, reps: int 
     ws = torch.empty((acl.acl_knn_gather_workspace(B, kb.Q, kb.N, kb.d, 8),), dtype=torch.uint8,
                      device=device)
 
-    def timed(fn):
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                fn()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(reps):
-                fn()
-            e1.record(stream)
-        e1.synchronize()
-        return round(e0.elapsed_time(e1) / reps * 1e3, 2)
-
+    timed = lambda fn: graph_time(torch, stream, fn, reps)
     res = {"workload": f"{B} images, 128x128 cells, {kb.N} tokens, {kb.Q} queries, d = {kb.d}, K = 8"}
     perm = acl.acl_token_order(xy, 128, 128, stream=stream)
     res["token_order"] = timed(lambda: acl.acl_token_order(xy, 128, 128, perm=perm, stream=stream))

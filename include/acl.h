@@ -269,7 +269,9 @@ acl_status acl_token_merge_fwd(const acl_bf16* feats, const float* coords, int B
  *   dW1 = sum_i f_i dh_i^T, db1 = sum dh_i, dw2 = sum ds_i gelu(z_i), db2 = sum ds_i
  *   (sums over all images).  All outputs are overwritten.
  * dmerged [B][k][d] bf16, dmcoords [B][k][2] fp32 in; dfeats [B][N][d] bf16, dcoords
- * [B][N][2], dW1 [d][h], db1 [h], dw2 [h], db2 [1] fp32 out.
+ * [B][N][2], dW1 [d][h], db1 [h], dw2 [h], db2 [1] fp32 out.  scores and assign are the
+ * forward's outputs; a token whose assign entry lies outside [0, k) belongs to no group and
+ * gets zero gradients.
  */
 acl_status acl_token_merge_bwd(const acl_bf16* feats, const float* coords, int B, int N, int d,
                                const float* w1, const float* b1, const float* w2, float b2,

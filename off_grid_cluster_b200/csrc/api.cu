@@ -231,12 +231,14 @@ void map_merge(acl::MergeArgs& m, const acl_bf16* feats, const float* coords, in
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     m.feats = BF(feats); m.xy = coords; m.B = B; m.N = N; m.d = d; m.h = h; m.k = k;
     m.w1 = w1; m.b1 = b1; m.w2 = w2; m.b2 = b2;
-    m.rank = reinterpret_cast<int32_t*>(ws + L.rank);
+    m.flag = reinterpret_cast<int32_t*>(ws + L.flag);
     m.members = reinterpret_cast<int32_t*>(ws + L.members);
     m.goff = reinterpret_cast<int32_t*>(ws + L.goff);
+    m.gstat = reinterpret_cast<float*>(ws + L.gstat);
+    m.g = reinterpret_cast<float*>(ws + L.g);
     m.ds = reinterpret_cast<float*>(ws + L.ds);
     m.dh = reinterpret_cast<float*>(ws + L.dh);
-    m.gz = reinterpret_cast<float*>(ws + L.gz);
+    m.e = reinterpret_cast<float*>(ws + L.e);
     m.part = reinterpret_cast<float*>(ws + L.part);
 }
 

@@ -135,17 +135,19 @@ struct MergeArgs {
     float* dw2;
     float* db2;
     // workspace
-    int32_t* rank;
-    int32_t* members;
-    int32_t* goff;
-    float* ds;
-    float* dh;
-    float* gz;
-    float* part;
+    int32_t* flag;       // [B][N] 1 for anchors
+    int32_t* members;    // [B][N] tokens by (assignment, id)
+    int32_t* goff;       // [B][k + 1]
+    float* gstat;        // [B][k][4] max score, 1 / sum, sum_G w g
+    float* g;            // [B][N] <dF, f> + <dX, x>
+    float* ds;           // [B][N]
+    float* dh;           // [B][N][h]
+    float* e;            // [B][N][h] ds * gelu(z)
+    float* part;         // parameter partial sums
 };
 
 struct MergeWorkspace {
-    size_t rank, members, goff, ds, dh, gz, part, total;
+    size_t flag, members, goff, gstat, g, ds, dh, e, part, total;
 };
 MergeWorkspace merge_workspace_layout(int B, int N, int d, int h, int k);
 size_t merge_smem_bytes(int N, int k, int d, int h);

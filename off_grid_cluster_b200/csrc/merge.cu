@@ -13,8 +13,17 @@
 //   g_i = <dF_j, f_i> + <dX_j, x_i>, ds_i = w_i (g_i - sum_G w g), dx_i = w_i dX_j,
 //   dh_i = ds_i w2 * gelu'(z_i), df_i = w_i dF_j + W1 dh_i,
 //   dW1 = sum_i f_i dh_i^T, db1 = sum dh_i, dw2 = sum ds_i gelu(z_i), db2 = sum ds_i.
-// No atomics in any sum: groups are listed by a sort, every token belongs to one group, and
-// the parameter gradients are reduced in two fixed-order stages.
+// No atomics in any sum: groups are listed by a counting sort whose order within a group is
+// fixed by ranking ids, every token belongs to one group, and the parameter gradients are
+// reduced in two fixed-order stages.
+//
+// Kernels.  Forward: scores (token-parallel, 4 lanes per token, W1 broadcast from shared
+// memory) -> rank by counting (anchor flags) -> assignment (each CTA rebuilds the anchor list
+// from the flags, then a nearest-anchor search with 4 lanes per token) -> groups (counting
+// sort) -> merge (one warp per anchor).  Backward: groups -> group statistics (one warp per
+// anchor: softmax max, 1/sum and sum_G w g) -> token pass (4 lanes per token: g, ds, the MLP
+// backward, dfeats) -> parameter partial sums (4x4 register tiles over token ranges) -> the
+// fixed-order sum of the parts.
 #include <float.h>
 
 #include "internal.h"
@@ -26,96 +35,274 @@ namespace {
 constexpr int kMergeWarps = 8;
 constexpr int kMergeThreads = 32 * kMergeWarps;
 constexpr int kSortThreads = 1024;
-constexpr int kParamParts = 64;   // token ranges of the first parameter-gradient stage
-constexpr int kParamTile = 32;    // tokens staged per step of that stage
+constexpr int kSub = 4;                               // lanes per token (token-parallel kernels)
+constexpr int kTokPerWarp = 32 / kSub;
+constexpr int kTokPerCta = kMergeWarps * kTokPerWarp;
+constexpr int kTokCtasPerSm = 4;                      // grid cap of the token-parallel kernels
+constexpr int kAssignSub = 4;                         // lanes per token in the nearest-anchor search
+constexpr int kParamParts = 296;                      // token ranges of the parameter partial sums
+constexpr int kParamTile = 32;                        // tokens staged per step of that stage
+constexpr size_t kW1SmemMax = 96 * 1024;              // W1 staged in shared memory up to this size
 
 __device__ __forceinline__ float gelu_f(float z) { return 0.5f * z * (1.f + erff(z * 0.70710678118654752f)); }
 __device__ __forceinline__ float gelu_grad_f(float z) {
     return 0.5f * (1.f + erff(z * 0.70710678118654752f)) + z * 0.39894228040143268f * expf(-0.5f * z * z);
 }
 
-__host__ __device__ __forceinline__ int pow2_ge(int n) {
-    int p = 1;
-    while (p < n) p <<= 1;
-    return p;
+// Hidden units are held 8 HP per lane: lane sub-index s (of kSub) owns the float4 groups
+// 4 s + 16 y (y < 2 HP), so the four lanes of a token read 64 contiguous bytes of a W1 row.
+// W1 in shared memory: rows of kHS(HP) floats (h padded with zeros, +4 so that rows two
+// apart start 32 bytes apart in the banks).
+template <int HP>
+constexpr int kHS = 32 * HP + 4;
+
+template <int HP>
+__device__ void stage_w1(float* w1s, const float* __restrict__ w1, int d, int h) {
+#pragma unroll 4
+    for (int i = threadIdx.x; i < d * kHS<HP>; i += blockDim.x) {
+        const int c = i / kHS<HP>, u = i - c * kHS<HP>;
+        w1s[i] = u < h ? w1[static_cast<size_t>(c) * h + u] : 0.f;
+    }
 }
 
-// Hidden pre-activations z_u = b1_u + sum_c f_c W1[c][u] of one token, lane l holding
-// u = l + 32 x (x < HP); f is read as bf16 pairs, two channels per lane, broadcast by shuffles.
-template <int HP>
-__device__ __forceinline__ void hidden_pre(const bf16* frow, int d, const float* w1, const float* b1,
-                                           int h, int lane, float (&z)[HP]) {
-#pragma unroll
-    for (int x = 0; x < HP; ++x) {
-        const int u = lane + 32 * x;
-        z[x] = u < h ? __ldg(b1 + u) : 0.f;
+// W1[c][u0 .. u0 + 3]: from the padded shared copy, or from global memory (rows of h).
+template <bool SM>
+__device__ __forceinline__ float4 w1_load4(const float* w, int stride, int h, int c, int u0) {
+    if constexpr (SM) {
+        return *reinterpret_cast<const float4*>(w + c * stride + u0);
+    } else {
+        const float* row = w + static_cast<size_t>(c) * h;
+        return make_float4(u0 < h ? __ldg(row + u0) : 0.f, u0 + 1 < h ? __ldg(row + u0 + 1) : 0.f,
+                           u0 + 2 < h ? __ldg(row + u0 + 2) : 0.f, u0 + 3 < h ? __ldg(row + u0 + 3) : 0.f);
     }
-    for (int c0 = 0; c0 < d; c0 += 64) {
-        const int c = c0 + 2 * lane;
-        uint32_t pair = 0u;
-        if (c < d) pair = *reinterpret_cast<const uint32_t*>(frow + c);
-        const int cn = min(64, d - c0);
-        for (int cc = 0; cc < cn; ++cc) {
-            const uint32_t pw = __shfl_sync(0xffffffffu, pair, cc >> 1);
-            const float fc = (cc & 1) ? bf16_hi(pw) : bf16_lo(pw);
-            const float* wr = w1 + static_cast<size_t>(c0 + cc) * h;
+}
+
+// Pre-activations z = b1 + W1^T f of one token for the units lane s owns (zero beyond h).
+template <int HP, bool SM>
+__device__ __forceinline__ void hidden4(const bf16* frow, int d, const float* w, int h,
+                                        const float* b1s, int s, float (&z)[8 * HP]) {
 #pragma unroll
-            for (int x = 0; x < HP; ++x) {
-                const int u = lane + 32 * x;
-                if (u < h) z[x] = fmaf(fc, __ldg(wr + u), z[x]);
+    for (int y = 0; y < 2 * HP; ++y) {
+        const float4 b = *reinterpret_cast<const float4*>(b1s + 4 * s + 16 * y);
+        z[4 * y] = b.x;
+        z[4 * y + 1] = b.y;
+        z[4 * y + 2] = b.z;
+        z[4 * y + 3] = b.w;
+    }
+    // 32 channels per step (d % 32 == 0), the next step's four 16-byte chunks loaded ahead
+    uint4 cur[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) cur[q] = ldg16(frow + 8 * q);
+    for (int c0 = 0; c0 < d; c0 += 32) {
+        uint4 nxt[4];
+        if (c0 + 32 < d) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) nxt[q] = ldg16(frow + c0 + 32 + 8 * q);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t fw[4] = {cur[q].x, cur[q].y, cur[q].z, cur[q].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float fc = (e & 1) ? bf16_hi(fw[e >> 1]) : bf16_lo(fw[e >> 1]);
+                const int c = c0 + 8 * q + e;
+#pragma unroll
+                for (int y = 0; y < 2 * HP; ++y) {
+                    const float4 w4 = w1_load4<SM>(w, kHS<HP>, h, c, 4 * s + 16 * y);
+                    z[4 * y] = fmaf(fc, w4.x, z[4 * y]);
+                    z[4 * y + 1] = fmaf(fc, w4.y, z[4 * y + 1]);
+                    z[4 * y + 2] = fmaf(fc, w4.z, z[4 * y + 2]);
+                    z[4 * y + 3] = fmaf(fc, w4.w, z[4 * y + 3]);
+                }
             }
+        }
+        if (c0 + 32 < d) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
         }
     }
 }
 
-// 1. scores: one warp per token.
+// b1 and w2 in shared memory, zero beyond h.
 template <int HP>
+__device__ __forceinline__ void stage_bias(float* b1s, float* w2s, const float* __restrict__ b1,
+                                           const float* __restrict__ w2, int h) {
+    for (int u = threadIdx.x; u < 32 * HP; u += blockDim.x) {
+        b1s[u] = u < h ? b1[u] : 0.f;
+        w2s[u] = u < h ? w2[u] : 0.f;
+    }
+}
+
+// 1. scores: four lanes per token, eight tokens per warp, warps striding over the tokens.
+template <int HP, bool SM>
 __global__ void __launch_bounds__(kMergeThreads)
     merge_scores_kernel(const bf16* __restrict__ feats, int T, int d, const float* __restrict__ w1,
                         const float* __restrict__ b1, const float* __restrict__ w2, float b2, int h,
                         float* __restrict__ scores) {
-    const int lane = threadIdx.x & 31;
-    const long long t = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
-    if (t >= T) return;  // whole warps
-    float z[HP];
-    hidden_pre<HP>(feats + static_cast<size_t>(t) * d, d, w1, b1, h, lane, z);
-    float s = 0.f;
+    extern __shared__ __align__(16) float w1s[];  // [d][kHS] when SM
+    __shared__ __align__(16) float b1s[32 * HP];
+    __shared__ __align__(16) float w2s[32 * HP];
+    stage_bias<HP>(b1s, w2s, b1, w2, h);
+    if constexpr (SM) stage_w1<HP>(w1s, w1, d, h);
+    __syncthreads();
+    const float* w = SM ? w1s : w1;
+    const int lane = threadIdx.x & 31, s = lane & (kSub - 1), tw = lane / kSub;
+    const int warp_g = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+    for (int base = warp_g * kTokPerWarp; base < T; base += gridDim.x * kTokPerCta) {  // warp-uniform
+        const int t = base + tw;
+        const bool live = t < T;
+        float z[8 * HP];
+        hidden4<HP, SM>(feats + static_cast<size_t>(live ? t : base) * d, d, w, h, b1s, s, z);
+        float acc = 0.f;
 #pragma unroll
-    for (int x = 0; x < HP; ++x) {
-        const int u = lane + 32 * x;
-        if (u < h) s = fmaf(__ldg(w2 + u), gelu_f(z[x]), s);
+        for (int y = 0; y < 2 * HP; ++y)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc = fmaf(w2s[4 * s + 16 * y + e], gelu_f(z[4 * y + e]), acc);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (live && s == 0) scores[t] = acc + b2;
     }
-    s = warp_sum(s);
-    if (lane == 0) scores[t] = s + b2;
 }
 
+// Order-preserving map of an fp32 score to uint32 (-0 and +0 equal).
 __device__ __forceinline__ uint32_t order_bits_f(float f) {
     uint32_t u = __float_as_uint(f);
     if ((u & 0x7FFFFFFFu) == 0) u = 0;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Ascending bitonic sort of P u64 keys in shared memory by the whole block.
-__device__ void bitonic_u64(uint64_t* keys, int P) {
-    for (int k = 2; k <= P; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = threadIdx.x; i < P; i += blockDim.x) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const uint64_t a = keys[i], b = keys[ixj];
-                    if ((a > b) == ((i & k) == 0)) {
-                        keys[i] = b;
-                        keys[ixj] = a;
-                    }
-                }
-            }
-            __syncthreads();
+// 2. anchors by counting: token i is ranked after every j with a larger score, or an equal
+//    score and a lower id; it is an anchor when fewer than k tokens rank ahead of it.
+//    kSub lanes per token, lane s over the 16-byte groups of scores = s (mod kSub).
+//    flag[i] = 1 for anchors, else 0.
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_rank_kernel(const float* __restrict__ scores, int N, int k, int32_t* __restrict__ flag) {
+    extern __shared__ __align__(16) uint32_t ord[];  // [N rounded up to 4], zero padding
+    const int b = blockIdx.y;
+    const float* sb = scores + static_cast<size_t>(b) * N;
+    const int N4 = (N + 3) & ~3;
+    for (int j = threadIdx.x; j < N4; j += kMergeThreads) ord[j] = j < N ? order_bits_f(sb[j]) : 0u;
+    __syncthreads();
+    const int s = threadIdx.x & (kSub - 1);
+    const int i = (blockIdx.x * kMergeThreads + threadIdx.x) / kSub;
+    const int iw = i & ~(kTokPerWarp - 1);  // first token of this warp (a multiple of 8)
+    if (iw >= N) return;                    // whole warps
+    const uint32_t oi = i < N ? ord[i] : 0u;
+    int ahead = 0;
+    for (int g = s; g < iw / 4; g += kSub) {  // j < i: ahead iff o_j >= o_i
+        const uint4 o = *reinterpret_cast<const uint4*>(ord + 4 * g);
+        ahead += (o.x >= oi) + (o.y >= oi) + (o.z >= oi) + (o.w >= oi);
+    }
+    if (s == 0) {
+        const int wend = min(iw + kTokPerWarp, N);
+        for (int j = iw; j < wend; ++j) {
+            const uint32_t o = ord[j];
+            ahead += (o > oi) || (o == oi && j < i);
         }
     }
+    for (int g = (iw + kTokPerWarp) / 4 + s; g < N4 / 4; g += kSub) {  // j > i: o_j > o_i (padding 0)
+        const uint4 o = *reinterpret_cast<const uint4*>(ord + 4 * g);
+        ahead += (o.x > oi) + (o.y > oi) + (o.z > oi) + (o.w > oi);
+    }
+    ahead += __shfl_xor_sync(0xffffffffu, ahead, 1);
+    ahead += __shfl_xor_sync(0xffffffffu, ahead, 2);
+    if (i < N && s == 0) flag[static_cast<size_t>(b) * N + i] = ahead < k ? 1 : 0;
 }
 
-// Exclusive prefix sum of data[0..n) by the whole block; returns the total.
-__device__ int merge_scan(int* data, int n, int* scratch) {
+// 3. assignment.  Every CTA rebuilds its image's anchor list (ascending id) from the flags
+//    by a block scan; CTA 0 of the image writes it out.  Then kAssignSub lanes per token, lane
+//    p scanning anchors j = p (mod kAssignSub) with an fp32 prefilter and the exact fp64
+//    decision; the lanes' bests are combined by (fp64 distance, anchor id).
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_assign_kernel(const float* __restrict__ xy, int N, int k, const int32_t* __restrict__ flag,
+                        int32_t* __restrict__ anchors, int32_t* __restrict__ assign) {
+    extern __shared__ __align__(16) float2 axy[];  // [k]
+    constexpr int kTok = kMergeThreads / kAssignSub;
+    __shared__ int wsum[kMergeWarps];
+    __shared__ int myrank[kTok];
+    const int b = blockIdx.y, i0 = blockIdx.x * kTok;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float2* xb = reinterpret_cast<const float2*>(xy) + static_cast<size_t>(b) * N;
+    const int32_t* fb = flag + static_cast<size_t>(b) * N;
+    const int per = (N + kMergeThreads - 1) / kMergeThreads;
+    const int j0 = min(N, threadIdx.x * per), j1 = min(N, j0 + per);
+    int cnt = 0;
+    for (int jb = j0; jb < j1; jb += 8) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) cnt += (jb + q < j1) ? (fb[jb + q] != 0) : 0;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int r = incl - cnt;
+    for (int w = 0; w < warp; ++w) r += wsum[w];
+    for (int jb = j0; jb < j1; jb += 8) {  // flags and coordinates of 8 tokens loaded at once
+        int f8[8];
+        float2 p8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            f8[q] = (jb + q < j1) ? fb[jb + q] : 0;
+            p8[q] = (jb + q < j1) ? xb[jb + q] : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int j = jb + q;
+            if (j >= j1) break;
+            const bool is_anchor = f8[q] != 0 && r < k;
+            if (j >= i0 && j < i0 + kTok) myrank[j - i0] = is_anchor ? r : -1;
+            if (is_anchor) {
+                axy[r] = p8[q];
+                if (blockIdx.x == 0) anchors[static_cast<size_t>(b) * k + r] = j;
+                ++r;
+            }
+        }
+    }
+    __syncthreads();
+    const int sub = threadIdx.x % kAssignSub;
+    const int i = i0 + threadIdx.x / kAssignSub;
+    const bool live = i < N;
+    const int ri = live ? myrank[i - i0] : 0;
+    const float2 p = live ? xb[i] : make_float2(0.f, 0.f);
+    const double px = p.x, py = p.y;
+    double best = DBL_MAX;
+    float bestf = FLT_MAX;
+    int bj = 0x7fffffff;
+    if (live && ri < 0) {
+        for (int j = sub; j < k; j += kAssignSub) {
+            const float2 a = axy[j];
+            const float dxf = p.x - a.x, dyf = p.y - a.y;
+            const float d2f = fmaf(dxf, dxf, dyf * dyf);
+            if (d2f <= bestf) {   // a candidate beyond the fp32 bound cannot be nearer in fp64
+                const double dx = __dsub_rn(px, static_cast<double>(a.x));
+                const double dy = __dsub_rn(py, static_cast<double>(a.y));
+                const double d2 = __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy));
+                if (d2 < best) {  // strict: ties keep the lower anchor id
+                    best = d2;
+                    bj = j;
+                    bestf = static_cast<float>(best) * (1.0f + 1.0f / 1048576.0f);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 1; o < kAssignSub; o <<= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+        if (ob < best || (ob == best && oj < bj)) {
+            best = ob;
+            bj = oj;
+        }
+    }
+    if (live && sub == 0) assign[static_cast<size_t>(b) * N + i] = ri >= 0 ? ri : bj;
+}
+
+// Exclusive prefix sum of data[0..n) by the whole block; data[n] = the total.
+__device__ void block_scan_excl(int* data, int n, int* scratch) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int per = (n + blockDim.x - 1) / blockDim.x;
     const int p0 = tid * per;
@@ -150,121 +337,81 @@ __device__ int merge_scan(int* data, int n, int* scratch) {
             run += v;
         }
     }
-    const int total = scratch[32];
+    if (tid == 0) data[n] = scratch[32];
     __syncthreads();
-    return total;
 }
 
-// 2. anchors: per image, the k largest scores (ties by id), listed by ascending id; rank[i]
-//    = the anchor rank of token i, or -1.
-__global__ void __launch_bounds__(kSortThreads)
-    merge_topk_kernel(const float* __restrict__ scores, int N, int k, int32_t* __restrict__ anchors,
-                      int32_t* __restrict__ rank) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int b = blockIdx.x, P = pow2_ge(N);
-    uint64_t* keys = reinterpret_cast<uint64_t*>(smem);          // [P]
-    int* flag = reinterpret_cast<int*>(keys + P);                 // [N]
-    int* scratch = flag + N;                                      // [40]
-    const float* sb = scores + static_cast<size_t>(b) * N;
-    for (int i = threadIdx.x; i < P; i += kSortThreads)
-        keys[i] = i < N ? ((static_cast<uint64_t>(~order_bits_f(sb[i])) << 32) | static_cast<uint32_t>(i))
-                        : ~0ull;
-    __syncthreads();
-    bitonic_u64(keys, P);   // ascending: score descending, then id ascending
-    for (int i = threadIdx.x; i < N; i += kSortThreads) flag[i] = 0;
-    __syncthreads();
-    for (int j = threadIdx.x; j < k; j += kSortThreads) flag[keys[j] & 0xffffffffu] = 1;
-    __syncthreads();
-    merge_scan(flag, N, scratch);   // flag[i] = number of anchors with a smaller id
-    int32_t* ab = anchors + static_cast<size_t>(b) * k;
-    int32_t* rb = rank + static_cast<size_t>(b) * N;
-    for (int i = threadIdx.x; i < N; i += kSortThreads) {
-        const int before = flag[i];
-        const int after = i + 1 < N ? flag[i + 1] : k;
-        const bool is_anchor = after > before;
-        rb[i] = is_anchor ? before : -1;
-        if (is_anchor) ab[before] = i;
-    }
-}
-
-// 3. assignment: one thread per token; the CTA holds its image's anchor coordinates.
-__global__ void __launch_bounds__(kMergeThreads)
-    merge_assign_kernel(const float* __restrict__ xy, int N, int k, const int32_t* __restrict__ anchors,
-                        const int32_t* __restrict__ rank, int32_t* __restrict__ assign) {
-    extern __shared__ __align__(16) float2 axy[];  // [k]
-    const int b = blockIdx.y;
-    const float2* xb = reinterpret_cast<const float2*>(xy) + static_cast<size_t>(b) * N;
-    const int32_t* ab = anchors + static_cast<size_t>(b) * k;
-    for (int j = threadIdx.x; j < k; j += kMergeThreads) axy[j] = xb[ab[j]];
-    __syncthreads();
-    const int i = blockIdx.x * kMergeThreads + threadIdx.x;
-    if (i >= N) return;
-    const int r = rank[static_cast<size_t>(b) * N + i];
-    if (r >= 0) {
-        assign[static_cast<size_t>(b) * N + i] = r;
-        return;
-    }
-    const float2 p = xb[i];
-    const double px = p.x, py = p.y;
-    double best = DBL_MAX;
-    float bestf = FLT_MAX;
-    int bj = 0;
-    for (int j = 0; j < k; ++j) {
-        const float2 a = axy[j];
-        const float dxf = p.x - a.x, dyf = p.y - a.y;
-        const float d2f = fmaf(dxf, dxf, dyf * dyf);
-        if (d2f <= bestf) {   // a candidate beyond the fp32 bound cannot be nearer in fp64
-            const double dx = __dsub_rn(px, static_cast<double>(a.x));
-            const double dy = __dsub_rn(py, static_cast<double>(a.y));
-            const double d2 = __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy));
-            if (d2 < best) {  // strict: ties keep the lower anchor id
-                best = d2;
-                bj = j;
-                bestf = static_cast<float>(best) * (1.0f + 1.0f / 1048576.0f);
-            }
-        }
-    }
-    assign[static_cast<size_t>(b) * N + i] = bj;
-}
-
-// 4. groups: per image, the tokens sorted by (assign, id) -> members [N] and the group
-//    offsets goff [k + 1].
+// 4. groups: per image, a counting sort of the tokens by assignment -> members [N] (each
+//    group's tokens by ascending id) and the offsets goff [k + 1].  Slots taken by shared-
+//    memory atomics only place a token in its group's segment; its final position is its rank
+//    by id within the group, so the result does not depend on the atomics' order.  A token
+//    whose assignment is outside [0, k) is left out.
 __global__ void __launch_bounds__(kSortThreads)
     merge_groups_kernel(const int32_t* __restrict__ assign, int N, int k, int32_t* __restrict__ members,
                         int32_t* __restrict__ goff) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int b = blockIdx.x, P = pow2_ge(N);
-    uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
+    extern __shared__ __align__(16) int gsm[];
+    int* cnt = gsm;              // [k + 1]
+    int* slot = cnt + k + 1;     // [N]
+    int* seg = slot + N;         // [N]
+    __shared__ int scratch[40];
+    const int b = blockIdx.x;
     const int32_t* ab = assign + static_cast<size_t>(b) * N;
-    for (int i = threadIdx.x; i < P; i += kSortThreads)
-        keys[i] = i < N ? ((static_cast<uint64_t>(static_cast<uint32_t>(ab[i])) << 32) | static_cast<uint32_t>(i))
-                        : ~0ull;
+    for (int j = threadIdx.x; j <= k; j += kSortThreads) cnt[j] = 0;
     __syncthreads();
-    bitonic_u64(keys, P);
-    int32_t* mb = members + static_cast<size_t>(b) * N;
-    int32_t* gb = goff + static_cast<size_t>(b) * (k + 1);
     for (int i = threadIdx.x; i < N; i += kSortThreads) {
-        const int a = static_cast<int>(keys[i] >> 32);
-        mb[i] = static_cast<int32_t>(keys[i] & 0xffffffffu);
-        const int prev = i > 0 ? static_cast<int>(keys[i - 1] >> 32) : -1;
-        for (int g = prev + 1; g <= a; ++g) gb[g] = i;   // every group holds its anchor
+        const int a = ab[i];
+        slot[i] = (a >= 0 && a < k) ? atomicAdd(&cnt[a], 1) : -1;
     }
-    if (threadIdx.x == 0) gb[k] = N;
+    __syncthreads();
+    block_scan_excl(cnt, k, scratch);
+    int32_t* gb = goff + static_cast<size_t>(b) * (k + 1);
+    for (int j = threadIdx.x; j <= k; j += kSortThreads) gb[j] = cnt[j];
+    for (int i = threadIdx.x; i < N; i += kSortThreads)
+        if (slot[i] >= 0) seg[cnt[ab[i]] + slot[i]] = i;
+    __syncthreads();
+    int32_t* mb = members + static_cast<size_t>(b) * N;
+    for (int i = threadIdx.x; i < N; i += kSortThreads) {
+        if (slot[i] < 0) continue;
+        const int a = ab[i], s0 = cnt[a], n = cnt[a + 1] - s0;
+        int pos = 0;
+        for (int x = 0; x < n; ++x) pos += seg[s0 + x] < i;
+        mb[s0 + pos] = i;
+    }
 }
 
-// Softmax weights of a group's members, lanes over members (groups of any size).
+// Softmax of a group's scores, lanes over members: max m, inv = 1 / sum_x exp(s_x - m) (lane
+// x adding members x, x + 32, ... in order, then a butterfly sum); member x's weight is
+// exp(s_x - m) * inv.
 __device__ __forceinline__ void group_softmax(const float* sb, const int32_t* mem, int n, int lane,
-                                              float& gmax, float& gsum) {
+                                              float& gmax, float& inv) {
     float m = -FLT_MAX;
     for (int x = lane; x < n; x += 32) m = fmaxf(m, sb[mem[x]]);
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float s = 0.f;
     for (int x = lane; x < n; x += 32) s += expf(sb[mem[x]] - m);
-    gsum = warp_sum(s);
     gmax = m;
+    inv = 1.f / warp_sum(s);
 }
 
-// 5. forward merge: one warp per anchor; lanes over channel pairs.
+// Members x0 + lane of a group (token id, weight, coordinates), 0 beyond n.
+struct MemberLane {
+    int t;
+    float w;
+    float2 p;
+};
+__device__ __forceinline__ MemberLane member_lane(const float* sb, const float2* xb, const int32_t* mem,
+                                                  int x, int n, float gmax, float inv) {
+    MemberLane r{0, 0.f, make_float2(0.f, 0.f)};
+    if (x < n) {
+        r.t = mem[x];
+        r.w = expf(sb[r.t] - gmax) * inv;
+        r.p = xb[r.t];
+    }
+    return r;
+}
+
+// 5. forward merge: one warp per anchor; members in rounds of 32 (lane x holding member x's
+//    id and weight), lanes over 4-channel groups.
 __global__ void __launch_bounds__(kMergeThreads)
     merge_fwd_kernel(const bf16* __restrict__ feats, const float* __restrict__ xy, int B, int N, int d,
                      int k, const float* __restrict__ scores, const int32_t* __restrict__ members,
@@ -274,216 +421,344 @@ __global__ void __launch_bounds__(kMergeThreads)
     if (ga >= static_cast<long long>(B) * k) return;
     const int b = static_cast<int>(ga / k), j = static_cast<int>(ga - static_cast<long long>(b) * k);
     const float* sb = scores + static_cast<size_t>(b) * N;
-    const int32_t* mem = members + static_cast<size_t>(b) * N;
     const int32_t* gb = goff + static_cast<size_t>(b) * (k + 1);
     const int g0 = gb[j], n = gb[j + 1] - g0;
-    float gmax, gsum;
-    group_softmax(sb, mem + g0, n, lane, gmax, gsum);
-    const float inv = 1.f / gsum;
+    const int32_t* mem = members + static_cast<size_t>(b) * N + g0;
+    const float2* xb = reinterpret_cast<const float2*>(xy) + static_cast<size_t>(b) * N;
+    float gmax, inv;
+    group_softmax(sb, mem, n, lane, gmax, inv);
     const bf16* fb = feats + static_cast<size_t>(b) * N * d;
-    for (int c0 = 0; c0 < d; c0 += 64) {
-        const int c = c0 + 2 * lane;
-        float a0 = 0.f, a1 = 0.f;
-        for (int x = 0; x < n; ++x) {
-            const int t = mem[g0 + x];
-            const float w = expf(sb[t] - gmax) * inv;
-            if (c < d) {
-                const uint32_t pr = *reinterpret_cast<const uint32_t*>(fb + static_cast<size_t>(t) * d + c);
-                a0 = fmaf(w, bf16_lo(pr), a0);
-                a1 = fmaf(w, bf16_hi(pr), a1);
+    bf16* out = merged + static_cast<size_t>(ga) * d;
+    float mx = 0.f, my = 0.f;
+    for (int c0 = 0; c0 < d; c0 += 128) {
+        const int c = c0 + 4 * lane;
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int x0 = 0; x0 < n; x0 += 32) {
+            const MemberLane ml = member_lane(sb, xb, mem, x0 + lane, n, gmax, inv);
+            if (c0 == 0) {
+                mx = fmaf(ml.w, ml.p.x, mx);
+                my = fmaf(ml.w, ml.p.y, my);
+            }
+            const int nn = min(32, n - x0);
+            for (int x = 0; x < nn; ++x) {
+                const int t = __shfl_sync(0xffffffffu, ml.t, x);
+                const float w = __shfl_sync(0xffffffffu, ml.w, x);
+                if (c < d) {
+                    const uint2 pr = *reinterpret_cast<const uint2*>(fb + static_cast<size_t>(t) * d + c);
+                    a[0] = fmaf(w, bf16_lo(pr.x), a[0]);
+                    a[1] = fmaf(w, bf16_hi(pr.x), a[1]);
+                    a[2] = fmaf(w, bf16_lo(pr.y), a[2]);
+                    a[3] = fmaf(w, bf16_hi(pr.y), a[3]);
+                }
             }
         }
         if (c < d) {
-            const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
-            *reinterpret_cast<__nv_bfloat162*>(merged + (static_cast<size_t>(b) * k + j) * d + c) = hv;
+            uint2 o;
+            o.x = pack_bf16(a[0], a[1]);
+            o.y = pack_bf16(a[2], a[3]);
+            *reinterpret_cast<uint2*>(out + c) = o;
         }
     }
-    if (lane < 2) {
-        const float2* xb = reinterpret_cast<const float2*>(xy) + static_cast<size_t>(b) * N;
-        float acc = 0.f;
-        for (int x = 0; x < n; ++x) {
-            const int t = mem[g0 + x];
-            const float2 p = xb[t];
-            acc = fmaf(expf(sb[t] - gmax) * inv, lane ? p.y : p.x, acc);
-        }
-        mxy[(static_cast<size_t>(b) * k + j) * 2 + lane] = acc;
-    }
+    mx = warp_sum(mx);
+    my = warp_sum(my);
+    if (lane == 0) reinterpret_cast<float2*>(mxy)[ga] = make_float2(mx, my);
 }
 
-// 6. backward per group: one warp per anchor, its members in order.  Writes dfeats (bf16),
-//    dcoords, and per token ds and dh (fp32, workspace) for the parameter gradients.
-template <int HP>
+// 6. backward group statistics: one warp per anchor -> gstat = {max score, 1 / sum of
+//    exp(s - max), sum_G w g} with g_i = <dF_j, f_i> + <dX_j, x_i> (members four at a time,
+//    lanes over 4-channel groups, then butterfly sums), summed in member order; g_i is stored
+//    so that the token pass uses the very values summed here (a one-token group then gets
+//    ds = 0 exactly).
 __global__ void __launch_bounds__(kMergeThreads)
-    merge_bwd_group_kernel(const bf16* __restrict__ feats, const float* __restrict__ xy, int B, int N,
-                           int d, int k, const float* __restrict__ w1, const float* __restrict__ b1,
-                           const float* __restrict__ w2, int h, const float* __restrict__ scores,
-                           const int32_t* __restrict__ members, const int32_t* __restrict__ goff,
-                           const bf16* __restrict__ dmerged, const float* __restrict__ dmxy,
-                           bf16* __restrict__ dfeats, float* __restrict__ dxy, float* __restrict__ ds_out,
-                           float* __restrict__ dh_out, float* __restrict__ gz_out) {
+    merge_gstat_kernel(const bf16* __restrict__ feats, const float* __restrict__ xy, int B, int N, int d,
+                       int k, const float* __restrict__ scores, const int32_t* __restrict__ members,
+                       const int32_t* __restrict__ goff, const bf16* __restrict__ dmerged,
+                       const float* __restrict__ dmxy, float4* __restrict__ gstat,
+                       float* __restrict__ g_out) {
     const int lane = threadIdx.x & 31;
     const long long ga = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
     if (ga >= static_cast<long long>(B) * k) return;
     const int b = static_cast<int>(ga / k), j = static_cast<int>(ga - static_cast<long long>(b) * k);
     const float* sb = scores + static_cast<size_t>(b) * N;
-    const int32_t* mem = members + static_cast<size_t>(b) * N;
     const int32_t* gb = goff + static_cast<size_t>(b) * (k + 1);
     const int g0 = gb[j], n = gb[j + 1] - g0;
-    float gmax, gsum;
-    group_softmax(sb, mem + g0, n, lane, gmax, gsum);
-    const float inv = 1.f / gsum;
-    const bf16* fb = feats + static_cast<size_t>(b) * N * d;
-    const bf16* dF = dmerged + (static_cast<size_t>(b) * k + j) * d;
-    const float dX0 = dmxy[(static_cast<size_t>(b) * k + j) * 2], dX1 = dmxy[(static_cast<size_t>(b) * k + j) * 2 + 1];
+    const int32_t* mem = members + static_cast<size_t>(b) * N + g0;
     const float2* xb = reinterpret_cast<const float2*>(xy) + static_cast<size_t>(b) * N;
-    // sum_G w g, g_i = <dF, f_i> + <dX, x_i>
+    float gmax, inv;
+    group_softmax(sb, mem, n, lane, gmax, inv);
+    const bf16* fb = feats + static_cast<size_t>(b) * N * d;
+    const bf16* dF = dmerged + static_cast<size_t>(ga) * d;
+    const float2 dX = reinterpret_cast<const float2*>(dmxy)[ga];
+    float* gb_out = g_out + static_cast<size_t>(b) * N;
     float sg = 0.f;
-    for (int x = 0; x < n; ++x) {
-        const int t = mem[g0 + x];
-        float acc = 0.f;
-        for (int c = 2 * lane; c < d; c += 64) {
-            const uint32_t pf = *reinterpret_cast<const uint32_t*>(fb + static_cast<size_t>(t) * d + c);
-            const uint32_t pg = *reinterpret_cast<const uint32_t*>(dF + c);
-            acc = fmaf(bf16_lo(pf), bf16_lo(pg), acc);
-            acc = fmaf(bf16_hi(pf), bf16_hi(pg), acc);
-        }
-        const float2 p = xb[t];
-        const float gi = warp_sum(acc) + dX0 * p.x + dX1 * p.y;
-        sg = fmaf(expf(sb[t] - gmax) * inv, gi, sg);
-    }
-    for (int x = 0; x < n; ++x) {
-        const int t = mem[g0 + x];
-        const size_t gt = static_cast<size_t>(b) * N + t;
-        const bf16* frow = fb + static_cast<size_t>(t) * d;
-        float acc = 0.f;
-        for (int c = 2 * lane; c < d; c += 64) {
-            const uint32_t pf = *reinterpret_cast<const uint32_t*>(frow + c);
-            const uint32_t pg = *reinterpret_cast<const uint32_t*>(dF + c);
-            acc = fmaf(bf16_lo(pf), bf16_lo(pg), acc);
-            acc = fmaf(bf16_hi(pf), bf16_hi(pg), acc);
-        }
-        const float2 p = xb[t];
-        const float gi = warp_sum(acc) + dX0 * p.x + dX1 * p.y;
-        const float w = expf(sb[t] - gmax) * inv;
-        const float ds = w * (gi - sg);
-        // MLP backward of this token
-        float z[HP], dh[HP];
-        hidden_pre<HP>(frow, d, w1, b1, h, lane, z);
+    for (int x0 = 0; x0 < n; x0 += 32) {
+        const MemberLane ml = member_lane(sb, xb, mem, x0 + lane, n, gmax, inv);
+        const int nn = min(32, n - x0);
+        for (int x1 = 0; x1 < nn; x1 += 4) {
+            int tq[4];
+            float part[4];
 #pragma unroll
-        for (int y = 0; y < HP; ++y) {
-            const int u = lane + 32 * y;
-            dh[y] = u < h ? ds * __ldg(w2 + u) * gelu_grad_f(z[y]) : 0.f;
-            if (u < h) {
-                dh_out[gt * h + u] = dh[y];
-                gz_out[gt * h + u] = gelu_f(z[y]);
+            for (int q = 0; q < 4; ++q) {
+                tq[q] = __shfl_sync(0xffffffffu, ml.t, min(x1 + q, nn - 1));
+                part[q] = 0.f;
             }
-        }
-        if (lane == 0) ds_out[gt] = ds;
-        if (lane < 2) reinterpret_cast<float*>(dxy)[gt * 2 + lane] = w * (lane ? dX1 : dX0);
-        // df = w dF + W1 dh: lane owns channel pairs; dh broadcast by shuffles
-        for (int c0 = 0; c0 < d; c0 += 64) {
-            const int c = c0 + 2 * lane;
-            float a0 = 0.f, a1 = 0.f;
-            if (c < d) {
-                const uint32_t pg = *reinterpret_cast<const uint32_t*>(dF + c);
-                a0 = w * bf16_lo(pg);
-                a1 = w * bf16_hi(pg);
-            }
+            for (int c = 4 * lane; c < d; c += 128) {
+                const uint2 g = *reinterpret_cast<const uint2*>(dF + c);
 #pragma unroll
-            for (int y = 0; y < HP; ++y) {
-                for (int ul = 0; ul < 32; ++ul) {
-                    const int u = ul + 32 * y;
-                    const float dhu = __shfl_sync(0xffffffffu, dh[y], ul);
-                    if (u < h && c < d) {
-                        a0 = fmaf(__ldg(w1 + static_cast<size_t>(c) * h + u), dhu, a0);
-                        a1 = fmaf(__ldg(w1 + static_cast<size_t>(c + 1) * h + u), dhu, a1);
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    const uint2 f = *reinterpret_cast<const uint2*>(fb + static_cast<size_t>(tq[q]) * d + c);
+                    part[q] = fmaf(bf16_lo(f.x), bf16_lo(g.x), part[q]);
+                    part[q] = fmaf(bf16_hi(f.x), bf16_hi(g.x), part[q]);
+                    part[q] = fmaf(bf16_lo(f.y), bf16_lo(g.y), part[q]);
+                    part[q] = fmaf(bf16_hi(f.y), bf16_hi(g.y), part[q]);
                 }
             }
-            if (c < d)
-                *reinterpret_cast<__nv_bfloat162*>(dfeats + gt * d + c) = __floats2bfloat162_rn(a0, a1);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) part[q] += __shfl_xor_sync(0xffffffffu, part[q], o);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int x = x1 + q;
+                const float px = __shfl_sync(0xffffffffu, ml.p.x, min(x, nn - 1));
+                const float py = __shfl_sync(0xffffffffu, ml.p.y, min(x, nn - 1));
+                const float wq = __shfl_sync(0xffffffffu, ml.w, min(x, nn - 1));
+                if (x < nn) {
+                    const float gi = part[q] + dX.x * px + dX.y * py;
+                    if (lane == 0) gb_out[tq[q]] = gi;
+                    sg = fmaf(wq, gi, sg);
+                }
+            }
         }
+    }
+    if (lane == 0) gstat[ga] = make_float4(gmax, inv, sg, 0.f);
+}
+
+// 7. backward token pass: four lanes per token.  w = exp(s - max) / sum, g from the group
+//    statistics pass, ds = w (g - sum_G w g), dx = w dX;
+//    z again, dh = ds w2 gelu'(z) and e = ds gelu(z) for the lane's units (written for the
+//    parameter sums, and dh to shared memory for the token's four lanes); then dfeats = w dF
+//    + W1 dh with lane s on the channel pairs 8 m + 2 s.  A token whose assignment is outside
+//    [0, k) gets w = 0, so all its gradients are zero.
+template <int HP, bool SM>
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_bwd_token_kernel(const bf16* __restrict__ feats, const float* __restrict__ xy, int T, int N,
+                           int d, int k, int h, const float* __restrict__ w1, const float* __restrict__ b1,
+                           const float* __restrict__ w2, const float* __restrict__ scores,
+                           const int32_t* __restrict__ assign, const float4* __restrict__ gstat,
+                           const float* __restrict__ gtok, const bf16* __restrict__ dmerged, const float* __restrict__ dmxy,
+                           bf16* __restrict__ dfeats, float* __restrict__ dxy, float* __restrict__ ds_out,
+                           float* __restrict__ dh_out, float* __restrict__ e_out) {
+    constexpr int HS = kHS<HP>;
+    extern __shared__ __align__(16) float dyn[];
+    float* dhs = dyn;                                 // [kTokPerCta][HS]
+    float* w1s = dyn + kTokPerCta * HS;               // [d][HS] when SM
+    __shared__ __align__(16) float b1s[32 * HP];
+    __shared__ __align__(16) float w2s[32 * HP];
+    stage_bias<HP>(b1s, w2s, b1, w2, h);
+    if constexpr (SM) stage_w1<HP>(w1s, w1, d, h);
+    __syncthreads();
+    const float* w = SM ? w1s : w1;
+    const int lane = threadIdx.x & 31, s = lane & (kSub - 1), tw = lane / kSub;
+    float* mydh = dhs + ((threadIdx.x >> 5) * kTokPerWarp + tw) * HS;
+    const int h4 = (h + 3) & ~3;
+    const int warp_g = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+    for (int base = warp_g * kTokPerWarp; base < T; base += gridDim.x * kTokPerCta) {  // warp-uniform
+        const int t0 = base + tw;
+        const bool live = t0 < T;
+        const int t = live ? t0 : base;
+        const int b = t / N;
+        const int a = assign[t];
+        const bool ok = live && a >= 0 && a < k;
+        const size_t ga = static_cast<size_t>(b) * k + (ok ? a : 0);
+        const float4 gs = gstat[ga];
+        const float wt = ok ? expf(scores[t] - gs.x) * gs.y : 0.f;
+        const bf16* frow = feats + static_cast<size_t>(t) * d;
+        const bf16* dF = dmerged + ga * d;
+        const float2 dX = reinterpret_cast<const float2*>(dmxy)[ga];
+        const float ds = ok ? wt * (gtok[t] - gs.z) : 0.f;
+        float z[8 * HP];
+        hidden4<HP, SM>(frow, d, w, h, b1s, s, z);
+#pragma unroll
+        for (int y = 0; y < 2 * HP; ++y) {
+            const int u0 = 4 * s + 16 * y;
+            float dh4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float zz = z[4 * y + e];
+                dh4[e] = ds * w2s[u0 + e] * gelu_grad_f(zz);
+                if (live && u0 + e < h) {
+                    dh_out[static_cast<size_t>(t) * h + u0 + e] = dh4[e];
+                    e_out[static_cast<size_t>(t) * h + u0 + e] = ds * gelu_f(zz);
+                }
+            }
+            *reinterpret_cast<float4*>(mydh + u0) = make_float4(dh4[0], dh4[1], dh4[2], dh4[3]);
+        }
+        if (live && s == 0) {
+            ds_out[t] = ds;
+            reinterpret_cast<float2*>(dxy)[t] = make_float2(wt * dX.x, wt * dX.y);
+        }
+        __syncwarp();
+        for (int c = 2 * s; c < d; c += 2 * kSub) {
+            const uint32_t pg = *reinterpret_cast<const uint32_t*>(dF + c);
+            float a0 = wt * bf16_lo(pg), a1 = wt * bf16_hi(pg);
+#pragma unroll 4
+            for (int u0 = 0; u0 < h4; u0 += 4) {
+                const float4 dh4 = *reinterpret_cast<const float4*>(mydh + u0);
+                const float4 wa = w1_load4<SM>(w, HS, h, c, u0);
+                const float4 wb = w1_load4<SM>(w, HS, h, c + 1, u0);
+                a0 = fmaf(wa.x, dh4.x, a0);
+                a0 = fmaf(wa.y, dh4.y, a0);
+                a0 = fmaf(wa.z, dh4.z, a0);
+                a0 = fmaf(wa.w, dh4.w, a0);
+                a1 = fmaf(wb.x, dh4.x, a1);
+                a1 = fmaf(wb.y, dh4.y, a1);
+                a1 = fmaf(wb.z, dh4.z, a1);
+                a1 = fmaf(wb.w, dh4.w, a1);
+            }
+            if (live)
+                *reinterpret_cast<__nv_bfloat162*>(dfeats + static_cast<size_t>(t) * d + c) =
+                    __floats2bfloat162_rn(a0, a1);
+        }
+        __syncwarp();  // the token's dh is read before the next token overwrites it
     }
 }
 
-// 7. parameter gradients, stage 1: CTA p sums tokens [p T / P, (p + 1) T / P) in order;
-//    thread tid owns outputs o = tid, tid + 256, ... of [dW1 (d*h) | db1 (h) | dw2 (h) | db2].
-__global__ void __launch_bounds__(kMergeThreads)
+// 8. parameter gradients, stage 1: CTA x sums tokens [x T / P, (x + 1) T / P) in order into
+//    4 x 4 register tiles of a (d + 3) x h output matrix: rows c < d give dW1 (left f_c,
+//    right dh), row d gives db1 (left 1, right dh), row d + 1 gives dw2 (left 1, right e),
+//    row d + 2 gives db2 (left ds, column 0).  Part layout [P][dW1 (d*h) | db1 | dw2 | db2].
+__global__ void __launch_bounds__(1024)
     merge_param_part_kernel(const bf16* __restrict__ feats, int T, int d, int h,
                             const float* __restrict__ ds, const float* __restrict__ dh,
-                            const float* __restrict__ gz, float* __restrict__ part) {
-    extern __shared__ __align__(16) float tile[];  // [kParamTile][d] f, then [kParamTile][h] dh, gz
-    float* ft = tile;
-    float* dht = ft + kParamTile * d;
-    float* gzt = dht + kParamTile * h;
-    float* dst = gzt + kParamTile * h;
+                            const float* __restrict__ ev, float* __restrict__ part) {
+    extern __shared__ __align__(16) float tile[];
+    const int h4 = (h + 3) & ~3;
+    float* fs = tile;                        // [kParamTile][d]
+    float* dhs = fs + kParamTile * d;        // [kParamTile][h4]
+    float* es = dhs + kParamTile * h4;       // [kParamTile][h4]
+    float* dss = es + kParamTile * h4;       // [kParamTile]
+    const int RB = d / 4 + 1, CB = h4 / 4;
+    const int tid = blockIdx.y * blockDim.x + threadIdx.x;
+    const bool active = tid < RB * CB;
+    const int rb = tid / CB, cb = tid - rb * CB;
     const int p = blockIdx.x;
     const int t0 = static_cast<int>(static_cast<long long>(p) * T / kParamParts);
     const int t1 = static_cast<int>(static_cast<long long>(p + 1) * T / kParamParts);
-    const int nout = d * h + 2 * h + 1;
-    constexpr int kPer = 16;  // outputs per thread held in registers per pass
-    for (int ob = 0; ob < nout; ob += kMergeThreads * kPer) {
-        float acc[kPer];
+    const int d8 = d / 8;
+    float acc[4][4];
 #pragma unroll
-        for (int q = 0; q < kPer; ++q) acc[q] = 0.f;
-        for (int tt = t0; tt < t1; tt += kParamTile) {
-            const int nt = min(kParamTile, t1 - tt);
-            __syncthreads();
-            for (int i = threadIdx.x; i < nt * d; i += kMergeThreads) {
-                const int r = i / d, c = i - r * d;
-                ft[r * d + c] = __bfloat162float(feats[static_cast<size_t>(tt + r) * d + c]);
-            }
-            for (int i = threadIdx.x; i < nt * h; i += kMergeThreads) {
-                const int r = i / h, u = i - r * h;
-                dht[r * h + u] = dh[static_cast<size_t>(tt + r) * h + u];
-                gzt[r * h + u] = gz[static_cast<size_t>(tt + r) * h + u];
-            }
-            for (int i = threadIdx.x; i < nt; i += kMergeThreads) dst[i] = ds[tt + i];
-            __syncthreads();
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int q = 0; q < kPer; ++q) {
-                const int o = ob + q * kMergeThreads + threadIdx.x;
-                if (o >= nout) continue;
-                float a = acc[q];
-                if (o < d * h) {
-                    const int c = o / h, u = o - c * h;
-                    for (int r = 0; r < nt; ++r) a = fmaf(ft[r * d + c], dht[r * h + u], a);
-                } else if (o < d * h + h) {
-                    const int u = o - d * h;
-                    for (int r = 0; r < nt; ++r) a += dht[r * h + u];
-                } else if (o < d * h + 2 * h) {
-                    const int u = o - d * h - h;
-                    for (int r = 0; r < nt; ++r) a = fmaf(dst[r], gzt[r * h + u], a);
-                } else {
-                    for (int r = 0; r < nt; ++r) a += dst[r];
-                }
-                acc[q] = a;
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int tt = t0; tt < t1; tt += kParamTile) {
+        const int nt = min(kParamTile, t1 - tt);
+        __syncthreads();
+#pragma unroll 4
+        for (int q = threadIdx.x; q < nt * d8; q += blockDim.x) {
+            const int r = q / d8, c8 = q - r * d8;
+            const uint4 v = ldg16(feats + static_cast<size_t>(tt + r) * d + 8 * c8);
+            float* dst = fs + r * d + 8 * c8;
+            *reinterpret_cast<float4*>(dst) = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+            *reinterpret_cast<float4*>(dst + 4) = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+        }
+#pragma unroll 4
+        for (int q = threadIdx.x; q < nt * h4; q += blockDim.x) {
+            const int r = q / h4, u = q - r * h4;
+            const size_t g = static_cast<size_t>(tt + r) * h + u;
+            dhs[q] = u < h ? dh[g] : 0.f;
+            es[q] = u < h ? ev[g] : 0.f;
+        }
+        for (int q = threadIdx.x; q < nt; q += blockDim.x) dss[q] = ds[tt + q];
+        __syncthreads();
+        if (!active) continue;
+        if (rb < RB - 1) {
+            for (int r = 0; r < nt; ++r) {
+                const float4 l = *reinterpret_cast<const float4*>(fs + r * d + 4 * rb);
+                const float4 v = *reinterpret_cast<const float4*>(dhs + r * h4 + 4 * cb);
+                const float lv[4] = {l.x, l.y, l.z, l.w}, rv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(lv[i], rv[j], acc[i][j]);
+            }
+        } else {
+            for (int r = 0; r < nt; ++r) {
+                const float4 v = *reinterpret_cast<const float4*>(dhs + r * h4 + 4 * cb);
+                const float4 e4 = *reinterpret_cast<const float4*>(es + r * h4 + 4 * cb);
+                const float sd = dss[r];
+                acc[0][0] += v.x; acc[0][1] += v.y; acc[0][2] += v.z; acc[0][3] += v.w;
+                acc[1][0] += e4.x; acc[1][1] += e4.y; acc[1][2] += e4.z; acc[1][3] += e4.w;
+                acc[2][0] += sd;
             }
         }
+    }
+    if (!active) return;
+    const size_t nout = static_cast<size_t>(d) * h + 2 * h + 1;
+    float* pp = part + static_cast<size_t>(p) * nout;
 #pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const int o = ob + q * kMergeThreads + threadIdx.x;
-            if (o < nout) part[static_cast<size_t>(p) * nout + o] = acc[q];
+    for (int j = 0; j < 4; ++j) {
+        const int u = 4 * cb + j;
+        if (u >= h) continue;
+        if (rb < RB - 1) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pp[static_cast<size_t>(4 * rb + i) * h + u] = acc[i][j];
+        } else {
+            pp[static_cast<size_t>(d) * h + u] = acc[0][j];
+            pp[static_cast<size_t>(d) * h + h + u] = acc[1][j];
+            if (u == 0) pp[static_cast<size_t>(d) * h + 2 * h] = acc[2][0];
         }
     }
 }
 
-// 8. parameter gradients, stage 2: the parts summed in order.
+// 9. parameter gradients, stage 2: CTA over 32 outputs; warp w sums parts w, w + 8, ... in
+//    order, then the eight warp sums are added in warp order.
 __global__ void __launch_bounds__(kMergeThreads)
     merge_param_reduce_kernel(const float* __restrict__ part, int d, int h, float* __restrict__ dw1,
                               float* __restrict__ db1, float* __restrict__ dw2, float* __restrict__ db2) {
+    __shared__ float red[kMergeWarps][32];
     const int nout = d * h + 2 * h + 1;
-    const int o = blockIdx.x * kMergeThreads + threadIdx.x;
-    if (o >= nout) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int o = blockIdx.x * 32 + lane;
     float a = 0.f;
-    for (int p = 0; p < kParamParts; ++p) a += part[static_cast<size_t>(p) * nout + o];
-    if (o < d * h) dw1[o] = a;
-    else if (o < d * h + h) db1[o - d * h] = a;
-    else if (o < d * h + 2 * h) dw2[o - d * h - h] = a;
-    else *db2 = a;
+    if (o < nout)
+#pragma unroll 8
+        for (int p = warp; p < kParamParts; p += kMergeWarps) a += part[static_cast<size_t>(p) * nout + o];
+    red[warp][lane] = a;
+    __syncthreads();
+    if (warp != 0 || o >= nout) return;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) s += red[w][lane];
+    if (o < d * h) dw1[o] = s;
+    else if (o < d * h + h) db1[o - d * h] = s;
+    else if (o < d * h + 2 * h) dw2[o - d * h - h] = s;
+    else *db2 = s;
 }
 
-size_t sort_smem(int N) { return 8 * static_cast<size_t>(pow2_ge(N)) + 4 * static_cast<size_t>(N) + 40 * 4; }
+int hp_of(int h) { return h <= 32 ? 1 : h <= 64 ? 2 : h <= 128 ? 4 : 8; }
+size_t w1_smem(int d, int h) { return sizeof(float) * static_cast<size_t>(d) * (32 * hp_of(h) + 4); }
+bool w1_in_smem(int d, int h) { return w1_smem(d, h) <= kW1SmemMax; }
+size_t token_smem(int d, int h) {
+    return sizeof(float) * static_cast<size_t>(kTokPerCta) * (32 * hp_of(h) + 4) + (w1_in_smem(d, h) ? w1_smem(d, h) : 0);
+}
+size_t rank_smem(int N) { return 4 * static_cast<size_t>((N + 3) & ~3); }
+size_t groups_smem(int N, int k) { return 4 * (static_cast<size_t>(k) + 1 + 2 * static_cast<size_t>(N)); }
+size_t param_smem(int d, int h) {
+    return sizeof(float) * static_cast<size_t>(kParamTile) * (d + 2 * ((h + 3) & ~3) + 1);
+}
+int param_threads(int d, int h) {
+    const int tiles = (d / 4 + 1) * (((h + 3) & ~3) / 4);
+    return tiles >= 1024 ? 1024 : ((tiles + 31) / 32) * 32;
+}
+unsigned token_ctas(int T) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 148;
+    const long long need = (static_cast<long long>(T) + kTokPerCta - 1) / kTokPerCta;
+    const long long cap = static_cast<long long>(sms) * kTokCtasPerSm;
+    return static_cast<unsigned>(need < cap ? need : cap);
+}
 
 }  // namespace
 
@@ -492,52 +767,85 @@ MergeWorkspace merge_workspace_layout(int B, int N, int d, int h, int k) {
     const size_t T = static_cast<size_t>(B) * N;
     MergeWorkspace w;
     size_t off = 0;
-    w.rank = off;    off += up(sizeof(int32_t) * T);
+    w.flag = off;    off += up(sizeof(int32_t) * T);
     w.members = off; off += up(sizeof(int32_t) * T);
     w.goff = off;    off += up(sizeof(int32_t) * static_cast<size_t>(B) * (k + 1));
+    w.gstat = off;   off += up(sizeof(float) * 4 * static_cast<size_t>(B) * k);
+    w.g = off;       off += up(sizeof(float) * T);
     w.ds = off;      off += up(sizeof(float) * T);
     w.dh = off;      off += up(sizeof(float) * T * h);
-    w.gz = off;      off += up(sizeof(float) * T * h);
+    w.e = off;       off += up(sizeof(float) * T * h);
     w.part = off;    off += up(sizeof(float) * kParamParts * (static_cast<size_t>(d) * h + 2 * h + 1));
     w.total = off;
     return w;
 }
 
 size_t merge_smem_bytes(int N, int k, int d, int h) {
-    const size_t s = sort_smem(N);
-    const size_t a = 8 * static_cast<size_t>(k);
-    const size_t p = sizeof(float) * (static_cast<size_t>(kParamTile) * (d + 2 * h) + kParamTile);
-    size_t m = s > a ? s : a;
-    return m > p ? m : p;
+    const size_t c[] = {w1_in_smem(d, h) ? w1_smem(d, h) : 0, rank_smem(N), 8 * static_cast<size_t>(k),
+                        groups_smem(N, k), token_smem(d, h), param_smem(d, h)};
+    size_t m = 0;
+    for (size_t x : c) m = x > m ? x : m;
+    return m;
 }
 
-#define ACL_HP_SWITCH(h, CALL)                        \
-    switch (((h) + 31) / 32) {                        \
-        case 1: { constexpr int HP = 1; CALL; } break; \
-        case 2: { constexpr int HP = 2; CALL; } break; \
-        case 3: case 4: { constexpr int HP = 4; CALL; } break; \
-        default: { constexpr int HP = 8; CALL; } break; \
+#define ACL_HP_SWITCH(h, CALL)                                 \
+    switch (hp_of(h)) {                                        \
+        case 1: { constexpr int HP = 1; CALL; } break;         \
+        case 2: { constexpr int HP = 2; CALL; } break;         \
+        case 4: { constexpr int HP = 4; CALL; } break;         \
+        default: { constexpr int HP = 8; CALL; } break;        \
     }
+
+template <int HP, bool SM>
+cudaError_t launch_scores(const MergeArgs& m, int T, cudaStream_t st) {
+    const size_t sm = SM ? w1_smem(m.d, m.h) : 0;
+    cudaError_t e = ensure_smem<merge_scores_kernel<HP, SM>>(sm);
+    if (e != cudaSuccess) return e;
+    merge_scores_kernel<HP, SM><<<token_ctas(T), kMergeThreads, sm, st>>>(m.feats, T, m.d, m.w1, m.b1, m.w2,
+                                                                        m.b2, m.h, m.scores);
+    note_launch();
+    return cudaSuccess;
+}
+
+template <int HP, bool SM>
+cudaError_t launch_bwd_token(const MergeArgs& m, int T, cudaStream_t st) {
+    const size_t sm = token_smem(m.d, m.h);
+    cudaError_t e = ensure_smem<merge_bwd_token_kernel<HP, SM>>(sm);
+    if (e != cudaSuccess) return e;
+    merge_bwd_token_kernel<HP, SM><<<token_ctas(T), kMergeThreads, sm, st>>>(
+        m.feats, m.xy, T, m.N, m.d, m.k, m.h, m.w1, m.b1, m.w2, m.scores, m.assign,
+        reinterpret_cast<const float4*>(m.gstat), m.g, m.dmerged, m.dmxy, m.dfeats, m.dxy, m.ds, m.dh, m.e);
+    note_launch();
+    return cudaSuccess;
+}
+
+cudaError_t launch_groups(const MergeArgs& m, cudaStream_t st) {
+    const size_t gsm = groups_smem(m.N, m.k);
+    cudaError_t e = ensure_smem<merge_groups_kernel>(gsm);
+    if (e != cudaSuccess) return e;
+    merge_groups_kernel<<<m.B, kSortThreads, gsm, st>>>(m.assign, m.N, m.k, m.members, m.goff);
+    note_launch();
+    return cudaSuccess;
+}
 
 cudaError_t launch_merge_fwd(const MergeArgs& m, cudaStream_t st) {
     const int T = m.B * m.N;
-    cudaError_t e;
-    const unsigned sblocks = static_cast<unsigned>((T + kMergeWarps - 1) / kMergeWarps);
-    ACL_HP_SWITCH(m.h, (merge_scores_kernel<HP><<<sblocks, kMergeThreads, 0, st>>>(
-                           m.feats, T, m.d, m.w1, m.b1, m.w2, m.b2, m.h, m.scores)));
-    note_launch();
-    const size_t ssm = sort_smem(m.N);
-    if ((e = ensure_smem<merge_topk_kernel>(ssm)) != cudaSuccess) return e;
-    merge_topk_kernel<<<m.B, kSortThreads, ssm, st>>>(m.scores, m.N, m.k, m.anchors, m.rank);
+    cudaError_t e = cudaSuccess;
+    const bool sm = w1_in_smem(m.d, m.h);
+    ACL_HP_SWITCH(m.h, (e = sm ? launch_scores<HP, true>(m, T, st) : launch_scores<HP, false>(m, T, st)));
+    if (e != cudaSuccess) return e;
+    const size_t rsm = rank_smem(m.N);
+    if ((e = ensure_smem<merge_rank_kernel>(rsm)) != cudaSuccess) return e;
+    merge_rank_kernel<<<dim3((m.N + kTokPerCta - 1) / kTokPerCta, m.B), kMergeThreads, rsm, st>>>(
+        m.scores, m.N, m.k, m.flag);
     note_launch();
     const size_t asm_ = 8 * static_cast<size_t>(m.k);
     if ((e = ensure_smem<merge_assign_kernel>(asm_)) != cudaSuccess) return e;
-    merge_assign_kernel<<<dim3((m.N + kMergeThreads - 1) / kMergeThreads, m.B), kMergeThreads, asm_, st>>>(
-        m.xy, m.N, m.k, m.anchors, m.rank, m.assign);
+    constexpr int kAssignTok = kMergeThreads / kAssignSub;
+    merge_assign_kernel<<<dim3((m.N + kAssignTok - 1) / kAssignTok, m.B), kMergeThreads, asm_, st>>>(
+        m.xy, m.N, m.k, m.flag, m.anchors, m.assign);
     note_launch();
-    if ((e = ensure_smem<merge_groups_kernel>(ssm)) != cudaSuccess) return e;
-    merge_groups_kernel<<<m.B, kSortThreads, ssm, st>>>(m.assign, m.N, m.k, m.members, m.goff);
-    note_launch();
+    if ((e = launch_groups(m, st)) != cudaSuccess) return e;
     const long long na = static_cast<long long>(m.B) * m.k;
     merge_fwd_kernel<<<static_cast<unsigned>((na + kMergeWarps - 1) / kMergeWarps), kMergeThreads, 0, st>>>(
         m.feats, m.xy, m.B, m.N, m.d, m.k, m.scores, m.members, m.goff, m.merged, m.mxy);
@@ -547,25 +855,26 @@ cudaError_t launch_merge_fwd(const MergeArgs& m, cudaStream_t st) {
 
 cudaError_t launch_merge_bwd(const MergeArgs& m, cudaStream_t st) {
     const int T = m.B * m.N;
-    cudaError_t e;
-    const size_t ssm = sort_smem(m.N);
-    if ((e = ensure_smem<merge_groups_kernel>(ssm)) != cudaSuccess) return e;
-    merge_groups_kernel<<<m.B, kSortThreads, ssm, st>>>(m.assign, m.N, m.k, m.members, m.goff);
-    note_launch();
+    cudaError_t e = cudaSuccess;
+    if ((e = launch_groups(m, st)) != cudaSuccess) return e;
     const long long na = static_cast<long long>(m.B) * m.k;
-    const unsigned gblocks = static_cast<unsigned>((na + kMergeWarps - 1) / kMergeWarps);
-    ACL_HP_SWITCH(m.h, (merge_bwd_group_kernel<HP><<<gblocks, kMergeThreads, 0, st>>>(
-                           m.feats, m.xy, m.B, m.N, m.d, m.k, m.w1, m.b1, m.w2, m.h, m.scores,
-                           m.members, m.goff, m.dmerged, m.dmxy, m.dfeats, m.dxy, m.ds, m.dh, m.gz)));
+    merge_gstat_kernel<<<static_cast<unsigned>((na + kMergeWarps - 1) / kMergeWarps), kMergeThreads, 0, st>>>(
+        m.feats, m.xy, m.B, m.N, m.d, m.k, m.scores, m.members, m.goff, m.dmerged, m.dmxy,
+        reinterpret_cast<float4*>(m.gstat), m.g);
     note_launch();
-    const size_t psm = sizeof(float) * (static_cast<size_t>(kParamTile) * (m.d + 2 * m.h) + kParamTile);
+    const bool sm = w1_in_smem(m.d, m.h);
+    ACL_HP_SWITCH(m.h, (e = sm ? launch_bwd_token<HP, true>(m, T, st) : launch_bwd_token<HP, false>(m, T, st)));
+    if (e != cudaSuccess) return e;
+    const size_t psm = param_smem(m.d, m.h);
     if ((e = ensure_smem<merge_param_part_kernel>(psm)) != cudaSuccess) return e;
-    merge_param_part_kernel<<<kParamParts, kMergeThreads, psm, st>>>(m.feats, T, m.d, m.h, m.ds, m.dh,
-                                                                      m.gz, m.part);
+    const int pth = param_threads(m.d, m.h);
+    const int tiles = (m.d / 4 + 1) * (((m.h + 3) & ~3) / 4);
+    merge_param_part_kernel<<<dim3(kParamParts, (tiles + pth - 1) / pth), pth, psm, st>>>(
+        m.feats, T, m.d, m.h, m.ds, m.dh, m.e, m.part);
     note_launch();
     const int nout = m.d * m.h + 2 * m.h + 1;
-    merge_param_reduce_kernel<<<(nout + kMergeThreads - 1) / kMergeThreads, kMergeThreads, 0, st>>>(
-        m.part, m.d, m.h, m.dw1, m.db1, m.dw2, m.db2);
+    merge_param_reduce_kernel<<<(nout + 31) / 32, kMergeThreads, 0, st>>>(m.part, m.d, m.h, m.dw1, m.db1,
+                                                                        m.dw2, m.db2);
     note_launch();
     return cudaGetLastError();
 }

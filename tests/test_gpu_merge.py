@@ -71,3 +71,22 @@ def test_merge_is_bit_reproducible():
                                  dev(mb.dmcoords))
     for x, y in zip(g1, g2):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("d,hidden", [(64, 100), (64, 256), (1024, 8)])
+def test_merge_hidden_widths(d, hidden):
+    """Hidden widths that are not a multiple of 32 (padded units), the widest (256), and a W1
+    too large for shared memory (read from global memory)."""
+    rng = np.random.default_rng(11)
+    xy = rng.uniform(0, 20, size=(2, 300, 2)).astype(np.float32)
+    merge_both(synth.merge_batch(xy, d=d, hidden=hidden))
+
+
+def test_merge_score_ties_and_many_tokens():
+    """Tokens with identical features get bit-identical scores: the anchors among them are the
+    lowest ids.  N = 5000 spans many CTAs of the counting and assignment kernels."""
+    rng = np.random.default_rng(12)
+    xy = rng.uniform(0, 70, size=(1, 5000, 2)).astype(np.float32)
+    mb = synth.merge_batch(xy, d=32, hidden=8)
+    mb.feats[:, 100:400] = mb.feats[:, 99:100]
+    merge_both(mb)

@@ -94,6 +94,9 @@ def parse_args(argv=None):
                          "chains run as two concurrent branches of the step graph)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bounded CPU work of the oracle baseline (seconds)")
+    ap.add_argument("--only", choices=("token_merge",), default=None,
+                    help="time one extra part alone on one GPU and print its JSON (a short "
+                         "command to profile under ncu); no bench line")
     return ap.parse_args(argv)
 
 
@@ -450,7 +453,8 @@ def run_gpu(args, rank: int, world: int):
             inv_us[f"{name}_{key}"] = graph_time(
                 torch, stream, lambda: s0.op(name, stream, kind=kind), 20)
     hires = hires_gather_times(torch, acl, synth, device, stream) if world == 1 else None
-    merge_us = token_merge_times(torch, acl, synth, sb, device, stream) if world == 1 else None
+    merge_us = (token_merge_times(torch, acl, synth, sb, device, stream, measured_peaks())
+                if world == 1 else None)
     # keep the same load on the GPU until the clock sampler has several samples
     t_wall = time.time()
     it = 0
@@ -569,9 +573,20 @@ def graph_time(torch, stream, fn, reps: int = 10) -> float:
     return round(e0.elapsed_time(e1) / reps * 1e3, 2)
 
 
-def token_merge_times(torch, acl, synth, sb, device, stream, reps: int = 10) -> dict:
+def merge_bytes(B: int, N: int, d: int, k: int) -> dict:
+    """Algorithmic bytes of token merging, every tensor once: forward reads features (2d B)
+    and coordinates (8 B) per token and writes score, assignment (8 B) per token and the merged
+    row (2d + 8 B) and anchor id per anchor; backward reads features, coordinates, score and
+    assignment and writes dfeats and dcoords per token (4d + 24 B), reads dmerged (2d + 8 B)
+    per anchor."""
+    T, A = B * N, B * k
+    return {"fwd": T * (2 * d + 16) + A * (2 * d + 12), "bwd": T * (4 * d + 24) + A * (2 * d + 8)}
+
+
+def token_merge_times(torch, acl, synth, sb, device, stream, peaks: dict, reps: int = 10) -> dict:
     """Token merging of the stage-1 tokens into round(0.4 N) anchors (d = 128, hidden 32),
-    forward and backward, one call at a time with CUDA events."""
+    forward and backward, one call at a time with CUDA events; GB/s of the algorithmic bytes
+    and the fraction of the measured HBM copy bandwidth."""
     mb = synth.merge_batch(sb.attn.coords, d=128)
     T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
     f, xy = T(mb.feats, torch.bfloat16), T(mb.coords)
@@ -581,13 +596,20 @@ def token_merge_times(torch, acl, synth, sb, device, stream, reps: int = 10) -> 
                      dtype=torch.uint8, device=device)
     out = acl.acl_token_merge_fwd(f, xy, w1, b1, w2, mb.b2, mb.k, workspace=ws, stream=stream)
     timed = lambda fn: graph_time(torch, stream, fn, reps)
-    return {
+    res = {
         "workload": f"{mb.B} images, N = {mb.N} -> k = {mb.k}, d = {mb.d}, hidden {mb.h}",
         "fwd": timed(lambda: acl.acl_token_merge_fwd(f, xy, w1, b1, w2, mb.b2, mb.k, workspace=ws,
                                                      stream=stream)),
         "bwd": timed(lambda: acl.acl_token_merge_bwd(f, xy, w1, b1, w2, mb.b2, mb.k, out[0], out[2],
                                                      dm, dx, workspace=ws, stream=stream)),
     }
+    nbytes = merge_bytes(mb.B, mb.N, mb.d, mb.k)
+    res["roofline"] = {}
+    for key in ("fwd", "bwd"):
+        gbs = nbytes[key] / (res[key] * 1e-6) / 1e9
+        res["roofline"][key] = {"alg_bytes": nbytes[key], "GB_s": round(gbs, 1),
+                                "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    return res
 
 
 def hires_gather_times(torch, acl, synth, device, stream, B: int = 4, reps: int = 10) -> dict:
@@ -782,7 +804,26 @@ def main(argv=None):
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
+    if args.only:
+        run_only(args)
+        return
     run_gpu(args, rank, world)
+
+
+def run_only(args):
+    """One extra part on cuda:0 (an eager call, then each call captured as a CUDA graph and
+    replayed between CUDA events); prints its timing dict."""
+    import torch
+
+    import off_grid_cluster_b200 as acl
+    from off_grid_cluster_b200 import synth
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    sb = synth.step_batch(B=args.batch)
+    res = token_merge_times(torch, acl, synth, sb, device, stream, measured_peaks())
+    print(json.dumps({"part": args.only, **res}))
 
 
 if __name__ == "__main__":

@@ -27,6 +27,8 @@ retention rate, dims 128/256/512/768, 32-channel heads):
                   subsets, dims 128/256/512/768, layers 3/4/16/2.
 * ``decoder``  -- the sweep's four stages as KNN sources, 4096 queries per
                   image at cell centre + U(-1,1)^2, K = 8, p_h ~ U(0.5, 4).
+* ``dec_layer`` -- the decoder: the 2048 masked cells of each image as queries,
+                  four layers over the sweep's stages coarse to fine (D = 256).
 * ``step``     -- the stage1 batch plus a decoder gather over that same stage
                   (4096 queries per image, d = 128): one pass of every step.
 
@@ -50,7 +52,8 @@ TAG_Q, TAG_K, TAG_V, TAG_DO = 10, 11, 12, 13
 TAG_QUERY, TAG_FEAT, TAG_P, TAG_DOUT = 20, 21, 22, 23
 
 WORKLOAD_ID = {"tiny": 1, "stage1": 2, "stage3": 3, "sweep": 4, "decoder": 5,
-               "step": 6, "hires": 7, "merge": 8}
+               "step": 6, "hires": 7, "merge": 8, "dec_layer": 9}
+TAG_F0, TAG_WOFF, TAG_WO, TAG_DF = 30, 31, 32, 33
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -416,3 +419,60 @@ def merge_batch(coords: np.ndarray, d: int = 128, ds: float = 0.4, image0: int =
     dxy = np.stack([normal(stream_seed(wid, i, TAG_QUERY, 1), 2 * k).reshape(k, 2)
                     for i in imgs]).astype(np.float32)
     return MergeBatch(coords.astype(np.float32), feats, w1, b1, w2, b2, k, dm, dxy)
+
+
+@dataclass
+class DecoderBatch:
+    """The decoder over four encoder stages: B images, Q mask-token queries per image (the
+    masked cells of the 64 x 64 grid; reference positions at their centres) with D-channel
+    features, and per layer an offset head (W_off [D, 2], b_off [2]) and a projection
+    (W_o [d_s, D], bf16 values).  Layer l reads stage layer_stage[l]: coarse to fine."""
+    ref: np.ndarray               # [B, Q, 2] fp32
+    f0: np.ndarray                # [B, Q, D] fp32
+    stages: list                  # KnnBatch per stage (0 = finest): coords, feats, p
+    w_off: list                   # per layer [D, 2] fp32
+    b_off: list                   # per layer [2] fp32
+    w_o: list                     # per layer [d_s, D] bf16 values in fp32
+    df: np.ndarray                # [B, Q, D] fp32, gradient of the last layer's output
+    layer_stage: tuple = (3, 2, 1, 0)
+
+    @property
+    def B(self): return self.ref.shape[0]
+
+    @property
+    def Q(self): return self.ref.shape[1]
+
+    @property
+    def D(self): return self.f0.shape[2]
+
+
+def decoder_batch(B: int = 8, image0: int = 0, D: int = 256, n0: int = 2048,
+                  offset_scale: float = 1.0) -> DecoderBatch:
+    """Stages as in the sweep (nested subsets, dims 128/256/512/768) of a value-noise mask
+    keeping n0 of 4096 cells; the other cells are the queries.  f0, df ~ N(0, 1);
+    W_off ~ offset_scale N(0, 1/D) (offsets of about offset_scale cells), b_off ~ 0.1 N(0, 1);
+    W_o ~ N(0, 1/d_s) rounded to bf16."""
+    wid = WORKLOAD_ID["dec_layer"]
+    imgs = range(image0, image0 + B)
+    coords = sweep_coords(B, image0, n0=n0, wid=wid)
+    refs = []
+    for i in imgs:
+        vis = noise_mask(stream_seed(wid, i, TAG_MASK), 64, 64, n0)
+        masked = np.setdiff1d(np.arange(64 * 64), vis)
+        refs.append(np.stack([(masked % 64) + 0.5, (masked // 64) + 0.5], axis=1))
+    ref = np.stack(refs).astype(np.float32)
+    Q = ref.shape[1]
+    stages = [knn_batch(xy, SWEEP_DIMS[s], image0, s, wid=wid) for s, xy in enumerate(coords)]
+    f0 = np.stack([normal(stream_seed(wid, i, TAG_F0), Q * D).reshape(Q, D)
+                   for i in imgs]).astype(np.float32)
+    df = np.stack([normal(stream_seed(wid, i, TAG_DF), Q * D).reshape(Q, D)
+                   for i in imgs]).astype(np.float32)
+    w_off, b_off, w_o = [], [], []
+    for layer, st in enumerate((3, 2, 1, 0)):
+        w_off.append((offset_scale * normal(stream_seed(wid, 0, TAG_WOFF, layer), 2 * D)
+                      / math.sqrt(D)).reshape(D, 2).astype(np.float32))
+        b_off.append((0.1 * normal(stream_seed(wid, 0, TAG_WOFF, 16 + layer), 2)).astype(np.float32))
+        d = SWEEP_DIMS[st]
+        w_o.append(round_bf16(normal(stream_seed(wid, 0, TAG_WO, layer), d * D)
+                              / math.sqrt(d)).reshape(d, D))
+    return DecoderBatch(ref, f0, stages, w_off, b_off, w_o, df)

@@ -31,7 +31,9 @@ def lib():
         for name in ("orc_cluster_batch", "orc_neighbors_batch", "orc_attn_fwd_batch",
                      "orc_attn_bwd_batch", "orc_knn_table_batch", "orc_knn_fwd_batch",
                      "orc_knn_bwd_batch", "orc_set_threads", "orc_token_order_batch",
-                     "orc_merge_scores", "orc_merge_select", "orc_merge_fwd", "orc_merge_bwd"):
+                     "orc_merge_scores", "orc_merge_select", "orc_merge_fwd", "orc_merge_bwd",
+                     "orc_dec_offsets", "orc_dec_project", "orc_dec_project_bwd",
+                     "orc_dec_offsets_bwd"):
             getattr(L, name).restype = ct.c_int
         _lib = L
     return _lib
@@ -212,3 +214,52 @@ def merge_bwd(feats, xy, w1, b1, w2, b2, k, assign, dmerged, dmxy):
                                    ct.byref(t4)), "merge_bwd")
         dw1 += t1; db1 += t2; dw2 += t3; db2 += t4.value
     return df, dxy, dw1, db1, dw2, db2
+
+
+def decoder_offsets(ref, f, w_off, b_off):
+    """Sample positions q = r + f W_off + b_off in fp64 -> [B, Q, 2]."""
+    ref, f, w_off, b_off = _f32(ref), _f64(f), _f64(w_off), _f64(b_off)
+    B, Q, D = f.shape
+    q = np.empty((B, Q, 2))
+    for b in range(B):
+        _check(lib().orc_dec_offsets(_p(ref[b]), _p(f[b]), Q, D, _p(w_off), _p(b_off), _p(q[b])),
+               "dec_offsets")
+    return q
+
+
+def decoder_layer_fwd(ref, f, w_off, b_off, feats, xy, table, p, w_o, q=None):
+    """One decoder layer: (q fp64, v = the stage gather at q, f_out = f + v W_o).  The gather
+    samples at q rounded to fp32, or at the given fp32 q (the cell choice is an integer
+    decision: a caller comparing with another implementation passes that one's q)."""
+    q64 = decoder_offsets(ref, f, w_off, b_off)
+    qs = q64.astype(np.float32) if q is None else _f32(q)
+    v = knn_fwd(qs, feats, xy, table, p)
+    f, w_o = _f64(f), _f64(w_o)
+    B, Q, D = f.shape
+    d = v.shape[2]
+    f_out = np.empty((B, Q, D))
+    for b in range(B):
+        _check(lib().orc_dec_project(_p(f[b]), _p(v[b]), Q, D, d, _p(w_o), _p(f_out[b])),
+               "dec_project")
+    return q64, v, f_out
+
+
+def decoder_layer_bwd(f, w_off, feats, xy, table, p, w_o, q, v, df_out):
+    """Backward of one decoder layer at the fp32 sample positions q with gathered v:
+    (df_in, dW_off, db_off, dfeats, dp, dW_o); parameter gradients summed over images."""
+    f, w_off, w_o, v, df_out = _f64(f), _f64(w_off), _f64(w_o), _f64(v), _f64(df_out)
+    B, Q, D = f.shape
+    d = v.shape[2]
+    dv = np.empty((B, Q, d))
+    dw_o = np.zeros((d, D))
+    for b in range(B):
+        _check(lib().orc_dec_project_bwd(_p(v[b]), _p(df_out[b]), Q, D, d, _p(w_o), _p(dv[b]),
+                                         _p(dw_o)), "dec_project_bwd")
+    dfeats, dq, dp = knn_bwd(q, feats, xy, table, p, dv)
+    df_in = np.empty((B, Q, D))
+    dw_off = np.zeros((D, 2))
+    db_off = np.zeros(2)
+    for b in range(B):
+        _check(lib().orc_dec_offsets_bwd(_p(f[b]), _p(dq[b]), _p(df_out[b]), Q, D, _p(w_off),
+                                         _p(df_in[b]), _p(dw_off), _p(db_off)), "dec_offsets_bwd")
+    return df_in, dw_off, db_off, dfeats, dp, dw_o

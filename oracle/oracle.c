@@ -729,6 +729,86 @@ int orc_merge_bwd(const double* f, const float* xy, int N, int d, const double* 
     return 0;
 }
 
+/*
+ * Decoder layer (AFFMAE notes, "Key Designs" 2, the point-wise deformable cross-attention
+ * decoder): every mask-token query, with feature f and reference position r, predicts a 2D
+ * offset Delta = g(f), samples q = r + Delta, gathers the nearest visible tokens of an
+ * encoder stage around q with distance-softmax weights (the KNN gather above), and the
+ * decoder fuses the stages coarse to fine ("A Complete Example": stage 4 first, then stages
+ * 3 to 1).  The notes fix no more; the readings taken:
+ *   g is one linear map: Delta = f W_off + b_off, W_off [D][2], b_off [2];
+ *   the gathered feature v (the stage's d channels) is projected to the decoder width and
+ *   added to the query feature: f_out = f + v W_o, W_o [d][D] (a residual cross-attention
+ *   update whose attention weights are the distance softmax).
+ * Plain loops in fp64; every sum in index order.
+ */
+int orc_dec_offsets(const float* ref, const double* f, int Q, int D, const double* w_off,
+                    const double* b_off, double* q) {
+    if (Q < 0 || D < 1) return 1;
+    for (int i = 0; i < Q; ++i)
+        for (int j = 0; j < 2; ++j) {
+            double acc = (double)ref[(size_t)i * 2 + j] + b_off[j];
+            for (int c = 0; c < D; ++c) acc += f[(size_t)i * D + c] * w_off[(size_t)c * 2 + j];
+            q[(size_t)i * 2 + j] = acc;
+        }
+    return 0;
+}
+
+int orc_dec_project(const double* f, const double* v, int Q, int D, int d, const double* w_o,
+                    double* f_out) {
+    if (Q < 0 || D < 1 || d < 1) return 1;
+    for (int i = 0; i < Q; ++i)
+        for (int n = 0; n < D; ++n) {
+            double acc = f[(size_t)i * D + n];
+            for (int c = 0; c < d; ++c) acc += v[(size_t)i * d + c] * w_o[(size_t)c * D + n];
+            f_out[(size_t)i * D + n] = acc;
+        }
+    return 0;
+}
+
+/* dv = df_out W_o^T; dW_o += v^T df_out (accumulated, so images can be summed) */
+int orc_dec_project_bwd(const double* v, const double* df_out, int Q, int D, int d,
+                        const double* w_o, double* dv, double* dw_o) {
+    if (Q < 0 || D < 1 || d < 1) return 1;
+    for (int i = 0; i < Q; ++i)
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int n = 0; n < D; ++n) acc += df_out[(size_t)i * D + n] * w_o[(size_t)c * D + n];
+            dv[(size_t)i * d + c] = acc;
+        }
+    for (int c = 0; c < d; ++c)
+        for (int n = 0; n < D; ++n) {
+            double acc = 0.0;
+            for (int i = 0; i < Q; ++i) acc += v[(size_t)i * d + c] * df_out[(size_t)i * D + n];
+            dw_o[(size_t)c * D + n] += acc;
+        }
+    return 0;
+}
+
+/* df_in = df_out + dq W_off^T (the residual path plus the offset head);
+ * dW_off += f^T dq, db_off += sum_i dq_i (accumulated) */
+int orc_dec_offsets_bwd(const double* f, const double* dq, const double* df_out, int Q, int D,
+                        const double* w_off, double* df_in, double* dw_off, double* db_off) {
+    if (Q < 0 || D < 1) return 1;
+    for (int i = 0; i < Q; ++i)
+        for (int c = 0; c < D; ++c)
+            df_in[(size_t)i * D + c] = df_out[(size_t)i * D + c] +
+                                       dq[(size_t)i * 2] * w_off[(size_t)c * 2] +
+                                       dq[(size_t)i * 2 + 1] * w_off[(size_t)c * 2 + 1];
+    for (int c = 0; c < D; ++c)
+        for (int j = 0; j < 2; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < Q; ++i) acc += f[(size_t)i * D + c] * dq[(size_t)i * 2 + j];
+            dw_off[(size_t)c * 2 + j] += acc;
+        }
+    for (int j = 0; j < 2; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < Q; ++i) acc += dq[(size_t)i * 2 + j];
+        db_off[j] += acc;
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* batch drivers: images are independent; OpenMP over images only            */
 /* ------------------------------------------------------------------------ */

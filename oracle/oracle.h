@@ -66,4 +66,14 @@ int orc_knn_bwd_batch(const float* queries, int B, int Q, const double* feats,
                       int K, const double* p, int kind, const double* dout, double* dfeats,
                       double* dq, double* dp);
 int orc_token_order_batch(const float* xy, int B, int N, int GH, int GW, int32_t* perm);
+
+/* decoder layer: offsets q = r + f W_off + b_off, projection f_out = f + v W_o, backward */
+int orc_dec_offsets(const float* ref, const double* f, int Q, int D, const double* w_off,
+                    const double* b_off, double* q);
+int orc_dec_project(const double* f, const double* v, int Q, int D, int d, const double* w_o,
+                    double* f_out);
+int orc_dec_project_bwd(const double* v, const double* df_out, int Q, int D, int d,
+                        const double* w_o, double* dv, double* dw_o);
+int orc_dec_offsets_bwd(const double* f, const double* dq, const double* df_out, int Q, int D,
+                        const double* w_off, double* df_in, double* dw_off, double* db_off);
 #endif

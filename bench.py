@@ -49,6 +49,7 @@ sys.path.insert(0, ROOT)
 METRIC = "cluster-attn fwd+bwd tokens/s & KNN-gather queries/s; % of B200 HBM roofline"
 WORKLOAD = "stage1-1024px-b8-n2048-d128-h4-c8-m48 + decoder-knn-gather-q4096-k8"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 OPS = ("cluster", "neighbors", "attn_fwd", "attn_bwd", "knn_table", "knn_index", "knn_fwd",
        "knn_bwd")
 KERNELS = {
@@ -94,7 +95,7 @@ def parse_args(argv=None):
                          "chains run as two concurrent branches of the step graph)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bounded CPU work of the oracle baseline (seconds)")
-    ap.add_argument("--only", choices=("token_merge",), default=None,
+    ap.add_argument("--only", choices=("token_merge", "decoder"), default=None,
                     help="time one extra part alone on one GPU and print its JSON (a short "
                          "command to profile under ncu); no bench line")
     return ap.parse_args(argv)
@@ -127,8 +128,10 @@ def measured_peaks() -> dict:
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured (MEASURED_PEAKS.json)"}
-    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback 6.65 TB/s"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d.get("bf16_tflops", FALLBACK_BF16_TFLOPS)),
+                "source": "measured (MEASURED_PEAKS.json)"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "source": "fallback 6.65 TB/s, 1590 TFLOP/s"}
 
 
 def source_hash() -> str:
@@ -455,6 +458,7 @@ def run_gpu(args, rank: int, world: int):
     hires = hires_gather_times(torch, acl, synth, device, stream) if world == 1 else None
     merge_us = (token_merge_times(torch, acl, synth, sb, device, stream, measured_peaks())
                 if world == 1 else None)
+    dec_us = decoder_times(torch, acl, synth, device, stream, measured_peaks()) if world == 1 else None
     # keep the same load on the GPU until the clock sampler has several samples
     t_wall = time.time()
     it = 0
@@ -527,6 +531,7 @@ def run_gpu(args, rank: int, world: int):
                                "on the same gathers (set 0, one graph per call, L2-warm)"},
             "hires_gather_us": hires,
             "token_merge_us": merge_us,
+            "decoder_us": dec_us,
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -810,6 +815,67 @@ def main(argv=None):
     run_gpu(args, rank, world)
 
 
+def decoder_times(torch, acl, synth, device, stream, peaks: dict, B: int = 8, reps: int = 10) -> dict:
+    """The decoder's four layers (coarse to fine over stages 4..1; B images x 2048 mask-token
+    queries, D = 256, K = 8), forward and backward per layer and the whole chain, each call
+    captured as a CUDA graph and timed with CUDA events.  The projection GEMMs do
+    2 T d D FLOPs forward and 4 T d D backward (T = B Q); their rate is given against the
+    layer's whole time (a lower bound on the GEMM kernels' own rate) and the measured bf16
+    peak."""
+    db = synth.decoder_batch(B=B)
+    T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
+    ref, f0, df = T(db.ref), T(db.f0), T(db.df)
+    layers = []
+    for layer, s in enumerate(db.layer_stage):
+        st = db.stages[s]
+        xy = T(st.coords)
+        table = acl.acl_knn_table(xy, st.GH, st.GW, st.K, stream=stream)
+        layers.append(dict(w_off=T(db.w_off[layer]), b_off=T(db.b_off[layer]),
+                           w_o=T(db.w_o[layer], torch.bfloat16), feats=T(st.feats, torch.bfloat16),
+                           coords=xy, table=table, p=T(st.p), d=st.d, N=st.N))
+    Tq = db.B * db.Q
+    ws = torch.empty((max(acl.acl_decoder_layer_workspace(db.B, db.Q, L["N"], L["d"], db.D)
+                          for L in layers),), dtype=torch.uint8, device=device)
+    fs, saved = [f0], []
+    for L in layers:
+        q, v, f_out = acl.acl_decoder_layer_fwd(ref, fs[-1], L["w_off"], L["b_off"], L["w_o"],
+                                                L["feats"], L["coords"], L["table"], L["p"], stream=stream)
+        saved.append((q, v))
+        fs.append(f_out)
+    torch.cuda.synchronize()
+    stage_of = lambda l: db.layer_stage[l] + 1
+
+    def fwd(l):
+        L = layers[l]
+        return acl.acl_decoder_layer_fwd(ref, fs[l], L["w_off"], L["b_off"], L["w_o"], L["feats"],
+                                         L["coords"], L["table"], L["p"], f_out=fs[l + 1], stream=stream)
+
+    def bwd(l):
+        L = layers[l]
+        q, v = saved[l]
+        return acl.acl_decoder_layer_bwd(fs[l], L["w_off"], L["w_o"], L["feats"], L["coords"],
+                                         L["table"], L["p"], q, v, df, workspace=ws, stream=stream)
+
+    res = {"workload": f"{db.B} images x {db.Q} queries, D = {db.D}, K = 8, stages 4..1 "
+                       f"(N = {', '.join(str(L['N']) for L in layers)}; d = "
+                       f"{', '.join(str(L['d']) for L in layers)})", "layers": []}
+    tf, tb = 0.0, 0.0
+    for l, L in enumerate(layers):
+        uf = graph_time(torch, stream, lambda: fwd(l), reps)
+        ub = graph_time(torch, stream, lambda: bwd(l), reps)
+        tf += uf
+        tb += ub
+        flops_f, flops_b = 2.0 * Tq * L["d"] * db.D, 4.0 * Tq * L["d"] * db.D
+        res["layers"].append({"stage": stage_of(l), "d": L["d"], "fwd": uf, "bwd": ub,
+                              "gemm_tflops_fwd": round(flops_f / (uf * 1e-6) / 1e12, 1),
+                              "gemm_tflops_bwd": round(flops_b / (ub * 1e-6) / 1e12, 1)})
+    res["fwd_total"] = round(tf, 2)
+    res["bwd_total"] = round(tb, 2)
+    res["queries_per_s_fwd_bwd"] = round(Tq / ((tf + tb) * 1e-6), 1)
+    res["peak_bf16_tflops"] = peaks["bf16_tflops"]
+    return res
+
+
 def run_only(args):
     """One extra part on cuda:0 (an eager call, then each call captured as a CUDA graph and
     replayed between CUDA events); prints its timing dict."""
@@ -821,8 +887,11 @@ def run_only(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     stream = torch.cuda.Stream(device)
-    sb = synth.step_batch(B=args.batch)
-    res = token_merge_times(torch, acl, synth, sb, device, stream, measured_peaks())
+    if args.only == "token_merge":
+        sb = synth.step_batch(B=args.batch)
+        res = token_merge_times(torch, acl, synth, sb, device, stream, measured_peaks())
+    else:
+        res = decoder_times(torch, acl, synth, device, stream, measured_peaks(), B=args.batch)
     print(json.dumps({"part": args.only, **res}))
 
 

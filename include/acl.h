@@ -396,6 +396,47 @@ acl_status acl_knn_gather_bwd_indexed_ex(const float* queries, int B, int Q,
                                          float* dp, void* workspace, size_t ws_bytes,
                                          acl_stream_t stream);
 
+/*
+ * acl_decoder_layer_fwd -- one layer of the point-wise deformable cross-attention decoder
+ * (NEXT row f4).  Passage: AFFMAE notes, "Key Designs" 2 (each mask-token query predicts a 2D
+ * offset Delta = g(f) and samples q = r + Delta, gathers an encoder stage's nearest visible
+ * tokens around q with distance-softmax weights, the stages fused coarse to fine) and "A
+ * Complete Example" (stage 4 first, then stages 3 to 1).  Readings: g is linear, and the
+ * gathered feature is projected to the decoder width and added to the query feature:
+ *   q = r + f W_off + b_off                     (fp32)
+ *   v = acl_knn_gather_fwd of the stage at q    (exponential kernel, bf16 out)
+ *   f_out = f + v W_o                           (bf16 tensor-core products, fp32 sums)
+ * ref [B][Q][2], f_in [B][Q][D] fp32; W_off [D][2], b_off [2] fp32; W_o [d][D] bf16; the
+ * stage as for the gather (feats [B][N][d] bf16, coords [B][N][2], table [B][H][W][K], p
+ * [d/32]).  Out: q [B][Q][2] fp32, v [B][Q][d] bf16 (both needed by the backward), f_out
+ * [B][Q][D] fp32 (may equal f_in when no backward follows).  Stacking layers over stages 4..1
+ * is the caller's loop.  Limits: D % 128 == 0, 128 <= D <= 1024; d % 128 == 0 and the
+ * gather's limits; Q <= ACL_MAX_GATHER_Q, B Q <= 2^24.  The cell choice is an integer decision
+ * on the fp32 q.
+ */
+size_t acl_decoder_layer_workspace(int B, int Q, int N, int d, int D, int K);
+acl_status acl_decoder_layer_fwd(const float* ref, const float* f_in, int B, int Q, int D,
+                                 const float* w_off, const float* b_off, const acl_bf16* w_o,
+                                 const acl_bf16* feats, const float* coords, int N, int d,
+                                 const int32_t* table, int H, int W, int K, const float* p,
+                                 float* q, acl_bf16* v, float* f_out, acl_stream_t stream);
+/*
+ * Backward of one decoder layer at the forward's q and v:
+ *   dv = df_out W_o^T (bf16), dW_o = v^T df_out, the gather's backward of dv (dfeats, dq, dp),
+ *   df_in = df_out + dq W_off^T, dW_off = f_in^T dq, db_off = sum dq
+ * (parameter gradients summed over all queries in a fixed order: bit-reproducible).  Out:
+ * df_in [B][Q][D] (may equal df_out), dW_off [D][2], db_off [2], dW_o [d][D] fp32, dfeats
+ * [B][N][d] bf16, dp [d/32] fp32; all overwritten.  workspace: acl_decoder_layer_workspace
+ * bytes, 256-byte aligned.
+ */
+acl_status acl_decoder_layer_bwd(const float* f_in, int B, int Q, int D, const float* w_off,
+                                 const acl_bf16* w_o, const acl_bf16* feats, const float* coords,
+                                 int N, int d, const int32_t* table, int H, int W, int K,
+                                 const float* p, const float* q, const acl_bf16* v,
+                                 const float* df_out, float* df_in, float* dw_off, float* db_off,
+                                 float* dw_o, acl_bf16* dfeats, float* dp, void* workspace,
+                                 size_t ws_bytes, acl_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,6 +47,11 @@ SIGNATURES = {
     "acl_token_merge_bwd": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _F, _I, _I, _P, _P, _P, _P, _P,
                                  _P, _P, _P, _P, _P, _P, _Z, _P]),
     "acl_knn_gather_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "acl_decoder_layer_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "acl_decoder_layer_fwd": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I,
+                                   _I, _P, _P, _P, _P, _P]),
+    "acl_decoder_layer_bwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P,
+                                   _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "acl_knn_gather_fwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P]),
     "acl_knn_gather_bwd": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P,
                                 _P, _P, _Z, _P]),
@@ -342,6 +347,65 @@ def _gather_shapes(queries, feats, coords, table, p):
 
 
 ACL_KNN_EXP, ACL_KNN_INVPOW = 0, 1  # weight kernels: softmax(-p d), d^-p / sum d^-p
+
+
+def acl_decoder_layer_workspace(B: int, Q: int, N: int, d: int, D: int, K: int = 8) -> int:
+    return int(lib().acl_decoder_layer_workspace(B, Q, N, d, D, K))
+
+
+def _decoder_shapes(f_in, w_off, w_o, feats, coords, table, p):
+    _need(f_in, "f_in", torch.float32)
+    B, Q, D = f_in.shape
+    _need(feats, "feats", torch.bfloat16)
+    N, d = feats.shape[1:]
+    _need(coords, "coords", torch.float32, (B, N, 2))
+    _need(table, "table", torch.int32)
+    H, W, K = table.shape[1:]
+    _need(p, "p", torch.float32, (d // 32,))
+    _need(w_off, "w_off", torch.float32, (D, 2))
+    _need(w_o, "w_o", torch.bfloat16, (d, D))
+    return B, Q, D, N, d, H, W, K
+
+
+def acl_decoder_layer_fwd(ref, f_in, w_off, b_off, w_o, feats, coords, table, p, f_out=None,
+                          stream=None):
+    """One decoder layer -> (q [B,Q,2] f32, v [B,Q,d] bf16, f_out [B,Q,D] f32)."""
+    B, Q, D, N, d, H, W, K = _decoder_shapes(f_in, w_off, w_o, feats, coords, table, p)
+    _need(ref, "ref", torch.float32, (B, Q, 2))
+    _need(b_off, "b_off", torch.float32, (2,))
+    dev = f_in.device
+    q = torch.empty((B, Q, 2), dtype=torch.float32, device=dev)
+    v = torch.empty((B, Q, d), dtype=torch.bfloat16, device=dev)
+    f_out = _out(f_out, (B, Q, D), torch.float32, f_in, "f_out")
+    _call("acl_decoder_layer_fwd", _ptr(ref), _ptr(f_in), B, Q, D, _ptr(w_off), _ptr(b_off),
+          _ptr(w_o), _ptr(feats), _ptr(coords), N, d, _ptr(table), H, W, K, _ptr(p), _ptr(q),
+          _ptr(v), _ptr(f_out), _stream(stream))
+    return q, v, f_out
+
+
+def acl_decoder_layer_bwd(f_in, w_off, w_o, feats, coords, table, p, q, v, df_out, df_in=None,
+                          workspace=None, stream=None):
+    """Decoder layer backward -> (df_in [B,Q,D] f32, dW_off [D,2], db_off [2], dW_o [d,D] f32,
+    dfeats [B,N,d] bf16, dp [d/32] f32)."""
+    B, Q, D, N, d, H, W, K = _decoder_shapes(f_in, w_off, w_o, feats, coords, table, p)
+    _need(q, "q", torch.float32, (B, Q, 2))
+    _need(v, "v", torch.bfloat16, (B, Q, d))
+    _need(df_out, "df_out", torch.float32, (B, Q, D))
+    dev = f_in.device
+    df_in = _out(df_in, (B, Q, D), torch.float32, f_in, "df_in")
+    dw_off = torch.empty((D, 2), dtype=torch.float32, device=dev)
+    db_off = torch.empty((2,), dtype=torch.float32, device=dev)
+    dw_o = torch.empty((d, D), dtype=torch.float32, device=dev)
+    dfeats = torch.empty_like(feats)
+    dp = torch.empty((d // 32,), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(acl_decoder_layer_workspace(B, Q, N, d, D, K), 1),
+                                dtype=torch.uint8, device=dev)
+    _call("acl_decoder_layer_bwd", _ptr(f_in), B, Q, D, _ptr(w_off), _ptr(w_o), _ptr(feats),
+          _ptr(coords), N, d, _ptr(table), H, W, K, _ptr(p), _ptr(q), _ptr(v), _ptr(df_out),
+          _ptr(df_in), _ptr(dw_off), _ptr(db_off), _ptr(dw_o), _ptr(dfeats), _ptr(dp),
+          _ptr(workspace), workspace.numel(), _stream(stream))
+    return df_in, dw_off, db_off, dw_o, dfeats, dp
 
 
 def acl_knn_gather_fwd(queries, feats, coords, table, p, out=None, stream=None,

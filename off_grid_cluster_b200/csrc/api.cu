@@ -88,6 +88,30 @@ acl_status setup_gather_bwd(const float* queries, int B, int Q, const acl_bf16* 
     return ACL_OK;
 }
 
+// Validation shared by the decoder-layer entry points (positions = ref or q).
+acl_status check_decoder(const float* positions, const float* f_in, int B, int Q, int D,
+                         const float* w_off, const acl_bf16* w_o, const acl_bf16* feats,
+                         const float* coords, int N, int d, const int32_t* table, int H, int W,
+                         int K, const float* p) {
+    acl_status st = check_gather(positions, B, Q, feats, coords, N, d, table, H, W, K, p);
+    if (st != ACL_OK) return st;
+    if ((Q > 0 && !f_in) || !w_off || !w_o) return ACL_ERR_INVALID_ARG;
+    if (D < 128 || D % 128 != 0 || d % 128 != 0) return ACL_ERR_INVALID_ARG;
+    if (D > 1024 || Q > ACL_MAX_GATHER_Q || N > ACL_MAX_TABLE_N) return ACL_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * Q > (1LL << 24)) return ACL_ERR_UNSUPPORTED;
+    if (!aligned(f_in, 16) || !aligned(w_off, 16) || !aligned(w_o, 16)) return ACL_ERR_INVALID_ARG;
+    return ACL_OK;
+}
+
+void map_decoder_stage(acl::DecArgs& a, const float* f_in, int B, int Q, int D, const float* w_off,
+                       const acl_bf16* w_o, const acl_bf16* feats, const float* coords, int N, int d,
+                       const int32_t* table, int H, int W, int K, const float* p) {
+    a.f_in = f_in; a.B = B; a.Q = Q; a.D = D; a.d = d; a.w_off = w_off; a.w_o = BF(w_o);
+    acl::KnnArgs& k = a.knn;
+    k.feats = BF(feats); k.xy = coords; k.table = table; k.p = p;
+    k.B = B; k.Q = Q; k.N = N; k.d = d; k.GH = H; k.GW = W; k.K = K; k.kind = 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -371,6 +395,60 @@ acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16
                               acl_stream_t stream) {
     return acl_knn_gather_bwd_ex(queries, B, Q, feats, coords, N, d, table, H, W, K, p, ACL_KNN_EXP,
                                  dOut, dfeats, dqueries, dp, workspace, ws_bytes, stream);
+}
+
+size_t acl_decoder_layer_workspace(int B, int Q, int N, int d, int D, int K) {
+    if (B < 1 || Q < 0 || N < 1 || d < 128 || d % 128 != 0 || D < 128 || D % 128 != 0 || K < 1)
+        return 0;
+    return acl::dec_workspace_layout(B, Q, N, d, D, K).total;
+}
+
+acl_status acl_decoder_layer_fwd(const float* ref, const float* f_in, int B, int Q, int D,
+                                 const float* w_off, const float* b_off, const acl_bf16* w_o,
+                                 const acl_bf16* feats, const float* coords, int N, int d,
+                                 const int32_t* table, int H, int W, int K, const float* p,
+                                 float* q, acl_bf16* v, float* f_out, acl_stream_t stream) {
+    acl_status st = check_decoder(ref, f_in, B, Q, D, w_off, w_o, feats, coords, N, d, table, H,
+                                  W, K, p);
+    if (st != ACL_OK) return st;
+    if (!b_off || (Q > 0 && (!q || !v || !f_out))) return ACL_ERR_INVALID_ARG;
+    if (!aligned(q, 8) || !aligned(v, 16) || !aligned(f_out, 16)) return ACL_ERR_INVALID_ARG;
+    acl::DecArgs a = {};
+    map_decoder_stage(a, f_in, B, Q, D, w_off, w_o, feats, coords, N, d, table, H, W, K, p);
+    a.ref = ref; a.b_off = b_off; a.q = q; a.v = BFm(v); a.f_out = f_out;
+    return cuda_status(acl::launch_dec_fwd(a, S(stream)));
+}
+
+acl_status acl_decoder_layer_bwd(const float* f_in, int B, int Q, int D, const float* w_off,
+                                 const acl_bf16* w_o, const acl_bf16* feats, const float* coords,
+                                 int N, int d, const int32_t* table, int H, int W, int K,
+                                 const float* p, const float* q, const acl_bf16* v,
+                                 const float* df_out, float* df_in, float* dw_off, float* db_off,
+                                 float* dw_o, acl_bf16* dfeats, float* dp, void* workspace,
+                                 size_t ws_bytes, acl_stream_t stream) {
+    acl_status st = check_decoder(q, f_in, B, Q, D, w_off, w_o, feats, coords, N, d, table, H, W,
+                                  K, p);
+    if (st != ACL_OK) return st;
+    if ((Q > 0 && (!v || !df_out || !df_in)) || !dw_off || !db_off || !dw_o || !dfeats || !dp)
+        return ACL_ERR_INVALID_ARG;
+    if (!aligned(v, 16) || !aligned(df_out, 16) || !aligned(df_in, 16) || !aligned(dfeats, 16) ||
+        !aligned(dw_off, 8))
+        return ACL_ERR_INVALID_ARG;
+    const acl::DecWorkspace L = acl::dec_workspace_layout(B, Q, N, d, D, K);
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < L.total) return ACL_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    acl::DecArgs a = {};
+    map_decoder_stage(a, f_in, B, Q, D, w_off, w_o, feats, coords, N, d, table, H, W, K, p);
+    a.q = const_cast<float*>(q); a.v = const_cast<acl::bf16*>(BF(v)); a.df_out = df_out;
+    a.df_in = df_in; a.dw_off = dw_off; a.db_off = db_off; a.dw_o = dw_o;
+    a.dfb = reinterpret_cast<acl::bf16*>(ws + L.dfb);
+    a.dv = reinterpret_cast<acl::bf16*>(ws + L.dv);
+    a.dq = reinterpret_cast<float*>(ws + L.dq);
+    a.wo_part = reinterpret_cast<float*>(ws + L.wo_part);
+    a.off_part = reinterpret_cast<float*>(ws + L.off_part);
+    a.knn.dfeats = BFm(dfeats); a.knn.dp = dp;
+    map_knn_workspace(a.knn, ws + L.knn, acl::knn_workspace_layout(B, Q, N, d, K));
+    return cuda_status(acl::launch_dec_bwd(a, S(stream)));
 }
 
 }  // extern "C"

@@ -154,6 +154,39 @@ size_t merge_smem_bytes(int N, int k, int d, int h);
 cudaError_t launch_merge_fwd(const MergeArgs& m, cudaStream_t st);
 cudaError_t launch_merge_bwd(const MergeArgs& m, cudaStream_t st);
 
+struct DecArgs {
+    const float* ref;     // [B][Q][2] reference positions
+    const float* f_in;    // [B][Q][D] query features
+    int B, Q, D, d;
+    const float* w_off;   // [D][2]
+    const float* b_off;   // [2]
+    const bf16* w_o;      // [d][D]
+    float* q;             // [B][Q][2] sample positions (forward out, backward in)
+    bf16* v;              // [B][Q][d] gathered features (forward out, backward in)
+    float* f_out;         // [B][Q][D]
+    // backward
+    const float* df_out;
+    float* df_in;
+    float* dw_off;
+    float* db_off;
+    float* dw_o;          // [d][D]
+    // backward workspace
+    bf16* dfb;            // [B][Q][D] df_out in bf16
+    bf16* dv;             // [B][Q][d]
+    float* dq;            // [B][Q][2]
+    float* wo_part;       // [splits][d][D]
+    float* off_part;      // [parts][2 D + 2]
+    KnnArgs knn;          // the stage: feats, coords, table, p, sizes; dfeats, dp, workspace
+};
+
+struct DecWorkspace {
+    size_t dfb, dv, dq, wo_part, off_part, knn, total;
+};
+DecWorkspace dec_workspace_layout(int B, int Q, int N, int d, int D, int K);
+int dec_wo_splits(int T, int d, int D);
+cudaError_t launch_dec_fwd(const DecArgs& a, cudaStream_t st);
+cudaError_t launch_dec_bwd(const DecArgs& a, cudaStream_t st);
+
 size_t knn_table_smem_bytes(int N, int nbins);
 size_t token_order_smem_bytes(int N);
 cudaError_t launch_token_order(const float* xy, int B, int N, int GH, int GW, int32_t* perm,

@@ -757,12 +757,15 @@ int orc_dec_offsets(const float* ref, const double* f, int Q, int D, const doubl
 int orc_dec_project(const double* f, const double* v, int Q, int D, int d, const double* w_o,
                     double* f_out) {
     if (Q < 0 || D < 1 || d < 1) return 1;
-    for (int i = 0; i < Q; ++i)
-        for (int n = 0; n < D; ++n) {
-            double acc = f[(size_t)i * D + n];
-            for (int c = 0; c < d; ++c) acc += v[(size_t)i * d + c] * w_o[(size_t)c * D + n];
-            f_out[(size_t)i * D + n] = acc;
+    /* f_out[i][n] = f[i][n] + sum over c in order of v[i][c] w_o[c][n]; rows of w_o read whole */
+    for (int i = 0; i < Q; ++i) {
+        double* out = f_out + (size_t)i * D;
+        for (int n = 0; n < D; ++n) out[n] = f[(size_t)i * D + n];
+        for (int c = 0; c < d; ++c) {
+            const double a = v[(size_t)i * d + c];
+            for (int n = 0; n < D; ++n) out[n] += a * w_o[(size_t)c * D + n];
         }
+    }
     return 0;
 }
 
@@ -776,12 +779,17 @@ int orc_dec_project_bwd(const double* v, const double* df_out, int Q, int D, int
             for (int n = 0; n < D; ++n) acc += df_out[(size_t)i * D + n] * w_o[(size_t)c * D + n];
             dv[(size_t)i * d + c] = acc;
         }
-    for (int c = 0; c < d; ++c)
-        for (int n = 0; n < D; ++n) {
-            double acc = 0.0;
-            for (int i = 0; i < Q; ++i) acc += v[(size_t)i * d + c] * df_out[(size_t)i * D + n];
-            dw_o[(size_t)c * D + n] += acc;
+    /* each dW_o[c][n] sums v[i][c] df_out[i][n] over i in order, then joins the running total */
+    double* acc = (double*)calloc((size_t)d * D, sizeof(double));
+    if (!acc) return 2;
+    for (int i = 0; i < Q; ++i)
+        for (int c = 0; c < d; ++c) {
+            const double a = v[(size_t)i * d + c];
+            double* row = acc + (size_t)c * D;
+            for (int n = 0; n < D; ++n) row[n] += a * df_out[(size_t)i * D + n];
         }
+    for (size_t x = 0; x < (size_t)d * D; ++x) dw_o[x] += acc[x];
+    free(acc);
     return 0;
 }
 

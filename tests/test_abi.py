@@ -121,6 +121,30 @@ def test_token_merge_validation():
     assert bwd(wsb=16) == WORKSPACE
 
 
+def test_decoder_layer_validation():
+    """Every case below is rejected before any launch (the pointers are fake)."""
+    L = _lib()
+    ws = acl.acl_decoder_layer_workspace(2, 2048, 131, 768, 256, 8)
+    assert ws > 0
+    assert acl.acl_decoder_layer_workspace(2, 2048, 131, 96, 256, 8) == 0   # d % 128
+    assert acl.acl_decoder_layer_workspace(2, 2048, 131, 768, 200, 8) == 0  # D % 128
+    fwd = lambda D=256, d=768, N=131, f=P, ref=P, out=P, wo=P: L.acl_decoder_layer_fwd(
+        ref, f, 2, 2048, D, P, P, wo, P, P, N, d, P, 64, 64, 8, P, out, P, P, None)
+    assert fwd(f=None) == INVALID and fwd(ref=None) == INVALID and fwd(wo=None) == INVALID
+    assert fwd(D=200) == INVALID and fwd(d=96) == INVALID
+    assert fwd(D=1152) == UNSUPPORTED
+    assert fwd(N=16385) == UNSUPPORTED
+    assert fwd(f=P + 8) == INVALID
+    assert fwd(out=None) == INVALID
+    bwd = lambda wsb=ws, w=P, dw=P: L.acl_decoder_layer_bwd(
+        P, 2, 2048, 256, P, P, P, P, 131, 768, P, 64, 64, 8, P, P, P, P, P, dw, P, P, P, P, w,
+        wsb, None)
+    assert bwd(dw=None) == INVALID
+    assert bwd(wsb=ws - 1) == WORKSPACE
+    assert bwd(w=None) == WORKSPACE
+    assert bwd(w=P + 16) == WORKSPACE
+
+
 def test_token_order_validation():
     L = _lib()
     assert L.acl_token_order(None, 1, 10, 8, 8, P, None) == INVALID

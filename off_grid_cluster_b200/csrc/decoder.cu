@@ -230,46 +230,81 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// Offset-head backward, stage 1: CTA p takes queries [p T / P, (p + 1) T / P) in order; thread c
-// owns channel c: df_in = df_out + dq W_off^T, and its sums of f_c dq; thread 0 also sums dq.
+// Offset-head backward, stage 1: CTA p takes queries [p T / P, (p + 1) T / P); its D threads
+// are 4 row groups x D/4 channel quads, row group r taking queries t0 + r, t0 + r + 4, ... in
+// order: df_in = df_out + dq W_off^T (float4 rows), and per quad the sums of f_c dq and (quad
+// 0) of dq; the four row groups' sums are then added in row-group order.
 __global__ void __launch_bounds__(1024)
     dec_offsets_bwd_kernel(const float* __restrict__ f, const float* __restrict__ dq,
                            const float* __restrict__ df_out, int T, int D, const float* __restrict__ w_off,
                            float* __restrict__ df_in, float* __restrict__ part) {
-    const int c = threadIdx.x;
+    extern __shared__ float red[];  // [4][2 D + 2]
+    const int nq = D / 4;
+    const int rg = threadIdx.x / nq, cq = threadIdx.x - rg * nq;
     const int p = blockIdx.x;
     const int t0 = static_cast<int>(static_cast<long long>(p) * T / kDecParts);
     const int t1 = static_cast<int>(static_cast<long long>(p + 1) * T / kDecParts);
-    const float2 w = reinterpret_cast<const float2*>(w_off)[c];
-    float sx = 0.f, sy = 0.f, bx = 0.f, by = 0.f;
-#pragma unroll 4
-    for (int t = t0; t < t1; ++t) {
+    const float4 wa = reinterpret_cast<const float4*>(w_off)[2 * cq];      // channels 4cq, 4cq+1
+    const float4 wb = reinterpret_cast<const float4*>(w_off)[2 * cq + 1];  // channels 4cq+2, 4cq+3
+    float sx[4] = {0.f, 0.f, 0.f, 0.f}, sy[4] = {0.f, 0.f, 0.f, 0.f}, bx = 0.f, by = 0.f;
+#pragma unroll 2
+    for (int t = t0 + rg; t < t1; t += 4) {
         const float2 g = reinterpret_cast<const float2*>(dq)[t];
-        const size_t o = static_cast<size_t>(t) * D + c;
-        const float fv = f[o];
-        df_in[o] = df_out[o] + (g.x * w.x + g.y * w.y);
-        sx = fmaf(fv, g.x, sx);
-        sy = fmaf(fv, g.y, sy);
+        const size_t o = static_cast<size_t>(t) * nq + cq;
+        const float4 fv = reinterpret_cast<const float4*>(f)[o];
+        const float4 dv = reinterpret_cast<const float4*>(df_out)[o];
+        float4 r;
+        r.x = dv.x + (g.x * wa.x + g.y * wa.y);
+        r.y = dv.y + (g.x * wa.z + g.y * wa.w);
+        r.z = dv.z + (g.x * wb.x + g.y * wb.y);
+        r.w = dv.w + (g.x * wb.z + g.y * wb.w);
+        reinterpret_cast<float4*>(df_in)[o] = r;
+        const float fa[4] = {fv.x, fv.y, fv.z, fv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sx[e] = fmaf(fa[e], g.x, sx[e]);
+            sy[e] = fmaf(fa[e], g.y, sy[e]);
+        }
         bx += g.x;
         by += g.y;
     }
-    float* pp = part + static_cast<size_t>(p) * (2 * D + 2);
-    reinterpret_cast<float2*>(pp)[c] = make_float2(sx, sy);
-    if (c == 0) reinterpret_cast<float2*>(pp)[D] = make_float2(bx, by);
+    const int n = 2 * D + 2;
+    float* my = red + rg * n;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        my[2 * (4 * cq + e)] = sx[e];
+        my[2 * (4 * cq + e) + 1] = sy[e];
+    }
+    if (cq == 0) {
+        my[2 * D] = bx;
+        my[2 * D + 1] = by;
+    }
+    __syncthreads();
+    float* pp = part + static_cast<size_t>(p) * n;
+    for (int o = threadIdx.x; o < n; o += blockDim.x) pp[o] = ((red[o] + red[n + o]) + red[2 * n + o]) + red[3 * n + o];
 }
 
-// Stage 2: the parts summed in order -> dW_off [D][2], db_off [2].
+// Stage 2: CTA over 32 outputs; warp w adds parts w, w + 8, ... in order, then the eight warp
+// sums are added in warp order -> dW_off [D][2], db_off [2].
 __global__ void __launch_bounds__(256)
     dec_offsets_reduce_kernel(const float* __restrict__ part, int D, float* __restrict__ dw_off,
                               float* __restrict__ db_off) {
-    const int o = blockIdx.x * 256 + threadIdx.x;
+    __shared__ float wsum[8][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int o = blockIdx.x * 32 + lane;
     const int n = 2 * D + 2;
-    if (o >= n) return;
     float a = 0.f;
+    if (o < n)
 #pragma unroll 8
-    for (int p = 0; p < kDecParts; ++p) a += part[static_cast<size_t>(p) * n + o];
-    if (o < 2 * D) dw_off[o] = a;
-    else db_off[o - 2 * D] = a;
+        for (int p = warp; p < kDecParts; p += 8) a += part[static_cast<size_t>(p) * n + o];
+    wsum[warp][lane] = a;
+    __syncthreads();
+    if (warp != 0 || o >= n) return;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += wsum[w][lane];
+    if (o < 2 * D) dw_off[o] = sum;
+    else db_off[o - 2 * D] = sum;
 }
 
 // dW_o = the split parts summed in order.
@@ -371,10 +406,12 @@ cudaError_t launch_dec_bwd(const DecArgs& a, cudaStream_t st) {
     k.dout = a.dv;
     k.dq = a.dq;
     if ((e = launch_knn_bwd(k, st)) != cudaSuccess) return e;
-    dec_offsets_bwd_kernel<<<kDecParts, a.D, 0, st>>>(a.f_in, a.dq, a.df_out, T, a.D, a.w_off, a.df_in,
-                                                       a.off_part);
+    const size_t osm = sizeof(float) * 4 * (2 * static_cast<size_t>(a.D) + 2);
+    if ((e = ensure_smem<dec_offsets_bwd_kernel>(osm)) != cudaSuccess) return e;
+    dec_offsets_bwd_kernel<<<kDecParts, a.D, osm, st>>>(a.f_in, a.dq, a.df_out, T, a.D, a.w_off, a.df_in,
+                                                         a.off_part);
     note_launch();
-    dec_offsets_reduce_kernel<<<(2 * a.D + 2 + 255) / 256, 256, 0, st>>>(a.off_part, a.D, a.dw_off, a.db_off);
+    dec_offsets_reduce_kernel<<<(2 * a.D + 2 + 31) / 32, 256, 0, st>>>(a.off_part, a.D, a.dw_off, a.db_off);
     note_launch();
     return cudaGetLastError();
 }

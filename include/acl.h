@@ -53,7 +53,7 @@ typedef enum {
     ACL_ERR_UNSUPPORTED = 3,   /* valid arguments outside what the kernels implement   */
     ACL_ERR_WORKSPACE = 4,     /* workspace pointer null or smaller than required     */
     ACL_ERR_DEVICE_CHECK = 5,  /* reserved: device-side consistency check failed      */
-    ACL_ERR_TIMEOUT = 6        /* reserved: a bounded device wait gave up              */
+    ACL_ERR_TIMEOUT = 6        /* a bounded device wait gave up (acl_device_check)     */
 } acl_status;
 
 /* Same type as cudaStream_t (both are pointers to struct CUstream_st). */
@@ -415,6 +415,13 @@ acl_status acl_knn_gather_bwd_indexed_ex(const float* queries, int B, int Q,
  * on the fp32 q.
  */
 size_t acl_decoder_layer_workspace(int B, int Q, int N, int d, int D, int K);
+/*
+ * acl_device_check -- synchronises the current device, then reports (and clears) whether
+ * any bounded device-side wait of the library's tensor-core kernels gave up since the last
+ * call: ACL_ERR_TIMEOUT if so (the affected outputs are zero, not garbage), ACL_OK if not,
+ * ACL_ERR_CUDA if synchronising failed.
+ */
+acl_status acl_device_check(void);
 acl_status acl_decoder_layer_fwd(const float* ref, const float* f_in, int B, int Q, int D,
                                  const float* w_off, const float* b_off, const acl_bf16* w_o,
                                  const acl_bf16* feats, const float* coords, int N, int d,

@@ -48,6 +48,7 @@ SIGNATURES = {
                                  _P, _P, _P, _P, _P, _P, _Z, _P]),
     "acl_knn_gather_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "acl_decoder_layer_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "acl_device_check": (_I, []),
     "acl_decoder_layer_fwd": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I,
                                    _I, _P, _P, _P, _P, _P]),
     "acl_decoder_layer_bwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P,
@@ -347,6 +348,11 @@ def _gather_shapes(queries, feats, coords, table, p):
 
 
 ACL_KNN_EXP, ACL_KNN_INVPOW = 0, 1  # weight kernels: softmax(-p d), d^-p / sum d^-p
+
+
+def acl_device_check() -> None:
+    """Synchronise the device; raise if a bounded device-side wait gave up."""
+    _call("acl_device_check")
 
 
 def acl_decoder_layer_workspace(B: int, Q: int, N: int, d: int, D: int, K: int = 8) -> int:

@@ -397,6 +397,13 @@ acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16
                                  dOut, dfeats, dqueries, dp, workspace, ws_bytes, stream);
 }
 
+acl_status acl_device_check(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return ACL_ERR_CUDA;
+    unsigned int n = 0;
+    if (acl::read_tc_timeouts(&n) != cudaSuccess) return ACL_ERR_CUDA;
+    return n ? ACL_ERR_TIMEOUT : ACL_OK;
+}
+
 size_t acl_decoder_layer_workspace(int B, int Q, int N, int d, int D, int K) {
     if (B < 1 || Q < 0 || N < 1 || d < 128 || d % 128 != 0 || D < 128 || D % 128 != 0 || K < 1)
         return 0;

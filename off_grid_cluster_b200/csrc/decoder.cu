@@ -13,10 +13,9 @@
 //   KNN backward of dv -> dfeats, dq, dp,
 //   df_in = df_out + dq W_off^T, dW_off = f^T dq, db_off = sum dq (fixed-order sums).
 //
-// The GEMMs: mma.sync m16n8k16 bf16 -> fp32, 128 x 128 CTA tiles, 32-deep k-steps through a
-// 3-stage cp.async pipeline; each operand is staged in its stored layout (k-contiguous rows
-// of 64 bytes, or k-rows of 128 elements, 256 bytes) with an XOR swizzle and fragments are
-// read by ldmatrix (.trans for k-row tiles), so no operand is transposed in memory.
+// The GEMMs run on the tcgen05 tensor cores with the accumulator in tensor memory; each
+// operand is staged in its stored layout (K-major or MN-major shared-memory descriptors), so
+// no operand is transposed in memory.
 #include <float.h>
 
 #include "internal.h"
@@ -25,10 +24,6 @@ namespace acl {
 
 namespace {
 
-constexpr int kGM = 128, kGN = 128, kGK = 32, kGStages = 3, kGThreads = 256;
-constexpr int kGTileBytes = kGM * kGK * 2;          // 8 KB, either layout
-constexpr int kGStageBytes = 2 * kGTileBytes;       // A and B
-constexpr int kGSmem = kGStages * kGStageBytes;     // 48 KB
 constexpr int kDecParts = 296;                      // query ranges of the offset-head sums
 constexpr int kMaxSplits = 16;                      // k-splits of the dW_o GEMM
 
@@ -47,140 +42,237 @@ struct GemmArgs {
     size_t part_stride;
 };
 
-// k-row tile [32][128]: 16-byte chunk ch of k-row kr at chunk ch ^ (kr & 7), so the 8 rows an
-// ldmatrix.trans reads fall in 8 distinct bank groups.
-__device__ __forceinline__ uint32_t tile256_off(int kr, int ch) {
-    return static_cast<uint32_t>(kr * 256 + ((ch ^ (kr & 7)) << 4));
+// ---------------------------------------------------------------- tcgen05 GEMM
+//
+// The same products on the 5th-generation tensor cores: a 128 x 128 fp32 accumulator in
+// tensor memory (128 columns), 64-deep k-tiles staged by cp.async into shared memory in the
+// canonical 128-byte-swizzle layouts (K-major: 128-byte rows, 16-byte chunk c of row r at
+// c ^ (r mod 8); MN-major: two 64-element halves of 64 k-rows each, the same swizzle on the
+// k-row), 3 stages.  One thread issues the four k16 MMAs of a stage and commits them to the
+// stage's mbarrier; a stage is refilled only after that barrier completes.  Every wait is
+// bounded: a wait that gives up counts in tc_timeouts (read by acl_device_check) and the CTA
+// skips its remaining MMAs, waits once more for those in flight and frees its tensor memory.
+constexpr int kTM = 128, kTN = 128, kTK = 64, kTStages = 3, kTThreads = 256;
+constexpr int kTTileBytes = kTM * kTK * 2;                  // 16 KB, A or B
+constexpr int kTStageBytes = 2 * kTTileBytes;
+constexpr int kTSmem = kTStages * kTStageBytes + 1024 + 64;  // + alignment slack, barriers, slot
+constexpr long long kTWaitCycles = 1000000000LL;
+constexpr uint32_t kTmemCols = 128;
+
+__device__ unsigned int tc_timeouts;
+
+// Shared-memory matrix descriptor: start, leading and stride byte offsets in 16-byte units,
+// descriptor version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo16, uint32_t sbo16) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(lbo16 & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>(sbo16 & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Operand descriptor of k16 step j of a staged tile: K-major tiles advance 32 bytes inside the
+// swizzle atom (8-row groups 1024 bytes apart); MN-major tiles advance 16 k-rows (2048 bytes),
+// their two 64-element halves 8192 bytes apart and 8-k-row groups 1024 bytes apart.
+template <bool MN>
+__device__ __forceinline__ uint64_t tile_desc(uint32_t tile, int j) {
+    return MN ? umma_desc(tile + 2048u * j, 8192u >> 4, 1024u >> 4) : umma_desc(tile + 32u * j, 1u, 1024u >> 4);
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, majors, N / 8, M / 16.
+template <bool AMN, bool BMN>
+__host__ __device__ constexpr uint32_t tc_idesc() {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((AMN ? 1u : 0u) << 15) | ((BMN ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(kTN >> 3) << 17) | (static_cast<uint32_t>(kTM >> 4) << 24);
 }
 
-// One operand tile, 512 chunks of 16 bytes (two per thread).  KROW: stored [K][rows] (rows
-// contiguous; the tile is 32 k-rows x 128), else [rows][K] (the tile is 128 rows x 32 k).
-// Chunks outside [0, rows) x [k0, kend) are zero-filled.  rows % 8 == 0 for KROW and
-// kend % 8 == 0 otherwise, so a chunk is wholly inside or outside.
-template <bool KROW>
-__device__ __forceinline__ void gemm_load_tile(uint32_t sbase, const bf16* __restrict__ src, int ld,
-                                               int row0, int rows, int k0, int kend, int tid) {
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Wait for the phase of the given parity to complete, giving up after kTWaitCycles SM clocks
+// (about half a second): try_wait itself returns after a bounded suspension.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (clock64() - t0 > kTWaitCycles) return false;
+    }
+}
+
+// Stage one operand tile (1024 chunks of 16 bytes, 4 per thread).  MN: stored [K][MN]
+// (MN contiguous), rows = extent of MN; else stored [MN][K].  Out-of-range chunks are zeroed.
+template <bool MN>
+__device__ __forceinline__ void tc_load_tile(uint32_t tile, const bf16* __restrict__ src, int ld, int mn0,
+                                             int rows, int k0, int kend, int tid) {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int q = tid + i * kGThreads;
-        if constexpr (!KROW) {
-            const int r = q >> 2, ch = q & 3;
-            const int gr = row0 + r, gk = k0 + 8 * ch;
+    for (int i = 0; i < 1024 / kTThreads; ++i) {
+        const int q = tid + i * kTThreads;
+        if constexpr (!MN) {
+            const int r = q >> 3, c = q & 7;
+            const int gr = mn0 + r, gk = k0 + 8 * c;
             const bool ok = gr < rows && gk < kend;
-            cp_async16(sbase + tile64_off(r, ch), ok ? src + static_cast<size_t>(gr) * ld + gk : src, ok);
+            cp_async16(tile + r * 128 + ((c ^ (r & 7)) << 4), ok ? src + static_cast<size_t>(gr) * ld + gk : src, ok);
         } else {
-            const int kr = q >> 4, ch = q & 15;
-            const int gk = k0 + kr, gc = row0 + 8 * ch;
+            const int kr = q >> 4, mc = q & 15, h = mc >> 3, c = mc & 7;
+            const int gk = k0 + kr, gc = mn0 + 8 * mc;
             const bool ok = gk < kend && gc < rows;
-            cp_async16(sbase + tile256_off(kr, ch), ok ? src + static_cast<size_t>(gk) * ld + gc : src, ok);
+            cp_async16(tile + h * 8192 + kr * 128 + ((c ^ (kr & 7)) << 4),
+                       ok ? src + static_cast<size_t>(gk) * ld + gc : src, ok);
         }
     }
 }
 
-template <bool AKROW, bool BKROW, int EPI>
-__global__ void __launch_bounds__(kGThreads)
-    dec_gemm_kernel(const GemmArgs g) {
-    extern __shared__ __align__(128) uint8_t gsm[];
-    const uint32_t s0 = smem_addr(gsm);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int m0 = blockIdx.y * kGM, n0 = blockIdx.x * kGN;
-    const int wm = (warp >> 2) * 64, wn = (warp & 3) * 32;
+template <bool AMN, bool BMN, int EPI>
+__global__ void __launch_bounds__(kTThreads)
+    tc_gemm_kernel(const GemmArgs g) {
+    extern __shared__ uint8_t tsm[];
+    const uint32_t raw = smem_addr(tsm);
+    const uint32_t s0 = (raw + 1023u) & ~1023u;
+    const uint32_t bar0 = s0 + kTStages * kTStageBytes;
+    const uint32_t slot = bar0 + 8 * kTStages;
+    const volatile uint32_t* slot_p = reinterpret_cast<const volatile uint32_t*>(tsm + (slot - raw));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m0 = blockIdx.y * kTM, n0 = blockIdx.x * kTN;
     const int kz0 = blockIdx.z * g.kchunk;
     const int kz1 = min(g.K, kz0 + g.kchunk);
-    const int nk = kz1 > kz0 ? (kz1 - kz0 + kGK - 1) / kGK : 0;
+    const int nk = kz1 > kz0 ? (kz1 - kz0 + kTK - 1) / kTK : 0;
 
-    auto load_stage = [&](int stage, int kt) {
-        const uint32_t sa = s0 + stage * kGStageBytes, sb = sa + kGTileBytes;
-        const int k0 = kz0 + kt * kGK;
-        gemm_load_tile<AKROW>(sa, g.A, g.lda, m0, g.M, k0, kz1, tid);
-        gemm_load_tile<BKROW>(sb, g.B, g.ldb, n0, g.N, k0, kz1, tid);
+    if (tid == 0) {
+        for (int s = 0; s < kTStages; ++s)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar0 + 8 * s), "r"(1) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *slot_p;
+
+    auto load = [&](int stage, int kt) {
+        const uint32_t sa = s0 + stage * kTStageBytes, sb = sa + kTTileBytes;
+        const int k0 = kz0 + kt * kTK;
+        tc_load_tile<AMN>(sa, g.A, g.lda, m0, g.M, k0, kz1, tid);
+        tc_load_tile<BMN>(sb, g.B, g.ldb, n0, g.N, k0, kz1, tid);
     };
-
-    float acc[4][4][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-
-#pragma unroll
-    for (int s = 0; s < kGStages - 1; ++s) {
-        if (s < nk) load_stage(s, s);
+    for (int s = 0; s < kTStages - 1; ++s) {
+        if (s < nk) load(s, s);
         cp_async_commit();
     }
-    const int mi = lane >> 3, r8 = lane & 7;
+    bool ok = true;
+    int issued = 0;  // k-tiles whose MMAs were issued
     for (int kt = 0; kt < nk; ++kt) {
-        cp_async_wait<kGStages - 2>();
-        __syncthreads();
-        const int nxt = kt + kGStages - 1;
-        if (nxt < nk) load_stage(nxt % kGStages, nxt);
-        cp_async_commit();
-        const uint32_t sa = s0 + (kt % kGStages) * kGStageBytes, sb = sa + kGTileBytes;
+        cp_async_wait<kTStages - 2>();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (!__syncthreads_and(ok)) break;  // a wait gave up somewhere: stop issuing
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t sa = s0 + (kt % kTStages) * kTStageBytes, sb = sa + kTTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kGK; kk += 16) {
-            uint32_t af[4][4], bfr[4][2];
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt) {
-                if constexpr (!AKROW) {
-                    const int row = wm + 16 * mt + (lane & 15), ch = (kk >> 3) + (lane >> 4);
-                    ldsm_x4(sa + tile64_off(row, ch), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-                } else {
-                    const int kr = kk + r8 + 8 * (mi >> 1), ch = ((wm + 16 * mt) >> 3) + (mi & 1);
-                    ldsm_x4_t(sa + tile256_off(kr, ch), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-                }
+            for (int j = 0; j < kTK / 16; ++j) {
+                const uint64_t ad = tile_desc<AMN>(sa, j), bd = tile_desc<BMN>(sb, j);
+                const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\t"
+                    "setp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+                    ::"r"(tmem), "l"(ad), "l"(bd), "r"(tc_idesc<AMN, BMN>()), "r"(acc), "r"(0u), "r"(0u), "r"(0u),
+                    "r"(0u)
+                    : "memory");
             }
-#pragma unroll
-            for (int pr = 0; pr < 2; ++pr) {
-                if constexpr (!BKROW) {
-                    const int row = wn + 16 * pr + 8 * (mi >> 1) + r8, ch = (kk >> 3) + (mi & 1);
-                    ldsm_x4(sb + tile64_off(row, ch), bfr[2 * pr][0], bfr[2 * pr][1], bfr[2 * pr + 1][0],
-                            bfr[2 * pr + 1][1]);
-                } else {
-                    const int kr = kk + r8 + 8 * (mi & 1), ch = ((wn + 16 * pr) >> 3) + (mi >> 1);
-                    ldsm_x4_t(sb + tile256_off(kr, ch), bfr[2 * pr][0], bfr[2 * pr][1], bfr[2 * pr + 1][0],
-                              bfr[2 * pr + 1][1]);
-                }
-            }
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-                    mma_bf16(acc[mt][nt], af[mt][0], af[mt][1], af[mt][2], af[mt][3], bfr[nt][0], bfr[nt][1]);
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             bar0 + 8 * (kt % kTStages))
+                         : "memory");
         }
+        issued = kt + 1;
+        const int nxt = kt + kTStages - 1;
+        if (nxt < nk) {
+            if (kt >= 1) ok = ok && mbar_wait(bar0 + 8 * ((kt - 1) % kTStages), ((kt - 1) / kTStages) & 1);
+            if (ok) load(nxt % kTStages, nxt);
+        }
+        cp_async_commit();
     }
     cp_async_wait<0>();
-
-    const int gq = lane >> 2, tq = lane & 3;
+    // the last commit covers every MMA issued before it
+    if (issued > 0) {
+        const bool done = mbar_wait(bar0 + 8 * ((issued - 1) % kTStages), ((issued - 1) / kTStages) & 1);
+        ok = ok && done;
+    }
+    ok = __syncthreads_and(ok) != 0;
+    tc_fence_after();
+    const bool have = ok && nk > 0 && issued == nk;
+    // warp w reads tensor-memory lanes 32 (w mod 4) .. + 31 (its rows), columns of half w / 4
+    const int row = m0 + 32 * (warp & 3) + lane;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    const int c0 = (warp >> 2) * (kTN / 2);
+#pragma unroll 1
+    for (int cj = c0; cj < c0 + kTN / 2; cj += 16) {
+        uint32_t v[16];
+        if (have) {
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                "%13, %14, %15}, [%16];\n"
+                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                  "=r"(v[15])
+                : "r"(taddr + cj));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        } else {
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int r = m0 + wm + 16 * mt + gq + 8 * h;
-            if (r >= g.M) continue;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int c = n0 + wn + 8 * nt + 2 * tq;
-                const float x0 = acc[mt][nt][2 * h], x1 = acc[mt][nt][2 * h + 1];
-                const size_t o = static_cast<size_t>(r) * g.ldc + c;
-                if constexpr (EPI == kEpiResid) {
-                    const float2 rv = *reinterpret_cast<const float2*>(g.R + o);
-                    *reinterpret_cast<float2*>(g.Cf + o) = make_float2(x0 + rv.x, x1 + rv.y);
-                } else if constexpr (EPI == kEpiBf16) {
-                    *reinterpret_cast<uint32_t*>(g.Cb + o) = pack_bf16(x0, x1);
-                } else {
-                    *reinterpret_cast<float2*>(g.Cf + blockIdx.z * g.part_stride + o) = make_float2(x0, x1);
-                }
-            }
+            for (int e = 0; e < 16; ++e) v[e] = 0u;
         }
+        if (row >= g.M) continue;
+        const size_t o = static_cast<size_t>(row) * g.ldc + n0 + cj;
+        if constexpr (EPI == kEpiResid) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4) {
+                const float4 r4 = *reinterpret_cast<const float4*>(g.R + o + e);
+                *reinterpret_cast<float4*>(g.Cf + o + e) =
+                    make_float4(__uint_as_float(v[e]) + r4.x, __uint_as_float(v[e + 1]) + r4.y,
+                                __uint_as_float(v[e + 2]) + r4.z, __uint_as_float(v[e + 3]) + r4.w);
+            }
+        } else if constexpr (EPI == kEpiBf16) {
+            uint4 w0, w1;
+            w0.x = pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1]));
+            w0.y = pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3]));
+            w0.z = pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5]));
+            w0.w = pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7]));
+            w1.x = pack_bf16(__uint_as_float(v[8]), __uint_as_float(v[9]));
+            w1.y = pack_bf16(__uint_as_float(v[10]), __uint_as_float(v[11]));
+            w1.z = pack_bf16(__uint_as_float(v[12]), __uint_as_float(v[13]));
+            w1.w = pack_bf16(__uint_as_float(v[14]), __uint_as_float(v[15]));
+            *reinterpret_cast<uint4*>(g.Cb + o) = w0;
+            *reinterpret_cast<uint4*>(g.Cb + o + 8) = w1;
+        } else {
+            float* dst = g.Cf + blockIdx.z * g.part_stride + o;
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+                *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                                                  __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+    if (!ok && tid == 0) atomicAdd(&tc_timeouts, 1u);
 }
 
-template <bool AKROW, bool BKROW, int EPI>
-cudaError_t launch_gemm(const GemmArgs& g, int splits, cudaStream_t st) {
-    cudaError_t e = ensure_smem<dec_gemm_kernel<AKROW, BKROW, EPI>>(kGSmem);
+template <bool AMN, bool BMN, int EPI>
+cudaError_t launch_tc_gemm(const GemmArgs& g, int splits, cudaStream_t st) {
+    cudaError_t e = ensure_smem<tc_gemm_kernel<AMN, BMN, EPI>>(kTSmem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(g.N / kGN, (g.M + kGM - 1) / kGM, splits);
-    dec_gemm_kernel<AKROW, BKROW, EPI><<<grid, kGThreads, kGSmem, st>>>(g);
+    const dim3 grid(g.N / kTN, (g.M + kTM - 1) / kTM, splits);
+    tc_gemm_kernel<AMN, BMN, EPI><<<grid, kTThreads, kTSmem, st>>>(g);
     note_launch();
     return cudaGetLastError();
 }
@@ -327,12 +419,19 @@ int sm_count() {
 }  // namespace
 
 int dec_wo_splits(int T, int d, int D) {
-    const int tiles = (d / kGM) * (D / kGN);
+    const int tiles = (d / kTM) * (D / kTN);
     int s = (2 * 148 + tiles - 1) / tiles;
-    const int kt = (T + kGK - 1) / kGK;
+    const int kt = (T + kTK - 1) / kTK;
     if (s > kt) s = kt;
     if (s > kMaxSplits) s = kMaxSplits;
     return s < 1 ? 1 : s;
+}
+
+cudaError_t read_tc_timeouts(unsigned int* count) {
+    cudaError_t e = cudaMemcpyFromSymbol(count, tc_timeouts, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(tc_timeouts, &zero, sizeof(unsigned int));
 }
 
 DecWorkspace dec_workspace_layout(int B, int Q, int N, int d, int D, int K) {
@@ -367,7 +466,7 @@ cudaError_t launch_dec_fwd(const DecArgs& a, cudaStream_t st) {
     g.B = a.w_o; g.ldb = a.D;               // [d][D], k-rows
     g.M = T; g.N = a.D; g.K = a.d; g.kchunk = a.d;
     g.R = a.f_in; g.Cf = a.f_out; g.ldc = a.D;
-    return launch_gemm<false, true, kEpiResid>(g, 1, st);
+    return launch_tc_gemm<false, true, kEpiResid>(g, 1, st);
 }
 
 cudaError_t launch_dec_bwd(const DecArgs& a, cudaStream_t st) {
@@ -386,17 +485,17 @@ cudaError_t launch_dec_bwd(const DecArgs& a, cudaStream_t st) {
         g.B = a.w_o; g.ldb = a.D;
         g.M = T; g.N = a.d; g.K = a.D; g.kchunk = a.D;
         g.Cb = a.dv; g.ldc = a.d;
-        if ((e = launch_gemm<false, false, kEpiBf16>(g, 1, st)) != cudaSuccess) return e;
+        if ((e = launch_tc_gemm<false, false, kEpiBf16>(g, 1, st)) != cudaSuccess) return e;
     }
     // dW_o = v^T df: A(m = d, k = T) = v[k][m] (k-rows), B(k = T, n = D) = df[k][n] (k-rows)
     const int splits = dec_wo_splits(T, a.d, a.D);
-    const int kt = (T + kGK - 1) / kGK;
+    const int kt = (T + kTK - 1) / kTK;
     GemmArgs w = {};
     w.A = a.v; w.lda = a.d;
     w.B = a.dfb; w.ldb = a.D;
-    w.M = a.d; w.N = a.D; w.K = T; w.kchunk = ((kt + splits - 1) / splits) * kGK;
+    w.M = a.d; w.N = a.D; w.K = T; w.kchunk = ((kt + splits - 1) / splits) * kTK;
     w.Cf = a.wo_part; w.ldc = a.D; w.part_stride = static_cast<size_t>(a.d) * a.D;
-    if ((e = launch_gemm<true, true, kEpiPart>(w, splits, st)) != cudaSuccess) return e;
+    if ((e = launch_tc_gemm<true, true, kEpiPart>(w, splits, st)) != cudaSuccess) return e;
     const size_t nw = static_cast<size_t>(a.d) * a.D;
     dec_split_reduce_kernel<<<static_cast<unsigned>((nw + 255) / 256), 256, 0, st>>>(a.wo_part, nw, splits, a.dw_o);
     note_launch();

@@ -184,6 +184,8 @@ struct DecWorkspace {
 };
 DecWorkspace dec_workspace_layout(int B, int Q, int N, int d, int D, int K);
 int dec_wo_splits(int T, int d, int D);
+// reads and clears the count of bounded tensor-core waits that gave up (synchronous)
+cudaError_t read_tc_timeouts(unsigned int* count);
 cudaError_t launch_dec_fwd(const DecArgs& a, cudaStream_t st);
 cudaError_t launch_dec_bwd(const DecArgs& a, cudaStream_t st);
 

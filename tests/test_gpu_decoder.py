@@ -33,6 +33,7 @@ def layer_both(ref, f_in, w_off, b_off, w_o, st, df, table=None):
     err = np.abs(host(f_out) - f_ref).max()
     assert err <= FWD_ATOL, f"f_out: max abs err {err:.3e}"
     grads = acl.acl_decoder_layer_bwd(f_d, woff_d, wo_d, q=q, v=v, df_out=dev(df), **g)
+    acl.acl_device_check()  # no bounded tensor-core wait gave up
     refs = oracle.decoder_layer_bwd(f_in, w_off, st.feats, st.coords, table, st.p, w_o, q_h, v_ref, df)
     for name, got, want in zip(("df_in", "dW_off", "db_off", "dfeats", "dp", "dW_o"),
                                (grads[0], grads[1], grads[2], grads[4], grads[5], grads[3]), refs):

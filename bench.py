@@ -65,10 +65,12 @@ KERNELS = {
 # DRAM bytes per launch measured by ncu for each call (sum over its kernels), with the
 # sha256 of the CUDA source the counters were taken on; a stale hash reports null.
 NCU_TRAFFIC: dict[str, tuple[float, str, str]] = {
-    "attn_fwd": (13202176.0, "139177723ccca99c", "profiles/attn_kernels_step_workload.md"),
-    "attn_bwd": (35377408.0, "139177723ccca99c", "profiles/attn_kernels_step_workload.md"),
-    "knn_table": (178432.0, "139177723ccca99c", "profiles/knn_kernels_step_workload.md"),
+    # call: (DRAM bytes read + written per launch, hash of the sources of its kernels, summary)
+    "attn_fwd": (13202176.0, "77c27f1c2b1cfe11", "profiles/attn_kernels_step_workload.md"),
+    "attn_bwd": (35377408.0, "77c27f1c2b1cfe11", "profiles/attn_kernels_step_workload.md"),
 }
+# the files whose code makes each call's kernels (the traffic goes stale when they change)
+TRAFFIC_SOURCES = {"attn_fwd": ("attn.cu", "common.cuh"), "attn_bwd": ("attn.cu", "common.cuh")}
 
 
 # --------------------------------------------------------------------------- helpers
@@ -134,10 +136,11 @@ def measured_peaks() -> dict:
             "source": "fallback 6.65 TB/s, 1590 TFLOP/s"}
 
 
-def source_hash() -> str:
+def source_hash(names=None) -> str:
+    """Hash of the named CUDA sources (all of them when names is None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "off_grid_cluster_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(names if names is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -483,7 +486,7 @@ def run_gpu(args, rank: int, world: int):
     achieved = abytes[dom_name] / (per_op[dom] * 1e-3) / 1e9
     traffic = None
     traffic_src = None
-    if dom_name in NCU_TRAFFIC and NCU_TRAFFIC[dom_name][1] == source_hash():
+    if dom_name in NCU_TRAFFIC and NCU_TRAFFIC[dom_name][1] == source_hash(TRAFFIC_SOURCES[dom_name]):
         traffic, traffic_src = NCU_TRAFFIC[dom_name][0], NCU_TRAFFIC[dom_name][2]
     breakdown = {}
     for j, name in enumerate(OPS):

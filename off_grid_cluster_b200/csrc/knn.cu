@@ -788,7 +788,7 @@ constexpr int kCsrListCap = 12288;  // entries of a slice listed in shared memor
 constexpr int kHeavyEntries = 96;  // tokens with more entries are reduced by a whole CTA
 constexpr int kChunkUnits = 64;   // work units (1 per token + 1 per entry) per light chunk
 constexpr int kChunkIds = 192;    // staged ids per warp (>= kChunkUnits + kHeavyEntries)
-constexpr int kHeavyCtas = 128;   // CTAs of the token pass that take the heavy tokens
+constexpr int kHeavyCtas = 128;   // CTAs of the token pass that take the heavy tokens (default)
 static_assert(kChunkUnits <= kHeavyEntries + 1, "a chunk's tokens other than its last must be light");
 static_assert(kChunkIds >= kChunkUnits + kHeavyEntries, "a chunk's light entries must fit the staging");
 
@@ -1033,7 +1033,7 @@ __global__ void __launch_bounds__(kCsrThreads)
 //     starts in it.  One lane group per chunk stages the entry ids of its tokens in shared
 //     memory (one round of independent loads), then walks them with the next batch's w and
 //     dOut loads in flight, summing each token's entries in ascending order;
-//   heavy tokens (listed per CSR slice): the first kHeavyCtas CTAs take them in a fixed
+//   heavy tokens (listed per CSR slice): the first hctas CTAs (heavy_ctas) take them in a fixed
 //     stride; all 8 warps x (32 / LPQ) lane groups stream every S-th entry, combined by a
 //     fixed shuffle tree and a fixed-order pass over warps.
 // Every token's sum is formed the same way on every run: bit-reproducible.  The first NH
@@ -1061,18 +1061,18 @@ __device__ __forceinline__ void token_streams(const KnnArgs& a, int b, int lo, i
         const int mine = (kk < n) ? __ldg(csr + lo + sid + nstreams * kk) : 0;
         const int cnt = min(LPQ, n - k0);
         int u = 0;
-        for (; u + 4 <= cnt; u += 4) {
-            float wv[4];
-            uint4 gv[4];
+        for (; u + 8 <= cnt; u += 8) {
+            float wv[8];
+            uint4 gv[8];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
+            for (int x = 0; x < 8; ++x) {
                 const int e = __shfl_sync(gmask, mine, u + x, LPQ);
                 const int q = e >> 4, j = e & 15;
                 wv[x] = __ldg(wb + q * KN + j * NH);
                 gv[x] = on ? ldg16(gb + q * a.d) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
-            for (int x = 0; x < 4; ++x) fma8(acc, wv[x], gv[x]);
+            for (int x = 0; x < 8; ++x) fma8(acc, wv[x], gv[x]);
         }
         for (; u < cnt; ++u) {
             const int e = __shfl_sync(gmask, mine, u, LPQ);
@@ -1119,7 +1119,8 @@ __device__ void heavy_token(const KnnArgs& a, int b, int t, int l2, float (*part
 }
 
 __global__ void __launch_bounds__(kGatherThreads, 4)
-    knn_bwd_token_kernel(const KnnArgs a, int lpq_log2, int query_blocks, int nlists, int chunks) {
+    knn_bwd_token_kernel(const KnnArgs a, int lpq_log2, int query_blocks, int nlists, int chunks,
+                         int hctas) {
     constexpr int STEPS = 4;  // warp steps whose loads are in flight together
     __shared__ float part[kGatherWarps][256];
     __shared__ int hpre[kGatherThreads];
@@ -1127,7 +1128,7 @@ __global__ void __launch_bounds__(kGatherThreads, 4)
     __shared__ int ids_smem[kGatherWarps][kChunkIds];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NH = a.d >> 5;
-    if (static_cast<int>(blockIdx.x) < kHeavyCtas) {
+    if (static_cast<int>(blockIdx.x) < hctas) {
         const int h = blockIdx.x;
         if (h < NH) {
             float acc = 0.f;
@@ -1143,7 +1144,7 @@ __global__ void __launch_bounds__(kGatherThreads, 4)
             }
             __syncthreads();
         }
-        // heavy items h, h + kHeavyCtas, ... of the concatenated per-(image, slice) lists,
+        // heavy items h, h + hctas, ... of the concatenated per-(image, slice) lists,
         // scanned kGatherThreads lists at a time
         const int slices = nlists / a.B;
         int run = 0;
@@ -1152,8 +1153,8 @@ __global__ void __launch_bounds__(kGatherThreads, 4)
             hpre[threadIdx.x] = (static_cast<int>(threadIdx.x) < nl) ? a.heavy_count[l0 + threadIdx.x] : 0;
             __syncthreads();
             const int tot = block_scan(hpre, kGatherThreads, scan_scratch);  // hpre: exclusive
-            int i = run + ((h - run % kHeavyCtas) + kHeavyCtas) % kHeavyCtas;  // first i >= run, i = h mod
-            for (; i < run + tot; i += kHeavyCtas) {
+            int i = run + ((h - run % hctas) + hctas) % hctas;  // first i >= run, i = h mod hctas
+            for (; i < run + tot; i += hctas) {
                 const int r = i - run;
                 int li = 0, hl = nl - 1;  // last list whose prefix is <= r
                 while (li < hl) {
@@ -1175,7 +1176,7 @@ __global__ void __launch_bounds__(kGatherThreads, 4)
     // loaded together, and the slots are combined by a fixed xor tree at the token's end.
     const int LPQ = 1 << lpq_log2, EPS = 32 >> lpq_log2;
     const int slot = lane >> lpq_log2, sub = lane & (LPQ - 1);
-    const int gid = (static_cast<int>(blockIdx.x) - kHeavyCtas) * kGatherWarps + warp;
+    const int gid = (static_cast<int>(blockIdx.x) - hctas) * kGatherWarps + warp;
     const int b = gid / chunks;
     if (b >= a.B) return;  // whole warps leave together
     const int c = gid - b * chunks;
@@ -1254,6 +1255,15 @@ __global__ void __launch_bounds__(kGatherThreads, 4)
         }
         __syncwarp();
     }
+}
+
+// CTAs of the token pass that take the heavy tokens: kHeavyCtas when a token has few entries
+// on average (heavy tokens are rare), four per SM when it has more than half the heavy
+// threshold (most tokens heavy, e.g. a coarse stage gathered by many queries).  Every heavy
+// token is summed by one CTA in the same order whatever this count.
+int heavy_ctas(int Q, int K, int N) {
+    const double mean = static_cast<double>(Q) * K / (N > 0 ? N : 1);
+    return mean > 0.5 * kHeavyEntries ? 4 * 148 : kHeavyCtas;
 }
 
 // light chunks of the token pass per image: (Q*K entries + N tokens) / kChunkUnits + 1
@@ -1457,9 +1467,10 @@ cudaError_t launch_knn_bwd_indexed(const KnnArgs& a, cudaStream_t st) {
     const int chunks = knn_chunks(a.Q, a.K, a.N);
     const int qb = static_cast<int>(qblocks);
     const long long warps = static_cast<long long>(a.B) * chunks;
-    const unsigned tblocks = static_cast<unsigned>(kHeavyCtas + (warps + kGatherWarps - 1) / kGatherWarps);
+    const int hctas = heavy_ctas(a.Q, a.K, a.N);
+    const unsigned tblocks = static_cast<unsigned>(hctas + (warps + kGatherWarps - 1) / kGatherWarps);
     const int nlists = a.B * slices;
-    knn_bwd_token_kernel<<<tblocks, kGatherThreads, 0, st>>>(a, l2, qb, nlists, chunks);
+    knn_bwd_token_kernel<<<tblocks, kGatherThreads, 0, st>>>(a, l2, qb, nlists, chunks, hctas);
     note_launch();
     return cudaGetLastError();
 }

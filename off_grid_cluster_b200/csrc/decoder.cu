@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kTThreads)
     const uint32_t slot = bar0 + 8 * kTStages;
     const volatile uint32_t* slot_p = reinterpret_cast<const volatile uint32_t*>(tsm + (slot - raw));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m0 = blockIdx.y * kTM, n0 = blockIdx.x * kTN;
+    const int m0 = blockIdx.x * kTM, n0 = blockIdx.y * kTN;  // M tiles on x: up to 2^31 - 1
     const int kz0 = blockIdx.z * g.kchunk;
     const int kz1 = min(g.K, kz0 + g.kchunk);
     const int nk = kz1 > kz0 ? (kz1 - kz0 + kTK - 1) / kTK : 0;
@@ -271,7 +271,7 @@ template <bool AMN, bool BMN, int EPI>
 cudaError_t launch_tc_gemm(const GemmArgs& g, int splits, cudaStream_t st) {
     cudaError_t e = ensure_smem<tc_gemm_kernel<AMN, BMN, EPI>>(kTSmem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(g.N / kTN, (g.M + kTM - 1) / kTM, splits);
+    const dim3 grid((g.M + kTM - 1) / kTM, g.N / kTN, splits);
     tc_gemm_kernel<AMN, BMN, EPI><<<grid, kTThreads, kTSmem, st>>>(g);
     note_launch();
     return cudaGetLastError();

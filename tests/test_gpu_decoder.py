@@ -103,3 +103,22 @@ def test_decoder_is_bit_reproducible():
         outs.append((q, v, f_out) + tuple(grads))
     for x, y in zip(*outs):
         assert torch.equal(x, y)
+
+
+def test_decoder_no_queries():
+    """Q = 0: the forward has nothing to write; the backward's parameter and stage gradients
+    are zero sums."""
+    db = synth.decoder_batch(B=1)
+    st = db.stages[3]
+    table = dev(oracle.knn_table(st.coords, st.GH, st.GW, st.K))
+    g = dict(feats=bf16(st.feats), coords=dev(st.coords), table=table, p=dev(st.p))
+    ref = torch.empty((1, 0, 2), dtype=torch.float32, device="cuda")
+    f0 = torch.empty((1, 0, db.D), dtype=torch.float32, device="cuda")
+    q, v, f_out = acl.acl_decoder_layer_fwd(ref, f0, dev(db.w_off[0]), dev(db.b_off[0]),
+                                            bf16(db.w_o[0]), **g)
+    assert q.numel() == 0 and v.numel() == 0 and f_out.numel() == 0
+    grads = acl.acl_decoder_layer_bwd(f0, dev(db.w_off[0]), bf16(db.w_o[0]), q=q, v=v,
+                                      df_out=torch.empty_like(f0), **g)
+    acl.acl_device_check()
+    for t in grads[1:]:
+        assert torch.count_nonzero(t).item() == 0

@@ -302,6 +302,222 @@ __global__ void __launch_bounds__(kMergeThreads)
 }
 
 // Exclusive prefix sum of data[0..n) by the whole block; data[n] = the total.
+__device__ void block_scan_excl(int* data, int n, int* scratch);
+
+// 3b. assignment by a binned search, one thread per token (k <= kBinnedMaxK).  The CTA
+//     rebuilds the anchor list as above, then counting-sorts the anchors into square bins of
+//     side s, a power of two, aligned to multiples of s (bin = floor(x / s): exact), about two
+//     anchors per bin over the anchors' bounding box.  A token scans rings of bins around its
+//     own (clamped) bin, an fp32 prefilter before the exact fp64 (distance, anchor rank)
+//     comparison; after each ring it stops once its best distance is below the squared
+//     distance to the edge of the scanned rectangle (an anchor outside lies at least that far
+//     on one axis, and rounding is monotone; a side on the grid's border bounds nothing).
+//     The result equals the brute-force definition.  A CTA whose anchor box is not finite
+//     falls back to the full scan.
+constexpr int kBinThreads = 128;
+constexpr int kBinnedMaxK = 4096;
+constexpr int kBinsMax = 2048;
+
+__global__ void __launch_bounds__(kBinThreads)
+    merge_assign_binned_kernel(const float* __restrict__ xy, int N, int k, const int32_t* __restrict__ flag,
+                               int32_t* __restrict__ anchors, int32_t* __restrict__ assign) {
+    extern __shared__ __align__(16) uint8_t bsm[];
+    float2* axy = reinterpret_cast<float2*>(bsm);   // [k] by rank
+    float2* sxy = axy + k;                           // [k] in bin order
+    int* srank = reinterpret_cast<int*>(sxy + k);    // [k] in bin order
+    int* cnt = srank + k;                            // [kBinsMax + 1]
+    __shared__ int wsum[kBinThreads / 32];
+    __shared__ int myrank[kBinThreads];
+    __shared__ float box[4][kBinThreads / 32];
+    __shared__ int scan_scratch[40];
+    __shared__ int grid_i[5];  // bx0, by0, nbx, nby, full scan
+    __shared__ float grid_f[1];
+    const int b = blockIdx.y, i0 = blockIdx.x * kBinThreads;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float2* xb = reinterpret_cast<const float2*>(xy) + static_cast<size_t>(b) * N;
+    const int32_t* fb = flag + static_cast<size_t>(b) * N;
+    // anchor list (ascending id) by a block scan of the flags
+    const int per = (N + kBinThreads - 1) / kBinThreads;
+    const int j0 = min(N, tid * per), j1 = min(N, j0 + per);
+    int c = 0;
+    for (int j = j0; j < j1; ++j) c += fb[j] != 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int r = incl - c;
+    for (int w = 0; w < warp; ++w) r += wsum[w];
+    for (int jb = j0; jb < j1; jb += 8) {
+        int f8[8];
+        float2 p8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            f8[q] = (jb + q < j1) ? fb[jb + q] : 0;
+            p8[q] = (jb + q < j1) ? xb[jb + q] : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int j = jb + q;
+            if (j >= j1) break;
+            const bool is_anchor = f8[q] != 0 && r < k;
+            if (j >= i0 && j < i0 + kBinThreads) myrank[j - i0] = is_anchor ? r : -1;
+            if (is_anchor) {
+                axy[r] = p8[q];
+                if (blockIdx.x == 0) anchors[static_cast<size_t>(b) * k + r] = j;
+                ++r;
+            }
+        }
+    }
+    __syncthreads();
+    // bounding box of the anchors
+    float mnx = FLT_MAX, mxx = -FLT_MAX, mny = FLT_MAX, mxy = -FLT_MAX;
+    bool fin = true;
+    for (int a = tid; a < k; a += kBinThreads) {
+        const float2 p = axy[a];
+        fin = fin && isfinite(p.x) && isfinite(p.y);
+        mnx = fminf(mnx, p.x); mxx = fmaxf(mxx, p.x);
+        mny = fminf(mny, p.y); mxy = fmaxf(mxy, p.y);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mnx = fminf(mnx, __shfl_xor_sync(0xffffffffu, mnx, o));
+        mxx = fmaxf(mxx, __shfl_xor_sync(0xffffffffu, mxx, o));
+        mny = fminf(mny, __shfl_xor_sync(0xffffffffu, mny, o));
+        mxy = fmaxf(mxy, __shfl_xor_sync(0xffffffffu, mxy, o));
+    }
+    const bool all_fin = __syncthreads_and(fin) != 0;
+    if (lane == 0) {
+        box[0][warp] = mnx; box[1][warp] = mxx; box[2][warp] = mny; box[3][warp] = mxy;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        for (int w = 1; w < kBinThreads / 32; ++w) {
+            mnx = fminf(mnx, box[0][w]); mxx = fmaxf(mxx, box[1][w]);
+            mny = fminf(mny, box[2][w]); mxy = fmaxf(mxy, box[3][w]);
+        }
+        int full = !all_fin;
+        float sv = 1.f;
+        int bx0 = 0, by0 = 0, nbx = 1, nby = 1;
+        if (!full) {
+            // about two anchors per bin, at most kBinsMax bins, |bin index| < 2^30
+            const int target = max(1, min(kBinsMax, k / 2));
+            const float ext = fmaxf(fmaxf(mxx - mnx, mxy - mny), 1e-30f);
+            sv = exp2f(ceilf(log2f(ext / sqrtf(static_cast<float>(target)))));
+            for (int it = 0; it < 300; ++it) {
+                const float fx0 = floorf(mnx / sv), fx1 = floorf(mxx / sv);
+                const float fy0 = floorf(mny / sv), fy1 = floorf(mxy / sv);
+                const bool ok = fabsf(fx0) < 1073741824.f && fabsf(fx1) < 1073741824.f &&
+                                fabsf(fy0) < 1073741824.f && fabsf(fy1) < 1073741824.f &&
+                                (fx1 - fx0 + 1.f) * (fy1 - fy0 + 1.f) <= static_cast<float>(target);
+                if (ok) {
+                    bx0 = static_cast<int>(fx0); by0 = static_cast<int>(fy0);
+                    nbx = static_cast<int>(fx1 - fx0) + 1; nby = static_cast<int>(fy1 - fy0) + 1;
+                    break;
+                }
+                sv *= 2.f;
+                if (it == 299) full = 1;
+            }
+        }
+        grid_i[0] = bx0; grid_i[1] = by0; grid_i[2] = nbx; grid_i[3] = nby; grid_i[4] = full;
+        grid_f[0] = sv;
+    }
+    __syncthreads();
+    const int bx0 = grid_i[0], by0 = grid_i[1], nbx = grid_i[2], nby = grid_i[3];
+    const bool full = grid_i[4] != 0;
+    const float sv = grid_f[0];
+    const float inv_s = 1.f / sv;  // exact: a power of two
+    auto bin_x = [&](float v) { return min(max(static_cast<int>(floorf(v * inv_s)) - bx0, 0), nbx - 1); };
+    auto bin_y = [&](float v) { return min(max(static_cast<int>(floorf(v * inv_s)) - by0, 0), nby - 1); };
+    const int nbins = nbx * nby;
+    if (!full) {
+        for (int i = tid; i <= nbins; i += kBinThreads) cnt[i] = 0;
+        __syncthreads();
+        for (int a = tid; a < k; a += kBinThreads) {
+            const float2 p = axy[a];
+            atomicAdd(&cnt[bin_y(p.y) * nbx + bin_x(p.x)], 1);
+        }
+        __syncthreads();
+        block_scan_excl(cnt, nbins, scan_scratch);  // cnt[bin] = start
+        for (int a = tid; a < k; a += kBinThreads) {
+            const float2 p = axy[a];
+            const int pos = atomicAdd(&cnt[bin_y(p.y) * nbx + bin_x(p.x)], 1);
+            sxy[pos] = p;
+            srank[pos] = a;
+        }
+        __syncthreads();  // cnt[bin] = end of bin; start = cnt[bin - 1]
+    }
+    const int i = i0 + tid;
+    if (i >= N) return;
+    const int ri = myrank[tid];
+    if (ri >= 0) {
+        assign[static_cast<size_t>(b) * N + i] = ri;
+        return;
+    }
+    const float2 p = xb[i];
+    const double px = p.x, py = p.y;
+    double best = DBL_MAX;
+    float bestf = FLT_MAX;
+    int bj = 0x7fffffff;
+    auto visit = [&](float2 a, int rank) {
+        const float dxf = p.x - a.x, dyf = p.y - a.y;
+        const float d2f = fmaf(dxf, dxf, dyf * dyf);
+        if (d2f <= bestf) {   // a candidate beyond the fp32 bound cannot be nearer in fp64
+            const double dx = __dsub_rn(px, static_cast<double>(a.x));
+            const double dy = __dsub_rn(py, static_cast<double>(a.y));
+            const double d2 = __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy));
+            if (d2 < best || (d2 == best && rank < bj)) {
+                best = d2;
+                bj = rank;
+                bestf = static_cast<float>(best) * (1.0f + 1.0f / 1048576.0f);
+            }
+        }
+    };
+    // a token whose scaled coordinates are not finite or not below 2^30 in magnitude takes the
+    // full scan (its bin index would not be exact)
+    const float fpx = floorf(p.x * inv_s), fpy = floorf(p.y * inv_s);
+    if (full || !(fabsf(fpx) < 1073741824.f && fabsf(fpy) < 1073741824.f)) {
+        for (int a = 0; a < k; ++a) visit(axy[a], a);
+    } else {
+        const int pbx = bin_x(p.x), pby = bin_y(p.y);
+        const double s = static_cast<double>(sv);
+        auto scan_bin = [&](int bx, int by) {
+            const int bin = by * nbx + bx;
+            const int a0 = bin > 0 ? cnt[bin - 1] : 0, a1 = cnt[bin];
+            for (int a = a0; a < a1; ++a) visit(sxy[a], srank[a]);
+        };
+        const int maxring = max(nbx, nby);
+        for (int rho = 0; rho <= maxring; ++rho) {
+            const int xl = pbx - rho, xh = pbx + rho, yl = pby - rho, yh = pby + rho;
+            const int cxl = max(xl, 0), cxh = min(xh, nbx - 1);
+            if (rho == 0) {
+                scan_bin(pbx, pby);
+            } else {
+                if (yl >= 0)
+                    for (int bx = cxl; bx <= cxh; ++bx) scan_bin(bx, yl);
+                if (yh < nby)
+                    for (int bx = cxl; bx <= cxh; ++bx) scan_bin(bx, yh);
+                for (int by = max(yl + 1, 0); by <= min(yh - 1, nby - 1); ++by) {
+                    if (xl >= 0) scan_bin(xl, by);
+                    if (xh < nbx) scan_bin(xh, by);
+                }
+            }
+            double m = DBL_MAX;
+            if (xl > 0) m = fmin(m, __dsub_rn(px, static_cast<double>(bx0 + xl) * s));
+            if (xh < nbx - 1) m = fmin(m, __dsub_rn(static_cast<double>(bx0 + xh + 1) * s, px));
+            if (yl > 0) m = fmin(m, __dsub_rn(py, static_cast<double>(by0 + yl) * s));
+            if (yh < nby - 1) m = fmin(m, __dsub_rn(static_cast<double>(by0 + yh + 1) * s, py));
+            if (m == DBL_MAX) break;                   // the whole grid is scanned
+            if (best < __dmul_rn(m, m)) break;         // nothing outside can be nearer or tie
+        }
+    }
+    assign[static_cast<size_t>(b) * N + i] = bj;
+}
+
+// Exclusive prefix sum of data[0..n) by the whole block; data[n] = the total.
 __device__ void block_scan_excl(int* data, int n, int* scratch) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int per = (n + blockDim.x - 1) / blockDim.x;
@@ -743,6 +959,7 @@ size_t token_smem(int d, int h) {
     return sizeof(float) * static_cast<size_t>(kTokPerCta) * (32 * hp_of(h) + 4) + (w1_in_smem(d, h) ? w1_smem(d, h) : 0);
 }
 size_t rank_smem(int N) { return 4 * static_cast<size_t>((N + 3) & ~3); }
+size_t binned_smem(int k) { return 20 * static_cast<size_t>(k) + 4 * (kBinsMax + 1); }
 size_t groups_smem(int N, int k) { return 4 * (static_cast<size_t>(k) + 1 + 2 * static_cast<size_t>(N)); }
 size_t param_smem(int d, int h) {
     return sizeof(float) * static_cast<size_t>(kParamTile) * (d + 2 * ((h + 3) & ~3) + 1);
@@ -781,7 +998,8 @@ MergeWorkspace merge_workspace_layout(int B, int N, int d, int h, int k) {
 }
 
 size_t merge_smem_bytes(int N, int k, int d, int h) {
-    const size_t c[] = {w1_in_smem(d, h) ? w1_smem(d, h) : 0, rank_smem(N), 8 * static_cast<size_t>(k),
+    const size_t c[] = {w1_in_smem(d, h) ? w1_smem(d, h) : 0, rank_smem(N),
+                        k <= kBinnedMaxK ? binned_smem(k) : 8 * static_cast<size_t>(k),
                         groups_smem(N, k), token_smem(d, h), param_smem(d, h)};
     size_t m = 0;
     for (size_t x : c) m = x > m ? x : m;
@@ -839,6 +1057,19 @@ cudaError_t launch_merge_fwd(const MergeArgs& m, cudaStream_t st) {
     merge_rank_kernel<<<dim3((m.N + kTokPerCta - 1) / kTokPerCta, m.B), kMergeThreads, rsm, st>>>(
         m.scores, m.N, m.k, m.flag);
     note_launch();
+    if (m.k <= kBinnedMaxK) {
+        const size_t bsm = binned_smem(m.k);
+        if ((e = ensure_smem<merge_assign_binned_kernel>(bsm)) != cudaSuccess) return e;
+        merge_assign_binned_kernel<<<dim3((m.N + kBinThreads - 1) / kBinThreads, m.B), kBinThreads, bsm, st>>>(
+            m.xy, m.N, m.k, m.flag, m.anchors, m.assign);
+        note_launch();
+        if ((e = launch_groups(m, st)) != cudaSuccess) return e;
+        const long long na2 = static_cast<long long>(m.B) * m.k;
+        merge_fwd_kernel<<<static_cast<unsigned>((na2 + kMergeWarps - 1) / kMergeWarps), kMergeThreads, 0, st>>>(
+            m.feats, m.xy, m.B, m.N, m.d, m.k, m.scores, m.members, m.goff, m.merged, m.mxy);
+        note_launch();
+        return cudaGetLastError();
+    }
     const size_t asm_ = 8 * static_cast<size_t>(m.k);
     if ((e = ensure_smem<merge_assign_kernel>(asm_)) != cudaSuccess) return e;
     constexpr int kAssignTok = kMergeThreads / kAssignSub;

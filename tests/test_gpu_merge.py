@@ -90,3 +90,22 @@ def test_merge_score_ties_and_many_tokens():
     mb = synth.merge_batch(xy, d=32, hidden=8)
     mb.feats[:, 100:400] = mb.feats[:, 99:100]
     merge_both(mb)
+
+
+def test_merge_binned_search_extremes():
+    """The binned nearest-anchor search: 200 coincident tokens, far outliers (a bin grid
+    stretched over 10^6 cells), and integer-lattice coordinates (many exact distance ties)."""
+    rng = np.random.default_rng(21)
+    xy = rng.uniform(0, 8, size=(2, 400, 2)).astype(np.float32)
+    xy[0, :200] = 3.25
+    xy[0, 390] = (1.0e6, -2.5e5)
+    xy[0, 391] = (-7.0e5, 3.0e5)
+    xy[1] = np.round(xy[1] * 2.0) / 2.0
+    merge_both(synth.merge_batch(xy, d=32, hidden=8))
+
+
+def test_merge_many_anchors_full_scan():
+    """k above the binned search's limit (4500 anchors) takes the full-scan kernel."""
+    rng = np.random.default_rng(22)
+    xy = rng.uniform(0, 100, size=(1, 10000, 2)).astype(np.float32)
+    merge_both(synth.merge_batch(xy, d=32, hidden=8, ds=0.45))

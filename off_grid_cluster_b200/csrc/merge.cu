@@ -164,6 +164,267 @@ __global__ void __launch_bounds__(kMergeThreads)
     }
 }
 
+// ---------------------------------------------------------- tensor-core MLP
+//
+// For d a multiple of 64 up to 256 and h a multiple of 16 up to 64, the hidden layer runs on
+// the tensor cores:
+// one warp per 16 tokens, z (16 x h) = F (16 x d, bf16: exact) . W1 by m16n8k16 bf16 MMAs with
+// fp32 accumulation, W1 split into bf16 hi + lo (hi = bf16(w), lo = bf16(w - hi): about 16
+// significant bits, two MMAs per tile).  The features are staged per warp by cp.async in
+// shared-memory rows of d + 8 elements and W1 as [h][d + 8] (unit rows), both read by
+// ldmatrix without bank conflicts.
+constexpr int kMmaMaxD = 256, kMmaMaxH = 64;
+
+// the backward's dfeats pass takes 64 channels at a time, so d % 64 == 0
+bool mlp_mma_ok(int d, int h) { return d % 64 == 0 && d <= kMmaMaxD && h % 16 == 0 && h <= kMmaMaxH; }
+
+struct MlpSmem {
+    size_t w1t_hi, w1t_lo, w1_hi, w1_lo, b1, w2, f, total;
+};
+// bwd: also W1 as [d][h + 8] (channel rows) hi + lo, the B operand of dh . W1^T
+__host__ __device__ inline MlpSmem mlp_smem(int d, int h, bool bwd) {
+    MlpSmem L;
+    size_t o = 0;
+    const size_t wt = static_cast<size_t>(h) * (d + 8) * 2, w = static_cast<size_t>(d) * (h + 8) * 2;
+    L.w1t_hi = o; o += wt;
+    L.w1t_lo = o; o += wt;
+    L.w1_hi = o; o += bwd ? w : 0;
+    L.w1_lo = o; o += bwd ? w : 0;
+    o = (o + 15) & ~size_t(15);
+    L.b1 = o; o += 4 * static_cast<size_t>(h);
+    L.w2 = o; o += 4 * static_cast<size_t>(h);
+    o = (o + 15) & ~size_t(15);
+    L.f = o; o += static_cast<size_t>(kMergeWarps) * 16 * (d + 8) * 2;
+    L.total = o;
+    return L;
+}
+
+__device__ void stage_mlp(const MlpSmem& L, uint8_t* sm, const float* __restrict__ w1, const float* __restrict__ b1,
+                          const float* __restrict__ w2, int d, int h, bool bwd) {
+    bf16* th = reinterpret_cast<bf16*>(sm + L.w1t_hi);
+    bf16* tl = reinterpret_cast<bf16*>(sm + L.w1t_lo);
+    bf16* wh = reinterpret_cast<bf16*>(sm + L.w1_hi);
+    bf16* wl = reinterpret_cast<bf16*>(sm + L.w1_lo);
+    for (int i = threadIdx.x; i < d * h; i += blockDim.x) {
+        const int c = i / h, u = i - c * h;
+        const float w = w1[i];
+        const bf16 hi = __float2bfloat16_rn(w);
+        const bf16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+        th[u * (d + 8) + c] = hi;
+        tl[u * (d + 8) + c] = lo;
+        if (bwd) {
+            wh[c * (h + 8) + u] = hi;
+            wl[c * (h + 8) + u] = lo;
+        }
+    }
+    float* b1s = reinterpret_cast<float*>(sm + L.b1);
+    float* w2s = reinterpret_cast<float*>(sm + L.w2);
+    for (int u = threadIdx.x; u < h; u += blockDim.x) {
+        b1s[u] = b1[u];
+        w2s[u] = w2[u];
+    }
+}
+
+// 16 feature rows (tokens t0 .. t0 + 15 of T) into the warp's tile; rows past T are zero.
+__device__ __forceinline__ void load_f_tile(uint32_t tile, const bf16* __restrict__ feats, int t0, int T, int d,
+                                            int lane) {
+    const int cpr = d / 8;  // 16-byte chunks per row
+    for (int q = lane; q < 16 * cpr; q += 32) {
+        const int r = q / cpr, ch = q - r * cpr;
+        const bool ok = t0 + r < T;
+        cp_async16(tile + (r * (d + 8) + ch * 8) * 2, ok ? feats + static_cast<size_t>(t0 + r) * d + ch * 8 : feats, ok);
+    }
+    cp_async_commit();
+}
+
+// z = F . W1 for the warp's 16-token tile: lane (g, t) holds rows g and g + 8, units 8 nt + 2t, +1.
+template <int NT>
+__device__ __forceinline__ void z_mma(uint32_t ftile, uint32_t whi, uint32_t wlo, int d, int lane,
+                                      float (&acc)[NT][4]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    const int rb = (d + 8) * 2;  // row bytes of the feature and W1 tiles
+    const int mi = lane >> 3, r8 = lane & 7;
+    for (int ks = 0; ks < d / 16; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(ftile + (lane & 15) * rb + (2 * ks + (lane >> 4)) * 16, a0, a1, a2, a3);
+#pragma unroll
+        for (int pr = 0; pr < NT / 2; ++pr) {
+            const uint32_t off = (16 * pr + 8 * (mi >> 1) + r8) * rb + (2 * ks + (mi & 1)) * 16;
+            uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+            ldsm_x4(whi + off, h0, h1, h2, h3);
+            ldsm_x4(wlo + off, l0, l1, l2, l3);
+            mma_bf16(acc[2 * pr], a0, a1, a2, a3, h0, h1);
+            mma_bf16(acc[2 * pr], a0, a1, a2, a3, l0, l1);
+            mma_bf16(acc[2 * pr + 1], a0, a1, a2, a3, h2, h3);
+            mma_bf16(acc[2 * pr + 1], a0, a1, a2, a3, l2, l3);
+        }
+    }
+}
+
+// 1'. scores on the tensor cores: warps stride over 16-token tiles.
+template <int NT>
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_scores_mma_kernel(const bf16* __restrict__ feats, int T, int d, const float* __restrict__ w1,
+                            const float* __restrict__ b1, const float* __restrict__ w2, float b2,
+                            float* __restrict__ scores) {
+    extern __shared__ __align__(16) uint8_t msm[];
+    constexpr int h = 8 * NT;
+    const MlpSmem L = mlp_smem(d, h, false);
+    stage_mlp(L, msm, w1, b1, w2, d, h, false);
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t base = smem_addr(msm);
+    const uint32_t ftile = base + static_cast<uint32_t>(L.f) + warp * 16 * (d + 8) * 2;
+    const float* b1s = reinterpret_cast<const float*>(msm + L.b1);
+    const float* w2s = reinterpret_cast<const float*>(msm + L.w2);
+    for (int t0 = (blockIdx.x * kMergeWarps + warp) * 16; t0 < T; t0 += gridDim.x * kMergeWarps * 16) {
+        load_f_tile(ftile, feats, t0, T, d, lane);
+        cp_async_wait<0>();
+        __syncwarp();
+        float acc[NT][4];
+        z_mma<NT>(ftile, base + static_cast<uint32_t>(L.w1t_hi), base + static_cast<uint32_t>(L.w1t_lo), d, lane, acc);
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int u = 8 * nt + 2 * t + e;
+                s0 = fmaf(w2s[u], gelu_f(acc[nt][e] + b1s[u]), s0);
+                s1 = fmaf(w2s[u], gelu_f(acc[nt][2 + e] + b1s[u]), s1);
+            }
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+        if (t == 0) {
+            if (t0 + g < T) scores[t0 + g] = s0 + b2;
+            if (t0 + g + 8 < T) scores[t0 + g + 8] = s1 + b2;
+        }
+        __syncwarp();  // the tile is read before the next one is loaded
+    }
+}
+
+// 7'. backward token pass on the tensor cores: one warp per 16 tokens.  Lane (g, t) owns rows g
+//     and g + 8: their weight, ds, dx; z again by z_mma; dh = ds w2 gelu'(z) and e = ds gelu(z)
+//     for its units (written for the parameter sums); then dfeats = w dF + dh . W1^T with dh
+//     (bf16 hi + lo, straight from the accumulator layout) as the A operand and W1 ([d][h + 8],
+//     hi + lo) as B, 64 channels at a time, three MMAs per tile (hi.hi, hi.lo, lo.hi).
+template <int NT>
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_bwd_token_mma_kernel(const bf16* __restrict__ feats, const float* __restrict__ xy, int T, int N,
+                               int d, int k, const float* __restrict__ w1, const float* __restrict__ b1,
+                               const float* __restrict__ w2, const float* __restrict__ scores,
+                               const int32_t* __restrict__ assign, const float4* __restrict__ gstat,
+                               const float* __restrict__ gtok, const bf16* __restrict__ dmerged,
+                               const float* __restrict__ dmxy, bf16* __restrict__ dfeats, float* __restrict__ dxy,
+                               float* __restrict__ ds_out, float* __restrict__ dh_out, float* __restrict__ e_out) {
+    extern __shared__ __align__(16) uint8_t msm[];
+    constexpr int h = 8 * NT;
+    const MlpSmem L = mlp_smem(d, h, true);
+    stage_mlp(L, msm, w1, b1, w2, d, h, true);
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3, mi = lane >> 3, r8 = lane & 7;
+    const uint32_t base = smem_addr(msm);
+    const uint32_t ftile = base + static_cast<uint32_t>(L.f) + warp * 16 * (d + 8) * 2;
+    const uint32_t wh = base + static_cast<uint32_t>(L.w1_hi), wl = base + static_cast<uint32_t>(L.w1_lo);
+    const float* b1s = reinterpret_cast<const float*>(msm + L.b1);
+    const float* w2s = reinterpret_cast<const float*>(msm + L.w2);
+    constexpr int rbw = (h + 8) * 2;  // row bytes of W1 [d][h + 8]
+    for (int t0 = (blockIdx.x * kMergeWarps + warp) * 16; t0 < T; t0 += gridDim.x * kMergeWarps * 16) {
+        load_f_tile(ftile, feats, t0, T, d, lane);
+        // rows g and g + 8: weight, ds, anchor row
+        float wt[2], ds[2];
+        size_t arow[2];
+        bool live[2];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const int tk = t0 + g + 8 * rr;
+            live[rr] = tk < T;
+            const int tc = live[rr] ? tk : t0;
+            const int bimg = tc / N;
+            const int a = assign[tc];
+            const bool ok = live[rr] && a >= 0 && a < k;
+            arow[rr] = static_cast<size_t>(bimg) * k + (ok ? a : 0);
+            const float4 gs = gstat[arow[rr]];
+            wt[rr] = ok ? expf(scores[tc] - gs.x) * gs.y : 0.f;
+            ds[rr] = ok ? wt[rr] * (gtok[tc] - gs.z) : 0.f;
+            if (live[rr] && t == 0) {
+                ds_out[tk] = ds[rr];
+                const float2 dX = reinterpret_cast<const float2*>(dmxy)[arow[rr]];
+                reinterpret_cast<float2*>(dxy)[tk] = make_float2(wt[rr] * dX.x, wt[rr] * dX.y);
+            }
+        }
+        cp_async_wait<0>();
+        __syncwarp();
+        float acc[NT][4];
+        z_mma<NT>(ftile, base + static_cast<uint32_t>(L.w1t_hi), base + static_cast<uint32_t>(L.w1t_lo), d, lane, acc);
+        // dh and e for the lane's units; dh packed as the A operand (hi, lo) of dh . W1^T
+        uint32_t ahi[NT / 2][4], alo[NT / 2][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float dh[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int u = 8 * nt + 2 * t + (e & 1), rr = e >> 1;
+                const float z = acc[nt][e] + b1s[u];
+                dh[e] = ds[rr] * w2s[u] * gelu_grad_f(z);
+                if (live[rr]) {
+                    const size_t o = static_cast<size_t>(t0 + g + 8 * rr) * h + u;
+                    dh_out[o] = dh[e];
+                    e_out[o] = ds[rr] * gelu_f(z);
+                }
+            }
+            const uint32_t h01 = pack_bf16(dh[0], dh[1]), h23 = pack_bf16(dh[2], dh[3]);
+            const uint32_t l01 = pack_bf16(dh[0] - bf16_lo(h01), dh[1] - bf16_hi(h01));
+            const uint32_t l23 = pack_bf16(dh[2] - bf16_lo(h23), dh[3] - bf16_hi(h23));
+            const int ks = nt >> 1, hf = nt & 1;  // n-tile 2 ks: A regs 0, 1; n-tile 2 ks + 1: regs 2, 3
+            ahi[ks][2 * hf] = h01;
+            ahi[ks][2 * hf + 1] = h23;
+            alo[ks][2 * hf] = l01;
+            alo[ks][2 * hf + 1] = l23;
+        }
+        // dfeats, 64 channels at a time
+        for (int c0 = 0; c0 < d; c0 += 64) {
+            float dfa[8][4];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) dfa[nt][0] = dfa[nt][1] = dfa[nt][2] = dfa[nt][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < NT / 2; ++ks) {
+#pragma unroll
+                for (int pr = 0; pr < 4; ++pr) {
+                    const uint32_t off = (c0 + 16 * pr + 8 * (mi >> 1) + r8) * rbw + (2 * ks + (mi & 1)) * 16;
+                    uint32_t x0, x1, x2, x3, y0, y1, y2, y3;
+                    ldsm_x4(wh + off, x0, x1, x2, x3);
+                    ldsm_x4(wl + off, y0, y1, y2, y3);
+                    mma_bf16(dfa[2 * pr], ahi[ks][0], ahi[ks][1], ahi[ks][2], ahi[ks][3], x0, x1);
+                    mma_bf16(dfa[2 * pr], ahi[ks][0], ahi[ks][1], ahi[ks][2], ahi[ks][3], y0, y1);
+                    mma_bf16(dfa[2 * pr], alo[ks][0], alo[ks][1], alo[ks][2], alo[ks][3], x0, x1);
+                    mma_bf16(dfa[2 * pr + 1], ahi[ks][0], ahi[ks][1], ahi[ks][2], ahi[ks][3], x2, x3);
+                    mma_bf16(dfa[2 * pr + 1], ahi[ks][0], ahi[ks][1], ahi[ks][2], ahi[ks][3], y2, y3);
+                    mma_bf16(dfa[2 * pr + 1], alo[ks][0], alo[ks][1], alo[ks][2], alo[ks][3], x2, x3);
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const int c = c0 + 8 * nt + 2 * t;
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    if (!live[rr]) continue;
+                    const uint32_t pg = *reinterpret_cast<const uint32_t*>(dmerged + arow[rr] * d + c);
+                    const float v0 = fmaf(wt[rr], bf16_lo(pg), dfa[nt][2 * rr]);
+                    const float v1 = fmaf(wt[rr], bf16_hi(pg), dfa[nt][2 * rr + 1]);
+                    *reinterpret_cast<uint32_t*>(dfeats + static_cast<size_t>(t0 + g + 8 * rr) * d + c) =
+                        pack_bf16(v0, v1);
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
 // Order-preserving map of an fp32 score to uint32 (-0 and +0 equal).
 __device__ __forceinline__ uint32_t order_bits_f(float f) {
     uint32_t u = __float_as_uint(f);
@@ -998,7 +1259,8 @@ MergeWorkspace merge_workspace_layout(int B, int N, int d, int h, int k) {
 }
 
 size_t merge_smem_bytes(int N, int k, int d, int h) {
-    const size_t c[] = {w1_in_smem(d, h) ? w1_smem(d, h) : 0, rank_smem(N),
+    const size_t c[] = {w1_in_smem(d, h) ? w1_smem(d, h) : 0, mlp_mma_ok(d, h) ? mlp_smem(d, h, true).total : 0,
+                        rank_smem(N),
                         k <= kBinnedMaxK ? binned_smem(k) : 8 * static_cast<size_t>(k),
                         groups_smem(N, k), token_smem(d, h), param_smem(d, h)};
     size_t m = 0;
@@ -1023,6 +1285,52 @@ cudaError_t launch_scores(const MergeArgs& m, int T, cudaStream_t st) {
                                                                         m.b2, m.h, m.scores);
     note_launch();
     return cudaSuccess;
+}
+
+template <int NT>
+cudaError_t launch_scores_mma_nt(const MergeArgs& m, int T, cudaStream_t st) {
+    const size_t sm = mlp_smem(m.d, m.h, false).total;
+    cudaError_t e = ensure_smem<merge_scores_mma_kernel<NT>>(sm);
+    if (e != cudaSuccess) return e;
+    const long long tiles = (static_cast<long long>(T) + 15) / 16;
+    const long long need = (tiles + kMergeWarps - 1) / kMergeWarps;
+    const unsigned ctas = static_cast<unsigned>(need < 2 * 148 ? need : 2 * 148);
+    merge_scores_mma_kernel<NT><<<ctas, kMergeThreads, sm, st>>>(m.feats, T, m.d, m.w1, m.b1, m.w2, m.b2, m.scores);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scores_mma(const MergeArgs& m, int T, cudaStream_t st) {
+    switch (m.h / 8) {
+        case 2: return launch_scores_mma_nt<2>(m, T, st);
+        case 4: return launch_scores_mma_nt<4>(m, T, st);
+        case 6: return launch_scores_mma_nt<6>(m, T, st);
+        default: return launch_scores_mma_nt<8>(m, T, st);
+    }
+}
+
+template <int NT>
+cudaError_t launch_bwd_token_mma_nt(const MergeArgs& m, int T, cudaStream_t st) {
+    const size_t sm = mlp_smem(m.d, m.h, true).total;
+    cudaError_t e = ensure_smem<merge_bwd_token_mma_kernel<NT>>(sm);
+    if (e != cudaSuccess) return e;
+    const long long tiles = (static_cast<long long>(T) + 15) / 16;
+    const long long need = (tiles + kMergeWarps - 1) / kMergeWarps;
+    const unsigned ctas = static_cast<unsigned>(need < 2 * 148 ? need : 2 * 148);
+    merge_bwd_token_mma_kernel<NT><<<ctas, kMergeThreads, sm, st>>>(
+        m.feats, m.xy, T, m.N, m.d, m.k, m.w1, m.b1, m.w2, m.scores, m.assign,
+        reinterpret_cast<const float4*>(m.gstat), m.g, m.dmerged, m.dmxy, m.dfeats, m.dxy, m.ds, m.dh, m.e);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_token_mma(const MergeArgs& m, int T, cudaStream_t st) {
+    switch (m.h / 8) {
+        case 2: return launch_bwd_token_mma_nt<2>(m, T, st);
+        case 4: return launch_bwd_token_mma_nt<4>(m, T, st);
+        case 6: return launch_bwd_token_mma_nt<6>(m, T, st);
+        default: return launch_bwd_token_mma_nt<8>(m, T, st);
+    }
 }
 
 template <int HP, bool SM>
@@ -1050,7 +1358,11 @@ cudaError_t launch_merge_fwd(const MergeArgs& m, cudaStream_t st) {
     const int T = m.B * m.N;
     cudaError_t e = cudaSuccess;
     const bool sm = w1_in_smem(m.d, m.h);
-    ACL_HP_SWITCH(m.h, (e = sm ? launch_scores<HP, true>(m, T, st) : launch_scores<HP, false>(m, T, st)));
+    if (mlp_mma_ok(m.d, m.h)) {
+        e = launch_scores_mma(m, T, st);
+    } else {
+        ACL_HP_SWITCH(m.h, (e = sm ? launch_scores<HP, true>(m, T, st) : launch_scores<HP, false>(m, T, st)));
+    }
     if (e != cudaSuccess) return e;
     const size_t rsm = rank_smem(m.N);
     if ((e = ensure_smem<merge_rank_kernel>(rsm)) != cudaSuccess) return e;
@@ -1094,7 +1406,11 @@ cudaError_t launch_merge_bwd(const MergeArgs& m, cudaStream_t st) {
         reinterpret_cast<float4*>(m.gstat), m.g);
     note_launch();
     const bool sm = w1_in_smem(m.d, m.h);
-    ACL_HP_SWITCH(m.h, (e = sm ? launch_bwd_token<HP, true>(m, T, st) : launch_bwd_token<HP, false>(m, T, st)));
+    if (mlp_mma_ok(m.d, m.h)) {
+        e = launch_bwd_token_mma(m, T, st);
+    } else {
+        ACL_HP_SWITCH(m.h, (e = sm ? launch_bwd_token<HP, true>(m, T, st) : launch_bwd_token<HP, false>(m, T, st)));
+    }
     if (e != cudaSuccess) return e;
     const size_t psm = param_smem(m.d, m.h);
     if ((e = ensure_smem<merge_param_part_kernel>(psm)) != cudaSuccess) return e;

@@ -73,10 +73,11 @@ def test_merge_is_bit_reproducible():
         assert torch.equal(x, y)
 
 
-@pytest.mark.parametrize("d,hidden", [(64, 100), (64, 256), (1024, 8)])
+@pytest.mark.parametrize("d,hidden", [(64, 100), (64, 256), (1024, 8), (64, 16), (192, 48)])
 def test_merge_hidden_widths(d, hidden):
-    """Hidden widths that are not a multiple of 32 (padded units), the widest (256), and a W1
-    too large for shared memory (read from global memory)."""
+    """Hidden widths that are not a multiple of 32 (padded units), the widest (256), a W1 too
+    large for shared memory (read from global memory), and the smallest and an odd-tile shape
+    of the tensor-core MLP (d = 64, h = 16; d = 192, h = 48)."""
     rng = np.random.default_rng(11)
     xy = rng.uniform(0, 20, size=(2, 300, 2)).astype(np.float32)
     merge_both(synth.merge_batch(xy, d=d, hidden=hidden))

@@ -1061,18 +1061,18 @@ __device__ __forceinline__ void token_streams(const KnnArgs& a, int b, int lo, i
         const int mine = (kk < n) ? __ldg(csr + lo + sid + nstreams * kk) : 0;
         const int cnt = min(LPQ, n - k0);
         int u = 0;
-        for (; u + 8 <= cnt; u += 8) {
-            float wv[8];
-            uint4 gv[8];
+        for (; u + 4 <= cnt; u += 4) {
+            float wv[4];
+            uint4 gv[4];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
+            for (int x = 0; x < 4; ++x) {
                 const int e = __shfl_sync(gmask, mine, u + x, LPQ);
                 const int q = e >> 4, j = e & 15;
                 wv[x] = __ldg(wb + q * KN + j * NH);
                 gv[x] = on ? ldg16(gb + q * a.d) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
-            for (int x = 0; x < 8; ++x) fma8(acc, wv[x], gv[x]);
+            for (int x = 0; x < 4; ++x) fma8(acc, wv[x], gv[x]);
         }
         for (; u < cnt; ++u) {
             const int e = __shfl_sync(gmask, mine, u, LPQ);

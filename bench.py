@@ -97,7 +97,7 @@ def parse_args(argv=None):
                          "chains run as two concurrent branches of the step graph)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bounded CPU work of the oracle baseline (seconds)")
-    ap.add_argument("--only", choices=("token_merge", "decoder"), default=None,
+    ap.add_argument("--only", choices=("token_merge", "decoder", "configs"), default=None,
                     help="time one extra part alone on one GPU and print its JSON (a short "
                          "command to profile under ncu); no bench line")
     return ap.parse_args(argv)
@@ -462,6 +462,7 @@ def run_gpu(args, rank: int, world: int):
     merge_us = (token_merge_times(torch, acl, synth, sb, device, stream, measured_peaks())
                 if world == 1 else None)
     dec_us = decoder_times(torch, acl, synth, device, stream, measured_peaks()) if world == 1 else None
+    cfg_us = config_times(torch, acl, synth, device, stream, measured_peaks()) if world == 1 else None
     # keep the same load on the GPU until the clock sampler has several samples
     t_wall = time.time()
     it = 0
@@ -535,6 +536,7 @@ def run_gpu(args, rank: int, world: int):
             "hires_gather_us": hires,
             "token_merge_us": merge_us,
             "decoder_us": dec_us,
+            "configs": cfg_us,
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -879,6 +881,94 @@ def decoder_times(torch, acl, synth, device, stream, peaks: dict, B: int = 8, re
     return res
 
 
+def config_times(torch, acl, synth, device, stream, peaks: dict, reps: int = 10) -> dict:
+    """The five seeded configurations' hot-path calls, one call at a time, each captured as a
+    CUDA graph and timed with CUDA events: cluster attention fwd + bwd tokens/s per layer
+    (configs 1-4; the sweep as sum over stages of its layers x one layer's time, all layers of
+    a stage having the same shapes) and the KNN gather fwd + bwd queries/s over the four stages
+    (config 5), each with its fraction of the measured HBM copy bandwidth on the algorithmic
+    bytes (`algorithmic_bytes`).  Clustering, neighbour and KNN tables are timed beside."""
+    T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
+    timed = lambda fn: graph_time(torch, stream, fn, reps)
+    hbm = peaks["hbm_gbs"]
+
+    def attn_layer(ab):
+        xy = T(ab.coords)
+        q, k, v, do = (T(x, torch.bfloat16) for x in (ab.q, ab.k, ab.v, ab.do))
+        bias = T(ab.bias)
+        cl = acl.acl_cluster(xy, stream=stream)
+        nb = acl.acl_neighbors(xy, cl, stream=stream)
+        o, lse = acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, stream=stream)
+        ws = torch.empty((acl.acl_cluster_attn_workspace(ab.B, ab.N, ab.H, 8, 48),), dtype=torch.uint8,
+                         device=device)
+        t_cl = timed(lambda: acl.acl_cluster(xy, clusters=cl, stream=stream))
+        t_nb = timed(lambda: acl.acl_neighbors(xy, cl, nbr=nb, stream=stream))
+        t_f = timed(lambda: acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, O=o, lse=lse,
+                                                     stream=stream))
+        t_b = timed(lambda: acl.acl_cluster_attn_bwd(q, k, v, xy, cl, nb, bias, ab.scale, o, do, lse,
+                                                     workspace=ws, stream=stream))
+        by = algorithmic_bytes(ab.B, ab.N, ab.H, 1, 32, 8, 1, 1)
+        return {"tokens": ab.B * ab.N, "cluster_us": t_cl, "neighbors_us": t_nb, "fwd_us": t_f, "bwd_us": t_b,
+                "alg_MB": round((by["attn_fwd"] + by["attn_bwd"]) / 1e6, 2)}
+
+    def attn_summary(r, layers=1):
+        t = (r["fwd_us"] + r["bwd_us"]) * 1e-6
+        gbs = r["alg_MB"] * 1e6 / t / 1e9
+        return {"tokens_per_s_fwd_bwd": round(r["tokens"] / t, 1), "GB_s": round(gbs, 1),
+                "frac": round(gbs / hbm, 4), **r}
+
+    res = {}
+    c1 = attn_summary(attn_layer(synth.attn_tiny()))
+    c1["config"] = "tiny: 1 image, 16 x 16 grid, H = 4 (launch-bound)"
+    res["c1"] = c1
+    c2 = attn_summary(attn_layer(synth.attn_stage1(B=8)))
+    c2["config"] = "stage 1: 8 images x 2048 tokens, H = 4"
+    res["c2"] = c2
+    c3 = attn_summary(attn_layer(synth.attn_stage3(B=64)))
+    c3["config"] = "stage 3: 64 images x 328 tokens, H = 16"
+    res["c3"] = c3
+    coords = synth.sweep_coords(B=16)
+    tot_t, tot_tok, tot_b, stages = 0.0, 0, 0.0, []
+    for st, xy in enumerate(coords):
+        r = attn_layer(synth.attn_sweep_layer(xy, st, 0))
+        L = synth.SWEEP_LAYERS[st]
+        t = (r["fwd_us"] + r["bwd_us"]) * 1e-6
+        tot_t += L * t
+        tot_tok += L * r["tokens"]
+        tot_b += L * r["alg_MB"] * 1e6
+        stages.append({"stage": st + 1, "N": xy.shape[1], "H": synth.SWEEP_DIMS[st] // 32, "layers": L,
+                       "fwd_us": r["fwd_us"], "bwd_us": r["bwd_us"], "cluster_us": r["cluster_us"],
+                       "neighbors_us": r["neighbors_us"],
+                       "frac": round(r["alg_MB"] * 1e6 / t / 1e9 / hbm, 4)})
+    res["c4"] = {"config": "sweep: 16 images, stages 2048/819/328/131, layers 3/4/16/2",
+                 "tokens_per_s_fwd_bwd": round(tot_tok / tot_t, 1), "sweep_us": round(tot_t * 1e6, 1),
+                 "GB_s": round(tot_b / tot_t / 1e9, 1), "frac": round(tot_b / tot_t / 1e9 / hbm, 4),
+                 "stages": stages}
+    kt, kq, kb, kst = 0.0, 0, 0.0, []
+    for st, kbt in enumerate(synth.knn_decoder(B=16)):
+        xy, f = T(kbt.coords), T(kbt.feats, torch.bfloat16)
+        qq, pp, dout = T(kbt.queries), T(kbt.p), T(kbt.dout, torch.bfloat16)
+        table = acl.acl_knn_table(xy, kbt.GH, kbt.GW, kbt.K, stream=stream)
+        out = acl.acl_knn_gather_fwd(qq, f, xy, table, pp, stream=stream)
+        ws = torch.empty((acl.acl_knn_gather_workspace(kbt.B, kbt.Q, kbt.N, kbt.d, kbt.K),),
+                         dtype=torch.uint8, device=device)
+        t_t = timed(lambda: acl.acl_knn_table(xy, kbt.GH, kbt.GW, kbt.K, table=table, stream=stream))
+        t_f = timed(lambda: acl.acl_knn_gather_fwd(qq, f, xy, table, pp, out=out, stream=stream))
+        t_b = timed(lambda: acl.acl_knn_gather_bwd(qq, f, xy, table, pp, dout, workspace=ws, stream=stream))
+        by = algorithmic_bytes(kbt.B, kbt.N, 1, kbt.Q, kbt.d, kbt.K, kbt.GH, kbt.GW)
+        bts = by["knn_fwd"] + by["knn_bwd"]
+        t = (t_f + t_b) * 1e-6
+        kt += t
+        kq += kbt.B * kbt.Q
+        kb += bts
+        kst.append({"stage": st + 1, "N": kbt.N, "d": kbt.d, "table_us": t_t, "fwd_us": t_f, "bwd_us": t_b,
+                    "frac": round(bts / t / 1e9 / hbm, 4)})
+    res["c5"] = {"config": "decoder gather: 16 images x 4096 queries over the four stages, K = 8",
+                 "queries_per_s_fwd_bwd": round(kq / kt, 1), "gather_us": round(kt * 1e6, 1),
+                 "GB_s": round(kb / kt / 1e9, 1), "frac": round(kb / kt / 1e9 / hbm, 4), "stages": kst}
+    return res
+
+
 def run_only(args):
     """One extra part on cuda:0 (an eager call, then each call captured as a CUDA graph and
     replayed between CUDA events); prints its timing dict."""
@@ -893,8 +983,10 @@ def run_only(args):
     if args.only == "token_merge":
         sb = synth.step_batch(B=args.batch)
         res = token_merge_times(torch, acl, synth, sb, device, stream, measured_peaks())
-    else:
+    elif args.only == "decoder":
         res = decoder_times(torch, acl, synth, device, stream, measured_peaks(), B=args.batch)
+    else:
+        res = config_times(torch, acl, synth, device, stream, measured_peaks())
     print(json.dumps({"part": args.only, **res}))
 
 

@@ -212,7 +212,16 @@ __global__ void __launch_bounds__(kTThreads)
     const int row = m0 + 32 * (warp & 3) + lane;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
     const int c0 = (warp >> 2) * (kTN / 2);
-#pragma unroll 1
+    // the residual's 64 columns of this row, loaded before the accumulator is read back
+    float4 rv[kTN / 8];
+    if constexpr (EPI == kEpiResid) {
+        if (row < g.M) {
+            const float4* rp = reinterpret_cast<const float4*>(g.R + static_cast<size_t>(row) * g.ldc + n0 + c0);
+#pragma unroll
+            for (int e = 0; e < kTN / 8; ++e) rv[e] = rp[e];
+        }
+    }
+#pragma unroll
     for (int cj = c0; cj < c0 + kTN / 2; cj += 16) {
         uint32_t v[16];
         if (have) {
@@ -233,7 +242,7 @@ __global__ void __launch_bounds__(kTThreads)
         if constexpr (EPI == kEpiResid) {
 #pragma unroll
             for (int e = 0; e < 16; e += 4) {
-                const float4 r4 = *reinterpret_cast<const float4*>(g.R + o + e);
+                const float4 r4 = rv[(cj - c0 + e) / 4];
                 *reinterpret_cast<float4*>(g.Cf + o + e) =
                     make_float4(__uint_as_float(v[e]) + r4.x, __uint_as_float(v[e + 1]) + r4.y,
                                 __uint_as_float(v[e + 2]) + r4.z, __uint_as_float(v[e + 3]) + r4.w);

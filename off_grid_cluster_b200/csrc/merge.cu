@@ -887,6 +887,31 @@ __device__ __forceinline__ MemberLane member_lane(const float* sb, const float2*
     return r;
 }
 
+// Softmax statistics and the first round of members (lane x < 32) together: for a group of
+// at most 32 members one round of loads serves both (the same operations in the same order
+// as group_softmax followed by member_lane, which larger groups use).
+__device__ __forceinline__ MemberLane group_first_round(const float* sb, const float2* xb, const int32_t* mem,
+                                                        int n, int lane, float& gmax, float& inv) {
+    if (n > 32) {
+        group_softmax(sb, mem, n, lane, gmax, inv);
+        return member_lane(sb, xb, mem, lane, n, gmax, inv);
+    }
+    MemberLane r{0, 0.f, make_float2(0.f, 0.f)};
+    float sc = 0.f;
+    if (lane < n) {
+        r.t = mem[lane];
+        sc = sb[r.t];
+        r.p = xb[r.t];
+    }
+    float m = lane < n ? fmaxf(-FLT_MAX, sc) : -FLT_MAX;
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float e = lane < n ? 0.f + expf(sc - m) : 0.f;
+    gmax = m;
+    inv = 1.f / warp_sum(e);
+    if (lane < n) r.w = expf(sc - m) * inv;
+    return r;
+}
+
 // 5. forward merge: one warp per anchor; members in rounds of 32 (lane x holding member x's
 //    id and weight), lanes over 4-channel groups.
 __global__ void __launch_bounds__(kMergeThreads)
@@ -903,7 +928,7 @@ __global__ void __launch_bounds__(kMergeThreads)
     const int32_t* mem = members + static_cast<size_t>(b) * N + g0;
     const float2* xb = reinterpret_cast<const float2*>(xy) + static_cast<size_t>(b) * N;
     float gmax, inv;
-    group_softmax(sb, mem, n, lane, gmax, inv);
+    const MemberLane ml0 = group_first_round(sb, xb, mem, n, lane, gmax, inv);
     const bf16* fb = feats + static_cast<size_t>(b) * N * d;
     bf16* out = merged + static_cast<size_t>(ga) * d;
     float mx = 0.f, my = 0.f;
@@ -911,7 +936,7 @@ __global__ void __launch_bounds__(kMergeThreads)
         const int c = c0 + 4 * lane;
         float a[4] = {0.f, 0.f, 0.f, 0.f};
         for (int x0 = 0; x0 < n; x0 += 32) {
-            const MemberLane ml = member_lane(sb, xb, mem, x0 + lane, n, gmax, inv);
+            const MemberLane ml = x0 == 0 ? ml0 : member_lane(sb, xb, mem, x0 + lane, n, gmax, inv);
             if (c0 == 0) {
                 mx = fmaf(ml.w, ml.p.x, mx);
                 my = fmaf(ml.w, ml.p.y, my);
@@ -962,14 +987,14 @@ __global__ void __launch_bounds__(kMergeThreads)
     const int32_t* mem = members + static_cast<size_t>(b) * N + g0;
     const float2* xb = reinterpret_cast<const float2*>(xy) + static_cast<size_t>(b) * N;
     float gmax, inv;
-    group_softmax(sb, mem, n, lane, gmax, inv);
+    const MemberLane ml0 = group_first_round(sb, xb, mem, n, lane, gmax, inv);
     const bf16* fb = feats + static_cast<size_t>(b) * N * d;
     const bf16* dF = dmerged + static_cast<size_t>(ga) * d;
     const float2 dX = reinterpret_cast<const float2*>(dmxy)[ga];
     float* gb_out = g_out + static_cast<size_t>(b) * N;
     float sg = 0.f;
     for (int x0 = 0; x0 < n; x0 += 32) {
-        const MemberLane ml = member_lane(sb, xb, mem, x0 + lane, n, gmax, inv);
+        const MemberLane ml = x0 == 0 ? ml0 : member_lane(sb, xb, mem, x0 + lane, n, gmax, inv);
         const int nn = min(32, n - x0);
         for (int x1 = 0; x1 < nn; x1 += 4) {
             int tq[4];

@@ -117,3 +117,39 @@ def test_backward_finite_differences():
         xm[0, i, c] -= np.float32(e)
         ref = (_loss(mb, assign, xy=xp) - _loss(mb, assign, xy=xm)) / (2 * e)
         assert dxy[0, i, c] == pytest.approx(ref, rel=1e-5, abs=1e-6)
+
+
+def test_extreme_retention_rates():
+    """k = N: every token is its own anchor, so merging is the identity and the MLP gets no
+    gradient (a one-token group's softmax weight is constant); k = 1: one group, the merge is
+    the softmax-of-scores average of all tokens (numpy)."""
+    rng = np.random.default_rng(9)
+    xy = rng.uniform(0, 10, size=(1, 60, 2)).astype(np.float32)
+    mb = synth.merge_batch(xy, d=32, ds=1.0)
+    assert mb.k == 60
+    s = oracle.merge_scores(mb.feats, mb.w1, mb.b1, mb.w2, mb.b2)
+    anchors, assign = oracle.merge_select(s, mb.coords, mb.k)
+    np.testing.assert_array_equal(anchors[0], np.arange(60))
+    np.testing.assert_array_equal(assign[0], np.arange(60))
+    m, mxy = oracle.merge_fwd(mb.feats, mb.coords, s, mb.k, assign)
+    np.testing.assert_allclose(m[0], mb.feats[0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(mxy[0], mb.coords[0], rtol=0, atol=1e-12)
+    dm = np.ones((1, 60, 32))
+    df, dxy, dw1, db1, dw2, db2 = oracle.merge_bwd(mb.feats, mb.coords, mb.w1, mb.b1, mb.w2, mb.b2,
+                                                   mb.k, assign, dm, np.ones((1, 60, 2)))
+    np.testing.assert_allclose(df[0], 1.0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dxy[0], 1.0, rtol=0, atol=1e-12)
+    for g in (dw1, db1, dw2):
+        assert np.abs(g).max() <= 1e-12
+    assert abs(db2) <= 1e-12
+
+    one = synth.merge_batch(xy, d=32, ds=1.0 / 60.0)
+    assert one.k == 1
+    s1 = oracle.merge_scores(one.feats, one.w1, one.b1, one.w2, one.b2)
+    _, as1 = oracle.merge_select(s1, one.coords, 1)
+    assert np.all(as1 == 0)
+    m1, mxy1 = oracle.merge_fwd(one.feats, one.coords, s1, 1, as1)
+    w = np.exp(s1[0] - s1[0].max())
+    w /= w.sum()
+    np.testing.assert_allclose(m1[0, 0], w @ one.feats[0].astype(np.float64), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(mxy1[0, 0], w @ one.coords[0].astype(np.float64), rtol=1e-12, atol=1e-12)

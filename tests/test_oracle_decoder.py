@@ -87,3 +87,35 @@ def test_layer_backward_finite_differences():
             xm[idx] -= eps
             fd = (loss(**{name: xp}) - loss(**{name: xm})) / (2 * eps)
             assert abs(fd - grad[idx]) <= 1e-2 * scale, (name, idx, fd, grad[idx])
+
+
+def test_two_layer_chain_finite_differences():
+    """Two layers over two different stages: the gradient of the first layer's input, taken as
+    layer 2's df_in fed to layer 1 as its df_out, against central differences of the composed
+    loss (pins the coarse-to-fine chaining of the backward)."""
+    t1, t2 = tiny(seed=1), tiny(seed=2, N=14)
+    f0 = t1["f"]
+
+    def chain(f):
+        _, v1, f1 = oracle.decoder_layer_fwd(t1["ref"], f, t1["w_off"], t1["b_off"], t1["feats"],
+                                             t1["xy"], t1["table"], t1["p"], t1["w_o"])
+        q2, v2, f2 = oracle.decoder_layer_fwd(t2["ref"], f1, t2["w_off"], t2["b_off"], t2["feats"],
+                                              t2["xy"], t2["table"], t2["p"], t2["w_o"])
+        return v1, f1, q2, v2, f2
+
+    v1, f1, q2, v2, f2 = chain(f0)
+    q1 = oracle.decoder_offsets(t1["ref"], f0, t1["w_off"], t1["b_off"]).astype(np.float32)
+    df1 = oracle.decoder_layer_bwd(f1, t2["w_off"], t2["feats"], t2["xy"], t2["table"], t2["p"],
+                                   t2["w_o"], q2.astype(np.float32), v2, t2["df"])[0]
+    df0 = oracle.decoder_layer_bwd(f0, t1["w_off"], t1["feats"], t1["xy"], t1["table"], t1["p"],
+                                   t1["w_o"], q1, v1, df1)[0]
+    scale = np.abs(df0).max()
+    rng = np.random.default_rng(3)
+    eps = 1e-3
+    for _ in range(8):
+        idx = tuple(rng.integers(0, s) for s in f0.shape)
+        fp, fm = f0.copy(), f0.copy()
+        fp[idx] += eps
+        fm[idx] -= eps
+        fd = (np.sum(t2["df"] * chain(fp)[4]) - np.sum(t2["df"] * chain(fm)[4])) / (2 * eps)
+        assert abs(fd - df0[idx]) <= 1e-2 * scale, (idx, fd, df0[idx])

@@ -7,36 +7,41 @@
 //   s_ij = scale <q_i, k_j> + a_h dx + b_h dy - c_h (dx^2 + dy^2),  dx = x_j - x_i,
 //   O_i = softmax_j(s_ij) V,  lse_i = log sum_j exp(s_ij).
 //
-// Work unit: one warp owns one (image, cluster, head): the cluster's C = 8 queries
-// against its M <= 64 neighbourhood keys, D = 32.  The whole neighbourhood fits
-// one tile, so the softmax is exact in registers (no running rescale).  The
-// contractions run on the tensor cores as m16n8k16 bf16 MMAs with the operands
-// swapped so that the 8 queries sit on the MMA's N = 8 side and keys on M:
-//   S^T (M x 8)  = K (M x 32) . Q^T          -- 2 k-steps per 16-key tile
-//   O^T (32 x 8) = V^T (32 x M) . P^T        -- P^T comes from the S^T
-//                  accumulators by an in-register 8x8 transpose (movmatrix)
-// so no tile is padded beyond M's rounding to 16.
+// Work decomposition: every warp is an independent, persistent pipeline.  An item is one
+// (image, cluster, head); a warp walks a contiguous range of items, cluster-major, so it
+// takes consecutive heads of a cluster and then the next cluster.  Per item it gathers
+// the cluster's M key rows of K and V and its 8 query rows of Q (64 bytes = one head of
+// one token each) with 16-byte cp.async into one of two private stages, in slot order,
+// while the previous item computes; the neighbour rows and coordinates of the clusters
+// ahead are fetched into registers one and two clusters early.  No barrier, no shared
+// state between warps: the only waits are the warp's own copies.
 //
-// A CTA runs kUC = 4 consecutive clusters x kUH = 2 heads (8 warps).  Consecutive
-// clusters are siblings of the bisection tree and their neighbourhoods overlap, so the
-// CTA gathers the union of the group's neighbour blocks once (16-byte cp.async of
-// 128-byte token rows = the two heads) into XOR-swizzled shared tiles, and each warp
-// addresses its own 48 keys inside the union through a block map; ldmatrix reads them
-// without bank conflicts.  This halves the L2 -> SM traffic of the 6x-reused rows.
+// Per warp and item: the cluster's 8 queries against its M <= 64 keys, D = 32, on the
+// tensor cores as m16n8k16 bf16 MMAs with the operands swapped so that the 8 queries
+// sit on the MMA's N = 8 side and keys on M (no padded rows):
+//   S^T (M x 8)  = K (M x 32) . Q^T
+//   O^T (32 x 8) = V^T (32 x M) . P^T        (P^T from the S^T accumulators by an
+//                                             in-register 8x8 transpose, movmatrix;
+//                                             P carried as bf16 hi + lo, ~16 bits)
+//   l   (1 x 8)  = 1^T . P^T                 (row sums as one more MMA row)
+// The bias is expanded around a local origin so that it costs three FMAs per score:
+//   a dx + b dy - c (dx^2 + dy^2) = u_j + 2c x_i x_j + 2c y_i y_j + w_i,
+//   u_j = a x_j + b y_j - c (x_j^2 + y_j^2),  w_i = -a x_i - b y_i - c (x_i^2 + y_i^2);
+// w_i is constant along the softmax row, so it drops out of P and is added to lse.
 //
-// Backward (recompute, FA2-style, no atomics):
-//   pass 1, query-major (same CTA shape as the forward): recompute P from lse,
-//     dP^T = V . dO^T, Delta = rowsum(P o dP) (equal to <dO, O>, but exact in fp32
-//     because the whole key row is in the tile, and O need not be read),
-//     dS = P (dP - Delta), dQ^T = K^T . dS^T, per-(cluster, head) partial sums of the
-//     bias gradient.  One extra column of CTAs builds, per image, the reverse
-//     neighbourhood index: for every key cluster, the query clusters that list it.
-//   pass 2, key-major: CTA = 4 key clusters x 2 heads; the union of the query clusters
-//     in their reverse lists is gathered once, and each warp walks its own list two
-//     query clusters at a time (16 queries = one MMA M tile): S = Q K_h^T,
-//     dP = dO V_h^T, dV^T += dO^T P, dK^T += Q^T dS.  Extra CTAs reduce the bias
-//     partials in a fixed order.  A group whose lists overflow the union tile falls back
-//     to per-warp direct loads.
+// Backward (recompute, FA2-style, no atomics, every sum in a fixed order):
+//   prep (one CTA per image): the reverse neighbourhood index -- for every key cluster,
+//     the query clusters that list it, ascending, and their tokens.
+//   query pass (the forward's items): P = exp(s - lse), dP^T = V . dO^T,
+//     Delta_i = sum_j P dP (equal to <dO_i, O_i>, exact in fp32 because the whole key
+//     row is in the tile, so O is not read), dS = P (dP - Delta), dQ^T = K^T . dS^T,
+//     per-(cluster, head) partial sums of the bias gradient.
+//   key pass: an item is (image, key cluster, head, chunk of up to kChunk listed query
+//     clusters); the warp gathers its own K and V rows and the chunk's Q and dO rows and
+//     walks the chunk two query clusters at a time (16 queries = one MMA M tile):
+//     S = Q K^T, dP = dO V^T, dV^T += dO^T P, dK^T += Q^T dS, the sums carried over the
+//     chunks of a (key cluster, head) in list order.  Extra CTAs reduce the bias partials
+//     in a fixed order.
 #include <math.h>
 
 #include "internal.h"
@@ -45,340 +50,539 @@ namespace acl {
 
 namespace {
 
+constexpr int kWarps = 4;               // warps per CTA (independent pipelines)
+constexpr int kThreads = 32 * kWarps;
+constexpr int kRowB = 64;               // bytes of one head of one token (32 bf16)
+constexpr int kChunk = 6;               // listed query clusters per key-pass item
 
-// ------------------------------------------------------------------ layouts
+// ---------------------------------------------------------------- small helpers
 
-constexpr int kBwdKWarpBytes = 3584;
+__device__ __forceinline__ float sfu_ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float sfu_lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float sfu_rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
 
-// bf16 pair (hi) of two floats and the bf16 pair of their remainders (lo): hi + lo keeps
-// about 16 significant bits.
+// 4-byte global->shared copy; zero-filled when !valid.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
+    int n = valid ? 4 : 0;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(n)
+                 : "memory");
+}
+
+// bf16 pair (hi) of two floats and the bf16 pair of their remainders (lo).
 __device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uint32_t& lo) {
     hi = pack_bf16(x0, x1);
     lo = pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
 }
 
-// Write an (e x 8-token) fp32 accumulator pair, transposed to token rows, as bf16 rows of
-// `dst` (token-major [tok][H][32]) through a 512-byte staging tile.
-__device__ __forceinline__ void store_rows_t(const float (&acc)[2][4], float s0, float s1,
-                                             uint8_t* stage, const int* ids, size_t tok0, int H,
-                                             int h, bf16* dst, int lane) {
-    const int gq = lane >> 2, tq = lane & 3;
-    const uint32_t w0 = movm_t(pack_bf16(acc[0][0] * s0, acc[0][1] * s1));
-    const uint32_t w1 = movm_t(pack_bf16(acc[0][2] * s0, acc[0][3] * s1));
-    const uint32_t w2 = movm_t(pack_bf16(acc[1][0] * s0, acc[1][1] * s1));
-    const uint32_t w3 = movm_t(pack_bf16(acc[1][2] * s0, acc[1][3] * s1));
-    __syncwarp();
-    uint32_t* row = reinterpret_cast<uint32_t*>(stage + gq * 64);
-    row[tq] = w0;
-    row[4 + tq] = w1;
-    row[8 + tq] = w2;
-    row[12 + tq] = w3;
-    __syncwarp();
-    const int r = lane >> 2, ch = lane & 3;
-    const int id = ids[r];
-    if (id >= 0) {
-        const uint4 v = *reinterpret_cast<const uint4*>(stage + r * 64 + ch * 16);
-        *reinterpret_cast<uint4*>(dst + ((tok0 + id) * H + h) * 32 + ch * 8) = v;
-    }
-    __syncwarp();
+// Sum of three per-lane values over the warp with 9 shuffles: after the first two rounds
+// lane l holds a partial of value (l >> 3) & 3 (value 3 is a dummy zero).
+__device__ __forceinline__ void warp_sum3(float& x0, float& x1, float& x2, int lane) {
+    const bool hi16 = lane & 16;
+    float k0 = hi16 ? x2 : x0, k1 = hi16 ? 0.f : x1;
+    const float s0 = hi16 ? x0 : x2, s1 = hi16 ? x1 : 0.f;
+    k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    const bool hi8 = lane & 8;
+    float k = hi8 ? k1 : k0;
+    const float s = hi8 ? k0 : k1;
+    k += __shfl_xor_sync(0xffffffffu, s, 8);
+    k += __shfl_xor_sync(0xffffffffu, k, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    x0 = __shfl_sync(0xffffffffu, k, 0);
+    x1 = __shfl_sync(0xffffffffu, k, 8);
+    x2 = __shfl_sync(0xffffffffu, k, 16);
 }
 
-// Same, for key-major accumulators whose per-column scale is uniform.
-__device__ __forceinline__ void store_rows_t1(const float (&acc)[2][4], float s, uint8_t* stage,
-                                              const int* ids, size_t tok0, int H, int h, bf16* dst,
-                                              int lane) {
-    store_rows_t(acc, s, s, stage, ids, tok0, H, h, dst, lane);
+__device__ __forceinline__ int valid_tok(int t, int N) { return (t >= 0 && t < N) ? t : -1; }
+
+__device__ __forceinline__ float2 sh2(float2 v, int src) {
+    return make_float2(__shfl_sync(0xffffffffu, v.x, src), __shfl_sync(0xffffffffu, v.y, src));
 }
 
-// ------------------------------------------------- forward, neighbourhood unions
-//
-// One CTA per (image, group of kUC consecutive clusters, group of kUH heads); warp w owns
-// cluster w / kUH and head w % kUH of the group.  Consecutive clusters are siblings of the
-// bisection tree, so their neighbourhoods overlap: the CTA de-duplicates the group's
-// neighbour blocks (a block is one whole cluster, named by its first token), gathers each
-// union row's K and V once (kUH heads = 128 contiguous bytes per token) and every warp
-// reads its own neighbourhood out of the union tile through a block map.  Rows are
-// 128 bytes with the 16-byte chunk index XOR-ed by (row & 7); a neighbourhood block is 8
-// consecutive union rows, so the 8 rows of every ldmatrix hit 8 distinct bank groups.
-// Empty blocks map to 8 zero rows at the end of the tile.
-constexpr int kUC = 4;
-constexpr int kUH = 2;
-constexpr int kUWarps = kUC * kUH;
-constexpr int kUThreads = 32 * kUWarps;
-constexpr int kURow = 64 * kUH;  // bytes per union row
+// Tiles are rows of 64 bytes (one head of one token) in slot order; the 16-byte chunk c of
+// row r sits at r * 64 + ((c ^ ((r >> 1) & 3)) << 4) (tile64_off), so the 8 rows of every
+// ldmatrix fall in 8 distinct bank groups.  Lane l gathers chunk l & 3 of rows
+// (l >> 2) + 8 k; for those rows the swizzle depends on the lane only.
+__device__ __forceinline__ uint32_t gather_lane_off(int lane) {
+    return static_cast<uint32_t>((lane >> 2) * kRowB + (((lane & 3) ^ ((lane >> 3) & 3)) << 4));
+}
 
-struct UnionLayout {
-    int ks, vs, qs, stage, utok, uxy, qtok, qxy, krow, nbs, total;
+// ldmatrix lane offsets (bytes) of the tiles in slot order, for sub-matrix mi = lane >> 3:
+//   ls[kk]: rows 16 i + 8 (mi & 1) + (lane & 7), chunk 2 kk + (mi >> 1)  (A operand, + 1024 i)
+//   lt[m]:  rows 16 i + 8 (mi >> 1) + (lane & 7), chunk 2 m + (mi & 1)   (transposed A, + 1024 i)
+//   oq:     row lane & 7, chunk mi                                        (B operand, 8 rows)
+struct LaneOffs {
+    uint32_t ls0, ls1, lt0, lt1, oq;
 };
-__host__ __device__ __forceinline__ UnionLayout union_layout(int R, int MT) {
-    UnionLayout L;
-    const int rows = kUC * R * 8 + 8;  // union rows + a zero block
-    int o = 0;
-    L.ks = o; o += rows * kURow;
-    L.vs = o; o += rows * kURow;
-    L.qs = o; o += kUC * 8 * kURow;
-    L.stage = o; o += kUWarps * 512;
-    L.utok = o; o += 4 * (rows - 8);
-    L.uxy = o; o += 8 * (rows - 8);
-    L.qtok = o; o += 4 * kUC * 8;
-    L.qxy = o; o += 8 * kUC * 8;
-    L.krow = o; o += 4 * kUC * MT;
-    L.nbs = o; o += 4 * kUC * R * 8;        // the group's neighbour rows
-    L.total = (o + 15) & ~15;
-    return L;
+__device__ __forceinline__ LaneOffs lane_offs(int lane) {
+    const int mi = lane >> 3, r7 = lane & 7, sw = (r7 >> 1) & 3;
+    LaneOffs o;
+    o.ls0 = (mi & 1) * 512 + r7 * kRowB + (((0 + (mi >> 1)) ^ sw) << 4);
+    o.ls1 = (mi & 1) * 512 + r7 * kRowB + (((2 + (mi >> 1)) ^ sw) << 4);
+    o.lt0 = (mi >> 1) * 512 + r7 * kRowB + (((0 + (mi & 1)) ^ sw) << 4);
+    o.lt1 = (mi >> 1) * 512 + r7 * kRowB + (((2 + (mi & 1)) ^ sw) << 4);
+    o.oq = r7 * kRowB + ((mi ^ sw) << 4);
+    return o;
 }
 
-__device__ __forceinline__ uint32_t urow_off(int row, int ch) {
-    return static_cast<uint32_t>(row * kURow + ((ch ^ (row & 7)) << 4));
+// The tokens of one cluster's neighbourhood as a warp holds them: lane l has slots l and
+// l + 32 of the neighbour row (a, b) and slot l of the cluster row (q, lanes < 8); raw
+// values, made valid where used.
+struct Toks {
+    int a, b, q;
+};
+__device__ __forceinline__ Toks load_toks(const AttnArgs& a, int b, int g, int lane) {
+    Toks t;
+    const int32_t* nb = a.nbr + (static_cast<size_t>(b) * a.G + g) * a.M;
+    t.a = lane < a.M ? __ldg(nb + lane) : -1;
+    t.b = lane + 32 < a.M ? __ldg(nb + lane + 32) : -1;
+    t.q = lane < 8 ? __ldg(a.clusters + (static_cast<size_t>(b) * a.G + g) * 8 + lane) : -1;
+    return t;
 }
-
-// Union setup shared by the forward-shaped kernels: the neighbour rows of the CTA's kUC
-// clusters (one global round, into shared memory), their blocks de-duplicated by first
-// token (every warp computes the same map in registers, so no barrier is needed before
-// it is used), union row tokens, the per-cluster key-slot -> union row map and the
-// group's query tokens.  Coordinates follow with the tiles (union_coords_async).  All
-// threads of the CTA call it; returns the number of distinct blocks.
-__device__ __forceinline__ int union_setup(const AttnArgs& a, int b, int g0, int MT, const UnionLayout& L,
-                                           uint8_t* smem) {
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int G = a.G, N = a.N, M = a.M, R = a.R;
-    const int nblk = kUC * R;
-    int* utok = reinterpret_cast<int*>(smem + L.utok);
-    int* qtok = reinterpret_cast<int*>(smem + L.qtok);
-    int* krow = reinterpret_cast<int*>(smem + L.krow);
-    int* nbs = reinterpret_cast<int*>(smem + L.nbs);
-    for (int i = tid; i < nblk * 8; i += blockDim.x) {
-        const int cw = i / M, m = i - cw * M;
-        const int g = g0 + cw;
-        int t = -1;
-        if (g < G) {
-            t = a.nbr[(static_cast<size_t>(b) * G + g) * M + m];
-            if (t < 0 || t >= N) t = -1;
-        }
-        nbs[i] = t;
-    }
-    for (int i = tid; i < kUC * 8; i += blockDim.x) {
-        const int g = g0 + (i >> 3);
-        int id = -1;
-        if (g < G) {
-            id = a.clusters[(static_cast<size_t>(b) * G + g) * 8 + (i & 7)];
-            if (id < 0 || id >= N) id = -1;
-        }
-        qtok[i] = id;
-    }
-    __syncthreads();
-    // lane j < nblk: block j's union index, or the index of its first occurrence (the
-    // lowest lane holding the same first token)
-    const int f = lane < nblk ? nbs[lane * 8] : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, f);
-    const int lead = __ffs(peers) - 1;
-    const int dup = (f >= 0 && lead != lane) ? lead : -1;
-    const bool isnew = f >= 0 && lead == lane;
-    const unsigned newmask = __ballot_sync(0xffffffffu, isnew);
-    int u = isnew ? __popc(newmask & ((1u << lane) - 1u)) : -1;
-    const int ud = __shfl_sync(0xffffffffu, u, dup >= 0 ? dup : 0);
-    if (dup >= 0) u = ud;
-    const int nU = __popc(newmask);
-    for (int base = 0; base < nblk * 8; base += blockDim.x) {
-        const int i = base + tid;
-        const int blk = min(i >> 3, 31);
-        const int ub = __shfl_sync(0xffffffffu, u, blk);
-        const bool first = __shfl_sync(0xffffffffu, isnew ? 1 : 0, blk) != 0;
-        if (i < nblk * 8 && first) utok[ub * 8 + (i & 7)] = nbs[i];
-    }
-    for (int base = 0; base < kUC * MT; base += blockDim.x) {
-        const int i = base + tid;
-        const int cw = i / MT, m = i - cw * MT;
-        const int blk = min(cw * R + (m >> 3), 31);
-        const int ub = __shfl_sync(0xffffffffu, u, blk);
-        if (i < kUC * MT) krow[i] = (m < M && ub >= 0) ? ub * 8 + (m & 7) : -1;
-    }
-    __syncthreads();
-    return nU;
-}
-
-// Coordinates of the union rows and of the group's queries, as asynchronous copies in
-// the caller's current cp.async group (rows without a token read as (0, 0)).
-__device__ __forceinline__ void union_coords_async(const AttnArgs& a, int b, int nU, const UnionLayout& L,
-                                                   uint8_t* smem) {
-    const int* utok = reinterpret_cast<const int*>(smem + L.utok);
-    const int* qtok = reinterpret_cast<const int*>(smem + L.qtok);
+// Their coordinates (zero for empty slots).
+struct TokXY {
+    float2 a, b, q;
+};
+__device__ __forceinline__ TokXY load_xy(const AttnArgs& a, int b, const Toks& t) {
     const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(b) * a.N;
-    for (int i = threadIdx.x; i < nU * 8; i += blockDim.x) {
-        const int t = utok[i];
-        cp_async8(smem_addr(smem + L.uxy) + 8 * i, xyb + (t >= 0 ? t : 0), t >= 0);
-    }
-    for (int i = threadIdx.x; i < kUC * 8; i += blockDim.x) {
-        const int t = qtok[i];
-        cp_async8(smem_addr(smem + L.qxy) + 8 * i, xyb + (t >= 0 ? t : 0), t >= 0);
+    const int ta = valid_tok(t.a, a.N), tb = valid_tok(t.b, a.N), tq = valid_tok(t.q, a.N);
+    TokXY x;
+    x.a = ta >= 0 ? __ldg(xyb + ta) : make_float2(0.f, 0.f);
+    x.b = tb >= 0 ? __ldg(xyb + tb) : make_float2(0.f, 0.f);
+    x.q = tq >= 0 ? __ldg(xyb + tq) : make_float2(0.f, 0.f);
+    return x;
+}
+
+// The next cluster after (b, g).
+__device__ __forceinline__ void next_cluster(int& b, int& g, int G) {
+    if (++g == G) {
+        g = 0;
+        ++b;
     }
 }
+
+// ------------------------------------------------------------- cluster items
+
+// Per-warp stage of the forward (BWD = false) and query pass (BWD = true): the M key rows of
+// K and V, the 8 query rows of Q (and dO), and the 8 queries' lse.
+template <int MT, bool BWD>
+struct QTile {
+    static constexpr int K = 0;
+    static constexpr int V = MT * kRowB;
+    static constexpr int Q = 2 * MT * kRowB;
+    static constexpr int DO = Q + 8 * kRowB;
+    static constexpr int LSE = DO + (BWD ? 8 * kRowB : 0);
+    static constexpr int STAGE = LSE + (BWD ? 32 : 0);
+    static constexpr int WARP = 2 * STAGE;
+};
+
+// One cluster's rows as the gather needs them: the tokens of rows gq + 8 k (made valid),
+// and of query row gq.
+template <int NK>
+struct Rows {
+    int rt[NK];
+    int qt;
+};
+template <int NK>
+__device__ __forceinline__ Rows<NK> cluster_rows(const Toks& t, int lane, int N) {
+    Rows<NK> r;
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+        r.rt[k] = valid_tok(__shfl_sync(0xffffffffu, k < 4 ? t.a : t.b, (lane >> 2) + 8 * (k & 3)), N);
+    r.qt = valid_tok(__shfl_sync(0xffffffffu, t.q, lane >> 2), N);
+    return r;
+}
+
+// Gather head h of a cluster of image b into the stage at sb (a shared address).
+template <int MT, bool BWD>
+__device__ __forceinline__ void gather_cluster(const AttnArgs& a, int b, int h, const Rows<MT / 8>& r,
+                                               uint32_t sb, int lane) {
+    using T = QTile<MT, BWD>;
+    const uint32_t lo = gather_lane_off(lane);
+    const size_t rowel = static_cast<size_t>(a.H) * 32;
+    const size_t tok0 = static_cast<size_t>(b) * a.N;
+    const size_t hoff = static_cast<size_t>(h) * 32 + (lane & 3) * 8;
+#pragma unroll
+    for (int k = 0; k < MT / 8; ++k) {
+        const int t = r.rt[k];
+        const size_t src = t >= 0 ? (tok0 + t) * rowel + hoff : 0;
+        cp_async16(sb + T::K + 512 * k + lo, a.k + src, t >= 0);
+        cp_async16(sb + T::V + 512 * k + lo, a.v + src, t >= 0);
+    }
+    const int t = r.qt;
+    const size_t src = t >= 0 ? (tok0 + t) * rowel + hoff : 0;
+    cp_async16(sb + T::Q + lo, a.q + src, t >= 0);
+    if (BWD) {
+        cp_async16(sb + T::DO + lo, a.dout + src, t >= 0);
+        if ((lane & 3) == 0)
+            cp_async4(sb + T::LSE + 4 * (lane >> 2), a.lse_in + (t >= 0 ? (tok0 + t) * a.H + h : 0), t >= 0);
+    }
+}
+
+// Per-lane geometry of one cluster, reused for every head: the lane's keys k = 2 i + hi
+// (slot gq + 8 k) and query columns 2 tq, 2 tq + 1 in local coordinates (origin: the
+// cluster's first slot), and the query tokens the lane writes.
+template <int MTILES>
+struct Geo {
+    float kx[2 * MTILES], ky[2 * MTILES];
+    unsigned kval;
+    float qx[2], qy[2];
+    int qo;      // query row gq (O / dQ rows)
+    int ql[2];   // query columns 2 tq, 2 tq + 1 (lse / Delta)
+};
 
 template <int MTILES>
-__global__ void __launch_bounds__(kUThreads) attn_fwd_union_kernel(const AttnArgs a) {
-    constexpr int MT = 16 * MTILES;
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int R = a.R;
-    const UnionLayout L = union_layout(R, MT);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int cg = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-    const int G = a.G, N = a.N, H = a.H;
-    const int g0 = cg * kUC;
-    const int nblk = kUC * R;
-    const int ZR = nblk * 8;
-    uint8_t* ks = smem + L.ks;
-    uint8_t* vs = smem + L.vs;
-    uint8_t* qs = smem + L.qs;
-    const int* utok = reinterpret_cast<const int*>(smem + L.utok);
-    const float2* uxy = reinterpret_cast<const float2*>(smem + L.uxy);
-    const int* qtok = reinterpret_cast<const int*>(smem + L.qtok);
-    const float2* qxy = reinterpret_cast<const float2*>(smem + L.qxy);
-    const int* krow = reinterpret_cast<const int*>(smem + L.krow);
-    const size_t tok0 = static_cast<size_t>(b) * N;
-
-    // 1-3. the group's neighbour rows, de-duplicated blocks, union rows and block map
-    const int nU = union_setup(a, b, g0, MT, L, smem);
-    // 4. gather the union's K and V rows, the group's Q rows, and zero the spare block;
-    //    thread tid copies 16-byte chunk tid % 8 of rows tid / 8, tid / 8 + 32, ...
-    const int hlo = hg * kUH;
-    const int ch = tid & 7;
-    const bool ch_ok = hlo + (ch >> 2) < H;
-    const size_t cbase = (tok0 * H + hlo) * 32 + ch * 8;
-    const size_t tstride = static_cast<size_t>(H) * 32;
-    const int urows = nU * 8;
-    for (int row = tid >> 3; row < urows + 8; row += kUThreads / 8) {
-        const int t = row < urows ? utok[row] : -1;
-        const bool ok = t >= 0 && ch_ok;
-        const int drow = row < urows ? row : ZR + (row - urows);
-        cp_async16(smem_addr(ks) + urow_off(drow, ch), a.k + (ok ? cbase + t * tstride : 0), ok);
-    }
-    for (int row = tid >> 3; row < kUC * 8; row += kUThreads / 8) {
-        const int t = qtok[row];
-        const bool ok = t >= 0 && ch_ok;
-        cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + (ok ? cbase + t * tstride : 0), ok);
-    }
-    union_coords_async(a, b, nU, L, smem);
-    cp_async_commit();  // group 0: K, Q, coordinates
-    for (int row = tid >> 3; row < urows + 8; row += kUThreads / 8) {
-        const int t = row < urows ? utok[row] : -1;
-        const bool ok = t >= 0 && ch_ok;
-        const int drow = row < urows ? row : ZR + (row - urows);
-        cp_async16(smem_addr(vs) + urow_off(drow, ch), a.v + (ok ? cbase + t * tstride : 0), ok);
-    }
-    cp_async_commit();  // group 1: V (lands while S and the softmax run)
-    cp_async_wait<1>();
-    __syncthreads();
-
-    // 5. one (cluster, head) per warp
-    const int cw = warp / kUH, hw = warp % kUH;
-    const int g = g0 + cw;
-    // a warp past the last cluster or head computes on masked data and stores nothing (it
-    // must still reach the barrier before the V tile is read)
-    const bool active = g < G && hlo + hw < H;
-    const int h = active ? hlo + hw : 0;
-    const int gq = lane >> 2, tq = lane & 3, mi = lane >> 3;
-    const int* kr = krow + cw * MT;
-    // row bases of the neighbourhood blocks this lane addresses
-    // row 0 of each neighbourhood block this lane addresses: (mi & 1) picks the block of
-    // the S / dQ operands, (mi >> 1) the block of the transposed V / K operands
-    int base_s[MTILES], base_t[MTILES];
+__device__ __forceinline__ Geo<MTILES> make_geo(const Toks& t, const TokXY& x, const int (&rt)[2 * MTILES], int lane,
+                                                int N) {
+    const int gq = lane >> 2, tq = lane & 3;
+    Geo<MTILES> g;
+    const float2 o = sh2(x.q, 0);
+    g.kval = 0u;
 #pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-        const int s0 = 2 * i + (mi & 1), s1 = 2 * i + (mi >> 1);
-        const int r0 = (s0 * 8 < a.M) ? kr[s0 * 8] : -1;
-        const int r1 = (s1 * 8 < a.M) ? kr[s1 * 8] : -1;
-        base_s[i] = r0 >= 0 ? r0 : ZR;
-        base_t[i] = r1 >= 0 ? r1 : ZR;
+    for (int k = 0; k < 2 * MTILES; ++k) {
+        const float2 p = sh2(k < 4 ? x.a : x.b, gq + 8 * (k & 3));
+        const bool ok = rt[k] >= 0;
+        g.kx[k] = ok ? p.x - o.x : 0.f;
+        g.ky[k] = ok ? p.y - o.y : 0.f;
+        g.kval |= ok ? (1u << k) : 0u;
     }
-    uint32_t qf0, qf1, qf2, qf3;
-    ldsm_x4(smem_addr(qs) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), qf0, qf1, qf2, qf3);
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        const float2 p = sh2(x.q, 2 * tq + c);
+        g.qx[c] = p.x - o.x;
+        g.qy[c] = p.y - o.y;
+        g.ql[c] = valid_tok(__shfl_sync(0xffffffffu, t.q, 2 * tq + c), N);
+    }
+    g.qo = valid_tok(__shfl_sync(0xffffffffu, t.q, gq), N);
+    return g;
+}
+
+// ------------------------------------------------------------------ forward
+
+template <int MTILES>
+__device__ __forceinline__ void fwd_item(const AttnArgs& a, int b, int h, uint32_t sb, const LaneOffs& lo,
+                                         const Geo<MTILES>& g, int lane) {
+    using T = QTile<16 * MTILES, false>;
+    const int gq = lane >> 2, tq = lane & 3;
+    const uint32_t kb = sb + T::K, vb = sb + T::V, qb = sb + T::Q;
+    const float an = __ldg(a.bias + 3 * h), bn = __ldg(a.bias + 3 * h + 1), cn = __ldg(a.bias + 3 * h + 2);
+    const float a2 = an * kLog2e, b2 = bn * kLog2e, c2 = cn * kLog2e;
+    const float sc = a.scale * kLog2e;
+    float u[2 * MTILES];
+#pragma unroll
+    for (int k = 0; k < 2 * MTILES; ++k)
+        u[k] = ((g.kval >> k) & 1u)
+                   ? fmaf(a2, g.kx[k], fmaf(b2, g.ky[k], -c2 * fmaf(g.kx[k], g.kx[k], g.ky[k] * g.ky[k])))
+                   : -INFINITY;
+    const float X[2] = {2.f * c2 * g.qx[0], 2.f * c2 * g.qx[1]};
+    const float Y[2] = {2.f * c2 * g.qy[0], 2.f * c2 * g.qy[1]};
+
+    uint32_t qf[4];
+    ldsm_x4(qb + lo.oq, qf[0], qf[1], qf[2], qf[3]);
     float sacc[MTILES][4];
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) {
         sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            const int row = base_s[i] + (lane & 7);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(smem_addr(ks) + urow_off(row, hw * 4 + 2 * kk + (mi >> 1)), a0, a1, a2, a3);
-            mma_bf16(sacc[i], a0, a1, a2, a3, kk ? qf2 : qf0, kk ? qf3 : qf1);
-        }
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4(kb + 1024 * i + lo.ls0, r0, r1, r2, r3);
+        mma_bf16(sacc[i], r0, r1, r2, r3, qf[0], qf[1]);
+        ldsm_x4(kb + 1024 * i + lo.ls1, r0, r1, r2, r3);
+        mma_bf16(sacc[i], r0, r1, r2, r3, qf[2], qf[3]);
     }
-    const float sc = a.scale * kLog2e;
-    const float ba = a.bias[3 * h] * kLog2e, bb = a.bias[3 * h + 1] * kLog2e,
-                bc = a.bias[3 * h + 2] * kLog2e;
-    const float2 qa = qxy[cw * 8 + 2 * tq], qb = qxy[cw * 8 + 2 * tq + 1];
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+    float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) {
 #pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-            const int row = kr[16 * i + gq + 8 * hi];
-            const bool kv = row >= 0 && utok[row] >= 0;
-            const float2 kp = kv ? uxy[row] : make_float2(0.f, 0.f);
-            float dx = kp.x - qa.x, dy = kp.y - qa.y;
-            const float v0 = sacc[i][2 * hi] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
-            dx = kp.x - qb.x;
-            dy = kp.y - qb.y;
-            const float v1 = sacc[i][2 * hi + 1] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
-            sacc[i][2 * hi] = kv ? v0 : -INFINITY;
-            sacc[i][2 * hi + 1] = kv ? v1 : -INFINITY;
-            mx0 = fmaxf(mx0, sacc[i][2 * hi]);
-            mx1 = fmaxf(mx1, sacc[i][2 * hi + 1]);
+        for (int j = 0; j < 4; ++j) {
+            const int k = 2 * i + (j >> 1), c = j & 1;
+            const float t = fmaf(sacc[i][j], sc, fmaf(X[c], g.kx[k], fmaf(Y[c], g.ky[k], u[k])));
+            sacc[i][j] = t;
+            mx[c] = fmaxf(mx[c], t);
         }
     }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
+        mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
     }
-    const float m0 = (mx0 == -INFINITY) ? 0.f : mx0;
-    const float m1 = (mx1 == -INFINITY) ? 0.f : mx1;
-    float l0 = 0.f, l1 = 0.f;
-    uint32_t pbh[MTILES][2], pbl[MTILES][2];
+    const float m0 = mx[0] == -INFINITY ? 0.f : mx[0];
+    const float m1 = mx[1] == -INFINITY ? 0.f : mx[1];
+    uint32_t ph[MTILES][2], pl[MTILES][2];
 #pragma unroll
     for (int i = 0; i < MTILES; ++i) {
-        const float p0 = exp2f(sacc[i][0] - m0), p1 = exp2f(sacc[i][1] - m1);
-        const float p2 = exp2f(sacc[i][2] - m0), p3 = exp2f(sacc[i][3] - m1);
-        l0 += p0 + p2;
-        l1 += p1 + p3;
+        const float p0 = sfu_ex2(sacc[i][0] - m0), p1 = sfu_ex2(sacc[i][1] - m1);
+        const float p2 = sfu_ex2(sacc[i][2] - m0), p3 = sfu_ex2(sacc[i][3] - m1);
         uint32_t h01, l01, h23, l23;
         split_bf16(p0, p1, h01, l01);
         split_bf16(p2, p3, h23, l23);
-        pbh[i][0] = movm_t(h01);
-        pbl[i][0] = movm_t(l01);
-        pbh[i][1] = movm_t(h23);
-        pbl[i][1] = movm_t(l23);
+        ph[i][0] = movm_t(h01);
+        ph[i][1] = movm_t(h23);
+        pl[i][0] = movm_t(l01);
+        pl[i][1] = movm_t(l23);
     }
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    }
-    cp_async_wait<0>();
-    __syncthreads();  // V tile complete (all threads reach this: no early exit above)
-    float oacc[2][4];
+    float oacc[2][4], lacc[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t ones = gq == 0 ? 0x3F803F80u : 0u;  // row 0 of the A operand = 1
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
         oacc[m][0] = oacc[m][1] = oacc[m][2] = oacc[m][3] = 0.f;
 #pragma unroll
         for (int i = 0; i < MTILES; ++i) {
-            const int row = base_t[i] + (lane & 7);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(smem_addr(vs) + urow_off(row, hw * 4 + 2 * m + (mi & 1)), a0, a1, a2, a3);
-            mma_bf16(oacc[m], a0, a1, a2, a3, pbl[i][0], pbl[i][1]);
-            mma_bf16(oacc[m], a0, a1, a2, a3, pbh[i][0], pbh[i][1]);
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4_t(vb + 1024 * i + (m ? lo.lt1 : lo.lt0), r0, r1, r2, r3);
+            mma_bf16(oacc[m], r0, r1, r2, r3, pl[i][0], pl[i][1]);
+            mma_bf16(oacc[m], r0, r1, r2, r3, ph[i][0], ph[i][1]);
         }
     }
-    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
-    const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
-    if (!active) return;
-    store_rows_t(oacc, i0, i1, smem + L.stage + warp * 512, qtok + cw * 8, tok0, H, h, a.o, lane);
-    if (gq == 0) {
-        const int q0 = qtok[cw * 8 + 2 * tq], q1 = qtok[cw * 8 + 2 * tq + 1];
-        if (q0 >= 0) a.lse[(tok0 + q0) * H + h] = l0 > 0.f ? (m0 + log2f(l0)) * kLn2 : -INFINITY;
-        if (q1 >= 0) a.lse[(tok0 + q1) * H + h] = l1 > 0.f ? (m1 + log2f(l1)) * kLn2 : -INFINITY;
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+        mma_bf16(lacc, ones, 0u, ones, 0u, pl[i][0], pl[i][1]);
+        mma_bf16(lacc, ones, 0u, ones, 0u, ph[i][0], ph[i][1]);
     }
+    // lanes 0..3 hold l of columns 2 tq, 2 tq + 1
+    const float l0 = __shfl_sync(0xffffffffu, lacc[0], tq);
+    const float l1 = __shfl_sync(0xffffffffu, lacc[1], tq);
+    const float i0 = l0 > 0.f ? sfu_rcp(l0) : 0.f;
+    const float i1 = l1 > 0.f ? sfu_rcp(l1) : 0.f;
+    const size_t tok0 = static_cast<size_t>(b) * a.N;
+    // O^T (dims x queries) -> rows of O: after the transpose lane (g, t) holds dims
+    // 2t, 2t + 1 (+ 8, + 16, + 24) of query g
+    const uint32_t w0 = movm_t(pack_bf16(oacc[0][0] * i0, oacc[0][1] * i1));
+    const uint32_t w1 = movm_t(pack_bf16(oacc[0][2] * i0, oacc[0][3] * i1));
+    const uint32_t w2 = movm_t(pack_bf16(oacc[1][0] * i0, oacc[1][1] * i1));
+    const uint32_t w3 = movm_t(pack_bf16(oacc[1][2] * i0, oacc[1][3] * i1));
+    if (g.qo >= 0) {
+        uint32_t* dst = reinterpret_cast<uint32_t*>(a.o + ((tok0 + g.qo) * a.H + h) * 32) + tq;
+        dst[0] = w0;
+        dst[4] = w1;
+        dst[8] = w2;
+        dst[12] = w3;
+    }
+    if (gq == 0) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const float l = lacc[c];
+            const float mc = c ? m1 : m0;
+            // w_i in natural units: the query-constant part of the expanded bias
+            const float wq = -(an * g.qx[c] + bn * g.qy[c] + cn * fmaf(g.qx[c], g.qx[c], g.qy[c] * g.qy[c]));
+            if (g.ql[c] >= 0)
+                a.lse[(tok0 + g.ql[c]) * a.H + h] = l > 0.f ? (mc + sfu_lg2(l)) * kLn2 + wq : -INFINITY;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- query pass
+
+template <int MTILES>
+__device__ __forceinline__ void query_item(const AttnArgs& a, int b, int gabs, int h, uint32_t sb,
+                                           const float* lse_s, const LaneOffs& lo, const Geo<MTILES>& g,
+                                           int lane) {
+    using T = QTile<16 * MTILES, true>;
+    const int gq = lane >> 2, tq = lane & 3;
+    const uint32_t kb = sb + T::K, vb = sb + T::V, qb = sb + T::Q, db_ = sb + T::DO;
+    const float an = __ldg(a.bias + 3 * h), bn = __ldg(a.bias + 3 * h + 1), cn = __ldg(a.bias + 3 * h + 2);
+    const float a2 = an * kLog2e, b2 = bn * kLog2e, c2 = cn * kLog2e;
+    const float sc = a.scale * kLog2e;
+    float u[2 * MTILES];
+#pragma unroll
+    for (int k = 0; k < 2 * MTILES; ++k)
+        u[k] = ((g.kval >> k) & 1u)
+                   ? fmaf(a2, g.kx[k], fmaf(b2, g.ky[k], -c2 * fmaf(g.kx[k], g.kx[k], g.ky[k] * g.ky[k])))
+                   : -INFINITY;
+    float X[2], Y[2], Lq[2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        X[c] = 2.f * c2 * g.qx[c];
+        Y[c] = 2.f * c2 * g.qy[c];
+        const float l = lse_s[2 * tq + c];
+        const bool ok = g.ql[c] >= 0 && l != -INFINITY;
+        // P = exp2(t - L'), L' = lse log2e - w2 with w2 the query-constant bias part
+        const float qr2 = fmaf(g.qx[c], g.qx[c], g.qy[c] * g.qy[c]);
+        Lq[c] = ok ? fmaf(l, kLog2e, fmaf(a2, g.qx[c], fmaf(b2, g.qy[c], c2 * qr2))) : INFINITY;
+    }
+    uint32_t qf[4], df[4];
+    ldsm_x4(qb + lo.oq, qf[0], qf[1], qf[2], qf[3]);
+    ldsm_x4(db_ + lo.oq, df[0], df[1], df[2], df[3]);
+    float sacc[MTILES][4], dp[MTILES][4];
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+        sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
+        dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            uint32_t r0, r1, r2, r3;
+            const uint32_t off = 1024 * i + (kk ? lo.ls1 : lo.ls0);
+            ldsm_x4(kb + off, r0, r1, r2, r3);
+            mma_bf16(sacc[i], r0, r1, r2, r3, qf[2 * kk], qf[2 * kk + 1]);
+            ldsm_x4(vb + off, r0, r1, r2, r3);
+            mma_bf16(dp[i], r0, r1, r2, r3, df[2 * kk], df[2 * kk + 1]);
+        }
+    }
+    float pd[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int k = 2 * i + (j >> 1), c = j & 1;
+            const float t = fmaf(sacc[i][j], sc, fmaf(X[c], g.kx[k], fmaf(Y[c], g.ky[k], u[k])));
+            const float p = sfu_ex2(t - Lq[c]);
+            sacc[i][j] = p;
+            pd[c] = fmaf(p, dp[i][j], pd[c]);
+        }
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        pd[0] += __shfl_xor_sync(0xffffffffu, pd[0], o);
+        pd[1] += __shfl_xor_sync(0xffffffffu, pd[1], o);
+    }
+    // dS and the bias-gradient sums per query column: S0 = sum dS, Sx = sum dS x_j, ...
+    float S0[2] = {0.f, 0.f}, Sx[2] = {0.f, 0.f}, Sy[2] = {0.f, 0.f}, Sr[2] = {0.f, 0.f};
+    uint32_t dsb[MTILES][2];
+#pragma unroll
+    for (int i = 0; i < MTILES; ++i) {
+        float ds[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int k = 2 * i + (j >> 1), c = j & 1;
+            const float v = sacc[i][j] * (dp[i][j] - pd[c]);
+            ds[j] = v;
+            S0[c] += v;
+            Sx[c] = fmaf(v, g.kx[k], Sx[c]);
+            Sy[c] = fmaf(v, g.ky[k], Sy[c]);
+            Sr[c] = fmaf(v, fmaf(g.kx[k], g.kx[k], g.ky[k] * g.ky[k]), Sr[c]);
+        }
+        dsb[i][0] = movm_t(pack_bf16(ds[0], ds[1]));
+        dsb[i][1] = movm_t(pack_bf16(ds[2], ds[3]));
+    }
+    // sum_j dS (x_j - x_i) = Sx - x_i S0;  sum_j dS |p_j - p_i|^2 = Sr - 2 x_i Sx - 2 y_i Sy + r_i S0
+    float ga = 0.f, gb = 0.f, gc = 0.f;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        ga += Sx[c] - g.qx[c] * S0[c];
+        gb += Sy[c] - g.qy[c] * S0[c];
+        gc += Sr[c] - 2.f * (g.qx[c] * Sx[c] + g.qy[c] * Sy[c]) +
+              fmaf(g.qx[c], g.qx[c], g.qy[c] * g.qy[c]) * S0[c];
+    }
+    warp_sum3(ga, gb, gc, lane);
+    const size_t tok0 = static_cast<size_t>(b) * a.N;
+    if (lane == 0) {
+        float* part = a.dbias_part + ((static_cast<size_t>(b) * a.G + gabs) * a.H + h) * 3;
+        part[0] = ga;
+        part[1] = gb;
+        part[2] = -gc;
+    }
+    if (gq == 0) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+            if (g.ql[c] >= 0) a.delta[(tok0 + g.ql[c]) * a.H + h] = pd[c];
+    }
+    float dq[2][4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        dq[m][0] = dq[m][1] = dq[m][2] = dq[m][3] = 0.f;
+#pragma unroll
+        for (int i = 0; i < MTILES; ++i) {
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4_t(kb + 1024 * i + (m ? lo.lt1 : lo.lt0), r0, r1, r2, r3);
+            mma_bf16(dq[m], r0, r1, r2, r3, dsb[i][0], dsb[i][1]);
+        }
+    }
+    const float scl = a.scale;
+    const uint32_t w0 = movm_t(pack_bf16(dq[0][0] * scl, dq[0][1] * scl));
+    const uint32_t w1 = movm_t(pack_bf16(dq[0][2] * scl, dq[0][3] * scl));
+    const uint32_t w2 = movm_t(pack_bf16(dq[1][0] * scl, dq[1][1] * scl));
+    const uint32_t w3 = movm_t(pack_bf16(dq[1][2] * scl, dq[1][3] * scl));
+    if (g.qo >= 0) {
+        uint32_t* dst = reinterpret_cast<uint32_t*>(a.dq + ((tok0 + g.qo) * a.H + h) * 32) + tq;
+        dst[0] = w0;
+        dst[4] = w1;
+        dst[8] = w2;
+        dst[12] = w3;
+    }
+}
+
+// ------------------------------------------- forward / query pass: the warp pipeline
+
+// One warp's items [i0, i1) (item = (image, cluster, head), cluster-major).  While item i
+// computes, item i + 1 is in flight; the neighbour rows of the cluster after next and the
+// coordinates of the next cluster load into registers at every cluster start.
+template <int MTILES, bool BWD>
+__device__ __forceinline__ void cluster_items(const AttnArgs& a, long long i0, long long i1, uint8_t* wsm) {
+    constexpr int MT = 16 * MTILES, NK = MT / 8;
+    using T = QTile<MT, BWD>;
+    const int lane = threadIdx.x & 31;
+    const int H = a.H, G = a.G, N = a.N;
+    const LaneOffs lo = lane_offs(lane);
+    const uint32_t wb = smem_addr(wsm);
+    long long c = i0 / H;                 // global cluster index b * G + g
+    int h = static_cast<int>(i0 - c * H);
+    const long long c_last = (i1 - 1) / H;
+    const int h_last_end = static_cast<int>(i1 - 1 - c_last * H) + 1;
+    int b = static_cast<int>(c / G), g = static_cast<int>(c - static_cast<long long>(b) * G);
+    int b1 = b, g1 = g;
+    next_cluster(b1, g1, G);
+    int b2 = b1, g2 = g1;
+    next_cluster(b2, g2, G);
+    Toks cur = load_toks(a, b, g, lane);
+    Toks nx = c + 1 <= c_last ? load_toks(a, b1, g1, lane) : Toks{-1, -1, -1};
+    TokXY cxy = load_xy(a, b, cur);
+    Rows<NK> rows = cluster_rows<NK>(cur, lane, N);
+    int st = 0;
+    gather_cluster<MT, BWD>(a, b, h, rows, wb, lane);
+    cp_async_commit();
+    for (;;) {
+        const bool lastc = c == c_last;
+        const int hend = lastc ? h_last_end : H;
+        const Toks nn = c + 2 <= c_last ? load_toks(a, b2, g2, lane) : Toks{-1, -1, -1};
+        const TokXY nxy = c + 1 <= c_last ? load_xy(a, b1, nx) : TokXY{};
+        const Geo<MTILES> geo = make_geo<MTILES>(cur, cxy, rows.rt, lane, N);
+        Rows<NK> nrows = rows;
+        for (; h < hend; ++h) {
+            cp_async_wait<0>();
+            __syncwarp();
+            const uint32_t sb = wb + st * T::STAGE, nb = wb + (st ^ 1) * T::STAGE;
+            if (h + 1 < hend) {
+                gather_cluster<MT, BWD>(a, b, h + 1, rows, nb, lane);
+                cp_async_commit();
+            } else if (!lastc) {
+                nrows = cluster_rows<NK>(nx, lane, N);
+                gather_cluster<MT, BWD>(a, b1, 0, nrows, nb, lane);
+                cp_async_commit();
+            }
+            if (BWD)
+                query_item<MTILES>(a, b, g, h, sb, reinterpret_cast<const float*>(wsm + st * T::STAGE + T::LSE), lo,
+                                   geo, lane);
+            else
+                fwd_item<MTILES>(a, b, h, sb, lo, geo, lane);
+            __syncwarp();
+            st ^= 1;
+        }
+        if (lastc) break;
+        ++c;
+        h = 0;
+        b = b1;
+        g = g1;
+        b1 = b2;
+        g1 = g2;
+        next_cluster(b2, g2, G);
+        cur = nx;
+        nx = nn;
+        cxy = nxy;
+        rows = nrows;
+    }
+    cp_async_wait<0>();
 }
 
 // ------------------------------------------------------ block-wide int scan
@@ -422,9 +626,14 @@ __device__ int block_scan_excl(int* data, int n, int* scratch) {
     return total;
 }
 
+// ------------------------------------------------------------------ prep
+
 // Reverse neighbourhood index of image b: for each key cluster h, the query clusters g
-// whose table lists h, ascending in g.  Runs in one CTA; dynamic smem >= 4*(G+1)+160 B.
-__device__ void build_reverse_index(const AttnArgs& a, int b, uint8_t* smem) {
+// whose table lists h, ascending in g, and the 8 tokens of each listed cluster (made
+// valid).  One CTA per image; dynamic smem >= 4 * (G + 1) + 160 bytes.
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int b = blockIdx.x;
     const int tid = threadIdx.x, nt = blockDim.x;
     const int N = a.N, G = a.G, R = a.R, M = a.M;
     int* cnt = reinterpret_cast<int*>(smem);
@@ -434,6 +643,7 @@ __device__ void build_reverse_index(const AttnArgs& a, int b, uint8_t* smem) {
     const int32_t* nb = a.nbr + static_cast<size_t>(b) * G * M;
     int32_t* off = a.rev_off + static_cast<size_t>(b) * (G + 1);
     int32_t* lst = a.rev_list + static_cast<size_t>(b) * G * R;
+    int32_t* rtok = a.rev_tok + static_cast<size_t>(b) * G * R * 8;
     for (int i = tid; i < N; i += nt) tc[i] = -1;
     for (int i = tid; i <= G; i += nt) cnt[i] = 0;
     __syncthreads();
@@ -471,627 +681,411 @@ __device__ void build_reverse_index(const AttnArgs& a, int b, uint8_t* smem) {
             lst[j + 1] = v;
         }
     }
-}
-
-// ------------------------------------------------------ backward, key-major
-
-// Key-major backward of one (image, key cluster, head) by one warp, loading the query
-// rows of each pair of listed query clusters straight into its own 3.5 KB of shared memory.
-__device__ void key_major_direct(const AttnArgs& a, int b, int kc, int h, int lane, uint8_t* w) {
-    const int H = a.H;
-    const size_t tok0 = static_cast<size_t>(b) * a.N;
-    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + tok0;
-
-    uint8_t* ks = w;            // 8 rows
-    uint8_t* vs = w + 512;      // 8 rows
-    uint8_t* qs = w + 1024;     // 16 rows
-    uint8_t* dos = w + 2048;    // 16 rows
-    int* kid = reinterpret_cast<int*>(w + 3072);
-    float2* kxy = reinterpret_cast<float2*>(w + 3104);
-    int* qid = reinterpret_cast<int*>(w + 3168);
-    float2* qxy = reinterpret_cast<float2*>(w + 3232);
-    float* qL = reinterpret_cast<float*>(w + 3360);
-    float* qD = reinterpret_cast<float*>(w + 3424);
-
-    if (lane < 8) {
-        int id = a.clusters[(static_cast<size_t>(b) * a.G + kc) * 8 + lane];
-        if (id < 0 || id >= a.N) id = -1;
-        kid[lane] = id;
-        kxy[lane] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
-    }
-    __syncwarp();
-    {
-        const int row = lane >> 2, ch = lane & 3;
-        const int id = kid[row];
-        const size_t off = ((tok0 + (id >= 0 ? id : 0)) * H + h) * 32 + ch * 8;
-        cp_async16(smem_addr(ks) + tile64_off(row, ch), a.k + off, id >= 0);
-        cp_async16(smem_addr(vs) + tile64_off(row, ch), a.v + off, id >= 0);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncwarp();
-    uint32_t kf0, kf1, kf2, kf3, vf0, vf1, vf2, vf3;
-    ldsm_x4(smem_addr(ks) + tile64_off(lane & 7, lane >> 3), kf0, kf1, kf2, kf3);
-    ldsm_x4(smem_addr(vs) + tile64_off(lane & 7, lane >> 3), vf0, vf1, vf2, vf3);
-
-    const int gq = lane >> 2, tq = lane & 3;
-    const float sc = a.scale * kLog2e;
-    const float ba = a.bias[3 * h] * kLog2e, bb = a.bias[3 * h + 1] * kLog2e,
-                bc = a.bias[3 * h + 2] * kLog2e;
-    const float2 kp0 = kxy[2 * tq], kp1 = kxy[2 * tq + 1];
-    const int lo = a.rev_off[static_cast<size_t>(b) * (a.G + 1) + kc];
-    const int hi_ = a.rev_off[static_cast<size_t>(b) * (a.G + 1) + kc + 1];
-    const int32_t* lst = a.rev_list + static_cast<size_t>(b) * a.G * a.R;
-    float dk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    float dv[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    const int mi = lane >> 3;
-
-    for (int e = lo; e < hi_; e += 2) {
-        if (lane < 16) {
-            const int gg = (lane < 8) ? lst[e] : (e + 1 < hi_ ? lst[e + 1] : -1);
-            int id = gg >= 0 ? a.clusters[(static_cast<size_t>(b) * a.G + gg) * 8 + (lane & 7)] : -1;
-            if (id < 0 || id >= a.N) id = -1;
-            qid[lane] = id;
-            qxy[lane] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
-            float L = id >= 0 ? a.lse_in[(tok0 + id) * H + h] * kLog2e : INFINITY;
-            if (L == -INFINITY) L = INFINITY;
-            qL[lane] = L;
-            qD[lane] = id >= 0 ? a.delta[(tok0 + id) * H + h] : 0.f;
-        }
-        __syncwarp();
-#pragma unroll
-        for (int c = lane; c < 64; c += 32) {
-            const int row = c >> 2, ch = c & 3;
-            const int id = qid[row];
-            const size_t off = ((tok0 + (id >= 0 ? id : 0)) * H + h) * 32 + ch * 8;
-            cp_async16(smem_addr(qs) + tile64_off(row, ch), a.q + off, id >= 0);
-            cp_async16(smem_addr(dos) + tile64_off(row, ch), a.dout + off, id >= 0);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-        __syncwarp();
-
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, pacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            const int row = (lane & 7) + 8 * (mi & 1);
-            const int ch = 2 * kk + (mi >> 1);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(smem_addr(qs) + tile64_off(row, ch), a0, a1, a2, a3);
-            mma_bf16(sacc, a0, a1, a2, a3, kk ? kf2 : kf0, kk ? kf3 : kf1);
-            ldsm_x4(smem_addr(dos) + tile64_off(row, ch), a0, a1, a2, a3);
-            mma_bf16(pacc, a0, a1, a2, a3, kk ? vf2 : vf0, kk ? vf3 : vf1);
-        }
-        // element j: query row gq + 8*(j>>1), key 2*tq + (j&1)
-        float p[4], ds[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int qr = gq + 8 * (j >> 1);
-            const float2 qp = qxy[qr];
-            const float2 kp = (j & 1) ? kp1 : kp0;
-            const float dx = kp.x - qp.x, dy = kp.y - qp.y;
-            const float lg = sacc[j] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
-            p[j] = exp2f(lg - qL[qr]);
-            ds[j] = p[j] * (pacc[j] - qD[qr]);
-        }
-        const uint32_t pb0 = movm_t(pack_bf16(p[0], p[1]));
-        const uint32_t pb1 = movm_t(pack_bf16(p[2], p[3]));
-        const uint32_t sb0 = movm_t(pack_bf16(ds[0], ds[1]));
-        const uint32_t sb1 = movm_t(pack_bf16(ds[2], ds[3]));
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            const int row = (lane & 7) + 8 * (mi >> 1);
-            const int ch = 2 * m + (mi & 1);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(smem_addr(dos) + tile64_off(row, ch), a0, a1, a2, a3);
-            mma_bf16(dv[m], a0, a1, a2, a3, pb0, pb1);
-            ldsm_x4_t(smem_addr(qs) + tile64_off(row, ch), a0, a1, a2, a3);
-            mma_bf16(dk[m], a0, a1, a2, a3, sb0, sb1);
-        }
-        __syncwarp();
-    }
-    store_rows_t1(dk, a.scale, qs, kid, tok0, H, h, a.dk, lane);
-    store_rows_t1(dv, 1.f, qs, kid, tok0, H, h, a.dv, lane);
-}
-
-
-// ------------------------------------------------ backward with neighbourhood unions
-
-
-// Query-major pass with neighbourhood unions (same CTA shape as the forward), plus one
-// extra CTA column that builds each image's reverse neighbourhood index.
-template <int MTILES>
-__global__ void __launch_bounds__(kUThreads) attn_bwd_query_union_kernel(const AttnArgs a, int ncg) {
-    constexpr int MT = 16 * MTILES;
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int cg = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-    if (cg >= ncg) {
-        if (hg == 0) build_reverse_index(a, b, smem);
-        return;
-    }
-    const int R = a.R;
-    const UnionLayout L = union_layout(R, MT);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int G = a.G, N = a.N, H = a.H;
-    const int g0 = cg * kUC;
-    const int ZR = kUC * R * 8;
-    uint8_t* ks = smem + L.ks;
-    uint8_t* vs = smem + L.vs;
-    uint8_t* qs = smem + L.qs;
-    uint8_t* dos = smem + L.stage;  // dO tile (kUC * 8 rows) in the staging area
-    uint8_t* stage = smem + L.total;  // per-warp output staging after the layout
-    const size_t tok0 = static_cast<size_t>(b) * N;
-    const int nU = union_setup(a, b, g0, MT, L, smem);
-    const int* utok = reinterpret_cast<const int*>(smem + L.utok);
-    const float2* uxy = reinterpret_cast<const float2*>(smem + L.uxy);
-    const int* qtok = reinterpret_cast<const int*>(smem + L.qtok);
-    const float2* qxy = reinterpret_cast<const float2*>(smem + L.qxy);
-    const int* krow = reinterpret_cast<const int*>(smem + L.krow);
-    const int hlo = hg * kUH;
-    {
-        // thread tid copies 16-byte chunk tid % 8 of rows tid / 8, tid / 8 + 32, ...
-        const int ch = tid & 7;
-        const bool ch_ok = hlo + (ch >> 2) < H;
-        const size_t cbase = (tok0 * H + hlo) * 32 + ch * 8;
-        const size_t tstride = static_cast<size_t>(H) * 32;
-        const int urows = nU * 8;
-        for (int row = tid >> 3; row < urows + 8; row += kUThreads / 8) {
-            const int t = row < urows ? utok[row] : -1;
-            const bool ok = t >= 0 && ch_ok;
-            const int drow = row < urows ? row : ZR + (row - urows);
-            const size_t off = ok ? cbase + t * tstride : 0;
-            cp_async16(smem_addr(ks) + urow_off(drow, ch), a.k + off, ok);
-            cp_async16(smem_addr(vs) + urow_off(drow, ch), a.v + off, ok);
-        }
-        for (int row = tid >> 3; row < kUC * 8; row += kUThreads / 8) {
-            const int t = qtok[row];
-            const bool ok = t >= 0 && ch_ok;
-            const size_t off = ok ? cbase + t * tstride : 0;
-            cp_async16(smem_addr(qs) + urow_off(row, ch), a.q + off, ok);
-            cp_async16(smem_addr(dos) + urow_off(row, ch), a.dout + off, ok);
-        }
-    }
-    union_coords_async(a, b, nU, L, smem);
-    cp_async_commit();
-    cp_async_wait<0>();
     __syncthreads();
+    for (int i = tid; i < total * 8; i += nt) rtok[i] = valid_tok(cl[lst[i >> 3] * 8 + (i & 7)], N);
+}
 
-    const int cw = warp / kUH, hw = warp % kUH;
-    const int g = g0 + cw, h = hlo + hw;
-    if (g >= G || h >= H) return;
-    const int gq = lane >> 2, tq = lane & 3, mi = lane >> 3;
-    const int* kr = krow + cw * MT;
-    // row 0 of each neighbourhood block this lane addresses: (mi & 1) picks the block of
-    // the S / dQ operands, (mi >> 1) the block of the transposed V / K operands
-    int base_s[MTILES], base_t[MTILES];
+// ------------------------------------------------------------------ key pass
+
+// Per-warp stage of the key pass: the key cluster's own K and V rows, the chunk's Q and dO
+// rows (kChunk listed clusters), and the chunk rows' parameters (lse and Delta land in .x
+// and .y and become (X, Y, L', Delta) in place).
+struct KTile {
+    static constexpr int K = 0;
+    static constexpr int V = 8 * kRowB;
+    static constexpr int Q = 16 * kRowB;
+    static constexpr int DO = Q + 8 * kChunk * kRowB;
+    static constexpr int PRM = DO + 8 * kChunk * kRowB;
+    static constexpr int STAGE = PRM + 16 * 8 * kChunk;
+    static constexpr int WARP = 2 * STAGE;
+};
+
+// One pair of query clusters (16 queries) against the warp's 8 keys.  rb1 / rb2: rows of
+// the two query blocks in the Q / dO tiles at qb / dob; p1 / p2: parameter rows
+// (X, Y, L', Delta) of the lane's queries gq in each block.
+__device__ __forceinline__ void key_pair(uint32_t qb, uint32_t dob, int rb1, int rb2, float4 p1, float4 p2,
+                                         const uint32_t (&kf)[4], const uint32_t (&vf)[4], const float (&kx)[2],
+                                         const float (&ky)[2], const float (&u)[2], float sc, float (&dk)[2][4],
+                                         float (&dv)[2][4]) {
+    const int lane = threadIdx.x & 31, mi = lane >> 3;
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f}, pacc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int rs = ((mi & 1) ? rb2 : rb1) + (lane & 7);
 #pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-        const int s0 = 2 * i + (mi & 1), s1 = 2 * i + (mi >> 1);
-        const int r0 = (s0 * 8 < a.M) ? kr[s0 * 8] : -1;
-        const int r1 = (s1 * 8 < a.M) ? kr[s1 * 8] : -1;
-        base_s[i] = r0 >= 0 ? r0 : ZR;
-        base_t[i] = r1 >= 0 ? r1 : ZR;
+    for (int kk = 0; kk < 2; ++kk) {
+        const uint32_t off = tile64_off(rs, 2 * kk + (mi >> 1));
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4(qb + off, r0, r1, r2, r3);
+        mma_bf16(sacc, r0, r1, r2, r3, kf[2 * kk], kf[2 * kk + 1]);
+        ldsm_x4(dob + off, r0, r1, r2, r3);
+        mma_bf16(pacc, r0, r1, r2, r3, vf[2 * kk], vf[2 * kk + 1]);
     }
-    const int q0 = qtok[cw * 8 + 2 * tq], q1 = qtok[cw * 8 + 2 * tq + 1];
-    float L0 = q0 >= 0 ? a.lse_in[(tok0 + q0) * H + h] * kLog2e : INFINITY;
-    float L1 = q1 >= 0 ? a.lse_in[(tok0 + q1) * H + h] * kLog2e : INFINITY;
-    if (L0 == -INFINITY) L0 = INFINITY;
-    if (L1 == -INFINITY) L1 = INFINITY;
-    uint32_t qf0, qf1, qf2, qf3, df0, df1, df2, df3;
-    ldsm_x4(smem_addr(qs) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), qf0, qf1, qf2, qf3);
-    ldsm_x4(smem_addr(dos) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), df0, df1, df2, df3);
-    float sacc[MTILES][4], dp[MTILES][4];
+    // element j: query row gq of block (j >> 1), key 2 tq + (j & 1)
+    float p[4], ds[4];
 #pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-        sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
-        dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            const int row = base_s[i] + (lane & 7);
-            const uint32_t off = urow_off(row, hw * 4 + 2 * kk + (mi >> 1));
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(smem_addr(ks) + off, a0, a1, a2, a3);
-            mma_bf16(sacc[i], a0, a1, a2, a3, kk ? qf2 : qf0, kk ? qf3 : qf1);
-            ldsm_x4(smem_addr(vs) + off, a0, a1, a2, a3);
-            mma_bf16(dp[i], a0, a1, a2, a3, kk ? df2 : df0, kk ? df3 : df1);
-        }
+    for (int j = 0; j < 4; ++j) {
+        const float4 pr = (j >> 1) ? p2 : p1;
+        const int c = j & 1;
+        const float t = fmaf(sacc[j], sc, fmaf(pr.x, kx[c], fmaf(pr.y, ky[c], u[c])));
+        p[j] = sfu_ex2(t - pr.z);
+        ds[j] = p[j] * (pacc[j] - pr.w);
     }
-    const float sc = a.scale * kLog2e;
-    const float ba = a.bias[3 * h] * kLog2e, bb = a.bias[3 * h + 1] * kLog2e,
-                bc = a.bias[3 * h + 2] * kLog2e;
-    const float2 qa = qxy[cw * 8 + 2 * tq], qb = qxy[cw * 8 + 2 * tq + 1];
-    float pd0 = 0.f, pd1 = 0.f;
-#pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-            const int row = kr[16 * i + gq + 8 * hi];
-            const bool kv = row >= 0 && utok[row] >= 0;
-            const float2 kp = kv ? uxy[row] : make_float2(0.f, 0.f);
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const float2 qp = qq ? qb : qa;
-                const float dx = kp.x - qp.x, dy = kp.y - qp.y;
-                const int j = 2 * hi + qq;
-                const float lg = sacc[i][j] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
-                const float p = kv ? exp2f(lg - (qq ? L1 : L0)) : 0.f;
-                sacc[i][j] = p;
-                if (qq) pd1 += p * dp[i][j];
-                else pd0 += p * dp[i][j];
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-        pd0 += __shfl_xor_sync(0xffffffffu, pd0, o);
-        pd1 += __shfl_xor_sync(0xffffffffu, pd1, o);
-    }
-    if (gq == 0) {
-        if (q0 >= 0) a.delta[(tok0 + q0) * H + h] = pd0;
-        if (q1 >= 0) a.delta[(tok0 + q1) * H + h] = pd1;
-    }
-    float ga = 0.f, gb = 0.f, gc = 0.f;
-    uint32_t db[MTILES][2];
-#pragma unroll
-    for (int i = 0; i < MTILES; ++i) {
-        float ds[4];
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-            const int row = kr[16 * i + gq + 8 * hi];
-            const bool kv = row >= 0 && utok[row] >= 0;
-            const float2 kp = kv ? uxy[row] : make_float2(0.f, 0.f);
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const float2 qp = qq ? qb : qa;
-                const float dx = kp.x - qp.x, dy = kp.y - qp.y;
-                const int j = 2 * hi + qq;
-                const float v = sacc[i][j] * (dp[i][j] - (qq ? pd1 : pd0));
-                ds[j] = v;
-                ga += v * dx;
-                gb += v * dy;
-                gc += v * (dx * dx + dy * dy);
-            }
-        }
-        db[i][0] = movm_t(pack_bf16(ds[0], ds[1]));
-        db[i][1] = movm_t(pack_bf16(ds[2], ds[3]));
-    }
-    ga = warp_sum(ga);
-    gb = warp_sum(gb);
-    gc = warp_sum(gc);
-    if (lane == 0) {
-        float* part = a.dbias_part + ((static_cast<size_t>(b) * G + g) * H + h) * 3;
-        part[0] = ga;
-        part[1] = gb;
-        part[2] = -gc;
-    }
-    float dqacc[2][4];
+    const uint32_t pb0 = movm_t(pack_bf16(p[0], p[1]));
+    const uint32_t pb1 = movm_t(pack_bf16(p[2], p[3]));
+    const uint32_t sb0 = movm_t(pack_bf16(ds[0], ds[1]));
+    const uint32_t sb1 = movm_t(pack_bf16(ds[2], ds[3]));
+    const int rt = ((mi >> 1) ? rb2 : rb1) + (lane & 7);
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-        dqacc[m][0] = dqacc[m][1] = dqacc[m][2] = dqacc[m][3] = 0.f;
+        const uint32_t off = tile64_off(rt, 2 * m + (mi & 1));
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4_t(dob + off, r0, r1, r2, r3);
+        mma_bf16(dv[m], r0, r1, r2, r3, pb0, pb1);
+        ldsm_x4_t(qb + off, r0, r1, r2, r3);
+        mma_bf16(dk[m], r0, r1, r2, r3, sb0, sb1);
+    }
+}
+
+// Row parameters of a query token for head h: X = 2 c x, Y = 2 c y (log2 units, local
+// coordinates), L' = lse log2e - w2 (P = exp2(t - L')), Delta.
+__device__ __forceinline__ float4 row_params(float x, float y, bool valid, float lse, float delta, float a2,
+                                             float b2, float c2) {
+    const bool ok = valid && lse != -INFINITY;
+    float4 r;
+    r.x = ok ? 2.f * c2 * x : 0.f;
+    r.y = ok ? 2.f * c2 * y : 0.f;
+    r.z = ok ? fmaf(lse, kLog2e, fmaf(a2, x, fmaf(b2, y, c2 * fmaf(x, x, y * y)))) : INFINITY;
+    r.w = ok ? delta : 0.f;
+    return r;
+}
+
+// Store one warp's dK^T / dV^T accumulators (dims x keys) as rows of dK / dV.
+__device__ __forceinline__ void store_key_rows(const float (&acc)[2][4], float scl, int tok, size_t tok0,
+                                               int H, int h, bf16* dst_base) {
+    const int lane = threadIdx.x & 31, tq = lane & 3;
+    const uint32_t w0 = movm_t(pack_bf16(acc[0][0] * scl, acc[0][1] * scl));
+    const uint32_t w1 = movm_t(pack_bf16(acc[0][2] * scl, acc[0][3] * scl));
+    const uint32_t w2 = movm_t(pack_bf16(acc[1][0] * scl, acc[1][1] * scl));
+    const uint32_t w3 = movm_t(pack_bf16(acc[1][2] * scl, acc[1][3] * scl));
+    if (tok >= 0) {
+        uint32_t* dst = reinterpret_cast<uint32_t*>(dst_base + ((tok0 + tok) * H + h) * 32) + tq;
+        dst[0] = w0;
+        dst[4] = w1;
+        dst[8] = w2;
+        dst[12] = w3;
+    }
+}
+
+// A key-pass item: (image b, key cluster kc, head h, chunk ch) over the list entries
+// [e0, e0 + E) of kc (image-local).  It carries what the gather needs: the tokens of the
+// lane's gather rows (chunk rows gq + 8 k), of the lane's parameter rows lane and lane + 32,
+// of the own cluster row (lanes < 8), and the coordinates of the last two groups.
+struct KItem {
+    int b, kc, h, ch, nch, e0, E;
+    int qt[kChunk];
+    int pa, pb, kt;
+    float2 pxa, pxb, kxy;
+};
+
+// Tokens of an item (coordinates separately, an item later).
+__device__ __forceinline__ void kitem_tokens(const AttnArgs& a, KItem& it, int lane) {
+    const int G = a.G, N = a.N;
+    const int32_t* rtok = a.rev_tok + static_cast<size_t>(it.b) * G * a.R * 8;
+    const size_t base = (static_cast<size_t>(it.e0) + static_cast<size_t>(kChunk) * it.ch) * 8;
+    const int rem = (it.E - kChunk * it.ch) * 8;
+    const int n = rem > 8 * kChunk ? 8 * kChunk : rem;
+    const int gq = lane >> 2;
 #pragma unroll
-        for (int i = 0; i < MTILES; ++i) {
-            const int row = base_t[i] + (lane & 7);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(smem_addr(ks) + urow_off(row, hw * 4 + 2 * m + (mi & 1)), a0, a1, a2, a3);
-            mma_bf16(dqacc[m], a0, a1, a2, a3, db[i][0], db[i][1]);
+    for (int k = 0; k < kChunk; ++k) it.qt[k] = gq + 8 * k < n ? __ldg(rtok + base + gq + 8 * k) : -1;
+    it.pa = lane < n ? __ldg(rtok + base + lane) : -1;
+    it.pb = lane + 32 < n ? __ldg(rtok + base + lane + 32) : -1;
+    it.kt = lane < 8 ? valid_tok(__ldg(a.clusters + (static_cast<size_t>(it.b) * G + it.kc) * 8 + lane), N) : -1;
+}
+__device__ __forceinline__ void kitem_coords(const AttnArgs& a, KItem& it) {
+    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(it.b) * a.N;
+    it.pxa = it.pa >= 0 ? __ldg(xyb + it.pa) : make_float2(0.f, 0.f);
+    it.pxb = it.pb >= 0 ? __ldg(xyb + it.pb) : make_float2(0.f, 0.f);
+    it.kxy = it.kt >= 0 ? __ldg(xyb + it.kt) : make_float2(0.f, 0.f);
+}
+
+__device__ __forceinline__ void kitem_gather(const AttnArgs& a, const KItem& it, uint32_t sb, int lane) {
+    const uint32_t lo = gather_lane_off(lane);
+    const size_t rowel = static_cast<size_t>(a.H) * 32;
+    const size_t tok0 = static_cast<size_t>(it.b) * a.N;
+    const size_t hoff = static_cast<size_t>(it.h) * 32 + (lane & 3) * 8;
+    const int own = __shfl_sync(0xffffffffu, it.kt, lane >> 2);
+    {
+        const size_t src = own >= 0 ? (tok0 + own) * rowel + hoff : 0;
+        cp_async16(sb + KTile::K + lo, a.k + src, own >= 0);
+        cp_async16(sb + KTile::V + lo, a.v + src, own >= 0);
+    }
+#pragma unroll
+    for (int k = 0; k < kChunk; ++k) {
+        const int t = it.qt[k];
+        const size_t src = t >= 0 ? (tok0 + t) * rowel + hoff : 0;
+        cp_async16(sb + KTile::Q + 512 * k + lo, a.q + src, t >= 0);
+        cp_async16(sb + KTile::DO + 512 * k + lo, a.dout + src, t >= 0);
+    }
+    const uint32_t pr = sb + KTile::PRM;
+    const size_t sa = it.pa >= 0 ? (tok0 + it.pa) * a.H + it.h : 0;
+    cp_async4(pr + 16 * lane, a.lse_in + sa, it.pa >= 0);
+    cp_async4(pr + 16 * lane + 4, a.delta + sa, it.pa >= 0);
+    if (lane + 32 < 8 * kChunk) {
+        const size_t s2 = it.pb >= 0 ? (tok0 + it.pb) * a.H + it.h : 0;
+        cp_async4(pr + 16 * (lane + 32), a.lse_in + s2, it.pb >= 0);
+        cp_async4(pr + 16 * (lane + 32) + 4, a.delta + s2, it.pb >= 0);
+    }
+}
+
+// Advance `it` to the next item of the warp's units (b, kc, h) (cluster-major), whose last
+// is unit u_end - 1; returns false past the end.
+__device__ __forceinline__ bool kitem_next(const AttnArgs& a, KItem& it, long long& unit, long long u_end) {
+    if (it.ch + 1 < it.nch) {
+        ++it.ch;
+        return true;
+    }
+    if (unit + 1 >= u_end) return false;
+    ++unit;
+    it.ch = 0;
+    if (++it.h == a.H) {
+        it.h = 0;
+        if (++it.kc == a.G) {
+            it.kc = 0;
+            ++it.b;
+        }
+        const int32_t* roff = a.rev_off + static_cast<size_t>(it.b) * (a.G + 1);
+        it.e0 = __ldg(roff + it.kc);
+        it.E = __ldg(roff + it.kc + 1) - it.e0;
+        it.nch = it.E > 0 ? (it.E + kChunk - 1) / kChunk : 1;
+    }
+    return true;
+}
+
+// One key-pass item: row parameters in place, then the chunk's pairs; the accumulators
+// carry over the chunks of a (key cluster, head) and are stored after its last chunk.
+__device__ __forceinline__ void key_item(const AttnArgs& a, const KItem& it, uint32_t sb, float4* prm,
+                                         float (&dk)[2][4], float (&dv)[2][4], int lane) {
+    const int gq = lane >> 2, tq = lane & 3, mi = lane >> 3;
+    const float a2 = __ldg(a.bias + 3 * it.h) * kLog2e, b2 = __ldg(a.bias + 3 * it.h + 1) * kLog2e,
+                c2 = __ldg(a.bias + 3 * it.h + 2) * kLog2e;
+    const float sc = a.scale * kLog2e;
+    // local origin: the key cluster's first slot
+    const float2 org = sh2(it.kxy, 0);
+    {
+        const float4 r = prm[lane];
+        prm[lane] = row_params(it.pxa.x - org.x, it.pxa.y - org.y, it.pa >= 0, r.x, r.y, a2, b2, c2);
+        if (lane + 32 < 8 * kChunk) {
+            const float4 r2 = prm[lane + 32];
+            prm[lane + 32] = row_params(it.pxb.x - org.x, it.pxb.y - org.y, it.pb >= 0, r2.x, r2.y, a2, b2, c2);
         }
     }
-    store_rows_t(dqacc, a.scale, a.scale, stage + warp * 512, qtok + cw * 8, tok0, H, h, a.dq, lane);
+    __syncwarp();
+    uint32_t kf[4], vf[4];
+    const uint32_t oq = tile64_off(lane & 7, mi);
+    ldsm_x4(sb + KTile::K + oq, kf[0], kf[1], kf[2], kf[3]);
+    ldsm_x4(sb + KTile::V + oq, vf[0], vf[1], vf[2], vf[3]);
+    float kx[2], ky[2], u[2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        const float2 p = sh2(it.kxy, 2 * tq + c);
+        const bool ok = __shfl_sync(0xffffffffu, it.kt, 2 * tq + c) >= 0;
+        kx[c] = ok ? p.x - org.x : 0.f;
+        ky[c] = ok ? p.y - org.y : 0.f;
+        u[c] = ok ? fmaf(a2, kx[c], fmaf(b2, ky[c], -c2 * fmaf(kx[c], kx[c], ky[c] * ky[c]))) : -INFINITY;
+    }
+    const int nq = it.E - kChunk * it.ch;  // listed clusters from this chunk on
+    const int n = nq < kChunk ? nq : kChunk;
+    for (int e = 0; e < n; e += 2) {
+        const bool two = e + 1 < n;
+        const float4 p1 = prm[8 * e + gq];
+        // an absent second block reads the first block's rows with P = 0
+        const float4 p2 = two ? prm[8 * (e + 1) + gq] : make_float4(0.f, 0.f, INFINITY, 0.f);
+        key_pair(sb + KTile::Q, sb + KTile::DO, 8 * e, two ? 8 * (e + 1) : 8 * e, p1, p2, kf, vf, kx, ky, u, sc, dk,
+                 dv);
+    }
+    if (it.ch + 1 == it.nch) {
+        const int own = __shfl_sync(0xffffffffu, it.kt, gq);
+        const size_t tok0 = static_cast<size_t>(it.b) * a.N;
+        store_key_rows(dk, a.scale, own, tok0, a.H, it.h, a.dk);
+        store_key_rows(dv, 1.f, own, tok0, a.H, it.h, a.dv);
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dk[m][j] = dv[m][j] = 0.f;
+    }
 }
 
-// Key-major pass with query-cluster unions.  CTA = (kUC consecutive key clusters, kUH
-// heads, image).  The reverse lists of its key clusters are concatenated and their query
-// clusters de-duplicated; Q and dO rows of the union (plus lse and Delta) are gathered
-// once and every warp walks its own list two query clusters at a time out of the union
-// tile.  A group whose lists exceed the tile falls back to per-warp direct loading.
-constexpr int kKQ = 24;       // union query clusters held per CTA
-constexpr int kKEnt = 64;     // list entries per CTA
-struct KeyLayout {
-    int qs, dos, ks, vs, stage, ent, eu, es, qtok, qxy, qL, qD, ktok, kxy, misc, total;
-};
-__host__ __device__ __forceinline__ KeyLayout key_layout() {
-    KeyLayout L;
-    const int rows = kKQ * 8 + 8;
-    int o = 0;
-    L.qs = o; o += rows * kURow;
-    L.dos = o; o += rows * kURow;
-    L.ks = o; o += kUC * 8 * kURow;
-    L.vs = o; o += kUC * 8 * kURow;
-    L.stage = o; o += kUWarps * 512;
-    L.ent = o; o += 4 * kKEnt;
-    L.eu = o; o += 4 * kKEnt;
-    L.es = o; o += 4 * (kUC + 1 + kKEnt);  // [kUC] count, then first-occurrence flags
-    o = (o + 15) & ~15;
-    L.qtok = o; o += 4 * rows;
-    L.qxy = o; o += 8 * rows;
-    L.qL = o; o += 4 * rows * kUH;
-    L.qD = o; o += 4 * rows * kUH;
-    L.ktok = o; o += 4 * kUC * 8;
-    L.kxy = o; o += 8 * kUC * 8;
-    L.misc = o; o += 16;
-    L.total = (o + 15) & ~15;
-    return L;
+// One warp's units [u0, u1) of the key pass (unit = (image, key cluster, head)).  The
+// item cursor runs two items ahead: tokens two items early, coordinates and the gather one.
+__device__ __forceinline__ void key_units(const AttnArgs& a, long long u0, long long u1, uint8_t* wsm) {
+    const int lane = threadIdx.x & 31;
+    const int H = a.H, G = a.G;
+    const uint32_t wb = smem_addr(wsm);
+    KItem cur;
+    {
+        const long long c = u0 / H;
+        cur.h = static_cast<int>(u0 - c * H);
+        cur.b = static_cast<int>(c / G);
+        cur.kc = static_cast<int>(c - static_cast<long long>(cur.b) * G);
+        cur.ch = 0;
+        const int32_t* roff = a.rev_off + static_cast<size_t>(cur.b) * (G + 1);
+        cur.e0 = __ldg(roff + cur.kc);
+        cur.E = __ldg(roff + cur.kc + 1) - cur.e0;
+        cur.nch = cur.E > 0 ? (cur.E + kChunk - 1) / kChunk : 1;
+    }
+    kitem_tokens(a, cur, lane);
+    kitem_coords(a, cur);
+    KItem nx = cur;
+    long long unx = u0;
+    bool has_nx = kitem_next(a, nx, unx, u1);
+    if (has_nx) kitem_tokens(a, nx, lane);
+    int st = 0;
+    kitem_gather(a, cur, wb, lane);
+    cp_async_commit();
+    float dk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float dv[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (;;) {
+        KItem nn = nx;
+        long long unn = unx;
+        const bool has_nn = has_nx && kitem_next(a, nn, unn, u1);
+        if (has_nn) kitem_tokens(a, nn, lane);
+        if (has_nx) kitem_coords(a, nx);
+        cp_async_wait<0>();
+        __syncwarp();
+        if (has_nx) {
+            kitem_gather(a, nx, wb + (st ^ 1) * KTile::STAGE, lane);
+            cp_async_commit();
+        }
+        key_item(a, cur, wb + st * KTile::STAGE, reinterpret_cast<float4*>(wsm + st * KTile::STAGE + KTile::PRM), dk,
+                 dv, lane);
+        __syncwarp();
+        st ^= 1;
+        if (!has_nx) break;
+        cur = nx;
+        nx = nn;
+        unx = unn;
+        has_nx = has_nn;
+    }
+    cp_async_wait<0>();
 }
 
-__global__ void __launch_bounds__(kUThreads) attn_bwd_key_union_kernel(const AttnArgs a, int ncg) {
+// ------------------------------------------------------------- entry kernels
+
+// Resident warps per SM the kernels are built for: the forward 16 (4 CTAs of 4 warps, up
+// to 128 registers), the query pass's larger stage 12, the key pass 16.
+template <int MTILES>
+__global__ void __launch_bounds__(kThreads, MTILES <= 3 ? 4 : 2) attn_fwd_kernel(const AttnArgs a) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const long long PW = static_cast<long long>(gridDim.x) * kWarps;
+    const long long gw = static_cast<long long>(blockIdx.x) * kWarps + warp;
+    const long long W = static_cast<long long>(a.B) * a.G * a.H;
+    const long long i0 = gw * W / PW, i1 = (gw + 1) * W / PW;
+    if (i0 >= i1) return;
+    cluster_items<MTILES, false>(a, i0, i1, smem + warp * QTile<16 * MTILES, false>::WARP);
+}
+
+template <int MTILES>
+__global__ void __launch_bounds__(kThreads, MTILES <= 3 ? 3 : 2) attn_bwd_query_kernel(const AttnArgs a) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const long long PW = static_cast<long long>(gridDim.x) * kWarps;
+    const long long gw = static_cast<long long>(blockIdx.x) * kWarps + warp;
+    const long long W = static_cast<long long>(a.B) * a.G * a.H;
+    const long long i0 = gw * W / PW, i1 = (gw + 1) * W / PW;
+    if (i0 >= i1) return;
+    cluster_items<MTILES, true>(a, i0, i1, smem + warp * QTile<16 * MTILES, true>::WARP);
+}
+
+__global__ void __launch_bounds__(kThreads, 4) attn_bwd_key_kernel(const AttnArgs a, int P) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int cg = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-    const int G = a.G, N = a.N, H = a.H;
-    if (cg >= ncg) {
+    if (static_cast<int>(blockIdx.x) >= P) {
         // bias-gradient reduction: one CTA per (head, coefficient), fixed order
-        const int hj = cg - ncg;
-        if (hg != 0 || b != 0 || hj >= 3 * H) return;
+        const int hj = blockIdx.x - P;
         const int hh = hj / 3, j = hj % 3;
-        const int n = a.B * G;
+        const int n = a.B * a.G;
         float acc = 0.f;
 #pragma unroll 4
-        for (int i = tid; i < n; i += kUThreads) acc += a.dbias_part[(static_cast<size_t>(i) * H + hh) * 3 + j];
+        for (int i = tid; i < n; i += kThreads) acc += a.dbias_part[(static_cast<size_t>(i) * a.H + hh) * 3 + j];
         acc = warp_sum(acc);
         float* red = reinterpret_cast<float*>(smem);
         if (lane == 0) red[warp] = acc;
         __syncthreads();
         if (tid == 0) {
             float tot = 0.f;
-            for (int w = 0; w < kUWarps; ++w) tot += red[w];
+            for (int w = 0; w < kWarps; ++w) tot += red[w];
             a.dbias[hh * 3 + j] = tot;
         }
         return;
     }
-    const KeyLayout L = key_layout();
-    const int g0 = cg * kUC;
-    const int hlo = hg * kUH;
-    const int ZR = kKQ * 8;
-    const size_t tok0 = static_cast<size_t>(b) * N;
-    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + tok0;
-    int* ent = reinterpret_cast<int*>(smem + L.ent);
-    int* eu = reinterpret_cast<int*>(smem + L.eu);
-    int* es = reinterpret_cast<int*>(smem + L.es);
-    int* qtok = reinterpret_cast<int*>(smem + L.qtok);
-    float2* qxy = reinterpret_cast<float2*>(smem + L.qxy);
-    float* qL = reinterpret_cast<float*>(smem + L.qL);
-    float* qD = reinterpret_cast<float*>(smem + L.qD);
-    int* ktok = reinterpret_cast<int*>(smem + L.ktok);
-    float2* kxy = reinterpret_cast<float2*>(smem + L.kxy);
-    int* misc = reinterpret_cast<int*>(smem + L.misc);
-    const int32_t* roff = a.rev_off + static_cast<size_t>(b) * (G + 1);
-    const int32_t* rlist = a.rev_list + static_cast<size_t>(b) * G * a.R;
-    static_assert(kKEnt == 64 && kUC < 32, "warp 0 holds two list entries per lane");
-    if (warp == 0) {
-        // list offsets of the kUC key clusters (lane c), their prefix, then the entries
-        // (lanes hold entries lane and lane + 32) and their de-duplication in registers
-        int cnt = 0;
-        if (lane < kUC && g0 + lane < G) cnt = roff[g0 + lane + 1] - roff[g0 + lane];
-        const int start = (lane < kUC && g0 + lane < G) ? roff[g0 + lane] : 0;
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        const int ntot_w = __shfl_sync(0xffffffffu, incl, kUC - 1);
-        int e[2] = {-1, -1};
-        if (ntot_w <= kKEnt) {
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int i = x * 32 + lane;
-                int c = 0;  // the key cluster whose list holds entry i (all lanes shuffle)
-#pragma unroll
-                for (int cc = 1; cc < kUC; ++cc)
-                    c += (i >= __shfl_sync(0xffffffffu, incl - cnt, cc)) ? 1 : 0;
-                const int es_c = __shfl_sync(0xffffffffu, incl - cnt, c);
-                const int st_c = __shfl_sync(0xffffffffu, start, c);
-                if (i < ntot_w) e[x] = rlist[st_c + (i - es_c)];
-            }
-            // first occurrence of each entry's value (src = its index), in list order
-            int src[2] = {0x7fffffff, 0x7fffffff};
-#pragma unroll 8
-            for (int j = 0; j < kKEnt; ++j) {
-                const int vj = __shfl_sync(0xffffffffu, j < 32 ? e[0] : e[1], j & 31);
-#pragma unroll
-                for (int x = 0; x < 2; ++x)
-                    if (j < src[x] && vj == e[x] && j < ntot_w) src[x] = j;
-            }
-            int run = 0, ui[2];
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int i = x * 32 + lane;
-                const bool first = i < ntot_w && src[x] == i;
-                const unsigned m = __ballot_sync(0xffffffffu, first);
-                ui[x] = first ? run + __popc(m & ((1u << lane) - 1u)) : -1;
-                run += __popc(m);
-            }
-            // a repeated entry takes the union index of its first occurrence
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int i = x * 32 + lane;
-                const int s2 = (i < ntot_w) ? src[x] : i;
-                const int from0 = __shfl_sync(0xffffffffu, ui[0], s2 & 31);
-                const int from1 = __shfl_sync(0xffffffffu, ui[1], s2 & 31);
-                if (i < ntot_w) {
-                    ent[i] = e[x];
-                    eu[i] = (s2 < 32) ? from0 : from1;
-                    es[kUC + 1 + i] = (src[x] == i) ? 1 : 0;  // first occurrence
-                }
-            }
-            if (lane == 0) misc[0] = run;
-        }
-        if (lane <= kUC) es[lane] = incl - cnt;  // list start of key cluster lane; es[kUC] = total
-    } else {
-        for (int i = tid - 32; i < kUC * 8; i += kUThreads - 32) {
-            const int kc = g0 + (i >> 3);
-            int id = -1;
-            if (kc < G) {
-                id = a.clusters[(static_cast<size_t>(b) * G + kc) * 8 + (i & 7)];
-                if (id < 0 || id >= N) id = -1;
-            }
-            ktok[i] = id;
-            kxy[i] = id >= 0 ? xyb[id] : make_float2(0.f, 0.f);
-        }
-    }
-    __syncthreads();
-    const int ntot = es[kUC];
-    const bool fits = ntot <= kKEnt && misc[0] <= kKQ;
-    if (!fits) {
-        // fallback: every warp handles its (key cluster, head) with direct loads
-        const int cw = warp / kUH, hw = warp % kUH;
-        const int kc = g0 + cw, h = hlo + hw;
-        if (kc < G && h < H) key_major_direct(a, b, kc, h, lane, smem + warp * kBwdKWarpBytes);
-        return;
-    }
-    const int nU = misc[0];
-    // union query rows, their lse / Delta per head of the group
-    for (int i = tid; i < ntot * 8; i += kUThreads) {
-        const int e = i >> 3, sl = i & 7;
-        if (!es[kUC + 1 + e]) continue;  // a repeated list entry
-        const int row = eu[e] * 8 + sl;
-        int t = a.clusters[(static_cast<size_t>(b) * G + ent[e]) * 8 + sl];
-        if (t < 0 || t >= N) t = -1;
-        qtok[row] = t;
-        qxy[row] = t >= 0 ? xyb[t] : make_float2(0.f, 0.f);
-        for (int hw = 0; hw < kUH; ++hw) {
-            const int h = hlo + hw;
-            float Lv = INFINITY, Dv = 0.f;
-            if (t >= 0 && h < H) {
-                Lv = a.lse_in[(tok0 + t) * H + h] * kLog2e;
-                if (Lv == -INFINITY) Lv = INFINITY;
-                Dv = a.delta[(tok0 + t) * H + h];
-            }
-            qL[row * kUH + hw] = Lv;
-            qD[row * kUH + hw] = Dv;
-        }
-    }
-    for (int i = tid; i < 8 * kUH; i += kUThreads) {
-        qL[(ZR + (i / kUH)) * kUH + (i % kUH)] = INFINITY;
-        qD[(ZR + (i / kUH)) * kUH + (i % kUH)] = 0.f;
-    }
-    if (tid < 8) {
-        qtok[ZR + tid] = -1;
-        qxy[ZR + tid] = make_float2(0.f, 0.f);
-    }
-    __syncthreads();
-    uint8_t* qs = smem + L.qs;
-    uint8_t* dos = smem + L.dos;
-    uint8_t* ks = smem + L.ks;
-    uint8_t* vs = smem + L.vs;
-    {
-        // thread tid copies 16-byte chunk tid % 8 of rows tid / 8, tid / 8 + 32, ...
-        const int ch = tid & 7;
-        const bool ch_ok = hlo + (ch >> 2) < H;
-        const size_t cbase = (tok0 * H + hlo) * 32 + ch * 8;
-        const size_t tstride = static_cast<size_t>(H) * 32;
-        const int urows = nU * 8;
-        for (int row = tid >> 3; row < urows + 8; row += kUThreads / 8) {
-            const int drow = row < urows ? row : ZR + (row - urows);
-            const int t = qtok[drow];
-            const bool ok = t >= 0 && ch_ok;
-            const size_t off = ok ? cbase + t * tstride : 0;
-            cp_async16(smem_addr(qs) + urow_off(drow, ch), a.q + off, ok);
-            cp_async16(smem_addr(dos) + urow_off(drow, ch), a.dout + off, ok);
-        }
-        for (int row = tid >> 3; row < kUC * 8; row += kUThreads / 8) {
-            const int t = ktok[row];
-            const bool ok = t >= 0 && ch_ok;
-            const size_t off = ok ? cbase + t * tstride : 0;
-            cp_async16(smem_addr(ks) + urow_off(row, ch), a.k + off, ok);
-            cp_async16(smem_addr(vs) + urow_off(row, ch), a.v + off, ok);
-        }
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
+    const long long PW = static_cast<long long>(P) * kWarps;
+    const long long gw = static_cast<long long>(blockIdx.x) * kWarps + warp;
+    const long long W = static_cast<long long>(a.B) * a.G * a.H;
+    const long long u0 = gw * W / PW, u1 = (gw + 1) * W / PW;
+    if (u0 >= u1) return;
+    key_units(a, u0, u1, smem + warp * KTile::WARP);
+}
 
-    const int cw = warp / kUH, hw = warp % kUH;
-    const int kc = g0 + cw, h = hlo + hw;
-    if (kc >= G || h >= H) return;
-    const int gq = lane >> 2, tq = lane & 3, mi = lane >> 3;
-    uint32_t kf0, kf1, kf2, kf3, vf0, vf1, vf2, vf3;
-    ldsm_x4(smem_addr(ks) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), kf0, kf1, kf2, kf3);
-    ldsm_x4(smem_addr(vs) + urow_off(cw * 8 + (lane & 7), hw * 4 + mi), vf0, vf1, vf2, vf3);
-    const float sc = a.scale * kLog2e;
-    const float ba = a.bias[3 * h] * kLog2e, bb = a.bias[3 * h + 1] * kLog2e,
-                bc = a.bias[3 * h + 2] * kLog2e;
-    const float2 kp0 = kxy[cw * 8 + 2 * tq], kp1 = kxy[cw * 8 + 2 * tq + 1];
-    float dk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    float dv[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    const int e_end = es[cw + 1];
-    for (int e = es[cw]; e < e_end; e += 2) {
-        const int b1 = eu[e] * 8;
-        const int b2 = (e + 1 < e_end) ? eu[e + 1] * 8 : ZR;
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, pacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            const int row = ((mi & 1) ? b2 : b1) + (lane & 7);
-            const uint32_t off = urow_off(row, hw * 4 + 2 * kk + (mi >> 1));
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(smem_addr(qs) + off, a0, a1, a2, a3);
-            mma_bf16(sacc, a0, a1, a2, a3, kk ? kf2 : kf0, kk ? kf3 : kf1);
-            ldsm_x4(smem_addr(dos) + off, a0, a1, a2, a3);
-            mma_bf16(pacc, a0, a1, a2, a3, kk ? vf2 : vf0, kk ? vf3 : vf1);
-        }
-        float p[4], ds[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int qrow = ((j >> 1) ? b2 : b1) + gq;
-            const float2 qp = qxy[qrow];
-            const float2 kp = (j & 1) ? kp1 : kp0;
-            const float dx = kp.x - qp.x, dy = kp.y - qp.y;
-            const float lg = sacc[j] * sc + ba * dx + bb * dy - bc * (dx * dx + dy * dy);
-            p[j] = exp2f(lg - qL[qrow * kUH + hw]);
-            ds[j] = p[j] * (pacc[j] - qD[qrow * kUH + hw]);
-        }
-        const uint32_t pb0 = movm_t(pack_bf16(p[0], p[1]));
-        const uint32_t pb1 = movm_t(pack_bf16(p[2], p[3]));
-        const uint32_t sb0 = movm_t(pack_bf16(ds[0], ds[1]));
-        const uint32_t sb1 = movm_t(pack_bf16(ds[2], ds[3]));
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            const int row = ((mi >> 1) ? b2 : b1) + (lane & 7);
-            const uint32_t off = urow_off(row, hw * 4 + 2 * m + (mi & 1));
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(smem_addr(dos) + off, a0, a1, a2, a3);
-            mma_bf16(dv[m], a0, a1, a2, a3, pb0, pb1);
-            ldsm_x4_t(smem_addr(qs) + off, a0, a1, a2, a3);
-            mma_bf16(dk[m], a0, a1, a2, a3, sb0, sb1);
-        }
+// ---------------------------------------------------------------- launchers
+
+int sm_count() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        cached[dev] = n;
     }
-    uint8_t* stage = smem + L.stage + warp * 512;
-    store_rows_t1(dk, a.scale, stage, ktok + cw * 8, tok0, H, h, a.dk, lane);
-    store_rows_t1(dv, 1.f, stage, ktok + cw * 8, tok0, H, h, a.dv, lane);
+    return cached[dev];
+}
+
+// Persistent grid: resident CTAs per SM times the SM count, or fewer when there are fewer
+// items than warps.
+int grid_for(long long items, int per_sm) {
+    const long long slots = static_cast<long long>(sm_count()) * per_sm;
+    const long long need = (items + kWarps - 1) / kWarps;
+    return static_cast<int>(need < slots ? need : slots);
 }
 
 template <int MTILES>
-cudaError_t fwd_union_dispatch(const AttnArgs& a, cudaStream_t st) {
-    const size_t smem = static_cast<size_t>(union_layout(a.R, 16 * MTILES).total);
-    cudaError_t e = ensure_smem<attn_fwd_union_kernel<MTILES>>(smem);
+cudaError_t fwd_dispatch(const AttnArgs& a, cudaStream_t st) {
+    constexpr int per = MTILES <= 3 ? 4 : 2;
+    const size_t smem = static_cast<size_t>(kWarps) * QTile<16 * MTILES, false>::WARP;
+    cudaError_t e = ensure_smem<attn_fwd_kernel<MTILES>>(smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.G + kUC - 1) / kUC, (a.H + kUH - 1) / kUH, a.B);
-    attn_fwd_union_kernel<MTILES><<<grid, kUThreads, smem, st>>>(a);
+    const int grid = grid_for(static_cast<long long>(a.B) * a.G * a.H, per);
+    attn_fwd_kernel<MTILES><<<grid, kThreads, smem, st>>>(a);
     note_launch();
     return cudaGetLastError();
 }
 
 template <int MTILES>
 cudaError_t bwd_dispatch(const AttnArgs& a, cudaStream_t st) {
-    const int ncg = (a.G + kUC - 1) / kUC;
-    const int nhg = (a.H + kUH - 1) / kUH;
-    // query-major pass (+ one column of reverse-index CTAs)
-    size_t smem = static_cast<size_t>(union_layout(a.R, 16 * MTILES).total) + kUWarps * 512;
+    // prep: reverse index and its tokens, one CTA per image
     const size_t prep = 4 * static_cast<size_t>(a.G + 1) + 160;
-    if (prep > smem) smem = prep;
-    cudaError_t e = ensure_smem<attn_bwd_query_union_kernel<MTILES>>(smem);
+    cudaError_t e = ensure_smem<attn_bwd_prep_kernel>(prep);
     if (e != cudaSuccess) return e;
-    attn_bwd_query_union_kernel<MTILES><<<dim3(ncg + 1, nhg, a.B), kUThreads, smem, st>>>(a, ncg);
+    attn_bwd_prep_kernel<<<a.B, 256, prep, st>>>(a);
     note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // key-major pass (+ 3H bias-reduction CTAs in the first column block)
-    size_t smem2 = static_cast<size_t>(key_layout().total);
-    if (smem2 < static_cast<size_t>(kUWarps) * kBwdKWarpBytes) smem2 = static_cast<size_t>(kUWarps) * kBwdKWarpBytes;
-    e = ensure_smem<attn_bwd_key_union_kernel>(smem2);
+    // query pass
+    constexpr int per = MTILES <= 3 ? 3 : 2;
+    const size_t smem = static_cast<size_t>(kWarps) * QTile<16 * MTILES, true>::WARP;
+    e = ensure_smem<attn_bwd_query_kernel<MTILES>>(smem);
     if (e != cudaSuccess) return e;
-    const int extra = (3 * a.H + 0);
-    attn_bwd_key_union_kernel<<<dim3(ncg + extra, nhg, a.B), kUThreads, smem2, st>>>(a, ncg);
+    const long long items = static_cast<long long>(a.B) * a.G * a.H;
+    attn_bwd_query_kernel<MTILES><<<grid_for(items, per), kThreads, smem, st>>>(a);
+    note_launch();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // key pass (+ 3 H bias-reduction CTAs at the end of the grid)
+    const size_t smem2 = static_cast<size_t>(kWarps) * KTile::WARP;
+    e = ensure_smem<attn_bwd_key_kernel>(smem2);
+    if (e != cudaSuccess) return e;
+    const int P = grid_for(items, 4);
+    attn_bwd_key_kernel<<<P + 3 * a.H, kThreads, smem2, st>>>(a, P);
     note_launch();
     return cudaGetLastError();
 }
@@ -1109,16 +1103,17 @@ AttnWorkspace attn_workspace_layout(int B, int N, int H, int C, int M) {
     w.tok_cluster = off; off += up(sizeof(int32_t) * B * static_cast<size_t>(N));
     w.rev_off = off;     off += up(sizeof(int32_t) * B * (G + 1));
     w.rev_list = off;    off += up(sizeof(int32_t) * B * G * R);
+    w.rev_tok = off;     off += up(sizeof(int32_t) * B * G * R * 8);
     w.total = off;
     return w;
 }
 
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st) {
     switch ((a.M + 15) / 16) {
-        case 1: return fwd_union_dispatch<1>(a, st);
-        case 2: return fwd_union_dispatch<2>(a, st);
-        case 3: return fwd_union_dispatch<3>(a, st);
-        default: return fwd_union_dispatch<4>(a, st);
+        case 1: return fwd_dispatch<1>(a, st);
+        case 2: return fwd_dispatch<2>(a, st);
+        case 3: return fwd_dispatch<3>(a, st);
+        default: return fwd_dispatch<4>(a, st);
     }
 }
 

@@ -70,10 +70,11 @@ struct AttnArgs {
     int32_t* tok_cluster;  // [B][N]
     int32_t* rev_off;    // [B][G + 1]
     int32_t* rev_list;   // [B][G * R]
+    int32_t* rev_tok;    // [B][G * R][8] query tokens of every reverse-list entry
 };
 
 struct AttnWorkspace {
-    size_t delta, dbias_part, tok_cluster, rev_off, rev_list, total;
+    size_t delta, dbias_part, tok_cluster, rev_off, rev_list, rev_tok, total;
 };
 AttnWorkspace attn_workspace_layout(int B, int N, int H, int C, int M);
 

@@ -20,10 +20,12 @@ from tests.parity import LSE_ATOL, bf16, check_fwd, check_grad, dev, host
 pytestmark = pytest.mark.gpu
 
 
-def run_attn(a: synth.AttnBatch, M: int = 48, check_bwd: bool = True, scale=None):
+def run_attn(a: synth.AttnBatch, M: int = 48, check_bwd: bool = True, scale=None, cl=None, nb=None):
     scale = a.scale if scale is None else scale
-    cl = oracle.cluster(a.coords, 8)
-    nb = oracle.neighbors(a.coords, cl, M)
+    if cl is None:
+        cl = oracle.cluster(a.coords, 8)
+    if nb is None:
+        nb = oracle.neighbors(a.coords, cl, M)
     o_ref, lse_ref = oracle.attn_fwd(a.q, a.k, a.v, a.coords, cl, nb, a.bias, scale)
     Q, K, V, dO = bf16(a.q), bf16(a.k), bf16(a.v), bf16(a.do)
     xy, tcl, tnb, bias = dev(a.coords), dev(cl), dev(nb), dev(a.bias)
@@ -110,3 +112,64 @@ def test_zero_query_zero_bias_is_mean():
         keys = nb[0, g]
         for i in cl[0, g]:
             np.testing.assert_allclose(host(O)[0, i], v[keys].mean(axis=0), atol=1e-2)
+
+
+# Capacities of the kernels' shared-memory unions (blocks of 8 token rows), used below to
+# show that the hub table reaches every overflow path.
+FWD_STAGE_BLOCKS = 24     # forward / query pass: one pipeline stage
+KEY_STAGE_BLOCKS = 20     # key pass: one pipeline stage
+KEY_MAX_ENTRIES = 128     # key pass: reverse-list entries of one group
+
+
+def _groups(G):
+    ng = (G + 7) // 8
+    return [(gi * G // ng, (gi + 1) * G // ng) for gi in range(ng)]
+
+
+def hub_table(cl: np.ndarray, M: int, seed: int) -> np.ndarray:
+    """Neighbour table in which every cluster lists cluster 0 first, then itself, then
+    R - 2 other clusters at random (whole cluster rows, as the backward requires)."""
+    B, G, C = cl.shape
+    R = M // C
+    rng = np.random.default_rng(seed)
+    nb = np.full((B, G, M), -1, np.int32)
+    for b in range(B):
+        for g in range(G):
+            rest = [h for h in rng.permutation(G) if h not in (0, g)]
+            lst = ([0, g] if g else [0]) + rest
+            for r, h in enumerate(lst[:R]):
+                nb[b, g, r * C:(r + 1) * C] = cl[b, h]
+    return nb
+
+
+@pytest.mark.parametrize("M", [48, 64])
+def test_hub_table_overflow_paths(M):
+    """A hand-built table in which every cluster lists cluster 0.  The unions of a group's
+    neighbour blocks exceed one pipeline stage (single-buffered stage) and, at M = 64, two
+    stages (the group is processed in halves); the reverse list of cluster 0 holds every
+    cluster, so its key group overflows the key pass's union and takes the per-warp direct
+    path.  The assertions on the table's geometry show that each path is reached; the
+    parity checks cover all of them against the oracle."""
+    a = synth.attn_stage1(B=2, N=700, H=3)
+    cl = oracle.cluster(a.coords, 8)
+    nb = hub_table(cl, M, seed=11 + M)
+    B, G, _ = cl.shape
+    R = M // 8
+    fwd_unions, key_entries, key_unions = [], [], []
+    for b in range(B):
+        first = {int(cl[b, g, 0]): g for g in range(G)}
+        rev = [[] for _ in range(G)]
+        for g in range(G):
+            for r in range(R):
+                rev[first[int(nb[b, g, r * 8])]].append(g)
+        for c0, c1 in _groups(G):
+            fwd_unions.append(len({tuple(nb[b, g, r * 8:(r + 1) * 8]) for g in range(c0, c1) for r in range(R)}))
+            ents = [q for k in range(c0, c1) for q in rev[k]]
+            key_entries.append(len(ents))
+            key_unions.append(len(set(ents)))
+    assert max(fwd_unions) > FWD_STAGE_BLOCKS                    # single-buffered stage
+    if M == 64:
+        assert max(fwd_unions) > 2 * FWD_STAGE_BLOCKS            # halves of the group
+    assert max(key_entries) > KEY_MAX_ENTRIES or max(key_unions) > 2 * KEY_STAGE_BLOCKS  # direct
+    assert min(key_unions) <= 2 * KEY_STAGE_BLOCKS               # and a union path beside it
+    run_attn(a, M=M, cl=cl, nb=nb)

@@ -189,83 +189,100 @@ struct QTile {
     static constexpr int WARP = 2 * STAGE;
 };
 
-// One cluster's rows as the gather needs them: the tokens of rows gq + 8 k (made valid),
-// and of query row gq.
-template <int NK>
+// One cluster's rows as the gather needs them: the byte offsets of rows gq + 8 k and of
+// query row gq in a [B][N][H][32] bf16 tensor (at head 0), and a bit per row that marks a
+// token.  Off is 32-bit when every such tensor is smaller than 4 GiB.
+template <int NK, typename Off>
 struct Rows {
-    int rt[NK];
-    int qt;
+    Off ro[NK];
+    Off rq;
+    unsigned valid;  // bit k: row gq + 8 k; bit NK: query row gq
 };
-template <int NK>
-__device__ __forceinline__ Rows<NK> cluster_rows(const Toks& t, int lane, int N) {
-    Rows<NK> r;
+template <int NK, typename Off>
+__device__ __forceinline__ Rows<NK, Off> cluster_rows(const AttnArgs& a, const Toks& t, int b, int lane) {
+    Rows<NK, Off> r;
+    const Off rowb = static_cast<Off>(a.H) * 64u;
+    const Off base = static_cast<Off>(b) * static_cast<Off>(a.N);
+    r.valid = 0u;
 #pragma unroll
-    for (int k = 0; k < NK; ++k)
-        r.rt[k] = valid_tok(__shfl_sync(0xffffffffu, k < 4 ? t.a : t.b, (lane >> 2) + 8 * (k & 3)), N);
-    r.qt = valid_tok(__shfl_sync(0xffffffffu, t.q, lane >> 2), N);
+    for (int k = 0; k < NK; ++k) {
+        const int tk = __shfl_sync(0xffffffffu, k < 4 ? t.a : t.b, (lane >> 2) + 8 * (k & 3));
+        const bool ok = static_cast<unsigned>(tk) < static_cast<unsigned>(a.N);
+        r.ro[k] = ok ? (base + static_cast<Off>(tk)) * rowb : Off(0);
+        r.valid |= ok ? (1u << k) : 0u;
+    }
+    const int tq = __shfl_sync(0xffffffffu, t.q, lane >> 2);
+    const bool okq = static_cast<unsigned>(tq) < static_cast<unsigned>(a.N);
+    r.rq = okq ? (base + static_cast<Off>(tq)) * rowb : Off(0);
+    r.valid |= okq ? (1u << NK) : 0u;
     return r;
 }
 
-// Gather head h of a cluster of image b into the stage at sb (a shared address).
-template <int MT, bool BWD>
-__device__ __forceinline__ void gather_cluster(const AttnArgs& a, int b, int h, const Rows<MT / 8>& r,
-                                               uint32_t sb, int lane) {
+// Gather head h of a cluster into the stage at sb (a shared address): K and V rows, the Q
+// row (query pass: the dO row and the lse of the query too).
+template <int MT, bool BWD, typename Off>
+__device__ __forceinline__ void gather_cluster(const AttnArgs& a, int h, const Rows<MT / 8, Off>& r, uint32_t sb,
+                                               int lane) {
     using T = QTile<MT, BWD>;
     const uint32_t lo = gather_lane_off(lane);
-    const size_t rowel = static_cast<size_t>(a.H) * 32;
-    const size_t tok0 = static_cast<size_t>(b) * a.N;
-    const size_t hoff = static_cast<size_t>(h) * 32 + (lane & 3) * 8;
+    const size_t hb = static_cast<size_t>(h) * 64 + (lane & 3) * 16;
+    const char* kp = reinterpret_cast<const char*>(a.k) + hb;
+    const char* vp = reinterpret_cast<const char*>(a.v) + hb;
 #pragma unroll
     for (int k = 0; k < MT / 8; ++k) {
-        const int t = r.rt[k];
-        const size_t src = t >= 0 ? (tok0 + t) * rowel + hoff : 0;
-        cp_async16(sb + T::K + 512 * k + lo, a.k + src, t >= 0);
-        cp_async16(sb + T::V + 512 * k + lo, a.v + src, t >= 0);
+        const bool ok = (r.valid >> k) & 1u;
+        cp_async16(sb + T::K + 512 * k + lo, kp + r.ro[k], ok);
+        cp_async16(sb + T::V + 512 * k + lo, vp + r.ro[k], ok);
     }
-    const int t = r.qt;
-    const size_t src = t >= 0 ? (tok0 + t) * rowel + hoff : 0;
-    cp_async16(sb + T::Q + lo, a.q + src, t >= 0);
+    const bool okq = (r.valid >> (MT / 8)) & 1u;
+    cp_async16(sb + T::Q + lo, reinterpret_cast<const char*>(a.q) + hb + r.rq, okq);
     if (BWD) {
-        cp_async16(sb + T::DO + lo, a.dout + src, t >= 0);
+        cp_async16(sb + T::DO + lo, reinterpret_cast<const char*>(a.dout) + hb + r.rq, okq);
+        // lse[tok][h] = element (row byte offset / 64 bytes per head-row) + h
         if ((lane & 3) == 0)
-            cp_async4(sb + T::LSE + 4 * (lane >> 2), a.lse_in + (t >= 0 ? (tok0 + t) * a.H + h : 0), t >= 0);
+            cp_async4(sb + T::LSE + 4 * (lane >> 2), a.lse_in + (static_cast<size_t>(r.rq) >> 6) + h, okq);
     }
 }
 
 // Per-lane geometry of one cluster, reused for every head: the lane's keys k = 2 i + hi
 // (slot gq + 8 k) and query columns 2 tq, 2 tq + 1 in local coordinates (origin: the
-// cluster's first slot), and the query tokens the lane writes.
+// cluster's first slot), and the query tokens the lane writes (lanes < 8 write query
+// `lane`'s lse / Delta).
 template <int MTILES>
 struct Geo {
-    float kx[2 * MTILES], ky[2 * MTILES];
+    float kx[2 * MTILES], ky[2 * MTILES], kr[2 * MTILES];  // kr = kx^2 + ky^2
     unsigned kval;
     float qx[2], qy[2];
-    int qo;      // query row gq (O / dQ rows)
-    int ql[2];   // query columns 2 tq, 2 tq + 1 (lse / Delta)
+    float sx, sy;  // query `lane` (lanes < 8)
+    int qo;        // query row gq (O / dQ rows)
+    int qs;        // query `lane` (lanes < 8)
 };
 
 template <int MTILES>
-__device__ __forceinline__ Geo<MTILES> make_geo(const Toks& t, const TokXY& x, const int (&rt)[2 * MTILES], int lane,
-                                                int N) {
+__device__ __forceinline__ Geo<MTILES> make_geo(const Toks& t, const TokXY& x, unsigned valid, int lane, int N) {
     const int gq = lane >> 2, tq = lane & 3;
     Geo<MTILES> g;
     const float2 o = sh2(x.q, 0);
-    g.kval = 0u;
+    g.kval = valid;
 #pragma unroll
     for (int k = 0; k < 2 * MTILES; ++k) {
         const float2 p = sh2(k < 4 ? x.a : x.b, gq + 8 * (k & 3));
-        const bool ok = rt[k] >= 0;
+        const bool ok = (valid >> k) & 1u;
         g.kx[k] = ok ? p.x - o.x : 0.f;
         g.ky[k] = ok ? p.y - o.y : 0.f;
-        g.kval |= ok ? (1u << k) : 0u;
+        g.kr[k] = fmaf(g.kx[k], g.kx[k], g.ky[k] * g.ky[k]);
     }
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
         const float2 p = sh2(x.q, 2 * tq + c);
         g.qx[c] = p.x - o.x;
         g.qy[c] = p.y - o.y;
-        g.ql[c] = valid_tok(__shfl_sync(0xffffffffu, t.q, 2 * tq + c), N);
     }
+    g.sx = x.q.x - o.x;
+    g.sy = x.q.y - o.y;
+    g.qs = valid_tok(t.q, N);
+    // bits 16 + s: query slot s holds a token
+    g.kval |= __ballot_sync(0xffffffffu, lane < 8 && g.qs >= 0) << 16;
     g.qo = valid_tok(__shfl_sync(0xffffffffu, t.q, gq), N);
     return g;
 }
@@ -273,7 +290,7 @@ __device__ __forceinline__ Geo<MTILES> make_geo(const Toks& t, const TokXY& x, c
 // ------------------------------------------------------------------ forward
 
 template <int MTILES>
-__device__ __forceinline__ void fwd_item(const AttnArgs& a, int b, int h, uint32_t sb, const LaneOffs& lo,
+__device__ __forceinline__ void fwd_item(const AttnArgs& a, size_t tok0, int h, uint32_t sb, const LaneOffs& lo,
                                          const Geo<MTILES>& g, int lane) {
     using T = QTile<16 * MTILES, false>;
     const int gq = lane >> 2, tq = lane & 3;
@@ -284,9 +301,7 @@ __device__ __forceinline__ void fwd_item(const AttnArgs& a, int b, int h, uint32
     float u[2 * MTILES];
 #pragma unroll
     for (int k = 0; k < 2 * MTILES; ++k)
-        u[k] = ((g.kval >> k) & 1u)
-                   ? fmaf(a2, g.kx[k], fmaf(b2, g.ky[k], -c2 * fmaf(g.kx[k], g.kx[k], g.ky[k] * g.ky[k])))
-                   : -INFINITY;
+        u[k] = ((g.kval >> k) & 1u) ? fmaf(a2, g.kx[k], fmaf(b2, g.ky[k], -c2 * g.kr[k])) : -INFINITY;
     const float X[2] = {2.f * c2 * g.qx[0], 2.f * c2 * g.qx[1]};
     const float Y[2] = {2.f * c2 * g.qy[0], 2.f * c2 * g.qy[1]};
 
@@ -356,7 +371,6 @@ __device__ __forceinline__ void fwd_item(const AttnArgs& a, int b, int h, uint32
     const float l1 = __shfl_sync(0xffffffffu, lacc[1], tq);
     const float i0 = l0 > 0.f ? sfu_rcp(l0) : 0.f;
     const float i1 = l1 > 0.f ? sfu_rcp(l1) : 0.f;
-    const size_t tok0 = static_cast<size_t>(b) * a.N;
     // O^T (dims x queries) -> rows of O: after the transpose lane (g, t) holds dims
     // 2t, 2t + 1 (+ 8, + 16, + 24) of query g
     const uint32_t w0 = movm_t(pack_bf16(oacc[0][0] * i0, oacc[0][1] * i1));
@@ -370,23 +384,23 @@ __device__ __forceinline__ void fwd_item(const AttnArgs& a, int b, int h, uint32
         dst[8] = w2;
         dst[12] = w3;
     }
-    if (gq == 0) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const float l = lacc[c];
-            const float mc = c ? m1 : m0;
-            // w_i in natural units: the query-constant part of the expanded bias
-            const float wq = -(an * g.qx[c] + bn * g.qy[c] + cn * fmaf(g.qx[c], g.qx[c], g.qy[c] * g.qy[c]));
-            if (g.ql[c] >= 0)
-                a.lse[(tok0 + g.ql[c]) * a.H + h] = l > 0.f ? (mc + sfu_lg2(l)) * kLn2 + wq : -INFINITY;
-        }
+    // lse of query `lane` (lanes < 8): its column max and sum sit at lane lane / 2
+    {
+        const int src = (lane >> 1) & 3;
+        const float ma = __shfl_sync(0xffffffffu, m0, src), mb = __shfl_sync(0xffffffffu, m1, src);
+        const float la = __shfl_sync(0xffffffffu, lacc[0], src), lb = __shfl_sync(0xffffffffu, lacc[1], src);
+        const float mq = (lane & 1) ? mb : ma, lq = (lane & 1) ? lb : la;
+        // w_i in natural units: the query-constant part of the expanded bias
+        const float wq = -fmaf(an, g.sx, fmaf(bn, g.sy, cn * fmaf(g.sx, g.sx, g.sy * g.sy)));
+        if (lane < 8 && g.qs >= 0)
+            a.lse[(tok0 + g.qs) * a.H + h] = lq > 0.f ? fmaf(mq + sfu_lg2(lq), kLn2, wq) : -INFINITY;
     }
 }
 
 // ---------------------------------------------------------------- query pass
 
 template <int MTILES>
-__device__ __forceinline__ void query_item(const AttnArgs& a, int b, int gabs, int h, uint32_t sb,
+__device__ __forceinline__ void query_item(const AttnArgs& a, size_t tok0, size_t crow, int h, uint32_t sb,
                                            const float* lse_s, const LaneOffs& lo, const Geo<MTILES>& g,
                                            int lane) {
     using T = QTile<16 * MTILES, true>;
@@ -398,16 +412,16 @@ __device__ __forceinline__ void query_item(const AttnArgs& a, int b, int gabs, i
     float u[2 * MTILES];
 #pragma unroll
     for (int k = 0; k < 2 * MTILES; ++k)
-        u[k] = ((g.kval >> k) & 1u)
-                   ? fmaf(a2, g.kx[k], fmaf(b2, g.ky[k], -c2 * fmaf(g.kx[k], g.kx[k], g.ky[k] * g.ky[k])))
-                   : -INFINITY;
+        u[k] = ((g.kval >> k) & 1u) ? fmaf(a2, g.kx[k], fmaf(b2, g.ky[k], -c2 * g.kr[k])) : -INFINITY;
     float X[2], Y[2], Lq[2];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
         X[c] = 2.f * c2 * g.qx[c];
         Y[c] = 2.f * c2 * g.qy[c];
         const float l = lse_s[2 * tq + c];
-        const bool ok = g.ql[c] >= 0 && l != -INFINITY;
+        // a padding query (no token) has its lse slot zero-filled: mask it through the
+        // query-validity bits of the cluster
+        const bool ok = ((g.kval >> (16 + 2 * tq + c)) & 1u) && l != -INFINITY;
         // P = exp2(t - L'), L' = lse log2e - w2 with w2 the query-constant bias part
         const float qr2 = fmaf(g.qx[c], g.qx[c], g.qy[c] * g.qy[c]);
         Lq[c] = ok ? fmaf(l, kLog2e, fmaf(a2, g.qx[c], fmaf(b2, g.qy[c], c2 * qr2))) : INFINITY;
@@ -461,7 +475,7 @@ __device__ __forceinline__ void query_item(const AttnArgs& a, int b, int gabs, i
             S0[c] += v;
             Sx[c] = fmaf(v, g.kx[k], Sx[c]);
             Sy[c] = fmaf(v, g.ky[k], Sy[c]);
-            Sr[c] = fmaf(v, fmaf(g.kx[k], g.kx[k], g.ky[k] * g.ky[k]), Sr[c]);
+            Sr[c] = fmaf(v, g.kr[k], Sr[c]);
         }
         dsb[i][0] = movm_t(pack_bf16(ds[0], ds[1]));
         dsb[i][1] = movm_t(pack_bf16(ds[2], ds[3]));
@@ -476,17 +490,17 @@ __device__ __forceinline__ void query_item(const AttnArgs& a, int b, int gabs, i
               fmaf(g.qx[c], g.qx[c], g.qy[c] * g.qy[c]) * S0[c];
     }
     warp_sum3(ga, gb, gc, lane);
-    const size_t tok0 = static_cast<size_t>(b) * a.N;
     if (lane == 0) {
-        float* part = a.dbias_part + ((static_cast<size_t>(b) * a.G + gabs) * a.H + h) * 3;
+        float* part = a.dbias_part + (crow * a.H + h) * 3;
         part[0] = ga;
         part[1] = gb;
         part[2] = -gc;
     }
-    if (gq == 0) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-            if (g.ql[c] >= 0) a.delta[(tok0 + g.ql[c]) * a.H + h] = pd[c];
+    {
+        // Delta of query `lane` (lanes < 8) from the lanes holding its column
+        const int src = (lane >> 1) & 3;
+        const float da = __shfl_sync(0xffffffffu, pd[0], src), db = __shfl_sync(0xffffffffu, pd[1], src);
+        if (lane < 8 && g.qs >= 0) a.delta[(tok0 + g.qs) * a.H + h] = (lane & 1) ? db : da;
     }
     float dq[2][4];
 #pragma unroll
@@ -518,7 +532,7 @@ __device__ __forceinline__ void query_item(const AttnArgs& a, int b, int gabs, i
 // One warp's items [i0, i1) (item = (image, cluster, head), cluster-major).  While item i
 // computes, item i + 1 is in flight; the neighbour rows of the cluster after next and the
 // coordinates of the next cluster load into registers at every cluster start.
-template <int MTILES, bool BWD>
+template <int MTILES, bool BWD, typename Off>
 __device__ __forceinline__ void cluster_items(const AttnArgs& a, long long i0, long long i1, uint8_t* wsm) {
     constexpr int MT = 16 * MTILES, NK = MT / 8;
     using T = QTile<MT, BWD>;
@@ -526,51 +540,52 @@ __device__ __forceinline__ void cluster_items(const AttnArgs& a, long long i0, l
     const int H = a.H, G = a.G, N = a.N;
     const LaneOffs lo = lane_offs(lane);
     const uint32_t wb = smem_addr(wsm);
-    long long c = i0 / H;                 // global cluster index b * G + g
-    int h = static_cast<int>(i0 - c * H);
-    const long long c_last = (i1 - 1) / H;
-    const int h_last_end = static_cast<int>(i1 - 1 - c_last * H) + 1;
-    int b = static_cast<int>(c / G), g = static_cast<int>(c - static_cast<long long>(b) * G);
+    const long long c0 = i0 / H;          // global cluster index b * G + g
+    int h = static_cast<int>(i0 - c0 * H);
+    // clusters left after the current one, and the end head of the last
+    unsigned left = static_cast<unsigned>((i1 - 1) / H - c0);
+    const int h_last_end = static_cast<int>(i1 - 1 - ((i1 - 1) / H) * H) + 1;
+    int b = static_cast<int>(c0 / G), g = static_cast<int>(c0 - static_cast<long long>(b) * G);
     int b1 = b, g1 = g;
     next_cluster(b1, g1, G);
     int b2 = b1, g2 = g1;
     next_cluster(b2, g2, G);
     Toks cur = load_toks(a, b, g, lane);
-    Toks nx = c + 1 <= c_last ? load_toks(a, b1, g1, lane) : Toks{-1, -1, -1};
+    Toks nx = left >= 1 ? load_toks(a, b1, g1, lane) : Toks{-1, -1, -1};
     TokXY cxy = load_xy(a, b, cur);
-    Rows<NK> rows = cluster_rows<NK>(cur, lane, N);
+    Rows<NK, Off> rows = cluster_rows<NK, Off>(a, cur, b, lane);
     int st = 0;
-    gather_cluster<MT, BWD>(a, b, h, rows, wb, lane);
+    gather_cluster<MT, BWD, Off>(a, h, rows, wb, lane);
     cp_async_commit();
     for (;;) {
-        const bool lastc = c == c_last;
-        const int hend = lastc ? h_last_end : H;
-        const Toks nn = c + 2 <= c_last ? load_toks(a, b2, g2, lane) : Toks{-1, -1, -1};
-        const TokXY nxy = c + 1 <= c_last ? load_xy(a, b1, nx) : TokXY{};
-        const Geo<MTILES> geo = make_geo<MTILES>(cur, cxy, rows.rt, lane, N);
-        Rows<NK> nrows = rows;
+        const int hend = left == 0 ? h_last_end : H;
+        const Toks nn = left >= 2 ? load_toks(a, b2, g2, lane) : Toks{-1, -1, -1};
+        const TokXY nxy = left >= 1 ? load_xy(a, b1, nx) : TokXY{};
+        const Geo<MTILES> geo = make_geo<MTILES>(cur, cxy, rows.valid, lane, N);
+        Rows<NK, Off> nrows = rows;
+        const size_t tok0 = static_cast<size_t>(b) * N;
         for (; h < hend; ++h) {
             cp_async_wait<0>();
             __syncwarp();
             const uint32_t sb = wb + st * T::STAGE, nb = wb + (st ^ 1) * T::STAGE;
             if (h + 1 < hend) {
-                gather_cluster<MT, BWD>(a, b, h + 1, rows, nb, lane);
+                gather_cluster<MT, BWD, Off>(a, h + 1, rows, nb, lane);
                 cp_async_commit();
-            } else if (!lastc) {
-                nrows = cluster_rows<NK>(nx, lane, N);
-                gather_cluster<MT, BWD>(a, b1, 0, nrows, nb, lane);
+            } else if (left != 0) {
+                nrows = cluster_rows<NK, Off>(a, nx, b1, lane);
+                gather_cluster<MT, BWD, Off>(a, 0, nrows, nb, lane);
                 cp_async_commit();
             }
             if (BWD)
-                query_item<MTILES>(a, b, g, h, sb, reinterpret_cast<const float*>(wsm + st * T::STAGE + T::LSE), lo,
-                                   geo, lane);
+                query_item<MTILES>(a, tok0, static_cast<size_t>(b) * G + g, h, sb,
+                                   reinterpret_cast<const float*>(wsm + st * T::STAGE + T::LSE), lo, geo, lane);
             else
-                fwd_item<MTILES>(a, b, h, sb, lo, geo, lane);
+                fwd_item<MTILES>(a, tok0, h, sb, lo, geo, lane);
             __syncwarp();
             st ^= 1;
         }
-        if (lastc) break;
-        ++c;
+        if (left == 0) break;
+        --left;
         h = 0;
         b = b1;
         g = g1;
@@ -685,6 +700,95 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
     for (int i = tid; i < total * 8; i += nt) rtok[i] = valid_tok(cl[lst[i >> 3] * 8 + (i & 7)], N);
 }
 
+// The same index built in shared memory (one CTA per image) when the image fits: the
+// token -> cluster map, the cluster rows, the list entries and their key clusters all live
+// on chip, so the kernel makes one pass over its inputs and one over its outputs.
+// Shared ints: tc[N], cnt[G + 1], lst[G R], ek[G R], cls[8 G], scratch[40].
+size_t prep_smem_ints(int N, int G, int R) {
+    return static_cast<size_t>(N) + (G + 1) + 2ull * G * R + 8ull * G + 40;
+}
+
+__device__ void prep_image_smem(const AttnArgs& a, int b, uint8_t* smem) {
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int N = a.N, G = a.G, R = a.R, M = a.M;
+    int* tc = reinterpret_cast<int*>(smem);
+    int* cnt = tc + N;
+    int* lst = cnt + G + 1;
+    int* ek = lst + G * R;
+    int* cls = ek + G * R;
+    int* scratch = cls + 8 * G;
+    const int32_t* cl = a.clusters + static_cast<size_t>(b) * G * 8;
+    const int32_t* nb = a.nbr + static_cast<size_t>(b) * G * M;
+    int32_t* off = a.rev_off + static_cast<size_t>(b) * (G + 1);
+    int32_t* rlst = a.rev_list + static_cast<size_t>(b) * G * R;
+    int32_t* rtok = a.rev_tok + static_cast<size_t>(b) * G * R * 8;
+    for (int i = tid; i < N; i += nt) tc[i] = -1;
+    for (int i = tid; i <= G; i += nt) cnt[i] = 0;
+    // the first token of every neighbour block, eight loads in flight per thread
+    constexpr int kB = 8;
+    for (int e0 = tid; e0 < G * R; e0 += kB * nt) {
+#pragma unroll
+        for (int j = 0; j < kB; ++j) {
+            const int e = e0 + j * nt;
+            if (e < G * R) {
+                const int q = e / R;
+                ek[e] = __ldg(nb + static_cast<size_t>(q) * M + (e - q * R) * 8);
+            }
+        }
+    }
+    for (int i0 = tid; i0 < G * 8; i0 += kB * nt) {
+        int v[kB];
+#pragma unroll
+        for (int j = 0; j < kB; ++j) v[j] = i0 + j * nt < G * 8 ? __ldg(cl + i0 + j * nt) : -1;
+#pragma unroll
+        for (int j = 0; j < kB; ++j)
+            if (i0 + j * nt < G * 8) cls[i0 + j * nt] = valid_tok(v[j], N);
+    }
+    __syncthreads();
+    for (int i = tid; i < G * 8; i += nt) {
+        const int t = cls[i];
+        if (t >= 0) tc[t] = i >> 3;
+    }
+    __syncthreads();
+    for (int e = tid; e < G * R; e += nt) {
+        const int t0 = valid_tok(ek[e], N);
+        const int h = t0 >= 0 ? tc[t0] : -1;
+        ek[e] = h;
+        if (h >= 0) atomicAdd(&cnt[h], 1);
+    }
+    __syncthreads();
+    const int total = block_scan_excl(cnt, G, scratch);
+    for (int i = tid; i < G; i += nt) off[i] = cnt[i];
+    if (tid == 0) off[G] = total;
+    __syncthreads();  // every list start is read before the fill advances it
+    for (int e = tid; e < G * R; e += nt) {
+        const int h = ek[e];
+        if (h >= 0) lst[atomicAdd(&cnt[h], 1)] = e / R;
+    }
+    __syncthreads();
+    // cnt[h] is now the end of list h; sort every list so the order is fixed
+    for (int h = tid; h < G; h += nt) {
+        const int lo = h > 0 ? cnt[h - 1] : 0, hi = cnt[h];
+        for (int i = lo + 1; i < hi; ++i) {
+            const int v = lst[i];
+            int j = i - 1;
+            while (j >= lo && lst[j] > v) {
+                lst[j + 1] = lst[j];
+                --j;
+            }
+            lst[j + 1] = v;
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < total; i += nt) rlst[i] = lst[i];
+    for (int i = tid; i < total * 8; i += nt) rtok[i] = cls[lst[i >> 3] * 8 + (i & 7)];
+}
+
+__global__ void __launch_bounds__(256) attn_bwd_prep_smem_kernel(const AttnArgs a) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    prep_image_smem(a, blockIdx.x, smem);
+}
+
 // ------------------------------------------------------------------ key pass
 
 // Per-warp stage of the key pass: the key cluster's own K and V rows, the chunk's Q and dO
@@ -695,24 +799,24 @@ struct KTile {
     static constexpr int V = 8 * kRowB;
     static constexpr int Q = 16 * kRowB;
     static constexpr int DO = Q + 8 * kChunk * kRowB;
-    static constexpr int PRM = DO + 8 * kChunk * kRowB;
-    static constexpr int STAGE = PRM + 16 * 8 * kChunk;
+    static constexpr int PRM = DO + 8 * kChunk * kRowB;     // float4 [8 kChunk] row parameters
+    static constexpr int LSE = PRM + 16 * 8 * kChunk;       // float [8 kChunk] raw lse
+    static constexpr int DEL = LSE + 4 * 8 * kChunk;        // float [8 kChunk] raw Delta
+    static constexpr int STAGE = DEL + 4 * 8 * kChunk;
     static constexpr int WARP = 2 * STAGE;
 };
 
-// One pair of query clusters (16 queries) against the warp's 8 keys.  rb1 / rb2: rows of
-// the two query blocks in the Q / dO tiles at qb / dob; p1 / p2: parameter rows
+// One pair of query clusters (16 queries, rows 8 e .. 8 e + 15 of the Q / dO tiles at qb /
+// dob, i.e. byte offset pe = 512 e) against the warp's 8 keys; p1 / p2: parameter rows
 // (X, Y, L', Delta) of the lane's queries gq in each block.
-__device__ __forceinline__ void key_pair(uint32_t qb, uint32_t dob, int rb1, int rb2, float4 p1, float4 p2,
-                                         const uint32_t (&kf)[4], const uint32_t (&vf)[4], const float (&kx)[2],
-                                         const float (&ky)[2], const float (&u)[2], float sc, float (&dk)[2][4],
-                                         float (&dv)[2][4]) {
-    const int lane = threadIdx.x & 31, mi = lane >> 3;
+__device__ __forceinline__ void key_pair(uint32_t qb, uint32_t dob, uint32_t pe, const LaneOffs& lo, float4 p1,
+                                         float4 p2, const uint32_t (&kf)[4], const uint32_t (&vf)[4],
+                                         const float (&kx)[2], const float (&ky)[2], const float (&u)[2], float sc,
+                                         float (&dk)[2][4], float (&dv)[2][4]) {
     float sacc[4] = {0.f, 0.f, 0.f, 0.f}, pacc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int rs = ((mi & 1) ? rb2 : rb1) + (lane & 7);
 #pragma unroll
     for (int kk = 0; kk < 2; ++kk) {
-        const uint32_t off = tile64_off(rs, 2 * kk + (mi >> 1));
+        const uint32_t off = pe + (kk ? lo.ls1 : lo.ls0);
         uint32_t r0, r1, r2, r3;
         ldsm_x4(qb + off, r0, r1, r2, r3);
         mma_bf16(sacc, r0, r1, r2, r3, kf[2 * kk], kf[2 * kk + 1]);
@@ -733,10 +837,9 @@ __device__ __forceinline__ void key_pair(uint32_t qb, uint32_t dob, int rb1, int
     const uint32_t pb1 = movm_t(pack_bf16(p[2], p[3]));
     const uint32_t sb0 = movm_t(pack_bf16(ds[0], ds[1]));
     const uint32_t sb1 = movm_t(pack_bf16(ds[2], ds[3]));
-    const int rt = ((mi >> 1) ? rb2 : rb1) + (lane & 7);
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-        const uint32_t off = tile64_off(rt, 2 * m + (mi & 1));
+        const uint32_t off = pe + (m ? lo.lt1 : lo.lt0);
         uint32_t r0, r1, r2, r3;
         ldsm_x4_t(dob + off, r0, r1, r2, r3);
         mma_bf16(dv[m], r0, r1, r2, r3, pb0, pb1);
@@ -776,69 +879,106 @@ __device__ __forceinline__ void store_key_rows(const float (&acc)[2][4], float s
 }
 
 // A key-pass item: (image b, key cluster kc, head h, chunk ch) over the list entries
-// [e0, e0 + E) of kc (image-local).  It carries what the gather needs: the tokens of the
-// lane's gather rows (chunk rows gq + 8 k), of the lane's parameter rows lane and lane + 32,
-// of the own cluster row (lanes < 8), and the coordinates of the last two groups.
+// [e0, e0 + E) of kc (image-local).  It carries what the gather needs: the byte offsets
+// (head 0) of the lane's gather rows -- own row gq, chunk rows gq + 8 k -- with a validity
+// bit each, the tokens of the lane's parameter rows lane and lane + 32 and of the own
+// cluster row (lanes < 8), and their coordinates (loaded an item later).
+template <typename Off>
 struct KItem {
     int b, kc, h, ch, nch, e0, E;
-    int qt[kChunk];
+    Off qo[kChunk], ko;
+    unsigned valid;  // bit k: chunk row gq + 8 k; bit kChunk: own row gq
     int pa, pb, kt;
     float2 pxa, pxb, kxy;
 };
 
-// Tokens of an item (coordinates separately, an item later).
-__device__ __forceinline__ void kitem_tokens(const AttnArgs& a, KItem& it, int lane) {
+// Tokens and row offsets of an item (coordinates separately, an item later).
+template <typename Off>
+__device__ __forceinline__ void kitem_tokens(const AttnArgs& a, KItem<Off>& it, int lane) {
     const int G = a.G, N = a.N;
     const int32_t* rtok = a.rev_tok + static_cast<size_t>(it.b) * G * a.R * 8;
     const size_t base = (static_cast<size_t>(it.e0) + static_cast<size_t>(kChunk) * it.ch) * 8;
     const int rem = (it.E - kChunk * it.ch) * 8;
     const int n = rem > 8 * kChunk ? 8 * kChunk : rem;
     const int gq = lane >> 2;
-#pragma unroll
-    for (int k = 0; k < kChunk; ++k) it.qt[k] = gq + 8 * k < n ? __ldg(rtok + base + gq + 8 * k) : -1;
+    const Off rowb = static_cast<Off>(a.H) * 64u;
+    const Off tb = static_cast<Off>(it.b) * static_cast<Off>(N);
+    // lane l loads chunk rows l and l + 32 (parameter rows); gather rows gq + 8 k arrive by shuffle
     it.pa = lane < n ? __ldg(rtok + base + lane) : -1;
     it.pb = lane + 32 < n ? __ldg(rtok + base + lane + 32) : -1;
+    it.valid = 0u;
+#pragma unroll
+    for (int k = 0; k < kChunk; ++k) {
+        const int t = __shfl_sync(0xffffffffu, k < 4 ? it.pa : it.pb, gq + 8 * (k & 3));
+        it.qo[k] = t >= 0 ? (tb + static_cast<Off>(t)) * rowb : Off(0);
+        it.valid |= t >= 0 ? (1u << k) : 0u;
+    }
     it.kt = lane < 8 ? valid_tok(__ldg(a.clusters + (static_cast<size_t>(it.b) * G + it.kc) * 8 + lane), N) : -1;
+    const int own = __shfl_sync(0xffffffffu, it.kt, gq);
+    it.ko = own >= 0 ? (tb + static_cast<Off>(own)) * rowb : Off(0);
+    it.valid |= own >= 0 ? (1u << kChunk) : 0u;
 }
-__device__ __forceinline__ void kitem_coords(const AttnArgs& a, KItem& it) {
+template <typename Off>
+__device__ __forceinline__ void kitem_coords(const AttnArgs& a, KItem<Off>& it) {
     const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(it.b) * a.N;
     it.pxa = it.pa >= 0 ? __ldg(xyb + it.pa) : make_float2(0.f, 0.f);
     it.pxb = it.pb >= 0 ? __ldg(xyb + it.pb) : make_float2(0.f, 0.f);
     it.kxy = it.kt >= 0 ? __ldg(xyb + it.kt) : make_float2(0.f, 0.f);
 }
 
-__device__ __forceinline__ void kitem_gather(const AttnArgs& a, const KItem& it, uint32_t sb, int lane) {
+template <typename Off>
+__device__ __forceinline__ void kitem_gather(const AttnArgs& a, const KItem<Off>& it, uint32_t sb, int lane) {
     const uint32_t lo = gather_lane_off(lane);
-    const size_t rowel = static_cast<size_t>(a.H) * 32;
-    const size_t tok0 = static_cast<size_t>(it.b) * a.N;
-    const size_t hoff = static_cast<size_t>(it.h) * 32 + (lane & 3) * 8;
-    const int own = __shfl_sync(0xffffffffu, it.kt, lane >> 2);
-    {
-        const size_t src = own >= 0 ? (tok0 + own) * rowel + hoff : 0;
-        cp_async16(sb + KTile::K + lo, a.k + src, own >= 0);
-        cp_async16(sb + KTile::V + lo, a.v + src, own >= 0);
-    }
+    const size_t hb = static_cast<size_t>(it.h) * 64 + (lane & 3) * 16;
+    const char* kp = reinterpret_cast<const char*>(a.k) + hb;
+    const char* vp = reinterpret_cast<const char*>(a.v) + hb;
+    const char* qp = reinterpret_cast<const char*>(a.q) + hb;
+    const char* dp = reinterpret_cast<const char*>(a.dout) + hb;
+    const bool okk = (it.valid >> kChunk) & 1u;
+    cp_async16(sb + KTile::K + lo, kp + it.ko, okk);
+    cp_async16(sb + KTile::V + lo, vp + it.ko, okk);
 #pragma unroll
     for (int k = 0; k < kChunk; ++k) {
-        const int t = it.qt[k];
-        const size_t src = t >= 0 ? (tok0 + t) * rowel + hoff : 0;
-        cp_async16(sb + KTile::Q + 512 * k + lo, a.q + src, t >= 0);
-        cp_async16(sb + KTile::DO + 512 * k + lo, a.dout + src, t >= 0);
+        const bool ok = (it.valid >> k) & 1u;
+        cp_async16(sb + KTile::Q + 512 * k + lo, qp + it.qo[k], ok);
+        cp_async16(sb + KTile::DO + 512 * k + lo, dp + it.qo[k], ok);
     }
-    const uint32_t pr = sb + KTile::PRM;
+    const size_t tok0 = static_cast<size_t>(it.b) * a.N;
     const size_t sa = it.pa >= 0 ? (tok0 + it.pa) * a.H + it.h : 0;
-    cp_async4(pr + 16 * lane, a.lse_in + sa, it.pa >= 0);
-    cp_async4(pr + 16 * lane + 4, a.delta + sa, it.pa >= 0);
+    cp_async4(sb + KTile::LSE + 4 * lane, a.lse_in + sa, it.pa >= 0);
+    cp_async4(sb + KTile::DEL + 4 * lane, a.delta + sa, it.pa >= 0);
     if (lane + 32 < 8 * kChunk) {
         const size_t s2 = it.pb >= 0 ? (tok0 + it.pb) * a.H + it.h : 0;
-        cp_async4(pr + 16 * (lane + 32), a.lse_in + s2, it.pb >= 0);
-        cp_async4(pr + 16 * (lane + 32) + 4, a.delta + s2, it.pb >= 0);
+        cp_async4(sb + KTile::LSE + 4 * (lane + 32), a.lse_in + s2, it.pb >= 0);
+        cp_async4(sb + KTile::DEL + 4 * (lane + 32), a.delta + s2, it.pb >= 0);
     }
 }
 
-// Advance `it` to the next item of the warp's units (b, kc, h) (cluster-major), whose last
-// is unit u_end - 1; returns false past the end.
-__device__ __forceinline__ bool kitem_next(const AttnArgs& a, KItem& it, long long& unit, long long u_end) {
+// A window of list offsets held by the warp: lane j has (first entry, entry count) of the
+// global key cluster base + j (global index b G + kc), so advancing to the next key cluster
+// takes two shuffles instead of a dependent load.
+struct OffWin {
+    unsigned base;
+    int e0, E;
+};
+__device__ __forceinline__ void load_win(const AttnArgs& a, OffWin& w, unsigned base, int lane) {
+    w.base = base;
+    const unsigned c = base + lane;
+    const unsigned b = c / static_cast<unsigned>(a.G);
+    w.e0 = 0;
+    w.E = 0;
+    if (b < static_cast<unsigned>(a.B)) {
+        const int32_t* roff = a.rev_off + static_cast<size_t>(b) * (a.G + 1) + (c - b * a.G);
+        w.e0 = __ldg(roff);
+        w.E = __ldg(roff + 1) - w.e0;
+    }
+}
+
+// Advance `it` (global key cluster c) to the next item of the warp's units (b, kc, h)
+// (cluster-major), whose last is unit u_end - 1; returns false past the end.
+template <typename Off>
+__device__ __forceinline__ bool kitem_next(const AttnArgs& a, KItem<Off>& it, long long& unit, long long u_end,
+                                           unsigned& c, OffWin& w, int lane) {
     if (it.ch + 1 < it.nch) {
         ++it.ch;
         return true;
@@ -852,9 +992,10 @@ __device__ __forceinline__ bool kitem_next(const AttnArgs& a, KItem& it, long lo
             it.kc = 0;
             ++it.b;
         }
-        const int32_t* roff = a.rev_off + static_cast<size_t>(it.b) * (a.G + 1);
-        it.e0 = __ldg(roff + it.kc);
-        it.E = __ldg(roff + it.kc + 1) - it.e0;
+        ++c;
+        if (c - w.base >= 32u) load_win(a, w, c, lane);
+        it.e0 = __shfl_sync(0xffffffffu, w.e0, c - w.base);
+        it.E = __shfl_sync(0xffffffffu, w.E, c - w.base);
         it.nch = it.E > 0 ? (it.E + kChunk - 1) / kChunk : 1;
     }
     return true;
@@ -862,27 +1003,26 @@ __device__ __forceinline__ bool kitem_next(const AttnArgs& a, KItem& it, long lo
 
 // One key-pass item: row parameters in place, then the chunk's pairs; the accumulators
 // carry over the chunks of a (key cluster, head) and are stored after its last chunk.
-__device__ __forceinline__ void key_item(const AttnArgs& a, const KItem& it, uint32_t sb, float4* prm,
-                                         float (&dk)[2][4], float (&dv)[2][4], int lane) {
-    const int gq = lane >> 2, tq = lane & 3, mi = lane >> 3;
+template <typename Off>
+__device__ __forceinline__ void key_item(const AttnArgs& a, const KItem<Off>& it, uint32_t sb, uint8_t* stage,
+                                         const LaneOffs& lo, float (&dk)[2][4], float (&dv)[2][4], int lane) {
+    const int gq = lane >> 2, tq = lane & 3;
     const float a2 = __ldg(a.bias + 3 * it.h) * kLog2e, b2 = __ldg(a.bias + 3 * it.h + 1) * kLog2e,
                 c2 = __ldg(a.bias + 3 * it.h + 2) * kLog2e;
     const float sc = a.scale * kLog2e;
+    float4* prm = reinterpret_cast<float4*>(stage + KTile::PRM);
+    const float* lse = reinterpret_cast<const float*>(stage + KTile::LSE);
+    const float* del = reinterpret_cast<const float*>(stage + KTile::DEL);
     // local origin: the key cluster's first slot
     const float2 org = sh2(it.kxy, 0);
-    {
-        const float4 r = prm[lane];
-        prm[lane] = row_params(it.pxa.x - org.x, it.pxa.y - org.y, it.pa >= 0, r.x, r.y, a2, b2, c2);
-        if (lane + 32 < 8 * kChunk) {
-            const float4 r2 = prm[lane + 32];
-            prm[lane + 32] = row_params(it.pxb.x - org.x, it.pxb.y - org.y, it.pb >= 0, r2.x, r2.y, a2, b2, c2);
-        }
-    }
+    prm[lane] = row_params(it.pxa.x - org.x, it.pxa.y - org.y, it.pa >= 0, lse[lane], del[lane], a2, b2, c2);
+    if (lane + 32 < 8 * kChunk)
+        prm[lane + 32] = row_params(it.pxb.x - org.x, it.pxb.y - org.y, it.pb >= 0, lse[lane + 32], del[lane + 32], a2,
+                                    b2, c2);
     __syncwarp();
     uint32_t kf[4], vf[4];
-    const uint32_t oq = tile64_off(lane & 7, mi);
-    ldsm_x4(sb + KTile::K + oq, kf[0], kf[1], kf[2], kf[3]);
-    ldsm_x4(sb + KTile::V + oq, vf[0], vf[1], vf[2], vf[3]);
+    ldsm_x4(sb + KTile::K + lo.oq, kf[0], kf[1], kf[2], kf[3]);
+    ldsm_x4(sb + KTile::V + lo.oq, vf[0], vf[1], vf[2], vf[3]);
     float kx[2], ky[2], u[2];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
@@ -892,15 +1032,13 @@ __device__ __forceinline__ void key_item(const AttnArgs& a, const KItem& it, uin
         ky[c] = ok ? p.y - org.y : 0.f;
         u[c] = ok ? fmaf(a2, kx[c], fmaf(b2, ky[c], -c2 * fmaf(kx[c], kx[c], ky[c] * ky[c]))) : -INFINITY;
     }
-    const int nq = it.E - kChunk * it.ch;  // listed clusters from this chunk on
-    const int n = nq < kChunk ? nq : kChunk;
-    for (int e = 0; e < n; e += 2) {
-        const bool two = e + 1 < n;
-        const float4 p1 = prm[8 * e + gq];
-        // an absent second block reads the first block's rows with P = 0
-        const float4 p2 = two ? prm[8 * (e + 1) + gq] : make_float4(0.f, 0.f, INFINITY, 0.f);
-        key_pair(sb + KTile::Q, sb + KTile::DO, 8 * e, two ? 8 * (e + 1) : 8 * e, p1, p2, kf, vf, kx, ky, u, sc, dk,
-                 dv);
+    // listed clusters of this chunk; rows of absent ones are zero and their parameters give P = 0
+    const int n = min(it.E - kChunk * it.ch, kChunk);
+#pragma unroll
+    for (int e = 0; e < kChunk; e += 2) {
+        if (e < n)
+            key_pair(sb + KTile::Q, sb + KTile::DO, 512u * e, lo, prm[8 * e + gq], prm[8 * (e + 1) + gq], kf, vf, kx,
+                     ky, u, sc, dk, dv);
     }
     if (it.ch + 1 == it.nch) {
         const int own = __shfl_sync(0xffffffffu, it.kt, gq);
@@ -916,27 +1054,28 @@ __device__ __forceinline__ void key_item(const AttnArgs& a, const KItem& it, uin
 
 // One warp's units [u0, u1) of the key pass (unit = (image, key cluster, head)).  The
 // item cursor runs two items ahead: tokens two items early, coordinates and the gather one.
+template <typename Off>
 __device__ __forceinline__ void key_units(const AttnArgs& a, long long u0, long long u1, uint8_t* wsm) {
     const int lane = threadIdx.x & 31;
     const int H = a.H, G = a.G;
     const uint32_t wb = smem_addr(wsm);
-    KItem cur;
-    {
-        const long long c = u0 / H;
-        cur.h = static_cast<int>(u0 - c * H);
-        cur.b = static_cast<int>(c / G);
-        cur.kc = static_cast<int>(c - static_cast<long long>(cur.b) * G);
-        cur.ch = 0;
-        const int32_t* roff = a.rev_off + static_cast<size_t>(cur.b) * (G + 1);
-        cur.e0 = __ldg(roff + cur.kc);
-        cur.E = __ldg(roff + cur.kc + 1) - cur.e0;
-        cur.nch = cur.E > 0 ? (cur.E + kChunk - 1) / kChunk : 1;
-    }
+    const LaneOffs lo = lane_offs(lane);
+    KItem<Off> cur;
+    unsigned c = static_cast<unsigned>(u0 / H);  // global key cluster of the leading cursor
+    OffWin win;
+    load_win(a, win, c, lane);
+    cur.h = static_cast<int>(u0 - static_cast<long long>(c) * H);
+    cur.b = static_cast<int>(c / static_cast<unsigned>(G));
+    cur.kc = static_cast<int>(c - static_cast<unsigned>(cur.b) * G);
+    cur.ch = 0;
+    cur.e0 = __shfl_sync(0xffffffffu, win.e0, 0);
+    cur.E = __shfl_sync(0xffffffffu, win.E, 0);
+    cur.nch = cur.E > 0 ? (cur.E + kChunk - 1) / kChunk : 1;
     kitem_tokens(a, cur, lane);
     kitem_coords(a, cur);
-    KItem nx = cur;
+    KItem<Off> nx = cur;
     long long unx = u0;
-    bool has_nx = kitem_next(a, nx, unx, u1);
+    bool has_nx = kitem_next(a, nx, unx, u1, c, win, lane);
     if (has_nx) kitem_tokens(a, nx, lane);
     int st = 0;
     kitem_gather(a, cur, wb, lane);
@@ -944,9 +1083,9 @@ __device__ __forceinline__ void key_units(const AttnArgs& a, long long u0, long 
     float dk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     float dv[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     for (;;) {
-        KItem nn = nx;
+        KItem<Off> nn = nx;
         long long unn = unx;
-        const bool has_nn = has_nx && kitem_next(a, nn, unn, u1);
+        const bool has_nn = has_nx && kitem_next(a, nn, unn, u1, c, win, lane);
         if (has_nn) kitem_tokens(a, nn, lane);
         if (has_nx) kitem_coords(a, nx);
         cp_async_wait<0>();
@@ -955,8 +1094,7 @@ __device__ __forceinline__ void key_units(const AttnArgs& a, long long u0, long 
             kitem_gather(a, nx, wb + (st ^ 1) * KTile::STAGE, lane);
             cp_async_commit();
         }
-        key_item(a, cur, wb + st * KTile::STAGE, reinterpret_cast<float4*>(wsm + st * KTile::STAGE + KTile::PRM), dk,
-                 dv, lane);
+        key_item(a, cur, wb + st * KTile::STAGE, wsm + st * KTile::STAGE, lo, dk, dv, lane);
         __syncwarp();
         st ^= 1;
         if (!has_nx) break;
@@ -972,7 +1110,7 @@ __device__ __forceinline__ void key_units(const AttnArgs& a, long long u0, long 
 
 // Resident warps per SM the kernels are built for: the forward 16 (4 CTAs of 4 warps, up
 // to 128 registers), the query pass's larger stage 12, the key pass 16.
-template <int MTILES>
+template <int MTILES, typename Off>
 __global__ void __launch_bounds__(kThreads, MTILES <= 3 ? 4 : 2) attn_fwd_kernel(const AttnArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
@@ -981,21 +1119,28 @@ __global__ void __launch_bounds__(kThreads, MTILES <= 3 ? 4 : 2) attn_fwd_kernel
     const long long W = static_cast<long long>(a.B) * a.G * a.H;
     const long long i0 = gw * W / PW, i1 = (gw + 1) * W / PW;
     if (i0 >= i1) return;
-    cluster_items<MTILES, false>(a, i0, i1, smem + warp * QTile<16 * MTILES, false>::WARP);
+    cluster_items<MTILES, false, Off>(a, i0, i1, smem + warp * QTile<16 * MTILES, false>::WARP);
 }
 
-template <int MTILES>
-__global__ void __launch_bounds__(kThreads, MTILES <= 3 ? 3 : 2) attn_bwd_query_kernel(const AttnArgs a) {
+// The query pass; its first `nprep` CTAs build the reverse index of one image each (when
+// the index fits the kernel's shared memory) while the others run the items.
+template <int MTILES, typename Off>
+__global__ void __launch_bounds__(kThreads, MTILES <= 3 ? 3 : 2) attn_bwd_query_kernel(const AttnArgs a, int nprep) {
     extern __shared__ __align__(16) uint8_t smem[];
+    if (static_cast<int>(blockIdx.x) < nprep) {
+        prep_image_smem(a, blockIdx.x, smem);
+        return;
+    }
     const int warp = threadIdx.x >> 5;
-    const long long PW = static_cast<long long>(gridDim.x) * kWarps;
-    const long long gw = static_cast<long long>(blockIdx.x) * kWarps + warp;
+    const long long PW = static_cast<long long>(gridDim.x - nprep) * kWarps;
+    const long long gw = static_cast<long long>(blockIdx.x - nprep) * kWarps + warp;
     const long long W = static_cast<long long>(a.B) * a.G * a.H;
     const long long i0 = gw * W / PW, i1 = (gw + 1) * W / PW;
     if (i0 >= i1) return;
-    cluster_items<MTILES, true>(a, i0, i1, smem + warp * QTile<16 * MTILES, true>::WARP);
+    cluster_items<MTILES, true, Off>(a, i0, i1, smem + warp * QTile<16 * MTILES, true>::WARP);
 }
 
+template <typename Off>
 __global__ void __launch_bounds__(kThreads, 4) attn_bwd_key_kernel(const AttnArgs a, int P) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1023,7 +1168,7 @@ __global__ void __launch_bounds__(kThreads, 4) attn_bwd_key_kernel(const AttnArg
     const long long W = static_cast<long long>(a.B) * a.G * a.H;
     const long long u0 = gw * W / PW, u1 = (gw + 1) * W / PW;
     if (u0 >= u1) return;
-    key_units(a, u0, u1, smem + warp * KTile::WARP);
+    key_units<Off>(a, u0, u1, smem + warp * KTile::WARP);
 }
 
 // ---------------------------------------------------------------- launchers
@@ -1048,46 +1193,90 @@ int grid_for(long long items, int per_sm) {
     return static_cast<int>(need < slots ? need : slots);
 }
 
-template <int MTILES>
-cudaError_t fwd_dispatch(const AttnArgs& a, cudaStream_t st) {
+// The reverse index: in shared memory when an image fits, else through the workspace.
+cudaError_t launch_prep(const AttnArgs& a, cudaStream_t st) {
+    const size_t sm = 4 * prep_smem_ints(a.N, a.G, a.R);
+    cudaError_t e;
+    if (sm <= 200 * 1024) {
+        e = ensure_smem<attn_bwd_prep_smem_kernel>(sm);
+        if (e != cudaSuccess) return e;
+        attn_bwd_prep_smem_kernel<<<a.B, 256, sm, st>>>(a);
+    } else {
+        const size_t prep = 4 * static_cast<size_t>(a.G + 1) + 160;
+        e = ensure_smem<attn_bwd_prep_kernel>(prep);
+        if (e != cudaSuccess) return e;
+        attn_bwd_prep_kernel<<<a.B, 256, prep, st>>>(a);
+    }
+    note_launch();
+    return cudaGetLastError();
+}
+
+// 32-bit row offsets when every [B][N][H][32] bf16 tensor is smaller than 4 GiB.
+bool narrow_offsets(const AttnArgs& a) {
+    return static_cast<unsigned long long>(a.B) * a.N * a.H * 64ull < (1ull << 32);
+}
+
+template <int MTILES, typename Off>
+cudaError_t fwd_launch(const AttnArgs& a, cudaStream_t st) {
     constexpr int per = MTILES <= 3 ? 4 : 2;
     const size_t smem = static_cast<size_t>(kWarps) * QTile<16 * MTILES, false>::WARP;
-    cudaError_t e = ensure_smem<attn_fwd_kernel<MTILES>>(smem);
+    cudaError_t e = ensure_smem<attn_fwd_kernel<MTILES, Off>>(smem);
     if (e != cudaSuccess) return e;
     const int grid = grid_for(static_cast<long long>(a.B) * a.G * a.H, per);
-    attn_fwd_kernel<MTILES><<<grid, kThreads, smem, st>>>(a);
+    attn_fwd_kernel<MTILES, Off><<<grid, kThreads, smem, st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+}
+
+template <int MTILES>
+cudaError_t fwd_dispatch(const AttnArgs& a, cudaStream_t st) {
+    return narrow_offsets(a) ? fwd_launch<MTILES, uint32_t>(a, st) : fwd_launch<MTILES, uint64_t>(a, st);
+}
+
+// The query pass, with the reverse index built by its leading CTAs when an image's index
+// fits the kernel's shared memory (those CTAs take resident slots from the query items for
+// the few microseconds they run), else by a separate kernel first.
+template <int MTILES, typename Off>
+cudaError_t query_launch(const AttnArgs& a, cudaStream_t st) {
+    constexpr int per = MTILES <= 3 ? 3 : 2;
+    const size_t smem = static_cast<size_t>(kWarps) * QTile<16 * MTILES, true>::WARP;
+    const size_t prep = 4 * prep_smem_ints(a.N, a.G, a.R);
+    const long long slots = static_cast<long long>(sm_count()) * per;
+    int nprep = 0;
+    if (prep <= smem && 2LL * a.B <= slots) {
+        nprep = a.B;
+    } else {
+        const cudaError_t ep = launch_prep(a, st);
+        if (ep != cudaSuccess) return ep;
+    }
+    cudaError_t e = ensure_smem<attn_bwd_query_kernel<MTILES, Off>>(smem);
+    if (e != cudaSuccess) return e;
+    const long long items = static_cast<long long>(a.B) * a.G * a.H;
+    long long P = grid_for(items, per);
+    if (nprep > 0 && P + nprep > slots) P = slots - nprep;
+    attn_bwd_query_kernel<MTILES, Off><<<static_cast<unsigned>(P + nprep), kThreads, smem, st>>>(a, nprep);
+    note_launch();
+    return cudaGetLastError();
+}
+
+// Key pass (+ 3 H bias-reduction CTAs at the end of the grid).
+template <typename Off>
+cudaError_t key_launch(const AttnArgs& a, cudaStream_t st) {
+    const size_t smem = static_cast<size_t>(kWarps) * KTile::WARP;
+    cudaError_t e = ensure_smem<attn_bwd_key_kernel<Off>>(smem);
+    if (e != cudaSuccess) return e;
+    const long long items = static_cast<long long>(a.B) * a.G * a.H;
+    const int P = grid_for(items, 4);
+    attn_bwd_key_kernel<Off><<<P + 3 * a.H, kThreads, smem, st>>>(a, P);
     note_launch();
     return cudaGetLastError();
 }
 
 template <int MTILES>
 cudaError_t bwd_dispatch(const AttnArgs& a, cudaStream_t st) {
-    // prep: reverse index and its tokens, one CTA per image
-    const size_t prep = 4 * static_cast<size_t>(a.G + 1) + 160;
-    cudaError_t e = ensure_smem<attn_bwd_prep_kernel>(prep);
+    const cudaError_t e = narrow_offsets(a) ? query_launch<MTILES, uint32_t>(a, st) : query_launch<MTILES, uint64_t>(a, st);
     if (e != cudaSuccess) return e;
-    attn_bwd_prep_kernel<<<a.B, 256, prep, st>>>(a);
-    note_launch();
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // query pass
-    constexpr int per = MTILES <= 3 ? 3 : 2;
-    const size_t smem = static_cast<size_t>(kWarps) * QTile<16 * MTILES, true>::WARP;
-    e = ensure_smem<attn_bwd_query_kernel<MTILES>>(smem);
-    if (e != cudaSuccess) return e;
-    const long long items = static_cast<long long>(a.B) * a.G * a.H;
-    attn_bwd_query_kernel<MTILES><<<grid_for(items, per), kThreads, smem, st>>>(a);
-    note_launch();
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // key pass (+ 3 H bias-reduction CTAs at the end of the grid)
-    const size_t smem2 = static_cast<size_t>(kWarps) * KTile::WARP;
-    e = ensure_smem<attn_bwd_key_kernel>(smem2);
-    if (e != cudaSuccess) return e;
-    const int P = grid_for(items, 4);
-    attn_bwd_key_kernel<<<P + 3 * a.H, kThreads, smem2, st>>>(a, P);
-    note_launch();
-    return cudaGetLastError();
+    return narrow_offsets(a) ? key_launch<uint32_t>(a, st) : key_launch<uint64_t>(a, st);
 }
 
 }  // namespace

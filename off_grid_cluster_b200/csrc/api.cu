@@ -204,6 +204,7 @@ acl_status acl_cluster_attn_bwd(const acl_bf16* Q, const acl_bf16* K, const acl_
     a.rev_off = reinterpret_cast<int32_t*>(ws + L.rev_off);
     a.rev_list = reinterpret_cast<int32_t*>(ws + L.rev_list);
     a.rev_tok = reinterpret_cast<int32_t*>(ws + L.rev_tok);
+    a.kplan = reinterpret_cast<long long*>(ws + L.kplan);
     return cuda_status(acl::launch_attn_bwd(a, S(stream)));
 }
 

@@ -54,6 +54,7 @@ constexpr int kWarps = 4;               // warps per CTA (independent pipelines)
 constexpr int kThreads = 32 * kWarps;
 constexpr int kRowB = 64;               // bytes of one head of one token (32 bf16)
 constexpr int kChunk = 6;               // listed query clusters per key-pass item
+constexpr int kMaxPlanWarps = 8192;     // key-pass warps a workspace plan can describe
 
 // ---------------------------------------------------------------- small helpers
 
@@ -703,9 +704,9 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const AttnArgs a) {
 // The same index built in shared memory (one CTA per image) when the image fits: the
 // token -> cluster map, the cluster rows, the list entries and their key clusters all live
 // on chip, so the kernel makes one pass over its inputs and one over its outputs.
-// Shared ints: tc[N], cnt[G + 1], lst[G R], ek[G R], cls[8 G], scratch[40].
+// Shared ints: tc[N], cnt[G + 1], lst[G R], ek[G R], cls[8 G], pc[G + 1], scratch[40].
 size_t prep_smem_ints(int N, int G, int R) {
-    return static_cast<size_t>(N) + (G + 1) + 2ull * G * R + 8ull * G + 40;
+    return static_cast<size_t>(N) + (G + 1) + 2ull * G * R + 8ull * G + (G + 1) + 40;
 }
 
 __device__ void prep_image_smem(const AttnArgs& a, int b, uint8_t* smem) {
@@ -716,7 +717,8 @@ __device__ void prep_image_smem(const AttnArgs& a, int b, uint8_t* smem) {
     int* lst = cnt + G + 1;
     int* ek = lst + G * R;
     int* cls = ek + G * R;
-    int* scratch = cls + 8 * G;
+    int* pc = cls + 8 * G;
+    int* scratch = pc + G + 1;
     const int32_t* cl = a.clusters + static_cast<size_t>(b) * G * 8;
     const int32_t* nb = a.nbr + static_cast<size_t>(b) * G * M;
     int32_t* off = a.rev_off + static_cast<size_t>(b) * (G + 1);
@@ -779,9 +781,44 @@ __device__ void prep_image_smem(const AttnArgs& a, int b, uint8_t* smem) {
             lst[j + 1] = v;
         }
     }
+    // key-pass plan: chunk counts per key cluster and their prefix
+    for (int h = tid; h < G; h += nt) {
+        const int E = cnt[h] - (h > 0 ? cnt[h - 1] : 0);
+        pc[h] = E > 0 ? (E + kChunk - 1) / kChunk : 1;
+    }
     __syncthreads();
     for (int i = tid; i < total; i += nt) rlst[i] = lst[i];
     for (int i = tid; i < total * 8; i += nt) rtok[i] = cls[lst[i >> 3] * 8 + (i & 7)];
+    const int S = block_scan_excl(pc, G, scratch);
+    if (tid == 0) pc[G] = S;
+    __syncthreads();
+    if (a.kwarps >= a.B) {
+        // this image's warps of the key pass split its units (key cluster, head) in cluster-
+        // major order so that each gets the same number of chunk items (a unit of key cluster
+        // kc weighs its chunk count)
+        const long long PW = a.kwarps;
+        const int w0 = static_cast<int>((static_cast<long long>(b) * PW + a.B - 1) / a.B);
+        const int w1 = static_cast<int>((static_cast<long long>(b + 1) * PW + a.B - 1) / a.B);
+        const int k = w1 - w0;
+        const long long T = static_cast<long long>(a.H) * S;
+        const long long ub = static_cast<long long>(b) * G * a.H;
+        auto unit_at = [&](long long tau) -> long long {
+            int lo = 0, hi = G;  // largest kc with H pc[kc] <= tau
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (static_cast<long long>(a.H) * pc[mid] <= tau) lo = mid; else hi = mid;
+            }
+            const int nch = pc[lo + 1] - pc[lo];
+            const long long hh = (tau - static_cast<long long>(a.H) * pc[lo]) / nch;
+            return static_cast<long long>(lo) * a.H + hh;
+        };
+        for (int j = tid; j < k; j += nt) {
+            const long long u0 = unit_at(T * j / k);
+            const long long u1 = j + 1 == k ? static_cast<long long>(G) * a.H : unit_at(T * (j + 1) / k);
+            a.kplan[2 * (w0 + j)] = ub + u0;
+            a.kplan[2 * (w0 + j) + 1] = ub + u1;
+        }
+    }
 }
 
 __global__ void __launch_bounds__(256) attn_bwd_prep_smem_kernel(const AttnArgs a) {
@@ -892,20 +929,34 @@ struct KItem {
     float2 pxa, pxb, kxy;
 };
 
-// Tokens and row offsets of an item (coordinates separately, an item later).
+// The raw tokens of an item: the lane's parameter rows (chunk rows lane and lane + 32) and
+// the own cluster row (lanes < 8).  Nothing uses them before the next item step, so the
+// loads have a whole item to land.
 template <typename Off>
 __device__ __forceinline__ void kitem_tokens(const AttnArgs& a, KItem<Off>& it, int lane) {
-    const int G = a.G, N = a.N;
-    const int32_t* rtok = a.rev_tok + static_cast<size_t>(it.b) * G * a.R * 8;
+    const int32_t* rtok = a.rev_tok + static_cast<size_t>(it.b) * a.G * a.R * 8;
     const size_t base = (static_cast<size_t>(it.e0) + static_cast<size_t>(kChunk) * it.ch) * 8;
     const int rem = (it.E - kChunk * it.ch) * 8;
     const int n = rem > 8 * kChunk ? 8 * kChunk : rem;
-    const int gq = lane >> 2;
-    const Off rowb = static_cast<Off>(a.H) * 64u;
-    const Off tb = static_cast<Off>(it.b) * static_cast<Off>(N);
-    // lane l loads chunk rows l and l + 32 (parameter rows); gather rows gq + 8 k arrive by shuffle
     it.pa = lane < n ? __ldg(rtok + base + lane) : -1;
     it.pb = lane + 32 < n ? __ldg(rtok + base + lane + 32) : -1;
+    it.kt = lane < 8 ? __ldg(a.clusters + (static_cast<size_t>(it.b) * a.G + it.kc) * 8 + lane) : -1;
+}
+// An item step later: the tokens made valid, the coordinates requested.
+template <typename Off>
+__device__ __forceinline__ void kitem_coords(const AttnArgs& a, KItem<Off>& it) {
+    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(it.b) * a.N;
+    it.kt = valid_tok(it.kt, a.N);
+    it.pxa = it.pa >= 0 ? __ldg(xyb + it.pa) : make_float2(0.f, 0.f);
+    it.pxb = it.pb >= 0 ? __ldg(xyb + it.pb) : make_float2(0.f, 0.f);
+    it.kxy = it.kt >= 0 ? __ldg(xyb + it.kt) : make_float2(0.f, 0.f);
+}
+// The byte offsets (head 0) of the lane's gather rows: chunk rows gq + 8 k and own row gq.
+template <typename Off>
+__device__ __forceinline__ void kitem_rows(const AttnArgs& a, KItem<Off>& it, int lane) {
+    const int gq = lane >> 2;
+    const Off rowb = static_cast<Off>(a.H) * 64u;
+    const Off tb = static_cast<Off>(it.b) * static_cast<Off>(a.N);
     it.valid = 0u;
 #pragma unroll
     for (int k = 0; k < kChunk; ++k) {
@@ -913,17 +964,9 @@ __device__ __forceinline__ void kitem_tokens(const AttnArgs& a, KItem<Off>& it, 
         it.qo[k] = t >= 0 ? (tb + static_cast<Off>(t)) * rowb : Off(0);
         it.valid |= t >= 0 ? (1u << k) : 0u;
     }
-    it.kt = lane < 8 ? valid_tok(__ldg(a.clusters + (static_cast<size_t>(it.b) * G + it.kc) * 8 + lane), N) : -1;
     const int own = __shfl_sync(0xffffffffu, it.kt, gq);
     it.ko = own >= 0 ? (tb + static_cast<Off>(own)) * rowb : Off(0);
     it.valid |= own >= 0 ? (1u << kChunk) : 0u;
-}
-template <typename Off>
-__device__ __forceinline__ void kitem_coords(const AttnArgs& a, KItem<Off>& it) {
-    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(it.b) * a.N;
-    it.pxa = it.pa >= 0 ? __ldg(xyb + it.pa) : make_float2(0.f, 0.f);
-    it.pxb = it.pb >= 0 ? __ldg(xyb + it.pb) : make_float2(0.f, 0.f);
-    it.kxy = it.kt >= 0 ? __ldg(xyb + it.kt) : make_float2(0.f, 0.f);
 }
 
 template <typename Off>
@@ -1078,6 +1121,7 @@ __device__ __forceinline__ void key_units(const AttnArgs& a, long long u0, long 
     bool has_nx = kitem_next(a, nx, unx, u1, c, win, lane);
     if (has_nx) kitem_tokens(a, nx, lane);
     int st = 0;
+    kitem_rows(a, cur, lane);
     kitem_gather(a, cur, wb, lane);
     cp_async_commit();
     float dk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -1091,6 +1135,7 @@ __device__ __forceinline__ void key_units(const AttnArgs& a, long long u0, long 
         cp_async_wait<0>();
         __syncwarp();
         if (has_nx) {
+            kitem_rows(a, nx, lane);
             kitem_gather(a, nx, wb + (st ^ 1) * KTile::STAGE, lane);
             cp_async_commit();
         }
@@ -1165,8 +1210,16 @@ __global__ void __launch_bounds__(kThreads, 4) attn_bwd_key_kernel(const AttnArg
     }
     const long long PW = static_cast<long long>(P) * kWarps;
     const long long gw = static_cast<long long>(blockIdx.x) * kWarps + warp;
-    const long long W = static_cast<long long>(a.B) * a.G * a.H;
-    const long long u0 = gw * W / PW, u1 = (gw + 1) * W / PW;
+    long long u0, u1;
+    if (a.kwarps == PW && PW >= a.B) {
+        // the plan the reverse-index builders made: equal chunk items per warp
+        u0 = a.kplan[2 * gw];
+        u1 = a.kplan[2 * gw + 1];
+    } else {
+        const long long W = static_cast<long long>(a.B) * a.G * a.H;
+        u0 = gw * W / PW;
+        u1 = (gw + 1) * W / PW;
+    }
     if (u0 >= u1) return;
     key_units<Off>(a, u0, u1, smem + warp * KTile::WARP);
 }
@@ -1180,6 +1233,21 @@ int sm_count() {
     if (cached[dev] == 0) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// Resident CTAs per SM of a kernel at a dynamic shared-memory size (asked of the runtime
+// once per kernel and device).
+template <auto Kern>
+int resident(size_t smem) {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, kThreads, smem) != cudaSuccess || n < 1) n = 1;
         cached[dev] = n;
     }
     return cached[dev];
@@ -1218,10 +1286,10 @@ bool narrow_offsets(const AttnArgs& a) {
 
 template <int MTILES, typename Off>
 cudaError_t fwd_launch(const AttnArgs& a, cudaStream_t st) {
-    constexpr int per = MTILES <= 3 ? 4 : 2;
     const size_t smem = static_cast<size_t>(kWarps) * QTile<16 * MTILES, false>::WARP;
     cudaError_t e = ensure_smem<attn_fwd_kernel<MTILES, Off>>(smem);
     if (e != cudaSuccess) return e;
+    const int per = resident<attn_fwd_kernel<MTILES, Off>>(smem);
     const int grid = grid_for(static_cast<long long>(a.B) * a.G * a.H, per);
     attn_fwd_kernel<MTILES, Off><<<grid, kThreads, smem, st>>>(a);
     note_launch();
@@ -1238,8 +1306,10 @@ cudaError_t fwd_dispatch(const AttnArgs& a, cudaStream_t st) {
 // the few microseconds they run), else by a separate kernel first.
 template <int MTILES, typename Off>
 cudaError_t query_launch(const AttnArgs& a, cudaStream_t st) {
-    constexpr int per = MTILES <= 3 ? 3 : 2;
     const size_t smem = static_cast<size_t>(kWarps) * QTile<16 * MTILES, true>::WARP;
+    cudaError_t e = ensure_smem<attn_bwd_query_kernel<MTILES, Off>>(smem);
+    if (e != cudaSuccess) return e;
+    const int per = resident<attn_bwd_query_kernel<MTILES, Off>>(smem);
     const size_t prep = 4 * prep_smem_ints(a.N, a.G, a.R);
     const long long slots = static_cast<long long>(sm_count()) * per;
     int nprep = 0;
@@ -1249,8 +1319,6 @@ cudaError_t query_launch(const AttnArgs& a, cudaStream_t st) {
         const cudaError_t ep = launch_prep(a, st);
         if (ep != cudaSuccess) return ep;
     }
-    cudaError_t e = ensure_smem<attn_bwd_query_kernel<MTILES, Off>>(smem);
-    if (e != cudaSuccess) return e;
     const long long items = static_cast<long long>(a.B) * a.G * a.H;
     long long P = grid_for(items, per);
     if (nprep > 0 && P + nprep > slots) P = slots - nprep;
@@ -1261,19 +1329,30 @@ cudaError_t query_launch(const AttnArgs& a, cudaStream_t st) {
 
 // Key pass (+ 3 H bias-reduction CTAs at the end of the grid).
 template <typename Off>
+int key_grid(const AttnArgs& a) {
+    const size_t smem = static_cast<size_t>(kWarps) * KTile::WARP;
+    if (ensure_smem<attn_bwd_key_kernel<Off>>(smem) != cudaSuccess) return 1;
+    return grid_for(static_cast<long long>(a.B) * a.G * a.H, resident<attn_bwd_key_kernel<Off>>(smem));
+}
+
+template <typename Off>
 cudaError_t key_launch(const AttnArgs& a, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(kWarps) * KTile::WARP;
     cudaError_t e = ensure_smem<attn_bwd_key_kernel<Off>>(smem);
     if (e != cudaSuccess) return e;
-    const long long items = static_cast<long long>(a.B) * a.G * a.H;
-    const int P = grid_for(items, 4);
+    const int P = key_grid<Off>(a);
     attn_bwd_key_kernel<Off><<<P + 3 * a.H, kThreads, smem, st>>>(a, P);
     note_launch();
     return cudaGetLastError();
 }
 
 template <int MTILES>
-cudaError_t bwd_dispatch(const AttnArgs& a, cudaStream_t st) {
+cudaError_t bwd_dispatch(const AttnArgs& a0, cudaStream_t st) {
+    AttnArgs a = a0;
+    const long long kw =
+        static_cast<long long>(narrow_offsets(a) ? key_grid<uint32_t>(a) : key_grid<uint64_t>(a)) * kWarps;
+    const bool plan = kw <= kMaxPlanWarps && 4 * prep_smem_ints(a.N, a.G, a.R) <= 200 * 1024;
+    a.kwarps = plan ? static_cast<int>(kw) : 0;
     const cudaError_t e = narrow_offsets(a) ? query_launch<MTILES, uint32_t>(a, st) : query_launch<MTILES, uint64_t>(a, st);
     if (e != cudaSuccess) return e;
     return narrow_offsets(a) ? key_launch<uint32_t>(a, st) : key_launch<uint64_t>(a, st);
@@ -1293,6 +1372,7 @@ AttnWorkspace attn_workspace_layout(int B, int N, int H, int C, int M) {
     w.rev_off = off;     off += up(sizeof(int32_t) * B * (G + 1));
     w.rev_list = off;    off += up(sizeof(int32_t) * B * G * R);
     w.rev_tok = off;     off += up(sizeof(int32_t) * B * G * R * 8);
+    w.kplan = off;       off += up(sizeof(long long) * 2 * kMaxPlanWarps);
     w.total = off;
     return w;
 }

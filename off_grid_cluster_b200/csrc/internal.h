@@ -71,10 +71,12 @@ struct AttnArgs {
     int32_t* rev_off;    // [B][G + 1]
     int32_t* rev_list;   // [B][G * R]
     int32_t* rev_tok;    // [B][G * R][8] query tokens of every reverse-list entry
+    long long* kplan;    // [kwarps][2] key-pass unit range of every warp (see attn.cu)
+    int kwarps;          // warps of the key pass the plan is made for (0: no plan)
 };
 
 struct AttnWorkspace {
-    size_t delta, dbias_part, tok_cluster, rev_off, rev_list, rev_tok, total;
+    size_t delta, dbias_part, tok_cluster, rev_off, rev_list, rev_tok, kplan, total;
 };
 AttnWorkspace attn_workspace_layout(int B, int N, int H, int C, int M);
 

@@ -45,7 +45,7 @@
 #include <omp.h>
 #endif
 
-/* Thread count of the batch drivers (OpenMP over images); returns the count in use. */
+/* Thread count of the batch drivers (OpenMP); returns the count in use. */
 int orc_set_threads(int n) {
 #ifdef _OPENMP
     if (n > 0) omp_set_num_threads(n);
@@ -233,11 +233,13 @@ static int attn_logits(const double* q, const double* k, const float* xy,
     return any;
 }
 
-int orc_attn_fwd(const double* q, const double* k, const double* v, const float* xy,
-                 const int32_t* clusters, const int32_t* nbr, const double* bias,
-                 int N, int H, int D, int C, int M, double scale,
-                 double* o, double* lse) {
-    if (N < 1 || H < 1 || D < 1 || C < 1 || M < 1) return 1;
+/* The forward for heads [h0, h1) only (heads are independent; o and lse of the other
+ * heads are left untouched). */
+static int attn_fwd_heads(const double* q, const double* k, const double* v, const float* xy,
+                          const int32_t* clusters, const int32_t* nbr, const double* bias,
+                          int N, int H, int D, int C, int M, double scale, int h0, int h1,
+                          double* o, double* lse) {
+    if (N < 1 || H < 1 || D < 1 || C < 1 || M < 1 || h0 < 0 || h1 > H) return 1;
     int G = (N + C - 1) / C;
     double* s = (double*)malloc(sizeof(double) * (size_t)M);
     int* valid = (int*)malloc(sizeof(int) * (size_t)M);
@@ -247,7 +249,7 @@ int orc_attn_fwd(const double* q, const double* k, const double* v, const float*
         for (int sl = 0; sl < C; ++sl) {
             int32_t i = clusters[(size_t)g * C + sl];
             if (i < 0) continue;
-            for (int h = 0; h < H; ++h) {
+            for (int h = h0; h < h1; ++h) {
                 double* oi = o + ((size_t)i * H + h) * D;
                 for (int e = 0; e < D; ++e) oi[e] = 0.0;
                 if (!attn_logits(q, k, xy, nrow, bias, i, h, H, D, M, scale, s, valid)) {
@@ -272,6 +274,13 @@ int orc_attn_fwd(const double* q, const double* k, const double* v, const float*
     return 0;
 }
 
+int orc_attn_fwd(const double* q, const double* k, const double* v, const float* xy,
+                 const int32_t* clusters, const int32_t* nbr, const double* bias,
+                 int N, int H, int D, int C, int M, double scale,
+                 double* o, double* lse) {
+    return attn_fwd_heads(q, k, v, xy, clusters, nbr, bias, N, H, D, C, M, scale, 0, H, o, lse);
+}
+
 /*
  * Backward by recomputation, from the definition of the forward:
  *   P_ij = exp(s_ij - lse_i), dP_ij = <dO_i, v_j>, Delta_i = <dO_i, o_i>,
@@ -282,11 +291,16 @@ int orc_attn_fwd(const double* q, const double* k, const double* v, const float*
  * o and lse are this oracle's own forward results.  Coordinates get no
  * gradient.  dq, dk, dv are overwritten; dbias [H][3] is overwritten.
  */
-int orc_attn_bwd(const double* q, const double* k, const double* v, const float* xy,
-                 const int32_t* clusters, const int32_t* nbr, const double* bias,
-                 int N, int H, int D, int C, int M, double scale, const double* dout,
-                 double* dq, double* dk, double* dv, double* dbias) {
-    if (N < 1 || H < 1 || D < 1 || C < 1 || M < 1) return 1;
+/* The backward for heads [h0, h1) only: dq, dk, dv of those heads and dbias[h0..h1)
+ * are overwritten, the other heads are left untouched.  Every sum keeps the order of the
+ * all-heads loop (clusters, slots, then keys), since a head's sums never mix with
+ * another head's. */
+static int attn_bwd_heads(const double* q, const double* k, const double* v, const float* xy,
+                          const int32_t* clusters, const int32_t* nbr, const double* bias,
+                          int N, int H, int D, int C, int M, double scale, int h0, int h1,
+                          const double* dout, double* dq, double* dk, double* dv,
+                          double* dbias) {
+    if (N < 1 || H < 1 || D < 1 || C < 1 || M < 1 || h0 < 0 || h1 > H) return 1;
     int G = (N + C - 1) / C;
     size_t nel = (size_t)N * H * D;
     double* o = (double*)malloc(sizeof(double) * nel);
@@ -294,18 +308,24 @@ int orc_attn_bwd(const double* q, const double* k, const double* v, const float*
     double* s = (double*)malloc(sizeof(double) * (size_t)M);
     int* valid = (int*)malloc(sizeof(int) * (size_t)M);
     if (!o || !lse || !s || !valid) { free(o); free(lse); free(s); free(valid); return 2; }
-    int rc = orc_attn_fwd(q, k, v, xy, clusters, nbr, bias, N, H, D, C, M, scale, o, lse);
+    int rc = attn_fwd_heads(q, k, v, xy, clusters, nbr, bias, N, H, D, C, M, scale, h0, h1,
+                            o, lse);
     if (rc) { free(o); free(lse); free(s); free(valid); return rc; }
-    memset(dq, 0, sizeof(double) * nel);
-    memset(dk, 0, sizeof(double) * nel);
-    memset(dv, 0, sizeof(double) * nel);
-    memset(dbias, 0, sizeof(double) * (size_t)H * 3);
+    for (int t = 0; t < N; ++t)
+        for (int h = h0; h < h1; ++h)
+            for (int e = 0; e < D; ++e) {
+                size_t x = ((size_t)t * H + h) * D + e;
+                dq[x] = 0.0;
+                dk[x] = 0.0;
+                dv[x] = 0.0;
+            }
+    for (int h = h0; h < h1; ++h) dbias[3 * h] = dbias[3 * h + 1] = dbias[3 * h + 2] = 0.0;
     for (int g = 0; g < G; ++g) {
         const int32_t* nrow = nbr + (size_t)g * M;
         for (int sl = 0; sl < C; ++sl) {
             int32_t i = clusters[(size_t)g * C + sl];
             if (i < 0) continue;
-            for (int h = 0; h < H; ++h) {
+            for (int h = h0; h < h1; ++h) {
                 if (!attn_logits(q, k, xy, nrow, bias, i, h, H, D, M, scale, s, valid)) continue;
                 const double L = lse[(size_t)i * H + h];
                 const double* doi = dout + ((size_t)i * H + h) * D;
@@ -341,6 +361,14 @@ int orc_attn_bwd(const double* q, const double* k, const double* v, const float*
     }
     free(o); free(lse); free(s); free(valid);
     return 0;
+}
+
+int orc_attn_bwd(const double* q, const double* k, const double* v, const float* xy,
+                 const int32_t* clusters, const int32_t* nbr, const double* bias,
+                 int N, int H, int D, int C, int M, double scale, const double* dout,
+                 double* dq, double* dk, double* dv, double* dbias) {
+    return attn_bwd_heads(q, k, v, xy, clusters, nbr, bias, N, H, D, C, M, scale, 0, H, dout,
+                          dq, dk, dv, dbias);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -818,7 +846,7 @@ int orc_dec_offsets_bwd(const double* f, const double* dq, const double* df_out,
 }
 
 /* ------------------------------------------------------------------------ */
-/* batch drivers: images are independent; OpenMP over images only            */
+/* batch drivers: images are independent (attention: image x head)           */
 /* ------------------------------------------------------------------------ */
 
 int orc_cluster_batch(const float* xy, int B, int N, int C, int32_t* clusters) {
@@ -845,14 +873,17 @@ int orc_attn_fwd_batch(const double* q, const double* k, const double* v, const 
                        double* o, double* lse) {
     int G = (N + C - 1) / C, rc = 0;
     size_t st = (size_t)N * H * D;
-    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    #pragma omp parallel for collapse(2) schedule(dynamic) reduction(|:rc)
     for (int b = 0; b < B; ++b)
-        rc |= orc_attn_fwd(q + b * st, k + b * st, v + b * st, xy + (size_t)b * N * 2,
-                           clusters + (size_t)b * G * C, nbr + (size_t)b * G * M, bias,
-                           N, H, D, C, M, scale, o + b * st, lse + (size_t)b * N * H);
+        for (int h = 0; h < H; ++h)
+            rc |= attn_fwd_heads(q + b * st, k + b * st, v + b * st, xy + (size_t)b * N * 2,
+                                 clusters + (size_t)b * G * C, nbr + (size_t)b * G * M, bias,
+                                 N, H, D, C, M, scale, h, h + 1, o + b * st,
+                                 lse + (size_t)b * N * H);
     return rc;
 }
 
+/* dbias sums the images' partial sums in image order, after the parallel loop. */
 int orc_attn_bwd_batch(const double* q, const double* k, const double* v, const float* xy,
                        const int32_t* clusters, const int32_t* nbr, const double* bias,
                        int B, int N, int H, int D, int C, int M, double scale,
@@ -862,12 +893,13 @@ int orc_attn_bwd_batch(const double* q, const double* k, const double* v, const 
     size_t st = (size_t)N * H * D;
     double* part = (double*)calloc((size_t)B * H * 3, sizeof(double));
     if (!part) return 2;
-    #pragma omp parallel for schedule(dynamic) reduction(|:rc)
+    #pragma omp parallel for collapse(2) schedule(dynamic) reduction(|:rc)
     for (int b = 0; b < B; ++b)
-        rc |= orc_attn_bwd(q + b * st, k + b * st, v + b * st, xy + (size_t)b * N * 2,
-                           clusters + (size_t)b * G * C, nbr + (size_t)b * G * M, bias,
-                           N, H, D, C, M, scale, dout + b * st, dq + b * st, dk + b * st,
-                           dv + b * st, part + (size_t)b * H * 3);
+        for (int h = 0; h < H; ++h)
+            rc |= attn_bwd_heads(q + b * st, k + b * st, v + b * st, xy + (size_t)b * N * 2,
+                                 clusters + (size_t)b * G * C, nbr + (size_t)b * G * M, bias,
+                                 N, H, D, C, M, scale, h, h + 1, dout + b * st, dq + b * st,
+                                 dk + b * st, dv + b * st, part + (size_t)b * H * 3);
     for (int j = 0; j < H * 3; ++j) {
         double acc = 0.0;
         for (int b = 0; b < B; ++b) acc += part[(size_t)b * H * 3 + j];

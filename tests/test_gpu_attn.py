@@ -114,16 +114,11 @@ def test_zero_query_zero_bias_is_mean():
             np.testing.assert_allclose(host(O)[0, i], v[keys].mean(axis=0), atol=1e-2)
 
 
-# Capacities of the kernels' shared-memory unions (blocks of 8 token rows), used below to
-# show that the hub table reaches every overflow path.
-FWD_STAGE_BLOCKS = 24     # forward / query pass: one pipeline stage
-KEY_STAGE_BLOCKS = 20     # key pass: one pipeline stage
-KEY_MAX_ENTRIES = 128     # key pass: reverse-list entries of one group
-
-
-def _groups(G):
-    ng = (G + 7) // 8
-    return [(gi * G // ng, (gi + 1) * G // ng) for gi in range(ng)]
+# The key pass walks a key cluster's reverse list in chunks of this many listed query
+# clusters, carrying the dK / dV accumulators across chunks; its warps read list offsets
+# through a window of this many consecutive key clusters.
+KEY_CHUNK = 6
+OFFSET_WINDOW = 32
 
 
 def hub_table(cl: np.ndarray, M: int, seed: int) -> np.ndarray:
@@ -143,33 +138,30 @@ def hub_table(cl: np.ndarray, M: int, seed: int) -> np.ndarray:
 
 
 @pytest.mark.parametrize("M", [48, 64])
-def test_hub_table_overflow_paths(M):
-    """A hand-built table in which every cluster lists cluster 0.  The unions of a group's
-    neighbour blocks exceed one pipeline stage (single-buffered stage) and, at M = 64, two
-    stages (the group is processed in halves); the reverse list of cluster 0 holds every
-    cluster, so its key group overflows the key pass's union and takes the per-warp direct
-    path.  The assertions on the table's geometry show that each path is reached; the
-    parity checks cover all of them against the oracle."""
+def test_hub_table_long_reverse_lists(M):
+    """A hand-built table in which every cluster lists cluster 0.  The reverse list of
+    cluster 0 then holds every query cluster of the image, so its key-pass units run many
+    chunks with accumulators carried between them, while the other key clusters have short
+    lists; the per-warp plan balances chunk items, so one warp's range starts and ends in the
+    middle of the hub's list and the offset window is refilled across image boundaries.  The
+    assertions show the table has these shapes; the parity checks cover them against the
+    oracle."""
     a = synth.attn_stage1(B=2, N=700, H=3)
     cl = oracle.cluster(a.coords, 8)
     nb = hub_table(cl, M, seed=11 + M)
     B, G, _ = cl.shape
     R = M // 8
-    fwd_unions, key_entries, key_unions = [], [], []
+    lens = []
     for b in range(B):
         first = {int(cl[b, g, 0]): g for g in range(G)}
-        rev = [[] for _ in range(G)]
+        rev = [0] * G
         for g in range(G):
             for r in range(R):
-                rev[first[int(nb[b, g, r * 8])]].append(g)
-        for c0, c1 in _groups(G):
-            fwd_unions.append(len({tuple(nb[b, g, r * 8:(r + 1) * 8]) for g in range(c0, c1) for r in range(R)}))
-            ents = [q for k in range(c0, c1) for q in rev[k]]
-            key_entries.append(len(ents))
-            key_unions.append(len(set(ents)))
-    assert max(fwd_unions) > FWD_STAGE_BLOCKS                    # single-buffered stage
-    if M == 64:
-        assert max(fwd_unions) > 2 * FWD_STAGE_BLOCKS            # halves of the group
-    assert max(key_entries) > KEY_MAX_ENTRIES or max(key_unions) > 2 * KEY_STAGE_BLOCKS  # direct
-    assert min(key_unions) <= 2 * KEY_STAGE_BLOCKS               # and a union path beside it
+                rev[first[int(nb[b, g, r * 8])]] += 1
+        lens.append(rev)
+    lens = np.array(lens)
+    assert lens[:, 0].min() == G                          # the hub is listed by every cluster
+    assert lens.max() > 4 * KEY_CHUNK                     # many chunks for one unit
+    assert np.median(lens) <= KEY_CHUNK                   # and single-chunk units beside it
+    assert B * G > OFFSET_WINDOW                          # window refills
     run_attn(a, M=M, cl=cl, nb=nb)

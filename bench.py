@@ -1,33 +1,37 @@
 #!/usr/bin/env python
 """Benchmark of the off-grid cluster attention + KNN gather hot path on B200.
 
-One *step* is one pass of every step of the path over one batch of seeded
-synthetic input shaped like the AFFMAE pages' stage-1 workload at 1024 px
-(8 images, a 64 x 64 patch grid with a value-noise mask keeping 2048 tokens per
-image, dim 128 = 4 heads x 32, C = 8, M = 48), followed by the decoder's
-KNN gather over that stage (4096 queries per image at cell centre + U(-1,1)^2,
-K = 8, d = 128, one temperature per head):
+One *step* is one pass of every step of the path over the two largest seeded synthetic
+workloads, shaped like the AFFMAE pages' 1024 px encoder and decoder ("A Complete
+Example": a 64 x 64 patch grid, 2048 visible tokens, then 819 / 328 / 131 after each
+down-sampling):
 
-    attention chain: acl_cluster -> acl_neighbors -> acl_cluster_attn_fwd
-                     -> acl_cluster_attn_bwd
-    KNN chain:       acl_knn_table -> (acl_knn_gather_index || acl_knn_gather_fwd)
-                     -> acl_knn_gather_bwd_indexed
+  encoder sweep   16 images; four stages of 2048 / 819 / 328 / 131 tokens (nested random
+                  subsets, ratio 0.4) with dims 128 / 256 / 512 / 768 (4 / 8 / 16 / 24
+                  heads x 32) and 3 / 4 / 16 / 2 layers, C = 8, M = 48, distinct Q / K / V
+                  / dO buffers per layer.  Forward over the stages (acl_cluster ->
+                  acl_neighbors -> acl_cluster_attn_fwd per layer), then the backward in
+                  reverse (acl_cluster_attn_bwd per layer).
+  decoder gather  16 images x 4096 queries (cell centre + U(-1, 1)^2) over each of the
+                  four stages' tokens (d = 128 ... 768), K = 8, one temperature per head:
+                  acl_knn_table -> acl_knn_gather_fwd -> acl_knn_gather_bwd per stage.
 
-`value` is whole-job tokens/s: images x tokens processed by all ranks per second
-of the slowest rank's device time.  Inputs sit in HBM before timing starts;
-S input sets rotate so that the sets total at least 4x the L2 size.  Each set's
-two chains are captured as two CUDA graphs and replayed on two streams (the
-attention chain, the longer one, at the higher priority; the inverse index on a
-third stream inside the KNN graph).  CUDA events inside the graphs time every
-call; the roofline figure is taken for the call with the largest share of the
-step.  `e2e` runs the same calls through the C entry points with every step's
-inputs copied in from pinned host buffers and all of its outputs read back, the
-copies pipelined against the neighbouring steps' compute.
+`value` is the encoder sweep's cluster-attention tokens/s: token-layers (images x tokens,
+summed over the 25 layers, all ranks) per second of the sweep's device time; the sweep's
+time includes its clustering and neighbour tables.  `knn` gives the decoder gather's
+queries/s the same way (queries x stages over the gather's device time, tables included).
+Both spans are measured with CUDA events inside the timed steps; ms_per_step is their sum.
+The inputs of one step (about 1.4 GB) are larger than the 126 MB L2, so no flush is
+needed between steps; each step is one CUDA graph of the library calls with CUDA events
+between the calls.  `roofline` and `roofline_knn` name the call with the largest share of
+each span and divide its algorithmic bytes per launch by its mean launch time.  `e2e`
+runs the same calls through the public entry points with every step's inputs copied in
+from pinned host memory and all outputs read back, copies pipelined against compute.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl acl|reference]
 
-With --impl reference the fp64 CPU oracle is timed on the host cores on a
-bounded sample of the same workload (rank 0 only under torchrun).
+With --impl reference the fp64 CPU oracle is timed on the host cores on a bounded sample
+of the same workload (rank 0 only under torchrun).
 """
 from __future__ import annotations
 
@@ -47,30 +51,34 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "cluster-attn fwd+bwd tokens/s & KNN-gather queries/s; % of B200 HBM roofline"
-WORKLOAD = "stage1-1024px-b8-n2048-d128-h4-c8-m48 + decoder-knn-gather-q4096-k8"
+IMAGES = 16                                   # images per rank
+STAGE_TOKENS = (2048, 819, 328, 131)
+STAGE_DIMS = (128, 256, 512, 768)
+STAGE_LAYERS = (3, 4, 16, 2)
+QUERIES, KNN_K, GRID = 4096, 8, 64
+WORKLOAD = ("encoder-sweep-1024px-b16-n2048/819/328/131-d128/256/512/768-layers3/4/16/2-c8-m48"
+            " + decoder-knn-gather-b16-q4096-k8-over-the-4-stages")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-OPS = ("cluster", "neighbors", "attn_fwd", "attn_bwd", "knn_table", "knn_index", "knn_fwd",
-       "knn_bwd")
+# the kernels behind each call
 KERNELS = {
     "cluster": ["cluster_kernel"],
     "neighbors": ["neighbors_kernel"],
-    "attn_fwd": ["attn_fwd_union_kernel"],
-    "attn_bwd": ["attn_bwd_query_union_kernel", "attn_bwd_key_union_kernel"],
+    "attn_fwd": ["attn_fwd_kernel"],
+    "attn_bwd": ["attn_bwd_query_kernel", "attn_bwd_key_kernel"],
     "knn_table": ["knn_table_kernel"],
-    "knn_index": ["knn_csr_kernel"],
-    "knn_fwd": ["knn_fwd_shared_kernel"],
-    "knn_bwd": ["knn_bwd_query_shared_kernel", "knn_bwd_token_kernel"],
+    "knn_fwd": ["knn_fwd_*"],
+    "knn_bwd": ["knn_keys_kernel", "knn_csr_*", "knn_bwd_query_*", "knn_bwd_token_*"],
 }
-# DRAM bytes per launch measured by ncu for each call (sum over its kernels), with the
-# sha256 of the CUDA source the counters were taken on; a stale hash reports null.
-NCU_TRAFFIC: dict[str, tuple[float, str, str]] = {
-    # call: (DRAM bytes read + written per launch, hash of the sources of its kernels, summary)
-    "attn_fwd": (13202176.0, "77c27f1c2b1cfe11", "profiles/attn_kernels_step_workload.md"),
-    "attn_bwd": (35377408.0, "77c27f1c2b1cfe11", "profiles/attn_kernels_step_workload.md"),
+# the files whose code makes each call's kernels: a DRAM-traffic figure taken by ncu on
+# other sources than the current ones is stale and is reported as null
+TRAFFIC_SOURCES = {
+    "attn_fwd": ("attn.cu", "common.cuh", "internal.h"),
+    "attn_bwd": ("attn.cu", "common.cuh", "internal.h"),
+    "knn_fwd": ("knn.cu", "common.cuh", "internal.h"),
+    "knn_bwd": ("knn.cu", "common.cuh", "internal.h"),
 }
-# the files whose code makes each call's kernels (the traffic goes stale when they change)
-TRAFFIC_SOURCES = {"attn_fwd": ("attn.cu", "common.cuh"), "attn_bwd": ("attn.cu", "common.cuh")}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
 
 # --------------------------------------------------------------------------- helpers
@@ -85,21 +93,23 @@ def env_int(name: str, default: int) -> int:
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("acl", "reference"), default="acl")
-    ap.add_argument("--batch", type=int, default=8, help="images per rank (default 8)")
+    ap.add_argument("--batch", type=int, default=IMAGES, help="images per rank (default 16)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=50)
-    ap.add_argument("--serial", action="store_true",
-                    help="run all seven calls on one stream (default: the attention and KNN "
-                         "chains run as two concurrent branches of the step graph)")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the extra parts (per-layer configurations, token merging, "
+                         "high-resolution gather, decoder layers)")
+    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded CPU work of the oracle baseline (seconds)")
-    ap.add_argument("--only", choices=("token_merge", "decoder", "configs"), default=None,
-                    help="time one extra part alone on one GPU and print its JSON (a short "
-                         "command to profile under ncu); no bench line")
+    ap.add_argument("--only", choices=("token_merge", "decoder", "configs", "attn_stage", "knn_stage"),
+                    default=None,
+                    help="run one part alone on one GPU and print its JSON (a short command to "
+                         "profile under ncu); no bench line")
+    ap.add_argument("--stage", type=int, default=3, help="stage (1-4) of --only attn_stage / knn_stage")
     return ap.parse_args(argv)
 
 
@@ -131,7 +141,7 @@ def measured_peaks() -> dict:
         with open(path) as f:
             d = json.load(f)
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d.get("bf16_tflops", FALLBACK_BF16_TFLOPS)),
-                "source": "measured (MEASURED_PEAKS.json)"}
+                "source": "measured (copy bandwidth and bf16 GEMM on this pool's B200s)"}
     return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
             "source": "fallback 6.65 TB/s, 1590 TFLOP/s"}
 
@@ -146,22 +156,75 @@ def source_hash(names=None) -> str:
     return h.hexdigest()[:16]
 
 
-def algorithmic_bytes(B, N, H, Q, d, K, GH, GW, C=8, M=48) -> dict:
-    """Bytes each call must move at least once (every tensor counted once)."""
+# --------------------------------------------------------------------------- byte counts
+
+def attn_bytes(B: int, N: int, H: int) -> dict:
+    """Algorithmic bytes of one attention call, every tensor once: per (token, head) the
+    forward moves Q, K, V, O (64 B each in bf16) and the lse (4 B) = 260 B, the backward
+    Q, K, V, O, dO, lse and dQ, dK, dV = 516 B; per token 72 B of coordinates, cluster
+    list and neighbour-table share."""
+    return {"attn_fwd": B * N * (260 * H + 72), "attn_bwd": B * N * (516 * H + 72)}
+
+
+def knn_bytes(B: int, Q: int, N: int, d: int, K: int = KNN_K) -> dict:
+    """Algorithmic bytes of one gather call: per query the forward reads its position (8 B)
+    and table row (4K B) and writes d bf16 channels; the backward reads position, table row
+    and dOut and writes dq (8 B); per token the features (2d B) and coordinates (8 B) are
+    read once and the backward writes dF (2d B)."""
+    return {"knn_fwd": B * (Q * (8 + 4 * K + 2 * d) + N * (2 * d + 8)),
+            "knn_bwd": B * (Q * (8 + 4 * K + 8 + 2 * d) + N * (4 * d + 8))}
+
+
+def table_bytes(B: int, N: int, C: int = 8, M: int = 48, GH: int = GRID, GW: int = GRID,
+                K: int = KNN_K) -> dict:
+    """Clustering, neighbour table and KNN table: coordinates in, index tables out."""
     G = (N + C - 1) // C
-    per_tok_meta = 8 + 4 + 4 * M * G / N           # coords, cluster slot, neighbour-table share
-    return {
-        "cluster": B * N * (8 + 4),
-        "neighbors": B * (N * 8 + G * C * 4 + G * M * 4),
-        "attn_fwd": B * N * (H * (3 * 64 + 64 + 4) + per_tok_meta) + H * 12,
-        "attn_bwd": B * N * (H * (4 * 64 + 4 + 3 * 64) + per_tok_meta) + 2 * H * 12,
-        "knn_table": B * (N * 8 + GH * GW * K * 4),
-        "knn_index": B * (Q * 8 + GH * GW * K * 4 + Q * K * 4 + (N + 1) * 4),
-        "knn_fwd": B * (Q * (8 + 4 * K + 2 * d) + N * (2 * d + 8)) + 4 * d // 32,
-        "knn_bwd": B * (Q * (8 + 4 * K + 2 * d + 8) + N * (2 * d + 8 + 2 * d)) + 8 * d // 32,
-    }
+    return {"cluster": B * N * (8 + 4), "neighbors": B * (N * 8 + G * C * 4 + G * M * 4),
+            "knn_table": B * (N * 8 + GH * GW * K * 4)}
 
 
+def merge_bytes(B: int, N: int, d: int, k: int) -> dict:
+    """Algorithmic bytes of token merging, every tensor once: forward reads features (2d B)
+    and coordinates (8 B) per token and writes score, assignment (8 B) per token and the merged
+    row (2d + 8 B) and anchor id per anchor; backward reads features, coordinates, score and
+    assignment and writes dfeats and dcoords per token (4d + 24 B), reads dmerged (2d + 8 B)
+    per anchor."""
+    T, A = B * N, B * k
+    return {"fwd": T * (2 * d + 16) + A * (2 * d + 12), "bwd": T * (4 * d + 24) + A * (2 * d + 8)}
+
+
+def read_traffic(path: str = TRAFFIC_FILE) -> list[dict]:
+    """Rows of the committed ncu DRAM-traffic summary: lines `key = value; key = value ...`
+    with call, workload, read, write (bytes per launch) and src (hash of the call's sources
+    the counters were taken on); other lines are ignored."""
+    rows = []
+    if not os.path.exists(path):
+        return rows
+    with open(path) as f:
+        for line in f:
+            if not line.startswith("traffic:"):
+                continue
+            row = {}
+            for part in line[len("traffic:"):].split(";"):
+                if "=" in part:
+                    k, v = part.split("=", 1)
+                    row[k.strip()] = v.strip()
+            if {"call", "workload", "read", "write", "src"} <= row.keys():
+                rows.append(row)
+    return rows
+
+
+def traffic_for(call: str, workload: str, rows: list[dict]) -> dict | None:
+    """DRAM bytes per launch of `call` on `workload` if a capture on the current sources
+    exists, else None."""
+    if call not in TRAFFIC_SOURCES:
+        return None
+    h = source_hash(TRAFFIC_SOURCES[call])
+    for r in rows:
+        if r["call"] == call and r["workload"] == workload and r["src"] == h:
+            rd, wr = float(r["read"]), float(r["write"])
+            return {"read": rd, "write": wr, "total": rd + wr}
+    return None
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
 
@@ -210,121 +273,153 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
-# --------------------------------------------------------------------------- GPU arm
+# --------------------------------------------------------------------------- workload
 
-class StepSet:
-    """Device buffers of one input set plus the seven library calls of a step."""
+def _pinned(torch, x: np.ndarray, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(x)).to(dtype)
+    return t.pin_memory()
 
-    def __init__(self, sb, device, acl, torch):
-        a, k = sb.attn, sb.knn
-        T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
-        bf = torch.bfloat16
-        self.acl, self.torch = acl, torch
-        self.B, self.N, self.H, self.Q, self.d, self.K = a.B, a.N, a.H, k.Q, k.d, k.K
-        self.GH, self.GW, self.scale = k.GH, k.GW, a.scale
-        self.inputs = {
-            "coords": T(a.coords), "q": T(a.q, bf), "k": T(a.k, bf), "v": T(a.v, bf),
-            "do": T(a.do, bf), "bias": T(a.bias), "queries": T(k.queries),
-            "feats": T(k.feats, bf), "dout": T(k.dout, bf), "p": T(k.p),
-        }
-        B, N, H, G = self.B, self.N, self.H, (self.N + 7) // 8
+
+class HostWorkload:
+    """The seeded inputs of one rank's step in pinned host memory (bf16 tensors as bf16):
+    per encoder stage its coordinates, bias coefficients and every layer's Q / K / V / dO;
+    per decoder stage its queries, token features, coordinates, temperatures and dOut."""
+
+    def __init__(self, B: int, image0: int, torch, pin: bool = True, layers: int | None = None):
+        """`layers` limits the layers generated per stage (the oracle's sample needs one);
+        `pin` False keeps plain host tensors (no CUDA context needed)."""
+        from off_grid_cluster_b200 import synth
+        bf, f32 = torch.bfloat16, torch.float32
+        self.B = B
+        self.layer_counts = list(STAGE_LAYERS)
+        host = _pinned if pin else (lambda _t, x, dt: torch.from_numpy(np.ascontiguousarray(x)).to(dt))
+        self.stages = []
+        for s, xy in enumerate(synth.sweep_coords(B, image0)):
+            layers_s = []
+            for layer in range(STAGE_LAYERS[s] if layers is None else min(layers, STAGE_LAYERS[s])):
+                ab = synth.attn_sweep_layer(xy, s, layer, image0)
+                layers_s.append({n: host(torch, getattr(ab, n), bf) for n in ("q", "k", "v", "do")})
+            self.stages.append({"coords": host(torch, xy, f32), "bias": host(torch, ab.bias, f32),
+                                "scale": float(ab.scale), "N": int(xy.shape[1]), "H": int(ab.q.shape[2]),
+                                "layers": layers_s})
+        self.knn = []
+        for kb in synth.knn_decoder(B, image0):
+            self.knn.append({"queries": host(torch, kb.queries, f32), "feats": host(torch, kb.feats, bf),
+                             "coords": host(torch, kb.coords, f32), "p": host(torch, kb.p, f32),
+                             "dout": host(torch, kb.dout, bf), "N": int(kb.N), "d": int(kb.d),
+                             "Q": int(kb.Q), "GH": int(kb.GH), "GW": int(kb.GW), "K": int(kb.K)})
+
+    def token_layers(self) -> int:
+        return sum(self.B * st["N"] * L for st, L in zip(self.stages, self.layer_counts))
+
+    def query_stages(self) -> int:
+        return sum(self.B * k["Q"] for k in self.knn)
+
+
+class DeviceStep:
+    """Device copies of a HostWorkload's inputs, the outputs of every call and the calls of
+    one step in order (`calls`: (kind, stage, fn) with fn(stream) issuing one library call)."""
+
+    def __init__(self, hw: HostWorkload, device, torch, acl):
+        self.torch, self.acl, self.B = torch, acl, hw.B
+        dev = lambda t: t.to(device, non_blocking=False)
         e = lambda shape, dt: torch.empty(shape, dtype=dt, device=device)
-        self.outputs = {
-            "clusters": e((B, G, 8), torch.int32), "nbr": e((B, G, 48), torch.int32),
-            "o": e((B, N, H, 32), bf), "lse": e((B, N, H), torch.float32),
-            "dq": e((B, N, H, 32), bf), "dk": e((B, N, H, 32), bf), "dv": e((B, N, H, 32), bf),
-            "dbias": e((H, 3), torch.float32),
-            "table": e((B, self.GH, self.GW, self.K), torch.int32),
-            "out": e((B, self.Q, self.d), bf), "dfeats": e((B, N, self.d), bf),
-            "dqueries": e((B, self.Q, 2), torch.float32), "dp": e((self.d // 32,), torch.float32),
-        }
-        self.ws_attn = e((acl.acl_cluster_attn_workspace(B, N, H, 8, 48),), torch.uint8)
-        self.ws_knn = e((acl.acl_knn_gather_workspace(B, self.Q, N, self.d, self.K),), torch.uint8)
+        bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+        B = hw.B
+        self.ins, self.outs = [], []            # (device, host) input pairs; device outputs
+        self.stages = []
+        ws_attn = 0
+        for st in hw.stages:
+            N, H = st["N"], st["H"]
+            G = (N + 7) // 8
+            d = {"coords": dev(st["coords"]), "bias": dev(st["bias"]), "scale": st["scale"], "N": N, "H": H,
+                 "clusters": e((B, G, 8), i32), "nbr": e((B, G, 48), i32), "layers": []}
+            self.ins += [(d["coords"], st["coords"]), (d["bias"], st["bias"])]
+            self.outs += [d["clusters"], d["nbr"]]
+            for hl in st["layers"]:
+                L = {n: dev(hl[n]) for n in ("q", "k", "v", "do")}
+                self.ins += [(L[n], hl[n]) for n in ("q", "k", "v", "do")]
+                L.update(o=e((B, N, H, 32), bf), lse=e((B, N, H), f32), dq=e((B, N, H, 32), bf),
+                         dk=e((B, N, H, 32), bf), dv=e((B, N, H, 32), bf), dbias=e((H, 3), f32))
+                self.outs += [L[n] for n in ("o", "lse", "dq", "dk", "dv", "dbias")]
+                d["layers"].append(L)
+            ws_attn = max(ws_attn, acl.acl_cluster_attn_workspace(B, N, H, 8, 48))
+            self.stages.append(d)
+        self.knn = []
+        ws_knn = 0
+        for k in hw.knn:
+            d = {n: dev(k[n]) for n in ("queries", "feats", "coords", "p", "dout")}
+            self.ins += [(d[n], k[n]) for n in ("queries", "feats", "coords", "p", "dout")]
+            d.update(GH=k["GH"], GW=k["GW"], K=k["K"],
+                     table=e((B, k["GH"], k["GW"], k["K"]), i32), out=e((B, k["Q"], k["d"]), bf),
+                     dfeats=e((B, k["N"], k["d"]), bf), dq=e((B, k["Q"], 2), f32), dp=e((k["d"] // 32,), f32))
+            self.outs += [d[n] for n in ("table", "out", "dfeats", "dq", "dp")]
+            ws_knn = max(ws_knn, acl.acl_knn_gather_workspace(B, k["Q"], k["N"], k["d"], k["K"]))
+            self.knn.append(d)
+        # the calls run one at a time on one stream, so one workspace of each kind serves all
+        self.ws_attn = e((max(ws_attn, 1),), torch.uint8)
+        self.ws_knn = e((max(ws_knn, 1),), torch.uint8)
+        self.calls = self._calls()
 
     def bytes(self) -> int:
-        ts = list(self.inputs.values()) + list(self.outputs.values()) + [self.ws_attn, self.ws_knn]
+        ts = [t for t, _ in self.ins] + self.outs + [self.ws_attn, self.ws_knn]
         return sum(t.numel() * t.element_size() for t in ts)
 
-    def op(self, name: str, stream, kind: int = 0):
-        i, o, acl = self.inputs, self.outputs, self.acl
-        if name == "cluster":
-            acl.acl_cluster(i["coords"], 8, clusters=o["clusters"], stream=stream)
-        elif name == "neighbors":
-            acl.acl_neighbors(i["coords"], o["clusters"], 48, nbr=o["nbr"], stream=stream)
-        elif name == "attn_fwd":
-            acl.acl_cluster_attn_fwd(i["q"], i["k"], i["v"], i["coords"], o["clusters"], o["nbr"],
-                                     i["bias"], self.scale, O=o["o"], lse=o["lse"], stream=stream)
-        elif name == "attn_bwd":
-            acl.acl_cluster_attn_bwd(i["q"], i["k"], i["v"], i["coords"], o["clusters"], o["nbr"],
-                                     i["bias"], self.scale, o["o"], i["do"], o["lse"], o["dq"],
-                                     o["dk"], o["dv"], o["dbias"], workspace=self.ws_attn,
-                                     stream=stream)
-        elif name == "knn_table":
-            acl.acl_knn_table(i["coords"], self.GH, self.GW, self.K, table=o["table"], stream=stream)
-        elif name == "knn_fwd":
-            acl.acl_knn_gather_fwd(i["queries"], i["feats"], i["coords"], o["table"], i["p"],
-                                   out=o["out"], stream=stream, kind=kind)
-        elif name == "knn_index":
-            acl.acl_knn_gather_index(i["queries"], o["table"], self.N, self.d, self.ws_knn,
-                                     stream=stream)
-        elif name == "knn_bwd":
-            acl.acl_knn_gather_bwd_indexed(i["queries"], i["feats"], i["coords"], o["table"],
-                                           i["p"], i["dout"], self.ws_knn, dfeats=o["dfeats"],
-                                           dqueries=o["dqueries"], dp=o["dp"], stream=stream,
-                                           kind=kind)
-        else:
-            raise KeyError(name)
+    def _calls(self):
+        acl, calls = self.acl, []
+        for s, d in enumerate(self.stages):
+            calls.append(("cluster", s, lambda st, d=d: acl.acl_cluster(d["coords"], 8, clusters=d["clusters"],
+                                                                         stream=st)))
+            calls.append(("neighbors", s, lambda st, d=d: acl.acl_neighbors(d["coords"], d["clusters"], 48,
+                                                                             nbr=d["nbr"], stream=st)))
+            for L in d["layers"]:
+                calls.append(("attn_fwd", s, lambda st, d=d, L=L: acl.acl_cluster_attn_fwd(
+                    L["q"], L["k"], L["v"], d["coords"], d["clusters"], d["nbr"], d["bias"], d["scale"],
+                    O=L["o"], lse=L["lse"], stream=st)))
+        for s in reversed(range(len(self.stages))):
+            d = self.stages[s]
+            for L in reversed(d["layers"]):
+                calls.append(("attn_bwd", s, lambda st, d=d, L=L: acl.acl_cluster_attn_bwd(
+                    L["q"], L["k"], L["v"], d["coords"], d["clusters"], d["nbr"], d["bias"], d["scale"],
+                    L["o"], L["do"], L["lse"], L["dq"], L["dk"], L["dv"], L["dbias"],
+                    workspace=self.ws_attn, stream=st)))
+        for s, k in enumerate(self.knn):
+            calls.append(("knn_table", s, lambda st, k=k: acl.acl_knn_table(k["coords"], k["GH"], k["GW"], k["K"],
+                                                                             table=k["table"], stream=st)))
+            calls.append(("knn_fwd", s, lambda st, k=k: acl.acl_knn_gather_fwd(
+                k["queries"], k["feats"], k["coords"], k["table"], k["p"], out=k["out"], stream=st)))
+            calls.append(("knn_bwd", s, lambda st, k=k: acl.acl_knn_gather_bwd(
+                k["queries"], k["feats"], k["coords"], k["table"], k["p"], k["dout"], k["dfeats"], k["dq"],
+                k["dp"], workspace=self.ws_knn, stream=st)))
+        return calls
 
-    ATTN = ("cluster", "neighbors", "attn_fwd", "attn_bwd")
-    KNN = ("knn_table", "knn_index", "knn_fwd", "knn_bwd")
+    def first_knn(self) -> int:
+        return next(i for i, c in enumerate(self.calls) if c[0].startswith("knn"))
 
-    def chain(self, names, stream, events=None, s3=None):
-        """The calls of one chain in order on `stream`; with s3 the inverse index runs on
-        s3 after the table and the indexed backward waits for it."""
-        torch = self.torch
-        tab, idx = torch.cuda.Event(), torch.cuda.Event()
-        for name in names:
-            j = OPS.index(name)
-            st = s3 if (name == "knn_index" and s3 is not None) else stream
-            if name == "knn_index" and s3 is not None:
-                s3.wait_event(tab)
-            if name == "knn_bwd" and s3 is not None:
-                stream.wait_event(idx)
+    def step(self, stream, events=None):
+        """Every call of the step on `stream`; events[2j], events[2j + 1] bracket call j."""
+        for j, (_, _, fn) in enumerate(self.calls):
             if events is not None:
-                events[2 * j].record(st)
-            self.op(name, st)
+                events[2 * j].record(stream)
+            fn(stream)
             if events is not None:
-                events[2 * j + 1].record(st)
-            if name == "knn_table":
-                tab.record(stream)
-            if name == "knn_index":
-                idx.record(st)
+                events[2 * j + 1].record(stream)
 
-    def step(self, stream, events=None, streams=None):
-        """The eight calls.  With streams = (s2, s3) the KNN chain (table -> gather fwd ->
-        indexed bwd; the inverse index on s3 after the table) runs on s2 concurrently with
-        the attention chain (cluster -> neighbours -> attn fwd -> bwd) on stream;
-        events[2j], events[2j+1] bracket call j on its stream."""
-        if streams is None:
-            self.chain(OPS, stream, events)
-            return
-        torch = self.torch
-        s2, s3 = streams
-        fork, join = torch.cuda.Event(), torch.cuda.Event()
-        fork.record(stream)
-        s2.wait_event(fork)
-        self.chain(StepSet.ATTN, stream, events)
-        self.chain(StepSet.KNN, s2, events, s3=s3)
-        join.record(s2)
-        stream.wait_event(join)
 
+def call_workload(kind: str, B: int, N: int, H: int = 0, d: int = 0, Q: int = QUERIES) -> str:
+    """Canonical name of one launch shape (the key of the DRAM-traffic summary)."""
+    if kind.startswith("attn") or kind in ("cluster", "neighbors"):
+        return f"b{B}-n{N}-h{H}"
+    return f"b{B}-q{Q}-n{N}-d{d}"
+
+
+# --------------------------------------------------------------------------- GPU arm
 
 def run_gpu(args, rank: int, world: int):
     import torch
     import torch.distributed as dist
 
     import off_grid_cluster_b200 as acl
-    from off_grid_cluster_b200 import synth
 
     local = env_int("LOCAL_RANK", 0)
     torch.cuda.set_device(local)
@@ -337,87 +432,36 @@ def run_gpu(args, rank: int, world: int):
         if world > 1:
             dist.barrier()
 
-
     first, per_rank = shard_images(rank, world, args.batch)
-    sb = synth.step_batch(B=per_rank, image0=first)
+    hw = HostWorkload(per_rank, first, torch)
+    ds = DeviceStep(hw, device, torch, acl)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    base = StepSet(sb, device, acl, torch)
-    set_bytes = base.bytes()
-    n_sets = max(2, math.ceil(4 * l2 / set_bytes))
-    sets = [base] + [StepSet(sb, device, acl, torch) for _ in range(n_sets - 1)]
-    # the attention chain is the longer one: its stream gets the higher priority so its
-    # CTAs are scheduled first and the KNN chain fills the remaining SMs
-    # (a lower number is a higher priority; out-of-range values map to the nearest valid one)
-    stream = torch.cuda.Stream(device, priority=-100)
-    streams = None if args.serial else (torch.cuda.Stream(device, priority=0),
-                                        torch.cuda.Stream(device, priority=0))
-
-    # eager warm-up of every call (kernel attributes, lazy module loading), then capture
+    stream = torch.cuda.Stream(device)
+    # eager pass of every call (kernel attributes, lazy module loading), then capture
     with torch.cuda.stream(stream):
-        for s in sets:
-            s.step(stream)
+        ds.step(stream)
     stream.synchronize()
-    n_ev = 2 * len(OPS)
+    n_calls = len(ds.calls)
+    reps = max(1, min(args.steps, 3))       # graph copies with their own events, replayed in turn
     graphs, events = [], []
     launches0 = acl.acl_launch_count()
-    for s in sets:
-        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
-        if streams is None:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                s.step(stream, evs)
-            graphs.append((g,))
-        else:
-            # one graph per chain, replayed on its own stream (graph nodes run at the
-            # priority of the stream the graph is launched into)
-            ga, gk = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-            with torch.cuda.graph(ga, stream=stream):
-                s.chain(StepSet.ATTN, stream, evs)
-            with torch.cuda.graph(gk, stream=streams[0]):
-                s.chain(StepSet.KNN, streams[0], evs, s3=streams[1])
-            graphs.append((ga, gk))
+    for _ in range(reps):
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * n_calls)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            ds.step(stream, evs)
+        graphs.append(g)
         events.append(evs)
-    launches_per_step = (acl.acl_launch_count() - launches0) // len(sets)
-    # single-stream graphs of the same sets: the per-call breakdown and the roofline come
-    # from these, where no call shares the GPU with another
-    serial_graphs, serial_events = [], []
-    if streams is None:
-        serial_graphs, serial_events = [gs[0] for gs in graphs], events
-    else:
-        for s in sets:
-            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                s.step(stream, evs)
-            serial_graphs.append(g)
-            serial_events.append(evs)
+    launches_per_step = (acl.acl_launch_count() - launches0) // reps
     torch.cuda.synchronize()
 
     def replay(i):
-        gs = graphs[i % n_sets]
-        if len(gs) == 1:
-            with torch.cuda.stream(stream):
-                gs[0].replay()
-            return
         with torch.cuda.stream(stream):
-            gs[0].replay()
-        with torch.cuda.stream(streams[0]):
-            gs[1].replay()
+            graphs[i % reps].replay()
 
-    def fork():
-        if streams is not None:
-            streams[0].wait_stream(stream)
-
-    def join():
-        if streams is not None:
-            stream.wait_stream(streams[0])
-
-    fork()
     for w in range(args.warmup):
         replay(w)
-    join()
     torch.cuda.synchronize()
-
     props = torch.cuda.get_device_properties(device)
     uuid = getattr(props, "uuid", None)
     clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local)).start()
@@ -426,135 +470,178 @@ def run_gpu(args, rank: int, world: int):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    fork()
+    # the last `reps` replays fill every graph copy's events
     for it in range(args.steps):
         replay(it)
-    join()
     t1.record(stream)
     torch.cuda.synchronize()
     barrier()
     step_ms_local = t0.elapsed_time(t1) / max(args.steps, 1)
-    def per_call(evsets, used):
-        acc = np.zeros(len(OPS))
-        for s_i in range(used):
-            ev = evsets[s_i]
-            acc += np.array([ev[2 * j].elapsed_time(ev[2 * j + 1]) for j in range(len(OPS))])
-        return acc / max(used, 1)
-
-    # per-call durations inside the timed region (the last replay of every set); with
-    # concurrent chains each includes the time it shared the GPU with the other chain
-    per_op_concurrent = per_call(events, min(n_sets, args.steps))
-    # per-call durations with one call at a time: 2 rounds over the sets, after warm-up
-    with torch.cuda.stream(stream):
-        for it in range(3 * n_sets):
-            serial_graphs[it % n_sets].replay()
-    torch.cuda.synchronize()
-    per_op = per_call(serial_events, n_sets)
-    # the inverse-power weight kernel (the original AFF weighting) on the same gathers:
-    # forward and backward of set 0, one call at a time
-    inv_us = {}
-    s0 = sets[0]
-    for name in ("knn_fwd", "knn_bwd"):
-        for kind, key in ((acl.ACL_KNN_EXP, "exp"), (acl.ACL_KNN_INVPOW, "invpow")):
-            inv_us[f"{name}_{key}"] = graph_time(
-                torch, stream, lambda: s0.op(name, stream, kind=kind), 20)
-    hires = hires_gather_times(torch, acl, synth, device, stream) if world == 1 else None
-    merge_us = (token_merge_times(torch, acl, synth, sb, device, stream, measured_peaks())
-                if world == 1 else None)
-    dec_us = decoder_times(torch, acl, synth, device, stream, measured_peaks()) if world == 1 else None
-    cfg_us = config_times(torch, acl, synth, device, stream, measured_peaks()) if world == 1 else None
+    # per-call durations of the last timed replay of every graph copy
+    dur = np.zeros(n_calls)
+    span_a, span_k = 0.0, 0.0
+    kf = ds.first_knn()
+    for evs in events:
+        dur += np.array([evs[2 * j].elapsed_time(evs[2 * j + 1]) for j in range(n_calls)])
+        span_a += evs[0].elapsed_time(evs[2 * kf - 1])
+        span_k += evs[2 * kf].elapsed_time(evs[2 * n_calls - 1])
+    dur /= reps
+    span_a /= reps
+    span_k /= reps
     # keep the same load on the GPU until the clock sampler has several samples
     t_wall = time.time()
     it = 0
     while time.time() - t_wall < 0.8:
-        fork()
-        for _ in range(64):
+        for _ in range(8):
             replay(it)
             it += 1
-        join()
         stream.synchronize()
     torch.cuda.synchronize()
     clk = clocks.stop()
 
     step_ms = max_over_ranks(step_ms_local, world, device)
-    B, N, Q = per_rank, sb.attn.N, sb.knn.Q
-    tokens = world * B * N
-    value = tokens / (step_ms * 1e-3)
-    abytes = algorithmic_bytes(B, N, sb.attn.H, Q, sb.knn.d, sb.knn.K, sb.knn.GH, sb.knn.GW)
-    dom = int(np.argmax(per_op))
-    dom_name = OPS[dom]
+    span_a = max_over_ranks(span_a, world, device)
+    span_k = max_over_ranks(span_k, world, device)
     peaks = measured_peaks()
-    achieved = abytes[dom_name] / (per_op[dom] * 1e-3) / 1e9
-    traffic = None
-    traffic_src = None
-    if dom_name in NCU_TRAFFIC and NCU_TRAFFIC[dom_name][1] == source_hash(TRAFFIC_SOURCES[dom_name]):
-        traffic, traffic_src = NCU_TRAFFIC[dom_name][0], NCU_TRAFFIC[dom_name][2]
-    breakdown = {}
-    for j, name in enumerate(OPS):
-        gbs = abytes[name] / (per_op[j] * 1e-3) / 1e9
-        breakdown[name] = {"us": round(per_op[j] * 1e3, 2), "alg_MB": round(abytes[name] / 1e6, 3),
-                           "GB_s": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
-    attn_ms = per_op[OPS.index("attn_fwd")] + per_op[OPS.index("attn_bwd")]
-    knn_ms = sum(per_op[OPS.index(n)] for n in ("knn_index", "knn_fwd", "knn_bwd"))
+    hbm = peaks["hbm_gbs"]
+    B = per_rank
+    token_layers = world * hw.token_layers()
+    query_stages = world * hw.query_stages()
+    value = token_layers / (span_a * 1e-3)
+    knn_value = query_stages / (span_k * 1e-3)
+
+    # per (call, stage) groups: launches, mean launch time, algorithmic bytes per launch
+    groups = {}
+    for j, (kind, s, _) in enumerate(ds.calls):
+        g = groups.setdefault((kind, s), {"kind": kind, "stage": s, "launches": 0, "ms": 0.0})
+        g["launches"] += 1
+        g["ms"] += dur[j]
+    for (kind, s), g in groups.items():
+        if kind in ("knn_table", "knn_fwd", "knn_bwd"):
+            k = hw.knn[s]
+            by = {**knn_bytes(B, k["Q"], k["N"], k["d"], k["K"]), **table_bytes(B, k["N"])}
+            g["workload"] = call_workload(kind, B, k["N"], d=k["d"], Q=k["Q"])
+        else:
+            st = hw.stages[s]
+            by = {**attn_bytes(B, st["N"], st["H"]), **table_bytes(B, st["N"])}
+            g["workload"] = call_workload(kind, B, st["N"], H=st["H"])
+        g["bytes"] = by[kind]
+        g["us"] = g["ms"] / g["launches"] * 1e3
+        g["GB_s"] = g["bytes"] / (g["us"] * 1e-6) / 1e9
+        g["frac"] = g["GB_s"] / hbm
+    traffic_rows = read_traffic()
+
+    def roofline(kinds, what):
+        cand = [g for g in groups.values() if g["kind"] in kinds]
+        g = max(cand, key=lambda x: x["ms"])
+        tr = traffic_for(g["kind"], g["workload"], traffic_rows)
+        return {"bound": "hbm", "achieved": round(g["GB_s"], 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(g["frac"], 4), "traffic": None if tr is None else int(tr["total"]),
+                "traffic_read": None if tr is None else int(tr["read"]),
+                "traffic_write": None if tr is None else int(tr["write"]),
+                "traffic_basis": ("ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, one eager "
+                                  "launch of this shape on the current sources (--cache-control none)"
+                                  if tr is not None else "no capture on the current sources"),
+                "call": f"acl_{g['kind']}", "kernels": KERNELS[g["kind"]],
+                "launch_workload": g["workload"], "stage": g["stage"] + 1,
+                "launches_per_step": g["launches"], "share_of_span": round(g["ms"] / what, 4),
+                "alg_bytes_per_launch": int(g["bytes"]), "launch_us": round(g["us"], 3),
+                "peak_source": peaks["source"] + " (burst copy)", "of": "measured" if "measured" in peaks["source"]
+                else "fallback"}
+
+    attn_kinds = ("cluster", "neighbors", "attn_fwd", "attn_bwd")
+    knn_kinds = ("knn_table", "knn_fwd", "knn_bwd")
+    rf_attn = roofline(attn_kinds, span_a)
+    rf_knn = roofline(knn_kinds, span_k)
+
+    def span_of(kinds):
+        """(device ms per step, fraction of HBM) of every launch of the given calls"""
+        ms = sum(g["ms"] for g in groups.values() if g["kind"] in kinds)
+        by = sum(g["bytes"] * g["launches"] for g in groups.values() if g["kind"] in kinds)
+        return ms, by / (ms * 1e-3) / 1e9 / hbm
+    attn_fb_ms, attn_fb_frac = span_of(("attn_fwd", "attn_bwd"))
+    knn_fb_ms, knn_fb_frac = span_of(("knn_fwd", "knn_bwd"))
+    per_stage = []
+    for s, st in enumerate(hw.stages):
+        f, b = groups[("attn_fwd", s)], groups[("attn_bwd", s)]
+        per_stage.append({"stage": s + 1, "N": st["N"], "H": st["H"], "layers": f["launches"],
+                          "cluster_us": round(groups[("cluster", s)]["us"], 2),
+                          "neighbors_us": round(groups[("neighbors", s)]["us"], 2),
+                          "fwd_us": round(f["us"], 2), "bwd_us": round(b["us"], 2),
+                          "fwd_frac": round(f["frac"], 4), "bwd_frac": round(b["frac"], 4),
+                          "fwd_bwd_frac": round((f["bytes"] + b["bytes"]) / ((f["us"] + b["us"]) * 1e-6)
+                                                / 1e9 / hbm, 4)})
+    knn_stage = []
+    for s, k in enumerate(hw.knn):
+        t, f, b = groups[("knn_table", s)], groups[("knn_fwd", s)], groups[("knn_bwd", s)]
+        knn_stage.append({"stage": s + 1, "N": k["N"], "d": k["d"], "table_us": round(t["us"], 2),
+                          "fwd_us": round(f["us"], 2), "bwd_us": round(b["us"], 2),
+                          "fwd_frac": round(f["frac"], 4), "bwd_frac": round(b["frac"], 4),
+                          "fwd_bwd_frac": round((f["bytes"] + b["bytes"]) / ((f["us"] + b["us"]) * 1e-6)
+                                                / 1e9 / hbm, 4)})
+
+    extras = None
+    if world == 1 and not args.no_extras:
+        from off_grid_cluster_b200 import synth
+        extras = {
+            "configs": config_times(torch, acl, synth, device, stream, peaks),
+            "token_merge_us": token_merge_times(torch, acl, synth, device, stream, peaks),
+            "hires_gather_us": hires_gather_times(torch, acl, synth, device, stream),
+            "decoder_us": decoder_times(torch, acl, synth, device, stream, peaks),
+        }
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, base, stream, streams, torch, acl, tokens_per_step=world * B * N,
-                      sb=sb, device=device)
+        e2e = run_e2e(args, hw, ds, stream, torch, acl, device)
         e2e_ms = max_over_ranks(e2e.pop("_ms"), world, device)
-        e2e["value"] = round(world * B * N / (e2e_ms * 1e-3), 1)
-        e2e["ms_per_step"] = round(e2e_ms, 4)
+        e2e["ms_per_step"] = round(e2e_ms, 3)
+        e2e["value"] = round(token_layers / (e2e_ms * 1e-3), 1)
+        e2e["knn_value"] = round(query_stages / (e2e_ms * 1e-3), 1)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args, sb)
+        cpu = cpu_baseline(args, per_rank)
 
+    set_mb = ds.bytes() / 1e6
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; shapes of the pages' 1024 px stage-1 workload)",
-        "config": {"workload": WORKLOAD, "images_per_gpu": B, "tokens_per_image": N,
-                   "heads": sb.attn.H, "head_dim": 32, "C": 8, "M": 48,
-                   "queries_per_image": Q, "knn_d": sb.knn.d, "K": sb.knn.K, "grid": [64, 64],
-                   "l2": f"rotating {n_sets} input sets, {n_sets * set_bytes / 1e6:.0f} MB total "
-                         f">= 4 x L2 ({l2 / 1e6:.0f} MB)",
-                   "timing": "CUDA graph per set, CUDA events on the launching stream",
-                   "streams": "1" if args.serial else "3 (attention chain at high priority)",
+        "data": "synthetic (seeded; shapes of the pages' 1024 px encoder and decoder workloads)",
+        "config": {"workload": WORKLOAD, "images_per_gpu": B, "stage_tokens": [st["N"] for st in hw.stages],
+                   "stage_heads": [st["H"] for st in hw.stages],
+                   "stage_layers": [len(st["layers"]) for st in hw.stages], "head_dim": 32, "C": 8, "M": 48,
+                   "knn_queries_per_image": QUERIES, "knn_stage_d": [k["d"] for k in hw.knn], "K": KNN_K,
+                   "grid": [GRID, GRID],
+                   "l2": f"inputs + outputs of one step {set_mb:.0f} MB > L2 {l2 / 1e6:.0f} MB: no flush "
+                         f"between steps",
+                   "timing": f"one CUDA graph per step ({reps} copies replayed in turn), CUDA events on the "
+                             f"launching stream around the steps and between the calls",
                    "parallelism": f"replicas x{world} (images sharded, no collective)"},
+        "value_basis": "encoder token-layers of all ranks / the encoder sweep's device time per step "
+                       "(clustering and neighbour tables included; mean of the last timed steps, max over "
+                       "ranks)",
+        "segments_ms": {"encoder_sweep": round(span_a, 4), "decoder_gather": round(span_k, 4)},
+        "knn": {"value": round(knn_value, 1), "unit": "queries/s",
+                "basis": "decoder queries x stages of all ranks / the gather's device time per step "
+                         "(KNN tables included)",
+                "gather_fwd_bwd_queries_per_s": round(query_stages / (knn_fb_ms * 1e-3), 1),
+                "gather_fwd_bwd_frac": round(knn_fb_frac, 4), "stages": knn_stage},
+        "roofline": rf_attn,
+        "roofline_knn": rf_knn,
         "parts": {
-            "knn_queries_per_s": round(world * B * Q / (step_ms * 1e-3), 1),
-            "cluster_attn_fwd_bwd_tokens_per_s": round(world * B * N / (attn_ms * 1e-3), 1),
-            "knn_gather_fwd_bwd_queries_per_s": round(world * B * Q / (knn_ms * 1e-3), 1),
-            "per_call": breakdown,
-            "per_call_note": "one call at a time (single-stream graphs of the same sets, "
-                             "after the timed region); the step overlaps the two chains",
-            "per_call_concurrent_us": {n: round(per_op_concurrent[j] * 1e3, 2)
-                                       for j, n in enumerate(OPS)},
-            "knn_kernels_us": {**inv_us, "note": "exponential and inverse-power weight kernels "
-                               "on the same gathers (set 0, one graph per call, L2-warm)"},
-            "hires_gather_us": hires,
-            "token_merge_us": merge_us,
-            "decoder_us": dec_us,
-            "configs": cfg_us,
+            "attn_fwd_bwd_tokens_per_s": round(token_layers / (attn_fb_ms * 1e-3), 1),
+            "attn_fwd_bwd_frac": round(attn_fb_frac, 4),
+            "attn_stages": per_stage,
+            "extras": extras,
         },
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "traffic": traffic, "traffic_unit": "bytes per launch (ncu DRAM read + write)",
-                     "traffic_source": traffic_src, "kernel": f"acl_{dom_name} ({', '.join(KERNELS[dom_name])})",
-                     "alg_bytes_per_launch": int(abytes[dom_name]),
-                     "launch_us": round(per_op[dom] * 1e3, 3), "peak_source": peaks["source"]},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": clk,
     }
-    for gs in graphs:
-        for g in gs:
-            g.reset()
-    if streams is not None:
-        for g in serial_graphs:
-            g.reset()
+    for g in graphs:
+        g.reset()
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -583,21 +670,116 @@ def graph_time(torch, stream, fn, reps: int = 10) -> float:
     return round(e0.elapsed_time(e1) / reps * 1e3, 2)
 
 
-def merge_bytes(B: int, N: int, d: int, k: int) -> dict:
-    """Algorithmic bytes of token merging, every tensor once: forward reads features (2d B)
-    and coordinates (8 B) per token and writes score, assignment (8 B) per token and the merged
-    row (2d + 8 B) and anchor id per anchor; backward reads features, coordinates, score and
-    assignment and writes dfeats and dcoords per token (4d + 24 B), reads dmerged (2d + 8 B)
-    per anchor."""
-    T, A = B * N, B * k
-    return {"fwd": T * (2 * d + 16) + A * (2 * d + 12), "bwd": T * (4 * d + 24) + A * (2 * d + 8)}
+def run_e2e(args, hw: HostWorkload, ds: DeviceStep, stream, torch, acl, device) -> dict:
+    """The step through the public entry points from pinned host memory, copies inside.
+
+    Every step copies all of its inputs host -> device and all of its outputs device ->
+    host.  Two device sets and two copy streams pipeline the steps: the inputs of step
+    k + 1 travel in and the outputs of step k - 1 travel out while step k computes (PCIe
+    is full duplex), with events ordering each set's copy-in, compute and copy-out."""
+    sets = [ds, DeviceStep(hw, device, torch, acl)]
+    hout = [[torch.empty_like(t, device="cpu").pin_memory() for t in ds.outs] for _ in range(2)]
+    h2d = sum(h.numel() * h.element_size() for _, h in ds.ins)
+    d2h = sum(t.numel() * t.element_size() for t in ds.outs)
+    cp_in, cp_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    recorded = [False, False]
+
+    def one(k):
+        i = k % 2
+        S = sets[i]
+        if recorded[i]:
+            cp_in.wait_event(ev_done[i])    # step k - 2 has finished reading set i's inputs
+        with torch.cuda.stream(cp_in):
+            for dv, hv in S.ins:
+                dv.copy_(hv, non_blocking=True)
+        ev_in[i].record(cp_in)
+        stream.wait_event(ev_in[i])
+        if recorded[i]:
+            stream.wait_event(ev_out[i])    # step k - 2's outputs have left set i
+        with torch.cuda.stream(stream):
+            S.step(stream)
+        ev_done[i].record(stream)
+        cp_out.wait_event(ev_done[i])
+        with torch.cuda.stream(cp_out):
+            for dv, hv in zip(S.outs, hout[i]):
+                hv.copy_(dv, non_blocking=True)
+        ev_out[i].record(cp_out)
+        recorded[i] = True
+
+    def drain():
+        stream.wait_stream(cp_out)
+        stream.wait_stream(cp_in)
+
+    for k in range(3):
+        one(k)
+    drain()
+    torch.cuda.synchronize()
+    n = max(1, args.e2e_steps)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    cp_in.wait_stream(stream)
+    cp_out.wait_stream(stream)
+    for k in range(n):
+        one(k)
+    drain()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    return {"unit": "tokens/s", "knn_unit": "queries/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": n, "_ms": ms,
+            "pipelining": "2 device sets, copy-in / compute / copy-out streams; eager calls"}
 
 
-def token_merge_times(torch, acl, synth, sb, device, stream, peaks: dict, reps: int = 10) -> dict:
-    """Token merging of the stage-1 tokens into round(0.4 N) anchors (d = 128, hidden 32),
-    forward and backward, one call at a time with CUDA events; GB/s of the algorithmic bytes
-    and the fraction of the measured HBM copy bandwidth."""
-    mb = synth.merge_batch(sb.attn.coords, d=128)
+# --------------------------------------------------------------------------- extra parts
+
+def config_times(torch, acl, synth, device, stream, peaks: dict, reps: int = 10) -> dict:
+    """One layer of the three smaller attention workloads (the tiny 16 x 16 grid; 8 images x
+    2048 tokens, 4 heads; 64 images x 328 tokens, 16 heads), one call at a time, each
+    captured as a CUDA graph and timed with CUDA events; tokens/s of fwd + bwd and the
+    fraction of the measured HBM copy bandwidth on the algorithmic bytes (`attn_bytes`)."""
+    T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
+    timed = lambda fn: graph_time(torch, stream, fn, reps)
+    hbm = peaks["hbm_gbs"]
+
+    def attn_layer(ab, what):
+        xy = T(ab.coords)
+        q, k, v, do = (T(x, torch.bfloat16) for x in (ab.q, ab.k, ab.v, ab.do))
+        bias = T(ab.bias)
+        cl = acl.acl_cluster(xy, stream=stream)
+        nb = acl.acl_neighbors(xy, cl, stream=stream)
+        o, lse = acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, stream=stream)
+        ws = torch.empty((acl.acl_cluster_attn_workspace(ab.B, ab.N, ab.H, 8, 48),), dtype=torch.uint8,
+                         device=device)
+        t_cl = timed(lambda: acl.acl_cluster(xy, clusters=cl, stream=stream))
+        t_nb = timed(lambda: acl.acl_neighbors(xy, cl, nbr=nb, stream=stream))
+        t_f = timed(lambda: acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, O=o, lse=lse,
+                                                     stream=stream))
+        t_b = timed(lambda: acl.acl_cluster_attn_bwd(q, k, v, xy, cl, nb, bias, ab.scale, o, do, lse,
+                                                     workspace=ws, stream=stream))
+        by = attn_bytes(ab.B, ab.N, ab.H)
+        t = (t_f + t_b) * 1e-6
+        gbs = (by["attn_fwd"] + by["attn_bwd"]) / t / 1e9
+        return {"config": what, "tokens_per_s_fwd_bwd": round(ab.B * ab.N / t, 1), "cluster_us": t_cl,
+                "neighbors_us": t_nb, "fwd_us": t_f, "bwd_us": t_b,
+                "fwd_frac": round(by["attn_fwd"] / (t_f * 1e-6) / 1e9 / hbm, 4),
+                "bwd_frac": round(by["attn_bwd"] / (t_b * 1e-6) / 1e9 / hbm, 4),
+                "GB_s": round(gbs, 1), "frac": round(gbs / hbm, 4)}
+
+    return {
+        "tiny": attn_layer(synth.attn_tiny(), "1 image, 16 x 16 grid, H = 4 (launch-bound)"),
+        "stage1_b8": attn_layer(synth.attn_stage1(B=8), "8 images x 2048 tokens, H = 4"),
+        "stage3_b64": attn_layer(synth.attn_stage3(B=64), "64 images x 328 tokens, H = 16"),
+    }
+
+
+def token_merge_times(torch, acl, synth, device, stream, peaks: dict, reps: int = 10) -> dict:
+    """Token merging of 8 images' stage-1 tokens into round(0.4 N) anchors (d = 128, hidden
+    32), forward and backward, one call at a time with CUDA events; GB/s of the algorithmic
+    bytes and the fraction of the measured HBM copy bandwidth."""
+    mb = synth.merge_batch(synth.sweep_coords(B=8)[0], d=128)
     T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
     f, xy = T(mb.feats, torch.bfloat16), T(mb.coords)
     w1, b1, w2 = T(mb.w1), T(mb.b1), T(mb.w2)
@@ -620,8 +802,6 @@ def token_merge_times(torch, acl, synth, sb, device, stream, peaks: dict, reps: 
         res["roofline"][key] = {"alg_bytes": nbytes[key], "GB_s": round(gbs, 1),
                                 "frac": round(gbs / peaks["hbm_gbs"], 4)}
     return res
-
-
 def hires_gather_times(torch, acl, synth, device, stream, B: int = 4, reps: int = 10) -> dict:
     """Decoder gather at 128 x 128 cells (4 images, 8192 tokens, 16384 queries, d = 128):
     Z-order token order, then table + gather fwd + bwd in raster and in Z-order, one call at a
@@ -653,171 +833,6 @@ def hires_gather_times(torch, acl, synth, device, stream, B: int = 4, reps: int 
                                                             workspace=ws, stream=stream)),
         }
     return res
-
-
-def run_e2e(args, s: StepSet, stream, streams, torch, acl, tokens_per_step: int, sb=None,
-            device=None) -> dict:
-    """The step through the public entry points from pinned host memory, copies inside.
-
-    Every step copies its inputs host -> device and its results device -> host.  Two
-    device sets and two copy streams pipeline the steps: the inputs of step k + 1 travel
-    in and the results of step k - 1 travel out while step k computes (PCIe is full
-    duplex), with events ordering each set's copy-in, compute and copy-out."""
-    sets = [s, StepSet(sb, device, acl, torch)] if sb is not None else [s, s]
-    hin = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in s.inputs.items()}
-    for k, v in s.inputs.items():
-        hin[k].copy_(v)
-    hout = [{k: torch.empty_like(v, device="cpu").pin_memory() for k, v in s.outputs.items()}
-            for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in hin.values())
-    d2h = sum(t.numel() * t.element_size() for t in hout[0].values())
-    cp_in, cp_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    recorded = [False, False]
-
-    def one(k):
-        i = k % 2
-        S = sets[i]
-        if recorded[i]:
-            cp_in.wait_event(ev_done[i])    # step k - 2 has finished reading set i's inputs
-        with torch.cuda.stream(cp_in):
-            for name, v in hin.items():
-                S.inputs[name].copy_(v, non_blocking=True)
-        ev_in[i].record(cp_in)
-        stream.wait_event(ev_in[i])
-        if recorded[i]:
-            stream.wait_event(ev_out[i])    # step k - 2's results have left set i
-        with torch.cuda.stream(stream):
-            S.step(stream, None, streams)
-        ev_done[i].record(stream)
-        cp_out.wait_event(ev_done[i])
-        with torch.cuda.stream(cp_out):
-            for name, v in S.outputs.items():
-                hout[i][name].copy_(v, non_blocking=True)
-        ev_out[i].record(cp_out)
-        recorded[i] = True
-
-    def drain():
-        stream.wait_stream(cp_out)
-        stream.wait_stream(cp_in)
-
-    for k in range(4):
-        one(k)
-    drain()
-    torch.cuda.synchronize()
-    n = max(1, args.e2e_steps)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    cp_in.wait_stream(stream)
-    cp_out.wait_stream(stream)
-    for k in range(n):
-        one(k)
-    drain()
-    b.record(stream)
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / n
-    return {"value": tokens_per_step / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "steps": n, "_ms": ms,
-            "pipelining": "2 device sets, copy-in / compute / copy-out streams"}
-
-
-# --------------------------------------------------------------------------- CPU oracle
-
-def oracle_step(sb, images: slice | None = None) -> None:
-    """One pass of the hot path through the fp64 oracle (optionally on a subset of images)."""
-    import oracle
-    a, k = sb.attn, sb.knn
-    sl = images if images is not None else slice(None)
-    xy = a.coords[sl]
-    cl = oracle.cluster(xy, 8)
-    nb = oracle.neighbors(xy, cl, 48)
-    oracle.attn_fwd(a.q[sl], a.k[sl], a.v[sl], xy, cl, nb, a.bias, a.scale)
-    oracle.attn_bwd(a.q[sl], a.k[sl], a.v[sl], xy, cl, nb, a.bias, a.scale, a.do[sl])
-    table = oracle.knn_table(k.coords[sl], k.GH, k.GW, k.K)
-    oracle.knn_fwd(k.queries[sl], k.feats[sl], k.coords[sl], table, k.p)
-    oracle.knn_bwd(k.queries[sl], k.feats[sl], k.coords[sl], table, k.p, k.dout[sl])
-
-
-def cpu_baseline(args, sb) -> dict:
-    import oracle
-    cores = oracle.set_threads(os.cpu_count() or 1)
-    B, N = sb.attn.B, sb.attn.N
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        oracle_step(sb)
-        reps += 1
-        if time.perf_counter() - t0 >= args.cpu_seconds:
-            break
-    dt = time.perf_counter() - t0
-    # the same on one thread, over the first image only (a few seconds)
-    oracle.set_threads(1)
-    reps1, t1 = 0, time.perf_counter()
-    while True:
-        oracle_step(sb, images=slice(0, 1))
-        reps1 += 1
-        if time.perf_counter() - t1 >= max(2.0, args.cpu_seconds / 4):
-            break
-    dt1 = time.perf_counter() - t1
-    oracle.set_threads(cores)
-    return {"value": round(reps * B * N / dt, 1), "unit": "tokens/s", "cores": cores,
-            "kind": "oracle",
-            "sample": f"{reps} full step(s) of the workload ({B} images), fp64 C, OpenMP over images",
-            "value_1_thread": round(reps1 * N / dt1, 1),
-            "sample_1_thread": f"{reps1} step(s) of one image on 1 thread"}
-
-
-def run_reference(args, rank: int, world: int) -> None:
-    if rank != 0:
-        return
-    import oracle
-    from off_grid_cluster_b200 import synth
-    cores = oracle.set_threads(os.cpu_count() or 1)
-    sb = synth.step_batch(B=args.batch)
-    B, N = sb.attn.B, sb.attn.N
-    # bounded sample: images per step chosen so that warm-up + steps take about two minutes
-    t = time.perf_counter()
-    oracle_step(sb, slice(0, 1))
-    t_img = max(time.perf_counter() - t, 1e-3)
-    total = args.steps + args.warmup
-    per_step = int(max(1, min(B, 120.0 / (total * t_img))))
-    sl = slice(0, per_step)
-    for _ in range(args.warmup):
-        oracle_step(sb, sl)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(sb, sl)
-    dt = (time.perf_counter() - t0) / max(args.steps, 1)
-    value = per_step * N / dt
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded; shapes of the pages' 1024 px stage-1 workload)",
-        "config": {"workload": WORKLOAD, "images_per_gpu": B, "tokens_per_image": N,
-                   "sample_images_per_step": per_step},
-        "impl": "reference",
-        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores,
-                         "kind": "oracle",
-                         "sample": f"{per_step} of {B} images per step, fp64 C oracle"},
-        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-
-
-def main(argv=None):
-    args = parse_args(argv)
-    rank = env_int("RANK", 0)
-    world = env_int("WORLD_SIZE", 1)
-    if args.impl == "reference":
-        run_reference(args, rank, world)
-        return
-    if args.only:
-        run_only(args)
-        return
-    run_gpu(args, rank, world)
 
 
 def decoder_times(torch, acl, synth, device, stream, peaks: dict, B: int = 8, reps: int = 10) -> dict:
@@ -881,97 +896,168 @@ def decoder_times(torch, acl, synth, device, stream, peaks: dict, B: int = 8, re
     return res
 
 
-def config_times(torch, acl, synth, device, stream, peaks: dict, reps: int = 10) -> dict:
-    """The five seeded configurations' hot-path calls, one call at a time, each captured as a
-    CUDA graph and timed with CUDA events: cluster attention fwd + bwd tokens/s per layer
-    (configs 1-4; the sweep as sum over stages of its layers x one layer's time, all layers of
-    a stage having the same shapes) and the KNN gather fwd + bwd queries/s over the four stages
-    (config 5), each with its fraction of the measured HBM copy bandwidth on the algorithmic
-    bytes (`algorithmic_bytes`).  Clustering, neighbour and KNN tables are timed beside."""
-    T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
-    timed = lambda fn: graph_time(torch, stream, fn, reps)
-    hbm = peaks["hbm_gbs"]
 
-    def attn_layer(ab):
-        xy = T(ab.coords)
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def oracle_pass(hw: HostWorkload, images: int) -> dict:
+    """One pass of the hot path through the fp64 oracle on the first `images` images: per
+    encoder stage the clustering and neighbour table (seconds) and one layer's forward +
+    backward (seconds); per decoder stage the table, gather forward and backward."""
+    import oracle
+    sl = slice(0, images)
+    res = {"tables_s": [], "layer_s": [], "knn_s": []}
+    for st in hw.stages:
+        xy = st["coords"][sl].numpy()
+        L = st["layers"][0]
+        q, k, v, do = (L[n][sl].float().numpy().astype(np.float64) for n in ("q", "k", "v", "do"))
+        bias = st["bias"].numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        cl = oracle.cluster(xy, 8)
+        nb = oracle.neighbors(xy, cl, 48)
+        t1 = time.perf_counter()
+        oracle.attn_fwd(q, k, v, xy, cl, nb, bias, st["scale"])
+        oracle.attn_bwd(q, k, v, xy, cl, nb, bias, st["scale"], do)
+        t2 = time.perf_counter()
+        res["tables_s"].append(t1 - t0)
+        res["layer_s"].append(t2 - t1)
+    for kd in hw.knn:
+        qq, xy, p = kd["queries"][sl].numpy(), kd["coords"][sl].numpy(), kd["p"].numpy()
+        f = kd["feats"][sl].float().numpy().astype(np.float64)
+        g = kd["dout"][sl].float().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        table = oracle.knn_table(xy, kd["GH"], kd["GW"], kd["K"])
+        oracle.knn_fwd(qq, f, xy, table, p)
+        oracle.knn_bwd(qq, f, xy, table, p, g)
+        res["knn_s"].append(time.perf_counter() - t0)
+    return res
+
+
+def oracle_rates(hw: HostWorkload, images: int, passes: list[dict]) -> tuple[float, float]:
+    """(sweep tokens/s, gather queries/s) of the oracle from timed passes over `images`
+    images: each stage's clustering + neighbour table once and its layer's time times the
+    stage's layer count, as in the sweep."""
+    n = len(passes)
+    t_sweep = sum(sum(p["tables_s"][s] + hw.layer_counts[s] * p["layer_s"][s] for s in range(len(hw.stages)))
+                  for p in passes) / n
+    tokens = sum(images * st["N"] * L for st, L in zip(hw.stages, hw.layer_counts))
+    t_knn = sum(sum(p["knn_s"]) for p in passes) / n
+    queries = sum(images * kd["Q"] for kd in hw.knn)
+    return tokens / t_sweep, queries / t_knn
+
+
+def cpu_baseline(args, B: int) -> dict:
+    """The oracle on the host cores over a bounded sample of the rank's workload: one layer
+    of each encoder stage (scaled by the stage's layer count) and the gather over every
+    stage, for the first images of the batch, repeated for about --cpu-seconds."""
+    import torch
+
+    import oracle
+    hw = HostWorkload(B, 0, torch, pin=False, layers=1)
+    cores = oracle.set_threads(os.cpu_count() or 1)
+    images = min(B, max(1, cores))
+    passes, t0 = [], time.perf_counter()
+    while not passes or time.perf_counter() - t0 < args.cpu_seconds:
+        passes.append(oracle_pass(hw, images))
+    tok, qry = oracle_rates(hw, images, passes)
+    oracle.set_threads(1)
+    one = [oracle_pass(hw, 1)]
+    tok1, qry1 = oracle_rates(hw, 1, one)
+    oracle.set_threads(cores)
+    return {"value": round(tok, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "knn_value": round(qry, 1), "knn_unit": "queries/s",
+            "sample": f"{len(passes)} pass(es) over {images} of {B} images: each encoder stage's clustering, "
+                      f"neighbour table and one layer fwd + bwd (layer time x the stage's layer count), and "
+                      f"the decoder gather (table, fwd, bwd) over the four stages; fp64 C, OpenMP over "
+                      f"image x head (attention) and images (the rest)",
+            "value_1_thread": round(tok1, 1), "knn_value_1_thread": round(qry1, 1),
+            "sample_1_thread": "one pass over 1 image on 1 thread"}
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    import torch
+
+    import oracle
+    cores = oracle.set_threads(os.cpu_count() or 1)
+    hw = HostWorkload(args.batch, 0, torch, pin=False, layers=1)
+    # bounded sample: images per step chosen so that warm-up + steps take about 100 s
+    n0 = min(args.batch, cores)
+    t = time.perf_counter()
+    oracle_pass(hw, n0)
+    t0_pass = max(time.perf_counter() - t, 1e-3)
+    total = args.steps + args.warmup
+    images = int(max(1, min(args.batch, n0 * 100.0 / (total * t0_pass))))
+    for _ in range(args.warmup):
+        oracle_pass(hw, images)
+    t0 = time.perf_counter()
+    passes = [oracle_pass(hw, images) for _ in range(args.steps)]
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    tok, qry = oracle_rates(hw, images, passes)
+    line = {
+        "metric": METRIC, "value": round(tok, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; shapes of the pages' 1024 px encoder and decoder workloads)",
+        "config": {"workload": WORKLOAD, "images_per_gpu": args.batch, "sample_images_per_step": images,
+                   "stage_tokens": [st["N"] for st in hw.stages], "stage_layers": hw.layer_counts},
+        "impl": "reference",
+        "knn": {"value": round(qry, 1), "unit": "queries/s"},
+        "cpu_baseline": {"value": round(tok, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step {images} of {args.batch} images: each encoder stage's "
+                                   f"clustering, neighbour table and one layer fwd + bwd (layer time x the "
+                                   f"stage's layer count) and the decoder gather over the four stages; "
+                                   f"fp64 C oracle"},
+        "e2e": {"value": round(tok, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- one part alone
+
+def stage_calls(torch, acl, synth, device, stream, which: str, stage: int, B: int = IMAGES):
+    """The library calls of one encoder stage's layer (which = "attn") or one decoder stage's
+    gather (which = "knn") of the benchmark workload, as closures, after one eager call of
+    each; returns (name, fn) pairs."""
+    T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
+    s = stage - 1
+    if which == "attn":
+        xy_np = synth.sweep_coords(B)[s]
+        ab = synth.attn_sweep_layer(xy_np, s, 0)
+        xy, bias = T(xy_np), T(ab.bias)
         q, k, v, do = (T(x, torch.bfloat16) for x in (ab.q, ab.k, ab.v, ab.do))
-        bias = T(ab.bias)
         cl = acl.acl_cluster(xy, stream=stream)
         nb = acl.acl_neighbors(xy, cl, stream=stream)
         o, lse = acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, stream=stream)
         ws = torch.empty((acl.acl_cluster_attn_workspace(ab.B, ab.N, ab.H, 8, 48),), dtype=torch.uint8,
                          device=device)
-        t_cl = timed(lambda: acl.acl_cluster(xy, clusters=cl, stream=stream))
-        t_nb = timed(lambda: acl.acl_neighbors(xy, cl, nbr=nb, stream=stream))
-        t_f = timed(lambda: acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, O=o, lse=lse,
-                                                     stream=stream))
-        t_b = timed(lambda: acl.acl_cluster_attn_bwd(q, k, v, xy, cl, nb, bias, ab.scale, o, do, lse,
-                                                     workspace=ws, stream=stream))
-        by = algorithmic_bytes(ab.B, ab.N, ab.H, 1, 32, 8, 1, 1)
-        return {"tokens": ab.B * ab.N, "cluster_us": t_cl, "neighbors_us": t_nb, "fwd_us": t_f, "bwd_us": t_b,
-                "alg_MB": round((by["attn_fwd"] + by["attn_bwd"]) / 1e6, 2)}
-
-    def attn_summary(r, layers=1):
-        t = (r["fwd_us"] + r["bwd_us"]) * 1e-6
-        gbs = r["alg_MB"] * 1e6 / t / 1e9
-        return {"tokens_per_s_fwd_bwd": round(r["tokens"] / t, 1), "GB_s": round(gbs, 1),
-                "frac": round(gbs / hbm, 4), **r}
-
-    res = {}
-    c1 = attn_summary(attn_layer(synth.attn_tiny()))
-    c1["config"] = "tiny: 1 image, 16 x 16 grid, H = 4 (launch-bound)"
-    res["c1"] = c1
-    c2 = attn_summary(attn_layer(synth.attn_stage1(B=8)))
-    c2["config"] = "stage 1: 8 images x 2048 tokens, H = 4"
-    res["c2"] = c2
-    c3 = attn_summary(attn_layer(synth.attn_stage3(B=64)))
-    c3["config"] = "stage 3: 64 images x 328 tokens, H = 16"
-    res["c3"] = c3
-    coords = synth.sweep_coords(B=16)
-    tot_t, tot_tok, tot_b, stages = 0.0, 0, 0.0, []
-    for st, xy in enumerate(coords):
-        r = attn_layer(synth.attn_sweep_layer(xy, st, 0))
-        L = synth.SWEEP_LAYERS[st]
-        t = (r["fwd_us"] + r["bwd_us"]) * 1e-6
-        tot_t += L * t
-        tot_tok += L * r["tokens"]
-        tot_b += L * r["alg_MB"] * 1e6
-        stages.append({"stage": st + 1, "N": xy.shape[1], "H": synth.SWEEP_DIMS[st] // 32, "layers": L,
-                       "fwd_us": r["fwd_us"], "bwd_us": r["bwd_us"], "cluster_us": r["cluster_us"],
-                       "neighbors_us": r["neighbors_us"],
-                       "frac": round(r["alg_MB"] * 1e6 / t / 1e9 / hbm, 4)})
-    res["c4"] = {"config": "sweep: 16 images, stages 2048/819/328/131, layers 3/4/16/2",
-                 "tokens_per_s_fwd_bwd": round(tot_tok / tot_t, 1), "sweep_us": round(tot_t * 1e6, 1),
-                 "GB_s": round(tot_b / tot_t / 1e9, 1), "frac": round(tot_b / tot_t / 1e9 / hbm, 4),
-                 "stages": stages}
-    kt, kq, kb, kst = 0.0, 0, 0.0, []
-    for st, kbt in enumerate(synth.knn_decoder(B=16)):
-        xy, f = T(kbt.coords), T(kbt.feats, torch.bfloat16)
-        qq, pp, dout = T(kbt.queries), T(kbt.p), T(kbt.dout, torch.bfloat16)
-        table = acl.acl_knn_table(xy, kbt.GH, kbt.GW, kbt.K, stream=stream)
-        out = acl.acl_knn_gather_fwd(qq, f, xy, table, pp, stream=stream)
-        ws = torch.empty((acl.acl_knn_gather_workspace(kbt.B, kbt.Q, kbt.N, kbt.d, kbt.K),),
-                         dtype=torch.uint8, device=device)
-        t_t = timed(lambda: acl.acl_knn_table(xy, kbt.GH, kbt.GW, kbt.K, table=table, stream=stream))
-        t_f = timed(lambda: acl.acl_knn_gather_fwd(qq, f, xy, table, pp, out=out, stream=stream))
-        t_b = timed(lambda: acl.acl_knn_gather_bwd(qq, f, xy, table, pp, dout, workspace=ws, stream=stream))
-        by = algorithmic_bytes(kbt.B, kbt.N, 1, kbt.Q, kbt.d, kbt.K, kbt.GH, kbt.GW)
-        bts = by["knn_fwd"] + by["knn_bwd"]
-        t = (t_f + t_b) * 1e-6
-        kt += t
-        kq += kbt.B * kbt.Q
-        kb += bts
-        kst.append({"stage": st + 1, "N": kbt.N, "d": kbt.d, "table_us": t_t, "fwd_us": t_f, "bwd_us": t_b,
-                    "frac": round(bts / t / 1e9 / hbm, 4)})
-    res["c5"] = {"config": "decoder gather: 16 images x 4096 queries over the four stages, K = 8",
-                 "queries_per_s_fwd_bwd": round(kq / kt, 1), "gather_us": round(kt * 1e6, 1),
-                 "GB_s": round(kb / kt / 1e9, 1), "frac": round(kb / kt / 1e9 / hbm, 4), "stages": kst}
-    return res
+        grads = acl.acl_cluster_attn_bwd(q, k, v, xy, cl, nb, bias, ab.scale, o, do, lse, workspace=ws,
+                                         stream=stream)
+        return [("attn_fwd", lambda: acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, O=o, lse=lse,
+                                                              stream=stream)),
+                ("attn_bwd", lambda: acl.acl_cluster_attn_bwd(q, k, v, xy, cl, nb, bias, ab.scale, o, do, lse,
+                                                              *grads, workspace=ws, stream=stream))]
+    kb = synth.knn_decoder(B)[s]
+    xy, f = T(kb.coords), T(kb.feats, torch.bfloat16)
+    qq, pp, g = T(kb.queries), T(kb.p), T(kb.dout, torch.bfloat16)
+    table = acl.acl_knn_table(xy, kb.GH, kb.GW, kb.K, stream=stream)
+    out = acl.acl_knn_gather_fwd(qq, f, xy, table, pp, stream=stream)
+    ws = torch.empty((acl.acl_knn_gather_workspace(kb.B, kb.Q, kb.N, kb.d, kb.K),), dtype=torch.uint8,
+                     device=device)
+    grads = acl.acl_knn_gather_bwd(qq, f, xy, table, pp, g, workspace=ws, stream=stream)
+    return [("knn_table", lambda: acl.acl_knn_table(xy, kb.GH, kb.GW, kb.K, table=table, stream=stream)),
+            ("knn_fwd", lambda: acl.acl_knn_gather_fwd(qq, f, xy, table, pp, out=out, stream=stream)),
+            ("knn_bwd", lambda: acl.acl_knn_gather_bwd(qq, f, xy, table, pp, g, *grads, workspace=ws,
+                                                       stream=stream))]
 
 
 def run_only(args):
-    """One extra part on cuda:0 (an eager call, then each call captured as a CUDA graph and
-    replayed between CUDA events); prints its timing dict."""
+    """One part on cuda:0 and its timing dict as JSON.  attn_stage / knn_stage run one
+    stage's calls of the benchmark workload eagerly (one warm call each, then one more:
+    a short command for ncu, whose launch shapes match the bench's), then time each call
+    as a CUDA graph."""
     import torch
 
     import off_grid_cluster_b200 as acl
@@ -980,14 +1066,35 @@ def run_only(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     stream = torch.cuda.Stream(device)
+    peaks = measured_peaks()
     if args.only == "token_merge":
-        sb = synth.step_batch(B=args.batch)
-        res = token_merge_times(torch, acl, synth, sb, device, stream, measured_peaks())
+        res = token_merge_times(torch, acl, synth, device, stream, peaks)
     elif args.only == "decoder":
-        res = decoder_times(torch, acl, synth, device, stream, measured_peaks(), B=args.batch)
+        res = decoder_times(torch, acl, synth, device, stream, peaks, B=8)
+    elif args.only == "configs":
+        res = config_times(torch, acl, synth, device, stream, peaks)
     else:
-        res = config_times(torch, acl, synth, device, stream, measured_peaks())
+        which = "attn" if args.only == "attn_stage" else "knn"
+        calls = stage_calls(torch, acl, synth, device, stream, which, args.stage, args.batch)
+        with torch.cuda.stream(stream):
+            for _, fn in calls:
+                fn()
+        stream.synchronize()
+        res = {"stage": args.stage, "us": {name: graph_time(torch, stream, fn) for name, fn in calls}}
     print(json.dumps({"part": args.only, **res}))
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = env_int("RANK", 0)
+    world = env_int("WORLD_SIZE", 1)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if args.only:
+        run_only(args)
+        return
+    run_gpu(args, rank, world)
 
 
 if __name__ == "__main__":

@@ -1,22 +1,28 @@
 """Host-side logic of the benchmark (no GPU): the algorithmic byte counts that the roofline
-fractions divide by, the measured-peak loader, the traffic keying and the argument defaults."""
+fractions divide by, the measured-peak loader, the DRAM-traffic summary keying and the
+argument defaults."""
 import os
 
 import bench
 
 
-def test_step_algorithmic_bytes():
-    """The per-call bytes of the step workload (8 images x 2048 tokens, H = 4; Q = 4096,
-    d = 128, K = 8 on a 64 x 64 grid), every tensor counted once."""
-    by = bench.algorithmic_bytes(8, 2048, 4, 4096, 128, 8, 64, 64)
-    B, N, H, Q, d, K = 8, 2048, 4, 4096, 128, 8
-    G = N // 8
-    meta = 8 + 4 + 4 * 48 * G / N
-    assert by["cluster"] == B * N * 12
-    assert by["attn_fwd"] == B * N * (H * (3 * 64 + 64 + 4) + meta) + H * 12
-    assert by["attn_bwd"] == B * N * (H * (4 * 64 + 4 + 3 * 64) + meta) + 2 * H * 12
-    assert by["knn_fwd"] == B * (Q * (8 + 4 * K + 2 * d) + N * (2 * d + 8)) + 4 * d // 32
-    assert round(by["attn_bwd"] / 1e6, 3) == 30.212 and round(by["knn_fwd"] / 1e6, 3) == 14.025
+def test_attention_algorithmic_bytes():
+    """Per (token, head): fwd Q, K, V, O + lse = 260 B, bwd Q, K, V, O, dO, lse + dQ, dK, dV =
+    516 B; 72 B per token of coordinates, cluster list and neighbour-table share."""
+    by = bench.attn_bytes(16, 328, 16)
+    assert by["attn_fwd"] == 16 * 328 * (16 * (4 * 64 + 4) + 72)
+    assert by["attn_bwd"] == 16 * 328 * (16 * (6 * 64 + 4 + 2 * 64) + 72)
+    # the stage-1 layer of 8 images: 35.0 MB for the backward
+    assert round(bench.attn_bytes(8, 2048, 4)["attn_bwd"] / 1e6, 1) == 35.0
+
+
+def test_gather_algorithmic_bytes():
+    B, Q, N, d, K = 16, 4096, 131, 768, 8
+    by = bench.knn_bytes(B, Q, N, d, K)
+    assert by["knn_fwd"] == B * (Q * (8 + 4 * K + 2 * d) + N * (2 * d + 8))
+    assert by["knn_bwd"] == B * (Q * (8 + 4 * K + 8 + 2 * d) + N * (2 * d + 8 + 2 * d))
+    tb = bench.table_bytes(16, 2048)
+    assert tb["cluster"] == 16 * 2048 * 12 and tb["knn_table"] == 16 * (2048 * 8 + 64 * 64 * 8 * 4)
 
 
 def test_merge_bytes():
@@ -31,17 +37,35 @@ def test_peaks_have_both_denominators():
     assert p["hbm_gbs"] > 0 and p["bf16_tflops"] > 0 and p["source"]
 
 
-def test_traffic_is_keyed_to_the_kernels_own_sources(tmp_path):
+def test_traffic_is_keyed_to_call_shape_and_sources(tmp_path):
     names = bench.TRAFFIC_SOURCES["attn_bwd"]
     h = bench.source_hash(names)
     assert len(h) == 16 and h == bench.source_hash(names)
     assert h != bench.source_hash()  # a subset of the sources hashes differently
     for name in names:
         assert os.path.exists(os.path.join(bench.ROOT, "off_grid_cluster_b200", "csrc", name))
+    w = bench.call_workload("attn_bwd", 16, 328, H=16)
+    f = tmp_path / "t.txt"
+    f.write_text("# comment\n"
+                 f"traffic: call = attn_bwd; workload = {w}; read = 1000; write = 24; src = {h}\n"
+                 f"traffic: call = attn_fwd; workload = {w}; read = 5; write = 5; src = 0000000000000000\n")
+    rows = bench.read_traffic(str(f))
+    assert len(rows) == 2
+    assert bench.traffic_for("attn_bwd", w, rows) == {"read": 1000.0, "write": 24.0, "total": 1024.0}
+    assert bench.traffic_for("attn_fwd", w, rows) is None          # stale sources
+    assert bench.traffic_for("attn_bwd", "b8-n2048-h4", rows) is None
+    assert bench.read_traffic(str(tmp_path / "missing.txt")) == []
 
 
 def test_argument_defaults():
     a = bench.parse_args([])
-    assert (a.gpus, a.impl, a.only) == (1, "acl", None)
+    assert (a.gpus, a.impl, a.only, a.batch) == (1, "acl", None, 16)
     assert a.warmup >= 3 and a.steps >= 1
-    assert bench.parse_args(["--only", "configs"]).only == "configs"
+    assert bench.parse_args(["--only", "attn_stage", "--stage", "2"]).stage == 2
+
+
+def test_workload_constants_match_the_generators():
+    from off_grid_cluster_b200 import synth
+    assert tuple(bench.STAGE_LAYERS) == tuple(synth.SWEEP_LAYERS)
+    assert tuple(bench.STAGE_DIMS) == tuple(synth.SWEEP_DIMS)
+    assert tuple(x.shape[1] for x in synth.sweep_coords(B=1)) == bench.STAGE_TOKENS

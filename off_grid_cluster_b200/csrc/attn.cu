@@ -1226,32 +1226,6 @@ __global__ void __launch_bounds__(kThreads, 4) attn_bwd_key_kernel(const AttnArg
 
 // ---------------------------------------------------------------- launchers
 
-int sm_count() {
-    static int cached[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
-        cached[dev] = n;
-    }
-    return cached[dev];
-}
-
-// Resident CTAs per SM of a kernel at a dynamic shared-memory size (asked of the runtime
-// once per kernel and device).
-template <auto Kern>
-int resident(size_t smem) {
-    static int cached[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    if (cached[dev] == 0) {
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, kThreads, smem) != cudaSuccess || n < 1) n = 1;
-        cached[dev] = n;
-    }
-    return cached[dev];
-}
 
 // Persistent grid: resident CTAs per SM times the SM count, or fewer when there are fewer
 // items than warps.
@@ -1289,7 +1263,7 @@ cudaError_t fwd_launch(const AttnArgs& a, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(kWarps) * QTile<16 * MTILES, false>::WARP;
     cudaError_t e = ensure_smem<attn_fwd_kernel<MTILES, Off>>(smem);
     if (e != cudaSuccess) return e;
-    const int per = resident<attn_fwd_kernel<MTILES, Off>>(smem);
+    const int per = resident<attn_fwd_kernel<MTILES, Off>>(kThreads, smem);
     const int grid = grid_for(static_cast<long long>(a.B) * a.G * a.H, per);
     attn_fwd_kernel<MTILES, Off><<<grid, kThreads, smem, st>>>(a);
     note_launch();
@@ -1309,7 +1283,7 @@ cudaError_t query_launch(const AttnArgs& a, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(kWarps) * QTile<16 * MTILES, true>::WARP;
     cudaError_t e = ensure_smem<attn_bwd_query_kernel<MTILES, Off>>(smem);
     if (e != cudaSuccess) return e;
-    const int per = resident<attn_bwd_query_kernel<MTILES, Off>>(smem);
+    const int per = resident<attn_bwd_query_kernel<MTILES, Off>>(kThreads, smem);
     const size_t prep = 4 * prep_smem_ints(a.N, a.G, a.R);
     const long long slots = static_cast<long long>(sm_count()) * per;
     int nprep = 0;
@@ -1332,7 +1306,7 @@ template <typename Off>
 int key_grid(const AttnArgs& a) {
     const size_t smem = static_cast<size_t>(kWarps) * KTile::WARP;
     if (ensure_smem<attn_bwd_key_kernel<Off>>(smem) != cudaSuccess) return 1;
-    return grid_for(static_cast<long long>(a.B) * a.G * a.H, resident<attn_bwd_key_kernel<Off>>(smem));
+    return grid_for(static_cast<long long>(a.B) * a.G * a.H, resident<attn_bwd_key_kernel<Off>>(kThreads, smem));
 }
 
 template <typename Off>

@@ -418,13 +418,6 @@ __global__ void __launch_bounds__(256)
     out[o] = a;
 }
 
-int sm_count() {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        sms = 148;
-    return sms;
-}
-
 }  // namespace
 
 int dec_wo_splits(int T, int d, int D) {

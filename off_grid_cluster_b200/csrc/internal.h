@@ -37,6 +37,35 @@ cudaError_t ensure_smem(size_t bytes) {
     return e;
 }
 
+// Streaming multiprocessors of the current device (asked of the runtime once per device).
+inline int sm_count() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// Resident CTAs per SM of kernel `Kern` launched with `threads` threads and `smem` bytes of
+// dynamic shared memory (asked of the runtime once per kernel and device: a kernel must be
+// launched with one shape).
+template <auto Kern>
+int resident(int threads, size_t smem) {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, threads, smem) != cudaSuccess || n < 1) n = 1;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 size_t cluster_smem_bytes(int N, int C);
 cudaError_t launch_cluster(const float* xy, int B, int N, int C, int32_t* clusters,
                            cudaStream_t st);

@@ -320,8 +320,9 @@ struct Nbrs {
 // d_min = 0 that is the d -> 0 limit); p = 0 gives equal weights.
 __device__ __forceinline__ float knn_v(float d, int kind) { return kind ? log2f(d) : d * kLog2e; }
 __device__ __forceinline__ float knn_weight(float v, float vmin, float p) {
-    if (v == vmin || p == 0.f) return 1.f;
-    return exp2f(-p * (v - vmin));
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(-p * (v - vmin)));
+    return (v == vmin || p == 0.f) ? 1.f : y;
 }
 // -dz/dp for z = -p d (d) or z = -p ln d (ln d; 0 at d = 0), from v
 __device__ __forceinline__ float knn_dzdp(float v) { return v == -INFINITY ? 0.f : v * kLn2; }
@@ -377,42 +378,158 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8], float s) {
     return o;
 }
 
-template <int KT, int CH>
-__global__ void __launch_bounds__(kGatherThreads) knn_fwd_kernel(const KnnArgs a, int lpq_log2) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int LPQ = 1 << lpq_log2;
-    const int sub = lane & (LPQ - 1), grp = lane >> lpq_log2;
-    const long long total = static_cast<long long>(a.B) * a.Q;
-    const long long gq = (static_cast<long long>(blockIdx.x) * kGatherWarps + warp) * (32 >> lpq_log2) + grp;
-    if (gq >= total) return;  // no cross-lane communication below
-    const float2 qp = reinterpret_cast<const float2*>(a.queries)[gq];
-    Nbrs nb[KT];
-    const float vmin = knn_v(load_neighbours<KT>(a, gq, qp, nb), a.kind);
-    float v[KT];
-#pragma unroll
-    for (int j = 0; j < KT; ++j) v[j] = knn_v(nb[j].d, a.kind);
-    const int b = static_cast<int>(gq / a.Q);
-    const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d;
-#pragma unroll
-    for (int ch = 0; ch < CH; ++ch) {
-        const int c0 = ch * LPQ * 8 + sub * 8;
-        if (c0 >= a.d) break;
-        const float ph = a.p[c0 >> 5];
-        uint4 f[KT];
-#pragma unroll
-        for (int j = 0; j < KT; ++j)
-            f[j] = (nb[j].t >= 0) ? ldg16(fb + static_cast<size_t>(nb[j].t) * a.d + c0)
-                                  : make_uint4(0u, 0u, 0u, 0u);
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        float sum = 0.f;
+// Packed f32x2 arithmetic (fp32 pairs held in 64-bit registers).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t r) {
+    float2 v;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+// acc[i] += ww * (the two bf16 of f word i, widened to fp32): one row of 8 channels
+__device__ __forceinline__ void row_fma(uint64_t (&acc)[4], uint64_t ww, uint4 f) {
+    asm("{\n\t.reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t.reg .b64 p0, p1, p2, p3;\n\t"
+        "shl.b32 l0, %5, 16;\n\tand.b32 h0, %5, 0xffff0000;\n\t"
+        "shl.b32 l1, %6, 16;\n\tand.b32 h1, %6, 0xffff0000;\n\t"
+        "shl.b32 l2, %7, 16;\n\tand.b32 h2, %7, 0xffff0000;\n\t"
+        "shl.b32 l3, %8, 16;\n\tand.b32 h3, %8, 0xffff0000;\n\t"
+        "mov.b64 p0, {l0, h0};\n\tmov.b64 p1, {l1, h1};\n\t"
+        "mov.b64 p2, {l2, h2};\n\tmov.b64 p3, {l3, h3};\n\t"
+        "fma.rn.f32x2 %0, %4, p0, %0;\n\tfma.rn.f32x2 %1, %4, p1, %1;\n\t"
+        "fma.rn.f32x2 %2, %4, p2, %2;\n\tfma.rn.f32x2 %3, %4, p3, %3;\n\t}"
+        : "+l"(acc[0]), "+l"(acc[1]), "+l"(acc[2]), "+l"(acc[3])
+        : "l"(ww), "r"(f.x), "r"(f.y), "r"(f.z), "r"(f.w));
+}
+
+// Neighbour j of a query: token id (-1 for an empty slot or an id >= N) and weight
+// exponent v = knn_v(d) (+inf for an empty slot).
+__device__ __forceinline__ void one_neighbour(const KnnArgs& a, const int32_t* row, const float2* xyb,
+                                              float2 qp, int j, int& t, float& v) {
+    t = __ldg(row + j);
+    v = INFINITY;
+    if (t >= a.N) t = -1;
+    if (t >= 0) {
+        const float2 p = __ldg(xyb + t);
+        const float dx = qp.x - p.x, dy = qp.y - p.y;
+        v = knn_v(sqrtf(dx * dx + dy * dy), a.kind);
+    }
+}
+
+// All K neighbours of a query group's query in every lane of the group (slots K..KT-1
+// empty); returns the minimum v.  With K <= LPQ lane j of the group looks up neighbour j
+// and the group shares them by shuffles (all 32 lanes must call); otherwise every lane
+// looks up all K.
+template <int KT>
+__device__ __forceinline__ float query_neighbours(const KnnArgs& a, int b, bool live, float2 qp,
+                                                  int sub, int LPQ, int (&t)[KT], float (&v)[KT],
+                                                  int* own_t = nullptr, float* own_v = nullptr) {
+    const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
+    const int32_t* row = a.table + ((static_cast<size_t>(b) * a.GH + cy) * a.GW + cx) * a.K;
+    const float2* xyb = reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(b) * a.N;
+    float vmin = INFINITY;
+    if (a.K <= LPQ) {
+        int my_t = -1;
+        float my_v = INFINITY;
+        if (live && sub < a.K) one_neighbour(a, row, xyb, qp, sub, my_t, my_v);
+        if (own_t) *own_t = my_t;
+        if (own_v) *own_v = my_v;
+        vmin = my_v;
+        for (int o = 1; o < LPQ; o <<= 1) vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o, LPQ));
 #pragma unroll
         for (int j = 0; j < KT; ++j) {
-            const float w = (nb[j].t >= 0) ? knn_weight(v[j], vmin, ph) : 0.f;
-            sum += w;
-            fma8(acc, w, f[j]);
+            const int tj = __shfl_sync(0xffffffffu, my_t, j, LPQ);
+            const float vj = __shfl_sync(0xffffffffu, my_v, j, LPQ);
+            t[j] = j < a.K ? tj : -1;
+            v[j] = j < a.K ? vj : INFINITY;
         }
-        const float inv = sum > 0.f ? 1.f / sum : 0.f;
-        *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(gq) * a.d + c0) = pack8(acc, inv);
+    } else {
+#pragma unroll
+        for (int j = 0; j < KT; ++j) {
+            t[j] = -1;
+            v[j] = INFINITY;
+            if (live && j < a.K) one_neighbour(a, row, xyb, qp, j, t[j], v[j]);
+            vmin = fminf(vmin, v[j]);
+        }
+    }
+    return vmin;
+}
+
+// Forward.  A group of LPQ lanes owns a query; lane sub owns channels [8 (ch LPQ + sub),
+// +8) of pass ch (one 16-byte load per neighbour row and pass).  The K weights of the
+// lane's head are formed once per pass and the rows accumulate with packed f32x2 FMAs.
+// CTA c takes the `span` consecutive queries from c * span, so neighbouring queries (which
+// share most of their rows) run on one SM and meet each other's rows in L1.
+template <int KT, int CH>
+__global__ void __launch_bounds__(kGatherThreads, 2) knn_fwd_kernel(const KnnArgs a, int lpq_log2, long long span) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int LPQ = 1 << lpq_log2, QPW = 32 >> lpq_log2;
+    const int sub = lane & (LPQ - 1), grp = lane >> lpq_log2;
+    const long long total = static_cast<long long>(a.B) * a.Q;
+    const long long q0 = static_cast<long long>(blockIdx.x) * span;
+    const long long q1 = q0 + span < total ? q0 + span : total;
+    long long gq = q0 + static_cast<long long>(warp) * QPW + grp;
+    // image of query gq and its first query, advanced without divisions
+    int b = static_cast<int>(gq / a.Q);
+    long long qb = static_cast<long long>(b) * a.Q;
+    for (; gq - grp < q1; gq += kGatherWarps * QPW) {
+        while (gq - qb >= a.Q) {
+            ++b;
+            qb += a.Q;
+        }
+        const bool live = gq < q1;
+        const float2 qp = live ? __ldg(reinterpret_cast<const float2*>(a.queries) + gq) : make_float2(0.f, 0.f);
+        int t[KT];
+        float v[KT];
+        const float vmin = query_neighbours<KT>(a, live ? b : 0, live, qp, sub, LPQ, t, v);
+        if (!live) continue;  // no shuffles below
+        // per neighbour: the row's first channel of this lane and the weight exponent
+        // e = v_min - v (0 at the nearest, -inf for an empty slot): w = 2^(p e)
+        const bf16* rowp[KT];
+        float e[KT];
+        {
+            const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d + sub * 8;
+#pragma unroll
+            for (int j = 0; j < KT; ++j) {
+                rowp[j] = fb + static_cast<size_t>(t[j] < 0 ? 0 : t[j]) * a.d;
+                e[j] = t[j] < 0 ? -INFINITY : (v[j] == vmin ? 0.f : vmin - v[j]);
+            }
+        }
+        bf16* ob = a.out + static_cast<size_t>(gq) * a.d + sub * 8;
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch) {
+            // passes after the first exist only with LPQ = 32: pass ch starts at channel 256 ch
+            const int c0 = ch * 256 + sub * 8;
+            if (c0 >= a.d) break;
+            uint4 f[KT];
+#pragma unroll
+            for (int j = 0; j < KT; ++j) f[j] = t[j] >= 0 ? ldg16(rowp[j] + ch * 256) : make_uint4(0u, 0u, 0u, 0u);
+            const float ph = __ldg(a.p + (c0 >> 5));
+            const bool flat = ph == 0.f;  // p = 0: equal weights
+            float w[KT];
+            float sum = 0.f;
+#pragma unroll
+            for (int j = 0; j < KT; ++j) {
+                float y;
+                asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(ph * e[j]));
+                w[j] = t[j] < 0 ? 0.f : (flat ? 1.f : y);
+                sum += w[j];
+            }
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+            for (int j = 0; j < KT; ++j) row_fma(acc, f2_pack(w[j], w[j]), f[j]);
+            const float inv = sum > 0.f ? __fdividef(1.f, sum) : 0.f;
+            const float2 a0 = f2_unpack(acc[0]), a1 = f2_unpack(acc[1]), a2 = f2_unpack(acc[2]),
+                         a3 = f2_unpack(acc[3]);
+            uint4 o;
+            o.x = pack_bf16(a0.x * inv, a0.y * inv);
+            o.y = pack_bf16(a1.x * inv, a1.y * inv);
+            o.z = pack_bf16(a2.x * inv, a2.y * inv);
+            o.w = pack_bf16(a3.x * inv, a3.y * inv);
+            *reinterpret_cast<uint4*>(ob + ch * 256) = o;
+        }
     }
 }
 
@@ -587,47 +704,6 @@ __device__ __forceinline__ float own_neighbour(const KnnArgs& a, long long gq, b
     float vmin = v;
     for (int o = 1; o < LPQ; o <<= 1) vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o, LPQ));
     return vmin;
-}
-
-template <int KT, int CH>
-__global__ void __launch_bounds__(kGatherThreads)
-    knn_fwd_shared_kernel(const KnnArgs a, int lpq_log2, int iters) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int LPQ = 1 << lpq_log2, QPW = 32 >> lpq_log2;
-    const int sub = lane & (LPQ - 1), grp = lane >> lpq_log2;
-    const long long total = static_cast<long long>(a.B) * a.Q;
-    for (int it = 0; it < iters; ++it) {
-        const long long gq = ((static_cast<long long>(blockIdx.x) * iters + it) * kGatherWarps + warp) * QPW + grp;
-        if ((gq - grp) >= total) break;  // whole warp past the end (uniform)
-        const bool live = gq < total;
-        const float2 qp = live ? reinterpret_cast<const float2*>(a.queries)[gq] : make_float2(0.f, 0.f);
-        GroupNbrs nb[KT];
-        const float vmin = group_neighbours<KT>(a, gq, live, qp, sub, LPQ, nb);
-        if (!live) continue;
-        const int b = static_cast<int>(gq / a.Q);
-        const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d;
-#pragma unroll
-        for (int ch = 0; ch < CH; ++ch) {
-            const int c0 = ch * LPQ * 8 + sub * 8;
-            if (c0 >= a.d) break;
-            const float ph = a.p[c0 >> 5];
-            uint4 f[KT];
-#pragma unroll
-            for (int j = 0; j < KT; ++j)
-                f[j] = (nb[j].t >= 0) ? ldg16(fb + static_cast<size_t>(nb[j].t) * a.d + c0)
-                                      : make_uint4(0u, 0u, 0u, 0u);
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            float sum = 0.f;
-#pragma unroll
-            for (int j = 0; j < KT; ++j) {
-                const float w = (nb[j].t >= 0) ? knn_weight(nb[j].v, vmin, ph) : 0.f;
-                sum += w;
-                fma8(acc, w, f[j]);
-            }
-            const float inv = sum > 0.f ? 1.f / sum : 0.f;
-            *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(gq) * a.d + c0) = pack8(acc, inv);
-        }
-    }
 }
 
 template <int KT, int CH>
@@ -1318,18 +1394,6 @@ GatherPlan gather_plan(int B, int Q, int d, int K, bool bwd) {
 }
 
 template <int KT>
-cudaError_t fwd_shared_k(const KnnArgs& a, cudaStream_t st, const GatherPlan& g) {
-    const unsigned blocks = static_cast<unsigned>(g.blocks);
-    switch (g.ch) {
-        case 1: knn_fwd_shared_kernel<KT, 1><<<blocks, kGatherThreads, 0, st>>>(a, g.l2, g.iters); break;
-        case 2: knn_fwd_shared_kernel<KT, 2><<<blocks, kGatherThreads, 0, st>>>(a, g.l2, g.iters); break;
-        case 3: knn_fwd_shared_kernel<KT, 3><<<blocks, kGatherThreads, 0, st>>>(a, g.l2, g.iters); break;
-        default: knn_fwd_shared_kernel<KT, 4><<<blocks, kGatherThreads, 0, st>>>(a, g.l2, g.iters); break;
-    }
-    return cudaGetLastError();
-}
-
-template <int KT>
 cudaError_t bwdq_shared_k(const KnnArgs& a, cudaStream_t st, const GatherPlan& g, size_t smem) {
     const unsigned blocks = static_cast<unsigned>(g.blocks);
     switch (g.ch) {
@@ -1341,15 +1405,29 @@ cudaError_t bwdq_shared_k(const KnnArgs& a, cudaStream_t st, const GatherPlan& g
     return cudaGetLastError();
 }
 
-template <int KT>
-cudaError_t fwd_k(const KnnArgs& a, cudaStream_t st, int l2, int ch, unsigned blocks) {
-    switch (ch) {
-        case 1: knn_fwd_kernel<KT, 1><<<blocks, kGatherThreads, 0, st>>>(a, l2); break;
-        case 2: knn_fwd_kernel<KT, 2><<<blocks, kGatherThreads, 0, st>>>(a, l2); break;
-        case 3: knn_fwd_kernel<KT, 3><<<blocks, kGatherThreads, 0, st>>>(a, l2); break;
-        default: knn_fwd_kernel<KT, 4><<<blocks, kGatherThreads, 0, st>>>(a, l2); break;
-    }
+// The forward's persistent grid: at most one wave of resident CTAs, each taking a span of
+// consecutive queries (a multiple of the queries one pass of its warps takes).
+template <int KT, int CH>
+cudaError_t fwd_launch(const KnnArgs& a, cudaStream_t st, int l2) {
+    const long long total = static_cast<long long>(a.B) * a.Q;
+    const long long per_pass = static_cast<long long>(kGatherWarps) * (32 >> l2);
+    const long long passes = (total + per_pass - 1) / per_pass;
+    const long long slots = static_cast<long long>(sm_count()) * resident<knn_fwd_kernel<KT, CH>>(kGatherThreads, 0);
+    const long long blocks0 = passes < slots ? passes : slots;
+    const long long span = (passes + blocks0 - 1) / blocks0 * per_pass;
+    const unsigned blocks = static_cast<unsigned>((total + span - 1) / span);
+    knn_fwd_kernel<KT, CH><<<blocks, kGatherThreads, 0, st>>>(a, l2, span);
     return cudaGetLastError();
+}
+
+template <int KT>
+cudaError_t fwd_k(const KnnArgs& a, cudaStream_t st, int l2, int ch) {
+    switch (ch) {
+        case 1: return fwd_launch<KT, 1>(a, st, l2);
+        case 2: return fwd_launch<KT, 2>(a, st, l2);
+        case 3: return fwd_launch<KT, 3>(a, st, l2);
+        default: return fwd_launch<KT, 4>(a, st, l2);
+    }
 }
 
 template <int KT>
@@ -1418,13 +1496,10 @@ KnnWorkspace knn_workspace_layout(int B, int Q, int N, int d, int K) {
 }
 
 cudaError_t launch_knn_fwd(const KnnArgs& a, cudaStream_t st) {
-    const GatherPlan g = gather_plan(a.B, a.Q, a.d, a.K, false);
-    if (g.blocks == 0) return cudaSuccess;
-    cudaError_t e;
-    if (g.shared)
-        e = (a.K <= 8) ? fwd_shared_k<8>(a, st, g) : fwd_shared_k<16>(a, st, g);
-    else
-        e = (a.K <= 8) ? fwd_k<8>(a, st, g.l2, g.ch, g.blocks) : fwd_k<16>(a, st, g.l2, g.ch, g.blocks);
+    if (static_cast<long long>(a.B) * a.Q == 0) return cudaSuccess;
+    const int l2 = lpq_log2_for(a.d);
+    const int ch = (a.d + (8 << l2) - 1) / (8 << l2);
+    const cudaError_t e = (a.K <= 8) ? fwd_k<8>(a, st, l2, ch) : fwd_k<16>(a, st, l2, ch);
     note_launch();
     return e;
 }

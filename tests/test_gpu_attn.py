@@ -162,6 +162,6 @@ def test_hub_table_long_reverse_lists(M):
     lens = np.array(lens)
     assert lens[:, 0].min() == G                          # the hub is listed by every cluster
     assert lens.max() > 4 * KEY_CHUNK                     # many chunks for one unit
-    assert np.median(lens) <= KEY_CHUNK                   # and single-chunk units beside it
+    assert (lens <= KEY_CHUNK).sum() > lens.size // 4      # and many single-chunk units beside it
     assert B * G > OFFSET_WINDOW                          # window refills
     run_attn(a, M=M, cl=cl, nb=nb)

@@ -52,7 +52,7 @@ typedef enum {
     ACL_ERR_CUDA = 2,          /* a CUDA call or kernel launch failed                  */
     ACL_ERR_UNSUPPORTED = 3,   /* valid arguments outside what the kernels implement   */
     ACL_ERR_WORKSPACE = 4,     /* workspace pointer null or smaller than required     */
-    ACL_ERR_DEVICE_CHECK = 5,  /* reserved: device-side consistency check failed      */
+    ACL_ERR_DEVICE_CHECK = 5,  /* check build: a device-side range check failed        */
     ACL_ERR_TIMEOUT = 6        /* a bounded device wait gave up (acl_device_check)     */
 } acl_status;
 
@@ -193,6 +193,9 @@ acl_status acl_cluster_attn_bwd(const acl_bf16* Q, const acl_bf16* K, const acl_
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call before any
  *    stream capture on the device.
+ *  - The array used is the current device's: `stream` must belong to the current device
+ *    (a stream of another device returns ACL_ERR_INVALID_ARG; NULL is the current
+ *    device's legacy stream).
  *  - All calls share the one array, which keeps the last call's contents; nothing in it
  *    needs to start at zero (every scratch value is written before it is read).  Calls
  *    that overlap on the GPU (on different streams, without ordering) race on it.
@@ -416,12 +419,32 @@ acl_status acl_knn_gather_bwd_indexed_ex(const float* queries, int B, int Q,
  */
 size_t acl_decoder_layer_workspace(int B, int Q, int N, int d, int D, int K);
 /*
- * acl_device_check -- synchronises the current device, then reports (and clears) whether
- * any bounded device-side wait of the library's tensor-core kernels gave up since the last
- * call: ACL_ERR_TIMEOUT if so (the affected outputs are zero, not garbage), ACL_OK if not,
- * ACL_ERR_CUDA if synchronising failed.
+ * acl_device_check -- synchronises the current device, then reports (and clears) what the
+ * device recorded since the last call:
+ *   ACL_ERR_DEVICE_CHECK  (check build only, see acl_device_checks_enabled) a kernel met an
+ *                         index input outside its range: a token id outside [-1, N) in a
+ *                         cluster list, neighbour table or KNN table.  The kernels treat such
+ *                         an id as an empty slot in both builds; the check build reports it;
+ *   ACL_ERR_TIMEOUT       a bounded device-side wait of the tensor-core kernels gave up (the
+ *                         affected outputs are zero, not garbage);
+ *   ACL_OK                neither; ACL_ERR_CUDA if synchronising failed.
  */
 acl_status acl_device_check(void);
+/*
+ * acl_device_checks_enabled -- 1 in the check build of the library (libacl_check.so, compiled
+ * with ACL_DEVICE_CHECKS: every token id read from a cluster list, neighbour table or KNN
+ * table is range-checked on the device), 0 in the regular build.
+ */
+int acl_device_checks_enabled(void);
+/*
+ * acl_test_set_wait_limit -- test hook: the SM clocks after which a main-loop mbarrier wait of
+ * the tensor-core GEMM gives up (default 1e9, about half a second; 0 = give up at once;
+ * negative restores the default).  The wait for the MMAs
+ * still in flight before tensor memory is freed always keeps the default, so a lowered limit
+ * ends the kernel early with zero outputs and ACL_ERR_TIMEOUT from acl_device_check, never
+ * with a fault.  Synchronous; affects the current device.
+ */
+acl_status acl_test_set_wait_limit(long long cycles);
 acl_status acl_decoder_layer_fwd(const float* ref, const float* f_in, int B, int Q, int D,
                                  const float* w_off, const float* b_off, const acl_bf16* w_o,
                                  const acl_bf16* feats, const float* coords, int N, int d,

@@ -18,7 +18,10 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libacl.so")
+# the library to load: the regular build, or another build of the same sources named by
+# ACL_LIBRARY (the check build libacl_check.so, whose kernels range-check their index inputs)
+LIB_PATH = os.environ.get("ACL_LIBRARY") or os.path.join(_HERE, "libacl.so")
+CHECK_LIB_PATH = os.path.join(_HERE, "libacl_check.so")
 
 ACL_OK = 0
 _STATUS = {0: "ACL_OK", 1: "ACL_ERR_INVALID_ARG", 2: "ACL_ERR_CUDA", 3: "ACL_ERR_UNSUPPORTED",
@@ -49,6 +52,8 @@ SIGNATURES = {
     "acl_knn_gather_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "acl_decoder_layer_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
     "acl_device_check": (_I, []),
+    "acl_device_checks_enabled": (_I, []),
+    "acl_test_set_wait_limit": (_I, [ct.c_longlong]),
     "acl_decoder_layer_fwd": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I,
                                    _I, _P, _P, _P, _P, _P]),
     "acl_decoder_layer_bwd": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P,
@@ -351,8 +356,21 @@ ACL_KNN_EXP, ACL_KNN_INVPOW = 0, 1  # weight kernels: softmax(-p d), d^-p / sum 
 
 
 def acl_device_check() -> None:
-    """Synchronise the device; raise if a bounded device-side wait gave up."""
+    """Synchronise the device; raise AclError if a bounded device-side wait gave up
+    (ACL_ERR_TIMEOUT) or, in the check build, an index input was out of range
+    (ACL_ERR_DEVICE_CHECK)."""
     _call("acl_device_check")
+
+
+def acl_device_checks_enabled() -> bool:
+    """True in the check build of the library (device-side range checks)."""
+    return bool(lib().acl_device_checks_enabled())
+
+
+def acl_test_set_wait_limit(cycles: int) -> None:
+    """Test hook: give-up limit (SM clocks) of the tensor-core GEMM's main-loop waits; a
+    negative value restores the default."""
+    _call("acl_test_set_wait_limit", int(cycles))
 
 
 def acl_decoder_layer_workspace(B: int, Q: int, N: int, d: int, D: int, K: int = 8) -> int:

@@ -401,9 +401,24 @@ acl_status acl_knn_gather_bwd(const float* queries, int B, int Q, const acl_bf16
 
 acl_status acl_device_check(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return ACL_ERR_CUDA;
-    unsigned int n = 0;
-    if (acl::read_tc_timeouts(&n) != cudaSuccess) return ACL_ERR_CUDA;
+    unsigned int n = 0, fa = 0, fk = 0, fc = 0;
+    if (acl::read_tc_timeouts(&n) != cudaSuccess || acl::read_checks_attn(&fa) != cudaSuccess ||
+        acl::read_checks_knn(&fk) != cudaSuccess || acl::read_checks_cluster(&fc) != cudaSuccess)
+        return ACL_ERR_CUDA;
+    if (fa | fk | fc) return ACL_ERR_DEVICE_CHECK;
     return n ? ACL_ERR_TIMEOUT : ACL_OK;
+}
+
+int acl_device_checks_enabled(void) {
+#ifdef ACL_DEVICE_CHECKS
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+acl_status acl_test_set_wait_limit(long long cycles) {
+    return acl::set_tc_wait_cycles(cycles < 0 ? 1000000000LL : cycles) == cudaSuccess ? ACL_OK : ACL_ERR_CUDA;
 }
 
 size_t acl_decoder_layer_workspace(int B, int Q, int N, int d, int D, int K) {

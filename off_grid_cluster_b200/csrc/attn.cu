@@ -107,7 +107,10 @@ __device__ __forceinline__ void warp_sum3(float& x0, float& x1, float& x2, int l
     x2 = __shfl_sync(0xffffffffu, k, 16);
 }
 
-__device__ __forceinline__ int valid_tok(int t, int N) { return (t >= 0 && t < N) ? t : -1; }
+__device__ __forceinline__ int valid_tok(int t, int N) {
+    ACL_DEVICE_CHECK(t >= -1 && t < N);
+    return (t >= 0 && t < N) ? t : -1;
+}
 
 __device__ __forceinline__ float2 sh2(float2 v, int src) {
     return make_float2(__shfl_sync(0xffffffffu, v.x, src), __shfl_sync(0xffffffffu, v.y, src));
@@ -1368,5 +1371,7 @@ cudaError_t launch_attn_bwd(const AttnArgs& a, cudaStream_t st) {
         default: return bwd_dispatch<4>(a, st);
     }
 }
+
+ACL_CHECK_READER(read_checks_attn)
 
 }  // namespace acl

@@ -499,6 +499,7 @@ __global__ void __launch_bounds__(kNbrThreads)
         int cnt = 0;
         for (int s = 0; s < C; ++s) {
             const int t = cl[static_cast<size_t>(g) * C + s];
+            ACL_DEVICE_CHECK(t >= -1 && t < N);
             if (t < 0 || t >= N) continue;
             sx = __dadd_rn(sx, static_cast<double>(img[2 * t]));
             sy = __dadd_rn(sy, static_cast<double>(img[2 * t + 1]));
@@ -605,5 +606,7 @@ cudaError_t launch_neighbors(const float* xy, const int32_t* clusters, int B, in
     note_launch();
     return cudaGetLastError();
 }
+
+ACL_CHECK_READER(read_checks_cluster)
 
 }  // namespace acl

@@ -20,6 +20,33 @@ typedef __nv_bfloat16 bf16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Device-side consistency checks of the check build (compiled with -DACL_DEVICE_CHECKS):
+// ACL_DEVICE_CHECK(cond) records a failed condition in a flag word of the translation unit,
+// which acl_device_check reads (ACL_ERR_DEVICE_CHECK) and clears.  The kernels handle the
+// condition as the regular build does (an out-of-range token id is an empty slot); the check
+// build only reports it.  In the regular build the macro compiles to nothing.
+#ifdef ACL_DEVICE_CHECKS
+static __device__ unsigned int g_check_flags;
+#define ACL_DEVICE_CHECK(cond)                                       \
+    do {                                                             \
+        if (!(cond)) atomicOr(&::acl::g_check_flags, 1u);            \
+    } while (0)
+#define ACL_CHECK_READER(name)                                                      \
+    cudaError_t name(unsigned int* flags) {                                         \
+        cudaError_t e = cudaMemcpyFromSymbol(flags, ::acl::g_check_flags, sizeof(unsigned int)); \
+        if (e != cudaSuccess) return e;                                             \
+        const unsigned int zero = 0u;                                               \
+        return cudaMemcpyToSymbol(::acl::g_check_flags, &zero, sizeof(unsigned int)); \
+    }
+#else
+#define ACL_DEVICE_CHECK(cond) ((void)0)
+#define ACL_CHECK_READER(name)                      \
+    cudaError_t name(unsigned int* flags) {         \
+        *flags = 0u;                                \
+        return cudaSuccess;                         \
+    }
+#endif
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

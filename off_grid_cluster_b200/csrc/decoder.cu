@@ -60,6 +60,11 @@ constexpr long long kTWaitCycles = 1000000000LL;
 constexpr uint32_t kTmemCols = 128;
 
 __device__ unsigned int tc_timeouts;
+// SM clocks a main-loop wait may take before it gives up (kTWaitCycles unless a test lowers
+// it; 0 gives up at once).  The final wait
+// for the MMAs in flight always allows kTWaitCycles, so tensor memory is freed only after
+// the MMAs that use it have completed.
+__device__ long long tc_wait_cycles = kTWaitCycles;
 
 // Shared-memory matrix descriptor: start, leading and stride byte offsets in 16-byte units,
 // descriptor version 1, 128-byte swizzle.
@@ -84,9 +89,11 @@ __host__ __device__ constexpr uint32_t tc_idesc() {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Wait for the phase of the given parity to complete, giving up after kTWaitCycles SM clocks
-// (about half a second): try_wait itself returns after a bounded suspension.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase of the given parity to complete, giving up after `limit` SM clocks
+// (kTWaitCycles: about half a second): try_wait itself returns after a bounded suspension.
+// A limit of 0 gives up at once (a test's way to make every main-loop wait run out).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit = kTWaitCycles) {
+    if (limit <= 0) return false;
     const long long t0 = clock64();
     for (;;) {
         uint32_t done;
@@ -98,7 +105,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
             : "r"(bar), "r"(parity)
             : "memory");
         if (done) return true;
-        if (clock64() - t0 > kTWaitCycles) return false;
+        if (clock64() - t0 > limit) return false;
     }
 }
 
@@ -166,6 +173,7 @@ __global__ void __launch_bounds__(kTThreads)
         if (s < nk) load(s, s);
         cp_async_commit();
     }
+    const long long wait_limit = tc_wait_cycles;
     bool ok = true;
     int issued = 0;  // k-tiles whose MMAs were issued
     for (int kt = 0; kt < nk; ++kt) {
@@ -194,7 +202,7 @@ __global__ void __launch_bounds__(kTThreads)
         issued = kt + 1;
         const int nxt = kt + kTStages - 1;
         if (nxt < nk) {
-            if (kt >= 1) ok = ok && mbar_wait(bar0 + 8 * ((kt - 1) % kTStages), ((kt - 1) / kTStages) & 1);
+            if (kt >= 1) ok = ok && mbar_wait(bar0 + 8 * ((kt - 1) % kTStages), ((kt - 1) / kTStages) & 1, wait_limit);
             if (ok) load(nxt % kTStages, nxt);
         }
         cp_async_commit();
@@ -427,6 +435,10 @@ int dec_wo_splits(int T, int d, int D) {
     if (s > kt) s = kt;
     if (s > kMaxSplits) s = kMaxSplits;
     return s < 1 ? 1 : s;
+}
+
+cudaError_t set_tc_wait_cycles(long long cycles) {
+    return cudaMemcpyToSymbol(tc_wait_cycles, &cycles, sizeof(long long));
 }
 
 cudaError_t read_tc_timeouts(unsigned int* count) {

@@ -218,6 +218,12 @@ DecWorkspace dec_workspace_layout(int B, int Q, int N, int d, int D, int K);
 int dec_wo_splits(int T, int d, int D);
 // reads and clears the count of bounded tensor-core waits that gave up (synchronous)
 cudaError_t read_tc_timeouts(unsigned int* count);
+// sets the give-up limit of the tensor-core GEMM's main-loop waits (synchronous; tests)
+cudaError_t set_tc_wait_cycles(long long cycles);
+// read and clear the device-check flags of each kernel file (always 0 in the regular build)
+cudaError_t read_checks_attn(unsigned int* flags);
+cudaError_t read_checks_knn(unsigned int* flags);
+cudaError_t read_checks_cluster(unsigned int* flags);
 cudaError_t launch_dec_fwd(const DecArgs& a, cudaStream_t st);
 cudaError_t launch_dec_bwd(const DecArgs& a, cudaStream_t st);
 

@@ -343,6 +343,7 @@ __device__ __forceinline__ float load_neighbours(const KnnArgs& a, long long gq,
 #pragma unroll
     for (int j = 0; j < KT; ++j) {
         int t = (j < a.K) ? row[j] : -1;
+        ACL_DEVICE_CHECK(t >= -1 && t < a.N);
         if (t >= a.N) t = -1;
         nb[j].t = t;
         if (t >= 0) {
@@ -409,6 +410,7 @@ __device__ __forceinline__ void row_fma(uint64_t (&acc)[4], uint64_t ww, uint4 f
 __device__ __forceinline__ void one_neighbour(const KnnArgs& a, const int32_t* row, const float2* xyb,
                                               float2 qp, int j, int& t, float& v) {
     t = __ldg(row + j);
+    ACL_DEVICE_CHECK(t >= -1 && t < a.N);
     v = INFINITY;
     if (t >= a.N) t = -1;
     if (t >= 0) {
@@ -658,6 +660,7 @@ __device__ __forceinline__ float group_neighbours(const KnnArgs& a, long long gq
         const int b = static_cast<int>(gq / a.Q);
         const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
         t = a.table[((static_cast<size_t>(b) * a.GH + cy) * a.GW + cx) * a.K + sub];
+        ACL_DEVICE_CHECK(t >= -1 && t < a.N);
         if (t >= a.N) t = -1;
         if (t >= 0) {
             const float2 p = reinterpret_cast<const float2*>(a.xy)[static_cast<size_t>(b) * a.N + t];
@@ -690,6 +693,7 @@ __device__ __forceinline__ float own_neighbour(const KnnArgs& a, long long gq, b
         const int b = static_cast<int>(gq / a.Q);
         const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
         t = a.table[((static_cast<size_t>(b) * a.GH + cy) * a.GW + cx) * a.K + sub];
+        ACL_DEVICE_CHECK(t >= -1 && t < a.N);
         if (t >= a.N) t = -1;
         if (t >= 0) {
             const float2 p = reinterpret_cast<const float2*>(a.xy)[static_cast<size_t>(b) * a.N + t];
@@ -872,10 +876,9 @@ struct CsrSmem {
     size_t pre, off, hash, lanes, ckey, cent, scratch, total;
 };
 __host__ __device__ __forceinline__ CsrSmem csr_smem_layout(int NS) {
-    const size_t n2 = static_cast<size_t>((NS + 1) & ~1);
     CsrSmem L;
     L.pre = 0;
-    L.off = (2 * kCsrWarps * n2 + 15) & ~size_t(15);
+    L.off = (4 * kCsrWarps * static_cast<size_t>(NS) + 15) & ~size_t(15);
     L.hash = L.off + ((4 * static_cast<size_t>(NS + 1) + 15) & ~size_t(15));
     L.lanes = L.hash + 4 * static_cast<size_t>(kCsrHash) * kCsrWarps;
     L.ckey = L.lanes + 4 * 32 * static_cast<size_t>(kCsrWarps);
@@ -897,6 +900,7 @@ __global__ void __launch_bounds__(256) knn_keys_kernel(const KnnArgs a) {
     int32_t* out = a.keys + gq * a.K;
     for (int j = 0; j < a.K; ++j) {
         const int t = __ldg(row + j);
+        ACL_DEVICE_CHECK(t >= -1 && t < a.N);
         out[j] = (t >= a.N) ? -1 : t;
     }
 }
@@ -910,9 +914,11 @@ __global__ void __launch_bounds__(kCsrThreads)
     const int t_lo = static_cast<int>(static_cast<long long>(sl) * N / slices);
     const int t_hi = static_cast<int>(static_cast<long long>(sl + 1) * N / slices);
     const int NS = t_hi - t_lo;
-    const int NS2 = (NS + 1) & ~1;
+    const int NS2 = NS;
     const CsrSmem L = csr_smem_layout((N + slices - 1) / slices);
-    uint16_t* pre = reinterpret_cast<uint16_t*>(smem + L.pre);  // [warps][NS2]
+    // per (warp, token) entry counts, then prefixes: 32-bit, since a token repeated within
+    // table rows can collect up to Q K entries
+    uint32_t* pre = reinterpret_cast<uint32_t*>(smem + L.pre);  // [warps][NS]
     int* off = reinterpret_cast<int*>(smem + L.off);
     uint32_t* hb = reinterpret_cast<uint32_t*>(smem + L.hash) + warp * kCsrHash;
     int* ks = reinterpret_cast<int*>(smem + L.lanes) + warp * 32;
@@ -926,7 +932,7 @@ __global__ void __launch_bounds__(kCsrThreads)
     for (int i = lane; i < kCsrHash; i += 32) hb[i] = 0u;
     const int lo = static_cast<int>(static_cast<long long>(warp) * E / kCsrWarps);
     const int hi = static_cast<int>(static_cast<long long>(warp + 1) * E / kCsrWarps);
-    uint16_t* mine = pre + warp * NS2;
+    uint32_t* mine = pre + warp * NS2;
     const unsigned below_lanes = (1u << lane) - 1u;
     // pass 1: per warp, the entries of the slice and the entries below it
     int cnt = 0, below = 0;
@@ -988,16 +994,14 @@ __global__ void __launch_bounds__(kCsrThreads)
     const int l1 = static_cast<int>(static_cast<long long>(warp + 1) * n / kCsrWarps);
     if (listed) {
         for (int i = l0 + lane; i < l1; i += 32) {
-            const int idx = warp * NS2 + ckey[i];
-            atomicAdd(reinterpret_cast<uint32_t*>(pre) + (idx >> 1), 1u << (16 * (idx & 1)));
+            atomicAdd(pre + warp * NS2 + ckey[i], 1u);
         }
     } else {
         for (int base = lo; base < hi; base += 32) {
             const int e = base + lane;
             const int key = (e < hi) ? __ldg(keys + e) : -1;
             if (key >= t_lo && key < t_hi) {
-                const int idx = warp * NS2 + (key - t_lo);
-                atomicAdd(reinterpret_cast<uint32_t*>(pre) + (idx >> 1), 1u << (16 * (idx & 1)));
+                atomicAdd(pre + warp * NS2 + (key - t_lo), 1u);
             }
         }
     }
@@ -1005,8 +1009,8 @@ __global__ void __launch_bounds__(kCsrThreads)
     for (int t = tid; t < NS; t += kCsrThreads) {
         int run = 0;
         for (int w = 0; w < kCsrWarps; ++w) {
-            const int c = pre[w * NS2 + t];
-            pre[w * NS2 + t] = static_cast<uint16_t>(run);
+            const int c = static_cast<int>(pre[w * NS2 + t]);
+            pre[w * NS2 + t] = static_cast<uint32_t>(run);
             run += c;
         }
         off[t] = run;
@@ -1073,13 +1077,13 @@ __global__ void __launch_bounds__(kCsrThreads)
                 mm &= mm - 1u;
                 if (ks[l] == kk) peers |= 1u << l;
             }
-            before = mine[kk];
+            before = static_cast<int>(mine[kk]);
             const int q = e / K, j = e - q * K;
             csr[off[kk] + before + __popc(peers & below_lanes)] = (q << 4) | j;
         }
         __syncwarp();
         if (in && lane == __ffs(peers) - 1) {
-            mine[kk] = static_cast<uint16_t>(before + __popc(peers));
+            mine[kk] = static_cast<uint32_t>(before + __popc(peers));
             hb[h] = 0u;
         }
         __syncwarp();
@@ -1348,13 +1352,17 @@ int knn_chunks(int Q, int K, int N) {
 }
 
 // token slices of the CSR build per image (B * slices <= 148 CTAs, at most 16)
+// tokens per CSR slice at most, so that the build's shared memory (32-bit counts per warp
+// and token) fits
+constexpr int kCsrMaxSlice = 768;
 int csr_slices(int B, int N) {
     int slices = 148 / (B > 0 ? B : 1);
     if (slices > 16) slices = 16;
     if (slices < 1) slices = 1;
     if (slices > (N + 31) / 32) slices = (N + 31) / 32;
     if (slices < 1) slices = 1;
-    return slices;
+    const int need = (N + kCsrMaxSlice - 1) / kCsrMaxSlice;
+    return slices < need ? need : slices;
 }
 
 // lanes per query: d/8 rounded up to a power of two, capped at 32
@@ -1555,5 +1563,7 @@ cudaError_t launch_knn_bwd(const KnnArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     return launch_knn_bwd_indexed(a, st);
 }
+
+ACL_CHECK_READER(read_checks_knn)
 
 }  // namespace acl

@@ -48,6 +48,14 @@ extern "C" acl_status acl_cluster_attn_bwd_noalloc(
     const size_t need = acl_cluster_attn_workspace(B, N, H, C, M);
     if (need == 0) return ACL_ERR_INVALID_ARG;
     if (need > ACL_NOALLOC_ATTN_WS_BYTES) return ACL_ERR_UNSUPPORTED;
+    // the scratch address is the current device's: a stream of another device is refused
+    if (stream) {
+        int dev = 0, sdev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) != cudaSuccess)
+            return ACL_ERR_CUDA;
+        if (sdev != dev) return ACL_ERR_INVALID_ARG;
+    }
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return ACL_ERR_CUDA;
     return acl_cluster_attn_bwd(Q, K, V, coords, clusters, nbr, bias_coef, B, N, H, D, C, M, scale,

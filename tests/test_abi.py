@@ -41,6 +41,18 @@ def test_library_exports_every_declared_symbol():
     assert set(declared_functions()) == set(acl.SIGNATURES)
 
 
+def test_check_build_exports_the_same_symbols_and_reports_itself():
+    """The check build (ACL_DEVICE_CHECKS: device-side range checks of index inputs) is
+    built from the same sources and exports the same ABI; only it reports checks enabled."""
+    assert os.path.exists(acl.CHECK_LIB_PATH)
+    chk = ct.CDLL(acl.CHECK_LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(chk, n), n
+    chk.acl_device_checks_enabled.restype = ct.c_int
+    assert chk.acl_device_checks_enabled() == 1
+    assert acl.acl_device_checks_enabled() is False
+
+
 def test_status_strings_and_version():
     for code in range(7):
         s = acl.acl_status_string(code)

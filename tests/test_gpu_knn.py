@@ -120,6 +120,31 @@ def test_bwd_deterministic_and_overwrites():
         assert torch.equal(x, y)
 
 
+def test_repeated_ids_beyond_16_bit_counts():
+    """A hand-built table whose rows repeat token ids: every row lists token 0 six times, so
+    token 0 collects 6 Q = 72000 (query, slot) entries in one image, more than a 16-bit count
+    holds.  The inverse index and the token pass must still sum every entry once."""
+    rng = np.random.default_rng(5)
+    B, Q, N, d, K = 1, 12000, 16, 32, 8
+    xy = np.stack([rng.uniform(0, 64, N), rng.uniform(0, 64, N)], -1)[None].astype(np.float32)
+    queries = rng.uniform(0, 64, (B, Q, 2)).astype(np.float32)
+    feats = synth.round_bf16(rng.standard_normal((B, N, d)).astype(np.float32))
+    dout = synth.round_bf16(rng.standard_normal((B, Q, d)).astype(np.float32))
+    p = np.array([1.5], np.float32)
+    table = np.empty((B, 64, 64, K), np.int32)
+    table[..., :6] = 0
+    table[..., 6] = 1 + (np.arange(64 * 64).reshape(64, 64) % (N - 1))
+    table[..., 7] = -1                                    # and one empty slot per row
+    q, f, xyd, tt, pd = dev(queries), bf16(feats), dev(xy), dev(table), dev(p)
+    check_fwd(host(acl.acl_knn_gather_fwd(q, f, xyd, tt, pd)),
+              oracle.knn_fwd(queries, feats, xy, table, p), "out")
+    dF_r, dq_r, dp_r = oracle.knn_bwd(queries, feats, xy, table, p, dout)
+    dF, dq, dp = acl.acl_knn_gather_bwd(q, f, xyd, tt, pd, bf16(dout))
+    check_grad(host(dF), dF_r, "dfeats")
+    check_grad(host(dq), dq_r, "dqueries")
+    check_grad(host(dp), dp_r, "dp")
+
+
 def test_staged_backward_matches_one_call():
     """Index built on a side stream, then the indexed backward: bit-identical results."""
     sb = synth.step_batch(B=2)

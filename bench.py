@@ -105,10 +105,13 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded CPU work of the oracle baseline (seconds)")
-    ap.add_argument("--only", choices=("token_merge", "decoder", "configs", "attn_stage", "knn_stage"),
+    ap.add_argument("--only", choices=("token_merge", "decoder", "configs", "attn_stage", "knn_stage",
+                                       "attn_traffic", "knn_traffic"),
                     default=None,
                     help="run one part alone on one GPU and print its JSON (a short command to "
-                         "profile under ncu); no bench line")
+                         "profile under ncu); no bench line.  attn_traffic / knn_traffic run one "
+                         "stage's calls in the bench's order over inputs larger than L2, for a "
+                         "DRAM-traffic capture whose cache state matches the bench's")
     ap.add_argument("--stage", type=int, default=3, help="stage (1-4) of --only attn_stage / knn_stage")
     return ap.parse_args(argv)
 
@@ -372,6 +375,7 @@ class DeviceStep:
                                                                          stream=st)))
             calls.append(("neighbors", s, lambda st, d=d: acl.acl_neighbors(d["coords"], d["clusters"], 48,
                                                                              nbr=d["nbr"], stream=st)))
+        for s, d in enumerate(self.stages):
             for L in d["layers"]:
                 calls.append(("attn_fwd", s, lambda st, d=d, L=L: acl.acl_cluster_attn_fwd(
                     L["q"], L["k"], L["v"], d["coords"], d["clusters"], d["nbr"], d["bias"], d["scale"],
@@ -396,14 +400,30 @@ class DeviceStep:
     def first_knn(self) -> int:
         return next(i for i, c in enumerate(self.calls) if c[0].startswith("knn"))
 
-    def step(self, stream, events=None):
-        """Every call of the step on `stream`; events[2j], events[2j + 1] bracket call j."""
-        for j, (_, _, fn) in enumerate(self.calls):
+    def step(self, stream, events=None, side=None):
+        """Every call of the step on `stream`; events[2j], events[2j + 1] bracket call j (on the
+        stream the call runs on).  With a `side` stream the clustering and neighbour tables of
+        stages 2..4 run there, concurrently with the stage-1 layers (the clustering kernel
+        takes one CTA per image), and each stage's first layer waits for its own tables."""
+        torch = self.torch
+        ready = {}
+        if side is not None:
+            side.wait_stream(stream)
+        for j, (kind, s, fn) in enumerate(self.calls):
+            on_side = side is not None and kind in ("cluster", "neighbors") and s > 0
+            st = side if on_side else stream
+            if kind == "attn_fwd" and s in ready:
+                stream.wait_event(ready.pop(s))
             if events is not None:
-                events[2 * j].record(stream)
-            fn(stream)
+                events[2 * j].record(st)
+            fn(st)
             if events is not None:
-                events[2 * j + 1].record(stream)
+                events[2 * j + 1].record(st)
+            if on_side and kind == "neighbors":
+                ready[s] = torch.cuda.Event()
+                ready[s].record(side)
+        if side is not None:
+            stream.wait_stream(side)
 
 
 def call_workload(kind: str, B: int, N: int, H: int = 0, d: int = 0, Q: int = QUERIES) -> str:
@@ -437,9 +457,10 @@ def run_gpu(args, rank: int, world: int):
     ds = DeviceStep(hw, device, torch, acl)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     stream = torch.cuda.Stream(device)
+    side = torch.cuda.Stream(device)
     # eager pass of every call (kernel attributes, lazy module loading), then capture
     with torch.cuda.stream(stream):
-        ds.step(stream)
+        ds.step(stream, side=side)
     stream.synchronize()
     n_calls = len(ds.calls)
     reps = max(1, min(args.steps, 3))       # graph copies with their own events, replayed in turn
@@ -449,7 +470,7 @@ def run_gpu(args, rank: int, world: int):
         evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * n_calls)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            ds.step(stream, evs)
+            ds.step(stream, evs, side=side)
         graphs.append(g)
         events.append(evs)
     launches_per_step = (acl.acl_launch_count() - launches0) // reps
@@ -619,8 +640,8 @@ def run_gpu(args, rank: int, world: int):
                              f"launching stream around the steps and between the calls",
                    "parallelism": f"replicas x{world} (images sharded, no collective)"},
         "value_basis": "encoder token-layers of all ranks / the encoder sweep's device time per step "
-                       "(clustering and neighbour tables included; mean of the last timed steps, max over "
-                       "ranks)",
+                       "(clustering and neighbour tables included, those of stages 2-4 on a second stream "
+                       "beside the stage-1 layers; mean of the last timed steps, max over ranks)",
         "segments_ms": {"encoder_sweep": round(span_a, 4), "decoder_gather": round(span_k, 4)},
         "knn": {"value": round(knn_value, 1), "unit": "queries/s",
                 "basis": "decoder queries x stages of all ranks / the gather's device time per step "
@@ -682,6 +703,7 @@ def run_e2e(args, hw: HostWorkload, ds: DeviceStep, stream, torch, acl, device) 
     h2d = sum(h.numel() * h.element_size() for _, h in ds.ins)
     d2h = sum(t.numel() * t.element_size() for t in ds.outs)
     cp_in, cp_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    side = torch.cuda.Stream(device)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
@@ -700,7 +722,7 @@ def run_e2e(args, hw: HostWorkload, ds: DeviceStep, stream, torch, acl, device) 
         if recorded[i]:
             stream.wait_event(ev_out[i])    # step k - 2's outputs have left set i
         with torch.cuda.stream(stream):
-            S.step(stream)
+            S.step(stream, side=side)
         ev_done[i].record(stream)
         cp_out.wait_event(ev_done[i])
         with torch.cuda.stream(cp_out):
@@ -1053,6 +1075,34 @@ def stage_calls(torch, acl, synth, device, stream, which: str, stage: int, B: in
                                                        stream=stream))]
 
 
+def attn_traffic_run(torch, acl, synth, device, stream, stage: int, B: int = IMAGES) -> dict:
+    """One encoder stage's layer, copied until the copies exceed 3 x L2, run as the bench runs
+    its layers: every copy's forward, then the backward of the copies in reverse order.  The
+    last forward and the last backward then read inputs that have left L2, while each
+    backward's key pass still finds what its query pass brought in, as in the bench."""
+    T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
+    s = stage - 1
+    xy_np = synth.sweep_coords(B)[s]
+    ab = synth.attn_sweep_layer(xy_np, s, 0)
+    xy, bias = T(xy_np), T(ab.bias)
+    cl = acl.acl_cluster(xy, stream=stream)
+    nb = acl.acl_neighbors(xy, cl, stream=stream)
+    ws = torch.empty((acl.acl_cluster_attn_workspace(ab.B, ab.N, ab.H, 8, 48),), dtype=torch.uint8, device=device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    layer_bytes = 8 * ab.B * ab.N * ab.H * 64
+    n = max(2, math.ceil(3 * l2 / layer_bytes))
+    base = [T(x, torch.bfloat16) for x in (ab.q, ab.k, ab.v, ab.do)]
+    copies = [[t.clone() for t in base] for _ in range(n)]
+    outs = []
+    with torch.cuda.stream(stream):
+        for q, k, v, do in copies:
+            outs.append(acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, stream=stream))
+        for (q, k, v, do), (o, lse) in reversed(list(zip(copies, outs))):
+            acl.acl_cluster_attn_bwd(q, k, v, xy, cl, nb, bias, ab.scale, o, do, lse, workspace=ws, stream=stream)
+    stream.synchronize()
+    return {"stage": stage, "copies": n, "order": f"attn_fwd x {n}, then attn_bwd x {n} (query, key passes)"}
+
+
 def run_only(args):
     """One part on cuda:0 and its timing dict as JSON.  attn_stage / knn_stage run one
     stage's calls of the benchmark workload eagerly (one warm call each, then one more:
@@ -1073,6 +1123,15 @@ def run_only(args):
         res = decoder_times(torch, acl, synth, device, stream, peaks, B=8)
     elif args.only == "configs":
         res = config_times(torch, acl, synth, device, stream, peaks)
+    elif args.only == "attn_traffic":
+        res = attn_traffic_run(torch, acl, synth, device, stream, args.stage, args.batch)
+    elif args.only == "knn_traffic":
+        calls = stage_calls(torch, acl, synth, device, stream, "knn", args.stage, args.batch)
+        with torch.cuda.stream(stream):
+            for _, fn in calls:  # table, fwd, bwd in the bench's order (inputs above L2 size)
+                fn()
+        stream.synchronize()
+        res = {"stage": args.stage, "launches": [name for name, _ in calls] * 2}
     else:
         which = "attn" if args.only == "attn_stage" else "knn"
         calls = stage_calls(torch, acl, synth, device, stream, which, args.stage, args.batch)

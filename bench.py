@@ -106,7 +106,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded CPU work of the oracle baseline (seconds)")
     ap.add_argument("--only", choices=("token_merge", "decoder", "configs", "attn_stage", "knn_stage",
-                                       "attn_traffic", "knn_traffic"),
+                                       "attn_traffic", "knn_traffic", "attn_fwd_units"),
                     default=None,
                     help="run one part alone on one GPU and print its JSON (a short command to "
                          "profile under ncu); no bench line.  attn_traffic / knn_traffic run one "
@@ -1103,6 +1103,35 @@ def attn_traffic_run(torch, acl, synth, device, stream, stage: int, B: int = IMA
     return {"stage": stage, "copies": n, "order": f"attn_fwd x {n}, then attn_bwd x {n} (query, key passes)"}
 
 
+def attn_fwd_units(torch, acl, synth, device, stream, peaks: dict) -> dict:
+    """The attention forward on the tensor cores (acl_cluster_attn_fwd) and on the FMA pipes
+    only (acl_cluster_attn_fwd_ffma), one layer of 8 images x 2048 tokens x 4 heads: each
+    called eagerly twice (the second launches are the ones to profile), then timed as CUDA
+    graphs."""
+    T = lambda x, dt=None: torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dt)
+    ab = synth.attn_stage1(B=8)
+    xy, bias = T(ab.coords), T(ab.bias)
+    q, k, v = (T(x, torch.bfloat16) for x in (ab.q, ab.k, ab.v))
+    cl = acl.acl_cluster(xy, stream=stream)
+    nb = acl.acl_neighbors(xy, cl, stream=stream)
+    o, lse = acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, stream=stream)
+    calls = {"tensor_core": lambda: acl.acl_cluster_attn_fwd(q, k, v, xy, cl, nb, bias, ab.scale, O=o, lse=lse,
+                                                             stream=stream),
+             "ffma": lambda: acl.acl_cluster_attn_fwd_ffma(q, k, v, xy, cl, nb, bias, ab.scale, O=o, lse=lse,
+                                                           stream=stream)}
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            for fn in calls.values():
+                fn()
+    stream.synchronize()
+    by = attn_bytes(ab.B, ab.N, ab.H)["attn_fwd"]
+    res = {"workload": "8 images x 2048 tokens, H = 4, M = 48"}
+    for name, fn in calls.items():
+        us = graph_time(torch, stream, fn, 20)
+        res[name] = {"us": us, "frac": round(by / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
+    return res
+
+
 def run_only(args):
     """One part on cuda:0 and its timing dict as JSON.  attn_stage / knn_stage run one
     stage's calls of the benchmark workload eagerly (one warm call each, then one more:
@@ -1123,6 +1152,8 @@ def run_only(args):
         res = decoder_times(torch, acl, synth, device, stream, peaks, B=8)
     elif args.only == "configs":
         res = config_times(torch, acl, synth, device, stream, peaks)
+    elif args.only == "attn_fwd_units":
+        res = attn_fwd_units(torch, acl, synth, device, stream, peaks)
     elif args.only == "attn_traffic":
         res = attn_traffic_run(torch, acl, synth, device, stream, args.stage, args.batch)
     elif args.only == "knn_traffic":

@@ -148,6 +148,18 @@ acl_status acl_cluster_attn_fwd(const acl_bf16* Q, const acl_bf16* K, const acl_
                                 const int32_t* nbr, const float* bias_coef,
                                 int B, int N, int H, int D, int C, int M, float scale,
                                 acl_bf16* O, float* lse, acl_stream_t stream);
+/*
+ * acl_cluster_attn_fwd_ffma -- the same forward computed on the FMA pipes only (fp32 dot
+ * products and sums, no tensor-core instruction): the reference variant the tensor-core
+ * kernel of acl_cluster_attn_fwd is measured against (the pages' kernel choice, tensor cores
+ * or FMA on the 8 x 48 tiles, rests on that comparison).  Arguments, layouts, limits, errors
+ * and results as acl_cluster_attn_fwd (results equal up to fp32 rounding order).
+ */
+acl_status acl_cluster_attn_fwd_ffma(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V,
+                                     const float* coords, const int32_t* clusters,
+                                     const int32_t* nbr, const float* bias_coef,
+                                     int B, int N, int H, int D, int C, int M, float scale,
+                                     acl_bf16* O, float* lse, acl_stream_t stream);
 
 /*
  * acl_cluster_attn_bwd -- local cluster attention, backward (a4), recomputing

@@ -38,6 +38,8 @@ SIGNATURES = {
     "acl_cluster_attn_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "acl_cluster_attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F,
                                   _P, _P, _P]),
+    "acl_cluster_attn_fwd_ffma": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F,
+                                       _P, _P, _P]),
     "acl_cluster_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F,
                                   _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "acl_cluster_attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
@@ -203,6 +205,19 @@ def acl_cluster_attn_fwd(Q, K, V, coords, clusters, nbr, bias_coef, scale: float
     O = _out(O, (B, N, H, D), torch.bfloat16, Q, "O")
     lse = _out(lse, (B, N, H), torch.float32, Q, "lse")
     _call("acl_cluster_attn_fwd", _ptr(Q), _ptr(K), _ptr(V), _ptr(coords), _ptr(clusters),
+          _ptr(nbr), _ptr(bias_coef), B, N, H, D, C, M, scale, _ptr(O), _ptr(lse),
+          _stream(stream))
+    return O, lse
+
+
+def acl_cluster_attn_fwd_ffma(Q, K, V, coords, clusters, nbr, bias_coef, scale: float | None = None,
+                              O=None, lse=None, stream=None):
+    """The forward on the FMA pipes only (the tensor-core kernel's reference variant)."""
+    B, N, H, D, C, M = _attn_shapes(Q, K, V, coords, clusters, nbr, bias_coef)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    O = _out(O, (B, N, H, D), torch.bfloat16, Q, "O")
+    lse = _out(lse, (B, N, H), torch.float32, Q, "lse")
+    _call("acl_cluster_attn_fwd_ffma", _ptr(Q), _ptr(K), _ptr(V), _ptr(coords), _ptr(clusters),
           _ptr(nbr), _ptr(bias_coef), B, N, H, D, C, M, scale, _ptr(O), _ptr(lse),
           _stream(stream))
     return O, lse

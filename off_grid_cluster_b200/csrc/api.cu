@@ -175,6 +175,23 @@ acl_status acl_cluster_attn_fwd(const acl_bf16* Q, const acl_bf16* K, const acl_
     return cuda_status(acl::launch_attn_fwd(a, S(stream)));
 }
 
+acl_status acl_cluster_attn_fwd_ffma(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V,
+                                     const float* coords, const int32_t* clusters, const int32_t* nbr,
+                                     const float* bias_coef, int B, int N, int H, int D, int C, int M,
+                                     float scale, acl_bf16* O, float* lse, acl_stream_t stream) {
+    acl_status st = check_attn(Q, K, V, coords, clusters, nbr, bias_coef, B, N, H, D, C, M);
+    if (st != ACL_OK) return st;
+    if (!O || !lse) return ACL_ERR_INVALID_ARG;
+    if (!aligned(O, 16)) return ACL_ERR_INVALID_ARG;
+    acl::AttnArgs a = {};
+    a.q = BF(Q); a.k = BF(K); a.v = BF(V);
+    a.xy = coords; a.clusters = clusters; a.nbr = nbr; a.bias = bias_coef;
+    a.B = B; a.N = N; a.H = H; a.G = (N + C - 1) / C; a.M = M; a.R = M / C;
+    a.scale = scale;
+    a.o = BFm(O); a.lse = lse;
+    return cuda_status(acl::launch_attn_fwd_ffma(a, S(stream)));
+}
+
 acl_status acl_cluster_attn_bwd(const acl_bf16* Q, const acl_bf16* K, const acl_bf16* V,
                                 const float* coords, const int32_t* clusters, const int32_t* nbr,
                                 const float* bias_coef, int B, int N, int H, int D, int C, int M,

@@ -110,6 +110,8 @@ struct AttnWorkspace {
 AttnWorkspace attn_workspace_layout(int B, int N, int H, int C, int M);
 
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t st);
+// the same forward on the FMA pipes only (attn_ffma.cu): the tensor-core kernel's reference
+cudaError_t launch_attn_fwd_ffma(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_attn_bwd(const AttnArgs& a, cudaStream_t st);
 
 struct KnnArgs {

@@ -46,6 +46,29 @@ def test_tiny():
     run_attn(synth.attn_tiny())
 
 
+def ffma_fwd(a: synth.AttnBatch, M: int = 48):
+    """The FMA-only forward (the tensor-core kernel's reference variant) against the oracle."""
+    cl = oracle.cluster(a.coords, 8)
+    nb = oracle.neighbors(a.coords, cl, M)
+    o_ref, lse_ref = oracle.attn_fwd(a.q, a.k, a.v, a.coords, cl, nb, a.bias, a.scale)
+    O, lse = acl.acl_cluster_attn_fwd_ffma(bf16(a.q), bf16(a.k), bf16(a.v), dev(a.coords), dev(cl), dev(nb),
+                                           dev(a.bias), a.scale)
+    check_fwd(host(O), o_ref, "O (FMA variant)")
+    assert np.abs(host(lse) - lse_ref).max() <= LSE_ATOL
+
+
+@pytest.mark.parametrize("case", ["stage1_b8", "stage3", "M64_ragged", "tiny"])
+def test_ffma_forward_variant(case):
+    if case == "stage1_b8":
+        ffma_fwd(synth.attn_stage1(B=8))
+    elif case == "stage3":
+        ffma_fwd(synth.attn_stage3(B=8))
+    elif case == "M64_ragged":
+        ffma_fwd(synth.attn_stage1(B=2, N=701, H=3), M=64)
+    else:
+        ffma_fwd(synth.attn_tiny())
+
+
 def test_stage1_full_batch():
     # 8 images x 2048 tokens x 4 heads: the benchmark workload's attention, every output
     run_attn(synth.attn_stage1())

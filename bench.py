@@ -68,15 +68,16 @@ KERNELS = {
     "attn_bwd": ["attn_bwd_query_kernel", "attn_bwd_key_kernel"],
     "knn_table": ["knn_table_kernel"],
     "knn_fwd": ["knn_fwd_*"],
-    "knn_bwd": ["knn_keys_kernel", "knn_csr_*", "knn_bwd_query_*", "knn_bwd_token_*"],
+    "knn_index": ["knn_keys_kernel", "knn_csr_kernel"],
+    "knn_bwd": ["knn_bwd_query_*", "knn_bwd_token_*"],
 }
 # the files whose code makes each call's kernels: a DRAM-traffic figure taken by ncu on
 # other sources than the current ones is stale and is reported as null
 TRAFFIC_SOURCES = {
-    "attn_fwd": ("attn.cu", "common.cuh", "internal.h"),
-    "attn_bwd": ("attn.cu", "common.cuh", "internal.h"),
-    "knn_fwd": ("knn.cu", "common.cuh", "internal.h"),
-    "knn_bwd": ("knn.cu", "common.cuh", "internal.h"),
+    "attn_fwd": ("attn.cu", "common.cuh"),
+    "attn_bwd": ("attn.cu", "common.cuh"),
+    "knn_fwd": ("knn.cu", "common.cuh"),
+    "knn_bwd": ("knn.cu", "common.cuh"),
 }
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
@@ -175,7 +176,10 @@ def knn_bytes(B: int, Q: int, N: int, d: int, K: int = KNN_K) -> dict:
     and dOut and writes dq (8 B); per token the features (2d B) and coordinates (8 B) are
     read once and the backward writes dF (2d B)."""
     return {"knn_fwd": B * (Q * (8 + 4 * K + 2 * d) + N * (2 * d + 8)),
-            "knn_bwd": B * (Q * (8 + 4 * K + 8 + 2 * d) + N * (4 * d + 8))}
+            "knn_bwd": B * (Q * (8 + 4 * K + 8 + 2 * d) + N * (4 * d + 8)),
+            # inverse index: positions and table rows in, the entries' tokens and their
+            # token-sorted order out, one offset per token
+            "knn_index": B * (Q * (8 + 12 * K) + 4 * (N + 1))}
 
 
 def table_bytes(B: int, N: int, C: int = 8, M: int = 48, GH: int = GRID, GW: int = GRID,
@@ -357,15 +361,16 @@ class DeviceStep:
                      table=e((B, k["GH"], k["GW"], k["K"]), i32), out=e((B, k["Q"], k["d"]), bf),
                      dfeats=e((B, k["N"], k["d"]), bf), dq=e((B, k["Q"], 2), f32), dp=e((k["d"] // 32,), f32))
             self.outs += [d[n] for n in ("table", "out", "dfeats", "dq", "dp")]
-            ws_knn = max(ws_knn, acl.acl_knn_gather_workspace(B, k["Q"], k["N"], k["d"], k["K"]))
+            # each stage's inverse index lives in its own workspace from its build to its backward
+            d["ws"] = e((max(acl.acl_knn_gather_workspace(B, k["Q"], k["N"], k["d"], k["K"]), 1),), torch.uint8)
+            ws_knn += d["ws"].numel()
             self.knn.append(d)
-        # the calls run one at a time on one stream, so one workspace of each kind serves all
+        # the attention calls run one at a time on one stream: one workspace serves them all
         self.ws_attn = e((max(ws_attn, 1),), torch.uint8)
-        self.ws_knn = e((max(ws_knn, 1),), torch.uint8)
         self.calls = self._calls()
 
     def bytes(self) -> int:
-        ts = [t for t, _ in self.ins] + self.outs + [self.ws_attn, self.ws_knn]
+        ts = [t for t, _ in self.ins] + self.outs + [self.ws_attn] + [k["ws"] for k in self.knn]
         return sum(t.numel() * t.element_size() for t in ts)
 
     def _calls(self):
@@ -390,11 +395,13 @@ class DeviceStep:
         for s, k in enumerate(self.knn):
             calls.append(("knn_table", s, lambda st, k=k: acl.acl_knn_table(k["coords"], k["GH"], k["GW"], k["K"],
                                                                              table=k["table"], stream=st)))
+            calls.append(("knn_index", s, lambda st, k=k: acl.acl_knn_gather_index(
+                k["queries"], k["table"], k["feats"].shape[1], k["feats"].shape[2], k["ws"], stream=st)))
             calls.append(("knn_fwd", s, lambda st, k=k: acl.acl_knn_gather_fwd(
                 k["queries"], k["feats"], k["coords"], k["table"], k["p"], out=k["out"], stream=st)))
-            calls.append(("knn_bwd", s, lambda st, k=k: acl.acl_knn_gather_bwd(
-                k["queries"], k["feats"], k["coords"], k["table"], k["p"], k["dout"], k["dfeats"], k["dq"],
-                k["dp"], workspace=self.ws_knn, stream=st)))
+            calls.append(("knn_bwd", s, lambda st, k=k: acl.acl_knn_gather_bwd_indexed(
+                k["queries"], k["feats"], k["coords"], k["table"], k["p"], k["dout"], k["ws"], dfeats=k["dfeats"],
+                dqueries=k["dq"], dp=k["dp"], stream=st)))
         return calls
 
     def first_knn(self) -> int:
@@ -409,19 +416,33 @@ class DeviceStep:
         ready = {}
         if side is not None:
             side.wait_stream(stream)
+        # decoder gather: the table of stage 1 on the main stream; every stage's inverse index
+        # and the tables of stages 2..4 on the side stream (in stage order), so they overlap the
+        # gathers; a stage's forward waits for its table, its backward for its index
+        side_kinds = ("cluster", "neighbors", "knn_table", "knn_index")
         for j, (kind, s, fn) in enumerate(self.calls):
-            on_side = side is not None and kind in ("cluster", "neighbors") and s > 0
+            on_side = side is not None and kind in side_kinds and (s > 0 or kind == "knn_index")
             st = side if on_side else stream
-            if kind == "attn_fwd" and s in ready:
-                stream.wait_event(ready.pop(s))
+            if side is not None:
+                if kind == "attn_fwd" and ("nbr", s) in ready:
+                    stream.wait_event(ready.pop(("nbr", s)))
+                if kind == "knn_fwd" and ("table", s) in ready:
+                    stream.wait_event(ready.pop(("table", s)))
+                if kind == "knn_bwd" and ("index", s) in ready:
+                    stream.wait_event(ready.pop(("index", s)))
+                if kind == "knn_index" and s == 0:
+                    side.wait_event(ready.pop(("table0",)))
             if events is not None:
                 events[2 * j].record(st)
             fn(st)
             if events is not None:
                 events[2 * j + 1].record(st)
-            if on_side and kind == "neighbors":
-                ready[s] = torch.cuda.Event()
-                ready[s].record(side)
+            if side is not None:
+                tag = {"neighbors": "nbr", "knn_table": "table", "knn_index": "index"}.get(kind)
+                if tag is not None:
+                    ev = torch.cuda.Event()
+                    ev.record(st)
+                    ready[(tag, s) if (on_side or tag != "table") else ("table0",)] = ev
         if side is not None:
             stream.wait_stream(side)
 
@@ -538,7 +559,7 @@ def run_gpu(args, rank: int, world: int):
         g["launches"] += 1
         g["ms"] += dur[j]
     for (kind, s), g in groups.items():
-        if kind in ("knn_table", "knn_fwd", "knn_bwd"):
+        if kind in ("knn_table", "knn_index", "knn_fwd", "knn_bwd"):
             k = hw.knn[s]
             by = {**knn_bytes(B, k["Q"], k["N"], k["d"], k["K"]), **table_bytes(B, k["N"])}
             g["workload"] = call_workload(kind, B, k["N"], d=k["d"], Q=k["Q"])
@@ -571,7 +592,7 @@ def run_gpu(args, rank: int, world: int):
                 else "fallback"}
 
     attn_kinds = ("cluster", "neighbors", "attn_fwd", "attn_bwd")
-    knn_kinds = ("knn_table", "knn_fwd", "knn_bwd")
+    knn_kinds = ("knn_table", "knn_index", "knn_fwd", "knn_bwd")
     rf_attn = roofline(attn_kinds, span_a)
     rf_knn = roofline(knn_kinds, span_k)
 
@@ -581,7 +602,7 @@ def run_gpu(args, rank: int, world: int):
         by = sum(g["bytes"] * g["launches"] for g in groups.values() if g["kind"] in kinds)
         return ms, by / (ms * 1e-3) / 1e9 / hbm
     attn_fb_ms, attn_fb_frac = span_of(("attn_fwd", "attn_bwd"))
-    knn_fb_ms, knn_fb_frac = span_of(("knn_fwd", "knn_bwd"))
+    knn_fb_ms, knn_fb_frac = span_of(("knn_index", "knn_fwd", "knn_bwd"))
     per_stage = []
     for s, st in enumerate(hw.stages):
         f, b = groups[("attn_fwd", s)], groups[("attn_bwd", s)]
@@ -596,6 +617,7 @@ def run_gpu(args, rank: int, world: int):
     for s, k in enumerate(hw.knn):
         t, f, b = groups[("knn_table", s)], groups[("knn_fwd", s)], groups[("knn_bwd", s)]
         knn_stage.append({"stage": s + 1, "N": k["N"], "d": k["d"], "table_us": round(t["us"], 2),
+                          "index_us": round(groups[("knn_index", s)]["us"], 2),
                           "fwd_us": round(f["us"], 2), "bwd_us": round(b["us"], 2),
                           "fwd_frac": round(f["frac"], 4), "bwd_frac": round(b["frac"], 4),
                           "fwd_bwd_frac": round((f["bytes"] + b["bytes"]) / ((f["us"] + b["us"]) * 1e-6)
@@ -645,9 +667,10 @@ def run_gpu(args, rank: int, world: int):
         "segments_ms": {"encoder_sweep": round(span_a, 4), "decoder_gather": round(span_k, 4)},
         "knn": {"value": round(knn_value, 1), "unit": "queries/s",
                 "basis": "decoder queries x stages of all ranks / the gather's device time per step "
-                         "(KNN tables included)",
-                "gather_fwd_bwd_queries_per_s": round(query_stages / (knn_fb_ms * 1e-3), 1),
-                "gather_fwd_bwd_frac": round(knn_fb_frac, 4), "stages": knn_stage},
+                         "(KNN tables and inverse indexes included, those on a second stream beside "
+                         "the gathers)",
+                "gather_index_fwd_bwd_queries_per_s": round(query_stages / (knn_fb_ms * 1e-3), 1),
+                "gather_index_fwd_bwd_frac": round(knn_fb_frac, 4), "stages": knn_stage},
         "roofline": rf_attn,
         "roofline_knn": rf_knn,
         "parts": {

@@ -646,51 +646,12 @@ __global__ void __launch_bounds__(kGatherThreads) knn_bwd_query_kernel(const Knn
 // distances with width-limited shuffles, instead of every lane recomputing all K.  A CTA
 // walks `iters` consecutive blocks of queries, so neighbouring queries (which share most
 // of their tokens) run on one SM and find each other's feature rows in L1.
-struct GroupNbrs {
-    int t;
-    float v, ux, uy;  // id, weight exponent knn_v(d), (q - p) * knn_dq_factor(d)
-};
-
-template <int KT>
-__device__ __forceinline__ float group_neighbours(const KnnArgs& a, long long gq, bool live, float2 qp,
-                                                  int sub, int LPQ, GroupNbrs (&nb)[KT]) {
-    int t = -1;
-    float v = INFINITY, ux = 0.f, uy = 0.f;
-    if (live && sub < a.K) {
-        const int b = static_cast<int>(gq / a.Q);
-        const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
-        t = a.table[((static_cast<size_t>(b) * a.GH + cy) * a.GW + cx) * a.K + sub];
-        ACL_DEVICE_CHECK(t >= -1 && t < a.N);
-        if (t >= a.N) t = -1;
-        if (t >= 0) {
-            const float2 p = reinterpret_cast<const float2*>(a.xy)[static_cast<size_t>(b) * a.N + t];
-            const float dx = qp.x - p.x, dy = qp.y - p.y;
-            const float d = sqrtf(dx * dx + dy * dy);
-            v = knn_v(d, a.kind);
-            const float f = knn_dq_factor(d, a.kind);
-            ux = dx * f;
-            uy = dy * f;
-        }
-    }
-    float vmin = v;
-    for (int o = 1; o < LPQ; o <<= 1) vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o, LPQ));
-#pragma unroll
-    for (int j = 0; j < KT; ++j) {
-        nb[j].t = __shfl_sync(0xffffffffu, t, j, LPQ);
-        nb[j].v = __shfl_sync(0xffffffffu, v, j, LPQ);
-        nb[j].ux = __shfl_sync(0xffffffffu, ux, j, LPQ);
-        nb[j].uy = __shfl_sync(0xffffffffu, uy, j, LPQ);
-    }
-    return vmin;
-}
-
 // The neighbour that lane sub (< K) of a query's lane group owns: token id, weight
 // exponent v = knn_v(d), and (q - p) * knn_dq_factor(d); returns the group's minimum v.
-__device__ __forceinline__ float own_neighbour(const KnnArgs& a, long long gq, bool live, float2 qp,
+__device__ __forceinline__ float own_neighbour(const KnnArgs& a, int b, bool live, float2 qp,
                                                int sub, int LPQ, int& t, float& v, float& ux,
                                                float& uy) {
     if (live && sub < a.K) {
-        const int b = static_cast<int>(gq / a.Q);
         const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
         t = a.table[((static_cast<size_t>(b) * a.GH + cy) * a.GW + cx) * a.K + sub];
         ACL_DEVICE_CHECK(t >= -1 && t < a.N);
@@ -722,33 +683,63 @@ __global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 4 : 2)
     for (int i = threadIdx.x; i < nslots; i += kGatherThreads) sdp[i] = 0.f;
     __syncthreads();
     const long long total = static_cast<long long>(a.B) * a.Q;
+    // image of the lane's query and its first query, advanced without divisions
+    const long long gq0 = (static_cast<long long>(blockIdx.x) * iters * kGatherWarps + warp) * QPW + grp;
+    int bq = static_cast<int>(gq0 / a.Q);
+    long long qb = static_cast<long long>(bq) * a.Q;
     for (int it = 0; it < iters; ++it) {
-        const long long gq = ((static_cast<long long>(blockIdx.x) * iters + it) * kGatherWarps + warp) * QPW + grp;
+        const long long gq = gq0 + static_cast<long long>(it) * kGatherWarps * QPW;
         if ((gq - grp) >= total) break;  // uniform per warp
+        while (gq - qb >= a.Q) {
+            ++bq;
+            qb += a.Q;
+        }
         const bool live = gq < total;
+        const int b = live ? bq : 0;
         const float2 qp = live ? reinterpret_cast<const float2*>(a.queries)[gq] : make_float2(0.f, 0.f);
         // lane j < K of the group owns neighbour j; every lane gets all K token ids
         int my_t = -1;
         float my_v = INFINITY, my_ux = 0.f, my_uy = 0.f;
-        const float vmin = own_neighbour(a, gq, live, qp, sub, LPQ, my_t, my_v, my_ux, my_uy);
-        int tk[KT];
-#pragma unroll
-        for (int j = 0; j < KT; ++j) tk[j] = __shfl_sync(0xffffffffu, my_t, j, LPQ);
-        const int b = live ? static_cast<int>(gq / a.Q) : 0;
-        const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d;
+        const float vmin = own_neighbour(a, b, live, qp, sub, LPQ, my_t, my_v, my_ux, my_uy);
         const int r = sub & 3;  // lane within the 4 lanes of a head
         constexpr int KQ = KT / 4;  // neighbours per lane after the reduce-scatter: j = r + 4 u
+        // every neighbour's row (this lane's first channel; row 0 for an empty slot), and the
+        // token, weight exponent and dq factor of this lane's neighbours j = r + 4 u: fixed for
+        // the query, so taken once before the channel passes
+        const bf16* rowp[KT];
+        bool has[KT];
+        {
+            const bf16* fb = a.feats + static_cast<size_t>(b) * a.N * a.d + sub * 8;
+#pragma unroll
+            for (int j = 0; j < KT; ++j) {
+                const int tj = __shfl_sync(0xffffffffu, my_t, j, LPQ);
+                has[j] = live && tj >= 0;
+                rowp[j] = fb + static_cast<size_t>(tj < 0 ? 0 : tj) * a.d;
+            }
+        }
+        float vj[KQ], uxj[KQ], uyj[KQ];
+        bool okq[KQ];
+#pragma unroll
+        for (int u = 0; u < KQ; ++u) {
+            const int j = r + 4 * u;
+            const int t = __shfl_sync(0xffffffffu, my_t, j, LPQ);
+            vj[u] = __shfl_sync(0xffffffffu, my_v, j, LPQ);
+            uxj[u] = __shfl_sync(0xffffffffu, my_ux, j, LPQ);
+            uyj[u] = __shfl_sync(0xffffffffu, my_uy, j, LPQ);
+            okq[u] = live && j < a.K && t >= 0;
+        }
+        const bf16* gb = a.dout + static_cast<size_t>(live ? gq : 0) * a.d + sub * 8;
         float dqx = 0.f, dqy = 0.f;
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch) {
-            const int c0 = ch * LPQ * 8 + sub * 8;
+            // passes after the first exist only with LPQ = 32: pass ch starts at channel 256 ch
+            const int c0 = ch * 256 + sub * 8;
             const bool on = live && c0 < a.d;
             const int hh = on ? (c0 >> 5) : 0;
             const float ph = on ? a.p[hh] : 0.f;
             float g[8];
             {
-                const uint4 gv = on ? ldg16(a.dout + static_cast<size_t>(gq) * a.d + c0)
-                                    : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 gv = on ? ldg16(gb + ch * 256) : make_uint4(0u, 0u, 0u, 0u);
                 const uint32_t u[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -762,8 +753,7 @@ __global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 4 : 2)
                 uint4 f[KT];
 #pragma unroll
                 for (int j = 0; j < KT; ++j)
-                    f[j] = (on && tk[j] >= 0) ? ldg16(fb + static_cast<size_t>(tk[j]) * a.d + c0)
-                                              : make_uint4(0u, 0u, 0u, 0u);
+                    f[j] = (on && has[j]) ? ldg16(rowp[j] + ch * 256) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                 for (int j = 0; j < KT; ++j) {
                     const uint32_t u[4] = {f[j].x, f[j].y, f[j].z, f[j].w};
@@ -783,7 +773,7 @@ __global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 4 : 2)
                 const float keep = (r & 2) ? dwp[jhi] : dwp[jlo];
                 dh[s2] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
             }
-            float dw[KQ], w[KQ], vj[KQ], uxj[KQ], uyj[KQ];
+            float dw[KQ], w[KQ];
             bool okj[KQ];
             float sum = 0.f;
 #pragma unroll
@@ -791,12 +781,7 @@ __global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 4 : 2)
                 const float send = (r & 1) ? dh[2 * u] : dh[2 * u + 1];
                 const float keep = (r & 1) ? dh[2 * u + 1] : dh[2 * u];
                 dw[u] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-                const int j = r + 4 * u;
-                const int t = __shfl_sync(0xffffffffu, my_t, j, LPQ);
-                vj[u] = __shfl_sync(0xffffffffu, my_v, j, LPQ);
-                uxj[u] = __shfl_sync(0xffffffffu, my_ux, j, LPQ);
-                uyj[u] = __shfl_sync(0xffffffffu, my_uy, j, LPQ);
-                okj[u] = on && j < a.K && t >= 0;
+                okj[u] = on && okq[u];
                 w[u] = okj[u] ? knn_weight(vj[u], vmin, ph) : 0.f;
                 sum += w[u];
             }

@@ -53,7 +53,7 @@ namespace {
 constexpr int kWarps = 4;               // warps per CTA (independent pipelines)
 constexpr int kThreads = 32 * kWarps;
 constexpr int kRowB = 64;               // bytes of one head of one token (32 bf16)
-constexpr int kChunk = 6;               // listed query clusters per key-pass item
+constexpr int kChunk = 4;               // listed query clusters per key-pass item
 constexpr int kMaxPlanWarps = 8192;     // key-pass warps a workspace plan can describe
 
 // ---------------------------------------------------------------- small helpers

@@ -30,6 +30,8 @@
 #include <float.h>
 #include <math.h>
 
+#include <cuda_fp16.h>
+
 #include "internal.h"
 
 namespace acl {
@@ -827,6 +829,279 @@ __global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 4 : 2)
     }
 }
 
+// Query side of the backward on the tensor cores, for images of at most kUTMaxN tokens and
+// K <= 8: a CTA takes tiles of 16 consecutive queries of one image.  The tile's (query, slot)
+// entries name at most 128 tokens; their union U (ascending token id, found with a bitmap of
+// the image's tokens and prefix popcounts) is staged once for the tile, so one row of F serves
+// every query of the tile that lists it.  Per head, dW (16 x U) = dO_h (16 x 32) F_U,h^T is
+// one row of m16n8k16 bf16 products (fp32 accumulation; both operands exact in bf16), written
+// to the warp's shared dW tile in fp16 (2^-11 relative, far inside the gradients' tolerance;
+// it halves the tile, so four CTAs fit an SM); each (query, slot) then reads its dw at its
+// token's union position and the rest is the per-query algebra of the FMA query pass: w = 2^(p e) / S,
+// ds = w (dw - sum w dw), dp and dq partials, w stored as [q][slot][head].  Thread (q, k) of
+// the CTA's 128 builds the tile's entry (q, k); warp w takes heads w, w + 4, ...; dq adds the
+// warps' partials in warp order and dp leaves each warp in a fixed order: bit-reproducible.
+constexpr int kUTWarps = 4;
+constexpr int kUTThreads = 32 * kUTWarps;
+constexpr int kUTMaxN = 2048;             // bitmap capacity (tokens per image)
+constexpr int kUTUseN = 1024;             // images of at most this many tokens take this pass
+                                          // (at 2048 tokens the FMA pass measured faster)
+constexpr int kUTMaxU = 128;              // 16 queries x 8 slots
+constexpr int kUTDS = kUTMaxU + 4;        // row stride of a warp's dW tile (floats)
+constexpr int kUTFBytes = 16 * 1024;      // F rows of one head group
+constexpr int kUTMaxGroup = 8;            // heads staged together (dO: 1 KB each)
+
+struct UTSmem {
+    size_t bits, pre, utok, qloc, qe, qz, qu, dqred, dw, fbuf, dobuf, total;
+};
+__host__ __device__ __forceinline__ UTSmem ut_smem_layout() {
+    UTSmem L;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = (o + bytes + 127) & ~size_t(127);
+        return at;
+    };
+    L.bits = take(4 * (kUTMaxN / 32));
+    L.pre = take(4 * (kUTMaxN / 32 + 1));
+    L.utok = take(4 * kUTMaxU);
+    L.qloc = take(4 * kUTMaxU);
+    L.qe = take(4 * kUTMaxU);
+    L.qz = take(4 * kUTMaxU);
+    L.qu = take(8 * kUTMaxU);
+    L.dqred = take(8 * kUTWarps * 16);
+    L.dw = take(2 * kUTWarps * 16 * kUTDS);
+    L.fbuf = take(kUTFBytes);
+    L.dobuf = take(1024 * kUTMaxGroup);
+    L.total = o;
+    return L;
+}
+
+__global__ void __launch_bounds__(kUTThreads)
+    knn_bwd_query_union_kernel(const KnnArgs a, long long tiles_per_image, long long tile_span) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const UTSmem L = ut_smem_layout();
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L.bits);
+    int* pre = reinterpret_cast<int*>(smem + L.pre);
+    int* utok = reinterpret_cast<int*>(smem + L.utok);
+    int* qloc = reinterpret_cast<int*>(smem + L.qloc);
+    float* qe = reinterpret_cast<float*>(smem + L.qe);
+    float* qz = reinterpret_cast<float*>(smem + L.qz);
+    float2* qu = reinterpret_cast<float2*>(smem + L.qu);
+    float2* dqred = reinterpret_cast<float2*>(smem + L.dqred);
+    const uint32_t fb0 = smem_addr(smem + L.fbuf), db0 = smem_addr(smem + L.dobuf);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __half* dws = reinterpret_cast<__half*>(smem + L.dw) + warp * 16 * kUTDS;
+    const int NH = a.d >> 5, NW = (a.N + 31) >> 5;
+    const int K = a.K;
+    // this lane's four (query, slot) pairs in the per-head algebra: q = lane / 2, k = 4 (lane & 1) + i
+    const int pq = lane >> 1, pk0 = 4 * (lane & 1);
+    float dpa[8];  // dp partials of this warp's heads h = warp + 4 s (s < 8 covers NH <= 32)
+#pragma unroll
+    for (int s = 0; s < 8; ++s) dpa[s] = 0.f;
+    const long long total_tiles = static_cast<long long>(a.B) * tiles_per_image;
+    const long long t0 = static_cast<long long>(blockIdx.x) * tile_span;
+    const long long t1 = t0 + tile_span < total_tiles ? t0 + tile_span : total_tiles;
+    for (long long tile = t0; tile < t1; ++tile) {
+        const int b = static_cast<int>(tile / tiles_per_image);
+        const int qt0 = static_cast<int>(tile - static_cast<long long>(b) * tiles_per_image) * 16;
+        const int nq = min(16, a.Q - qt0);
+        // ---- the tile's entries: thread (q, k) = (tid / 8, tid % 8)
+        const int eq = tid >> 3, ek = tid & 7;
+        const bool qlive = eq < nq;
+        const long long gq_e = static_cast<long long>(b) * a.Q + qt0 + eq;
+        int t = -1;
+        float v = INFINITY, z = 0.f;
+        float2 u = make_float2(0.f, 0.f);
+        if (qlive && ek < K) {
+            const float2 qp = __ldg(reinterpret_cast<const float2*>(a.queries) + gq_e);
+            const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
+            t = __ldg(a.table + ((static_cast<size_t>(b) * a.GH + cy) * a.GW + cx) * K + ek);
+            ACL_DEVICE_CHECK(t >= -1 && t < a.N);
+            if (t >= a.N) t = -1;
+            if (t >= 0) {
+                const float2 p = __ldg(reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(b) * a.N + t);
+                const float dx = qp.x - p.x, dy = qp.y - p.y;
+                const float d = sqrtf(dx * dx + dy * dy);
+                v = knn_v(d, a.kind);
+                z = knn_dzdp(v);
+                const float f = knn_dq_factor(d, a.kind);
+                u = make_float2(dx * f, dy * f);
+            }
+        }
+        float vmin = v;
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, 1));
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, 2));
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, 4));
+        for (int i = tid; i < NW; i += kUTThreads) bits[i] = 0u;
+        __syncthreads();
+        if (t >= 0) atomicOr(&bits[t >> 5], 1u << (t & 31));
+        __syncthreads();
+        // exclusive prefix of the words' popcounts (warp 0; NW <= 64)
+        if (warp == 0) {
+            const int c0 = lane < NW ? __popc(bits[lane]) : 0;
+            const int c1 = lane + 32 < NW ? __popc(bits[lane + 32]) : 0;
+            int s0 = c0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, s0, o);
+                if (lane >= o) s0 += y;
+            }
+            const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+            int s1 = c1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, s1, o);
+                if (lane >= o) s1 += y;
+            }
+            if (lane < NW) pre[lane] = s0 - c0;
+            if (lane + 32 < NW) pre[lane + 32] = tot0 + s1 - c1;
+            if (lane == 31) pre[64] = tot0 + s1;
+        }
+        __syncthreads();
+        const int U = pre[64];
+        const int loc = t >= 0 ? pre[t >> 5] + __popc(bits[t >> 5] & ((1u << (t & 31)) - 1u)) : -1;
+        if (t >= 0) utok[loc] = t;  // entries of one token write the same value
+        qloc[tid] = loc;
+        qe[tid] = t < 0 ? -INFINITY : (v == vmin ? 0.f : vmin - v);
+        qz[tid] = z;
+        qu[tid] = u;
+        const int U8 = (U + 7) >> 3;  // n-tiles of 8 tokens
+        const int Upad = 8 * U8;
+        __syncthreads();
+        // this lane's pairs
+        int lk[4];
+        float le[4], lz[4];
+        float2 lu[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = pq * 8 + pk0 + i;
+            lk[i] = qloc[e];
+            le[i] = qe[e];
+            lz[i] = qz[e];
+            lu[i] = qu[e];
+        }
+        float cq[4] = {0.f, 0.f, 0.f, 0.f};
+        const size_t ftok0 = static_cast<size_t>(b) * a.N;
+        const long long gq0 = static_cast<long long>(b) * a.Q + qt0;
+        // ---- head groups: the group's F rows and dO rows are staged once for the CTA
+        const int hg = max(1, min(min(kUTMaxGroup, NH), kUTFBytes / max(64 * Upad, 64)));
+        for (int h0 = 0; h0 < NH; h0 += hg) {
+            const int ng = min(hg, NH - h0);
+            {
+                // thread: 16-byte chunk c of a 64-byte head row; rows in steps of 32 (no division)
+                const int c = tid & 3;
+                for (int r = tid >> 2; r < Upad; r += kUTThreads / 4) {
+                    const bool ok = r < U;
+                    const bf16* src = a.feats + (ftok0 + (ok ? utok[r] : 0)) * a.d + h0 * 32 + c * 8;
+                    for (int j = 0; j < ng; ++j)
+                        cp_async16(fb0 + j * Upad * 64 + tile64_off(r, c), src + j * 32, ok);
+                }
+                if (tid < 64) {
+                    const int r = tid >> 2;
+                    const bool ok = r < nq;
+                    const bf16* src = a.dout + static_cast<size_t>(gq0 + (ok ? r : 0)) * a.d + h0 * 32 + c * 8;
+                    for (int j = 0; j < ng; ++j) cp_async16(db0 + j * 1024 + tile64_off(r, c), src + j * 32, ok);
+                }
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            __syncthreads();
+            // warp w takes the heads h = w (mod 4)
+            for (int j = ((warp - h0) % kUTWarps + kUTWarps) % kUTWarps; j < ng; j += kUTWarps) {
+                const int h = h0 + j;
+                // dW_h = dO_h F_U,h^T into the warp's dW tile
+                uint32_t af[2][4];
+#pragma unroll
+                for (int s = 0; s < 2; ++s)
+                    ldsm_x4(db0 + j * 1024 + tile64_off(lane & 15, 2 * s + (lane >> 4)), af[s][0], af[s][1],
+                            af[s][2], af[s][3]);
+                const int g = lane >> 2, tq = lane & 3;
+                for (int nt = 0; nt < U8; ++nt) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(fb0 + j * Upad * 64 + tile64_off(nt * 8 + (lane & 7), lane >> 3), b0, b1, b2, b3);
+                    float c[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_bf16(c, af[0][0], af[0][1], af[0][2], af[0][3], b0, b1);
+                    mma_bf16(c, af[1][0], af[1][1], af[1][2], af[1][3], b2, b3);
+                    *reinterpret_cast<__half2*>(dws + g * kUTDS + nt * 8 + 2 * tq) = __floats2half2_rn(c[0], c[1]);
+                    *reinterpret_cast<__half2*>(dws + (g + 8) * kUTDS + nt * 8 + 2 * tq) = __floats2half2_rn(c[2], c[3]);
+                }
+                __syncwarp();
+                // the per-query algebra of this head for the lane's four pairs
+                const float ph = __ldg(a.p + h);
+                float w[4], dw[4];
+                float sum = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float y;
+                    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(ph * le[i]));
+                    w[i] = lk[i] < 0 ? 0.f : (ph == 0.f ? 1.f : y);
+                    dw[i] = lk[i] < 0 ? 0.f : __half2float(dws[pq * kUTDS + lk[i]]);
+                    sum += w[i];
+                }
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                const float inv = sum > 0.f ? __fdividef(1.f, sum) : 0.f;
+                float sdw = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    w[i] *= inv;
+                    sdw += w[i] * dw[i];
+                }
+                sdw += __shfl_xor_sync(0xffffffffu, sdw, 1);
+                float dph = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float ds = w[i] * (dw[i] - sdw);
+                    dph -= w[i] > 0.f ? ds * lz[i] : 0.f;
+                    cq[i] -= ph * ds;
+                }
+                const int slot = (h - warp) >> 2;  // h = warp + 4 slot
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    if (s == slot) dpa[s] += dph;
+                if (pq < nq) {
+                    float* wout = a.w + (static_cast<size_t>(gq0 + pq) * K + pk0) * NH + h;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (pk0 + i < K) wout[i * NH] = w[i];
+                }
+                __syncwarp();
+            }
+            __syncthreads();  // the group's buffers are reused
+        }
+        // dq: the lane's pairs, its partner lane, then the warps in order
+        float dqx = 0.f, dqy = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            dqx += cq[i] * lu[i].x;
+            dqy += cq[i] * lu[i].y;
+        }
+        dqx += __shfl_xor_sync(0xffffffffu, dqx, 1);
+        dqy += __shfl_xor_sync(0xffffffffu, dqy, 1);
+        if ((lane & 1) == 0) dqred[warp * 16 + pq] = make_float2(dqx, dqy);
+        __syncthreads();
+        if (tid < nq) {
+            float2 s = dqred[tid];
+#pragma unroll
+            for (int w2 = 1; w2 < kUTWarps; ++w2) {
+                s.x += dqred[w2 * 16 + tid].x;
+                s.y += dqred[w2 * 16 + tid].y;
+            }
+            reinterpret_cast<float2*>(a.dq)[gq0 + tid] = s;
+        }
+        __syncthreads();  // bits, lists and dq partials are rebuilt by the next tile
+    }
+    // dp: the lane partials of each of this warp's heads, summed over the warp in a fixed order
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        const int h = warp + 4 * s;
+        float x = dpa[s];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0 && h < NH) a.dp_part[static_cast<size_t>(blockIdx.x) * NH + h] = x;
+    }
+}
+
 // Stable counting sort of an image's (query, slot) entries by token id, integer only,
 // spread over `slices` CTAs per image: CTA (slice, b) owns the tokens [t_lo, t_hi).
 //   compaction: warp w scans the contiguous entry chunk [lo_w, hi_w) of the image twice
@@ -1522,7 +1797,25 @@ cudaError_t launch_knn_bwd_indexed(const KnnArgs& a, cudaStream_t st) {
     const unsigned qblocks = static_cast<unsigned>(ws.query_blocks);
     const GatherPlan g = gather_plan(a.B, a.Q, a.d, a.K, true);
     cudaError_t e = cudaSuccess;
-    if (qblocks > 0) {
+    int qb_used = static_cast<int>(qblocks);
+    if (qblocks > 0 && a.N <= kUTUseN && a.K <= 8) {
+        // tensor-core query pass over 16-query tiles (grid within the workspace's dp rows)
+        const size_t usmem = ut_smem_layout().total;
+        e = ensure_smem<knn_bwd_query_union_kernel>(usmem);
+        if (e != cudaSuccess) return e;
+        const long long tpi = (a.Q + 15) / 16;
+        const long long tiles = static_cast<long long>(a.B) * tpi;
+        long long grid = static_cast<long long>(sm_count()) * resident<knn_bwd_query_union_kernel>(kUTThreads, usmem);
+        if (grid > static_cast<long long>(qblocks)) grid = qblocks;
+        if (grid > tiles) grid = tiles;
+        const long long span = (tiles + grid - 1) / grid;
+        grid = (tiles + span - 1) / span;
+        qb_used = static_cast<int>(grid);
+        knn_bwd_query_union_kernel<<<static_cast<unsigned>(grid), kUTThreads, usmem, st>>>(a, tpi, span);
+        note_launch();
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    } else if (qblocks > 0) {
         const size_t smem = sizeof(float) * kGatherWarps * (32 >> l2) * NH;
         if (g.shared)
             e = (a.K <= 8) ? bwdq_shared_k<8>(a, st, g, smem) : bwdq_shared_k<16>(a, st, g, smem);
@@ -1533,7 +1826,7 @@ cudaError_t launch_knn_bwd_indexed(const KnnArgs& a, cudaStream_t st) {
     }
     const int slices = csr_slices(a.B, a.N);
     const int chunks = knn_chunks(a.Q, a.K, a.N);
-    const int qb = static_cast<int>(qblocks);
+    const int qb = qb_used;
     const long long warps = static_cast<long long>(a.B) * chunks;
     const int hctas = heavy_ctas(a.Q, a.K, a.N);
     const unsigned tblocks = static_cast<unsigned>(hctas + (warps + kGatherWarps - 1) / kGatherWarps);

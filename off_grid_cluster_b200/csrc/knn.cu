@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kTableThreads, KMAX <= 8 ? 2 : 1)
     knn_table_kernel(const float* __restrict__ xy, int N, int GH, int GW, int K, BinGrid bg,
                      int32_t* __restrict__ table) {
     static_assert(kTableSub == 4, "the merge below takes two levels");
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const int b = blockIdx.y, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int nbins = bg.nbx * bg.nby;
@@ -1102,6 +1102,237 @@ __global__ void __launch_bounds__(kUTThreads)
     }
 }
 
+// Forward on the tensor cores, for the images the union query pass serves (at most kUTUseN
+// tokens, K <= 8), over the same 16-query tiles and token unions.  Per head:
+//   out (16 x 32) = W_h (16 x U) F_U,h (U x 32),
+// W_h holding each query's normalised weights at the union positions of its tokens (slots
+// that repeat a token add up in slot order), split into bf16 hi + lo (about 16 significant
+// bits) and read by ldmatrix from a per-warp tile; m16n8k16 products accumulate in fp32.
+// F_U,h never passes through shared memory: lane (g, c) loads 16 bytes, channels 8c .. 8c + 7,
+// of union rows 16 s + g and 16 s + 8 + g, and movmatrix turns pair e of those registers
+// into the B operand of column tile e, whose column n holds channel 8 (n / 2) + 2 e + n % 2.
+// The accumulator of tile e then holds channels 8c + 2e, 8c + 2e + 1 of queries g and g + 8,
+// so each lane stores 16 contiguous bytes per query.  Warp w takes heads w, w + 4, ...
+constexpr int kUFDS = kUTMaxU + 8;  // row stride of a warp's W tiles (bf16; 272-byte rows)
+constexpr int kUFBatch = 2;         // k-steps (16 union rows each) whose rows load together
+
+struct UFSmem {
+    size_t bits, pre, utok, qloc, qe, wt, total;
+};
+__host__ __device__ __forceinline__ UFSmem uf_smem_layout() {
+    UFSmem L;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = (o + bytes + 127) & ~size_t(127);
+        return at;
+    };
+    L.bits = take(4 * (kUTMaxN / 32));
+    L.pre = take(4 * (kUTMaxN / 32 + 1));
+    L.utok = take(4 * kUTMaxU);
+    L.qloc = take(4 * kUTMaxU);
+    L.qe = take(4 * kUTMaxU);
+    L.wt = take(2 * 2 * 16 * kUFDS * kUTWarps);  // hi and lo tiles per warp
+    L.total = o;
+    return L;
+}
+
+__global__ void __launch_bounds__(kUTThreads, 5)
+    knn_fwd_union_kernel(const KnnArgs a, long long tiles_per_image, long long tile_span) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const UFSmem L = uf_smem_layout();
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L.bits);
+    int* pre = reinterpret_cast<int*>(smem + L.pre);
+    int* utok = reinterpret_cast<int*>(smem + L.utok);
+    int* qloc = reinterpret_cast<int*>(smem + L.qloc);
+    float* qe = reinterpret_cast<float*>(smem + L.qe);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    bf16* wh = reinterpret_cast<bf16*>(smem + L.wt) + warp * 2 * 16 * kUFDS;
+    bf16* wl = wh + 16 * kUFDS;
+    const uint32_t wh0 = smem_addr(wh), wl0 = smem_addr(wl);
+    const int NH = a.d >> 5, NW = (a.N + 31) >> 5;
+    const int K = a.K;
+    const int pq = lane >> 1, pk0 = 4 * (lane & 1);  // the lane's four (query, slot) pairs
+    const int g = lane >> 2, tq = lane & 3;
+    const uint32_t aoff = ((lane & 7) + ((lane >> 3) & 1) * 8) * (2 * kUFDS) + (lane >> 4) * 16;
+    const long long total_tiles = static_cast<long long>(a.B) * tiles_per_image;
+    const long long t0 = static_cast<long long>(blockIdx.x) * tile_span;
+    const long long t1 = t0 + tile_span < total_tiles ? t0 + tile_span : total_tiles;
+    for (long long tile = t0; tile < t1; ++tile) {
+        const int b = static_cast<int>(tile / tiles_per_image);
+        const int qt0 = static_cast<int>(tile - static_cast<long long>(b) * tiles_per_image) * 16;
+        const int nq = min(16, a.Q - qt0);
+        // ---- the tile's entries: thread (q, k) = (tid / 8, tid % 8)
+        const int eq = tid >> 3, ek = tid & 7;
+        const long long gq_e = static_cast<long long>(b) * a.Q + qt0 + eq;
+        int t = -1;
+        float v = INFINITY;
+        if (eq < nq && ek < K) {
+            const float2 qp = __ldg(reinterpret_cast<const float2*>(a.queries) + gq_e);
+            const int cy = quantise(qp.y, a.GH), cx = quantise(qp.x, a.GW);
+            t = __ldg(a.table + ((static_cast<size_t>(b) * a.GH + cy) * a.GW + cx) * K + ek);
+            ACL_DEVICE_CHECK(t >= -1 && t < a.N);
+            if (t >= a.N) t = -1;
+            if (t >= 0) {
+                const float2 p = __ldg(reinterpret_cast<const float2*>(a.xy) + static_cast<size_t>(b) * a.N + t);
+                const float dx = qp.x - p.x, dy = qp.y - p.y;
+                v = knn_v(sqrtf(dx * dx + dy * dy), a.kind);
+            }
+        }
+        float vmin = v;
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, 1));
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, 2));
+        vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, 4));
+        for (int i = tid; i < NW; i += kUTThreads) bits[i] = 0u;
+        __syncthreads();
+        if (t >= 0) atomicOr(&bits[t >> 5], 1u << (t & 31));
+        __syncthreads();
+        if (warp == 0) {
+            const int c0 = lane < NW ? __popc(bits[lane]) : 0;
+            const int c1 = lane + 32 < NW ? __popc(bits[lane + 32]) : 0;
+            int s0 = c0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, s0, o);
+                if (lane >= o) s0 += y;
+            }
+            const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+            int s1 = c1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, s1, o);
+                if (lane >= o) s1 += y;
+            }
+            if (lane < NW) pre[lane] = s0 - c0;
+            if (lane + 32 < NW) pre[lane + 32] = tot0 + s1 - c1;
+            if (lane == 31) pre[64] = tot0 + s1;
+        }
+        __syncthreads();
+        const int U = pre[64];
+        const int loc = t >= 0 ? pre[t >> 5] + __popc(bits[t >> 5] & ((1u << (t & 31)) - 1u)) : -1;
+        if (t >= 0) utok[loc] = t;  // entries of one token write the same value
+        qloc[tid] = loc;
+        qe[tid] = t < 0 ? -INFINITY : (v == vmin ? 0.f : vmin - v);
+        const int nks = (U + 15) >> 4;  // k-steps of 16 union rows
+        __syncthreads();
+        int lk[4];
+        float le[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            lk[i] = qloc[pq * 8 + pk0 + i];
+            le[i] = qe[pq * 8 + pk0 + i];
+        }
+        // the partner lane's slots (the query's other four) and, per own slot, whether it is the
+        // first slot of its token in the query's row: that slot writes the token's summed weight
+        int ok[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ok[i] = __shfl_xor_sync(0xffffffffu, lk[i], 1);
+        bool first[4];
+        bool dup = false;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            bool f = lk[i] >= 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (j < i && lk[j] == lk[i]) f = false;
+                if ((lane & 1) && ok[j] == lk[i]) f = false;  // slots 0..3 come first
+                if (lk[i] >= 0 && ((j != i && lk[j] == lk[i]) || ok[j] == lk[i])) dup = true;
+            }
+            first[i] = f;
+        }
+        dup = __any_sync(0xffffffffu, dup);
+        // the warp's W tiles start at zero; every head of the tile writes the same positions,
+        // so one clearing per tile suffices
+        {
+            bf16* zt = ((lane >> 4) ? wl : wh) + (lane & 15) * kUFDS;
+            for (int c = 0; c < 2 * nks; ++c) *reinterpret_cast<uint4*>(zt + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+        const bf16* fimg = a.feats + static_cast<size_t>(b) * a.N * a.d + 8 * tq;
+        bf16* oq = a.out + (static_cast<size_t>(b) * a.Q + qt0 + g) * a.d + 8 * tq;
+        for (int h = warp; h < NH; h += kUTWarps) {
+            const float ph = __ldg(a.p + h);
+            float w[4];
+            float sum = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float y;
+                asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(ph * le[i]));
+                w[i] = lk[i] < 0 ? 0.f : (ph == 0.f ? 1.f : y);
+                sum += w[i];
+            }
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            const float inv = sum > 0.f ? __fdividef(1.f, sum) : 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] *= inv;
+            float x[4] = {w[0], w[1], w[2], w[3]};
+            if (dup) {  // warp-uniform: some query repeats a token
+                float pw[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) pw[i] = __shfl_xor_sync(0xffffffffu, w[i], 1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float s = 0.f;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const bool mine = (lane & 1) ? (q >= 4) : (q < 4);
+                        const int lq = mine ? lk[q & 3] : ok[q & 3];
+                        if (lq == lk[i]) s += mine ? w[q & 3] : pw[q & 3];
+                    }
+                    x[i] = s;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (!first[i]) continue;
+                const bf16 hi = __float2bfloat16_rn(x[i]);
+                wh[pq * kUFDS + lk[i]] = hi;
+                wl[pq * kUFDS + lk[i]] = __float2bfloat16_rn(x[i] - __bfloat162float(hi));
+            }
+            __syncwarp();
+            float acc[4][4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[e][0] = acc[e][1] = acc[e][2] = acc[e][3] = 0.f;
+            const bf16* fh = fimg + h * 32;
+            for (int s0 = 0; s0 < nks; s0 += kUFBatch) {
+                uint4 f0[kUFBatch], f1[kUFBatch];
+#pragma unroll
+                for (int s = 0; s < kUFBatch; ++s) {
+                    // rows past the union repeat its last row: their W columns are zero
+                    const int r0 = min(16 * (s0 + s) + g, U - 1), r1 = min(16 * (s0 + s) + 8 + g, U - 1);
+                    f0[s] = ldg16(fh + static_cast<size_t>(utok[r0]) * a.d);
+                    f1[s] = ldg16(fh + static_cast<size_t>(utok[r1]) * a.d);
+                }
+#pragma unroll
+                for (int s = 0; s < kUFBatch; ++s) {
+                    if (s0 + s >= nks) break;
+                    uint32_t ah[4], al[4];
+                    ldsm_x4(wh0 + aoff + (s0 + s) * 32, ah[0], ah[1], ah[2], ah[3]);
+                    ldsm_x4(wl0 + aoff + (s0 + s) * 32, al[0], al[1], al[2], al[3]);
+                    const uint32_t p0[4] = {f0[s].x, f0[s].y, f0[s].z, f0[s].w};
+                    const uint32_t p1[4] = {f1[s].x, f1[s].y, f1[s].z, f1[s].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t b0 = movm_t(p0[e]), b1 = movm_t(p1[e]);
+                        mma_bf16(acc[e], ah[0], ah[1], ah[2], ah[3], b0, b1);
+                        mma_bf16(acc[e], al[0], al[1], al[2], al[3], b0, b1);
+                    }
+                }
+            }
+            if (g < nq)
+                *reinterpret_cast<uint4*>(oq + h * 32) =
+                    make_uint4(pack_bf16(acc[0][0], acc[0][1]), pack_bf16(acc[1][0], acc[1][1]),
+                               pack_bf16(acc[2][0], acc[2][1]), pack_bf16(acc[3][0], acc[3][1]));
+            if (g + 8 < nq)
+                *reinterpret_cast<uint4*>(oq + static_cast<size_t>(8) * a.d + h * 32) =
+                    make_uint4(pack_bf16(acc[0][2], acc[0][3]), pack_bf16(acc[1][2], acc[1][3]),
+                               pack_bf16(acc[2][2], acc[2][3]), pack_bf16(acc[3][2], acc[3][3]));
+            __syncwarp();  // the next head rewrites the W tiles
+        }
+        __syncthreads();  // utok, qloc and qe are rebuilt by the next tile
+    }
+}
+
 // Stable counting sort of an image's (query, slot) entries by token id, integer only,
 // spread over `slices` CTAs per image: CTA (slice, b) owns the tokens [t_lo, t_hi).
 //   compaction: warp w scans the contiguous entry chunk [lo_w, hi_w) of the image twice
@@ -1167,7 +1398,7 @@ __global__ void __launch_bounds__(256) knn_keys_kernel(const KnnArgs a) {
 
 __global__ void __launch_bounds__(kCsrThreads)
     knn_csr_kernel(const KnnArgs a, int slices, int chunks) {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const int b = blockIdx.y, sl = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = a.N, K = a.K;
@@ -1767,6 +1998,21 @@ cudaError_t launch_knn_fwd(const KnnArgs& a, cudaStream_t st) {
     if (static_cast<long long>(a.B) * a.Q == 0) return cudaSuccess;
     const int l2 = lpq_log2_for(a.d);
     const int ch = (a.d + (8 << l2) - 1) / (8 << l2);
+    if (a.N <= kUTUseN && a.K <= 8) {
+        // tensor-core forward over 16-query tiles, one wave of resident CTAs
+        const size_t usmem = uf_smem_layout().total;
+        const cudaError_t e = ensure_smem<knn_fwd_union_kernel>(usmem);
+        if (e != cudaSuccess) return e;
+        const long long tpi = (a.Q + 15) / 16;
+        const long long tiles = static_cast<long long>(a.B) * tpi;
+        long long grid = static_cast<long long>(sm_count()) * resident<knn_fwd_union_kernel>(kUTThreads, usmem);
+        if (grid > tiles) grid = tiles;
+        const long long span = (tiles + grid - 1) / grid;
+        grid = (tiles + span - 1) / span;
+        knn_fwd_union_kernel<<<static_cast<unsigned>(grid), kUTThreads, usmem, st>>>(a, tpi, span);
+        note_launch();
+        return cudaGetLastError();
+    }
     const cudaError_t e = (a.K <= 8) ? fwd_k<8>(a, st, l2, ch) : fwd_k<16>(a, st, l2, ch);
     note_launch();
     return e;

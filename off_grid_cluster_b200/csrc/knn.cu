@@ -30,7 +30,6 @@
 #include <float.h>
 #include <math.h>
 
-#include <cuda_fp16.h>
 
 #include "internal.h"
 
@@ -363,15 +362,6 @@ __device__ __forceinline__ float load_neighbours(const KnnArgs& a, long long gq,
     return dmin;
 }
 
-__device__ __forceinline__ void fma8(float (&acc)[8], float w, uint4 f) {
-    const uint32_t u[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        acc[2 * i] += w * bf16_lo(u[i]);
-        acc[2 * i + 1] += w * bf16_hi(u[i]);
-    }
-}
-
 __device__ __forceinline__ uint4 pack8(const float (&v)[8], float s) {
     uint4 o;
     o.x = pack_bf16(v[0] * s, v[1] * s);
@@ -405,6 +395,14 @@ __device__ __forceinline__ void row_fma(uint64_t (&acc)[4], uint64_t ww, uint4 f
         "fma.rn.f32x2 %2, %4, p2, %2;\n\tfma.rn.f32x2 %3, %4, p3, %3;\n\t}"
         : "+l"(acc[0]), "+l"(acc[1]), "+l"(acc[2]), "+l"(acc[3])
         : "l"(ww), "r"(f.x), "r"(f.y), "r"(f.z), "r"(f.w));
+}
+__device__ __forceinline__ void unpack_acc(const uint64_t (&acc)[4], float (&v)[8]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = f2_unpack(acc[i]);
+        v[2 * i] = x.x;
+        v[2 * i + 1] = x.y;
+    }
 }
 
 // Neighbour j of a query: token id (-1 for an empty slot or an id >= N) and weight
@@ -832,12 +830,12 @@ __global__ void __launch_bounds__(kGatherThreads, (KT <= 8 && CH == 1) ? 4 : 2)
 // Query side of the backward on the tensor cores, for images of at most kUTMaxN tokens and
 // K <= 8: a CTA takes tiles of 16 consecutive queries of one image.  The tile's (query, slot)
 // entries name at most 128 tokens; their union U (ascending token id, found with a bitmap of
-// the image's tokens and prefix popcounts) is staged once for the tile, so one row of F serves
+// the image's tokens and prefix popcounts) is the tile's set of F rows, so one row of F serves
 // every query of the tile that lists it.  Per head, dW (16 x U) = dO_h (16 x 32) F_U,h^T is
-// one row of m16n8k16 bf16 products (fp32 accumulation; both operands exact in bf16), written
-// to the warp's shared dW tile in fp16 (2^-11 relative, far inside the gradients' tolerance;
-// it halves the tile, so four CTAs fit an SM); each (query, slot) then reads its dw at its
-// token's union position and the rest is the per-query algebra of the FMA query pass: w = 2^(p e) / S,
+// one row of m16n8k16 bf16 products (fp32 accumulation; both operands exact in bf16) whose
+// operands are 16-byte loads of dO and F rows straight into the fragments, written to the
+// warp's shared dW tile in fp32; each (query, slot) then reads its dw at its token's union
+// position and the rest is the per-query algebra of the FMA query pass: w = 2^(p e) / S,
 // ds = w (dw - sum w dw), dp and dq partials, w stored as [q][slot][head].  Thread (q, k) of
 // the CTA's 128 builds the tile's entry (q, k); warp w takes heads w, w + 4, ...; dq adds the
 // warps' partials in warp order and dp leaves each warp in a fixed order: bit-reproducible.
@@ -848,13 +846,13 @@ constexpr int kUTUseN = 1024;             // images of at most this many tokens 
                                           // (at 2048 tokens the FMA pass measured faster)
 constexpr int kUTMaxU = 128;              // 16 queries x 8 slots
 constexpr int kUTDS = kUTMaxU + 4;        // row stride of a warp's dW tile (floats)
-constexpr int kUTFBytes = 16 * 1024;      // F rows of one head group
-constexpr int kUTMaxGroup = 8;            // heads staged together (dO: 1 KB each)
+constexpr int kUTBatch = 4;               // n-tiles (8 union rows each) whose rows load together
 
 struct UTSmem {
-    size_t bits, pre, utok, qloc, qe, qz, qu, dqred, dw, fbuf, dobuf, total;
+    size_t bits, pre, utok, qloc, qe, qz, qu, dqred, dw, wblk, total;
 };
-__host__ __device__ __forceinline__ UTSmem ut_smem_layout() {
+// wblk: the tile's w block, [query][slot][head] with rows of NH + 1 floats
+__host__ __device__ __forceinline__ UTSmem ut_smem_layout(int NH) {
     UTSmem L;
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -870,9 +868,8 @@ __host__ __device__ __forceinline__ UTSmem ut_smem_layout() {
     L.qz = take(4 * kUTMaxU);
     L.qu = take(8 * kUTMaxU);
     L.dqred = take(8 * kUTWarps * 16);
-    L.dw = take(2 * kUTWarps * 16 * kUTDS);
-    L.fbuf = take(kUTFBytes);
-    L.dobuf = take(1024 * kUTMaxGroup);
+    L.dw = take(4 * kUTWarps * 16 * kUTDS);
+    L.wblk = take(4 * 16 * 8 * (NH + 1));
     L.total = o;
     return L;
 }
@@ -880,7 +877,7 @@ __host__ __device__ __forceinline__ UTSmem ut_smem_layout() {
 __global__ void __launch_bounds__(kUTThreads)
     knn_bwd_query_union_kernel(const KnnArgs a, long long tiles_per_image, long long tile_span) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const UTSmem L = ut_smem_layout();
+    const UTSmem L = ut_smem_layout(a.d >> 5);
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L.bits);
     int* pre = reinterpret_cast<int*>(smem + L.pre);
     int* utok = reinterpret_cast<int*>(smem + L.utok);
@@ -889,22 +886,32 @@ __global__ void __launch_bounds__(kUTThreads)
     float* qz = reinterpret_cast<float*>(smem + L.qz);
     float2* qu = reinterpret_cast<float2*>(smem + L.qu);
     float2* dqred = reinterpret_cast<float2*>(smem + L.dqred);
-    const uint32_t fb0 = smem_addr(smem + L.fbuf), db0 = smem_addr(smem + L.dobuf);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    __half* dws = reinterpret_cast<__half*>(smem + L.dw) + warp * 16 * kUTDS;
+    float* dws = reinterpret_cast<float*>(smem + L.dw) + warp * 16 * kUTDS;
+    float* wblk = reinterpret_cast<float*>(smem + L.wblk);
     const int NH = a.d >> 5, NW = (a.N + 31) >> 5;
+    const int WS = NH + 1;  // row stride of the w block
+    // the w block copy: this thread's first float (row, column) and its step of kUTThreads floats
+    const int wr0 = tid / NH, wc0 = tid - (tid / NH) * NH;
+    const int wdr = kUTThreads / NH, wdc = kUTThreads - (kUTThreads / NH) * NH;
     const int K = a.K;
     // this lane's four (query, slot) pairs in the per-head algebra: q = lane / 2, k = 4 (lane & 1) + i
     const int pq = lane >> 1, pk0 = 4 * (lane & 1);
+    const int g = lane >> 2, tq = lane & 3;  // the mma fragments' row and column pair
     float dpa[8];  // dp partials of this warp's heads h = warp + 4 s (s < 8 covers NH <= 32)
 #pragma unroll
     for (int s = 0; s < 8; ++s) dpa[s] = 0.f;
     const long long total_tiles = static_cast<long long>(a.B) * tiles_per_image;
     const long long t0 = static_cast<long long>(blockIdx.x) * tile_span;
     const long long t1 = t0 + tile_span < total_tiles ? t0 + tile_span : total_tiles;
-    for (long long tile = t0; tile < t1; ++tile) {
-        const int b = static_cast<int>(tile / tiles_per_image);
-        const int qt0 = static_cast<int>(tile - static_cast<long long>(b) * tiles_per_image) * 16;
+    // image and first query of the tile, advanced without divisions
+    int b = static_cast<int>(t0 / tiles_per_image);
+    int qt0 = static_cast<int>(t0 - static_cast<long long>(b) * tiles_per_image) * 16;
+    for (long long tile = t0; tile < t1; ++tile, qt0 += 16) {
+        if (qt0 >= a.Q) {
+            qt0 = 0;
+            ++b;
+        }
         const int nq = min(16, a.Q - qt0);
         // ---- the tile's entries: thread (q, k) = (tid / 8, tid % 8)
         const int eq = tid >> 3, ek = tid & 7;
@@ -940,7 +947,6 @@ __global__ void __launch_bounds__(kUTThreads)
         // exclusive prefix of the words' popcounts (warp 0; NW <= 64)
         if (warp == 0) {
             const int c0 = lane < NW ? __popc(bits[lane]) : 0;
-            const int c1 = lane + 32 < NW ? __popc(bits[lane + 32]) : 0;
             int s0 = c0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -948,15 +954,20 @@ __global__ void __launch_bounds__(kUTThreads)
                 if (lane >= o) s0 += y;
             }
             const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
-            int s1 = c1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, s1, o);
-                if (lane >= o) s1 += y;
-            }
             if (lane < NW) pre[lane] = s0 - c0;
-            if (lane + 32 < NW) pre[lane + 32] = tot0 + s1 - c1;
-            if (lane == 31) pre[64] = tot0 + s1;
+            if (NW > 32) {
+                const int c1 = lane + 32 < NW ? __popc(bits[lane + 32]) : 0;
+                int s1 = c1;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, s1, o);
+                    if (lane >= o) s1 += y;
+                }
+                if (lane + 32 < NW) pre[lane + 32] = tot0 + s1 - c1;
+                if (lane == 31) pre[64] = tot0 + s1;
+            } else if (lane == 0) {
+                pre[64] = tot0;
+            }
         }
         __syncthreads();
         const int U = pre[64];
@@ -967,7 +978,6 @@ __global__ void __launch_bounds__(kUTThreads)
         qz[tid] = z;
         qu[tid] = u;
         const int U8 = (U + 7) >> 3;  // n-tiles of 8 tokens
-        const int Upad = 8 * U8;
         __syncthreads();
         // this lane's pairs
         int lk[4];
@@ -982,92 +992,77 @@ __global__ void __launch_bounds__(kUTThreads)
             lu[i] = qu[e];
         }
         float cq[4] = {0.f, 0.f, 0.f, 0.f};
-        const size_t ftok0 = static_cast<size_t>(b) * a.N;
+        // rows of the lane's fragments: dO rows g and g + 8 of the tile (the tail repeats the
+        // last query; those rows of dW are never read)
+        const bf16* fimg = a.feats + static_cast<size_t>(b) * a.N * a.d + 8 * tq;
+        const bf16* do0 = a.dout + (static_cast<size_t>(b) * a.Q + qt0 + min(g, nq - 1)) * a.d + 8 * tq;
+        const bf16* do1 = a.dout + (static_cast<size_t>(b) * a.Q + qt0 + min(g + 8, nq - 1)) * a.d + 8 * tq;
         const long long gq0 = static_cast<long long>(b) * a.Q + qt0;
-        // ---- head groups: the group's F rows and dO rows are staged once for the CTA
-        const int hg = max(1, min(min(kUTMaxGroup, NH), kUTFBytes / max(64 * Upad, 64)));
-        for (int h0 = 0; h0 < NH; h0 += hg) {
-            const int ng = min(hg, NH - h0);
+        // warp w takes the heads h = w (mod 4)
+        for (int h = warp; h < NH; h += kUTWarps) {
             {
-                // thread: 16-byte chunk c of a 64-byte head row; rows in steps of 32 (no division)
-                const int c = tid & 3;
-                for (int r = tid >> 2; r < Upad; r += kUTThreads / 4) {
-                    const bool ok = r < U;
-                    const bf16* src = a.feats + (ftok0 + (ok ? utok[r] : 0)) * a.d + h0 * 32 + c * 8;
-                    for (int j = 0; j < ng; ++j)
-                        cp_async16(fb0 + j * Upad * 64 + tile64_off(r, c), src + j * 32, ok);
-                }
-                if (tid < 64) {
-                    const int r = tid >> 2;
-                    const bool ok = r < nq;
-                    const bf16* src = a.dout + static_cast<size_t>(gq0 + (ok ? r : 0)) * a.d + h0 * 32 + c * 8;
-                    for (int j = 0; j < ng; ++j) cp_async16(db0 + j * 1024 + tile64_off(r, c), src + j * 32, ok);
+                // dW_h = dO_h F_U,h^T into the warp's dW tile.  Lane (g, c) holds channels
+                // 8c .. 8c + 7 of its rows as pairs e = 0..3; k-step s takes pairs 2s and 2s + 1
+                // as its two k-halves, for dO and F alike, so the sum over channels is unchanged.
+                const uint4 q0 = ldg16(do0 + h * 32), q1 = ldg16(do1 + h * 32);
+                const bf16* fh = fimg + h * 32;
+                for (int n0 = 0; n0 < U8; n0 += kUTBatch) {
+                    uint4 f[kUTBatch];
+#pragma unroll
+                    for (int x = 0; x < kUTBatch; ++x) {
+                        // rows past the union repeat its last row: those columns are never read
+                        const int r = min(8 * (n0 + x) + g, U - 1);
+                        f[x] = ldg16(fh + static_cast<size_t>(utok[r]) * a.d);
+                    }
+#pragma unroll
+                    for (int x = 0; x < kUTBatch; ++x) {
+                        const int nt = n0 + x;
+                        if (nt >= U8) break;
+                        float c[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_bf16(c, q0.x, q1.x, q0.y, q1.y, f[x].x, f[x].y);
+                        mma_bf16(c, q0.z, q1.z, q0.w, q1.w, f[x].z, f[x].w);
+                        *reinterpret_cast<float2*>(dws + g * kUTDS + nt * 8 + 2 * tq) = make_float2(c[0], c[1]);
+                        *reinterpret_cast<float2*>(dws + (g + 8) * kUTDS + nt * 8 + 2 * tq) = make_float2(c[2], c[3]);
+                    }
                 }
             }
-            cp_async_commit();
-            cp_async_wait<0>();
-            __syncthreads();
-            // warp w takes the heads h = w (mod 4)
-            for (int j = ((warp - h0) % kUTWarps + kUTWarps) % kUTWarps; j < ng; j += kUTWarps) {
-                const int h = h0 + j;
-                // dW_h = dO_h F_U,h^T into the warp's dW tile
-                uint32_t af[2][4];
+            __syncwarp();
+            // the per-query algebra of this head for the lane's four pairs
+            const float ph = __ldg(a.p + h);
+            float w[4], dw[4];
+            float sum = 0.f;
 #pragma unroll
-                for (int s = 0; s < 2; ++s)
-                    ldsm_x4(db0 + j * 1024 + tile64_off(lane & 15, 2 * s + (lane >> 4)), af[s][0], af[s][1],
-                            af[s][2], af[s][3]);
-                const int g = lane >> 2, tq = lane & 3;
-                for (int nt = 0; nt < U8; ++nt) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(fb0 + j * Upad * 64 + tile64_off(nt * 8 + (lane & 7), lane >> 3), b0, b1, b2, b3);
-                    float c[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_bf16(c, af[0][0], af[0][1], af[0][2], af[0][3], b0, b1);
-                    mma_bf16(c, af[1][0], af[1][1], af[1][2], af[1][3], b2, b3);
-                    *reinterpret_cast<__half2*>(dws + g * kUTDS + nt * 8 + 2 * tq) = __floats2half2_rn(c[0], c[1]);
-                    *reinterpret_cast<__half2*>(dws + (g + 8) * kUTDS + nt * 8 + 2 * tq) = __floats2half2_rn(c[2], c[3]);
-                }
-                __syncwarp();
-                // the per-query algebra of this head for the lane's four pairs
-                const float ph = __ldg(a.p + h);
-                float w[4], dw[4];
-                float sum = 0.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float y;
-                    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(ph * le[i]));
-                    w[i] = lk[i] < 0 ? 0.f : (ph == 0.f ? 1.f : y);
-                    dw[i] = lk[i] < 0 ? 0.f : __half2float(dws[pq * kUTDS + lk[i]]);
-                    sum += w[i];
-                }
-                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                const float inv = sum > 0.f ? __fdividef(1.f, sum) : 0.f;
-                float sdw = 0.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    w[i] *= inv;
-                    sdw += w[i] * dw[i];
-                }
-                sdw += __shfl_xor_sync(0xffffffffu, sdw, 1);
-                float dph = 0.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float ds = w[i] * (dw[i] - sdw);
-                    dph -= w[i] > 0.f ? ds * lz[i] : 0.f;
-                    cq[i] -= ph * ds;
-                }
-                const int slot = (h - warp) >> 2;  // h = warp + 4 slot
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    if (s == slot) dpa[s] += dph;
-                if (pq < nq) {
-                    float* wout = a.w + (static_cast<size_t>(gq0 + pq) * K + pk0) * NH + h;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (pk0 + i < K) wout[i * NH] = w[i];
-                }
-                __syncwarp();
+            for (int i = 0; i < 4; ++i) {
+                float y;
+                asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(ph * le[i]));
+                w[i] = lk[i] < 0 ? 0.f : (ph == 0.f ? 1.f : y);
+                dw[i] = lk[i] < 0 ? 0.f : dws[pq * kUTDS + lk[i]];
+                sum += w[i];
             }
-            __syncthreads();  // the group's buffers are reused
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            const float inv = sum > 0.f ? __fdividef(1.f, sum) : 0.f;
+            float sdw = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                w[i] *= inv;
+                sdw += w[i] * dw[i];
+            }
+            sdw += __shfl_xor_sync(0xffffffffu, sdw, 1);
+            float dph = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float ds = w[i] * (dw[i] - sdw);
+                dph -= w[i] > 0.f ? ds * lz[i] : 0.f;
+                cq[i] -= ph * ds;
+            }
+            const int slot = (h - warp) >> 2;  // h = warp + 4 slot
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                if (s == slot) dpa[s] += dph;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (pk0 + i < K) wblk[(pq * K + pk0 + i) * WS + h] = w[i];
+            __syncwarp();
         }
         // dq: the lane's pairs, its partner lane, then the warps in order
         float dqx = 0.f, dqy = 0.f;
@@ -1080,6 +1075,22 @@ __global__ void __launch_bounds__(kUTThreads)
         dqy += __shfl_xor_sync(0xffffffffu, dqy, 1);
         if ((lane & 1) == 0) dqred[warp * 16 + pq] = make_float2(dqx, dqy);
         __syncthreads();
+        // the tile's w block is contiguous in [q][slot][head]: float o of it sits at o + o / NH
+        // in the padded rows; o advances by the CTA's width, its row and column without divisions
+        {
+            float* wout = a.w + static_cast<size_t>(gq0) * K * NH;
+            const int n = nq * K * NH;
+            int r = wr0, c = wc0;
+            for (int o = tid; o < n; o += kUTThreads) {
+                wout[o] = wblk[o + r];
+                r += wdr;
+                c += wdc;
+                if (c >= NH) {
+                    c -= NH;
+                    ++r;
+                }
+            }
+        }
         if (tid < nq) {
             float2 s = dqred[tid];
 #pragma unroll
@@ -1158,9 +1169,14 @@ __global__ void __launch_bounds__(kUTThreads, 5)
     const long long total_tiles = static_cast<long long>(a.B) * tiles_per_image;
     const long long t0 = static_cast<long long>(blockIdx.x) * tile_span;
     const long long t1 = t0 + tile_span < total_tiles ? t0 + tile_span : total_tiles;
-    for (long long tile = t0; tile < t1; ++tile) {
-        const int b = static_cast<int>(tile / tiles_per_image);
-        const int qt0 = static_cast<int>(tile - static_cast<long long>(b) * tiles_per_image) * 16;
+    // image and first query of the tile, advanced without divisions
+    int b = static_cast<int>(t0 / tiles_per_image);
+    int qt0 = static_cast<int>(t0 - static_cast<long long>(b) * tiles_per_image) * 16;
+    for (long long tile = t0; tile < t1; ++tile, qt0 += 16) {
+        if (qt0 >= a.Q) {
+            qt0 = 0;
+            ++b;
+        }
         const int nq = min(16, a.Q - qt0);
         // ---- the tile's entries: thread (q, k) = (tid / 8, tid % 8)
         const int eq = tid >> 3, ek = tid & 7;
@@ -1183,13 +1199,23 @@ __global__ void __launch_bounds__(kUTThreads, 5)
         vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, 1));
         vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, 2));
         vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, 4));
+        // the entry is its token's first slot in the query's row unless an earlier slot holds
+        // the token; a repeated token anywhere in the tile sends every warp down the summing path
+        bool efirst = t >= 0, erep = false;
+#pragma unroll
+        for (int s = 1; s < 8; ++s) {
+            const int ts = __shfl_sync(0xffffffffu, t, (lane & ~7) | ((lane + s) & 7));
+            if (t >= 0 && ts == t) {
+                erep = true;
+                if (((lane + s) & 7) < ek) efirst = false;
+            }
+        }
         for (int i = tid; i < NW; i += kUTThreads) bits[i] = 0u;
         __syncthreads();
         if (t >= 0) atomicOr(&bits[t >> 5], 1u << (t & 31));
         __syncthreads();
-        if (warp == 0) {
+        if (warp == 0) {  // exclusive prefix of the bitmap words' counts (NW <= 64)
             const int c0 = lane < NW ? __popc(bits[lane]) : 0;
-            const int c1 = lane + 32 < NW ? __popc(bits[lane + 32]) : 0;
             int s0 = c0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -1197,50 +1223,40 @@ __global__ void __launch_bounds__(kUTThreads, 5)
                 if (lane >= o) s0 += y;
             }
             const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
-            int s1 = c1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, s1, o);
-                if (lane >= o) s1 += y;
-            }
             if (lane < NW) pre[lane] = s0 - c0;
-            if (lane + 32 < NW) pre[lane + 32] = tot0 + s1 - c1;
-            if (lane == 31) pre[64] = tot0 + s1;
+            if (NW > 32) {
+                const int c1 = lane + 32 < NW ? __popc(bits[lane + 32]) : 0;
+                int s1 = c1;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, s1, o);
+                    if (lane >= o) s1 += y;
+                }
+                if (lane + 32 < NW) pre[lane + 32] = tot0 + s1 - c1;
+                if (lane == 31) pre[64] = tot0 + s1;
+            } else if (lane == 0) {
+                pre[64] = tot0;
+            }
         }
         __syncthreads();
         const int U = pre[64];
         const int loc = t >= 0 ? pre[t >> 5] + __popc(bits[t >> 5] & ((1u << (t & 31)) - 1u)) : -1;
         if (t >= 0) utok[loc] = t;  // entries of one token write the same value
-        qloc[tid] = loc;
+        qloc[tid] = efirst ? loc : (t >= 0 ? loc | 0x40000000 : -1);  // bit 30: a later slot
         qe[tid] = t < 0 ? -INFINITY : (v == vmin ? 0.f : vmin - v);
         const int nks = (U + 15) >> 4;  // k-steps of 16 union rows
-        __syncthreads();
+        const bool dup = __syncthreads_or(erep) != 0;
+        // the lane's slots: union position, whether it writes the token's summed weight, exponent
         int lk[4];
+        bool first[4];
         float le[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            lk[i] = qloc[pq * 8 + pk0 + i];
+            const int r = qloc[pq * 8 + pk0 + i];
+            lk[i] = r < 0 ? -1 : (r & 0x3fffffff);
+            first[i] = r >= 0 && !(r & 0x40000000);
             le[i] = qe[pq * 8 + pk0 + i];
         }
-        // the partner lane's slots (the query's other four) and, per own slot, whether it is the
-        // first slot of its token in the query's row: that slot writes the token's summed weight
-        int ok[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) ok[i] = __shfl_xor_sync(0xffffffffu, lk[i], 1);
-        bool first[4];
-        bool dup = false;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            bool f = lk[i] >= 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (j < i && lk[j] == lk[i]) f = false;
-                if ((lane & 1) && ok[j] == lk[i]) f = false;  // slots 0..3 come first
-                if (lk[i] >= 0 && ((j != i && lk[j] == lk[i]) || ok[j] == lk[i])) dup = true;
-            }
-            first[i] = f;
-        }
-        dup = __any_sync(0xffffffffu, dup);
         // the warp's W tiles start at zero; every head of the tile writes the same positions,
         // so one clearing per tile suffices
         {
@@ -1266,10 +1282,14 @@ __global__ void __launch_bounds__(kUTThreads, 5)
 #pragma unroll
             for (int i = 0; i < 4; ++i) w[i] *= inv;
             float x[4] = {w[0], w[1], w[2], w[3]};
-            if (dup) {  // warp-uniform: some query repeats a token
+            if (dup) {  // CTA-uniform: some query of the tile repeats a token
                 float pw[4];
+                int ok[4];  // the partner lane's slots: the query's other four
 #pragma unroll
-                for (int i = 0; i < 4; ++i) pw[i] = __shfl_xor_sync(0xffffffffu, w[i], 1);
+                for (int i = 0; i < 4; ++i) {
+                    pw[i] = __shfl_xor_sync(0xffffffffu, w[i], 1);
+                    ok[i] = __shfl_xor_sync(0xffffffffu, lk[i], 1);
+                }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     float s = 0.f;
@@ -1612,7 +1632,7 @@ __global__ void __launch_bounds__(kCsrThreads)
 template <int CH>
 __device__ __forceinline__ void token_streams(const KnnArgs& a, int b, int lo, int hi, int sid,
                                              int nstreams, int sub, int LPQ, int ch,
-                                             float (&acc)[8]) {
+                                             uint64_t (&acc)[4]) {
     const int NH = a.d >> 5;
     const int KN = a.K * NH;
     const int c0 = ch * LPQ * 8 + sub * 8;
@@ -1623,7 +1643,7 @@ __device__ __forceinline__ void token_streams(const KnnArgs& a, int b, int lo, i
     const bf16* gb = a.dout + qbase * a.d + (on ? c0 : 0);
     const int32_t* csr = a.csr + static_cast<size_t>(b) * a.Q * a.K;
 #pragma unroll
-    for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+    for (int v = 0; v < 4; ++v) acc[v] = 0ull;
     // this stream's entries are lo + sid + nstreams * k; lanes of the group hold LPQ of them
     const int n = (hi - lo - sid + nstreams - 1) / nstreams;  // entries of this stream (>= 0)
     const unsigned gmask = (LPQ == 32) ? 0xffffffffu : (((1u << LPQ) - 1u) << (threadIdx.x & 31 & ~(LPQ - 1)));
@@ -1643,12 +1663,13 @@ __device__ __forceinline__ void token_streams(const KnnArgs& a, int b, int lo, i
                 gv[x] = on ? ldg16(gb + q * a.d) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
-            for (int x = 0; x < 4; ++x) fma8(acc, wv[x], gv[x]);
+            for (int x = 0; x < 4; ++x) row_fma(acc, f2_pack(wv[x], wv[x]), gv[x]);
         }
         for (; u < cnt; ++u) {
             const int e = __shfl_sync(gmask, mine, u, LPQ);
             const int q = e >> 4, j = e & 15;
-            fma8(acc, __ldg(wb + q * KN + j * NH), on ? ldg16(gb + q * a.d) : make_uint4(0u, 0u, 0u, 0u));
+            const float wv = __ldg(wb + q * KN + j * NH);
+            row_fma(acc, f2_pack(wv, wv), on ? ldg16(gb + q * a.d) : make_uint4(0u, 0u, 0u, 0u));
         }
     }
 }
@@ -1662,8 +1683,10 @@ __device__ void heavy_token(const KnnArgs& a, int b, int t, int l2, float (*part
     const int32_t* coff = a.csr_off + static_cast<size_t>(b) * (a.N + 1);
     const int lo = coff[t], hi = coff[t + 1];
     for (int ch = 0; ch < CH; ++ch) {
+        uint64_t acc2[4];
+        token_streams<1>(a, b, lo, hi, warp * S + grp, kGatherWarps * S, sub, LPQ, ch, acc2);
         float acc[8];
-        token_streams<1>(a, b, lo, hi, warp * S + grp, kGatherWarps * S, sub, LPQ, ch, acc);
+        unpack_acc(acc2, acc);
         for (int o = LPQ; o < 32; o <<= 1) {
 #pragma unroll
             for (int v = 0; v < 8; ++v) acc[v] += __shfl_xor_sync(0xffffffffu, acc[v], o);
@@ -1794,9 +1817,7 @@ __global__ void __launch_bounds__(kGatherThreads, 4)
             int lo = __shfl_sync(0xffffffffu, offv, 0);
             for (int k = 0; k < nl; ++k) {
                 const int hi = __shfl_sync(0xffffffffu, offv, k + 1);
-                float acc[8];
-#pragma unroll
-                for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+                uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
                 for (int i0 = lo; i0 < hi; i0 += STEPS * EPS) {
                     float w[STEPS];
                     uint4 g[STEPS];
@@ -1813,8 +1834,10 @@ __global__ void __launch_bounds__(kGatherThreads, 4)
                         }
                     }
 #pragma unroll
-                    for (int x = 0; x < STEPS; ++x) fma8(acc, w[x], g[x]);
+                    for (int x = 0; x < STEPS; ++x) row_fma(acc2, f2_pack(w[x], w[x]), g[x]);
                 }
+                float acc[8];
+                unpack_acc(acc2, acc);
                 for (int o = LPQ; o < 32; o <<= 1) {
 #pragma unroll
                     for (int v = 0; v < 8; ++v) acc[v] += __shfl_xor_sync(0xffffffffu, acc[v], o);
@@ -2046,7 +2069,7 @@ cudaError_t launch_knn_bwd_indexed(const KnnArgs& a, cudaStream_t st) {
     int qb_used = static_cast<int>(qblocks);
     if (qblocks > 0 && a.N <= kUTUseN && a.K <= 8) {
         // tensor-core query pass over 16-query tiles (grid within the workspace's dp rows)
-        const size_t usmem = ut_smem_layout().total;
+        const size_t usmem = ut_smem_layout(a.d >> 5).total;
         e = ensure_smem<knn_bwd_query_union_kernel>(usmem);
         if (e != cudaSuccess) return e;
         const long long tpi = (a.Q + 15) / 16;

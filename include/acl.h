@@ -314,6 +314,10 @@ size_t acl_knn_gather_workspace(int B, int Q, int N, int d, int K);
  * out [B][Q][d] bf16 out.
  * Limits: d % 32 == 0, 32 <= d <= ACL_MAX_GATHER_D, 1 <= K <= ACL_MAX_KNN_K,
  *         table entries in [-1, N).
+ * Non-finite features: for N <= 1024 and K <= 8 the sum runs as a tensor-core product
+ * over tiles of 16 consecutive queries, which multiplies every token listed by the tile
+ * by every query's weight (zeros included); a feature row holding Inf or NaN then makes
+ * the outputs of all 16 queries of such a tile non-finite.  Finite inputs are unaffected.
  */
 acl_status acl_knn_gather_fwd(const float* queries, int B, int Q, const acl_bf16* feats,
                               const float* coords, int N, int d, const int32_t* table,

@@ -1000,21 +1000,38 @@ __global__ void __launch_bounds__(kUTThreads)
         const bf16* do0 = a.dout + (static_cast<size_t>(b) * a.Q + qt0 + min(g, nq - 1)) * a.d + 8 * tq;
         const bf16* do1 = a.dout + (static_cast<size_t>(b) * a.Q + qt0 + min(g + 8, nq - 1)) * a.d + 8 * tq;
         const long long gq0 = static_cast<long long>(b) * a.Q + qt0;
+        // the fragments of a head: its dO rows and the first kUTBatch n-tiles of union rows
+        // (rows past the union repeat its last row: those columns are never read); the next
+        // head's are loaded while this one computes
+        uint4 nq0 = make_uint4(0u, 0u, 0u, 0u), nq1 = nq0, nf[kUTBatch];
+        auto fetch = [&](int hh) {
+            nq0 = ldg16(do0 + hh * 32);
+            nq1 = ldg16(do1 + hh * 32);
+#pragma unroll
+            for (int x = 0; x < kUTBatch; ++x)
+                nf[x] = U8 > 0 ? ldg16(fimg + hh * 32 + static_cast<size_t>(utok[min(8 * x + g, U - 1)]) * a.d)
+                               : make_uint4(0u, 0u, 0u, 0u);
+        };
+        if (warp < NH) fetch(warp);
         // warp w takes the heads h = w (mod 4)
         for (int h = warp; h < NH; h += kUTWarps) {
             {
                 // dW_h = dO_h F_U,h^T into the warp's dW tile.  Lane (g, c) holds channels
                 // 8c .. 8c + 7 of its rows as pairs e = 0..3; k-step s takes pairs 2s and 2s + 1
                 // as its two k-halves, for dO and F alike, so the sum over channels is unchanged.
-                const uint4 q0 = ldg16(do0 + h * 32), q1 = ldg16(do1 + h * 32);
+                const uint4 q0 = nq0, q1 = nq1;
+                uint4 f[kUTBatch];
+#pragma unroll
+                for (int x = 0; x < kUTBatch; ++x) f[x] = nf[x];
+                if (h + kUTWarps < NH) fetch(h + kUTWarps);
                 const bf16* fh = fimg + h * 32;
                 for (int n0 = 0; n0 < U8; n0 += kUTBatch) {
-                    uint4 f[kUTBatch];
+                    if (n0 > 0) {
 #pragma unroll
-                    for (int x = 0; x < kUTBatch; ++x) {
-                        // rows past the union repeat its last row: those columns are never read
-                        const int r = min(8 * (n0 + x) + g, U - 1);
-                        f[x] = ldg16(fh + static_cast<size_t>(utok[r]) * a.d);
+                        for (int x = 0; x < kUTBatch; ++x) {
+                            const int r = min(8 * (n0 + x) + g, U - 1);
+                            f[x] = ldg16(fh + static_cast<size_t>(utok[r]) * a.d);
+                        }
                     }
 #pragma unroll
                     for (int x = 0; x < kUTBatch; ++x) {
@@ -1269,6 +1286,18 @@ __global__ void __launch_bounds__(kUTThreads, 5)
         const bf16* fimg = a.feats + static_cast<size_t>(b) * a.N * a.d + 8 * tq;
         bf16* oq = a.out + (static_cast<size_t>(b) * a.Q + qt0 + g) * a.d + 8 * tq;
         for (int h = warp; h < NH; h += kUTWarps) {
+            const bf16* fh = fimg + h * 32;
+            // the first k-steps' rows load while the weights form (rows past the union repeat
+            // its last row: their W columns are zero)
+            uint4 f0[kUFBatch], f1[kUFBatch];
+            if (nks > 0) {
+#pragma unroll
+                for (int s = 0; s < kUFBatch; ++s) {
+                    const int r0 = min(16 * s + g, U - 1), r1 = min(16 * s + 8 + g, U - 1);
+                    f0[s] = ldg16(fh + static_cast<size_t>(utok[r0]) * a.d);
+                    f1[s] = ldg16(fh + static_cast<size_t>(utok[r1]) * a.d);
+                }
+            }
             const float ph = __ldg(a.p + h);
             float w[4];
             float sum = 0.f;
@@ -1315,15 +1344,14 @@ __global__ void __launch_bounds__(kUTThreads, 5)
             float acc[4][4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[e][0] = acc[e][1] = acc[e][2] = acc[e][3] = 0.f;
-            const bf16* fh = fimg + h * 32;
             for (int s0 = 0; s0 < nks; s0 += kUFBatch) {
-                uint4 f0[kUFBatch], f1[kUFBatch];
+                if (s0 > 0) {
 #pragma unroll
-                for (int s = 0; s < kUFBatch; ++s) {
-                    // rows past the union repeat its last row: their W columns are zero
-                    const int r0 = min(16 * (s0 + s) + g, U - 1), r1 = min(16 * (s0 + s) + 8 + g, U - 1);
-                    f0[s] = ldg16(fh + static_cast<size_t>(utok[r0]) * a.d);
-                    f1[s] = ldg16(fh + static_cast<size_t>(utok[r1]) * a.d);
+                    for (int s = 0; s < kUFBatch; ++s) {
+                        const int r0 = min(16 * (s0 + s) + g, U - 1), r1 = min(16 * (s0 + s) + 8 + g, U - 1);
+                        f0[s] = ldg16(fh + static_cast<size_t>(utok[r0]) * a.d);
+                        f1[s] = ldg16(fh + static_cast<size_t>(utok[r1]) * a.d);
+                    }
                 }
 #pragma unroll
                 for (int s = 0; s < kUFBatch; ++s) {

@@ -145,6 +145,33 @@ def test_repeated_ids_beyond_16_bit_counts():
     check_grad(host(dp), dp_r, "dp")
 
 
+@pytest.mark.parametrize("N,Q,K", [(1024, 1001, 8), (1025, 1001, 8), (700, 37, 5), (64, 145, 1)])
+def test_gather_union_tiles_ragged_and_scattered(N, Q, K):
+    """Images of at most 1024 tokens take the tensor-core union kernels, over tiles of 16
+    consecutive queries: ragged last tiles (Q % 16 != 0), queries in random order so that a
+    tile lists up to 16 x K distinct tokens, the 1024-token boundary (1025 takes the FMA
+    kernels), K < 8, both weight kernels, p = 0, and a bit-identical repeated backward."""
+    rng = np.random.default_rng(7 * N + Q)
+    B, d = 2, 96
+    xy = rng.uniform(0, 64, (B, N, 2)).astype(np.float32)
+    queries = rng.uniform(-1, 65, (B, Q, 2)).astype(np.float32)
+    feats = synth.round_bf16(rng.standard_normal((B, N, d)).astype(np.float32))
+    dout = synth.round_bf16(rng.standard_normal((B, Q, d)).astype(np.float32))
+    p = rng.uniform(0.5, 4.0, d // 32).astype(np.float32)
+    kb = synth.KnnBatch(queries, xy, feats, dout, p, 64, 64, K)
+    gather_both(kb)
+    gather_both(kb, kind=acl.ACL_KNN_INVPOW)
+    kb.p = np.zeros_like(kb.p)                               # plain mean
+    gather_both(kb)
+    kb.p = p
+    table = acl.acl_knn_table(dev(xy), 64, 64, K)
+    args = (dev(queries), bf16(feats), dev(xy), table, dev(p), bf16(dout))
+    r1 = acl.acl_knn_gather_bwd(*args)
+    r2 = acl.acl_knn_gather_bwd(*args)
+    for x, y in zip(r1, r2):
+        assert torch.equal(x, y)
+
+
 def test_staged_backward_matches_one_call():
     """Index built on a side stream, then the indexed backward: bit-identical results."""
     sb = synth.step_batch(B=2)

@@ -239,8 +239,8 @@ __device__ void bitonic_2lists(uint64_t* keys, int P) {
 }
 
 // Fallback sort for inputs with crowded buckets (many equal or clustered coordinates),
-// with 48-bit packed keys only.  Round 1 sorts (a, id) per list: T_x = tokens in (x, id)
-// order, T_y = tokens in (y, id) order.  Round 2 sorts the X list by (x, r) where r is a
+// with 48-bit packed keys only.  Pass 1 sorts (a, id) per list: T_x = tokens in (x, id)
+// order, T_y = tokens in (y, id) order.  Pass 2 sorts the X list by (x, r) where r is a
 // token's position in T_y -- so ties in x fall back to (y, id) -- and the Y list by (y, r)
 // with r its position in T_x; mapping r back through T_y / T_x gives the tokens.
 __device__ void fallback_sort(const float* xs, const float* ys, int N, int P, uint64_t* keys,

@@ -1,6 +1,6 @@
 """Host-side logic of the benchmark (no GPU): the algorithmic byte counts that the roofline
-fractions divide by, the measured-peak loader, the DRAM-traffic summary keying and the
-argument defaults."""
+fractions divide by, the measured-peak loader, the DRAM-traffic summary keying, the clock
+record and the argument defaults."""
 import os
 
 import bench
@@ -69,3 +69,31 @@ def test_workload_constants_match_the_generators():
     assert tuple(bench.STAGE_LAYERS) == tuple(synth.SWEEP_LAYERS)
     assert tuple(bench.STAGE_DIMS) == tuple(synth.SWEEP_DIMS)
     assert tuple(x.shape[1] for x in synth.sweep_coords(B=1)) == bench.STAGE_TOKENS
+
+
+def test_clock_sampler_reads_median_max_and_reasons(tmp_path):
+    """The clock record of a timed region: median SM clock under load, the highest
+    clocks.max.sm seen, and every throttle reason that was Active in any sample."""
+    path = tmp_path / "clocks.csv"
+    path.write_text(
+        "0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active\n"
+        "0, 1900, 1965, 998.0, 0x4, Not Active, Not Active, Not Active, Active\n"
+        "0, 1950, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n"
+        "garbage line\n"
+        "0, [N/A], 1965, 0, 0x0, Not Active, Active, Not Active, Not Active\n")
+
+    class FakeProc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    cs = bench.ClockSampler("GPU-0")
+    cs.proc, cs.path = FakeProc(), str(path)
+    rec = cs.stop()
+    assert rec["samples"] == 4
+    assert rec["sm_mhz"] == 1950.0 and rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert not path.exists()
+    assert bench.ClockSampler("GPU-0").stop()["reasons"] == ["nvidia-smi unavailable"]

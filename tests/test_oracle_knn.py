@@ -13,7 +13,8 @@ Pins, each independent of the oracle's own code:
 * queries outside the grid use the border cell (K = 1 copy);
 * with queries on cell centres the gather is the softmax over the KD-tree's
   exact neighbours and distances;
-* backward: central finite differences of L = <dOut, out> on the oracle.
+* backward: central finite differences of L = <dOut, out> on the oracle;
+* a token repeated in a table row takes the weights of all its slots (closed form).
 """
 import numpy as np
 import pytest
@@ -298,3 +299,24 @@ def test_invpow_half_precision_range_versus_exp_kernel():
         assert np.isfinite(w).all() and w.max() == np.float16(1.0)
         r = (dist.min() / dist) ** p                                # the ratio form
         assert np.isfinite(r).all() and r.max() == np.float16(1.0)
+
+
+def test_repeated_token_in_a_row_counts_once_per_slot():
+    """Table rows may repeat a token id (entries in [-1, N)); the softmax runs over the row's
+    slots, so a token in two slots takes both slots' weights, and an empty slot (-1) none:
+    closed form for the row [0, 0, 1, -1] at distances d0, d0, d1."""
+    xy = np.array([[[3.0, 2.0], [2.0, 6.0]]], dtype=np.float32)
+    q = np.array([[[2.0, 2.5]]], dtype=np.float32)
+    rng = np.random.default_rng(11)
+    feats = rng.standard_normal((1, 2, 32))
+    dout = rng.standard_normal((1, 1, 32))
+    table = _one_row_table(8, 8, [0, 0, 1, -1])
+    d0, d1 = np.hypot(1.0, 0.5), np.hypot(0.0, 3.5)
+    for p in (0.0, 0.7, 3.0):
+        e0, e1 = np.exp(-p * d0), np.exp(-p * d1)
+        w0, w1 = 2 * e0 / (2 * e0 + e1), e1 / (2 * e0 + e1)
+        out = oracle.knn_fwd(q, feats, xy, table, np.array([p]))[0, 0]
+        np.testing.assert_allclose(out, w0 * feats[0, 0] + w1 * feats[0, 1], rtol=1e-12)
+        dF, _, _ = oracle.knn_bwd(q, feats, xy, table, np.array([p]), dout)
+        np.testing.assert_allclose(dF[0, 0], w0 * dout[0, 0], rtol=1e-12)
+        np.testing.assert_allclose(dF[0, 1], w1 * dout[0, 0], rtol=1e-12)
